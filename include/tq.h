@@ -1,0 +1,259 @@
+/*
+ * tq.h -- C ABI of libtq, a B200 (sm_100a) implementation of the TurboQuant hot path.
+ *
+ * The method (TurboQuant: Online Vector Quantization with Near-optimal Distortion Rate,
+ * paper review, section "Method"): rotate each vector by a random orthogonal matrix Pi,
+ * quantize every rotated coordinate with a Lloyd-Max scalar codebook precomputed for the
+ * post-rotation coordinate law, and bit-pack the codes ("TurboQuant-mse").  The inner-
+ * product variant ("TurboQuant-prod") spends b-1 bits on that stage and one bit per
+ * projection on a Quantized-JL sketch of the residual, which makes inner products
+ * unbiased.  Attention reads the cache only through query-key inner products (review,
+ * "Problem"), so decode attention runs directly on the packed records.
+ * A SpectralQuant-style variant (SpectralQuant thread by @ashwingop, posts 4-6) replaces
+ * Pi by calibrated covariance eigenvectors, water-fills bits over the top signal dims and
+ * applies the QJL correction to those dims only.
+ *
+ * Conventions shared by every entry point:
+ *   - Every function returns a tq_status; nothing throws across the ABI.  On a non-OK
+ *     status tq_last_error() returns a thread-local message.
+ *   - Ownership: the caller owns every buffer.  The library never allocates, frees or
+ *     retains caller memory beyond the call (device work is stream-ordered).
+ *   - "device" pointers are CUDA device memory of the current device; "host" pointers
+ *     are ordinary host memory.  Device entry points are asynchronous on `stream`
+ *     (NULL = legacy default stream); arguments are validated on the host before any
+ *     launch and a failed validation launches nothing.
+ *   - Alignment: device pointers must be 16-byte aligned, else TQ_ERR_ALIGNMENT.
+ *   - Aliasing: an output that overlaps an input gives TQ_ERR_ALIAS.
+ *   - Device-side failures (a bounded wait that ran out) are recorded in a device status
+ *     word; tq_get_status() synchronizes the stream and returns it.  No kernel traps.
+ *   - Non-finite inputs give unspecified codes (never out-of-bounds accesses).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t / CUstream. */
+typedef struct CUstream_st* tq_stream;
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, inconsistent descriptor */
+  TQ_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+  TQ_ERR_ALIGNMENT = 3,     /* device pointer not 16-byte aligned */
+  TQ_ERR_ALIAS = 4,         /* an output overlaps an input */
+  TQ_ERR_CUDA = 5,          /* CUDA runtime error (message has the CUDA error string) */
+  TQ_ERR_TIMEOUT = 6,       /* a device-side bounded wait ran out (see tq_get_status) */
+  TQ_ERR_NOT_CONVERGED = 7, /* host iteration did not reach its tolerance */
+  TQ_ERR_WORKSPACE = 8      /* workspace pointer null or smaller than required */
+} tq_status;
+
+/* Coordinate law the codebook is solved for (review, Method: "known Beta distribution,
+ * converging to N(0, 1/d)"). */
+typedef enum { TQ_DIST_BETA_SPHERE = 0, TQ_DIST_GAUSSIAN = 1 } tq_dist;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+typedef enum { TQ_KIND_MSE = 0, TQ_KIND_PROD = 1, TQ_KIND_SPECTRAL = 2 } tq_kind;
+
+#define TQ_MAX_TOP 8
+
+/*
+ * Quantizer descriptor.  Plain data; all pointers are DEVICE pointers owned by the caller
+ * and read (never written) by the library.
+ *
+ *  MSE       bits = b (1..8).  centroids [2^b] ascending, boundaries [2^b-1] with
+ *            t_k = (c_k + c_{k+1})/2 (from tq_codebook_build).
+ *  PROD      bits = b total (1..9): b-1 MSE bits (centroids/boundaries of the (b-1)-bit
+ *            codebook; ignored when b = 1) plus m QJL sign bits; S [m*d] row-major,
+ *            i.i.d. N(0,1).  m must be a multiple of 32.
+ *  SPECTRAL  rot = calibrated eigenvectors (row j = eigenvector j, descending eigenvalue);
+ *            dims j < k_top use top_bits[j] bits (0..8), the rest tail_bits (1..4);
+ *            dim j's codebook is dim_sigma[j] * (standard-normal Lloyd-Max codebook);
+ *            unit_centroids / unit_boundaries hold those codebooks for 1..8 bits
+ *            concatenated (see tq_spectral_unit_codebooks).  qjl != 0 adds k_top sign bits
+ *            of S [k_top*k_top] applied to the top-k residual.
+ *  rot       [d*d] row-major fp32; the rotated vector is y = rot @ x.
+ */
+typedef struct {
+  int32_t kind;                 /* tq_kind */
+  int32_t d;                    /* vector dimension (2..4096) */
+  int32_t bits;                 /* MSE: bits; PROD: total bits; SPECTRAL: unused (0) */
+  int32_t m;                    /* PROD: QJL rows (multiple of 32); SPECTRAL: unused */
+  const float* rot;             /* [d*d] */
+  const float* S;               /* PROD [m*d]; SPECTRAL+qjl [k_top*k_top]; else NULL */
+  const float* centroids;       /* MSE/PROD */
+  const float* boundaries;      /* MSE/PROD */
+  int32_t k_top;                /* SPECTRAL: number of signal dims (1..TQ_MAX_TOP) */
+  int32_t tail_bits;            /* SPECTRAL: bits of dims >= k_top (1..4) */
+  int32_t qjl;                  /* SPECTRAL: 1 = QJL on the top-k residual */
+  int32_t top_bits[TQ_MAX_TOP]; /* SPECTRAL: bits of dims 0..k_top-1 */
+  const float* dim_sigma;       /* SPECTRAL: [d] sqrt(eigenvalue) per dim */
+  const float* unit_centroids;  /* SPECTRAL: [510] codebook of b bits at offset 2^b - 2 */
+  const float* unit_boundaries; /* SPECTRAL: [502] boundaries of b bits at offset 2^b - b - 1 */
+} tq_quantizer;
+
+/*
+ * Packed records, structure-of-arrays (each array indexed by record).  Record v owns
+ * codes[v*code_words .. +code_words), signs[v*sign_words ..), norms[v], rnorms[v]
+ * (word counts from tq_record_layout).  Code stream: code j occupies bits
+ * [j*b, j*b+b) of the record's little-endian uint32 stream, LSB first; unused bits 0.
+ * Signs: bit i%32 of word i/32 is 1 iff (S r)_i >= 0.  norms = ||x|| (fp32),
+ * rnorms = ||r|| of the QJL residual (fp32).  Spectral records: a head of
+ * ceil((sum top_bits + qjl*k_top)/32) words with the top-k codes LSB-first then the
+ * k_top sign bits, followed by ceil(d*tail_bits/32) words with dim j's code at bits
+ * [j*tail_bits, ...) (dims < k_top hold 0).  Unused arrays may be NULL.
+ * A KV cache is the same arrays laid out [B][Hkv][Nmax] records.
+ */
+typedef struct {
+  uint32_t* codes;
+  uint32_t* signs;
+  float* norms;
+  float* rnorms;
+} tq_packed;
+
+typedef struct {
+  int32_t code_words;   /* uint32 words of codes per record */
+  int32_t sign_words;   /* uint32 words of QJL signs per record (PROD) */
+  int32_t has_norms;    /* 1 if norms[] is written (MSE, PROD) */
+  int32_t has_rnorms;   /* 1 if rnorms[] is written (PROD, SPECTRAL with qjl) */
+} tq_layout;
+
+/* Library version string (static storage). */
+const char* tq_version(void);
+
+/* Thread-local message for the last non-OK status returned on this thread. */
+const char* tq_last_error(void);
+
+/*
+ * HOST.  Lloyd-Max codebook with 2^bits levels for one coordinate (review, Method:
+ * "solved once as a continuous 1-D k-means").  dist = TQ_DIST_BETA_SPHERE uses the
+ * exact marginal of a uniform point on S^{d-1} (d >= 2, sigma ignored);
+ * TQ_DIST_GAUSSIAN uses N(0, sigma^2) (sigma > 0, d ignored).  Iterates
+ * t_k = (c_k + c_{k+1})/2, c_k = E[t | cell k] until the largest move < 1e-13 * scale.
+ * Outputs (host, caller-allocated): centroids [2^bits] ascending, boundaries [2^bits-1];
+ * iterations may be NULL.  bits 1..8.  TQ_ERR_NOT_CONVERGED after 10^7 iterations.
+ */
+tq_status tq_codebook_build(int32_t d, int32_t bits, int32_t dist, double sigma,
+                            double* centroids, double* boundaries, int32_t* iterations);
+
+/*
+ * HOST.  Integer reverse water-filling (SpectralQuant thread, post 6: "[3,3,3,3] ->
+ * [5,3,2,2]"): starting from zero, each of budget_bits bits goes to
+ * argmax_j lambda_j * 4^(-b_j) (ties to the lowest j; dims capped at max_bits).
+ * lambda [k] host, bits_out [k] host.
+ */
+tq_status tq_waterfill(const double* lambda, int32_t k, int32_t budget_bits, int32_t max_bits,
+                       int32_t* bits_out);
+
+/*
+ * HOST.  SpectralQuant calibration (thread, post 4): eigen-decomposition of the second
+ * moment M = X^T X / n of n calibration rows X [n*d] (host, row-major fp32) by cyclic
+ * Jacobi rotations.  eigvecs_out [d*d] (row j = eigenvector j, sign fixed so its largest-
+ * magnitude entry is positive), eigvals_out [d] descending.  d <= 1024.
+ */
+tq_status tq_spectral_calibrate(const float* X, int64_t n, int32_t d,
+                                double* eigvecs_out, double* eigvals_out);
+
+/* HOST.  Standard-normal codebooks for 1..8 bits in the concatenated layout the
+ * SPECTRAL descriptor expects: centroids_out [510], boundaries_out [502]. */
+tq_status tq_spectral_unit_codebooks(double* centroids_out, double* boundaries_out);
+
+/* HOST.  Words per record and which norm arrays a quantizer writes. */
+tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out);
+
+/*
+ * DEVICE.  TurboQuant-mse quantize of n rows x [n*d] (dtype TQ_F32 / TQ_BF16 / TQ_F16,
+ * row-major): norms[v] = ||x_v||; y = rot @ (x_v/||x_v||); code_j = #{k : t_k < y_j};
+ * codes packed as described at tq_packed.  q->kind must be TQ_KIND_MSE.
+ * Appending a decode-time token is this call with `out` pointing at its cache slot.
+ */
+tq_status tq_quantize_mse(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n,
+                          tq_packed out, tq_stream stream);
+
+/*
+ * DEVICE.  TurboQuant-prod quantize (review, Method): the (bits-1)-bit MSE stage as above,
+ * residual r = y - c[code] in the rotated unit-scale domain, rnorms[v] = ||r||,
+ * sign_i = [(S r)_i >= 0].  q->kind must be TQ_KIND_PROD.
+ */
+tq_status tq_quantize_prod(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n,
+                           tq_packed out, tq_stream stream);
+
+/*
+ * DEVICE.  SpectralQuant-style quantize: z = rot @ x (no normalization), dim j coded with
+ * dim_sigma[j] * unit codebook of its bits; with qjl, r = z_top - c_hat_top,
+ * rnorms[v] = ||r||, sign_i = [(S r)_i >= 0] for i < k_top.  q->kind TQ_KIND_SPECTRAL.
+ */
+tq_status tq_quantize_spectral(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n,
+                               tq_packed out, tq_stream stream);
+
+/*
+ * DEVICE.  Reconstruction out [n*d] fp32: MSE x_hat = ||x|| rot^T c[code];
+ * PROD adds ||x|| rot^T (sqrt(pi/2)/m ||r|| S^T (2s-1)) (unbiased);
+ * SPECTRAL x_hat = rot^T c_hat (the QJL bits are not used).
+ */
+tq_status tq_dequantize(const tq_quantizer* q, tq_packed in, int64_t n, float* out,
+                        tq_stream stream);
+
+/*
+ * Workspace bytes needed by tq_score for nq queries against n records with topk (0 = dense).
+ */
+tq_status tq_score_workspace(const tq_quantizer* q, int64_t nq, int64_t n, int32_t topk,
+                             size_t* bytes);
+
+/*
+ * DEVICE.  Inner-product estimates of queries qv [nq*d] (dtype) against n packed records:
+ *   MSE       ||x|| <rot q, c[code]>
+ *   PROD      ||x|| (<rot q, c_hat> + sqrt(pi/2)/m ||r|| <S rot q, 2s-1>)   (unbiased)
+ *   SPECTRAL  sum_j (rot q)_j c_hat_j + sqrt(pi/2)/k ||r|| <S (rot q)_top, 2s-1>
+ * topk == 0: scores [nq*n] fp32 dense, ids unused.  topk in 1..64: for each query the
+ * topk records by descending estimate, ties to the lower id: ids [nq*topk] int32,
+ * scores [nq*topk].  workspace: device, >= tq_score_workspace bytes.
+ */
+tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t nq,
+                   tq_packed keys, int64_t n, int32_t topk, float* scores, int32_t* ids,
+                   void* workspace, size_t ws_bytes, tq_stream stream);
+
+/* Workspace bytes needed by tq_decode_attn for this shape. */
+tq_status tq_decode_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq, int32_t Hkv,
+                                   int64_t Nmax, size_t* bytes);
+
+/*
+ * DEVICE.  One decode-attention step straight from the packed cache:
+ *   for query head h (KV head h / (Hq/Hkv)), logit_i = scale * est(q_h, k_i) over the
+ *   first seq_lens[b] records, p = softmax(logit), out = sum_i p_i v_hat_i.
+ * q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), caches laid out
+ * [B][Hkv][Nmax] records, out [B*Hq*d] fp32.  Keys: MSE, PROD or SPECTRAL; values: MSE or
+ * SPECTRAL (without qjl).  This build runs d in {64, 128}, code bits <= 4, PROD m = d,
+ * Hq/Hkv in 1..16; other shapes give TQ_ERR_UNSUPPORTED.  Value norms must stay below
+ * 6.0e4 (the probability-weighted norm is a half-precision MMA operand).
+ */
+tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const void* q,
+                         int32_t dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,
+                         const int32_t* seq_lens, tq_packed kcache, tq_packed vcache,
+                         float scale, float* out, void* workspace, size_t ws_bytes,
+                         tq_stream stream);
+
+/*
+ * Synchronizes `stream`, then returns and clears the device status word of the current
+ * device: TQ_OK, or TQ_ERR_TIMEOUT if a bounded device wait ran out since the last call.
+ */
+tq_status tq_get_status(tq_stream stream);
+
+/*
+ * Test hook: iteration limit of every device-side bounded wait launched after this call
+ * (0 = default, about 2^26 polls).  Lowering it makes waits that are not immediately
+ * satisfied time out, which exercises the error path without hanging a GPU.
+ */
+tq_status tq_set_wait_limit(int64_t polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

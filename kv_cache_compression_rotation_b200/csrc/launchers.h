@@ -1,0 +1,24 @@
+// Host launchers for the templated kernels, each compiled in its own translation unit.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace tq {
+
+struct DecodeParams;
+struct UmmaQuantParams;
+
+// Launch decode_attn_kernel for (key format, key bits, value format, value bits) at D = 128.
+// Returns cudaErrorNotSupported (without launching) for a combination that is not built.
+cudaError_t launch_decode(const DecodeParams& p, int kfmt, int kb, int vfmt, int vb, dim3 grid,
+                          size_t smem, cudaStream_t stream);
+cudaError_t launch_decode_mse(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
+cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
+cudaError_t launch_decode_spec(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
+
+// Tensor-core quantize (d = 128, 16-bit input, MSE bits 1..4).
+cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& p, int bits, int grid,
+                                 cudaStream_t stream);
+
+}  // namespace tq

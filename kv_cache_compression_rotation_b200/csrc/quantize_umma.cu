@@ -1,0 +1,30 @@
+// Instantiations of the tensor-core quantize kernel.
+#include "launchers.h"
+#include "quantize_umma.cuh"
+
+namespace tq {
+namespace {
+
+template <int B>
+cudaError_t go(const CUtensorMap& map, const UmmaQuantParams& p, int grid, cudaStream_t s) {
+  auto k = umma_quantize_kernel<B>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kUmmaSmemBytes));
+  if (e != cudaSuccess) return e;
+  k<<<grid, kUmmaThreads, kUmmaSmemBytes, s>>>(map, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& p, int bits, int grid,
+                                 cudaStream_t s) {
+  switch (bits) {
+    case 1: return go<1>(map, p, grid, s);
+    case 2: return go<2>(map, p, grid, s);
+    case 3: return go<3>(map, p, grid, s);
+    case 4: return go<4>(map, p, grid, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace tq

@@ -1,0 +1,320 @@
+// Tensor-core quantize for d = 128, 16-bit input: TMA -> tcgen05.mma (TMEM) -> epilogue.
+//
+// TurboQuant review, "Method": y = Pi x / ||x||, then each coordinate is coded against
+// the Lloyd-Max boundaries.  The rotation is the only dense contraction of the path:
+//   Y[128 vectors x 128] = X[128 x 128] . Pi^T,   accumulated in TMEM (fp32).
+// Pi is fp32; the input is exact in bf16 (or fp16), so Pi is split as Pi_hi + Pi_lo
+// (both in the input's 16-bit type) and the tile takes two MMAs per k-step into the same
+// accumulator.  The split keeps every rotated coordinate within about 2^-17 ||x|| of
+// the fp32 product, far inside the 1e-5 decision band around a boundary.
+//
+// Roles in a persistent CTA (one per SM), 320 threads:
+//   warp 0      TMA producer: 128-row tiles of x into a 4-stage ring (128B swizzle)
+//   warp 1      TMEM allocator and single-thread MMA issuer (2 accumulator buffers)
+//   warps 2-5   epilogue group 0 (even tiles), warps 6-9 group 1 (odd tiles):
+//               one vector per thread: tcgen05.ld the row, ||y||, codes against
+//               ||y|| * t_k, pack LSB-first, store record + norm.
+// ||y|| equals ||x|| up to the orthogonality of the fp32 Pi (~1e-7 relative).
+// Every mbarrier wait is bounded; on timeout the CTA records TQ_ERR_TIMEOUT, drains
+// what it issued, frees TMEM and exits.
+#pragma once
+
+#include <cuda.h>
+
+#include "device_common.cuh"
+
+namespace tq {
+
+constexpr int kUmmaThreads = 320;
+constexpr int kUmmaStages = 4;
+constexpr int kUmmaTileRows = 128;
+constexpr int kUmmaD = 128;
+constexpr uint32_t kXStageBytes = kUmmaTileRows * kUmmaD * 2;      // 32 KB
+constexpr uint32_t kPiBytes = kUmmaD * kUmmaD * 2;                 // 32 KB per half
+// Drains (copies and MMAs this CTA already issued) always complete on their own; their
+// bound is fixed and independent of the test-adjustable wait limit.
+constexpr long long kDrainLimit = 1ll << 28;
+constexpr uint32_t kUmmaSmemBytes = 1024 /*align slack*/ + 2 * kPiBytes + kUmmaStages * kXStageBytes + 256;
+
+struct UmmaQuantParams {
+  const float* rot;        // [128*128] fp32
+  const float* boundaries; // [2^b - 1]
+  int64_t n;
+  int is_f16;              // 0 bf16, 1 fp16
+  uint32_t* codes;         // [n][W]
+  float* norms;            // [n]
+  int* status;
+  long long wait_limit;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; returns false (and records a timeout) if the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit, int* status,
+                                          volatile int* abort_flag) {
+  for (long long i = 0;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if (i >= limit || *abort_flag) {
+      report_status(status, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle layout
+// (8-row x 128-byte atoms, 1024 B apart).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);          // start address
+  desc |= static_cast<uint64_t>(1u) << 16;                          // leading byte offset (unused)
+  desc |= static_cast<uint64_t>(1024u >> 4) << 32;                  // stride byte offset
+  desc |= static_cast<uint64_t>(1u) << 46;                          // descriptor version
+  desc |= static_cast<uint64_t>(2u) << 61;                          // 128-byte swizzle
+  return desc;
+}
+
+// Instruction descriptor: D f32, A/B bf16 or f16, both K-major, M = 128, N = 128.
+__device__ __forceinline__ uint32_t idesc_m128n128(int is_f16) {
+  const uint32_t ab = is_f16 ? 0u : 1u;
+  return (1u << 4) | (ab << 7) | (ab << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+template <int B>
+__global__ void __launch_bounds__(kUmmaThreads, 1)
+umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantParams p) {
+  constexpr int K = 1 << B;
+  constexpr int NB = K - 1;
+  constexpr int W = kUmmaD * B / 32;             // code words per vector
+  extern __shared__ unsigned char usm_raw[];
+  const uint32_t raw = smem_u32(usm_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sm = usm_raw + (base - raw);
+  const uint32_t pi_hi = base, pi_lo = base + kPiBytes;
+  const uint32_t xs0 = base + 2 * kPiBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * kPiBytes + kUmmaStages * kXStageBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kUmmaStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kUmmaStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kUmmaStages + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kUmmaStages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* tsm = reinterpret_cast<float*>(tmem_slot + 2);   // boundaries [NB]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n_tiles = (p.n + kUmmaTileRows - 1) / kUmmaTileRows;
+
+  // Pi_hi / Pi_lo in the swizzled K-major layout: row = output dim n, k = input dim.
+  for (int i = tid; i < kUmmaD * kUmmaD; i += kUmmaThreads) {
+    const int nrow = i >> 7, k = i & 127;
+    const float v = __ldg(p.rot + i);
+    uint16_t hi, lo;
+    if (p.is_f16) {
+      const __half h = __float2half_rn(v);
+      const __half l = __float2half_rn(v - __half2float(h));
+      hi = __half_as_ushort(h); lo = __half_as_ushort(l);
+    } else {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+      hi = __bfloat16_as_ushort(h); lo = __bfloat16_as_ushort(l);
+    }
+    const int kb = k >> 6, kk = k & 63;
+    const uint32_t off = kb * (kUmmaD * 128) + nrow * 128 + ((((kk >> 3) ^ (nrow & 7))) << 4) + (kk & 7) * 2;
+    *reinterpret_cast<uint16_t*>(sm + off) = hi;
+    *reinterpret_cast<uint16_t*>(sm + kPiBytes + off) = lo;
+  }
+  if (tid < NB) tsm[tid] = __ldg(p.boundaries + tid);
+  if (tid == 0) {
+    for (int s = 0; s < kUmmaStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), 128); }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // generic-proxy writes of Pi must be visible to the tensor-core (async) proxy
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(tmem_slot)), "r"(256) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const long long lim = p.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      int issued = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        const int s = it % kUmmaStages, use = it / kUmmaStages;
+        if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, lim, p.status, abort_flag)) break;
+        mbar_expect_tx(full_bar(s), kXStageBytes);
+        const uint32_t dst = xs0 + s * kXStageBytes;
+        const int row = static_cast<int>(tile * kUmmaTileRows);
+        tma_load_2d(dst, &xmap, 0, row, full_bar(s));
+        tma_load_2d(dst + kXStageBytes / 2, &xmap, 64, row, full_bar(s));
+        ++issued;
+      }
+      // drain: every issued stage must land before the CTA can exit
+      for (int j = max(0, issued - kUmmaStages); j < issued; ++j) {
+        const int s = j % kUmmaStages, use = j / kUmmaStages;
+        for (long long i = 0; !mbar_try(full_bar(s), use & 1) && i < kDrainLimit; ++i) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_m128n128(p.is_f16);
+      int it = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        const int s = it % kUmmaStages, buf = it & 1, j = it >> 1;
+        if (j > 0 && !mbar_wait(tempty_bar(buf), (j - 1) & 1, lim, p.status, abort_flag)) break;
+        if (!mbar_wait(full_bar(s), (it / kUmmaStages) & 1, lim, p.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t xa = xs0 + s * kXStageBytes;
+        const uint32_t td = tmem_base + buf * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * (kXStageBytes / 2) + (kk & 3) * 32;
+          const uint32_t poff = (kk >> 2) * (kPiBytes / 2) + (kk & 3) * 32;
+          umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_hi + poff), idesc, kk > 0 ? 1u : 0u);
+          umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo + poff), idesc, 1u);
+        }
+        umma_commit(empty_bar(s));
+        umma_commit(tfull_bar(buf));
+      }
+      // wait for the tensor core to finish everything issued before TMEM is freed
+      if (it > 0) {
+        const int last = it - 1;
+        for (long long i = 0; !mbar_try(tfull_bar(last & 1), (last >> 1) & 1) && i < kDrainLimit; ++i) {}
+      }
+    }
+  } else {
+    const int grp = (warp - 2) >> 2;                   // 0: warps 2-5, 1: warps 6-9
+    const int lanebase = 32 * (warp & 3);              // TMEM lanes this warp may access
+    const int r = lanebase + lane;                     // row within the tile
+    float thr[NB];
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      if (buf != grp) continue;
+      const int j = it >> 1;
+      if (!mbar_wait(tfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 128;
+      // pass 1: ||y|| over the whole row
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(taddr + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+      const float nu = sqrtf(ss);
+#pragma unroll
+      for (int k = 0; k < NB; ++k) thr[k] = nu * tsm[k];
+      // pass 2: codes against ||y|| * t_k, packed LSB-first
+      uint32_t words[W];
+#pragma unroll
+      for (int w = 0; w < W; ++w) words[w] = 0u;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(taddr + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          int code = 0;
+#pragma unroll
+          for (int k = 0; k < NB; ++k) code += (v[i] > thr[k]) ? 1 : 0;
+          const int pos = (32 * c + i) * B;
+          words[pos >> 5] |= static_cast<uint32_t>(code) << (pos & 31);
+          if ((pos & 31) + B > 32) words[(pos >> 5) + 1] |= static_cast<uint32_t>(code) >> (32 - (pos & 31));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(buf));
+      const int64_t v = tile * kUmmaTileRows + r;
+      if (v < p.n) {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + v * W);
+#pragma unroll
+        for (int w = 0; w < W / 4; ++w)
+          dst[w] = make_uint4(words[4 * w], words[4 * w + 1], words[4 * w + 2], words[4 * w + 3]);
+        p.norms[v] = nu;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(256) : "memory");
+  }
+}
+
+}  // namespace tq

@@ -1,0 +1,641 @@
+// C ABI of libtq: argument validation, workspace planning and kernel launches.
+// The declarations and their contracts are in include/tq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "decode.cuh"
+#include "decode_aux.cuh"
+#include "device_common.cuh"
+#include "launchers.h"
+#include "quantize_simt.cuh"
+#include "quantize_umma.cuh"
+#include "score.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+
+__device__ int g_tq_status = 0;
+
+namespace {
+thread_local char g_msg[512] = "ok";
+std::atomic<long long> g_wait_limit{0};
+constexpr long long kDefaultWaitLimit = 1ll << 24;
+}  // namespace
+
+tq_status fail(tq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+int* device_status_ptr() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_tq_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(ptr);
+}
+
+long long wait_limit() {
+  const long long v = g_wait_limit.load();
+  return v > 0 ? v : kDefaultWaitLimit;
+}
+
+namespace {
+
+tq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  const void* p;
+  size_t bytes;
+};
+
+bool overlaps(Range a, Range b) {
+  if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+  return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+size_t dtype_size(int dtype) { return dtype == TQ_F32 ? 4 : 2; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+int spectral_head_bits(const tq_quantizer* q) {
+  int s = 0;
+  for (int j = 0; j < q->k_top; ++j) s += q->top_bits[j];
+  return s + (q->qjl ? q->k_top : 0);
+}
+
+tq_status check_quantizer(const tq_quantizer* q) {
+  if (!q) return fail(TQ_ERR_INVALID_ARG, "quantizer is NULL");
+  if (q->d < 2 || q->d > 4096) return fail(TQ_ERR_INVALID_ARG, "d must be in 2..4096 (got %d)", q->d);
+  if (!q->rot) return fail(TQ_ERR_INVALID_ARG, "rot is NULL");
+  if (!aligned16(q->rot)) return fail(TQ_ERR_ALIGNMENT, "rot is not 16-byte aligned");
+  switch (q->kind) {
+    case TQ_KIND_MSE:
+      if (q->bits < 1 || q->bits > 8) return fail(TQ_ERR_INVALID_ARG, "MSE bits must be 1..8");
+      if (!q->centroids || !q->boundaries) return fail(TQ_ERR_INVALID_ARG, "codebook is NULL");
+      break;
+    case TQ_KIND_PROD:
+      if (q->bits < 1 || q->bits > 9) return fail(TQ_ERR_INVALID_ARG, "PROD bits must be 1..9");
+      if (q->m < 32 || q->m > 4096 || (q->m & 31)) return fail(TQ_ERR_INVALID_ARG, "PROD m must be a multiple of 32 in 32..4096");
+      if (!q->S) return fail(TQ_ERR_INVALID_ARG, "S is NULL");
+      if (q->bits > 1 && (!q->centroids || !q->boundaries)) return fail(TQ_ERR_INVALID_ARG, "codebook is NULL");
+      break;
+    case TQ_KIND_SPECTRAL: {
+      if (q->k_top < 1 || q->k_top > TQ_MAX_TOP || q->k_top > q->d)
+        return fail(TQ_ERR_INVALID_ARG, "k_top must be 1..%d and <= d", TQ_MAX_TOP);
+      for (int j = 0; j < q->k_top; ++j)
+        if (q->top_bits[j] < 0 || q->top_bits[j] > 8) return fail(TQ_ERR_INVALID_ARG, "top_bits must be 0..8");
+      if (q->tail_bits < 1 || q->tail_bits > 4) return fail(TQ_ERR_INVALID_ARG, "tail_bits must be 1..4");
+      if (spectral_head_bits(q) > 96) return fail(TQ_ERR_INVALID_ARG, "spectral head exceeds 96 bits");
+      if (!q->dim_sigma || !q->unit_centroids || !q->unit_boundaries)
+        return fail(TQ_ERR_INVALID_ARG, "spectral codebook arrays are NULL");
+      if (q->qjl && !q->S) return fail(TQ_ERR_INVALID_ARG, "S is NULL (qjl)");
+      break;
+    }
+    default:
+      return fail(TQ_ERR_INVALID_ARG, "unknown quantizer kind %d", q->kind);
+  }
+  if (q->S && !aligned16(q->S)) return fail(TQ_ERR_ALIGNMENT, "S is not 16-byte aligned");
+  return TQ_OK;
+}
+
+tq_layout layout_of(const tq_quantizer* q) {
+  tq_layout L{};
+  if (q->kind == TQ_KIND_MSE) {
+    L.code_words = words_for(q->d, q->bits);
+    L.has_norms = 1;
+  } else if (q->kind == TQ_KIND_PROD) {
+    L.code_words = q->bits > 1 ? words_for(q->d, q->bits - 1) : 0;
+    L.sign_words = q->m / 32;
+    L.has_norms = 1;
+    L.has_rnorms = 1;
+  } else {
+    L.code_words = (spectral_head_bits(q) + 31) / 32 + words_for(q->d, q->tail_bits);
+    L.has_rnorms = q->qjl ? 1 : 0;
+  }
+  return L;
+}
+
+tq_status check_packed(const tq_packed& pk, const tq_layout& L, bool need_codes = true) {
+  if (need_codes && L.code_words > 0 && !pk.codes) return fail(TQ_ERR_INVALID_ARG, "codes is NULL");
+  if (L.sign_words > 0 && !pk.signs) return fail(TQ_ERR_INVALID_ARG, "signs is NULL");
+  if (L.has_norms && !pk.norms) return fail(TQ_ERR_INVALID_ARG, "norms is NULL");
+  if (L.has_rnorms && !pk.rnorms) return fail(TQ_ERR_INVALID_ARG, "rnorms is NULL");
+  const void* ps[4] = {pk.codes, pk.signs, pk.norms, pk.rnorms};
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return fail(TQ_ERR_ALIGNMENT, "packed array is not 16-byte aligned");
+  return TQ_OK;
+}
+
+void packed_ranges(const tq_packed& pk, const tq_layout& L, int64_t n, Range out[4]) {
+  out[0] = {pk.codes, static_cast<size_t>(n) * L.code_words * 4};
+  out[1] = {pk.signs, static_cast<size_t>(n) * L.sign_words * 4};
+  out[2] = {L.has_norms ? pk.norms : nullptr, static_cast<size_t>(n) * 4};
+  out[3] = {L.has_rnorms ? pk.rnorms : nullptr, static_cast<size_t>(n) * 4};
+}
+
+tq_status check_no_alias(const Range* outs, int nout, const Range* ins, int nin) {
+  for (int i = 0; i < nout; ++i) {
+    for (int j = 0; j < nin; ++j)
+      if (overlaps(outs[i], ins[j])) return fail(TQ_ERR_ALIAS, "an output overlaps an input");
+    for (int j = i + 1; j < nout; ++j)
+      if (overlaps(outs[i], outs[j])) return fail(TQ_ERR_ALIAS, "two outputs overlap");
+  }
+  return TQ_OK;
+}
+
+// ---- tensor map for the tensor-core quantize ----
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool umma_supported(const tq_quantizer* q, int dtype, int64_t n) {
+  if (q->kind != TQ_KIND_MSE || q->d != 128 || q->bits > 4) return false;
+  if (dtype != TQ_BF16 && dtype != TQ_F16) return false;
+  if (n < 1 || n >= (1ll << 31) - 256) return false;
+  if (std::getenv("TQ_FORCE_SIMT")) return false;
+  int dev = 0, major = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  return major == 10 && get_encode() != nullptr;
+}
+
+tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64_t n, tq_packed out,
+                          cudaStream_t stream, int want_kind) {
+  tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (q->kind != want_kind) return fail(TQ_ERR_INVALID_ARG, "quantizer kind does not match this entry point");
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return TQ_OK;
+  if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
+  if (!aligned16(x)) return fail(TQ_ERR_ALIGNMENT, "x is not 16-byte aligned");
+  if (q->d > 2048) return fail(TQ_ERR_UNSUPPORTED, "quantize supports d <= 2048 in this build");
+  const tq_layout L = layout_of(q);
+  if ((s = check_packed(out, L)) != TQ_OK) return s;
+  Range outs[4];
+  packed_ranges(out, L, n, outs);
+  const Range ins[1] = {{x, static_cast<size_t>(n) * q->d * dtype_size(dtype)}};
+  if ((s = check_no_alias(outs, 4, ins, 1)) != TQ_OK) return s;
+  int* status = device_status_ptr();
+
+  if (umma_supported(q, dtype, n)) {
+    auto encode = get_encode();
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {128, static_cast<cuuint64_t>(n)};
+    const cuuint64_t gstride[1] = {256};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(&map, dtype == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                              2, const_cast<void*>(x), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    UmmaQuantParams p{};
+    p.rot = q->rot;
+    p.boundaries = q->boundaries;
+    p.n = n;
+    p.is_f16 = dtype == TQ_F16;
+    p.codes = out.codes;
+    p.norms = out.norms;
+    p.status = status;
+    p.wait_limit = wait_limit();
+    const int64_t tiles = (n + 127) / 128;
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
+    const cudaError_t e = launch_umma_quantize(map, p, q->bits, grid, stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "umma quantize launch");
+  }
+
+  SimtQuantParams p{};
+  p.x = x; p.dtype = dtype; p.n = n; p.d = q->d; p.kind = q->kind;
+  p.rot = q->rot; p.S = q->S;
+  p.m = q->kind == TQ_KIND_PROD ? q->m : (q->kind == TQ_KIND_SPECTRAL && q->qjl ? q->k_top : 0);
+  p.centroids = q->centroids; p.boundaries = q->boundaries;
+  p.bmse = q->kind == TQ_KIND_MSE ? q->bits : (q->kind == TQ_KIND_PROD ? q->bits - 1 : 0);
+  p.k_top = q->k_top; p.tail_bits = q->tail_bits; p.qjl = q->qjl;
+  for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];
+  p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids; p.unit_t = q->unit_boundaries;
+  p.codes = out.codes; p.code_words = L.code_words;
+  p.signs = out.signs; p.sign_words = L.sign_words;
+  p.norms = L.has_norms ? out.norms : nullptr;
+  p.rnorms = L.has_rnorms ? out.rnorms : nullptr;
+  const int d = q->d;
+  int tv = static_cast<int>(std::min<int64_t>(16, std::max<int64_t>(1, 180000 / (9 * d + 12))));
+  p.tv = tv;
+  const size_t smem = static_cast<size_t>(tv) * d * 9 + static_cast<size_t>(tv) * 12 + 16;
+  cudaError_t e = cudaFuncSetAttribute(simt_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "simt quantize attribute");
+  const int64_t blocks = (n + tv - 1) / tv;
+  if (blocks > 0x7fffffff) return fail(TQ_ERR_INVALID_ARG, "n too large");
+  simt_quantize_kernel<<<static_cast<unsigned>(blocks), kSimtThreads, smem, stream>>>(p);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "simt quantize launch");
+}
+
+// ---- decode planning ----
+struct DecodePlan {
+  int chunk_len, n_chunks, qb_stride;
+  size_t off_qa, off_qb, off_qs, off_ml, off_o, bytes;
+};
+
+DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t Nmax) {
+  DecodePlan P{};
+  const int D = kq->d;
+  const int64_t units = static_cast<int64_t>(B) * Hkv;
+  const int64_t target = static_cast<int64_t>(sm_count()) * 6;
+  int64_t nch = std::max<int64_t>(1, (target + units - 1) / units);
+  int64_t cl = (Nmax + nch - 1) / nch;
+  cl = std::max<int64_t>(256, (cl + 63) / 64 * 64);
+  nch = (Nmax + cl - 1) / cl;
+  P.chunk_len = static_cast<int>(cl);
+  P.n_chunks = static_cast<int>(nch);
+  P.qb_stride = kq->kind == TQ_KIND_PROD ? kq->m : 16;
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t off = 0;
+  P.off_qa = off; off = al(off + rows * D * 4);
+  P.off_qb = off; off = al(off + rows * P.qb_stride * 4);
+  P.off_qs = off; off = al(off + rows * 2 * 4);
+  P.off_ml = off; off = al(off + rows * nch * 2 * 4);
+  P.off_o = off; off = al(off + rows * nch * D * 4);
+  P.bytes = off;
+  return P;
+}
+
+tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int B, int Hq, int Hkv, int64_t Nmax) {
+  tq_status s = check_quantizer(kq);
+  if (s != TQ_OK) return s;
+  if ((s = check_quantizer(vq)) != TQ_OK) return s;
+  if (B < 1 || Hkv < 1 || Hq < 1 || Nmax < 1) return fail(TQ_ERR_INVALID_ARG, "B, Hq, Hkv, Nmax must be >= 1");
+  if (Hq % Hkv) return fail(TQ_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (kq->d != vq->d) return fail(TQ_ERR_INVALID_ARG, "key and value d differ");
+  if (Nmax > (1ll << 30)) return fail(TQ_ERR_INVALID_ARG, "Nmax too large");
+  if (static_cast<int64_t>(B) * Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "B*Hkv > 65535");
+  if (kq->d != 128) return fail(TQ_ERR_UNSUPPORTED, "decode attention runs d = 128 in this build");
+  if (Hq / Hkv > 16) return fail(TQ_ERR_UNSUPPORTED, "Hq/Hkv > 16");
+  if (vq->kind == TQ_KIND_PROD) return fail(TQ_ERR_UNSUPPORTED, "values as PROD are not built");
+  if (vq->kind == TQ_KIND_SPECTRAL && vq->qjl) return fail(TQ_ERR_UNSUPPORTED, "spectral values with qjl");
+  if ((kq->kind == TQ_KIND_SPECTRAL) != (vq->kind == TQ_KIND_SPECTRAL))
+    return fail(TQ_ERR_UNSUPPORTED, "spectral keys need spectral values (and the reverse)");
+  if (kq->kind == TQ_KIND_PROD && (kq->m != 128 || kq->bits < 2 || kq->bits > 5))
+    return fail(TQ_ERR_UNSUPPORTED, "PROD keys need m = d and 2..5 bits");
+  if (kq->kind == TQ_KIND_MSE && kq->bits > 4) return fail(TQ_ERR_UNSUPPORTED, "key bits > 4");
+  if (vq->kind == TQ_KIND_MSE && vq->bits > 4) return fail(TQ_ERR_UNSUPPORTED, "value bits > 4");
+  if (kq->kind == TQ_KIND_SPECTRAL && (kq->tail_bits > 2 || kq->tail_bits != vq->tail_bits))
+    return fail(TQ_ERR_UNSUPPORTED, "spectral tail bits must be equal and <= 2");
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_version(void) { return "libtq 0.1 (sm_100a)"; }
+
+const char* tq_last_error(void) { return g_msg; }
+
+tq_status tq_codebook_build(int32_t d, int32_t bits, int32_t dist, double sigma, double* centroids,
+                            double* boundaries, int32_t* iterations) {
+  int it = 0;
+  const tq_status s = codebook_build(d, bits, dist, sigma, centroids, boundaries, &it);
+  if (iterations) *iterations = it;
+  return s;
+}
+
+tq_status tq_waterfill(const double* lambda, int32_t k, int32_t budget_bits, int32_t max_bits, int32_t* bits_out) {
+  return waterfill(lambda, k, budget_bits, max_bits, bits_out);
+}
+
+tq_status tq_spectral_calibrate(const float* X, int64_t n, int32_t d, double* eigvecs_out, double* eigvals_out) {
+  return spectral_calibrate(X, n, d, eigvecs_out, eigvals_out);
+}
+
+tq_status tq_spectral_unit_codebooks(double* centroids_out, double* boundaries_out) {
+  return spectral_unit_codebooks(centroids_out, boundaries_out);
+}
+
+tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out) {
+  const tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "layout output is NULL");
+  *out = layout_of(q);
+  return TQ_OK;
+}
+
+tq_status tq_quantize_mse(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
+                          tq_stream stream) {
+  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_MSE);
+}
+
+tq_status tq_quantize_prod(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
+                           tq_stream stream) {
+  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_PROD);
+}
+
+tq_status tq_quantize_spectral(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
+                               tq_stream stream) {
+  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_SPECTRAL);
+}
+
+tq_status tq_dequantize(const tq_quantizer* q, tq_packed in, int64_t n, float* out, tq_stream stream) {
+  tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return TQ_OK;
+  if (n > 0x7fffffff) return fail(TQ_ERR_INVALID_ARG, "n too large");
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  if (!aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "out is not 16-byte aligned");
+  const tq_layout L = layout_of(q);
+  if ((s = check_packed(in, L)) != TQ_OK) return s;
+  Range ins[4];
+  packed_ranges(in, L, n, ins);
+  const Range outs[1] = {{out, static_cast<size_t>(n) * q->d * 4}};
+  if ((s = check_no_alias(outs, 1, ins, 4)) != TQ_OK) return s;
+  DequantParams p{};
+  p.kind = q->kind; p.d = q->d; p.m = q->m;
+  p.bmse = q->kind == TQ_KIND_MSE ? q->bits : (q->kind == TQ_KIND_PROD ? q->bits - 1 : 0);
+  p.rot = q->rot; p.S = q->S; p.centroids = q->centroids;
+  p.codes = in.codes; p.code_words = L.code_words;
+  p.signs = in.signs; p.sign_words = L.sign_words;
+  p.norms = in.norms; p.rnorms = in.rnorms;
+  p.k_top = q->k_top; p.tail_bits = q->tail_bits; p.qjl = q->qjl;
+  for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];
+  p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids;
+  p.out = out; p.n = n;
+  const size_t smem = static_cast<size_t>(q->d) * 4;
+  dequant_kernel<<<static_cast<unsigned>(n), kSimtThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "dequantize launch");
+}
+
+static int64_t score_block(int64_t nq, int64_t n) {
+  int64_t qb = (1ll << 28) / (4 * std::max<int64_t>(n, 1));
+  qb = std::max<int64_t>(8, std::min<int64_t>(1024, qb)) / 8 * 8;
+  return std::min<int64_t>(qb, (nq + 7) / 8 * 8);
+}
+
+static int score_qu_stride(const tq_quantizer* q) {
+  if (q->kind == TQ_KIND_PROD) return q->m;
+  if (q->kind == TQ_KIND_SPECTRAL && q->qjl) return q->k_top;
+  return 0;
+}
+
+tq_status tq_score_workspace(const tq_quantizer* q, int64_t nq, int64_t n, int32_t topk, size_t* bytes) {
+  tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (!bytes || nq < 0 || n < 0) return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
+  size_t b = static_cast<size_t>(nq) * q->d * 4 + 256;
+  b += static_cast<size_t>(nq) * score_qu_stride(q) * 4 + 256;
+  if (topk > 0) b += static_cast<size_t>(score_block(nq, n)) * static_cast<size_t>(n) * 4 + 256;
+  *bytes = b;
+  return TQ_OK;
+}
+
+tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t nq, tq_packed keys, int64_t n,
+                   int32_t topk, float* scores, int32_t* ids, void* workspace, size_t ws_bytes, tq_stream stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (nq < 0 || n < 0) return fail(TQ_ERR_INVALID_ARG, "nq, n must be >= 0");
+  if (topk < 0 || topk > 32) return fail(TQ_ERR_UNSUPPORTED, "topk must be 0..32");
+  if (topk > 0 && topk > n) return fail(TQ_ERR_INVALID_ARG, "topk > n");
+  if (n > 0x7fffffff || nq > 0x7fffffff) return fail(TQ_ERR_INVALID_ARG, "sizes too large");
+  if (nq == 0 || n == 0) return TQ_OK;
+  if (!qv || !scores || (topk > 0 && !ids)) return fail(TQ_ERR_INVALID_ARG, "NULL query or output");
+  if (!aligned16(qv) || !aligned16(scores) || (ids && !aligned16(ids)))
+    return fail(TQ_ERR_ALIGNMENT, "query/output not 16-byte aligned");
+  if (q->d > 2048) return fail(TQ_ERR_UNSUPPORTED, "score supports d <= 2048");
+  const tq_layout L = layout_of(q);
+  if ((s = check_packed(keys, L)) != TQ_OK) return s;
+  size_t need = 0;
+  tq_score_workspace(q, nq, n, topk, &need);
+  if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  Range ins[6];
+  packed_ranges(keys, L, n, ins);
+  ins[4] = {qv, static_cast<size_t>(nq) * q->d * dtype_size(dtype)};
+  ins[5] = {workspace, ws_bytes};
+  Range outs[2] = {{scores, topk > 0 ? static_cast<size_t>(nq) * topk * 4 : static_cast<size_t>(nq) * n * 4},
+                   {topk > 0 ? ids : nullptr, static_cast<size_t>(nq) * topk * 4}};
+  if ((s = check_no_alias(outs, 2, ins, 6)) != TQ_OK) return s;
+
+  const int d = q->d;
+  const int qus = score_qu_stride(q);
+  char* ws = static_cast<char*>(workspace);
+  float* qr = reinterpret_cast<float*>(ws);
+  float* qu = qus ? reinterpret_cast<float*>(ws + (static_cast<size_t>(nq) * d * 4 + 255) / 256 * 256) : nullptr;
+  float* dense = reinterpret_cast<float*>(
+      ws + (static_cast<size_t>(nq) * d * 4 + 255) / 256 * 256 + (static_cast<size_t>(nq) * qus * 4 + 255) / 256 * 256);
+  score_qprep_kernel<<<static_cast<unsigned>(nq), 128, 2 * d * 4, stream>>>(
+      qv, dtype, d, q->kind, q->rot, q->S, q->m, q->k_top, qr, qu, qus);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "score qprep launch");
+  ScoreParams p{};
+  p.kind = q->kind; p.d = d; p.m = qus;
+  p.bmse = q->kind == TQ_KIND_MSE ? q->bits : (q->kind == TQ_KIND_PROD ? q->bits - 1 : 0);
+  p.codes = keys.codes; p.code_words = L.code_words;
+  p.signs = keys.signs; p.sign_words = L.sign_words;
+  p.norms = keys.norms; p.rnorms = keys.rnorms;
+  p.centroids = q->centroids;
+  p.k_top = q->k_top; p.tail_bits = q->tail_bits; p.qjl = q->qjl;
+  for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];
+  p.head_words = q->kind == TQ_KIND_SPECTRAL ? (spectral_head_bits(q) + 31) / 32 : 0;
+  p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids;
+  p.coef = q->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / q->m)
+                                   : static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, q->k_top));
+  p.qu_stride = std::max(qus, 1);
+  p.n = n;
+  const size_t smem = static_cast<size_t>(kScoreQT) * (d + p.qu_stride) * 4 + 256 * 4;
+  e = cudaFuncSetAttribute(score_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "score attribute");
+  const int64_t qb = topk > 0 ? score_block(nq, n) : nq;
+  for (int64_t q0 = 0; q0 < nq; q0 += qb) {
+    const int64_t nb = std::min(qb, nq - q0);
+    p.qr = qr + q0 * d;
+    p.qu = qu ? qu + q0 * qus : nullptr;
+    p.nq = nb;
+    p.out = topk > 0 ? dense : scores + q0 * n;
+    const dim3 grid(static_cast<unsigned>((n + kScoreThreads - 1) / kScoreThreads),
+                    static_cast<unsigned>((nb + kScoreQT - 1) / kScoreQT));
+    if (grid.y > 65535) return fail(TQ_ERR_UNSUPPORTED, "too many queries per block");
+    score_dense_kernel<<<grid, kScoreThreads, smem, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+    if (topk > 0) {
+      if (topk <= 16) topk_kernel<16><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+      else topk_kernel<32><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+    }
+  }
+  return TQ_OK;
+}
+
+tq_status tq_decode_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,
+                                   size_t* bytes) {
+  tq_status s = check_quantizer(kq);
+  if (s != TQ_OK) return s;
+  if (!bytes || B < 1 || Hq < 1 || Hkv < 1 || Nmax < 1) return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
+  *bytes = plan_decode(kq, B, Hq, Hkv, Nmax).bytes;
+  return TQ_OK;
+}
+
+tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const void* q, int32_t dtype, int32_t B,
+                         int32_t Hq, int32_t Hkv, int64_t Nmax, const int32_t* seq_lens, tq_packed kc,
+                         tq_packed vc, float scale, float* out, void* workspace, size_t ws_bytes,
+                         tq_stream stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  tq_status s = check_decode_shape(kq, vq, B, Hq, Hkv, Nmax);
+  if (s != TQ_OK) return s;
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
+  if (!aligned16(q) || !aligned16(seq_lens) || !aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "q/seq_lens/out alignment");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
+  const tq_layout LK = layout_of(kq), LV = layout_of(vq);
+  if ((s = check_packed(kc, LK)) != TQ_OK) return s;
+  if ((s = check_packed(vc, LV)) != TQ_OK) return s;
+  const DecodePlan P = plan_decode(kq, B, Hq, Hkv, Nmax);
+  if (!workspace || ws_bytes < P.bytes) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", P.bytes);
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  const int64_t recs = static_cast<int64_t>(B) * Hkv * Nmax;
+  Range ins[11];
+  packed_ranges(kc, LK, recs, ins);
+  packed_ranges(vc, LV, recs, ins + 4);
+  ins[8] = {q, static_cast<size_t>(B) * Hq * kq->d * dtype_size(dtype)};
+  ins[9] = {seq_lens, static_cast<size_t>(B) * 4};
+  ins[10] = {workspace, ws_bytes};
+  const Range outs[1] = {{out, static_cast<size_t>(B) * Hq * kq->d * 4}};
+  if ((s = check_no_alias(outs, 1, ins, 11)) != TQ_OK) return s;
+
+  const int D = kq->d, G = Hq / Hkv, rows = B * Hq;
+  char* ws = static_cast<char*>(workspace);
+  float* qa = reinterpret_cast<float*>(ws + P.off_qa);
+  float* qb = reinterpret_cast<float*>(ws + P.off_qb);
+  float* qs = reinterpret_cast<float*>(ws + P.off_qs);
+  float* pml = reinterpret_cast<float*>(ws + P.off_ml);
+  float* po = reinterpret_cast<float*>(ws + P.off_o);
+
+  QPrepParams qp{};
+  qp.q = q; qp.dtype = dtype; qp.rows = rows; qp.D = D; qp.kind = kq->kind;
+  qp.scale = scale * kLog2e;
+  qp.rot = kq->rot; qp.S = kq->S; qp.m = kq->m;
+  qp.dim_sigma = kq->dim_sigma; qp.k_top = kq->k_top; qp.qjl = kq->qjl;
+  qp.spec_coef = static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, kq->k_top));
+  qp.qa = qa; qp.qb = qb; qp.qs = qs; qp.qb_stride = P.qb_stride;
+  const size_t qsm = static_cast<size_t>(2 * D + std::max(D, P.qb_stride)) * 4;
+  qprep_kernel<<<rows, 128, qsm, stream>>>(qp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "qprep launch");
+
+  DecodeParams dp{};
+  dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.G = G; dp.Nmax = Nmax;
+  dp.chunk_len = P.chunk_len; dp.n_chunks = P.n_chunks; dp.seq_lens = seq_lens;
+  dp.kcodes = kc.codes; dp.k_words = LK.code_words; dp.ksigns = kc.signs; dp.k_sign_words = LK.sign_words;
+  dp.knorms = kc.norms; dp.krnorms = kc.rnorms;
+  dp.vcodes = vc.codes; dp.v_words = LV.code_words; dp.vnorms = vc.norms;
+  dp.unit_c = kq->kind == TQ_KIND_SPECTRAL ? kq->unit_centroids : nullptr;
+  int kfmt, kb, vfmt, vb;
+  if (kq->kind == TQ_KIND_SPECTRAL) {
+    kfmt = KFMT_SPEC; kb = kq->tail_bits;
+    dp.k_code_off = (spectral_head_bits(kq) + 31) / 32;
+    dp.kc = kq->unit_centroids + unit_c_off(kb);
+    dp.k_top_k = kq->k_top; dp.k_qjl = kq->qjl;
+    for (int j = 0; j < TQ_MAX_TOP; ++j) dp.k_top_bits[j] = kq->top_bits[j];
+  } else {
+    kfmt = kq->kind == TQ_KIND_PROD ? KFMT_PROD : KFMT_MSE;
+    kb = kq->kind == TQ_KIND_PROD ? kq->bits - 1 : kq->bits;
+    dp.k_code_off = 0;
+    dp.kc = kq->centroids;
+  }
+  if (vq->kind == TQ_KIND_SPECTRAL) {
+    vfmt = VFMT_SPEC; vb = vq->tail_bits;
+    dp.v_code_off = (spectral_head_bits(vq) + 31) / 32;
+    dp.vc = vq->unit_centroids + unit_c_off(vb);
+    dp.v_top = vq->k_top;
+    for (int j = 0; j < TQ_MAX_TOP; ++j) dp.v_top_bits[j] = vq->top_bits[j];
+    if (!dp.unit_c) dp.unit_c = vq->unit_centroids;
+  } else {
+    vfmt = VFMT_MSE; vb = vq->bits;
+    dp.v_code_off = 0;
+    dp.vc = vq->centroids;
+  }
+  dp.qa = qa; dp.qb = qb; dp.qs = qs; dp.qb_stride = P.qb_stride;
+  dp.qjl_coef = kq->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / kq->m) : 0.f;
+  dp.part_ml = pml; dp.part_o = po;
+  const dim3 grid(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv));
+  const size_t smem = decode_smem_bytes(D, kb, vb);
+  e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream);
+  if (e == cudaErrorNotSupported) return fail(TQ_ERR_UNSUPPORTED, "decode variant not built (kbits %d, vbits %d)", kb, vb);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+
+  CombineParams cp{};
+  cp.rows = rows; cp.D = D; cp.n_chunks = P.n_chunks;
+  cp.part_ml = pml; cp.part_o = po; cp.rot_v = vq->rot;
+  cp.v_sigma = vq->kind == TQ_KIND_SPECTRAL ? vq->dim_sigma : nullptr;
+  cp.out = out;
+  combine_kernel<<<rows, 128, static_cast<size_t>(D) * 4, stream>>>(cp);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "combine launch");
+}
+
+tq_status tq_get_status(tq_stream stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_tq_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_tq_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  if (v == TQ_ERR_TIMEOUT) return fail(TQ_ERR_TIMEOUT, "a device-side bounded wait timed out");
+  return v == 0 ? TQ_OK : fail(static_cast<tq_status>(v), "device reported status %d", v);
+}
+
+tq_status tq_set_wait_limit(int64_t polls) {
+  if (polls < 0) return fail(TQ_ERR_INVALID_ARG, "polls < 0");
+  g_wait_limit.store(polls);
+  return TQ_OK;
+}
+
+}  // extern "C"
+
+namespace tq {
+cudaError_t launch_decode(const DecodeParams& p, int kfmt, int kb, int vfmt, int vb, dim3 grid, size_t smem,
+                          cudaStream_t stream) {
+  if (kfmt == KFMT_MSE && vfmt == VFMT_MSE) return launch_decode_mse(p, kb, vb, grid, smem, stream);
+  if (kfmt == KFMT_PROD && vfmt == VFMT_MSE) return launch_decode_prod(p, kb, vb, grid, smem, stream);
+  if (kfmt == KFMT_SPEC && vfmt == VFMT_SPEC) return launch_decode_spec(p, kb, vb, grid, smem, stream);
+  return cudaErrorNotSupported;
+}
+}  // namespace tq

@@ -1,0 +1,25 @@
+// Internal declarations shared by the libtq translation units (host side).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+// Records a thread-local message and returns the status (for `return fail(...)`).
+tq_status fail(tq_status s, const char* fmt, ...);
+
+// Host math (host_math.cpp).
+tq_status codebook_build(int d, int bits, int dist, double sigma, double* c_out, double* t_out,
+                         int* iters_out);
+tq_status waterfill(const double* lambda, int k, int budget, int max_bits, int32_t* out);
+tq_status spectral_calibrate(const float* X, int64_t n, int d, double* vecs, double* vals);
+tq_status spectral_unit_codebooks(double* c_out, double* t_out);
+
+// Device-side status word and wait limit (tq_api.cu).
+int* device_status_ptr();      // address of the current device's status word
+long long wait_limit();        // polls per bounded wait
+
+}  // namespace tq

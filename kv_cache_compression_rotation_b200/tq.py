@@ -1,0 +1,312 @@
+"""ctypes binding of libtq (include/tq.h): argument marshalling only.
+
+Every computation runs in the CUDA library; PyTorch supplies device memory and the
+current stream.  If ``libtq.so`` is missing the first call raises -- there is no CPU
+fallback.  Build it with ``python -m kv_cache_compression_rotation_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK = 0
+STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_INVALID_ARG", 2: "TQ_ERR_UNSUPPORTED", 3: "TQ_ERR_ALIGNMENT",
+                4: "TQ_ERR_ALIAS", 5: "TQ_ERR_CUDA", 6: "TQ_ERR_TIMEOUT", 7: "TQ_ERR_NOT_CONVERGED",
+                8: "TQ_ERR_WORKSPACE"}
+DIST = {"beta": 0, "gaussian": 1}
+KIND_MSE, KIND_PROD, KIND_SPECTRAL = 0, 1, 2
+F32, BF16, F16 = 0, 1, 2
+MAX_TOP = 8
+
+EXPORTS = [
+    "tq_version", "tq_last_error", "tq_codebook_build", "tq_waterfill", "tq_spectral_calibrate",
+    "tq_spectral_unit_codebooks", "tq_record_layout", "tq_quantize_mse", "tq_quantize_prod",
+    "tq_quantize_spectral", "tq_dequantize", "tq_score_workspace", "tq_score",
+    "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit",
+]
+
+
+class TqError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Quantizer_t(C.Structure):
+    _fields_ = [
+        ("kind", C.c_int32), ("d", C.c_int32), ("bits", C.c_int32), ("m", C.c_int32),
+        ("rot", C.c_void_p), ("S", C.c_void_p), ("centroids", C.c_void_p), ("boundaries", C.c_void_p),
+        ("k_top", C.c_int32), ("tail_bits", C.c_int32), ("qjl", C.c_int32),
+        ("top_bits", C.c_int32 * MAX_TOP),
+        ("dim_sigma", C.c_void_p), ("unit_centroids", C.c_void_p), ("unit_boundaries", C.c_void_p),
+    ]
+
+
+class Packed_t(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("signs", C.c_void_p), ("norms", C.c_void_p), ("rnorms", C.c_void_p)]
+
+
+class Layout_t(C.Structure):
+    _fields_ = [("code_words", C.c_int32), ("sign_words", C.c_int32), ("has_norms", C.c_int32),
+                ("has_rnorms", C.c_int32)]
+
+
+_lib_handle = None
+
+
+def lib():
+    """Load libtq.so (raises if it was not built)."""
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libtq.so not found at {LIB_PATH}; build it with "
+                               "`python -m kv_cache_compression_rotation_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, i64, f64p = C.c_void_p, C.c_int32, C.c_int64, C.POINTER(C.c_double)
+        qp = C.POINTER(Quantizer_t)
+        sig = {
+            "tq_version": ([], C.c_char_p),
+            "tq_last_error": ([], C.c_char_p),
+            "tq_codebook_build": ([i32, i32, i32, C.c_double, f64p, f64p, C.POINTER(i32)], C.c_int),
+            "tq_waterfill": ([f64p, i32, i32, i32, C.POINTER(i32)], C.c_int),
+            "tq_spectral_calibrate": ([vp, i64, i32, f64p, f64p], C.c_int),
+            "tq_spectral_unit_codebooks": ([f64p, f64p], C.c_int),
+            "tq_record_layout": ([qp, C.POINTER(Layout_t)], C.c_int),
+            "tq_quantize_mse": ([qp, vp, i32, i64, Packed_t, vp], C.c_int),
+            "tq_quantize_prod": ([qp, vp, i32, i64, Packed_t, vp], C.c_int),
+            "tq_quantize_spectral": ([qp, vp, i32, i64, Packed_t, vp], C.c_int),
+            "tq_dequantize": ([qp, Packed_t, i64, vp, vp], C.c_int),
+            "tq_score_workspace": ([qp, i64, i64, i32, C.POINTER(C.c_size_t)], C.c_int),
+            "tq_score": ([qp, vp, i32, i64, Packed_t, i64, i32, vp, vp, vp, C.c_size_t, vp], C.c_int),
+            "tq_decode_attn_workspace": ([qp, i32, i32, i32, i64, C.POINTER(C.c_size_t)], C.c_int),
+            "tq_decode_attn": ([qp, qp, vp, i32, i32, i32, i32, i64, vp, Packed_t, Packed_t, C.c_float,
+                                vp, vp, C.c_size_t, vp], C.c_int),
+            "tq_get_status": ([vp], C.c_int),
+            "tq_set_wait_limit": ([i64], C.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib_handle = L
+    return _lib_handle
+
+
+def _check(status: int) -> None:
+    if status != TQ_OK:
+        raise TqError(status, lib().tq_last_error().decode())
+
+
+def _dptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}[t.dtype]
+
+
+def version() -> str:
+    return lib().tq_version().decode()
+
+
+# ------------------------------------------------------------------ host math
+def codebook_build(bits: int, dist: str = "beta", d: int = 0, sigma: float = 0.0):
+    """Lloyd-Max codebook: (centroids [2^b], boundaries [2^b-1], iterations) as float64."""
+    k = 1 << bits
+    c = np.zeros(k, dtype=np.float64)
+    t = np.zeros(k - 1, dtype=np.float64)
+    it = C.c_int32(0)
+    _check(lib().tq_codebook_build(d, bits, DIST[dist], float(sigma),
+                                   c.ctypes.data_as(C.POINTER(C.c_double)),
+                                   t.ctypes.data_as(C.POINTER(C.c_double)), C.byref(it)))
+    return c, t, it.value
+
+
+def waterfill(lam, budget: int, max_bits: int = 8) -> np.ndarray:
+    lam = np.ascontiguousarray(lam, dtype=np.float64)
+    out = np.zeros(lam.shape[0], dtype=np.int32)
+    _check(lib().tq_waterfill(lam.ctypes.data_as(C.POINTER(C.c_double)), lam.shape[0], budget, max_bits,
+                              out.ctypes.data_as(C.POINTER(C.c_int32))))
+    return out
+
+
+def spectral_calibrate(X: np.ndarray):
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    n, d = X.shape
+    vecs = np.zeros((d, d), dtype=np.float64)
+    vals = np.zeros(d, dtype=np.float64)
+    _check(lib().tq_spectral_calibrate(X.ctypes.data, n, d, vecs.ctypes.data_as(C.POINTER(C.c_double)),
+                                       vals.ctypes.data_as(C.POINTER(C.c_double))))
+    return vecs, vals
+
+
+def spectral_unit_codebooks():
+    c = np.zeros(510, dtype=np.float64)
+    t = np.zeros(502, dtype=np.float64)
+    _check(lib().tq_spectral_unit_codebooks(c.ctypes.data_as(C.POINTER(C.c_double)),
+                                            t.ctypes.data_as(C.POINTER(C.c_double))))
+    return c, t
+
+
+# ------------------------------------------------------------------ descriptors
+@dataclass
+class Packed:
+    """Packed records (structure of arrays) on the device."""
+    codes: object
+    signs: object = None
+    norms: object = None
+    rnorms: object = None
+
+    def as_c(self) -> Packed_t:
+        return Packed_t(_dptr(self.codes) if self.codes is not None and self.codes.numel() else None,
+                        _dptr(self.signs), _dptr(self.norms), _dptr(self.rnorms))
+
+
+class Quantizer:
+    """Device-resident quantizer descriptor (owns the tensors the C struct points at)."""
+
+    def __init__(self, kind: int, d: int, rot, *, bits=0, m=0, S=None, centroids=None, boundaries=None,
+                 k_top=0, tail_bits=0, qjl=0, top_bits=(), dim_sigma=None, unit_c=None, unit_t=None):
+        self.kind, self.d, self.bits, self.m = kind, d, bits, m
+        self._keep = [rot, S, centroids, boundaries, dim_sigma, unit_c, unit_t]
+        self.rot, self.S, self.centroids, self.boundaries = rot, S, centroids, boundaries
+        self.dim_sigma, self.unit_c, self.unit_t = dim_sigma, unit_c, unit_t
+        self.k_top, self.tail_bits, self.qjl, self.top_bits = k_top, tail_bits, qjl, tuple(top_bits)
+        tb = (C.c_int32 * MAX_TOP)(*(list(top_bits) + [0] * (MAX_TOP - len(top_bits))))
+        self.c = Quantizer_t(kind, d, bits, m, _dptr(rot), _dptr(S), _dptr(centroids), _dptr(boundaries),
+                             k_top, tail_bits, qjl, tb, _dptr(dim_sigma), _dptr(unit_c), _dptr(unit_t))
+
+    @property
+    def ref(self):
+        return C.byref(self.c)
+
+    @staticmethod
+    def _dev(a, device):
+        import torch
+        return torch.as_tensor(np.ascontiguousarray(a, dtype=np.float32), device=device).contiguous()
+
+    @classmethod
+    def mse(cls, rot, bits: int, dist: str = "beta", sigma: float = 0.0, device="cuda"):
+        d = rot.shape[0]
+        c, t, _ = codebook_build(bits, dist, d=d, sigma=sigma)
+        return cls(KIND_MSE, d, cls._dev(rot, device), bits=bits,
+                   centroids=cls._dev(c, device), boundaries=cls._dev(t, device))
+
+    @classmethod
+    def prod(cls, rot, S, bits: int, dist: str = "beta", sigma: float = 0.0, device="cuda"):
+        d = rot.shape[0]
+        m = S.shape[0]
+        cen = bnd = None
+        if bits > 1:
+            c, t, _ = codebook_build(bits - 1, dist, d=d, sigma=sigma)
+            cen, bnd = cls._dev(c, device), cls._dev(t, device)
+        return cls(KIND_PROD, d, cls._dev(rot, device), bits=bits, m=m, S=cls._dev(S, device),
+                   centroids=cen, boundaries=bnd)
+
+    @classmethod
+    def spectral(cls, eigvecs, eigvals, k_top: int, top_bits, tail_bits: int, qjl: bool, S_top=None,
+                 device="cuda"):
+        d = eigvecs.shape[0]
+        uc, ut = spectral_unit_codebooks()
+        sig = np.sqrt(np.maximum(np.asarray(eigvals, dtype=np.float64), 0.0))
+        return cls(KIND_SPECTRAL, d, cls._dev(eigvecs, device), S=None if S_top is None else cls._dev(S_top, device),
+                   k_top=k_top, tail_bits=tail_bits, qjl=1 if qjl else 0, top_bits=list(top_bits),
+                   dim_sigma=cls._dev(sig, device), unit_c=cls._dev(uc, device), unit_t=cls._dev(ut, device))
+
+    def layout(self) -> Layout_t:
+        L = Layout_t()
+        _check(lib().tq_record_layout(self.ref, C.byref(L)))
+        return L
+
+    def alloc(self, n: int, device="cuda") -> Packed:
+        """Zeroed packed arrays for n records."""
+        import torch
+        L = self.layout()
+        codes = torch.zeros((n, L.code_words), dtype=torch.int32, device=device)
+        signs = torch.zeros((n, L.sign_words), dtype=torch.int32, device=device) if L.sign_words else None
+        norms = torch.zeros(n, dtype=torch.float32, device=device) if L.has_norms else None
+        rnorms = torch.zeros(n, dtype=torch.float32, device=device) if L.has_rnorms else None
+        return Packed(codes, signs, norms, rnorms)
+
+
+# ------------------------------------------------------------------ device calls
+def quantize(q: Quantizer, x, out: Optional[Packed] = None, stream=None) -> Packed:
+    """tq_quantize_{mse,prod,spectral} of x [n, d] (fp32 / bf16 / fp16 CUDA tensor)."""
+    assert x.is_cuda and x.is_contiguous() and x.shape[-1] == q.d
+    n = x.numel() // q.d
+    out = q.alloc(n, x.device) if out is None else out
+    fn = {KIND_MSE: lib().tq_quantize_mse, KIND_PROD: lib().tq_quantize_prod,
+          KIND_SPECTRAL: lib().tq_quantize_spectral}[q.kind]
+    _check(fn(q.ref, x.data_ptr(), _dtype_code(x), n, out.as_c(), _stream(stream)))
+    return out
+
+
+def dequantize(q: Quantizer, packed: Packed, n: int, stream=None):
+    import torch
+    out = torch.empty((n, q.d), dtype=torch.float32, device=packed.codes.device)
+    _check(lib().tq_dequantize(q.ref, packed.as_c(), n, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def score(q: Quantizer, qv, packed: Packed, n: int, topk: int = 0, stream=None):
+    """Dense estimates [nq, n], or (scores [nq, topk], ids [nq, topk]) when topk > 0."""
+    import torch
+    nq = qv.numel() // q.d
+    ws = C.c_size_t(0)
+    _check(lib().tq_score_workspace(q.ref, nq, n, topk, C.byref(ws)))
+    work = torch.empty(max(ws.value, 16), dtype=torch.uint8, device=qv.device)
+    if topk == 0:
+        scores = torch.empty((nq, n), dtype=torch.float32, device=qv.device)
+        ids = None
+    else:
+        scores = torch.empty((nq, topk), dtype=torch.float32, device=qv.device)
+        ids = torch.empty((nq, topk), dtype=torch.int32, device=qv.device)
+    _check(lib().tq_score(q.ref, qv.data_ptr(), _dtype_code(qv), nq, packed.as_c(), n, topk, scores.data_ptr(),
+                          _dptr(ids), work.data_ptr(), ws.value, _stream(stream)))
+    return scores if topk == 0 else (scores, ids)
+
+
+def decode_workspace_bytes(kq: Quantizer, B: int, Hq: int, Hkv: int, Nmax: int) -> int:
+    ws = C.c_size_t(0)
+    _check(lib().tq_decode_attn_workspace(kq.ref, B, Hq, Hkv, Nmax, C.byref(ws)))
+    return ws.value
+
+
+def decode_attn(kq: Quantizer, vq: Quantizer, q, seq_lens, kcache: Packed, vcache: Packed, Nmax: int,
+                Hkv: int, scale: Optional[float] = None, out=None, workspace=None, stream=None):
+    """One decode-attention step; q [B, Hq, d], seq_lens int32 [B] on the device."""
+    import torch
+    B, Hq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = decode_workspace_bytes(kq, B, Hq, Hkv, Nmax)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device) if out is None else out
+    _check(lib().tq_decode_attn(kq.ref, vq.ref, q.data_ptr(), _dtype_code(q), B, Hq, Hkv, Nmax,
+                                seq_lens.data_ptr(), kcache.as_c(), vcache.as_c(), float(scale), out.data_ptr(),
+                                workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out
+
+
+def get_status(stream=None) -> int:
+    """Synchronize and return the device status code (0 = OK, 6 = a bounded wait timed out)."""
+    return lib().tq_get_status(_stream(stream))
+
+
+def set_wait_limit(polls: int) -> None:
+    _check(lib().tq_set_wait_limit(polls))

@@ -1,0 +1,150 @@
+"""GPU parity: quantize / dequantize through the C ABI against the oracle."""
+import math
+
+import numpy as np
+import pytest
+
+import tq_inputs as ti
+from oracle import quantizer as OQ
+from oracle import spectral as OSP
+from oracle.codebook import lloyd_max
+
+from _parity import as_u32, code_mismatches, sign_mismatches
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+K = pytest.importorskip("kv_cache_compression_rotation_b200")
+
+
+def _inputs(n, d, dtype, seed, zero_rows=()):
+    x = ti.anisotropic(n, d, ti.haar_rotation(d, seed + 1).astype(np.float64), seed, lam=None) \
+        if d == 128 else ti.iid_normal((n, d), seed) * 2.0
+    for r in zero_rows:
+        x[r] = 0.0
+    if dtype == "bf16":
+        xt, x64 = ti.to_bf16_f64(x)
+    elif dtype == "f16":
+        xt = torch.from_numpy(x.astype(np.float16))
+        x64 = xt.to(torch.float64).numpy()
+    else:
+        xt = torch.from_numpy(x.astype(np.float32))
+        x64 = xt.to(torch.float64).numpy()
+    return xt.cuda().contiguous(), x64
+
+
+MSE_CASES = [
+    # d, bits, dtype, n   (d=128 16-bit input, bits <= 4 runs the tensor-core kernel)
+    (128, 3, "f32", 4096),
+    (128, 4, "bf16", 1000),
+    (128, 4, "bf16", 128 * 148 * 2 + 37),
+    (128, 1, "bf16", 5000),
+    (128, 2, "bf16", 5000),
+    (128, 3, "bf16", 5000),
+    (128, 4, "f16", 3000),
+    (128, 4, "bf16", 1),
+    (8, 2, "f32", 777),
+    (32, 5, "f32", 300),
+    (96, 6, "bf16", 100),
+    (1536, 4, "bf16", 64),
+]
+
+
+@pytest.mark.parametrize("d,bits,dtype,n", MSE_CASES)
+def test_quantize_mse_parity(d, bits, dtype, n):
+    rot = ti.haar_rotation(d, 1000 + d)
+    x, x64 = _inputs(n, d, dtype, 4000 + d + bits, zero_rows=[0] if n > 10 else [])
+    q = K.Quantizer.mse(rot, bits)
+    out = K.quantize(q, x)
+    torch.cuda.synchronize()
+    assert K.get_status() == 0
+    c, t, _ = lloyd_max(bits, "beta", d=d)
+    ref = OQ.quantize_mse(x64, rot, c, t, bits)
+    bad, exempt, _ = code_mismatches(as_u32(out.codes), ref["codes"], d, bits, ref["y"], t)
+    assert bad == 0, f"{bad} code mismatches outside the band ({exempt} exempt)"
+    assert exempt <= max(2, 1e-4 * n * d)
+    nrm = out.norms.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(nrm - ref["norms"]) <= 1e-5 * np.maximum(ref["norms"], 1e-30))
+    # reconstruction from the GPU's own records matches the oracle's (records without exemptions)
+    xh = K.dequantize(q, out, n).cpu().numpy().astype(np.float64)
+    xr = OQ.dequantize_mse(ref["idx"], ref["norms"], rot, c)
+    same = np.all(as_u32(out.codes) == ref["codes"], axis=1)
+    err = np.max(np.abs(xh[same] - xr[same]), axis=1) / np.maximum(ref["norms"][same], 1e-30)
+    assert np.all(err < 1e-5)
+
+
+@pytest.mark.parametrize("d,bits,m,dtype,n", [(128, 3, 128, "bf16", 2000), (64, 2, 64, "f32", 500),
+                                              (128, 1, 128, "f32", 300), (128, 5, 256, "bf16", 400)])
+def test_quantize_prod_parity(d, bits, m, dtype, n):
+    rot = ti.haar_rotation(d, 1100 + d)
+    S = ti.gaussian_matrix(m, d, 2000 + d)
+    x, x64 = _inputs(n, d, dtype, 4100 + d + bits)
+    q = K.Quantizer.prod(rot, S, bits)
+    out = K.quantize(q, x)
+    if bits > 1:
+        c, t, _ = lloyd_max(bits - 1, "beta", d=d)
+    else:
+        c = t = None
+    ref = OQ.quantize_prod(x64, rot, S, c, t, bits)
+    skip = set()
+    if bits > 1:
+        bad, exempt, skip = code_mismatches(as_u32(out.codes), ref["codes"], d, bits - 1, ref["y"], t)
+        assert bad == 0
+    sbad, sex = sign_mismatches(as_u32(out.signs), ref["signs"], m, ref["proj"], S, skip)
+    assert sbad == 0, f"{sbad} sign mismatches outside the band"
+    assert sex <= max(3, 2e-3 * n)
+    rn = out.rnorms.cpu().numpy().astype(np.float64)
+    ok = np.array([i not in skip for i in range(n)])
+    assert np.all(np.abs(rn[ok] - ref["rnorms"][ok]) <= 1e-5 * np.maximum(ref["rnorms"][ok], 1e-6) + 1e-6)
+    nrm = out.norms.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(nrm - ref["norms"]) <= 1e-5 * ref["norms"])
+    xh = K.dequantize(q, out, n).cpu().numpy().astype(np.float64)
+    xr = OQ.dequantize_prod(ref["chat"], ref["s"], ref["norms"], ref["rnorms"], rot, S)
+    same = np.all(as_u32(out.signs) == ref["signs"], axis=1) & ok
+    err = np.max(np.abs(xh[same] - xr[same]), axis=1) / ref["norms"][same]
+    assert np.all(err < 1e-4)
+
+
+def _spectral_desc(qjl, d=128):
+    """Quantizer inputs: the generator's own basis and spectrum stand in for a calibration."""
+    U = ti.haar_rotation(d, 3004).astype(np.float64)
+    lam = d * ti.kv_spectrum(d)
+    S4 = ti.gaussian_matrix(4, 4, 2004)
+    rot = U.T.astype(np.float32)                     # row j = eigenvector j
+    desc = OSP.build_descriptor(rot.astype(np.float64), lam, 4, 12, 1, qjl, S4)
+    return U, rot, lam, S4, desc
+
+
+@pytest.mark.parametrize("qjl", [True, False])
+def test_quantize_spectral_parity(qjl):
+    d, n = 128, 3000
+    U, rot, lam, S4, desc = _spectral_desc(qjl)
+    xt, x64 = ti.to_bf16_f64(ti.anisotropic(n, d, U, 4004))
+    q = K.Quantizer.spectral(rot, lam, 4, list(desc["bits"][:4]), 1, qjl, S4 if qjl else None)
+    out = K.quantize(q, xt.cuda())
+    ref = OSP.quantize_spectral(x64, desc)
+    g = as_u32(out.codes)
+    rows = np.nonzero(np.any(g != ref["codes"], axis=1))[0]
+    # every differing record must have a coordinate within 1e-5 ||x|| of one of its dim's
+    # boundaries (or a QJL projection within 1e-5 ||S_i|| ||x|| of zero)
+    xn = np.linalg.norm(x64, axis=1)
+    for i in rows:
+        dmin = np.inf
+        for j in range(d):
+            b = int(desc["bits"][j])
+            tt = desc["books"][b][1] * desc["sigma"][j]
+            dmin = min(dmin, np.min(np.abs(ref["z"][i, j] - tt)))
+        if qjl:
+            dmin = min(dmin, np.min(np.abs(ref["proj"][i]) / np.linalg.norm(S4, axis=1)))
+        assert dmin <= 1e-5 * xn[i], f"record {i} differs outside the band"
+    assert len(rows) <= max(3, 1e-3 * n)
+    if qjl:
+        rn = out.rnorms.cpu().numpy()
+        ok = np.ones(n, dtype=bool)
+        ok[rows] = False
+        assert np.all(np.abs(rn[ok] - ref["rnorms"][ok]) <= 1e-5 * np.maximum(ref["rnorms"][ok], 1e-3))
+    xh = K.dequantize(q, out, n).cpu().numpy()
+    xr = OSP.dequantize_spectral(ref["chat"], desc)
+    ok = np.ones(n, dtype=bool)
+    ok[rows] = False
+    assert np.max(np.abs(xh[ok] - xr[ok])) < 1e-4 * np.max(np.abs(xr))

@@ -1,0 +1,82 @@
+"""GPU parity: inner-product estimates and exhaustive top-k vs the oracle."""
+import numpy as np
+import pytest
+
+import tq_inputs as ti
+from oracle import quantizer as OQ
+from oracle.codebook import lloyd_max
+from oracle.search import topk as otopk
+
+from _parity import as_u32
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+K = pytest.importorskip("kv_cache_compression_rotation_b200")
+
+
+def test_scores_c1_mse_fp32():
+    """Single head d=128, 4096 fp32 keys ~ N(0, 1/d), 64 queries, mse b=3."""
+    d, n, nq, b = 128, 4096, 64, 3
+    rot = ti.haar_rotation(d, 1001)
+    x = ti.iid_normal((n, d), 4001, std=1 / np.sqrt(d)).astype(np.float32)
+    qv = ti.iid_normal((nq, d), 6001, std=1 / np.sqrt(d)).astype(np.float32)
+    q = K.Quantizer.mse(rot, b)
+    pk = K.quantize(q, torch.from_numpy(x).cuda())
+    s = K.score(q, torch.from_numpy(qv).cuda(), pk, n).cpu().numpy().astype(np.float64)
+    c, t, _ = lloyd_max(b, "beta", d=d)
+    ref = OQ.quantize_mse(x.astype(np.float64), rot, c, t, b)
+    same = np.all(as_u32(pk.codes) == ref["codes"], axis=1)
+    est = OQ.estimate_mse(qv.astype(np.float64), rot, ref["idx"], ref["norms"], c)
+    scale = np.linalg.norm(qv, axis=1)[:, None] * np.linalg.norm(x, axis=1)[None, :]
+    assert np.all(np.abs(s - est)[:, same] <= 1e-3 * scale[:, same])
+    assert same.mean() > 0.99
+    # quality context: estimates vs exact inner products (MSE stage is biased by 1 - D_3)
+    exact = qv.astype(np.float64) @ x.astype(np.float64).T
+    slope = np.sum(est * exact) / np.sum(exact * exact)
+    assert 0.9 < slope < 1.0
+
+
+@pytest.mark.parametrize("d,bits,n,nq", [(128, 3, 3000, 16), (1536, 2, 2000, 8), (1536, 4, 1000, 8)])
+def test_scores_prod(d, bits, n, nq):
+    rot = ti.haar_rotation(d, 1005)
+    S = ti.gaussian_matrix(d, d, 2005)
+    x = ti.unit_gaussian(n, d, 8000).astype(np.float32)
+    qv = ti.unit_gaussian(nq, d, 8001).astype(np.float32)
+    q = K.Quantizer.prod(rot, S, bits)
+    pk = K.quantize(q, torch.from_numpy(x).cuda())
+    s = K.score(q, torch.from_numpy(qv).cuda(), pk, n).cpu().numpy().astype(np.float64)
+    c, t, _ = lloyd_max(bits - 1, "beta", d=d)
+    ref = OQ.quantize_prod(x.astype(np.float64), rot, S, c, t, bits)
+    same = np.all(as_u32(pk.codes) == ref["codes"], axis=1) & np.all(as_u32(pk.signs) == ref["signs"], axis=1)
+    est = OQ.estimate_prod(qv.astype(np.float64), rot, S, ref["chat"], ref["s"], ref["norms"], ref["rnorms"])
+    assert np.all(np.abs(s - est)[:, same] <= 1e-3)       # unit-norm q and x
+    assert same.mean() > 0.99
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_topk_search(bits):
+    """Exhaustive top-10 by estimated inner product (unit-norm Gaussian DB, d=1536)."""
+    d, n, nq, k = 1536, 20000, 12, 10
+    rot = ti.haar_rotation(d, 1005)
+    S = ti.gaussian_matrix(d, d, 2005)
+    x = ti.unit_gaussian(n, d, 8000).astype(np.float32)
+    qv = ti.unit_gaussian(nq, d, 8001).astype(np.float32)
+    q = K.Quantizer.prod(rot, S, bits)
+    pk = K.quantize(q, torch.from_numpy(x).cuda())
+    vals, ids = K.score(q, torch.from_numpy(qv).cuda(), pk, n, topk=k)
+    vals, ids = vals.cpu().numpy().astype(np.float64), ids.cpu().numpy()
+    c, t, _ = lloyd_max(bits - 1, "beta", d=d)
+    ref = OQ.quantize_prod(x.astype(np.float64), rot, S, c, t, bits)
+    est = OQ.estimate_prod(qv.astype(np.float64), rot, S, ref["chat"], ref["s"], ref["norms"], ref["rnorms"])
+    rid, rval = otopk(est, k)
+    tol = 1e-3
+    for i in range(nq):
+        # the GPU's list is sorted, its scores match the oracle's estimates of the same ids,
+        # and every id the oracle ranks clearly inside the top-k is present
+        assert np.all(np.diff(vals[i]) <= 0)
+        assert np.all(np.abs(vals[i] - est[i, ids[i]]) <= tol)
+        kth = rval[i, -1]
+        must = rid[i][rval[i] > kth + 2 * tol]
+        assert set(must.tolist()) <= set(ids[i].tolist())
+        assert np.all(est[i, ids[i]] >= kth - 2 * tol)

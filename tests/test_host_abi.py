@@ -1,0 +1,217 @@
+"""libtq host functions and C-ABI checks that need no GPU.
+
+The library must load and export every entry point include/tq.h declares; its host math
+(codebooks, water-filling, calibration) must agree with the oracle; argument validation
+must reject bad calls before any launch.
+"""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import tq_inputs as ti
+from oracle import spectral as OSP
+from oracle.codebook import lloyd_max
+
+K = pytest.importorskip("kv_cache_compression_rotation_b200")
+T = K.tq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(T.LIB_PATH):
+        from kv_cache_compression_rotation_b200 import build as B
+        B.build()
+    return T.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(T.EXPORTS)
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(T, "LIB_PATH", "/nonexistent/libtq.so")
+    monkeypatch.setattr(T, "_lib_handle", None)
+    with pytest.raises(RuntimeError):
+        T.lib()
+
+
+@pytest.mark.parametrize("dist,d,bits", [("beta", 128, b) for b in (1, 2, 3, 4, 5)] +
+                         [("beta", 1536, b) for b in (1, 2, 3, 4)] +
+                         [("beta", 8, b) for b in (1, 2, 3)] + [("beta", 2, 3), ("beta", 3, 2)] +
+                         [("gaussian", None, b) for b in (1, 2, 3, 4, 5)])
+def test_codebook_matches_oracle(lib, dist, d, bits):
+    sigma = 0.37 if dist == "gaussian" else 0.0
+    c, t, it = K.codebook_build(bits, dist, d=d or 0, sigma=sigma)
+    co, to, _ = lloyd_max(bits, dist, d=d, sigma=sigma or None)
+    # both stop at a largest move of 1e-13 * scale; the distance to the fixed point is
+    # that move over (1 - contraction rate), far below 1e-9 relative for b <= 5
+    assert np.max(np.abs(c - co) / np.abs(co)) < 1e-9
+    assert np.max(np.abs(t - to)) < 1e-9 * np.max(np.abs(co))
+    assert it >= 1
+
+
+def test_codebook_rejects_bad_args(lib):
+    with pytest.raises(T.TqError):
+        K.codebook_build(0, "beta", d=128)
+    with pytest.raises(T.TqError):
+        K.codebook_build(3, "beta", d=1)
+    with pytest.raises(T.TqError):
+        K.codebook_build(3, "gaussian", sigma=-1.0)
+
+
+def test_waterfill_matches_oracle(lib):
+    rng = np.random.Generator(np.random.PCG64(7))
+    for _ in range(50):
+        k = int(rng.integers(1, 9))
+        lam = rng.uniform(0.001, 1.0, size=k)
+        budget = int(rng.integers(0, 30))
+        assert list(K.waterfill(lam, budget, 8)) == list(OSP.waterfill(lam, budget, 8))
+    assert list(K.waterfill(ti.kv_spectrum(128)[:4], 12)) == [5, 3, 2, 2]
+
+
+def test_calibration_matches_oracle(lib):
+    d, n = 128, 4096
+    U = ti.haar_rotation(d, 3004).astype(np.float64)
+    X = ti.anisotropic(n, d, U, 7000).astype(np.float32)
+    v, w = K.spectral_calibrate(X)
+    vo, wo = OSP.calibrate(X.astype(np.float64))
+    assert np.max(np.abs(w - wo) / np.abs(wo).max()) < 1e-9
+    # well-separated leading eigenvectors agree exactly, including the sign rule
+    for j in range(4):
+        assert np.max(np.abs(v[j] - vo[j])) < 1e-8
+    # the tail is nearly degenerate: compare the projector onto it
+    P = v[4:].T @ v[4:]
+    Po = vo[4:].T @ vo[4:]
+    assert np.max(np.abs(P - Po)) < 1e-8
+    assert np.max(np.abs(v @ v.T - np.eye(d))) < 1e-10
+
+
+def test_unit_codebooks(lib):
+    c, t = K.spectral_unit_codebooks()
+    for b in range(1, 9):
+        co, to, _ = lloyd_max(b, "gaussian", sigma=1.0) if b <= 6 else (None, None, None)
+        if co is None:
+            continue
+        off_c, off_t = (1 << b) - 2, (1 << b) - b - 1
+        assert np.max(np.abs(c[off_c:off_c + (1 << b)] - co)) < 1e-9 * np.max(np.abs(co))
+        assert np.max(np.abs(t[off_t:off_t + (1 << b) - 1] - to)) < 1e-9 * np.max(np.abs(co))
+
+
+FAKE = 0x10000  # 16-byte aligned placeholder device address (never dereferenced here)
+
+
+def _q(kind, d=128, bits=3, m=0, **kw):
+    q = T.Quantizer_t()
+    q.kind, q.d, q.bits, q.m = kind, d, bits, m
+    q.rot = FAKE
+    q.centroids = FAKE + 0x1000
+    q.boundaries = FAKE + 0x2000
+    q.S = kw.get("S", None)
+    q.k_top = kw.get("k_top", 0)
+    q.tail_bits = kw.get("tail_bits", 0)
+    q.qjl = kw.get("qjl", 0)
+    for i, b in enumerate(kw.get("top_bits", [])):
+        q.top_bits[i] = b
+    q.dim_sigma = kw.get("dim_sigma", None)
+    q.unit_centroids = kw.get("unit_c", None)
+    q.unit_boundaries = kw.get("unit_t", None)
+    return q
+
+
+def _layout(lib, q):
+    L = T.Layout_t()
+    st = lib.tq_record_layout(C.byref(q), C.byref(L))
+    return st, L
+
+
+def test_record_layouts(lib):
+    st, L = _layout(lib, _q(T.KIND_MSE, bits=4))
+    assert st == 0 and (L.code_words, L.sign_words, L.has_norms, L.has_rnorms) == (16, 0, 1, 0)
+    st, L = _layout(lib, _q(T.KIND_MSE, bits=3))
+    assert st == 0 and L.code_words == 12
+    st, L = _layout(lib, _q(T.KIND_PROD, bits=3, m=128, S=FAKE))
+    assert st == 0 and (L.code_words, L.sign_words, L.has_norms, L.has_rnorms) == (8, 4, 1, 1)
+    st, L = _layout(lib, _q(T.KIND_PROD, d=1536, bits=2, m=1536, S=FAKE))
+    assert st == 0 and (L.code_words, L.sign_words) == (48, 48)
+    st, L = _layout(lib, _q(T.KIND_SPECTRAL, k_top=4, top_bits=[5, 3, 2, 2], tail_bits=1, qjl=1, S=FAKE,
+                             dim_sigma=FAKE, unit_c=FAKE, unit_t=FAKE))
+    assert st == 0 and (L.code_words, L.has_norms, L.has_rnorms) == (5, 0, 1)
+    st, L = _layout(lib, _q(T.KIND_SPECTRAL, k_top=4, top_bits=[5, 3, 2, 2], tail_bits=1, qjl=0,
+                             dim_sigma=FAKE, unit_c=FAKE, unit_t=FAKE))
+    assert st == 0 and (L.code_words, L.has_rnorms) == (5, 0)
+
+
+@pytest.mark.parametrize("mut,code", [
+    (lambda q: setattr(q, "d", 1), 1), (lambda q: setattr(q, "bits", 9), 1),
+    (lambda q: setattr(q, "rot", None), 1), (lambda q: setattr(q, "rot", FAKE + 4), 3),
+    (lambda q: setattr(q, "kind", 7), 1), (lambda q: setattr(q, "centroids", None), 1),
+])
+def test_descriptor_validation(lib, mut, code):
+    q = _q(T.KIND_MSE, bits=3)
+    mut(q)
+    st, _ = _layout(lib, q)
+    assert st == code
+    assert lib.tq_last_error()
+
+
+def test_quantize_validation_before_launch(lib):
+    q = _q(T.KIND_MSE, bits=3)
+    pk = T.Packed_t(FAKE + 0x100000, None, FAKE + 0x200000, None)
+    # kind mismatch, unknown dtype, misaligned input, aliasing output, n == 0 (no launch)
+    assert lib.tq_quantize_prod(C.byref(q), FAKE + 0x300000, 0, 10, pk, None) == 1
+    assert lib.tq_quantize_mse(C.byref(q), FAKE + 0x300000, 9, 10, pk, None) == 1
+    assert lib.tq_quantize_mse(C.byref(q), FAKE + 0x300002, 0, 10, pk, None) == 3
+    assert lib.tq_quantize_mse(C.byref(q), FAKE + 0x100000, 0, 10, pk, None) == 4
+    assert lib.tq_quantize_mse(C.byref(q), FAKE + 0x300000, 0, 0, pk, None) == 0
+    assert lib.tq_quantize_mse(C.byref(q), None, 0, 10, pk, None) == 1
+    bad = T.Packed_t(None, None, FAKE + 0x200000, None)
+    assert lib.tq_quantize_mse(C.byref(q), FAKE + 0x300000, 0, 10, bad, None) == 1
+
+
+def test_decode_validation_before_launch(lib):
+    kq = _q(T.KIND_MSE, bits=4)
+    vq = _q(T.KIND_MSE, bits=4)
+    pk = T.Packed_t(FAKE + 0x100000, None, FAKE + 0x200000, None)
+    pv = T.Packed_t(FAKE + 0x400000, None, FAKE + 0x500000, None)
+    ws = C.c_size_t(0)
+    assert lib.tq_decode_attn_workspace(C.byref(kq), 2, 8, 2, 1000, C.byref(ws)) == 0 and ws.value > 0
+    args = (FAKE + 0x600000, 1, 2, 8, 2, 1000, FAKE + 0x700000, pk, pv, C.c_float(0.1), FAKE + 0x800000)
+    # workspace too small
+    assert lib.tq_decode_attn(C.byref(kq), C.byref(vq), *args, FAKE + 0x900000, 16, None) == 8
+    # Hq not a multiple of Hkv
+    a2 = list(args); a2[3] = 3
+    assert lib.tq_decode_attn(C.byref(kq), C.byref(vq), *a2, FAKE + 0x900000, ws.value, None) == 1
+    # head dim outside this build
+    k64 = _q(T.KIND_MSE, d=64, bits=4); v64 = _q(T.KIND_MSE, d=64, bits=4)
+    assert lib.tq_decode_attn(C.byref(k64), C.byref(v64), *args, FAKE + 0x900000, 1 << 30, None) == 2
+    # output aliasing the query
+    a3 = list(args); a3[-1] = FAKE + 0x600000
+    assert lib.tq_decode_attn(C.byref(kq), C.byref(vq), *a3, FAKE + 0x900000, ws.value, None) == 4
+
+
+def test_score_validation(lib):
+    q = _q(T.KIND_MSE, bits=3)
+    pk = T.Packed_t(FAKE + 0x100000, None, FAKE + 0x200000, None)
+    ws = C.c_size_t(0)
+    assert lib.tq_score_workspace(C.byref(q), 4, 100, 10, C.byref(ws)) == 0
+    assert lib.tq_score(C.byref(q), FAKE + 0x300000, 0, 4, pk, 100, 40, FAKE + 0x400000, FAKE + 0x500000,
+                        FAKE + 0x600000, ws.value, None) == 2   # topk > 32
+    assert lib.tq_score(C.byref(q), FAKE + 0x300000, 0, 4, pk, 100, 10, FAKE + 0x400000, FAKE + 0x500000,
+                        FAKE + 0x600000, 8, None) == 8          # workspace
+    assert lib.tq_set_wait_limit(-1) == 1
+    assert lib.tq_set_wait_limit(0) == 0
