@@ -96,6 +96,9 @@ typedef struct {
   const float* dim_sigma;       /* SPECTRAL: [d] sqrt(eigenvalue) per dim */
   const float* unit_centroids;  /* SPECTRAL: [510] codebook of b bits at offset 2^b - 2 */
   const float* unit_boundaries; /* SPECTRAL: [502] boundaries of b bits at offset 2^b - b - 1 */
+  float lut_scale;              /* decode/score: shared scale s of the half-precision codebook
+                                   table (entries c_k / s); 0 means 1.  tq_lut_scale picks one
+                                   that keeps every entry within ~1e-4 of c_k. */
 } tq_quantizer;
 
 /*
@@ -163,6 +166,15 @@ tq_status tq_spectral_calibrate(const float* X, int64_t n, int32_t d,
 /* HOST.  Standard-normal codebooks for 1..8 bits in the concatenated layout the
  * SPECTRAL descriptor expects: centroids_out [510], boundaries_out [502]. */
 tq_status tq_spectral_unit_codebooks(double* centroids_out, double* boundaries_out);
+
+/*
+ * HOST.  Shared scale s in [1, 2) for representing `values` [count] (host) in half
+ * precision as s * half(v / s): searches s on a uniform grid of 2^22 points for the
+ * smallest worst-case relative rounding error over the distinct magnitudes.  Decode
+ * attention multiplies products back by s in fp32; the result is written to *scale_out.
+ * This is an encoding detail of the half-precision MMA operands, not part of the method.
+ */
+tq_status tq_lut_scale(const double* values, int32_t count, float* scale_out);
 
 /* HOST.  Words per record and which norm arrays a quantizer writes. */
 tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out);

@@ -18,6 +18,12 @@
 //                The CTA's four warps merge their (max, sum, o') and write one partial.
 //   combine      log-sum-exp merge of the chunks, then o = Pi_V^T o' once per head.
 //
+// Precision: every half-precision MMA operand that is not a table entry is split as
+// hi + lo (two MMAs into the same fp32 accumulator), and the table entries are c_k / s
+// with a shared scale s chosen so that each entry rounds to within ~1e-4 of c_k / s;
+// products are scaled back by s in fp32.  Without these, half-precision rounding of
+// q', p and c alone moves the attention output by ~1e-3 of its largest entry.
+//
 // Dimension mapping: the mma k index is a permutation of the head dims chosen so that
 // each thread reads one contiguous slice of a record; the query operand uses the same
 // permutation, so the inner product is unchanged.
@@ -66,6 +72,7 @@ struct DecodeParams {
   const float* qs;      // [B*Hq][2] scales of qa and qb
   int qb_stride;
   float qjl_coef;       // prod: sqrt(pi/2)/m
+  float k_scale, v_scale; // shared scales of the half-precision codebook tables (entries c/s)
   // partial results
   float* part_ml;       // [B*Hq][n_chunks][2]
   float* part_o;        // [B*Hq][n_chunks][D]
@@ -74,6 +81,15 @@ struct DecodeParams {
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// hi = half(lo_v, hi_v) and lo = half of the rounding residuals.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 back = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - back.x, x1 - back.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -156,18 +172,23 @@ decode_attn_kernel(const DecodeParams p) {
 
   for (int i = tid; i < KLUT * 32; i += kDecThreads) {
     const int e = i >> 5;
-    lutk[i] = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))), __ldg(p.kc + (e >> KB)));
+    lutk[i] = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) / p.k_scale, __ldg(p.kc + (e >> KB)) / p.k_scale);
   }
   for (int i = tid; i < VLUT * 32; i += kDecThreads) {
     const int e = i >> 5;
-    lutv[i] = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))), __ldg(p.vc + (e >> VB)));
+    lutv[i] = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
   }
   if (tid < 128) {
     const int e = tid >> 5;
     luts[tid] = pack_half2((e & 1) ? 1.f : -1.f, (e & 2) ? 1.f : -1.f);
   }
   if constexpr (KF == KFMT_SPEC || VF == VFMT_SPEC) {
-    for (int i = tid; i < 510; i += kDecThreads) uhalf[i] = __float2half_rn(__ldg(p.unit_c + i));
+    for (int i = tid; i < 510; i += kDecThreads) {
+      const float v = __ldg(p.unit_c + i);
+      const __half h = __float2half_rn(v);
+      uhalf[i] = h;
+      uhalf[510 + i] = __float2half_rn(v - __half2float(h));
+    }
   }
   __syncthreads();
 
@@ -177,26 +198,20 @@ decode_attn_kernel(const DecodeParams p) {
   const bool r0ok = row0 < G, r1ok = row1 < G;
   const int64_t qrow0 = static_cast<int64_t>(bb) * p.Hq + hk * G + row0;
   const int64_t qrow1 = static_cast<int64_t>(bb) * p.Hq + hk * G + row1;
-  uint32_t qa[KST][4];
+  uint32_t qa[KST][4], ql[KST][4];   // hi and lo halves of the query operand
 #pragma unroll
   for (int s = 0; s < KST; ++s) {
     const int dm = t * TDK + 4 * s;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-    if (r0ok) {
-      const float* q = p.qa + qrow0 * D + dm;
-      a0 = q[0]; a1 = q[1]; a2 = q[2]; a3 = q[3];
-    }
-    if (r1ok) {
-      const float* q = p.qa + qrow1 * D + dm;
-      b0 = q[0]; b1 = q[1]; b2 = q[2]; b3 = q[3];
-    }
-    qa[s][0] = pack_half2(a0, a1);
-    qa[s][1] = pack_half2(b0, b1);
-    qa[s][2] = pack_half2(a2, a3);
-    qa[s][3] = pack_half2(b2, b3);
+    float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+    if (r0ok) for (int i = 0; i < 4; ++i) a[i] = p.qa[qrow0 * D + dm + i];
+    if (r1ok) for (int i = 0; i < 4; ++i) b[i] = p.qa[qrow1 * D + dm + i];
+    split_pair(a[0], a[1], qa[s][0], ql[s][0]);
+    split_pair(b[0], b[1], qa[s][1], ql[s][1]);
+    split_pair(a[2], a[3], qa[s][2], ql[s][2]);
+    split_pair(b[2], b[3], qa[s][3], ql[s][3]);
   }
-  uint32_t qb[KST][4];     // prod: QJL operand with the same permutation
-  uint32_t qx[4];          // spectral: the extra head k-step
+  uint32_t qb[KST][4], qbl[KST][4];   // prod: QJL operand (hi, lo) with the same permutation
+  uint32_t qx[4], qxl[4];              // spectral: the extra head k-step (hi, lo)
   if constexpr (KF == KFMT_PROD) {
 #pragma unroll
     for (int s = 0; s < KST; ++s) {
@@ -204,10 +219,10 @@ decode_attn_kernel(const DecodeParams p) {
       float a[4] = {0.f, 0.f, 0.f, 0.f}, c[4] = {0.f, 0.f, 0.f, 0.f};
       if (r0ok) for (int i = 0; i < 4; ++i) a[i] = p.qb[qrow0 * p.qb_stride + dm + i];
       if (r1ok) for (int i = 0; i < 4; ++i) c[i] = p.qb[qrow1 * p.qb_stride + dm + i];
-      qb[s][0] = pack_half2(a[0], a[1]);
-      qb[s][1] = pack_half2(c[0], c[1]);
-      qb[s][2] = pack_half2(a[2], a[3]);
-      qb[s][3] = pack_half2(c[2], c[3]);
+      split_pair(a[0], a[1], qb[s][0], qbl[s][0]);
+      split_pair(c[0], c[1], qb[s][1], qbl[s][1]);
+      split_pair(a[2], a[3], qb[s][2], qbl[s][2]);
+      split_pair(c[2], c[3], qb[s][3], qbl[s][3]);
     }
   }
   if constexpr (KF == KFMT_SPEC) {
@@ -215,12 +230,12 @@ decode_attn_kernel(const DecodeParams p) {
     const int sl[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
     if (r0ok) for (int i = 0; i < 4; ++i) a[i] = p.qb[qrow0 * p.qb_stride + sl[i]];
     if (r1ok) for (int i = 0; i < 4; ++i) c[i] = p.qb[qrow1 * p.qb_stride + sl[i]];
-    qx[0] = pack_half2(a[0], a[1]);
-    qx[1] = pack_half2(c[0], c[1]);
-    qx[2] = pack_half2(a[2], a[3]);
-    qx[3] = pack_half2(c[2], c[3]);
+    split_pair(a[0], a[1], qx[0], qxl[0]);
+    split_pair(c[0], c[1], qx[1], qxl[1]);
+    split_pair(a[2], a[3], qx[2], qxl[2]);
+    split_pair(c[2], c[3], qx[3], qxl[3]);
   }
-  const float sa0 = r0ok ? p.qs[qrow0 * 2] : 0.f, sa1 = r1ok ? p.qs[qrow1 * 2] : 0.f;
+  const float sa0 = r0ok ? p.qs[qrow0 * 2] * p.k_scale : 0.f, sa1 = r1ok ? p.qs[qrow1 * 2] * p.k_scale : 0.f;
   const float sb0 = r0ok ? p.qs[qrow0 * 2 + 1] : 0.f, sb1 = r1ok ? p.qs[qrow1 * 2 + 1] : 0.f;
 
   // spectral head layout (bit offsets of the top dims inside the head words)
@@ -278,6 +293,7 @@ decode_attn_kernel(const DecodeParams p) {
         const uint32_t b0 = lutk[(pair_at<KB, NWK>(ks, 4 * s * KB) << 5) + lane];
         const uint32_t b1 = lutk[(pair_at<KB, NWK>(ks, (4 * s + 2) * KB) << 5) + lane];
         mma16816(acc, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
+        mma16816(acc, ql[s][0], ql[s][1], ql[s][2], ql[s][3], b0, b1);
       }
       float acc2[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (KF == KFMT_PROD) {
@@ -289,6 +305,7 @@ decode_attn_kernel(const DecodeParams p) {
           const uint32_t b0 = luts[(((sw >> (4 * s)) & 3u) << 5) + lane];
           const uint32_t b1 = luts[(((sw >> (4 * s + 2)) & 3u) << 5) + lane];
           mma16816(acc2, qb[s][0], qb[s][1], qb[s][2], qb[s][3], b0, b1);
+          mma16816(acc2, qbl[s][0], qbl[s][1], qbl[s][2], qbl[s][3], b0, b1);
         }
       }
       if constexpr (KF == KFMT_SPEC) {
@@ -307,11 +324,19 @@ decode_attn_kernel(const DecodeParams p) {
           const int j = 2 * t + i;
           if (j < p.k_top_k) {
             const int nb = p.k_top_bits[j];
-            if (nb > 0) hv[i] = __half2float(uhalf[unit_c_off(nb) + head_field(hw, kpos[j], nb)]);
+            if (nb > 0) {
+              const int e = unit_c_off(nb) + head_field(hw, kpos[j], nb);
+              hv[i] = __half2float(uhalf[e]) + __half2float(uhalf[510 + e]);
+            }
             if (p.k_qjl) hv[2 + i] = head_field(hw, kq_pos + j, 1) ? gk : -gk;
           }
         }
-        mma16816(acc2, qx[0], qx[1], qx[2], qx[3], pack_half2(hv[0], hv[1]), pack_half2(hv[2], hv[3]));
+        uint32_t bh0, bl0, bh1, bl1;
+        split_pair(hv[0], hv[1], bh0, bl0);
+        split_pair(hv[2], hv[3], bh1, bl1);
+        mma16816(acc2, qx[0], qx[1], qx[2], qx[3], bh0, bh1);
+        mma16816(acc2, qxl[0], qxl[1], qxl[2], qxl[3], bh0, bh1);
+        mma16816(acc2, qx[0], qx[1], qx[2], qx[3], bl0, bl1);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -359,16 +384,19 @@ decode_attn_kernel(const DecodeParams p) {
       l1 += pr[nt][2] + pr[nt][3];
     }
     // A operand of P.V: p * ||v|| as half (rows g, g+8; keys 2t,2t+1 | 8+2t,9+2t)
-    const uint32_t pa0 = pack_half2(pr[0][0] * vn[0], pr[0][1] * vn[1]);
-    const uint32_t pa1 = pack_half2(pr[0][2] * vn[0], pr[0][3] * vn[1]);
-    const uint32_t pa2 = pack_half2(pr[1][0] * vn[2], pr[1][1] * vn[3]);
-    const uint32_t pa3 = pack_half2(pr[1][2] * vn[2], pr[1][3] * vn[3]);
+    uint32_t pa0, pa1, pa2, pa3, pl0, pl1, pl2, pl3;
+    split_pair(pr[0][0] * vn[0], pr[0][1] * vn[1], pa0, pl0);
+    split_pair(pr[0][2] * vn[0], pr[0][3] * vn[1], pa1, pl1);
+    split_pair(pr[1][0] * vn[2], pr[1][1] * vn[3], pa2, pl2);
+    split_pair(pr[1][2] * vn[2], pr[1][3] * vn[3], pa3, pl3);
     // ---- P.V in the rotated domain ----
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
       const uint32_t e01 = field_at<VB, NWV>(vs[0], i * VB) | (field_at<VB, NWV>(vs[1], i * VB) << VB);
       const uint32_t e23 = field_at<VB, NWV>(vs[2], i * VB) | (field_at<VB, NWV>(vs[3], i * VB) << VB);
-      mma16816(o[i], pa0, pa1, pa2, pa3, lutv[(e01 << 5) + lane], lutv[(e23 << 5) + lane]);
+      const uint32_t b0 = lutv[(e01 << 5) + lane], b1 = lutv[(e23 << 5) + lane];
+      mma16816(o[i], pa0, pa1, pa2, pa3, b0, b1);
+      mma16816(o[i], pl0, pl1, pl2, pl3, b0, b1);
     }
     if constexpr (VF == VFMT_SPEC) {
       // head dims of the values: n-tile slot g = head dim g
@@ -381,11 +409,17 @@ decode_attn_kernel(const DecodeParams p) {
             const uint32_t* rec = p.vcodes + (rec0 + kc[i]) * p.v_words;
             uint32_t hw[3] = {0u, 0u, 0u};
             for (int w = 0; w < 3 && w < p.v_code_off; ++w) hw[w] = __ldg(rec + w);
-            hv[i] = __half2float(uhalf[unit_c_off(nb) + head_field(hw, vpos[g], nb)]);
+            const int e = unit_c_off(nb) + head_field(hw, vpos[g], nb);
+            hv[i] = (__half2float(uhalf[e]) + __half2float(uhalf[510 + e])) / p.v_scale;
           }
         }
       }
-      mma16816(oh, pa0, pa1, pa2, pa3, pack_half2(hv[0], hv[1]), pack_half2(hv[2], hv[3]));
+      uint32_t bh0, bl0, bh1, bl1;
+      split_pair(hv[0], hv[1], bh0, bl0);
+      split_pair(hv[2], hv[3], bh1, bl1);
+      mma16816(oh, pa0, pa1, pa2, pa3, bh0, bh1);
+      mma16816(oh, pl0, pl1, pl2, pl3, bh0, bh1);
+      mma16816(oh, pa0, pa1, pa2, pa3, bl0, bl1);
     }
   }
 
@@ -434,14 +468,14 @@ decode_attn_kernel(const DecodeParams p) {
       float a = 0.f;
 #pragma unroll
       for (int w = 0; w < kDecWarps; ++w) a += f[w] * mrg[w * 16 * (D + 2) + r * (D + 2) + 2 + j];
-      p.part_o[pi * D + j] = a;
+      p.part_o[pi * D + j] = a * p.v_scale;
     }
   }
 }
 
 // Dynamic shared memory of decode_attn_kernel<D, *, KB, *, VB>.
 inline size_t decode_smem_bytes(int D, int kb, int vb) {
-  const size_t tables = (static_cast<size_t>(1u << (2 * kb)) + (1u << (2 * vb)) + 4) * 32 * 4 + 1024;
+  const size_t tables = (static_cast<size_t>(1u << (2 * kb)) + (1u << (2 * vb)) + 4) * 32 * 4 + 2048;
   const size_t merge = static_cast<size_t>(kDecWarps) * 16 * (D + 2) * 4;
   return tables > merge ? tables : merge;
 }

@@ -215,6 +215,12 @@ tq_status codebook_build(int d, int bits, int dist, double sigma, double* c_out,
       move = std::max(move, std::fabs(cn[k] - c[k]));
     }
     c.swap(cn);
+    // both laws are symmetric: keep the codebook exactly odd so the middle boundary is 0
+    for (int k = 0; k < K / 2; ++k) {
+      const double v = 0.5 * (c[K - 1 - k] - c[k]);
+      c[k] = -v;
+      c[K - 1 - k] = v;
+    }
     if (move < 1e-13 * L.scale) {
       for (int k = 0; k < K; ++k) c_out[k] = c[k];
       for (int k = 0; k + 1 < K; ++k) t_out[k] = 0.5 * (c[k] + c[k + 1]);
@@ -314,6 +320,39 @@ tq_status spectral_calibrate(const float* X, int64_t n, int d, double* vecs, dou
     const double sgn = V[(size_t)arg * d + j] < 0 ? -1.0 : 1.0;
     for (int k = 0; k < d; ++k) vecs[(size_t)r * d + k] = sgn * V[(size_t)k * d + j];
   }
+  return TQ_OK;
+}
+
+tq_status lut_scale(const double* values, int count, float* scale_out) {
+  if (!values || !scale_out || count < 1) return fail(TQ_ERR_INVALID_ARG, "lut_scale: bad arguments");
+  std::vector<double> mags;
+  for (int i = 0; i < count; ++i) {
+    const double a = std::fabs(values[i]);
+    if (a > 0.0 && std::isfinite(a)) mags.push_back(a);
+  }
+  std::sort(mags.begin(), mags.end());
+  mags.erase(std::unique(mags.begin(), mags.end()), mags.end());
+  if (mags.empty()) { *scale_out = 1.0f; return TQ_OK; }
+  // relative rounding error of v to the nearest half-precision value (normal range)
+  auto rel_err = [](double v) {
+    int e;
+    std::frexp(v, &e);                       // v = f * 2^e, f in [0.5, 1)
+    const double ulp = std::ldexp(1.0, e - 11);
+    const double r = std::nearbyint(v / ulp) * ulp;
+    return std::fabs(r - v) / v;
+  };
+  const int steps = 1 << 22;
+  double best_s = 1.0, best = 1e9;
+  for (int i = 0; i < steps; ++i) {
+    const double sc = 1.0 + static_cast<double>(i) / steps;
+    double worst = 0.0;
+    for (double m : mags) {
+      worst = std::max(worst, rel_err(m / sc));
+      if (worst >= best) break;
+    }
+    if (worst < best) { best = worst; best_s = sc; }
+  }
+  *scale_out = static_cast<float>(best_s);
   return TQ_OK;
 }
 

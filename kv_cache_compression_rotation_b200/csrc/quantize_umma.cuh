@@ -276,8 +276,10 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
       }
       const float nu = sqrtf(ss);
+      // a zero row compares y = 0 against the unscaled boundaries (u = 0 by definition)
+      const float nthr = nu > 0.f ? nu : 1.f;
 #pragma unroll
-      for (int k = 0; k < NB; ++k) thr[k] = nu * tsm[k];
+      for (int k = 0; k < NB; ++k) thr[k] = nthr * tsm[k];
       // pass 2: codes against ||y|| * t_k, packed LSB-first
       uint32_t words[W];
 #pragma unroll

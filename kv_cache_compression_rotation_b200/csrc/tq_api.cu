@@ -346,6 +346,10 @@ tq_status tq_spectral_unit_codebooks(double* centroids_out, double* boundaries_o
   return spectral_unit_codebooks(centroids_out, boundaries_out);
 }
 
+tq_status tq_lut_scale(const double* values, int32_t count, float* scale_out) {
+  return lut_scale(values, count, scale_out);
+}
+
 tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out) {
   const tq_status s = check_quantizer(q);
   if (s != TQ_OK) return s;
@@ -522,6 +526,8 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
   if (!aligned16(q) || !aligned16(seq_lens) || !aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "q/seq_lens/out alignment");
   if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
+  if (!(kq->lut_scale >= 0.f) || !(vq->lut_scale >= 0.f) || !std::isfinite(kq->lut_scale) || !std::isfinite(vq->lut_scale))
+    return fail(TQ_ERR_INVALID_ARG, "lut_scale must be finite and >= 0");
   const tq_layout LK = layout_of(kq), LV = layout_of(vq);
   if ((s = check_packed(kc, LK)) != TQ_OK) return s;
   if ((s = check_packed(vc, LV)) != TQ_OK) return s;
@@ -592,6 +598,8 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   }
   dp.qa = qa; dp.qb = qb; dp.qs = qs; dp.qb_stride = P.qb_stride;
   dp.qjl_coef = kq->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / kq->m) : 0.f;
+  dp.k_scale = kq->lut_scale > 0.f ? kq->lut_scale : 1.f;
+  dp.v_scale = vq->lut_scale > 0.f ? vq->lut_scale : 1.f;
   dp.part_ml = pml; dp.part_o = po;
   const dim3 grid(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv));
   const size_t smem = decode_smem_bytes(D, kb, vb);

@@ -17,6 +17,7 @@ tq_status codebook_build(int d, int bits, int dist, double sigma, double* c_out,
 tq_status waterfill(const double* lambda, int k, int budget, int max_bits, int32_t* out);
 tq_status spectral_calibrate(const float* X, int64_t n, int d, double* vecs, double* vals);
 tq_status spectral_unit_codebooks(double* c_out, double* t_out);
+tq_status lut_scale(const double* values, int count, float* scale_out);
 
 // Device-side status word and wait limit (tq_api.cu).
 int* device_status_ptr();      // address of the current device's status word

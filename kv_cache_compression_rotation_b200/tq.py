@@ -30,7 +30,7 @@ EXPORTS = [
     "tq_version", "tq_last_error", "tq_codebook_build", "tq_waterfill", "tq_spectral_calibrate",
     "tq_spectral_unit_codebooks", "tq_record_layout", "tq_quantize_mse", "tq_quantize_prod",
     "tq_quantize_spectral", "tq_dequantize", "tq_score_workspace", "tq_score",
-    "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit",
+    "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
 ]
 
 
@@ -47,6 +47,7 @@ class Quantizer_t(C.Structure):
         ("k_top", C.c_int32), ("tail_bits", C.c_int32), ("qjl", C.c_int32),
         ("top_bits", C.c_int32 * MAX_TOP),
         ("dim_sigma", C.c_void_p), ("unit_centroids", C.c_void_p), ("unit_boundaries", C.c_void_p),
+        ("lut_scale", C.c_float),
     ]
 
 
@@ -91,6 +92,7 @@ def lib():
                                 vp, vp, C.c_size_t, vp], C.c_int),
             "tq_get_status": ([vp], C.c_int),
             "tq_set_wait_limit": ([i64], C.c_int),
+            "tq_lut_scale": ([f64p, i32, C.POINTER(C.c_float)], C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -155,6 +157,14 @@ def spectral_calibrate(X: np.ndarray):
     return vecs, vals
 
 
+def lut_scale(values) -> float:
+    """Shared scale s for a half-precision table of `values` (entries v / s)."""
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    out = C.c_float(0.0)
+    _check(lib().tq_lut_scale(v.ctypes.data_as(C.POINTER(C.c_double)), v.shape[0], C.byref(out)))
+    return float(out.value)
+
+
 def spectral_unit_codebooks():
     c = np.zeros(510, dtype=np.float64)
     t = np.zeros(502, dtype=np.float64)
@@ -181,7 +191,8 @@ class Quantizer:
     """Device-resident quantizer descriptor (owns the tensors the C struct points at)."""
 
     def __init__(self, kind: int, d: int, rot, *, bits=0, m=0, S=None, centroids=None, boundaries=None,
-                 k_top=0, tail_bits=0, qjl=0, top_bits=(), dim_sigma=None, unit_c=None, unit_t=None):
+                 k_top=0, tail_bits=0, qjl=0, top_bits=(), dim_sigma=None, unit_c=None, unit_t=None,
+                 lut_scale=0.0):
         self.kind, self.d, self.bits, self.m = kind, d, bits, m
         self._keep = [rot, S, centroids, boundaries, dim_sigma, unit_c, unit_t]
         self.rot, self.S, self.centroids, self.boundaries = rot, S, centroids, boundaries
@@ -189,7 +200,8 @@ class Quantizer:
         self.k_top, self.tail_bits, self.qjl, self.top_bits = k_top, tail_bits, qjl, tuple(top_bits)
         tb = (C.c_int32 * MAX_TOP)(*(list(top_bits) + [0] * (MAX_TOP - len(top_bits))))
         self.c = Quantizer_t(kind, d, bits, m, _dptr(rot), _dptr(S), _dptr(centroids), _dptr(boundaries),
-                             k_top, tail_bits, qjl, tb, _dptr(dim_sigma), _dptr(unit_c), _dptr(unit_t))
+                             k_top, tail_bits, qjl, tb, _dptr(dim_sigma), _dptr(unit_c), _dptr(unit_t),
+                             float(lut_scale))
 
     @property
     def ref(self):
@@ -205,18 +217,20 @@ class Quantizer:
         d = rot.shape[0]
         c, t, _ = codebook_build(bits, dist, d=d, sigma=sigma)
         return cls(KIND_MSE, d, cls._dev(rot, device), bits=bits,
-                   centroids=cls._dev(c, device), boundaries=cls._dev(t, device))
+                   centroids=cls._dev(c, device), boundaries=cls._dev(t, device), lut_scale=lut_scale(c))
 
     @classmethod
     def prod(cls, rot, S, bits: int, dist: str = "beta", sigma: float = 0.0, device="cuda"):
         d = rot.shape[0]
         m = S.shape[0]
         cen = bnd = None
+        sc = 0.0
         if bits > 1:
             c, t, _ = codebook_build(bits - 1, dist, d=d, sigma=sigma)
             cen, bnd = cls._dev(c, device), cls._dev(t, device)
+            sc = lut_scale(c)
         return cls(KIND_PROD, d, cls._dev(rot, device), bits=bits, m=m, S=cls._dev(S, device),
-                   centroids=cen, boundaries=bnd)
+                   centroids=cen, boundaries=bnd, lut_scale=sc)
 
     @classmethod
     def spectral(cls, eigvecs, eigvals, k_top: int, top_bits, tail_bits: int, qjl: bool, S_top=None,
@@ -226,7 +240,8 @@ class Quantizer:
         sig = np.sqrt(np.maximum(np.asarray(eigvals, dtype=np.float64), 0.0))
         return cls(KIND_SPECTRAL, d, cls._dev(eigvecs, device), S=None if S_top is None else cls._dev(S_top, device),
                    k_top=k_top, tail_bits=tail_bits, qjl=1 if qjl else 0, top_bits=list(top_bits),
-                   dim_sigma=cls._dev(sig, device), unit_c=cls._dev(uc, device), unit_t=cls._dev(ut, device))
+                   dim_sigma=cls._dev(sig, device), unit_c=cls._dev(uc, device), unit_t=cls._dev(ut, device),
+                   lut_scale=lut_scale(uc[(1 << tail_bits) - 2:(1 << (tail_bits + 1)) - 2]))
 
     def layout(self) -> Layout_t:
         L = Layout_t()

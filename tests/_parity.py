@@ -19,8 +19,13 @@ def as_u32(t) -> np.ndarray:
     return t.detach().cpu().numpy().view(np.uint32)
 
 
-def code_mismatches(gpu_words, ref_words, d, bits, y_ref, boundaries):
-    """Return (#mismatched coordinates outside the band, #exempt, rows with exemptions)."""
+def code_mismatches(gpu_words, ref_words, d, bits, y_ref, boundaries, skip_rows=()):
+    """Return (#mismatched coordinates outside the band, #exempt, rows with exemptions).
+
+    A mismatch is exempt only when the two codes are neighbours and the oracle's rotated
+    value lies within BAND of the boundary between them.  Rows in ``skip_rows`` (zero
+    vectors, whose every coordinate sits on the middle boundary) are not compared here.
+    """
     from oracle.quantizer import unpack_codes
     g = np.asarray(gpu_words, dtype=np.uint32)
     r = np.asarray(ref_words, dtype=np.uint32)
@@ -29,11 +34,14 @@ def code_mismatches(gpu_words, ref_words, d, bits, y_ref, boundaries):
     exempt_rows = set()
     t = np.asarray(boundaries, dtype=np.float64)
     for i in rows:
+        if int(i) in skip_rows:
+            continue
         cg = unpack_codes(g[i:i + 1], d, bits)[0]
         cr = unpack_codes(r[i:i + 1], d, bits)[0]
         for j in np.nonzero(cg != cr)[0]:
-            dist = np.min(np.abs(y_ref[i, j] - t)) if t.size else np.inf
-            if dist <= BAND:
+            lo = int(min(cg[j], cr[j]))
+            near = abs(int(cg[j]) - int(cr[j])) == 1 and abs(y_ref[i, j] - t[lo]) <= BAND
+            if near:
                 exempt += 1
                 exempt_rows.add(int(i))
             else:

@@ -60,9 +60,15 @@ def test_quantize_mse_parity(d, bits, dtype, n):
     assert K.get_status() == 0
     c, t, _ = lloyd_max(bits, "beta", d=d)
     ref = OQ.quantize_mse(x64, rot, c, t, bits)
-    bad, exempt, _ = code_mismatches(as_u32(out.codes), ref["codes"], d, bits, ref["y"], t)
+    zero = [0] if n > 10 else []
+    bad, exempt, _ = code_mismatches(as_u32(out.codes), ref["codes"], d, bits, ref["y"], t, skip_rows=zero)
     assert bad == 0, f"{bad} code mismatches outside the band ({exempt} exempt)"
     assert exempt <= max(2, 1e-4 * n * d)
+    # a zero vector has u = 0: every coordinate sits on the middle boundary t = 0 and
+    # takes the lower cell, code 2^(b-1) - 1
+    from oracle.quantizer import unpack_codes
+    for r in zero:
+        assert np.all(unpack_codes(as_u32(out.codes)[r:r + 1], d, bits) == (1 << (bits - 1)) - 1)
     nrm = out.norms.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(nrm - ref["norms"]) <= 1e-5 * np.maximum(ref["norms"], 1e-30))
     # reconstruction from the GPU's own records matches the oracle's (records without exemptions)
@@ -142,7 +148,8 @@ def test_quantize_spectral_parity(qjl):
         rn = out.rnorms.cpu().numpy()
         ok = np.ones(n, dtype=bool)
         ok[rows] = False
-        assert np.all(np.abs(rn[ok] - ref["rnorms"][ok]) <= 1e-5 * np.maximum(ref["rnorms"][ok], 1e-3))
+        # the top coordinates are O(sigma_0) ~ 10, so gamma carries absolute rounding ~1e-6 ||x||
+        assert np.all(np.abs(rn[ok] - ref["rnorms"][ok]) <= 1e-5 * xn[ok])
     xh = K.dequantize(q, out, n).cpu().numpy()
     xr = OSP.dequantize_spectral(ref["chat"], desc)
     ok = np.ones(n, dtype=bool)

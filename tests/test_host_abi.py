@@ -215,3 +215,13 @@ def test_score_validation(lib):
                         FAKE + 0x600000, 8, None) == 8          # workspace
     assert lib.tq_set_wait_limit(-1) == 1
     assert lib.tq_set_wait_limit(0) == 0
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_lut_scale_tightens_half_precision_codebook(lib, bits):
+    c, _, _ = K.codebook_build(bits, "beta", d=128)
+    s = T.lut_scale(c)
+    assert 1.0 <= s < 2.0
+    plain = np.max(np.abs(c.astype(np.float16).astype(np.float64) - c) / np.abs(c))
+    scaled = np.max(np.abs((c / s).astype(np.float16).astype(np.float64) * s - c) / np.abs(c))
+    assert scaled <= min(plain, 1.5e-4)
