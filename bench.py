@@ -38,12 +38,12 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-B, HKV, HQ, N, D, BITS = 8, 8, 32, 131072, 128, 4
+B, HKV, HQ, N, D, BITS = 8, 8, 32, 131072, 128, 4   # N may be lowered with --context
 METRIC = "quantized vectors/s and packed-KV decode-attn GB/s (% of B200 HBM roofline)"
 
 
 def algorithmic_bytes():
-    nvec = B * HKV * N
+    nvec = B * HKV * N   # noqa: F821 (N is module state, adjustable by --context)
     rec = D * BITS // 8 + 4                      # 64 B codes + 4 B norm
     q_bytes = nvec * (D * 2 + rec)               # read bf16 row, write record
     dec_bytes = 2 * nvec * rec                   # read K and V records
@@ -139,18 +139,27 @@ def run_tq(args, rank, world, local_rank):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     qk_ms, qv_ms, dec_ms = [], [], []
 
+    only = args.only
+
     def step(record):
         if record:
             ev[0].record(stream)
-        K.quantize(kq, kx, kc)
+        if only in ("all", "quantize"):
+            K.quantize(kq, kx, kc)
         if record:
             ev[1].record(stream)
-        K.quantize(vq, vx, vc)
+        if only in ("all", "quantize"):
+            K.quantize(vq, vx, vc)
         if record:
             ev[2].record(stream)
-        K.decode_attn(kq, vq, q, seq, kc, vc, N, HKV, out=out, workspace=ws)
+        if only in ("all", "decode"):
+            K.decode_attn(kq, vq, q, seq, kc, vc, N, HKV, out=out, workspace=ws)
         if record:
             ev[3].record(stream)
+
+    if only == "decode":          # the decode-only profile reads a cache quantized once here
+        K.quantize(kq, kx, kc)
+        K.quantize(vq, vx, vc)
 
     for _ in range(args.warmup):
         step(False)
@@ -328,7 +337,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--only", default="all", choices=["all", "quantize", "decode"],
+                    help="profiling aid: run one part of the step (the reported line is then partial)")
+    ap.add_argument("--context", type=int, default=N,
+                    help="profiling aid: context length (the headline workload uses 131072)")
     args = ap.parse_args()
+    globals()["N"] = args.context
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

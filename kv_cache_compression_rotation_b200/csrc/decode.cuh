@@ -102,8 +102,9 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
 }
 
 // Per-thread slice of a record: `NW` words starting at bit `base` of the record's stream,
-// re-aligned so that bit 0 of seg[0] is bit `base`.
-template <int NW>
+// re-aligned so that bit 0 of seg[0] is bit `base`.  GLOBAL selects the read-only global
+// load path; otherwise `rec` points into shared memory.
+template <int NW, bool GLOBAL = true>
 __device__ __forceinline__ void load_slice(const uint32_t* rec, int rec_words, int base,
                                            bool valid, uint32_t (&seg)[NW]) {
   const int w0 = base >> 5, sh = base & 31;
@@ -111,7 +112,9 @@ __device__ __forceinline__ void load_slice(const uint32_t* rec, int rec_words, i
 #pragma unroll
   for (int i = 0; i <= NW; ++i) {
     const int wi = w0 + i;
-    w[i] = (valid && wi < rec_words && (i < NW || sh != 0)) ? __ldg(rec + wi) : 0u;
+    const bool use = valid && wi < rec_words && (i < NW || sh != 0);
+    if constexpr (GLOBAL) w[i] = use ? __ldg(rec + wi) : 0u;
+    else w[i] = use ? rec[wi] : 0u;
   }
 #pragma unroll
   for (int i = 0; i < NW; ++i) seg[i] = __funnelshift_r(w[i], w[i + 1], sh);

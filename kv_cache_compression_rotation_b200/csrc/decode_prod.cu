@@ -1,39 +1,43 @@
-// Instantiations of decode_attn_kernel with keys in the prod format (D = 128).
-#include "decode.cuh"
+// Instantiations of the bulk-copy staged decode kernel with prod keys and MSE values (d = 128).
+#include "decode_tma.cuh"
 #include "launchers.h"
 
 namespace tq {
 namespace {
 
 template <int KB, int VB>
-cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s) {
-  auto k = decode_attn_kernel<128, KFMT_PROD, KB, VFMT_MSE, VB>;
+cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, int* status, long long lim) {
+  const bool g8 = p.G <= 8;
+  auto k = g8 ? decode_tma_kernel<KFMT_PROD, KB, VB, true> : decode_tma_kernel<KFMT_PROD, KB, VB, false>;
+  smem = decode_tma_smem_bytes(KB, VB, KFMT_PROD, 4, g8);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k<<<grid, kDecThreads, smem, s>>>(p);
+  k<<<grid, kTmaThreads, smem, s>>>(p, status, lim);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid, size_t, cudaStream_t s,
+                              int* status, long long lim) {
+  size_t smem = 0;
   switch (kb * 10 + vb) {
-    case 11: return go<1, 1>(p, grid, smem, s);
-    case 12: return go<1, 2>(p, grid, smem, s);
-    case 13: return go<1, 3>(p, grid, smem, s);
-    case 14: return go<1, 4>(p, grid, smem, s);
-    case 21: return go<2, 1>(p, grid, smem, s);
-    case 22: return go<2, 2>(p, grid, smem, s);
-    case 23: return go<2, 3>(p, grid, smem, s);
-    case 24: return go<2, 4>(p, grid, smem, s);
-    case 31: return go<3, 1>(p, grid, smem, s);
-    case 32: return go<3, 2>(p, grid, smem, s);
-    case 33: return go<3, 3>(p, grid, smem, s);
-    case 34: return go<3, 4>(p, grid, smem, s);
-    case 41: return go<4, 1>(p, grid, smem, s);
-    case 42: return go<4, 2>(p, grid, smem, s);
-    case 43: return go<4, 3>(p, grid, smem, s);
-    case 44: return go<4, 4>(p, grid, smem, s);
+    case 11: return go<1, 1>(p, grid, smem, s, status, lim);
+    case 12: return go<1, 2>(p, grid, smem, s, status, lim);
+    case 13: return go<1, 3>(p, grid, smem, s, status, lim);
+    case 14: return go<1, 4>(p, grid, smem, s, status, lim);
+    case 21: return go<2, 1>(p, grid, smem, s, status, lim);
+    case 22: return go<2, 2>(p, grid, smem, s, status, lim);
+    case 23: return go<2, 3>(p, grid, smem, s, status, lim);
+    case 24: return go<2, 4>(p, grid, smem, s, status, lim);
+    case 31: return go<3, 1>(p, grid, smem, s, status, lim);
+    case 32: return go<3, 2>(p, grid, smem, s, status, lim);
+    case 33: return go<3, 3>(p, grid, smem, s, status, lim);
+    case 34: return go<3, 4>(p, grid, smem, s, status, lim);
+    case 41: return go<4, 1>(p, grid, smem, s, status, lim);
+    case 42: return go<4, 2>(p, grid, smem, s, status, lim);
+    case 43: return go<4, 3>(p, grid, smem, s, status, lim);
+    case 44: return go<4, 4>(p, grid, smem, s, status, lim);
     default: return cudaErrorNotSupported;
   }
 }

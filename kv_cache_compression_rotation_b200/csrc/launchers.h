@@ -11,10 +11,14 @@ struct UmmaQuantParams;
 
 // Launch decode_attn_kernel for (key format, key bits, value format, value bits) at D = 128.
 // Returns cudaErrorNotSupported (without launching) for a combination that is not built.
+// MSE / PROD keys run the bulk-copy staged kernel (decode_tma.cuh), spectral keys the
+// direct-load kernel (decode.cuh).  `status`/`lim`: device status word and wait limit.
 cudaError_t launch_decode(const DecodeParams& p, int kfmt, int kb, int vfmt, int vb, dim3 grid,
-                          size_t smem, cudaStream_t stream);
-cudaError_t launch_decode_mse(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
-cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
+                          size_t smem, cudaStream_t stream, int* status, long long lim);
+cudaError_t launch_decode_mse(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s,
+                              int* status, long long lim);
+cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s,
+                               int* status, long long lim);
 cudaError_t launch_decode_spec(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
 
 // Tensor-core quantize (d = 128, 16-bit input, MSE bits 1..4).

@@ -12,8 +12,16 @@
 //   warp 0      TMA producer: 128-row tiles of x into a 4-stage ring (128B swizzle)
 //   warp 1      TMEM allocator and single-thread MMA issuer (2 accumulator buffers)
 //   warps 2-5   epilogue group 0 (even tiles), warps 6-9 group 1 (odd tiles):
-//               one vector per thread: tcgen05.ld the row, ||y||, codes against
-//               ||y|| * t_k, pack LSB-first, store record + norm.
+//               one vector per thread: tcgen05.ld the row, ||y||, then per coordinate
+//               u = y / ||y|| and its code, packed LSB-first; store record + norm.
+// Code assignment (b >= 2): [-R, R) with R = 1.25 t_max is cut into 32 equal cells,
+// narrower than the smallest gap between boundaries, so each cell holds at most one
+// boundary.  Lane g of every warp keeps cell g's entry: the boundary inside it (or a
+// huge value) with the number of boundaries below the cell in its 4 low mantissa bits
+// (a perturbation below 1e-6 of a unit-scale boundary).  A coordinate's code is then
+// one FFMA to find its cell, one warp shuffle to fetch the entry and one compare:
+// code = (#boundaries below the cell) + (u > boundary in the cell).  A codebook whose
+// gaps are narrower than the cells falls back to counting all boundaries.
 // ||y|| equals ||x|| up to the orthogonality of the fp32 Pi (~1e-7 relative).
 // Every mbarrier wait is bounded; on timeout the CTA records TQ_ERR_TIMEOUT, drains
 // what it issued, frees TMEM and exits.
@@ -34,6 +42,8 @@ constexpr uint32_t kPiBytes = kUmmaD * kUmmaD * 2;                 // 32 KB per 
 // Drains (copies and MMAs this CTA already issued) always complete on their own; their
 // bound is fixed and independent of the test-adjustable wait limit.
 constexpr long long kDrainLimit = 1ll << 28;
+// 32 cells over [-R, R): f in [0, 1] maps to floor(f * kCellSpan) in 0..31
+constexpr float kCellSpan = 31.9999f;
 constexpr uint32_t kUmmaSmemBytes = 1024 /*align slack*/ + 2 * kPiBytes + kUmmaStages * kXStageBytes + 256;
 
 struct UmmaQuantParams {
@@ -257,6 +267,27 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
     const int lanebase = 32 * (warp & 3);              // TMEM lanes this warp may access
     const int r = lanebase + lane;                     // row within the tile
     float thr[NB];
+    // cell table (identical in every warp): lane g holds the entry of cell g
+    bool use_cells = false;
+    float cell_scale = 0.f;
+    uint32_t cell_entry = 0u;
+    if (NB >= 3) {
+      const float R = 1.25f * tsm[NB - 1];
+      float min_gap = 3.0e38f;
+      for (int k = 0; k + 1 < NB; ++k) min_gap = fminf(min_gap, tsm[k + 1] - tsm[k]);
+      const float width = 2.f * R / kCellSpan;
+      use_cells = R > 0.f && width < 0.9f * min_gap;
+      cell_scale = 0.5f / R;
+      const float a = (static_cast<float>(lane) / kCellSpan - 0.5f) * 2.f * R;
+      const float b = (static_cast<float>(lane + 1) / kCellSpan - 0.5f) * 2.f * R;
+      uint32_t base_code = 0u;
+      float inside = 3.0e38f;
+      for (int k = 0; k < NB; ++k) {
+        if (tsm[k] < a) ++base_code;
+        else if (tsm[k] < b || lane == 31) inside = fminf(inside, tsm[k]);
+      }
+      cell_entry = (__float_as_uint(inside) & ~15u) | base_code;
+    }
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int buf = it & 1;
@@ -280,10 +311,12 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       const float nthr = nu > 0.f ? nu : 1.f;
 #pragma unroll
       for (int k = 0; k < NB; ++k) thr[k] = nthr * tsm[k];
-      // pass 2: codes against ||y|| * t_k, packed LSB-first
+      // pass 2: codes, packed LSB-first
       uint32_t words[W];
 #pragma unroll
       for (int w = 0; w < W; ++w) words[w] = 0u;
+      const float inv = nu > 0.f ? 1.f / nu : 1.f;     // a zero row keeps u = 0
+      const float fs = inv * cell_scale;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[32];
@@ -291,12 +324,21 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          int code = 0;
+          uint32_t code;
+          if (use_cells) {
+            const float f = __saturatef(fmaf(v[i], fs, 0.5f));
+            const float gcell = __fmaf_rz(f, kCellSpan, 8388608.0f);
+            const uint32_t e = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gcell));
+            code = (e & 15u) + ((v[i] * inv > __uint_as_float(e)) ? 1u : 0u);
+          } else {
+            int cnt = 0;
 #pragma unroll
-          for (int k = 0; k < NB; ++k) code += (v[i] > thr[k]) ? 1 : 0;
+            for (int k = 0; k < NB; ++k) cnt += (v[i] > thr[k]) ? 1 : 0;
+            code = static_cast<uint32_t>(cnt);
+          }
           const int pos = (32 * c + i) * B;
-          words[pos >> 5] |= static_cast<uint32_t>(code) << (pos & 31);
-          if ((pos & 31) + B > 32) words[(pos >> 5) + 1] |= static_cast<uint32_t>(code) >> (32 - (pos & 31));
+          words[pos >> 5] |= code << (pos & 31);
+          if ((pos & 31) + B > 32) words[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
         }
       }
       tc_fence_before();

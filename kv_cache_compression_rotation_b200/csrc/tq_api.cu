@@ -14,6 +14,7 @@
 
 #include "decode.cuh"
 #include "decode_aux.cuh"
+#include "decode_tma.cuh"
 #include "device_common.cuh"
 #include "launchers.h"
 #include "quantize_simt.cuh"
@@ -271,11 +272,25 @@ DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t N
   DecodePlan P{};
   const int D = kq->d;
   const int64_t units = static_cast<int64_t>(B) * Hkv;
-  const int64_t target = static_cast<int64_t>(sm_count()) * 6;
-  int64_t nch = std::max<int64_t>(1, (target + units - 1) / units);
-  int64_t cl = (Nmax + nch - 1) / nch;
-  cl = std::max<int64_t>(256, (cl + 63) / 64 * 64);
-  nch = (Nmax + cl - 1) / cl;
+  const int64_t sms = sm_count();
+  int64_t nch, cl;
+  if (kq->kind != TQ_KIND_SPECTRAL) {
+    // persistent bulk-copy kernel: about 16 work items per SM, chunks of whole 112-token
+    // stages, and (when the shape allows) an item count that is a multiple of the SMs
+    const int64_t stage = 112;
+    int64_t n0 = std::max<int64_t>(1, (16 * sms + units - 1) / units);
+    for (int64_t cand = n0; cand < n0 + 8 && cand <= Nmax; ++cand)
+      if ((units * cand) % sms == 0) { n0 = cand; break; }
+    cl = (Nmax + n0 - 1) / n0;
+    cl = std::max<int64_t>(stage, (cl + stage - 1) / stage * stage);
+    nch = (Nmax + cl - 1) / cl;
+  } else {
+    const int64_t target = sms * 6;
+    nch = std::max<int64_t>(1, (target + units - 1) / units);
+    cl = (Nmax + nch - 1) / nch;
+    cl = std::max<int64_t>(256, (cl + 63) / 64 * 64);
+    nch = (Nmax + cl - 1) / cl;
+  }
   P.chunk_len = static_cast<int>(cl);
   P.n_chunks = static_cast<int>(nch);
   P.qb_stride = kq->kind == TQ_KIND_PROD ? kq->m : 16;
@@ -601,9 +616,11 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   dp.k_scale = kq->lut_scale > 0.f ? kq->lut_scale : 1.f;
   dp.v_scale = vq->lut_scale > 0.f ? vq->lut_scale : 1.f;
   dp.part_ml = pml; dp.part_o = po;
-  const dim3 grid(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv));
+  const int64_t items = static_cast<int64_t>(B) * Hkv * P.n_chunks;
+  const dim3 grid = kfmt == KFMT_SPEC ? dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv))
+                                      : dim3(static_cast<unsigned>(std::min<int64_t>(items, sm_count())));
   const size_t smem = decode_smem_bytes(D, kb, vb);
-  e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream);
+  e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream, device_status_ptr(), wait_limit());
   if (e == cudaErrorNotSupported) return fail(TQ_ERR_UNSUPPORTED, "decode variant not built (kbits %d, vbits %d)", kb, vb);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
 
@@ -640,9 +657,9 @@ tq_status tq_set_wait_limit(int64_t polls) {
 
 namespace tq {
 cudaError_t launch_decode(const DecodeParams& p, int kfmt, int kb, int vfmt, int vb, dim3 grid, size_t smem,
-                          cudaStream_t stream) {
-  if (kfmt == KFMT_MSE && vfmt == VFMT_MSE) return launch_decode_mse(p, kb, vb, grid, smem, stream);
-  if (kfmt == KFMT_PROD && vfmt == VFMT_MSE) return launch_decode_prod(p, kb, vb, grid, smem, stream);
+                          cudaStream_t stream, int* status, long long lim) {
+  if (kfmt == KFMT_MSE && vfmt == VFMT_MSE) return launch_decode_mse(p, kb, vb, grid, smem, stream, status, lim);
+  if (kfmt == KFMT_PROD && vfmt == VFMT_MSE) return launch_decode_prod(p, kb, vb, grid, smem, stream, status, lim);
   if (kfmt == KFMT_SPEC && vfmt == VFMT_SPEC) return launch_decode_spec(p, kb, vb, grid, smem, stream);
   return cudaErrorNotSupported;
 }
