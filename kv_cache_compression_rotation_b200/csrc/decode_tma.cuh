@@ -301,15 +301,26 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       float sc[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // hi and lo query halves accumulate separately: two independent MMA chains
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, accl[4] = {0.f, 0.f, 0.f, 0.f};
         const uint32_t(&ks)[NWK] = nt ? ks1 : ks0;
 #pragma unroll
         for (int s2 = 0; s2 < KST; ++s2) {
-          const uint32_t b0 = lutk[(pair_at<KB, NWK>(ks, 4 * s2 * KB) << 5) + lane];
-          const uint32_t b1 = lutk[(pair_at<KB, NWK>(ks, (4 * s2 + 2) * KB) << 5) + lane];
+          uint32_t b0, b1;
+          if constexpr (KB == 4) {
+            // the pair of dims (4 s2, 4 s2 + 1) is byte 2 (s2 % 2) of word s2 / 2
+            const uint32_t w = ks[s2 >> 1];
+            b0 = lutk[(__byte_perm(w, 0u, 0x4440u + 2 * (s2 & 1)) << 5) + lane];
+            b1 = lutk[(__byte_perm(w, 0u, 0x4441u + 2 * (s2 & 1)) << 5) + lane];
+          } else {
+            b0 = lutk[(pair_at<KB, NWK>(ks, 4 * s2 * KB) << 5) + lane];
+            b1 = lutk[(pair_at<KB, NWK>(ks, (4 * s2 + 2) * KB) << 5) + lane];
+          }
           mma16816(acc, qa[s2][0], qa[s2][1], qa[s2][2], qa[s2][3], b0, b1);
-          mma16816(acc, ql[s2][0], ql[s2][1], ql[s2][2], ql[s2][3], b0, b1);
+          mma16816(accl, ql[s2][0], ql[s2][1], ql[s2][2], ql[s2][3], b0, b1);
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += accl[i];
         float acc2[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (KF == KFMT_PROD) {
           const uint32_t w = sw[nt];
@@ -375,13 +386,34 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         split_pair(pr[1][2] * vn[2], pr[1][3] * vn[3], pa3, pl3);
       }
       // ---- P.V in the rotated domain ----
+      if constexpr (VB == 4) {
+        // byte j of lo (hi) holds the codes of keys (t, t + 4) for dim 2j (2j + 1) of a word
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        const uint32_t e01 = field_at<VB, NWV>(vs[0], i * VB) | (field_at<VB, NWV>(vs[1], i * VB) << VB);
-        const uint32_t e23 = field_at<VB, NWV>(vs[2], i * VB) | (field_at<VB, NWV>(vs[3], i * VB) << VB);
-        const uint32_t b0 = lutv[(e01 << 5) + lane], b1 = lutv[(e23 << 5) + lane];
-        mma16816(o[i], pa0, pa1, pa2, pa3, b0, b1);
-        mma16816(o[i], pl0, pl1, pl2, pl3, b0, b1);
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t a0 = vs[0][w], a1 = vs[1][w], c0 = vs[2][w], c1 = vs[3][w];
+          const uint32_t lo01 = (a0 & 0x0F0F0F0Fu) | ((a1 << 4) & 0xF0F0F0F0u);
+          const uint32_t hi01 = ((a0 >> 4) & 0x0F0F0F0Fu) | (a1 & 0xF0F0F0F0u);
+          const uint32_t lo23 = (c0 & 0x0F0F0F0Fu) | ((c1 << 4) & 0xF0F0F0F0u);
+          const uint32_t hi23 = ((c0 >> 4) & 0x0F0F0F0Fu) | (c1 & 0xF0F0F0F0u);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = 8 * w + j;                  // n-tile = dim within this thread's 16
+            const uint32_t x01 = (j & 1) ? hi01 : lo01, x23 = (j & 1) ? hi23 : lo23;
+            const uint32_t b0 = lutv[(__byte_perm(x01, 0u, 0x4440u + (j >> 1)) << 5) + lane];
+            const uint32_t b1 = lutv[(__byte_perm(x23, 0u, 0x4440u + (j >> 1)) << 5) + lane];
+            mma16816(o[i], pa0, pa1, pa2, pa3, b0, b1);
+            mma16816(o[i], pl0, pl1, pl2, pl3, b0, b1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+          const uint32_t e01 = field_at<VB, NWV>(vs[0], i * VB) | (field_at<VB, NWV>(vs[1], i * VB) << VB);
+          const uint32_t e23 = field_at<VB, NWV>(vs[2], i * VB) | (field_at<VB, NWV>(vs[3], i * VB) << VB);
+          const uint32_t b0 = lutv[(e01 << 5) + lane], b1 = lutv[(e23 << 5) + lane];
+          mma16816(o[i], pa0, pa1, pa2, pa3, b0, b1);
+          mma16816(o[i], pl0, pl1, pl2, pl3, b0, b1);
+        }
       }
     }
 

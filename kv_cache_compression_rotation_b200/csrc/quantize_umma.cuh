@@ -151,6 +151,19 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// B packed words of one 32-coordinate chunk (the chunk starts 4 * B bytes into the record).
+template <int B>
+__device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B]) {
+  if constexpr (B == 4) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (B == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < B; ++i) dst[i] = w[i];
+  }
+}
+
 template <int B>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
 umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantParams p) {
@@ -296,61 +309,74 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       if (!mbar_wait(tfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 128;
-      // pass 1: ||y|| over the whole row
-      float ss = 0.f;
+      const int64_t v = tile * kUmmaTileRows + r;
+      // pass 1: ||y|| over the whole row (independent partial sums keep the FMA pipe busy)
+      float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(taddr + 32 * c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
-      }
-      const float nu = sqrtf(ss);
-      // a zero row compares y = 0 against the unscaled boundaries (u = 0 by definition)
-      const float nthr = nu > 0.f ? nu : 1.f;
-#pragma unroll
-      for (int k = 0; k < NB; ++k) thr[k] = nthr * tsm[k];
-      // pass 2: codes, packed LSB-first
-      uint32_t words[W];
-#pragma unroll
-      for (int w = 0; w < W; ++w) words[w] = 0u;
-      const float inv = nu > 0.f ? 1.f / nu : 1.f;     // a zero row keeps u = 0
-      const float fs = inv * cell_scale;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(taddr + 32 * c, v);
+      for (int c = 0; c < 4; c += 2) {
+        float va[32], vb[32];
+        tmem_ld32(taddr + 32 * c, va);
+        tmem_ld32(taddr + 32 * (c + 1), vb);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          uint32_t code;
-          if (use_cells) {
-            const float f = __saturatef(fmaf(v[i], fs, 0.5f));
-            const float gcell = __fmaf_rz(f, kCellSpan, 8388608.0f);
-            const uint32_t e = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gcell));
-            code = (e & 15u) + ((v[i] * inv > __uint_as_float(e)) ? 1u : 0u);
-          } else {
-            int cnt = 0;
-#pragma unroll
-            for (int k = 0; k < NB; ++k) cnt += (v[i] > thr[k]) ? 1 : 0;
-            code = static_cast<uint32_t>(cnt);
-          }
-          const int pos = (32 * c + i) * B;
-          words[pos >> 5] |= code << (pos & 31);
-          if ((pos & 31) + B > 32) words[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
+          ss[i & 3] = fmaf(va[i], va[i], ss[i & 3]);
+          ss[(i + 2) & 3] = fmaf(vb[i], vb[i], ss[(i + 2) & 3]);
         }
       }
+      const float nu = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
+      const float inv = nu > 0.f ? 1.f / nu : 1.f;     // a zero row keeps u = 0
+      uint32_t* dst = p.codes + v * W;
+      // pass 2: codes of 32 coordinates at a time, B packed words per chunk
+      if (use_cells) {
+        const float fs = inv * cell_scale;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float y[32];
+          tmem_ld32(taddr + 32 * c, y);
+          tmem_wait_ld();
+          uint32_t wc[B];
+#pragma unroll
+          for (int w = 0; w < B; ++w) wc[w] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float f = __saturatef(fmaf(y[i], fs, 0.5f));
+            const float gcell = __fmaf_rz(f, kCellSpan, 8388608.0f);
+            const uint32_t e = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gcell));
+            const uint32_t code = (e & 15u) + ((y[i] * inv > __uint_as_float(e)) ? 1u : 0u);
+            const int pos = i * B;
+            wc[pos >> 5] |= code << (pos & 31);
+            if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
+          }
+          if (v < p.n) store_words<B>(dst + c * B, wc);
+        }
+      } else {
+        const float nthr = nu > 0.f ? nu : 1.f;
+#pragma unroll
+        for (int k = 0; k < NB; ++k) thr[k] = nthr * tsm[k];
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float y[32];
+          tmem_ld32(taddr + 32 * c, y);
+          tmem_wait_ld();
+          uint32_t wc[B];
+#pragma unroll
+          for (int w = 0; w < B; ++w) wc[w] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            int cnt = 0;
+#pragma unroll
+            for (int k = 0; k < NB; ++k) cnt += (y[i] > thr[k]) ? 1 : 0;
+            const int pos = i * B;
+            wc[pos >> 5] |= static_cast<uint32_t>(cnt) << (pos & 31);
+            if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] |= static_cast<uint32_t>(cnt) >> (32 - (pos & 31));
+          }
+          if (v < p.n) store_words<B>(dst + c * B, wc);
+        }
+      }
+      if (v < p.n) p.norms[v] = nu;
       tc_fence_before();
       mbar_arrive(tempty_bar(buf));
-      const int64_t v = tile * kUmmaTileRows + r;
-      if (v < p.n) {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes + v * W);
-#pragma unroll
-        for (int w = 0; w < W / 4; ++w)
-          dst[w] = make_uint4(words[4 * w], words[4 * w + 1], words[4 * w + 2], words[4 * w + 3]);
-        p.norms[v] = nu;
-      }
     }
   }
   tc_fence_before();
