@@ -7,9 +7,8 @@ namespace {
 
 template <int KB, int VB>
 cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, int* status, long long lim) {
-  const bool g8 = p.G <= 8;
-  auto k = g8 ? decode_tma_kernel<KFMT_MSE, KB, VB, true> : decode_tma_kernel<KFMT_MSE, KB, VB, false>;
-  smem = decode_tma_smem_bytes(KB, VB, KFMT_MSE, 4, g8);
+  auto k = decode_tma_kernel<KFMT_MSE, KB, VB>;
+  smem = decode_tma_smem_bytes(KB, VB, KFMT_MSE, 4);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   k<<<grid, kTmaThreads, smem, s>>>(p, status, lim);

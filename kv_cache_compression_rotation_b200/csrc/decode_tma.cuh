@@ -1,17 +1,27 @@
 // Decode attention with bulk-copy (TMA engine) staging of the packed cache, d = 128.
 //
-// Same computation as decode_attn_kernel (decode.cuh) for MSE or PROD keys and MSE
-// values; the difference is how the records reach the SM.  One producer warp streams
-// each chunk of the context in stages of 112 tokens with cp.async.bulk (key codes,
-// value codes, norms; prod adds sign words and residual norms), four stages deep, into
-// shared memory; seven consumer warps each take 16 tokens of a stage, read their
-// record slices with vector shared loads, release the stage, and run the lookup-table
-// dequantization, the two mma.sync products and the online softmax from registers.
-// Keeping ~70 KB of copies in flight per SM is what lets the stream run near HBM rate.
+// Computes, for MSE or PROD keys and MSE values, the same step as decode_attn_kernel
+// (decode.cuh): logit = scale * est(q, k_i), online softmax, o' = sum p ||v|| c[code_v].
 //
-// Within a 16-token unit the score tile's columns are permuted (column n of n-tile nt
-// is token 8 nt + n/2 + 4 (n mod 2)) so that the value-slice loads of a warp touch both
-// halves of the banks evenly; the P.V operand uses the same permutation.
+// Streaming.  Persistent CTAs (one per SM) walk work items (batch * kv-head, head block,
+// context chunk).  One producer warp copies each item in stages of 112 tokens with
+// cp.async.bulk (key codes, value codes, norms; prod adds sign words and residual norms)
+// into a 4-deep shared-memory ring; seven consumer warps each take 16 tokens of a stage,
+// pull their record slices into registers, release the stage and compute.
+//
+// Math per 16-token unit, all on mma.sync m16n8k16 (fp16 in, fp32 accumulate):
+//   scores  S[16 tokens x 8 heads] = K_hat[16 x 128] . Q'^T     (A = table-decoded keys)
+//   P       exp2(S - m) * ||v||, transposed in registers with movmatrix
+//   values  O'^T[128 dims x 8 heads] += V_hat^T[128 x 16] . P^T (A = table-decoded values)
+// Tokens and value dims sit on the MMA's M side (16 rows), the query heads of the GQA
+// group on N (8 columns), so a 4-head group fills half of each MMA instead of a quarter.
+// Table decoding: one 32-bit shared load turns a pair of codes into half2 codebook values
+// (table replicated per lane, so a warp's 32 loads hit 32 banks).
+// Precision: the query operand and P are split hi + lo (two MMAs into one accumulator),
+// table entries are c / s with a searched shared scale s (see tq_lut_scale).
+// Token order inside a unit: score row r holds token r/2 + 4 (r mod 2) + 8 (r / 8)
+// (rows 0..7) which spreads a warp's value-slice loads over both halves of the banks;
+// the k-index of P^T follows the score rows through the transpose.
 // All waits are bounded (TQ_ERR_TIMEOUT on expiry); a CTA that times out drains the
 // copies it issued before it exits.
 #pragma once
@@ -24,6 +34,7 @@ constexpr int kTmaConsumerWarps = 7;
 constexpr int kTmaThreads = (kTmaConsumerWarps + 1) * 32;
 constexpr int kTmaStageTokens = kTmaConsumerWarps * 16;
 constexpr int kTmaStages = 4;
+constexpr int kTmaHeadBlock = 8;     // query heads per work item (MMA N)
 
 __device__ __forceinline__ uint32_t tma_smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -56,6 +67,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Transpose of an 8x8 matrix of halves held one row-pair per thread (mma fragment layout).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 struct TmaStageLayout {
   uint32_t kcodes, vcodes, knorm, vnorm, ksign, krn, bytes;
 };
@@ -74,32 +92,30 @@ __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int k
   return L;
 }
 
-inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, int ksw, bool g8) {
+inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, int ksw) {
   const size_t tables = (static_cast<size_t>(1u << (2 * kb)) + (1u << (2 * vb)) + 4) * 32 * 4;
   const TmaStageLayout L = tma_stage_layout(128 * kb / 32, 128 * vb / 32, kf, ksw);
-  const size_t merge = static_cast<size_t>(kTmaConsumerWarps) * (g8 ? 8 : 16) * (128 + 2) * 4;
+  const size_t merge = static_cast<size_t>(kTmaConsumerWarps) * kTmaHeadBlock * (128 + 2) * 4;
   return tables + static_cast<size_t>(kTmaStages) * L.bytes + merge + 2 * kTmaStages * 8 + 64 + 16;
 }
 
-// G8: the GQA group has at most 8 query heads, so mma rows 8..15 are known to be zero.
-// Persistent: CTA c processes work items c, c + gridDim.x, ... where item = (batch *
-// kv-head, chunk); the lookup tables are built once per CTA and the stage ring runs on
-// across items.  The consumer warps merge each item's partial with a named barrier of
-// their own, so the producer keeps streaming the next item meanwhile.
-template <int KF, int KB, int VB, bool G8>
+// Head blocks per GQA group (work items split groups larger than 8 heads).
+__host__ __device__ inline int tma_head_blocks(int G) { return (G + kTmaHeadBlock - 1) / kTmaHeadBlock; }
+
+template <int KF, int KB, int VB>
 __global__ void __launch_bounds__(kTmaThreads, 1)
 decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int D = 128;
-  constexpr int KST = D / 16;
-  constexpr int TDK = D / 4;
+  constexpr int KST = D / 16;                 // mma k-steps over the key dims
+  constexpr int TDK = D / 4;                  // key dims per thread
   constexpr int NWK = (TDK * KB + 31) / 32;
-  constexpr int TDV = D / 8;
+  constexpr int TDV = D / 8;                  // value dims per thread
   constexpr int NWV = (TDV * VB + 31) / 32;
-  constexpr int NT = D / 8;
+  constexpr int MT = D / 16;                  // P.V M-tiles (16 dims each)
   constexpr int KLUT = 1 << (2 * KB), VLUT = 1 << (2 * VB);
   constexpr int KW = D * KB / 32, VW = D * VB / 32;     // record words
   constexpr int KSW = 4;                                // prod sign words (m = 128)
-  constexpr int MROWS = G8 ? 8 : 16;
+  constexpr int HB = kTmaHeadBlock;
   constexpr int CONSUMERS = kTmaConsumerWarps * 32;
   extern __shared__ __align__(128) uint32_t tsm_[];
   uint32_t* lutk = tsm_;
@@ -108,7 +124,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   unsigned char* stage0 = reinterpret_cast<unsigned char*>(luts + 4 * 32);
   const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW);
   float* mrg = reinterpret_cast<float*>(stage0 + static_cast<size_t>(kTmaStages) * SL.bytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(mrg + kTmaConsumerWarps * MROWS * (D + 2));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mrg + kTmaConsumerWarps * HB * (D + 2));
   int* nb_count = reinterpret_cast<int*>(bars + 2 * kTmaStages);   // [kTmaStages] tokens with staged norms
   int* nb_off = nb_count + kTmaStages;                                 // [kTmaStages] their offset in the stage
   volatile int* abort_flag = nb_off + kTmaStages;
@@ -119,11 +135,16 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int n_items = p.B * p.Hkv * p.n_chunks;
+  const int G = p.G;
+  const int nhb = tma_head_blocks(G);
+  const int n_items = p.B * p.Hkv * nhb * p.n_chunks;
   const int64_t total_recs = static_cast<int64_t>(p.B) * p.Hkv * p.Nmax;
-  auto item_range = [&](int item, int& bh, int& chunk, int& k0, int& k1) {
-    bh = item / p.n_chunks;
-    chunk = item - bh * p.n_chunks;
+  // item -> (bh, head block, chunk, token range)
+  auto item_range = [&](int item, int& bh, int& hblk, int& chunk, int& k0, int& k1) {
+    chunk = item % p.n_chunks;
+    const int rest = item / p.n_chunks;
+    hblk = rest % nhb;
+    bh = rest / nhb;
     const int bb = bh / p.Hkv;
     const int len = static_cast<int>(min(static_cast<int64_t>(p.seq_lens[bb]), p.Nmax));
     k0 = chunk * p.chunk_len;
@@ -158,8 +179,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       int gs = 0;                                   // global stage counter of this CTA
       bool stop = false;
       for (int item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
-        int bh, chunk, k0, k1;
-        item_range(item, bh, chunk, k0, k1);
+        int bh, hblk, chunk, k0, k1;
+        item_range(item, bh, hblk, chunk, k0, k1);
         const int64_t rec0 = static_cast<int64_t>(bh) * p.Nmax;
         for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
           const int s = gs % kTmaStages, use = gs / kTmaStages;
@@ -202,58 +223,52 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   }
 
   // ---------------- consumers ----------------
-  const int G = p.G;
-  const int row0 = g, row1 = g + 8;
-  const bool r0ok = row0 < G, r1ok = !G8 && row1 < G;
-  const int kA = (g >> 1) + 4 * (g & 1);        // score n-tile 0 column g; n-tile 1 adds 8
-  const int kc[4] = {t, t + 4, 8 + t, 12 + t};  // columns 2t, 2t+1 of n-tiles 0 and 1
+  // score-tile row g holds token pg of the unit, row g + 8 token 8 + pg
+  const int pg = (g >> 1) + 4 * (g & 1);
+  // value-operand k-indices 2t, 2t+1, 2t+8, 2t+9 are the tokens of score rows 2t, 2t+1, ...
+  const int kv[4] = {t, t + 4, 8 + t, 12 + t};
   int gs = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    int bh, chunk, k0, k1;
-    item_range(item, bh, chunk, k0, k1);
+    int bh, hblk, chunk, k0, k1;
+    item_range(item, bh, hblk, chunk, k0, k1);
     const int bb = bh / p.Hkv, hk = bh - bb * p.Hkv;
     const int64_t rec0 = static_cast<int64_t>(bh) * p.Nmax;
-    const int64_t qrow0 = static_cast<int64_t>(bb) * p.Hq + hk * G + row0;
-    const int64_t qrow1 = static_cast<int64_t>(bb) * p.Hq + hk * G + row1;
-    uint32_t qa[KST][4], ql[KST][4];
+    const int h0 = hblk * HB;                         // first head of this block in the group
+    const int nh = min(HB, G - h0);
+    const int64_t qbase = static_cast<int64_t>(bb) * p.Hq + hk * G + h0;
+    // query operand (B of the score MMA): column g = head h0 + g
+    const bool hok = g < nh;
+    uint32_t qh[KST][2], ql[KST][2];
 #pragma unroll
     for (int s = 0; s < KST; ++s) {
       const int dm = t * TDK + 4 * s;
-      float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
-      if (r0ok) for (int i = 0; i < 4; ++i) a[i] = p.qa[qrow0 * D + dm + i];
-      if (r1ok) for (int i = 0; i < 4; ++i) b[i] = p.qa[qrow1 * D + dm + i];
-      split_pair(a[0], a[1], qa[s][0], ql[s][0]);
-      split_pair(a[2], a[3], qa[s][2], ql[s][2]);
-      if constexpr (G8) {
-        qa[s][1] = ql[s][1] = qa[s][3] = ql[s][3] = 0u;
-      } else {
-        split_pair(b[0], b[1], qa[s][1], ql[s][1]);
-        split_pair(b[2], b[3], qa[s][3], ql[s][3]);
-      }
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+      if (hok) for (int i = 0; i < 4; ++i) a[i] = p.qa[(qbase + g) * D + dm + i];
+      split_pair(a[0], a[1], qh[s][0], ql[s][0]);
+      split_pair(a[2], a[3], qh[s][1], ql[s][1]);
     }
-    // QJL operand: one half-precision pass suffices, since its term is the residual part
-    // of the score (a 2^-12 relative error on it is ~1e-5 of the score)
-    uint32_t qb[KST][4];
+    uint32_t qb[KST][2];
     if constexpr (KF == KFMT_PROD) {
 #pragma unroll
       for (int s = 0; s < KST; ++s) {
         const int dm = t * TDK + 4 * s;
-        float a[4] = {0.f, 0.f, 0.f, 0.f}, c[4] = {0.f, 0.f, 0.f, 0.f};
-        if (r0ok) for (int i = 0; i < 4; ++i) a[i] = p.qb[qrow0 * p.qb_stride + dm + i];
-        if (r1ok) for (int i = 0; i < 4; ++i) c[i] = p.qb[qrow1 * p.qb_stride + dm + i];
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        if (hok) for (int i = 0; i < 4; ++i) a[i] = p.qb[(qbase + g) * p.qb_stride + dm + i];
         qb[s][0] = pack_half2(a[0], a[1]);
-        qb[s][1] = G8 ? 0u : pack_half2(c[0], c[1]);
-        qb[s][2] = pack_half2(a[2], a[3]);
-        qb[s][3] = G8 ? 0u : pack_half2(c[2], c[3]);
+        qb[s][1] = pack_half2(a[2], a[3]);
       }
     }
-    const float sa0 = r0ok ? p.qs[qrow0 * 2] * p.k_scale : 0.f, sa1 = r1ok ? p.qs[qrow1 * 2] * p.k_scale : 0.f;
-    const float sb0 = r0ok ? p.qs[qrow0 * 2 + 1] : 0.f, sb1 = r1ok ? p.qs[qrow1 * 2 + 1] : 0.f;
+    // this thread's score columns are heads 2t, 2t+1 of the block
+    const bool c0ok = 2 * t < nh, c1ok = 2 * t + 1 < nh;
+    const float sa0 = c0ok ? p.qs[(qbase + 2 * t) * 2] * p.k_scale : 0.f;
+    const float sa1 = c1ok ? p.qs[(qbase + 2 * t + 1) * 2] * p.k_scale : 0.f;
+    const float sb0 = c0ok ? p.qs[(qbase + 2 * t) * 2 + 1] * p.qjl_coef : 0.f;
+    const float sb1 = c1ok ? p.qs[(qbase + 2 * t + 1) * 2 + 1] * p.qjl_coef : 0.f;
 
-    float o[NT][4];
+    float o[MT][4];
 #pragma unroll
-    for (int i = 0; i < NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads 2t, 2t+1
 
     for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
       const int s = gs % kTmaStages;
@@ -267,190 +282,182 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       const int nn = nb_count[s], noff = nb_off[s];
       const int u0 = warp * 16;                      // first token of this warp's unit (stage-local)
       // ---- pull this warp's slices out of the stage ----
+      const int ka = u0 + pg, kb2 = u0 + 8 + pg;     // tokens of score rows g, g + 8
+      const bool oka = ka < cnt, okb = kb2 < cnt;
       uint32_t ks0[NWK], ks1[NWK];
-      load_slice<NWK, false>(skc + (u0 + kA) * KW, KW, t * TDK * KB, u0 + kA < cnt, ks0);
-      load_slice<NWK, false>(skc + (u0 + 8 + kA) * KW, KW, t * TDK * KB, u0 + 8 + kA < cnt, ks1);
+      load_slice<NWK, false>(skc + ka * KW, KW, t * TDK * KB, oka, ks0);
+      load_slice<NWK, false>(skc + kb2 * KW, KW, t * TDK * KB, okb, ks1);
+      auto norm_of = [&](const float* staged, const float* global, int lk, bool ok) {
+        return ok ? (lk < nn ? staged[noff + lk] : __ldg(global + rec0 + t0 + lk)) : 0.f;
+      };
+      const float kn0 = norm_of(skn, p.knorms, ka, oka), kn1 = norm_of(skn, p.knorms, kb2, okb);
+      const float vn0 = norm_of(svn, p.vnorms, ka, oka), vn1 = norm_of(svn, p.vnorms, kb2, okb);
+      float gm0 = 0.f, gm1 = 0.f;
+      uint32_t sw0 = 0u, sw1 = 0u;
+      if constexpr (KF == KFMT_PROD) {
+        const float* srn = reinterpret_cast<const float*>(sb + SL.krn);
+        gm0 = norm_of(srn, p.krnorms, ka, oka);
+        gm1 = norm_of(srn, p.krnorms, kb2, okb);
+        const uint32_t* ssg = reinterpret_cast<const uint32_t*>(sb + SL.ksign);
+        sw0 = oka ? ssg[ka * KSW + t] : 0u;
+        sw1 = okb ? ssg[kb2 * KSW + t] : 0u;
+      }
       uint32_t vs[4][NWV];
-      float kn[4], vn[4], gm[4];
-      uint32_t sw[2] = {0u, 0u};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int lk = u0 + kc[i];
-        const bool ok = lk < cnt;
-        load_slice<NWV, false>(svc + lk * VW, VW, g * TDV * VB, ok, vs[i]);
-        const int64_t gi = rec0 + t0 + lk;
-        kn[i] = ok ? (lk < nn ? skn[noff + lk] : __ldg(p.knorms + gi)) : 0.f;
-        vn[i] = ok ? (lk < nn ? svn[noff + lk] : __ldg(p.vnorms + gi)) : 0.f;
-        if constexpr (KF == KFMT_PROD) {
-          const float* srn = reinterpret_cast<const float*>(sb + SL.krn);
-          gm[i] = ok ? (lk < nn ? srn[noff + lk] : __ldg(p.krnorms + gi)) : 0.f;
-        } else {
-          gm[i] = 0.f;
-        }
-      }
-      if constexpr (KF == KFMT_PROD) {
-        const uint32_t* ssg = reinterpret_cast<const uint32_t*>(sb + SL.ksign);
-        sw[0] = (u0 + kA < cnt) ? ssg[(u0 + kA) * KSW + t] : 0u;
-        sw[1] = (u0 + 8 + kA < cnt) ? ssg[(u0 + 8 + kA) * KSW + t] : 0u;
+        const int lk = u0 + kv[i];
+        load_slice<NWV, false>(svc + lk * VW, VW, g * TDV * VB, lk < cnt, vs[i]);
       }
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(s)) : "memory");
       if (u0 >= cnt) continue;
 
-      // ---- scores ----
-      float sc[2][4];
+      // ---- scores: S[16 tokens x 8 heads] ----
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, accl[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        // hi and lo query halves accumulate separately: two independent MMA chains
-        float acc[4] = {0.f, 0.f, 0.f, 0.f}, accl[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t(&ks)[NWK] = nt ? ks1 : ks0;
+      for (int s2 = 0; s2 < KST; ++s2) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (KB == 4) {
+          // dims (4 s2, 4 s2 + 1) are byte 2 (s2 % 2) of word s2 / 2; (+2, +3) the next byte
+          const uint32_t w0 = ks0[s2 >> 1], w1 = ks1[s2 >> 1];
+          const uint32_t sel = 0x4440u + 2 * (s2 & 1);
+          a0 = lutk[(__byte_perm(w0, 0u, sel) << 5) + lane];
+          a1 = lutk[(__byte_perm(w1, 0u, sel) << 5) + lane];
+          a2 = lutk[(__byte_perm(w0, 0u, sel + 1) << 5) + lane];
+          a3 = lutk[(__byte_perm(w1, 0u, sel + 1) << 5) + lane];
+        } else {
+          a0 = lutk[(pair_at<KB, NWK>(ks0, 4 * s2 * KB) << 5) + lane];
+          a1 = lutk[(pair_at<KB, NWK>(ks1, 4 * s2 * KB) << 5) + lane];
+          a2 = lutk[(pair_at<KB, NWK>(ks0, (4 * s2 + 2) * KB) << 5) + lane];
+          a3 = lutk[(pair_at<KB, NWK>(ks1, (4 * s2 + 2) * KB) << 5) + lane];
+        }
+        mma16816(acc, a0, a1, a2, a3, qh[s2][0], qh[s2][1]);
+        mma16816(accl, a0, a1, a2, a3, ql[s2][0], ql[s2][1]);
+      }
+      float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (KF == KFMT_PROD) {
 #pragma unroll
         for (int s2 = 0; s2 < KST; ++s2) {
-          uint32_t b0, b1;
-          if constexpr (KB == 4) {
-            // the pair of dims (4 s2, 4 s2 + 1) is byte 2 (s2 % 2) of word s2 / 2
-            const uint32_t w = ks[s2 >> 1];
-            b0 = lutk[(__byte_perm(w, 0u, 0x4440u + 2 * (s2 & 1)) << 5) + lane];
-            b1 = lutk[(__byte_perm(w, 0u, 0x4441u + 2 * (s2 & 1)) << 5) + lane];
-          } else {
-            b0 = lutk[(pair_at<KB, NWK>(ks, 4 * s2 * KB) << 5) + lane];
-            b1 = lutk[(pair_at<KB, NWK>(ks, (4 * s2 + 2) * KB) << 5) + lane];
-          }
-          mma16816(acc, qa[s2][0], qa[s2][1], qa[s2][2], qa[s2][3], b0, b1);
-          mma16816(accl, ql[s2][0], ql[s2][1], ql[s2][2], ql[s2][3], b0, b1);
+          const uint32_t a0 = luts[(((sw0 >> (4 * s2)) & 3u) << 5) + lane];
+          const uint32_t a1 = luts[(((sw1 >> (4 * s2)) & 3u) << 5) + lane];
+          const uint32_t a2 = luts[(((sw0 >> (4 * s2 + 2)) & 3u) << 5) + lane];
+          const uint32_t a3 = luts[(((sw1 >> (4 * s2 + 2)) & 3u) << 5) + lane];
+          mma16816(acc2, a0, a1, a2, a3, qb[s2][0], qb[s2][1]);
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += accl[i];
-        float acc2[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (KF == KFMT_PROD) {
-          const uint32_t w = sw[nt];
-#pragma unroll
-          for (int s2 = 0; s2 < KST; ++s2) {
-            const uint32_t b0 = luts[(((w >> (4 * s2)) & 3u) << 5) + lane];
-            const uint32_t b1 = luts[(((w >> (4 * s2 + 2)) & 3u) << 5) + lane];
-            mma16816(acc2, qb[s2][0], qb[s2][1], qb[s2][2], qb[s2][3], b0, b1);
-          }
-        }
+      }
+      // acc[0], acc[1]: token row g, heads 2t, 2t+1; acc[2], acc[3]: token row g + 8
+      float sc[4];
+      {
+        const float kr[4] = {kn0, kn0, kn1, kn1};
+        const float gr[4] = {gm0, gm0, gm1, gm1};
+        const float sa[4] = {sa0, sa1, sa0, sa1}, sbq[4] = {sb0, sb1, sb0, sb1};
+        const bool ok[4] = {oka, oka, okb, okb};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int ci = nt * 2 + (i & 1);
-          const float sa = (i < 2) ? sa0 : sa1, sbv = (i < 2) ? sb0 : sb1;
-          float v;
-          if constexpr (KF == KFMT_PROD) v = kn[ci] * (sa * acc[i] + p.qjl_coef * gm[ci] * sbv * acc2[i]);
-          else v = kn[ci] * sa * acc[i];
-          sc[nt][i] = (u0 + kc[ci] < cnt) ? v : -INFINITY;
+          float v = sa[i] * (acc[i] + accl[i]);
+          if constexpr (KF == KFMT_PROD) v += gr[i] * sbq[i] * acc2[i];
+          sc[i] = ok[i] ? kr[i] * v : -INFINITY;
         }
       }
-      // ---- online softmax (log2 domain) ----
-      float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      const float mn0 = fmaxf(m0, mx0);
-      if (mn0 > m0) {
-        const float f = exp2f(m0 - mn0);
-        l0 *= f;
+      // ---- online softmax per head (log2 domain), reduced over the 8 token rows ----
+      float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
-        for (int i = 0; i < NT; ++i) { o[i][0] *= f; o[i][1] *= f; }
+      for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      if (mn0 > m0 || mn1 > m1) {
+        const float f0 = exp2f(m0 - mn0), f1 = exp2f(m1 - mn1);
+        l0 *= f0;
+        l1 *= f1;
+#pragma unroll
+        for (int i = 0; i < MT; ++i) { o[i][0] *= f0; o[i][2] *= f0; o[i][1] *= f1; o[i][3] *= f1; }
         m0 = mn0;
+        m1 = mn1;
       }
-      if constexpr (!G8) {
-        float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn1 = fmaxf(m1, mx1);
-        if (G > 8 && mn1 > m1) {
-          const float f = exp2f(m1 - mn1);
-          l1 *= f;
-#pragma unroll
-          for (int i = 0; i < NT; ++i) { o[i][2] *= f; o[i][3] *= f; }
-          m1 = mn1;
-        }
-      }
-      float pr[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        pr[nt][0] = r0ok ? exp2f(sc[nt][0] - m0) : 0.f;
-        pr[nt][1] = r0ok ? exp2f(sc[nt][1] - m0) : 0.f;
-        pr[nt][2] = r1ok ? exp2f(sc[nt][2] - m1) : 0.f;
-        pr[nt][3] = r1ok ? exp2f(sc[nt][3] - m1) : 0.f;
-        l0 += pr[nt][0] + pr[nt][1];
-        l1 += pr[nt][2] + pr[nt][3];
-      }
-      uint32_t pa0, pa1, pa2, pa3, pl0, pl1, pl2, pl3;
-      split_pair(pr[0][0] * vn[0], pr[0][1] * vn[1], pa0, pl0);
-      split_pair(pr[1][0] * vn[2], pr[1][1] * vn[3], pa2, pl2);
-      if constexpr (G8) {
-        pa1 = pl1 = pa3 = pl3 = 0u;
-      } else {
-        split_pair(pr[0][2] * vn[0], pr[0][3] * vn[1], pa1, pl1);
-        split_pair(pr[1][2] * vn[2], pr[1][3] * vn[3], pa3, pl3);
-      }
-      // ---- P.V in the rotated domain ----
+      const float p00 = c0ok ? exp2f(sc[0] - m0) : 0.f, p01 = c1ok ? exp2f(sc[1] - m1) : 0.f;
+      const float p10 = c0ok ? exp2f(sc[2] - m0) : 0.f, p11 = c1ok ? exp2f(sc[3] - m1) : 0.f;
+      l0 += p00 + p10;
+      l1 += p01 + p11;
+      // P^T (16 tokens x 8 heads) as the B operand: transpose the two 8x8 halves
+      uint32_t pth, ptl, pbh, pbl;
+      split_pair(p00 * vn0, p01 * vn0, pth, ptl);
+      split_pair(p10 * vn1, p11 * vn1, pbh, pbl);
+      const uint32_t b0h = movmatrix_t(pth), b1h = movmatrix_t(pbh);
+      const uint32_t b0l = movmatrix_t(ptl), b1l = movmatrix_t(pbl);
+      // ---- O'^T[128 dims x 8 heads] += V_hat^T . P^T ----
+      // M-tile i: row g = dim TDV g + i (first word of the slice), row g + 8 = dim TDV g + 8 + i
       if constexpr (VB == 4) {
-        // byte j of lo (hi) holds the codes of keys (t, t + 4) for dim 2j (2j + 1) of a word
+        // byte j of lo (hi) holds the codes of one token pair for dim 2j (2j + 1) of a word
+        uint32_t lo[2][2], hi[2][2];   // [token pair][word]
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-          const uint32_t a0 = vs[0][w], a1 = vs[1][w], c0 = vs[2][w], c1 = vs[3][w];
-          const uint32_t lo01 = (a0 & 0x0F0F0F0Fu) | ((a1 << 4) & 0xF0F0F0F0u);
-          const uint32_t hi01 = ((a0 >> 4) & 0x0F0F0F0Fu) | (a1 & 0xF0F0F0F0u);
-          const uint32_t lo23 = (c0 & 0x0F0F0F0Fu) | ((c1 << 4) & 0xF0F0F0F0u);
-          const uint32_t hi23 = ((c0 >> 4) & 0x0F0F0F0Fu) | (c1 & 0xF0F0F0F0u);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int i = 8 * w + j;                  // n-tile = dim within this thread's 16
-            const uint32_t x01 = (j & 1) ? hi01 : lo01, x23 = (j & 1) ? hi23 : lo23;
-            const uint32_t b0 = lutv[(__byte_perm(x01, 0u, 0x4440u + (j >> 1)) << 5) + lane];
-            const uint32_t b1 = lutv[(__byte_perm(x23, 0u, 0x4440u + (j >> 1)) << 5) + lane];
-            mma16816(o[i], pa0, pa1, pa2, pa3, b0, b1);
-            mma16816(o[i], pl0, pl1, pl2, pl3, b0, b1);
+          for (int kp = 0; kp < 2; ++kp) {
+            const uint32_t x = vs[2 * kp][w], y = vs[2 * kp + 1][w];
+            lo[kp][w] = (x & 0x0F0F0F0Fu) | ((y << 4) & 0xF0F0F0F0u);
+            hi[kp][w] = ((x >> 4) & 0x0F0F0F0Fu) | (y & 0xF0F0F0F0u);
           }
+        }
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          const uint32_t sel = 0x4440u + (i >> 1);
+          const uint32_t a0 = lutv[(__byte_perm((i & 1) ? hi[0][0] : lo[0][0], 0u, sel) << 5) + lane];
+          const uint32_t a1 = lutv[(__byte_perm((i & 1) ? hi[0][1] : lo[0][1], 0u, sel) << 5) + lane];
+          const uint32_t a2 = lutv[(__byte_perm((i & 1) ? hi[1][0] : lo[1][0], 0u, sel) << 5) + lane];
+          const uint32_t a3 = lutv[(__byte_perm((i & 1) ? hi[1][1] : lo[1][1], 0u, sel) << 5) + lane];
+          mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
+          mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < NT; ++i) {
-          const uint32_t e01 = field_at<VB, NWV>(vs[0], i * VB) | (field_at<VB, NWV>(vs[1], i * VB) << VB);
-          const uint32_t e23 = field_at<VB, NWV>(vs[2], i * VB) | (field_at<VB, NWV>(vs[3], i * VB) << VB);
-          const uint32_t b0 = lutv[(e01 << 5) + lane], b1 = lutv[(e23 << 5) + lane];
-          mma16816(o[i], pa0, pa1, pa2, pa3, b0, b1);
-          mma16816(o[i], pl0, pl1, pl2, pl3, b0, b1);
+        for (int i = 0; i < MT; ++i) {
+          const uint32_t e00 = field_at<VB, NWV>(vs[0], i * VB) | (field_at<VB, NWV>(vs[1], i * VB) << VB);
+          const uint32_t e01 = field_at<VB, NWV>(vs[0], (8 + i) * VB) | (field_at<VB, NWV>(vs[1], (8 + i) * VB) << VB);
+          const uint32_t e10 = field_at<VB, NWV>(vs[2], i * VB) | (field_at<VB, NWV>(vs[3], i * VB) << VB);
+          const uint32_t e11 = field_at<VB, NWV>(vs[2], (8 + i) * VB) | (field_at<VB, NWV>(vs[3], (8 + i) * VB) << VB);
+          const uint32_t a0 = lutv[(e00 << 5) + lane], a1 = lutv[(e01 << 5) + lane];
+          const uint32_t a2 = lutv[(e10 << 5) + lane], a3 = lutv[(e11 << 5) + lane];
+          mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
+          mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
         }
       }
     }
 
     // ---- merge this item across the consumer warps (named barrier 1) ----
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    float* wm = mrg + warp * MROWS * (D + 2);
-    if (t == 0) {
-      wm[row0 * (D + 2)] = m0; wm[row0 * (D + 2) + 1] = l0;
-      if constexpr (!G8) { wm[row1 * (D + 2)] = m1; wm[row1 * (D + 2) + 1] = l1; }
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
+    }
+    float* wm = mrg + warp * HB * (D + 2);          // [head][m, l, o'[D]]
+    if (g == 0) {
+      wm[(2 * t) * (D + 2)] = m0; wm[(2 * t) * (D + 2) + 1] = l0;
+      wm[(2 * t + 1) * (D + 2)] = m1; wm[(2 * t + 1) * (D + 2) + 1] = l1;
     }
 #pragma unroll
-    for (int i = 0; i < NT; ++i) {
-      wm[row0 * (D + 2) + 2 + (2 * t) * TDV + i] = o[i][0];
-      wm[row0 * (D + 2) + 2 + (2 * t + 1) * TDV + i] = o[i][1];
-      if constexpr (!G8) {
-        wm[row1 * (D + 2) + 2 + (2 * t) * TDV + i] = o[i][2];
-        wm[row1 * (D + 2) + 2 + (2 * t + 1) * TDV + i] = o[i][3];
-      }
+    for (int i = 0; i < MT; ++i) {
+      wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = o[i][0];
+      wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = o[i][1];
+      wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][2];
+      wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][3];
     }
     asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
-    for (int idx = tid; idx < G * D; idx += CONSUMERS) {
+    for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
       const int r = idx / D, j = idx - r * D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kTmaConsumerWarps; ++w) M = fmaxf(M, mrg[(w * MROWS + r) * (D + 2)]);
+      for (int w = 0; w < kTmaConsumerWarps; ++w) M = fmaxf(M, mrg[(w * HB + r) * (D + 2)]);
       float a = 0.f, L = 0.f;
 #pragma unroll
       for (int w = 0; w < kTmaConsumerWarps; ++w) {
-        const float* row = mrg + (w * MROWS + r) * (D + 2);
+        const float* row = mrg + (w * HB + r) * (D + 2);
         const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
         L += f * row[1];
         a += f * row[2 + j];
       }
-      const int64_t qi = static_cast<int64_t>(bb) * p.Hq + hk * G + r;
+      const int64_t qi = qbase + r;
       const int64_t pi = qi * p.n_chunks + chunk;
       if (j == 0) { p.part_ml[pi * 2] = M; p.part_ml[pi * 2 + 1] = L; }
       p.part_o[pi * D + j] = a * p.v_scale;

@@ -276,11 +276,13 @@ DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t N
   int64_t nch, cl;
   if (kq->kind != TQ_KIND_SPECTRAL) {
     // persistent bulk-copy kernel: about 16 work items per SM, chunks of whole 112-token
-    // stages, and (when the shape allows) an item count that is a multiple of the SMs
+    // stages, and (when the shape allows) an item count that is a multiple of the SMs;
+    // a work item covers one block of up to 8 query heads of a GQA group
     const int64_t stage = 112;
-    int64_t n0 = std::max<int64_t>(1, (16 * sms + units - 1) / units);
+    const int64_t wu = units * tma_head_blocks(Hq / Hkv);
+    int64_t n0 = std::max<int64_t>(1, (16 * sms + wu - 1) / wu);
     for (int64_t cand = n0; cand < n0 + 8 && cand <= Nmax; ++cand)
-      if ((units * cand) % sms == 0) { n0 = cand; break; }
+      if ((wu * cand) % sms == 0) { n0 = cand; break; }
     cl = (Nmax + n0 - 1) / n0;
     cl = std::max<int64_t>(stage, (cl + stage - 1) / stage * stage);
     nch = (Nmax + cl - 1) / cl;
@@ -616,7 +618,7 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   dp.k_scale = kq->lut_scale > 0.f ? kq->lut_scale : 1.f;
   dp.v_scale = vq->lut_scale > 0.f ? vq->lut_scale : 1.f;
   dp.part_ml = pml; dp.part_o = po;
-  const int64_t items = static_cast<int64_t>(B) * Hkv * P.n_chunks;
+  const int64_t items = static_cast<int64_t>(B) * Hkv * tma_head_blocks(G) * P.n_chunks;
   const dim3 grid = kfmt == KFMT_SPEC ? dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv))
                                       : dim3(static_cast<unsigned>(std::min<int64_t>(items, sm_count())));
   const size_t smem = decode_smem_bytes(D, kb, vb);
