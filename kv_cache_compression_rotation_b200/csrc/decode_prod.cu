@@ -11,7 +11,7 @@ cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, in
   smem = decode_tma_smem_bytes(KB, VB, KFMT_PROD, 4);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k<<<grid, kTmaThreads, smem, s>>>(p, status, lim);
+  k<<<grid, (tma_consumers(KFMT_PROD) + 1) * 32, smem, s>>>(p, status, lim);
   return cudaGetLastError();
 }
 

@@ -4,9 +4,9 @@
 // (decode.cuh): logit = scale * est(q, k_i), online softmax, o' = sum p ||v|| c[code_v].
 //
 // Streaming.  Persistent CTAs (one per SM) walk work items (batch * kv-head, head block,
-// context chunk).  One producer warp copies each item in stages of 112 tokens with
+// context chunk).  One producer warp copies each item in stages of 16 tokens per consumer warp with
 // cp.async.bulk (key codes, value codes, norms; prod adds sign words and residual norms)
-// into a 4-deep shared-memory ring; seven consumer warps each take 16 tokens of a stage,
+// into a 4-deep shared-memory ring; 11 (prod: 7) consumer warps each take 16 tokens of a stage,
 // pull their record slices into registers, release the stage and compute.
 //
 // Math per 16-token unit, all on mma.sync m16n8k16 (fp16 in, fp32 accumulate):
@@ -30,9 +30,10 @@
 
 namespace tq {
 
-constexpr int kTmaConsumerWarps = 7;
-constexpr int kTmaThreads = (kTmaConsumerWarps + 1) * 32;
-constexpr int kTmaStageTokens = kTmaConsumerWarps * 16;
+// Consumer warps per CTA: MSE keys fit 11 (plus the producer: 12 warps of <= 168
+// registers fill the register file); PROD keys need more registers and run 7.
+__host__ __device__ constexpr int tma_consumers(int kf) { return kf == KFMT_PROD ? 7 : 11; }
+__host__ __device__ constexpr int tma_stage_tokens(int kf) { return tma_consumers(kf) * 16; }
 constexpr int kTmaStages = 4;
 constexpr int kTmaHeadBlock = 8;     // query heads per work item (MMA N)
 
@@ -80,31 +81,51 @@ struct TmaStageLayout {
 
 // Byte offsets of the arrays of one stage (all 16-byte aligned).
 __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int kf, int ksw) {
+  const int st = tma_stage_tokens(kf);
   TmaStageLayout L{};
   uint32_t o = 0;
-  L.kcodes = o; o += kTmaStageTokens * kw * 4;
-  L.vcodes = o; o += kTmaStageTokens * vw * 4;
-  L.knorm = o; o += (kTmaStageTokens + 4) * 4;
-  L.vnorm = o; o += (kTmaStageTokens + 4) * 4;
-  L.ksign = o; o += (kf == KFMT_PROD) ? kTmaStageTokens * ksw * 4 : 0;
-  L.krn = o; o += (kf == KFMT_PROD) ? (kTmaStageTokens + 4) * 4 : 0;
+  L.kcodes = o; o += st * kw * 4;
+  L.vcodes = o; o += st * vw * 4;
+  L.knorm = o; o += (st + 4) * 4;
+  L.vnorm = o; o += (st + 4) * 4;
+  L.ksign = o; o += (kf == KFMT_PROD) ? st * ksw * 4 : 0;
+  L.krn = o; o += (kf == KFMT_PROD) ? (st + 4) * 4 : 0;
   L.bytes = o;
   return L;
 }
 
 inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, int ksw) {
-  const size_t tables = (static_cast<size_t>(1u << (2 * kb)) + (1u << (2 * vb)) + 4) * 32 * 4;
+  const size_t ne = static_cast<size_t>(1u << (2 * (kb > vb ? kb : vb)));
+  const size_t tables = (ne * 64 + 4 * 32) * 4;
   const TmaStageLayout L = tma_stage_layout(128 * kb / 32, 128 * vb / 32, kf, ksw);
-  const size_t merge = static_cast<size_t>(kTmaConsumerWarps) * kTmaHeadBlock * (128 + 2) * 4;
+  const size_t merge = static_cast<size_t>(tma_consumers(kf)) * kTmaHeadBlock * (128 + 2) * 4;
   return tables + static_cast<size_t>(kTmaStages) * L.bytes + merge + 2 * kTmaStages * 8 + 64 + 16;
 }
 
 // Head blocks per GQA group (work items split groups larger than 8 heads).
 __host__ __device__ inline int tma_head_blocks(int G) { return (G + kTmaHeadBlock - 1) / kTmaHeadBlock; }
 
+__device__ __forceinline__ uint32_t tab_ld(const char* tab, uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(tab + off);
+}
+
+// Byte k of w as table entry index, combined with this lane's byte offset `lo8` (< 256).
+__device__ __forceinline__ uint32_t tab_off(uint32_t w, uint32_t lo8, int k) {
+  return __byte_perm(w, lo8, 0x7604u | (static_cast<uint32_t>(k) << 4));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int KF, int KB, int VB>
-__global__ void __launch_bounds__(kTmaThreads, 1)
+__global__ void __launch_bounds__((tma_consumers(KF) + 1) * 32, 1)
 decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
+  constexpr int kTmaConsumerWarps = tma_consumers(KF);
+  constexpr int kTmaThreads = (kTmaConsumerWarps + 1) * 32;
+  constexpr int kTmaStageTokens = tma_stage_tokens(KF);
   constexpr int D = 128;
   constexpr int KST = D / 16;                 // mma k-steps over the key dims
   constexpr int TDK = D / 4;                  // key dims per thread
@@ -117,10 +138,12 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int KSW = 4;                                // prod sign words (m = 128)
   constexpr int HB = kTmaHeadBlock;
   constexpr int CONSUMERS = kTmaConsumerWarps * 32;
+  constexpr int NE = KLUT > VLUT ? KLUT : VLUT;        // table entries
   extern __shared__ __align__(128) uint32_t tsm_[];
-  uint32_t* lutk = tsm_;
-  uint32_t* lutv = lutk + KLUT * 32;
-  uint32_t* luts = lutv + VLUT * 32;
+  // table entry e is 256 B: the key value pair for lanes 0..31, then the value pair; a
+  // lookup address is (e << 8) | (lane * 4) [+ 128], one byte permute from the code word
+  const char* tab = reinterpret_cast<const char*>(tsm_);
+  uint32_t* luts = tsm_ + NE * 64;
   unsigned char* stage0 = reinterpret_cast<unsigned char*>(luts + 4 * 32);
   const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW);
   float* mrg = reinterpret_cast<float*>(stage0 + static_cast<size_t>(kTmaStages) * SL.bytes);
@@ -159,13 +182,16 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int i = tid; i < KLUT * 32; i += kTmaThreads) {
-    const int e = i >> 5;
-    lutk[i] = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) / p.k_scale, __ldg(p.kc + (e >> KB)) / p.k_scale);
-  }
-  for (int i = tid; i < VLUT * 32; i += kTmaThreads) {
-    const int e = i >> 5;
-    lutv[i] = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
+  for (int i = tid; i < NE * 64; i += kTmaThreads) {
+    const int e = i >> 6;
+    uint32_t val = 0u;
+    if ((i & 32) == 0) {
+      if (e < KLUT)
+        val = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) / p.k_scale, __ldg(p.kc + (e >> KB)) / p.k_scale);
+    } else if (e < VLUT) {
+      val = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
+    }
+    tsm_[i] = val;
   }
   if (tid < 128) {
     const int e = tid >> 5;
@@ -227,6 +253,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   const int pg = (g >> 1) + 4 * (g & 1);
   // value-operand k-indices 2t, 2t+1, 2t+8, 2t+9 are the tokens of score rows 2t, 2t+1, ...
   const int kv[4] = {t, t + 4, 8 + t, 12 + t};
+  const uint32_t klo = static_cast<uint32_t>(lane) * 4u, vlo = klo + 128u;
   int gs = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     int bh, hblk, chunk, k0, k1;
@@ -320,16 +347,16 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         if constexpr (KB == 4) {
           // dims (4 s2, 4 s2 + 1) are byte 2 (s2 % 2) of word s2 / 2; (+2, +3) the next byte
           const uint32_t w0 = ks0[s2 >> 1], w1 = ks1[s2 >> 1];
-          const uint32_t sel = 0x4440u + 2 * (s2 & 1);
-          a0 = lutk[(__byte_perm(w0, 0u, sel) << 5) + lane];
-          a1 = lutk[(__byte_perm(w1, 0u, sel) << 5) + lane];
-          a2 = lutk[(__byte_perm(w0, 0u, sel + 1) << 5) + lane];
-          a3 = lutk[(__byte_perm(w1, 0u, sel + 1) << 5) + lane];
+          const int k = 2 * (s2 & 1);
+          a0 = tab_ld(tab, tab_off(w0, klo, k));
+          a1 = tab_ld(tab, tab_off(w1, klo, k));
+          a2 = tab_ld(tab, tab_off(w0, klo, k + 1));
+          a3 = tab_ld(tab, tab_off(w1, klo, k + 1));
         } else {
-          a0 = lutk[(pair_at<KB, NWK>(ks0, 4 * s2 * KB) << 5) + lane];
-          a1 = lutk[(pair_at<KB, NWK>(ks1, 4 * s2 * KB) << 5) + lane];
-          a2 = lutk[(pair_at<KB, NWK>(ks0, (4 * s2 + 2) * KB) << 5) + lane];
-          a3 = lutk[(pair_at<KB, NWK>(ks1, (4 * s2 + 2) * KB) << 5) + lane];
+          a0 = tab_ld(tab, (pair_at<KB, NWK>(ks0, 4 * s2 * KB) << 8) | klo);
+          a1 = tab_ld(tab, (pair_at<KB, NWK>(ks1, 4 * s2 * KB) << 8) | klo);
+          a2 = tab_ld(tab, (pair_at<KB, NWK>(ks0, (4 * s2 + 2) * KB) << 8) | klo);
+          a3 = tab_ld(tab, (pair_at<KB, NWK>(ks1, (4 * s2 + 2) * KB) << 8) | klo);
         }
         mma16816(acc, a0, a1, a2, a3, qh[s2][0], qh[s2][1]);
         mma16816(accl, a0, a1, a2, a3, ql[s2][0], ql[s2][1]);
@@ -368,7 +395,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       }
       const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
       if (mn0 > m0 || mn1 > m1) {
-        const float f0 = exp2f(m0 - mn0), f1 = exp2f(m1 - mn1);
+        const float f0 = ex2(m0 - mn0), f1 = ex2(m1 - mn1);
         l0 *= f0;
         l1 *= f1;
 #pragma unroll
@@ -376,8 +403,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         m0 = mn0;
         m1 = mn1;
       }
-      const float p00 = c0ok ? exp2f(sc[0] - m0) : 0.f, p01 = c1ok ? exp2f(sc[1] - m1) : 0.f;
-      const float p10 = c0ok ? exp2f(sc[2] - m0) : 0.f, p11 = c1ok ? exp2f(sc[3] - m1) : 0.f;
+      const float p00 = c0ok ? ex2(sc[0] - m0) : 0.f, p01 = c1ok ? ex2(sc[1] - m1) : 0.f;
+      const float p10 = c0ok ? ex2(sc[2] - m0) : 0.f, p11 = c1ok ? ex2(sc[3] - m1) : 0.f;
       l0 += p00 + p10;
       l1 += p01 + p11;
       // P^T (16 tokens x 8 heads) as the B operand: transpose the two 8x8 halves
@@ -402,11 +429,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         }
 #pragma unroll
         for (int i = 0; i < MT; ++i) {
-          const uint32_t sel = 0x4440u + (i >> 1);
-          const uint32_t a0 = lutv[(__byte_perm((i & 1) ? hi[0][0] : lo[0][0], 0u, sel) << 5) + lane];
-          const uint32_t a1 = lutv[(__byte_perm((i & 1) ? hi[0][1] : lo[0][1], 0u, sel) << 5) + lane];
-          const uint32_t a2 = lutv[(__byte_perm((i & 1) ? hi[1][0] : lo[1][0], 0u, sel) << 5) + lane];
-          const uint32_t a3 = lutv[(__byte_perm((i & 1) ? hi[1][1] : lo[1][1], 0u, sel) << 5) + lane];
+          const int k = i >> 1;
+          const uint32_t a0 = tab_ld(tab, tab_off((i & 1) ? hi[0][0] : lo[0][0], vlo, k));
+          const uint32_t a1 = tab_ld(tab, tab_off((i & 1) ? hi[0][1] : lo[0][1], vlo, k));
+          const uint32_t a2 = tab_ld(tab, tab_off((i & 1) ? hi[1][0] : lo[1][0], vlo, k));
+          const uint32_t a3 = tab_ld(tab, tab_off((i & 1) ? hi[1][1] : lo[1][1], vlo, k));
           mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
           mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
         }
@@ -417,8 +444,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           const uint32_t e01 = field_at<VB, NWV>(vs[0], (8 + i) * VB) | (field_at<VB, NWV>(vs[1], (8 + i) * VB) << VB);
           const uint32_t e10 = field_at<VB, NWV>(vs[2], i * VB) | (field_at<VB, NWV>(vs[3], i * VB) << VB);
           const uint32_t e11 = field_at<VB, NWV>(vs[2], (8 + i) * VB) | (field_at<VB, NWV>(vs[3], (8 + i) * VB) << VB);
-          const uint32_t a0 = lutv[(e00 << 5) + lane], a1 = lutv[(e01 << 5) + lane];
-          const uint32_t a2 = lutv[(e10 << 5) + lane], a3 = lutv[(e11 << 5) + lane];
+          const uint32_t a0 = tab_ld(tab, (e00 << 8) | vlo), a1 = tab_ld(tab, (e01 << 8) | vlo);
+          const uint32_t a2 = tab_ld(tab, (e10 << 8) | vlo), a3 = tab_ld(tab, (e11 << 8) | vlo);
           mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
           mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
         }
