@@ -105,8 +105,53 @@ inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, int ksw) {
 // Head blocks per GQA group (work items split groups larger than 8 heads).
 __host__ __device__ inline int tma_head_blocks(int G) { return (G + kTmaHeadBlock - 1) / kTmaHeadBlock; }
 
-__device__ __forceinline__ uint32_t tab_ld(const char* tab, uint32_t off) {
-  return *reinterpret_cast<const uint32_t*>(tab + off);
+// Explicit shared-space loads (32-bit shared addresses): the stage and table reads must
+// be LDS, never generic loads through the global path.
+__device__ __forceinline__ uint32_t tab_ld(uint32_t tab, uint32_t off) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(tab + off));
+  return v;
+}
+__device__ __forceinline__ uint32_t sld32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float sldf(uint32_t a) { return __uint_as_float(sld32(a)); }
+
+// Slice of NW words of a record in shared memory starting at word w0 (aligned slices).
+template <int NW>
+__device__ __forceinline__ void sld_words(uint32_t a, bool valid, uint32_t (&w)[NW]) {
+  if constexpr (NW == 4) {
+    uint32_t x0 = 0, x1 = 0, x2 = 0, x3 = 0;
+    if (valid) asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(a) : "memory");
+    w[0] = x0; w[1] = x1; w[2] = x2; w[3] = x3;
+  } else if constexpr (NW == 2) {
+    uint32_t x0 = 0, x1 = 0;
+    if (valid) asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x0), "=r"(x1) : "r"(a) : "memory");
+    w[0] = x0; w[1] = x1;
+  } else {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) w[i] = valid ? sld32(a + 4 * i) : 0u;
+  }
+}
+
+// General slice (any bit offset): NW words starting at bit `base` of the record at `rec`.
+template <int NW>
+__device__ __forceinline__ void sld_slice(uint32_t rec, int rec_words, int base, bool valid, uint32_t (&seg)[NW]) {
+  const int w0 = base >> 5, sh = base & 31;
+  if (sh == 0 && (w0 * 4) % (NW == 4 ? 16 : (NW == 2 ? 8 : 4)) == 0) {
+    sld_words<NW>(rec + 4 * w0, valid, seg);
+    return;
+  }
+  uint32_t w[NW + 1];
+#pragma unroll
+  for (int i = 0; i <= NW; ++i) {
+    const int wi = w0 + i;
+    w[i] = (valid && wi < rec_words && (i < NW || sh != 0)) ? sld32(rec + 4 * wi) : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < NW; ++i) seg[i] = __funnelshift_r(w[i], w[i + 1], sh);
 }
 
 // Byte k of w as table entry index, combined with this lane's byte offset `lo8` (< 256).
@@ -142,8 +187,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   extern __shared__ __align__(128) uint32_t tsm_[];
   // table entry e is 256 B: the key value pair for lanes 0..31, then the value pair; a
   // lookup address is (e << 8) | (lane * 4) [+ 128], one byte permute from the code word
-  const char* tab = reinterpret_cast<const char*>(tsm_);
+  const uint32_t tab = tma_smem_u32(tsm_);
   uint32_t* luts = tsm_ + NE * 64;
+  const uint32_t luts_a = tma_smem_u32(luts);
   unsigned char* stage0 = reinterpret_cast<unsigned char*>(luts + 4 * 32);
   const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW);
   float* mrg = reinterpret_cast<float*>(stage0 + static_cast<size_t>(kTmaStages) * SL.bytes);
@@ -300,11 +346,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
       const int s = gs % kTmaStages;
       if (!tma_mbar_wait(full_bar(s), (gs / kTmaStages) & 1, wait_lim, status, abort_flag)) break;
-      const unsigned char* sb = stage0 + static_cast<size_t>(s) * SL.bytes;
-      const uint32_t* skc = reinterpret_cast<const uint32_t*>(sb + SL.kcodes);
-      const uint32_t* svc = reinterpret_cast<const uint32_t*>(sb + SL.vcodes);
-      const float* skn = reinterpret_cast<const float*>(sb + SL.knorm);
-      const float* svn = reinterpret_cast<const float*>(sb + SL.vnorm);
+      const uint32_t sb = tma_smem_u32(stage0) + static_cast<uint32_t>(s) * SL.bytes;
       const int cnt = min(kTmaStageTokens, k1 - t0);
       const int nn = nb_count[s], noff = nb_off[s];
       const int u0 = warp * 16;                      // first token of this warp's unit (stage-local)
@@ -312,28 +354,26 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       const int ka = u0 + pg, kb2 = u0 + 8 + pg;     // tokens of score rows g, g + 8
       const bool oka = ka < cnt, okb = kb2 < cnt;
       uint32_t ks0[NWK], ks1[NWK];
-      load_slice<NWK, false>(skc + ka * KW, KW, t * TDK * KB, oka, ks0);
-      load_slice<NWK, false>(skc + kb2 * KW, KW, t * TDK * KB, okb, ks1);
-      auto norm_of = [&](const float* staged, const float* global, int lk, bool ok) {
-        return ok ? (lk < nn ? staged[noff + lk] : __ldg(global + rec0 + t0 + lk)) : 0.f;
+      sld_slice<NWK>(sb + SL.kcodes + ka * KW * 4, KW, t * TDK * KB, oka, ks0);
+      sld_slice<NWK>(sb + SL.kcodes + kb2 * KW * 4, KW, t * TDK * KB, okb, ks1);
+      auto norm_of = [&](uint32_t staged, const float* global, int lk, bool ok) {
+        return ok ? (lk < nn ? sldf(staged + 4 * (noff + lk)) : __ldg(global + rec0 + t0 + lk)) : 0.f;
       };
-      const float kn0 = norm_of(skn, p.knorms, ka, oka), kn1 = norm_of(skn, p.knorms, kb2, okb);
-      const float vn0 = norm_of(svn, p.vnorms, ka, oka), vn1 = norm_of(svn, p.vnorms, kb2, okb);
+      const float kn0 = norm_of(sb + SL.knorm, p.knorms, ka, oka), kn1 = norm_of(sb + SL.knorm, p.knorms, kb2, okb);
+      const float vn0 = norm_of(sb + SL.vnorm, p.vnorms, ka, oka), vn1 = norm_of(sb + SL.vnorm, p.vnorms, kb2, okb);
       float gm0 = 0.f, gm1 = 0.f;
       uint32_t sw0 = 0u, sw1 = 0u;
       if constexpr (KF == KFMT_PROD) {
-        const float* srn = reinterpret_cast<const float*>(sb + SL.krn);
-        gm0 = norm_of(srn, p.krnorms, ka, oka);
-        gm1 = norm_of(srn, p.krnorms, kb2, okb);
-        const uint32_t* ssg = reinterpret_cast<const uint32_t*>(sb + SL.ksign);
-        sw0 = oka ? ssg[ka * KSW + t] : 0u;
-        sw1 = okb ? ssg[kb2 * KSW + t] : 0u;
+        gm0 = norm_of(sb + SL.krn, p.krnorms, ka, oka);
+        gm1 = norm_of(sb + SL.krn, p.krnorms, kb2, okb);
+        sw0 = oka ? sld32(sb + SL.ksign + (ka * KSW + t) * 4) : 0u;
+        sw1 = okb ? sld32(sb + SL.ksign + (kb2 * KSW + t) * 4) : 0u;
       }
       uint32_t vs[4][NWV];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int lk = u0 + kv[i];
-        load_slice<NWV, false>(svc + lk * VW, VW, g * TDV * VB, lk < cnt, vs[i]);
+        sld_slice<NWV>(sb + SL.vcodes + lk * VW * 4, VW, g * TDV * VB, lk < cnt, vs[i]);
       }
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(s)) : "memory");
@@ -365,10 +405,10 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       if constexpr (KF == KFMT_PROD) {
 #pragma unroll
         for (int s2 = 0; s2 < KST; ++s2) {
-          const uint32_t a0 = luts[(((sw0 >> (4 * s2)) & 3u) << 5) + lane];
-          const uint32_t a1 = luts[(((sw1 >> (4 * s2)) & 3u) << 5) + lane];
-          const uint32_t a2 = luts[(((sw0 >> (4 * s2 + 2)) & 3u) << 5) + lane];
-          const uint32_t a3 = luts[(((sw1 >> (4 * s2 + 2)) & 3u) << 5) + lane];
+          const uint32_t a0 = tab_ld(luts_a, ((((sw0 >> (4 * s2)) & 3u) << 5) + lane) * 4);
+          const uint32_t a1 = tab_ld(luts_a, ((((sw1 >> (4 * s2)) & 3u) << 5) + lane) * 4);
+          const uint32_t a2 = tab_ld(luts_a, ((((sw0 >> (4 * s2 + 2)) & 3u) << 5) + lane) * 4);
+          const uint32_t a3 = tab_ld(luts_a, ((((sw1 >> (4 * s2 + 2)) & 3u) << 5) + lane) * 4);
           mma16816(acc2, a0, a1, a2, a3, qb[s2][0], qb[s2][1]);
         }
       }
