@@ -251,6 +251,29 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
                          float scale, float* out, void* workspace, size_t ws_bytes,
                          tq_stream stream);
 
+/* Size of the fixed device scratch array behind tq_decode_attn_fixed_ws (8 MiB per device). */
+#define TQ_DECODE_FIXED_WS_BYTES (8u << 20)
+
+/*
+ * DEVICE.  The same step as tq_decode_attn, with the same arguments, results and errors,
+ * but it allocates nothing and takes no workspace: its scratch is one file-scope device
+ * array of TQ_DECODE_FIXED_WS_BYTES in this library (one per device).  The pages have no
+ * counterpart of this call; it serves callers that cannot hand over device scratch.
+ *   - A shape whose tq_decode_attn_workspace exceeds TQ_DECODE_FIXED_WS_BYTES returns
+ *     TQ_ERR_WORKSPACE before any launch (the 128k-token workload with B = 8, Hq = 32
+ *     needs about 4.9 MB).
+ *   - The first call on a device, with that device current, looks up the array address
+ *     (cudaGetSymbolAddress); make it before any latency-critical loop.  A failed lookup
+ *     returns TQ_ERR_CUDA.
+ *   - All calls on one device share the array: calls that can overlap in time (other
+ *     streams, unordered host threads) race on it; calls in order on one stream do not.
+ *     Nothing in it has to start at zero.
+ */
+tq_status tq_decode_attn_fixed_ws(const tq_quantizer* kq, const tq_quantizer* vq, const void* q,
+                                  int32_t dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,
+                                  const int32_t* seq_lens, tq_packed kcache, tq_packed vcache,
+                                  float scale, float* out, tq_stream stream);
+
 /*
  * Synchronizes `stream`, then returns and clears the device status word of the current
  * device: TQ_OK, or TQ_ERR_TIMEOUT if a bounded device wait ran out since the last call.

@@ -31,6 +31,7 @@ EXPORTS = [
     "tq_spectral_unit_codebooks", "tq_record_layout", "tq_quantize_mse", "tq_quantize_prod",
     "tq_quantize_spectral", "tq_dequantize", "tq_score_workspace", "tq_score",
     "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
+    "tq_decode_attn_fixed_ws",
 ]
 
 
@@ -90,6 +91,8 @@ def lib():
             "tq_decode_attn_workspace": ([qp, i32, i32, i32, i64, C.POINTER(C.c_size_t)], C.c_int),
             "tq_decode_attn": ([qp, qp, vp, i32, i32, i32, i32, i64, vp, Packed_t, Packed_t, C.c_float,
                                 vp, vp, C.c_size_t, vp], C.c_int),
+            "tq_decode_attn_fixed_ws": ([qp, qp, vp, i32, i32, i32, i32, i64, vp, Packed_t, Packed_t,
+                                         C.c_float, vp, vp], C.c_int),
             "tq_get_status": ([vp], C.c_int),
             "tq_set_wait_limit": ([i64], C.c_int),
             "tq_lut_scale": ([f64p, i32, C.POINTER(C.c_float)], C.c_int),
