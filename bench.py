@@ -60,57 +60,108 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """SM clock and clock-event reasons of one GPU, polled through NVML (read-only queries)
+    every few milliseconds while the timed region runs; falls back to nvidia-smi."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index: str):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, uuid: str, period_s: float = 0.002):
+        self.uuid = uuid
+        self.period = period_s
+        self.samples = []          # (sm_mhz, reason bits)
+        self.max_mhz = None
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            get_r = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                             int(get_r(h))))
+                    except Exception:
+                        pass
+                    self._stop.wait(self.period)
+            self.source = "nvml"
+        except Exception:
+            poll = self._poll_smi
+            self.source = "nvidia-smi"
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        bits = [0x8, 0x40, 0x20, 0x4]
+        while not self._stop.is_set():
+            try:
+                r = subprocess.run(["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={fields}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                f = [x.strip() for x in r.stdout.strip().split(",")]
+                m = sum(b for b, v in zip(bits, f[2:6]) if v.lower() == "active")
+                self.samples.append((float(f[0]), m))
+                self.max_mhz = float(f[1])
+            except Exception:
+                pass
+            self._stop.wait(0.05)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=10)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [c for c, _ in self.samples]
+        reasons = sorted(n for n, b in self.REASONS.items() if any(r & b for _, r in self.samples))
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": self.source}
+
+
+def profiled_traffic(summary_name: str, sources, scale: float):
+    """Per-launch DRAM bytes (read + write) recorded by an ncu capture in profiles/<summary_name>,
+    scaled by ``scale`` (units of the timed launch / units of the captured launch).  None when
+    the summary is missing or the kernel sources changed since the capture (the summary holds
+    the sha256 of the listed source files at capture time)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary_name)
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for rel in sources:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    fields = {}
+    with open(path) as f:
+        for ln in f:
+            if ln.startswith("- ") and ": " in ln:
+                k, v = ln[2:].split(": ", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel sources sha256") != h.hexdigest():
+        return None
+    try:
+        return float(fields["dram bytes per launch"]) * scale
+    except (KeyError, ValueError):
+        return None
+
+
+QUANT_SOURCES = ["kv_cache_compression_rotation_b200/csrc/quantize_umma.cuh",
+                 "kv_cache_compression_rotation_b200/csrc/quantize_umma.cu",
+                 "kv_cache_compression_rotation_b200/csrc/device_common.cuh"]
+DECODE_SOURCES = ["kv_cache_compression_rotation_b200/csrc/decode_tma.cuh",
+                  "kv_cache_compression_rotation_b200/csrc/decode.cuh",
+                  "kv_cache_compression_rotation_b200/csrc/decode_mse.cu",
+                  "kv_cache_compression_rotation_b200/csrc/device_common.cuh"]
 
 
 def run_tq(args, rank, world, local_rank):
@@ -257,10 +308,13 @@ def run_tq(args, rank, world, local_rank):
                             "note": "tq_decode_attn = query prep + decode + combine launches"},
         },
         "roofline": {"bound": "hbm", "kernel": "umma_quantize_kernel<4>", "achieved": q_gbs, "peak": peak,
-                     "peak_source": peak_kind, "unit": "GB/s", "frac": q_gbs / peak, "traffic": None},
-        "roofline_decode": {"bound": "hbm", "kernel": "decode_attn_kernel<128,mse4,mse4> (+qprep, combine)",
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": q_gbs / peak,
+                     "algorithmic_bytes": q_bytes,
+                     "traffic": profiled_traffic("umma_quantize_kernel_ctx32k.md", QUANT_SOURCES, N / 32768)},
+        "roofline_decode": {"bound": "hbm", "kernel": "decode_tma_kernel<mse4,mse4> (+qprep, combine)",
                             "achieved": d_gbs, "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                            "frac": d_gbs / peak, "traffic": None},
+                            "frac": d_gbs / peak, "algorithmic_bytes": dec_bytes,
+                            "traffic": profiled_traffic("decode_tma_kernel_ctx32k.md", DECODE_SOURCES, N / 32768)},
         "e2e": e2e,
         "gpu_launches": args.steps * 5,
         "clocks": clocks,
@@ -341,8 +395,11 @@ def main():
                     help="profiling aid: run one part of the step (the reported line is then partial)")
     ap.add_argument("--context", type=int, default=N,
                     help="profiling aid: context length (the headline workload uses 131072)")
+    ap.add_argument("--batch", type=int, default=B,
+                    help="profiling aid: batch size (the headline workload uses 8)")
     args = ap.parse_args()
     globals()["N"] = args.context
+    globals()["B"] = args.batch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

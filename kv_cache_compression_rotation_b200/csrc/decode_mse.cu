@@ -5,14 +5,21 @@
 namespace tq {
 namespace {
 
-template <int KB, int VB>
-cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, int* status, long long lim) {
-  auto k = decode_tma_kernel<KFMT_MSE, KB, VB>;
+template <int KB, int VB, bool PK>
+cudaError_t go_pk(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, int* status, long long lim) {
+  auto k = decode_tma_kernel<KFMT_MSE, KB, VB, PK>;
   smem = decode_tma_smem_bytes(KB, VB, KFMT_MSE, 4);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   k<<<grid, (tma_consumers(KFMT_MSE) + 1) * 32, smem, s>>>(p, status, lim);
   return cudaGetLastError();
+}
+
+// GQA groups of at most 4 heads take the packed-column variant
+template <int KB, int VB>
+cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, int* status, long long lim) {
+  return p.G <= 4 ? go_pk<KB, VB, true>(p, grid, smem, s, status, lim)
+                  : go_pk<KB, VB, false>(p, grid, smem, s, status, lim);
 }
 
 }  // namespace
