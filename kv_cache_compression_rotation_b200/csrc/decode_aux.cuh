@@ -94,4 +94,144 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
   }
 }
 
+// ---- d = 128 versions: 8 query rows per CTA of 256 threads ----
+
+// ys[r][j] = scale * sum_k M[j][k] xs[r][k] for 8 rows r and 128 outputs j (M row-major,
+// 128 x 128; xs, ys in shared memory).  Warp w produces j in [16 w, 16 w + 16); lane l
+// holds xs[r][4 l .. 4 l + 3].  Each group of 4 outputs x 8 rows is 32 partial dot products
+// per lane, summed across the warp by a halving exchange that leaves total l in lane l.
+__device__ __forceinline__ void matvec8x128(const float* __restrict__ M, const float* xs, float* ys, float scale,
+                                            int warp, int lane) {
+  float4 xv[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) xv[r] = *reinterpret_cast<const float4*>(xs + r * 128 + 4 * lane);
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    float v[32];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+      const float4 m = __ldg(reinterpret_cast<const float4*>(M + (16 * warp + 4 * pass + d) * 128 + 4 * lane));
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        v[d * 8 + r] = fmaf(m.w, xv[r].w, fmaf(m.z, xv[r].z, fmaf(m.y, xv[r].y, m.x * xv[r].x)));
+    }
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) {
+      const bool up = (lane & sh) != 0;
+#pragma unroll
+      for (int i = 0; i < sh; ++i) {
+        const float send = up ? v[i] : v[i + sh];
+        const float keep = up ? v[i + sh] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+      }
+    }
+    // lane l now holds the total of value l = 8 d + r
+    ys[(lane & 7) * 128 + 16 * warp + 4 * pass + (lane >> 3)] = v[0] * scale;
+  }
+}
+
+// qprep_kernel for MSE and PROD keys with d = 128 (same outputs).
+__global__ void __launch_bounds__(256) qprep128_kernel(QPrepParams p) {
+  __shared__ __align__(16) float xs[8 * 128], ys[8 * 128], us[8 * 128];
+  const int r0 = blockIdx.x * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 8 * 128; i += 256) {
+    const int r = i >> 7, j = i & 127;
+    xs[i] = (r0 + r < p.rows) ? load_elem(p.q, p.dtype, static_cast<int64_t>(r0 + r) * 128 + j) : 0.f;
+  }
+  __syncthreads();
+  matvec8x128(p.rot, xs, ys, p.scale, warp, lane);
+  __syncthreads();
+  const bool prod = p.kind == TQ_KIND_PROD;
+  if (prod) {
+    matvec8x128(p.S, ys, us, 1.f, warp, lane);
+    __syncthreads();
+  }
+  const int r = r0 + warp;                         // warp w normalizes row w
+  if (r >= p.rows) return;
+  const float4 a = *reinterpret_cast<const float4*>(ys + warp * 128 + 4 * lane);
+  float ma = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
+  ma = warp_max(ma);
+  const float sa = ma > 0.f ? ma : 1.f;
+  reinterpret_cast<float4*>(p.qa + static_cast<int64_t>(r) * 128)[lane] =
+      make_float4(a.x / sa, a.y / sa, a.z / sa, a.w / sa);
+  float sb = 1.f;
+  const int n2 = p.qb_stride;
+  if (prod) {                                       // n2 = m = 128
+    const float4 u = *reinterpret_cast<const float4*>(us + warp * 128 + 4 * lane);
+    float mb = fmaxf(fmaxf(fabsf(u.x), fabsf(u.y)), fmaxf(fabsf(u.z), fabsf(u.w)));
+    mb = warp_max(mb);
+    sb = mb > 0.f ? mb : 1.f;
+    reinterpret_cast<float4*>(p.qb + static_cast<int64_t>(r) * n2)[lane] =
+        make_float4(u.x / sb, u.y / sb, u.z / sb, u.w / sb);
+  } else {
+    for (int i = lane; i < n2; i += 32) p.qb[static_cast<int64_t>(r) * n2 + i] = 0.f;
+  }
+  if (lane == 0) { p.qs[r * 2] = sa; p.qs[r * 2 + 1] = sb; }
+}
+
+// combine_kernel with d = 128: 8 rows per CTA; dynamic shared memory holds the chunk
+// weights 2^(m_c - M) / L of the 8 rows ([8][n_chunks] floats).
+__global__ void __launch_bounds__(256) combine128_kernel(CombineParams p) {
+  extern __shared__ __align__(16) float cw[];
+  __shared__ __align__(16) float ov[128 * 8];     // o' transposed: [j][row]
+  const int r0 = blockIdx.x * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nch = p.n_chunks;
+  {
+    float* w = cw + warp * nch;
+    const int r = r0 + warp;
+    if (r < p.rows) {
+      const float* ml = p.part_ml + static_cast<int64_t>(r) * nch * 2;
+      float M = -INFINITY;
+      for (int c = lane; c < nch; c += 32) M = fmaxf(M, ml[c * 2]);
+      M = warp_max(M);
+      float L = 0.f;
+      for (int c = lane; c < nch; c += 32) {
+        const float mc = ml[c * 2];
+        const float e = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        w[c] = e;
+        L += e * ml[c * 2 + 1];
+      }
+      L = warp_sum(L);
+      const float invL = L > 0.f ? 1.f / L : 0.f;
+      for (int c = lane; c < nch; c += 32) w[c] *= invL;
+    } else {
+      for (int c = lane; c < nch; c += 32) w[c] = 0.f;
+    }
+  }
+  __syncthreads();
+  {
+    const int r = r0 + warp;                       // thread: row warp, dims 4 lane .. 4 lane + 3
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < p.rows) {
+      const float* w = cw + warp * nch;
+      const float4* po = reinterpret_cast<const float4*>(p.part_o + static_cast<int64_t>(r) * nch * 128) + lane;
+      for (int c = 0; c < nch; ++c) {
+        const float wc = w[c];
+        const float4 x = __ldg(po + c * 32);
+        a.x = fmaf(wc, x.x, a.x); a.y = fmaf(wc, x.y, a.y); a.z = fmaf(wc, x.z, a.z); a.w = fmaf(wc, x.w, a.w);
+      }
+      if (p.v_sigma) {
+        a.x *= p.v_sigma[4 * lane]; a.y *= p.v_sigma[4 * lane + 1];
+        a.z *= p.v_sigma[4 * lane + 2]; a.w *= p.v_sigma[4 * lane + 3];
+      }
+    }
+    ov[(4 * lane) * 8 + warp] = a.x;
+    ov[(4 * lane + 1) * 8 + warp] = a.y;
+    ov[(4 * lane + 2) * 8 + warp] = a.z;
+    ov[(4 * lane + 3) * 8 + warp] = a.w;
+  }
+  __syncthreads();
+  const int k = tid & 127, rb = (tid >> 7) * 4;    // thread: output dim k of rows rb .. rb + 3
+  float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+  for (int j = 0; j < 128; ++j) {
+    const float m = __ldg(p.rot_v + j * 128 + k);
+    const float4 o = *reinterpret_cast<const float4*>(ov + j * 8 + rb);
+    o0 = fmaf(o.x, m, o0); o1 = fmaf(o.y, m, o1); o2 = fmaf(o.z, m, o2); o3 = fmaf(o.w, m, o3);
+  }
+  const float res[4] = {o0, o1, o2, o3};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (r0 + rb + i < p.rows) p.out[static_cast<int64_t>(r0 + rb + i) * 128 + k] = res[i];
+}
+
 }  // namespace tq

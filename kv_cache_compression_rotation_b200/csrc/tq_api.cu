@@ -577,7 +577,10 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   qp.spec_coef = static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, kq->k_top));
   qp.qa = qa; qp.qb = qb; qp.qs = qs; qp.qb_stride = P.qb_stride;
   const size_t qsm = static_cast<size_t>(2 * D + std::max(D, P.qb_stride)) * 4;
-  qprep_kernel<<<rows, 128, qsm, stream>>>(qp);
+  if (kq->kind != TQ_KIND_SPECTRAL && D == 128)
+    qprep128_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(qp);
+  else
+    qprep_kernel<<<rows, 128, qsm, stream>>>(qp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "qprep launch");
 
@@ -631,7 +634,16 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   cp.part_ml = pml; cp.part_o = po; cp.rot_v = vq->rot;
   cp.v_sigma = vq->kind == TQ_KIND_SPECTRAL ? vq->dim_sigma : nullptr;
   cp.out = out;
-  combine_kernel<<<rows, 128, static_cast<size_t>(D) * 4, stream>>>(cp);
+  const size_t csm = static_cast<size_t>(8) * P.n_chunks * 4;
+  if (D == 128 && csm <= 160 * 1024) {
+    if (csm > 48 * 1024) {
+      e = cudaFuncSetAttribute(combine128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(csm));
+      if (e != cudaSuccess) return cuda_fail(e, "combine attribute");
+    }
+    combine128_kernel<<<(rows + 7) / 8, 256, csm, stream>>>(cp);
+  } else {
+    combine_kernel<<<rows, 128, static_cast<size_t>(D) * 4, stream>>>(cp);
+  }
   e = cudaGetLastError();
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "combine launch");
 }
