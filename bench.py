@@ -50,6 +50,27 @@ def algorithmic_bytes():
     return nvec, q_bytes, dec_bytes
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank time over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, bytes_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job algorithmic GB/s: every rank moves the same bytes per step."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch of the workload."""
+    return 17 * rank
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -172,7 +193,7 @@ def run_tq(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     torch.backends.cuda.matmul.allow_tf32 = False
-    seed_off = 17 * rank
+    seed_off = rank_seed_offset(rank)
     nvec, q_bytes, dec_bytes = algorithmic_bytes()
     rot = ti.haar_rotation(D, ti.SEEDS["rotation"] + 3)
     U = ti.haar_rotation(D, ti.SEEDS["basis"] + 3)
@@ -234,18 +255,13 @@ def run_tq(args, rank, world, local_rank):
         end.record(stream)
         torch.cuda.synchronize(dev)
     assert K.get_status() == 0
-    total_ms = start.elapsed_time(end)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), dev)
     ms_step = total_ms / args.steps
     t_qk = float(np.mean([a.elapsed_time(b) for a, b in qk_ms]))
     t_qv = float(np.mean([a.elapsed_time(b) for a, b in qv_ms]))
     t_dec = float(np.mean([a.elapsed_time(b) for a, b in dec_ms]))
     step_bytes = 2 * q_bytes + dec_bytes
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = weak_scaling_value(world, step_bytes, ms_step)
     peak, peak_kind = measured_peaks()
     q_gbs = q_bytes / (0.5 * (t_qk + t_qv) * 1e-3) / 1e9
     d_gbs = dec_bytes / (t_dec * 1e-3) / 1e9
@@ -279,13 +295,8 @@ def run_tq(args, rank, world, local_rank):
             e2e_step()
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = s0.elapsed_time(s1) / ne
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * step_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e_ms,
+        e_ms = max_over_ranks(s0.elapsed_time(s1) / ne, dev)
+        e2e = {"value": weak_scaling_value(world, step_bytes, e_ms), "unit": "GB/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2,
                "d2h_bytes_per_step": oh.numel() * 4}
         del kh, vh

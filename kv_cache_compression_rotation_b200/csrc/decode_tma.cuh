@@ -10,18 +10,23 @@
 // pull their record slices into registers, release the stage and compute.
 //
 // Math per 16-token unit, all on mma.sync m16n8k16 (fp16 in, fp32 accumulate):
-//   scores  S[16 tokens x 8 heads] = K_hat[16 x 128] . Q'^T     (A = table-decoded keys)
+//   scores  S[16 tokens x 8 columns] = K_hat[16 x 128] . Q'^T     (A = table-decoded keys)
 //   P       exp2(S - m) * ||v||, transposed in registers with movmatrix
-//   values  O'^T[128 dims x 8 heads] += V_hat^T[128 x 16] . P^T (A = table-decoded values)
-// Tokens and value dims sit on the MMA's M side (16 rows), the query heads of the GQA
-// group on N (8 columns), so a 4-head group fills half of each MMA instead of a quarter.
+//   values  O'^T[128 dims x 8 columns] += V_hat^T[128 x 16] . P^T (A = table-decoded values)
+// Tokens and value dims sit on the MMA's M side (16 rows), the query heads on N.  For GQA
+// groups of at most 4 heads the 8 columns are 4 heads x (hi, lo) parts of the split
+// operands (see PK below); larger groups take 8 heads per work item.
 // Table decoding: one 32-bit shared load turns a pair of codes into half2 codebook values
-// (table replicated per lane, so a warp's 32 loads hit 32 banks).
-// Precision: the query operand and P are split hi + lo (two MMAs into one accumulator),
-// table entries are c / s with a searched shared scale s (see tq_lut_scale).
+// (table replicated per lane, so a warp's 32 loads hit 32 banks; the table sits at a
+// 64 KB-aligned shared address, so one byte permute of the code word is the address).
+// Precision: the query operand and P are split hi + lo (one accumulator), table entries
+// are c / s with a searched shared scale s (see tq_lut_scale).
 // Token order inside a unit: score row r holds token r/2 + 4 (r mod 2) + 8 (r / 8)
 // (rows 0..7) which spreads a warp's value-slice loads over both halves of the banks;
 // the k-index of P^T follows the score rows through the transpose.
+// Scheduling: the cross-row max runs only when a score of the warp exceeds its running
+// max (warp vote), and the value half of unit i - 1 is issued next to the key half of
+// unit i, so table loads, MMAs and softmax arithmetic of two units interleave.
 // All waits are bounded (TQ_ERR_TIMEOUT on expiry); a CTA that times out drains the
 // copies it issued before it exits.
 #pragma once
