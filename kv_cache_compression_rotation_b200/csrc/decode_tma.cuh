@@ -76,7 +76,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // Transpose of an 8x8 matrix of halves held one row-pair per thread (mma fragment layout).
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 
@@ -463,28 +463,49 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       const int u0 = warp * 16;                      // first token of this warp's unit (stage-local)
       // ---- pull this warp's slices out of the stage ----
       const int ka = u0 + pg, kb2 = u0 + 8 + pg;     // tokens of score rows g, g + 8
-      const bool oka = ka < cnt, okb = kb2 < cnt;
+      bool oka = true, okb = true;
       uint32_t ks0[NWK], ks1[NWK];
-      sld_slice<NWK>(sb + SL.kcodes + ka * KW * 4, KW, t * TDK * KB, oka, ks0);
-      sld_slice<NWK>(sb + SL.kcodes + kb2 * KW * 4, KW, t * TDK * KB, okb, ks1);
-      auto norm_of = [&](uint32_t staged, const float* global, int lk, bool ok) {
-        return ok ? (lk < nn ? sldf(staged + 4 * (noff + lk)) : __ldg(global + rec0 + t0 + lk)) : 0.f;
-      };
-      const float kn0 = norm_of(sb + SL.knorm, p.knorms, ka, oka), kn1 = norm_of(sb + SL.knorm, p.knorms, kb2, okb);
-      const float vn0 = norm_of(sb + SL.vnorm, p.vnorms, ka, oka), vn1 = norm_of(sb + SL.vnorm, p.vnorms, kb2, okb);
+      float kn0, kn1, vn0, vn1;
       float gm0 = 0.f, gm1 = 0.f;
       uint32_t sw0 = 0u, sw1 = 0u;
-      if constexpr (KF == KFMT_PROD) {
-        gm0 = norm_of(sb + SL.krn, p.krnorms, ka, oka);
-        gm1 = norm_of(sb + SL.krn, p.krnorms, kb2, okb);
-        sw0 = oka ? sld32(sb + SL.ksign + (ka * KSW + t) * 4) : 0u;
-        sw1 = okb ? sld32(sb + SL.ksign + (kb2 * KSW + t) * 4) : 0u;
-      }
       uint32_t vs[4][NWV];
+      if (cnt == kTmaStageTokens && nn >= cnt) {
+        // a whole stage with every norm staged (all but the last stage of a chunk): no
+        // per-token checks
+        sld_slice<NWK>(sb + SL.kcodes + ka * KW * 4, KW, t * TDK * KB, true, ks0);
+        sld_slice<NWK>(sb + SL.kcodes + kb2 * KW * 4, KW, t * TDK * KB, true, ks1);
+        kn0 = sldf(sb + SL.knorm + 4 * (noff + ka)); kn1 = sldf(sb + SL.knorm + 4 * (noff + kb2));
+        vn0 = sldf(sb + SL.vnorm + 4 * (noff + ka)); vn1 = sldf(sb + SL.vnorm + 4 * (noff + kb2));
+        if constexpr (KF == KFMT_PROD) {
+          gm0 = sldf(sb + SL.krn + 4 * (noff + ka));
+          gm1 = sldf(sb + SL.krn + 4 * (noff + kb2));
+          sw0 = sld32(sb + SL.ksign + (ka * KSW + t) * 4);
+          sw1 = sld32(sb + SL.ksign + (kb2 * KSW + t) * 4);
+        }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int lk = u0 + kv[i];
-        sld_slice<NWV>(sb + SL.vcodes + lk * VW * 4, VW, g * TDV * VB, lk < cnt, vs[i]);
+        for (int i = 0; i < 4; ++i)
+          sld_slice<NWV>(sb + SL.vcodes + (u0 + kv[i]) * VW * 4, VW, g * TDV * VB, true, vs[i]);
+      } else {
+        oka = ka < cnt;
+        okb = kb2 < cnt;
+        sld_slice<NWK>(sb + SL.kcodes + ka * KW * 4, KW, t * TDK * KB, oka, ks0);
+        sld_slice<NWK>(sb + SL.kcodes + kb2 * KW * 4, KW, t * TDK * KB, okb, ks1);
+        auto norm_of = [&](uint32_t staged, const float* global, int lk, bool ok) {
+          return ok ? (lk < nn ? sldf(staged + 4 * (noff + lk)) : __ldg(global + rec0 + t0 + lk)) : 0.f;
+        };
+        kn0 = norm_of(sb + SL.knorm, p.knorms, ka, oka); kn1 = norm_of(sb + SL.knorm, p.knorms, kb2, okb);
+        vn0 = norm_of(sb + SL.vnorm, p.vnorms, ka, oka); vn1 = norm_of(sb + SL.vnorm, p.vnorms, kb2, okb);
+        if constexpr (KF == KFMT_PROD) {
+          gm0 = norm_of(sb + SL.krn, p.krnorms, ka, oka);
+          gm1 = norm_of(sb + SL.krn, p.krnorms, kb2, okb);
+          sw0 = oka ? sld32(sb + SL.ksign + (ka * KSW + t) * 4) : 0u;
+          sw1 = okb ? sld32(sb + SL.ksign + (kb2 * KSW + t) * 4) : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int lk = u0 + kv[i];
+          sld_slice<NWV>(sb + SL.vcodes + lk * VW * 4, VW, g * TDV * VB, lk < cnt, vs[i]);
+        }
       }
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(s)) : "memory");

@@ -299,7 +299,10 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         if (tsm[k] < a) ++base_code;
         else if (tsm[k] < b || lane == 31) inside = fminf(inside, tsm[k]);
       }
-      cell_entry = (__float_as_uint(inside) & ~15u) | base_code;
+      // the boundary is kept in the cell coordinate f = u / (2R) + 1/2 (in [0, 1]), where
+      // the code assignment compares it with f directly
+      const float inside_f = inside < 1.0e38f ? fmaf(inside, 0.5f / R, 0.5f) : 3.0e38f;
+      cell_entry = (__float_as_uint(inside_f) & ~15u) | base_code;
     }
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
@@ -343,7 +346,8 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
             const float f = __saturatef(fmaf(y[i], fs, 0.5f));
             const float gcell = __fmaf_rz(f, kCellSpan, 8388608.0f);
             const uint32_t e = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gcell));
-            const uint32_t code = (e & 15u) + ((y[i] * inv > __uint_as_float(e)) ? 1u : 0u);
+            // + 1 when f lies above the cell's boundary: the sign bit of (boundary - f)
+            const uint32_t code = (e & 15u) + (__float_as_uint(__uint_as_float(e) - f) >> 31);
             const int pos = i * B;
             wc[pos >> 5] |= code << (pos & 31);
             if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
