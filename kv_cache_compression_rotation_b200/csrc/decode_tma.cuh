@@ -21,8 +21,10 @@
 // 64 KB-aligned shared address, so one byte permute of the code word is the address).
 // Precision: the query operand and P are split hi + lo (one accumulator), table entries
 // are c / s with a searched shared scale s (see tq_lut_scale).
-// Token order inside a unit: score row r holds token r/2 + 4 (r mod 2) + 8 (r / 8)
-// (rows 0..7) which spreads a warp's value-slice loads over both halves of the banks;
+// Token order inside a unit: score rows r and r + 8 hold tokens tau(r) and 8 + tau(r), with
+// tau = [0, 5, 1, 4, 2, 7, 3, 6]: the two rows a quarter-warp reads in one 16-byte key
+// slice load are tokens of opposite parity (64-byte records: opposite bank halves), and
+// the four tokens a half-warp reads in one value slice load cover both halves twice;
 // the k-index of P^T follows the score rows through the transpose.
 // Scheduling: the cross-row max runs only when a score of the warp exceeds its running
 // max (warp vote), and the value half of unit i - 1 is issued next to the key half of
@@ -332,9 +334,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
 
   // ---------------- consumers ----------------
   // score-tile row g holds token pg of the unit, row g + 8 token 8 + pg
-  const int pg = (g >> 1) + 4 * (g & 1);
+  const int pg = (g & 1) ? ((g >> 1) ^ 5) : (g >> 1);
   // value-operand k-indices 2t, 2t+1, 2t+8, 2t+9 are the tokens of score rows 2t, 2t+1, ...
-  const int kv[4] = {t, t + 4, 8 + t, 12 + t};
+  const int kv[4] = {t, t ^ 5, 8 + t, 8 + (t ^ 5)};
   const uint32_t klo = tabA | static_cast<uint32_t>(lane) * 4u, vlo = klo + 128u;
   // MMA column of this lane's B operand (g) and of its accumulators (2t, 2t + 1)
   const int qcol = PK ? (g & 3) : g;               // head (in the block) of B column g
