@@ -8,10 +8,10 @@ namespace {
 template <int KB, int VB, bool PK>
 cudaError_t go_pk(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s, int* status, long long lim) {
   auto k = decode_tma_kernel<KFMT_MSE, KB, VB, PK>;
-  smem = decode_tma_smem_bytes(KB, VB, KFMT_MSE, 4);
+  smem = decode_tma_smem_bytes(KB, VB, KFMT_MSE, PK);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k<<<grid, (tma_consumers(KFMT_MSE) + 1) * 32, smem, s>>>(p, status, lim);
+  k<<<grid, (tma_consumers(KFMT_MSE, PK) + 1) * 32, smem, s>>>(p, status, lim);
   return cudaGetLastError();
 }
 

@@ -37,11 +37,14 @@
 
 namespace tq {
 
-// Consumer warps per CTA: MSE keys fit 11 (plus the producer: 12 warps of <= 168
-// registers fill the register file); PROD keys need more registers and run 7.
-__host__ __device__ constexpr int tma_consumers(int kf) { return kf == KFMT_PROD ? 7 : 11; }
-__host__ __device__ constexpr int tma_stage_tokens(int kf) { return tma_consumers(kf) * 16; }
-constexpr int kTmaStages = 4;
+// Work split.  With packed columns (GQA groups of at most 4 heads) every consumer warp takes
+// two 16-token units of a stage (8 consumer warps, 3 stages of 256 tokens); otherwise one
+// unit (11 consumer warps for MSE keys, 4 stages).  PROD keys need more registers and run
+// 7 consumer warps.  Plus one producer warp.
+__host__ __device__ constexpr int tma_units(bool pk) { return pk ? 2 : 1; }
+__host__ __device__ constexpr int tma_consumers(int kf, bool pk) { return kf == KFMT_PROD ? 7 : (pk ? 8 : 11); }
+__host__ __device__ constexpr int tma_stage_tokens(int kf, bool pk) { return tma_consumers(kf, pk) * 16 * tma_units(pk); }
+__host__ __device__ constexpr int tma_stages(bool pk) { return pk ? 3 : 4; }
 constexpr int kTmaHeadBlock = 8;     // query heads per work item (MMA N)
 
 __device__ __forceinline__ uint32_t tma_smem_u32(const void* p) {
@@ -87,8 +90,8 @@ struct TmaStageLayout {
 };
 
 // Byte offsets of the arrays of one stage (all 16-byte aligned).
-__host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int kf, int ksw) {
-  const int st = tma_stage_tokens(kf);
+__host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int kf, int ksw, bool pk) {
+  const int st = tma_stage_tokens(kf, pk);
   TmaStageLayout L{};
   uint32_t o = 0;
   L.kcodes = o; o += st * kw * 4;
@@ -102,19 +105,23 @@ __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int k
 }
 
 // Shared memory of one CTA.  The lookup table must start at a 64 KB-aligned shared
-// address (a byte permute then forms the complete lookup address); the small arrays
-// (merge buffer, sign table, barriers) sit in the gap below it when they fit, so the
-// request covers a gap of up to 64 KB plus the table and the stage ring.
+// address (a byte permute then forms the complete lookup address).  The small arrays
+// (merge buffer, sign table, barriers) and as many stages as fit go into the gap below
+// the table, the rest after it; the kernel checks the layout against the allocation.
 __host__ __device__ inline uint32_t tma_table_bytes(int kb, int vb) {
   return (1u << (2 * (kb > vb ? kb : vb))) * 256u;
 }
-__host__ __device__ inline uint32_t tma_misc_bytes(int kf) {
-  const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf)) * 8u * (128u + 2u) * 4u;
-  return merge + 4u * 32u * 4u + 2u * 4u * 8u + 64u;
+__host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u : 8u; }
+__host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk) {
+  const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf, pk)) * tma_merge_rows(pk) * (128u + 2u) * 4u;
+  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u;
+  return (v + 127u) & ~127u;
 }
-inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, int ksw) {
-  const TmaStageLayout L = tma_stage_layout(128 * kb / 32, 128 * vb / 32, kf, ksw);
-  return 65536 + tma_table_bytes(kb, vb) + 4 * static_cast<size_t>(L.bytes);
+inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, bool pk) {
+  const TmaStageLayout L = tma_stage_layout(128 * kb / 32, 128 * vb / 32, kf, 4, pk);
+  const size_t want = 65536 + tma_table_bytes(kb, vb) + static_cast<size_t>(tma_stages(pk)) * L.bytes +
+                      tma_misc_bytes(kf, pk);
+  return want < 232448 ? want : 232448;
 }
 
 // Head blocks per GQA group (work items split groups larger than 8 heads).
@@ -186,11 +193,13 @@ __device__ __forceinline__ float ex2(float x) {
 // columns of the value MMA (summed in the merge).  Without PK the 8 columns are 8 heads and
 // the hi / lo parts take separate MMAs.
 template <int KF, int KB, int VB, bool PK>
-__global__ void __launch_bounds__((tma_consumers(KF) + 1) * 32, 1)
+__global__ void __launch_bounds__((tma_consumers(KF, PK) + 1) * 32, 1)
 decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
-  constexpr int kTmaConsumerWarps = tma_consumers(KF);
-  constexpr int kTmaThreads = (kTmaConsumerWarps + 1) * 32;
-  constexpr int kTmaStageTokens = tma_stage_tokens(KF);
+  constexpr int NC = tma_consumers(KF, PK);   // consumer warps
+  constexpr int U = tma_units(PK);            // 16-token units per consumer warp per stage
+  constexpr int NS = tma_stages(PK);          // ring stages
+  constexpr int kTmaThreads = (NC + 1) * 32;
+  constexpr int kTmaStageTokens = tma_stage_tokens(KF, PK);
   constexpr int D = 128;
   constexpr int KST = D / 16;                 // mma k-steps over the key dims
   constexpr int TDK = D / 4;                  // key dims per thread
@@ -202,7 +211,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int KW = D * KB / 32, VW = D * VB / 32;     // record words
   constexpr int KSW = 4;                                // prod sign words (m = 128)
   constexpr int HB = PK ? 4 : kTmaHeadBlock;            // query heads per work item
-  constexpr int CONSUMERS = kTmaConsumerWarps * 32;
+  constexpr int RW = static_cast<int>(tma_merge_rows(PK));   // merge rows per warp
+  constexpr int CONSUMERS = NC * 32;
   constexpr int NE = KLUT > VLUT ? KLUT : VLUT;        // table entries
   constexpr uint32_t TAB = static_cast<uint32_t>(NE) * 256u;
   extern __shared__ __align__(128) unsigned char tsm_[];
@@ -211,34 +221,47 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   // Table entry e is 256 B: the key value pair for lanes 0..31, then the value pair.  With the
   // table base B (a multiple of 64 KB), the lookup address of a code pair byte x for this lane
   // is B | x << 8 | lane * 4 [+ 128]: one byte permute, no add.
-  const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW);
+  const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW, PK);
   const uint32_t base = tma_smem_u32(tsm_);
   uint32_t dyn;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
   const uint32_t gap = (0u - base) & 0xFFFFu;
   const uint32_t tabA = base + gap;
-  const uint32_t stageA = tabA + TAB;
-  const uint32_t miscA = gap >= tma_misc_bytes(KF) ? base : stageA + kTmaStages * SL.bytes;
-  const uint32_t endA = max(stageA + kTmaStages * SL.bytes, miscA + tma_misc_bytes(KF));
-  if (endA > base + dyn) {                        // the request did not cover this layout
+  // first fit: misc block, then each stage, into the gap; the rest after the table
+  uint32_t gap_used = 0u, after = tabA + TAB;
+  auto place = [&](uint32_t bytes) {
+    if (gap_used + bytes <= gap) { const uint32_t a0 = base + gap_used; gap_used += bytes; return a0; }
+    const uint32_t a0 = after;
+    after += bytes;
+    return a0;
+  };
+  const uint32_t miscA = place(tma_misc_bytes(KF, PK));
+  uint32_t stA[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < NS; ++i) stA[i] = place(SL.bytes);
+  if (after > base + dyn) {                       // the request did not cover this layout
     if (threadIdx.x == 0) report_status(status, TQ_ERR_UNSUPPORTED);
     return;
   }
+  auto stage_addr = [&](int st) {
+    return NS == 3 ? (st == 0 ? stA[0] : (st == 1 ? stA[1] : stA[2]))
+                   : (st < 2 ? (st == 0 ? stA[0] : stA[1]) : (st == 2 ? stA[2] : stA[3]));
+  };
   auto gen = [&](uint32_t a) { return tsm_ + (a - base); };   // generic pointer of a shared address
   uint32_t* tab_g = reinterpret_cast<uint32_t*>(gen(tabA));
-  float* mrg = reinterpret_cast<float*>(gen(miscA));             // [warp][8 columns][m, l, o'[D]]
-  const uint32_t mrg_bytes = kTmaConsumerWarps * 8 * (D + 2) * 4;
+  float* mrg = reinterpret_cast<float*>(gen(miscA));             // [warp][RW rows][m, l, o'[D]]
+  const uint32_t mrg_bytes = NC * RW * (D + 2) * 4;
   uint32_t* luts = reinterpret_cast<uint32_t*>(gen(miscA + mrg_bytes));
   const uint32_t luts_a = miscA + mrg_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gen(miscA + mrg_bytes + 512));
-  int* nb_count = reinterpret_cast<int*>(bars + 2 * kTmaStages);   // [kTmaStages] tokens with staged norms
-  int* nb_off = nb_count + kTmaStages;                                 // [kTmaStages] their offset in the stage
-  volatile int* abort_flag = nb_off + kTmaStages;
+  int* nb_count = reinterpret_cast<int*>(bars + 2 * NS);   // [NS] tokens with staged norms
+  int* nb_off = nb_count + NS;                              // [NS] their offset in the stage
+  volatile int* abort_flag = nb_off + NS;
   volatile int* consumers_stop = abort_flag + 1;   // uniform exit decision of the consumer warps
   const uint32_t bar0 = tma_smem_u32(bars);
   const uint32_t nb_a = tma_smem_u32(nb_count);
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kTmaStages + s); };
+  auto full_bar = [&](int st) { return bar0 + 8u * st; };
+  auto empty_bar = [&](int st) { return bar0 + 8u * (NS + st); };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -259,9 +282,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   };
 
   if (tid == 0) {
-    for (int s = 0; s < kTmaStages; ++s) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(full_bar(s)), "r"(1));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty_bar(s)), "r"(kTmaConsumerWarps));
+    for (int st = 0; st < NS; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(full_bar(st)), "r"(1));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty_bar(st)), "r"(NC));
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -283,7 +306,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   }
   __syncthreads();
 
-  if (warp == kTmaConsumerWarps) {
+  if (warp == NC) {
     // ---------------- producer ----------------
     if (lane == 0) {
       int gs = 0;                                   // global stage counter of this CTA
@@ -293,8 +316,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         item_range(item, bh, hblk, chunk, k0, k1);
         const int64_t rec0 = static_cast<int64_t>(bh) * p.Nmax;
         for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
-          const int s = gs % kTmaStages, use = gs / kTmaStages;
-          if (use > 0 && !tma_mbar_wait(empty_bar(s), (use - 1) & 1, wait_lim, status, abort_flag)) {
+          const int st = gs % NS, use = gs / NS;
+          if (use > 0 && !tma_mbar_wait(empty_bar(st), (use - 1) & 1, wait_lim, status, abort_flag)) {
             stop = true;
             break;
           }
@@ -306,13 +329,13 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           const int off = static_cast<int>(r & 3);
           int nn = (off + cnt + 3) & ~3;
           if (r - off + nn > total_recs) nn = (off + cnt) & ~3;
-          nb_count[s] = max(0, nn - off);
-          nb_off[s] = off;
+          nb_count[st] = max(0, nn - off);
+          nb_off[st] = off;
           uint32_t bytes = cnt * (KW + VW) * 4 + 2 * nn * 4;
           if (KF == KFMT_PROD) bytes += cnt * KSW * 4 + nn * 4;
-          const uint32_t fb = full_bar(s);
+          const uint32_t fb = full_bar(st);
           asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
-          const uint32_t sb = stageA + static_cast<uint32_t>(s) * SL.bytes;
+          const uint32_t sb = stage_addr(st);
           bulk_g2s(sb + SL.kcodes, p.kcodes + r * KW, cnt * KW * 4, fb);
           bulk_g2s(sb + SL.vcodes, p.vcodes + r * VW, cnt * VW * 4, fb);
           if (nn > 0) {
@@ -326,8 +349,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         }
       }
       // drain: the copies this CTA issued land before it may exit
-      for (int j = max(0, gs - kTmaStages); j < gs; ++j)
-        for (long long i = 0; !tma_mbar_try(full_bar(j % kTmaStages), (j / kTmaStages) & 1) && i < (1ll << 28); ++i) {}
+      for (int j = max(0, gs - NS); j < gs; ++j)
+        for (long long i = 0; !tma_mbar_try(full_bar(j % NS), (j / NS) & 1) && i < (1ll << 28); ++i) {}
     }
     return;
   }
@@ -356,8 +379,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     const bool hok = qcol < nh;
     uint32_t qh[KST][2], ql[PK ? 1 : KST][2];
 #pragma unroll
-    for (int s = 0; s < KST; ++s) {
-      const int dm = t * TDK + 4 * s;
+    for (int k = 0; k < KST; ++k) {
+      const int dm = t * TDK + 4 * k;
       float a[4] = {0.f, 0.f, 0.f, 0.f};
       if (hok) {
         const float4 v = __ldg(reinterpret_cast<const float4*>(p.qa + (qbase + qcol) * D + dm));
@@ -367,18 +390,18 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       split_pair(a[0], a[1], h01, l01);
       split_pair(a[2], a[3], h23, l23);
       if constexpr (PK) {
-        qh[s][0] = qlo ? l01 : h01;
-        qh[s][1] = qlo ? l23 : h23;
+        qh[k][0] = qlo ? l01 : h01;
+        qh[k][1] = qlo ? l23 : h23;
       } else {
-        qh[s][0] = h01; qh[s][1] = h23;
-        ql[s][0] = l01; ql[s][1] = l23;
+        qh[k][0] = h01; qh[k][1] = h23;
+        ql[k][0] = l01; ql[k][1] = l23;
       }
     }
     uint32_t qb[KST][2];
     if constexpr (KF == KFMT_PROD) {
 #pragma unroll
-      for (int s = 0; s < KST; ++s) {
-        const int dm = t * TDK + 4 * s;
+      for (int k = 0; k < KST; ++k) {
+        const int dm = t * TDK + 4 * k;
         float a[4] = {0.f, 0.f, 0.f, 0.f};
         if (hok) {
           const float4 v = __ldg(reinterpret_cast<const float4*>(p.qb + (qbase + qcol) * p.qb_stride + dm));
@@ -388,11 +411,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           uint32_t h01, l01, h23, l23;
           split_pair(a[0], a[1], h01, l01);
           split_pair(a[2], a[3], h23, l23);
-          qb[s][0] = qlo ? l01 : h01;
-          qb[s][1] = qlo ? l23 : h23;
+          qb[k][0] = qlo ? l01 : h01;
+          qb[k][1] = qlo ? l23 : h23;
         } else {
-          qb[s][0] = pack_half2(a[0], a[1]);
-          qb[s][1] = pack_half2(a[2], a[3]);
+          qb[k][0] = pack_half2(a[0], a[1]);
+          qb[k][1] = pack_half2(a[2], a[3]);
         }
       }
     }
@@ -407,180 +430,148 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
 #pragma unroll
     for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads h0, h0 + 1
-    // Software pipeline: the value half of unit i - 1 (its value slices and P operand,
-    // kept here) is issued next to the key half of unit i.  A zero P makes the first
-    // pass a no-op, so the loop body has no branch around it.
-    uint32_t pvs[4][NWV];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int w = 0; w < NWV; ++w) pvs[i][w] = 0u;
-    uint32_t pb0h = 0u, pb1h = 0u, pb0l = 0u, pb1l = 0u;
-    // O'^T[128 dims x 8 columns] += V_hat^T . P^T for the pending unit
-    // M-tile i: row g = dim TDV g + i (first word of the slice), row g + 8 = dim TDV g + 8 + i
-    auto value_half = [&]() {
-      if constexpr (VB == 4) {
-        // byte j of lo (hi) holds the codes of one token pair for dim 2j (2j + 1) of a word
-        uint32_t lo[2][2], hi[2][2];   // [token pair][word]
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-#pragma unroll
-          for (int kp = 0; kp < 2; ++kp) {
-            const uint32_t x = pvs[2 * kp][w], y = pvs[2 * kp + 1][w];
-            lo[kp][w] = (x & 0x0F0F0F0Fu) | ((y << 4) & 0xF0F0F0F0u);
-            hi[kp][w] = ((x >> 4) & 0x0F0F0F0Fu) | (y & 0xF0F0F0F0u);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          const int k = i >> 1;
-          const uint32_t a0 = tab_ld(tab_off((i & 1) ? hi[0][0] : lo[0][0], vlo, k));
-          const uint32_t a1 = tab_ld(tab_off((i & 1) ? hi[0][1] : lo[0][1], vlo, k));
-          const uint32_t a2 = tab_ld(tab_off((i & 1) ? hi[1][0] : lo[1][0], vlo, k));
-          const uint32_t a3 = tab_ld(tab_off((i & 1) ? hi[1][1] : lo[1][1], vlo, k));
-          mma16816(o[i], a0, a1, a2, a3, pb0h, pb1h);
-          if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, pb0l, pb1l);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          const uint32_t e00 = field_at<VB, NWV>(pvs[0], i * VB) | (field_at<VB, NWV>(pvs[1], i * VB) << VB);
-          const uint32_t e01 = field_at<VB, NWV>(pvs[0], (8 + i) * VB) | (field_at<VB, NWV>(pvs[1], (8 + i) * VB) << VB);
-          const uint32_t e10 = field_at<VB, NWV>(pvs[2], i * VB) | (field_at<VB, NWV>(pvs[3], i * VB) << VB);
-          const uint32_t e11 = field_at<VB, NWV>(pvs[2], (8 + i) * VB) | (field_at<VB, NWV>(pvs[3], (8 + i) * VB) << VB);
-          const uint32_t a0 = tab_ld((e00 << 8) | vlo), a1 = tab_ld((e01 << 8) | vlo);
-          const uint32_t a2 = tab_ld((e10 << 8) | vlo), a3 = tab_ld((e11 << 8) | vlo);
-          mma16816(o[i], a0, a1, a2, a3, pb0h, pb1h);
-          if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, pb0l, pb1l);
-        }
-      }
-    };
 
     for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
-      const int s = gs % kTmaStages;
-      if (!tma_mbar_wait(full_bar(s), (gs / kTmaStages) & 1, wait_lim, status, abort_flag)) break;
-      const uint32_t sb = stageA + static_cast<uint32_t>(s) * SL.bytes;
+      const int st = gs % NS;
+      if (!tma_mbar_wait(full_bar(st), (gs / NS) & 1, wait_lim, status, abort_flag)) break;
+      const uint32_t sb = stage_addr(st);
       const int cnt = min(kTmaStageTokens, k1 - t0);
-      const int nn = static_cast<int>(sld32(nb_a + 4u * s)), noff = static_cast<int>(sld32(nb_a + 4u * (kTmaStages + s)));
-      const int u0 = warp * 16;                      // first token of this warp's unit (stage-local)
+      const int nn = static_cast<int>(sld32(nb_a + 4u * st)), noff = static_cast<int>(sld32(nb_a + 4u * (NS + st)));
+      const int w0 = warp * 16 * U;                  // first token of this warp (stage-local)
       // ---- pull this warp's slices out of the stage ----
-      const int ka = u0 + pg, kb2 = u0 + 8 + pg;     // tokens of score rows g, g + 8
-      bool oka = true, okb = true;
-      uint32_t ks0[NWK], ks1[NWK];
-      float kn0, kn1, vn0, vn1;
-      float gm0 = 0.f, gm1 = 0.f;
-      uint32_t sw0 = 0u, sw1 = 0u;
-      uint32_t vs[4][NWV];
+      bool ok[U][2];
+      uint32_t ks[U][2][NWK];
+      float kn[U][2], vn[U][2], gm[U][2];
+      uint32_t sw[U][2];
+      uint32_t vs[U][4][NWV];
       if (cnt == kTmaStageTokens && nn >= cnt) {
         // a whole stage with every norm staged (all but the last stage of a chunk): no
         // per-token checks
-        sld_slice<NWK>(sb + SL.kcodes + ka * KW * 4, KW, t * TDK * KB, true, ks0);
-        sld_slice<NWK>(sb + SL.kcodes + kb2 * KW * 4, KW, t * TDK * KB, true, ks1);
-        kn0 = sldf(sb + SL.knorm + 4 * (noff + ka)); kn1 = sldf(sb + SL.knorm + 4 * (noff + kb2));
-        vn0 = sldf(sb + SL.vnorm + 4 * (noff + ka)); vn1 = sldf(sb + SL.vnorm + 4 * (noff + kb2));
-        if constexpr (KF == KFMT_PROD) {
-          gm0 = sldf(sb + SL.krn + 4 * (noff + ka));
-          gm1 = sldf(sb + SL.krn + 4 * (noff + kb2));
-          sw0 = sld32(sb + SL.ksign + (ka * KSW + t) * 4);
-          sw1 = sld32(sb + SL.ksign + (kb2 * KSW + t) * 4);
-        }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          sld_slice<NWV>(sb + SL.vcodes + (u0 + kv[i]) * VW * 4, VW, g * TDV * VB, true, vs[i]);
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int tk = w0 + 16 * u + 8 * h + pg;     // token of score row g + 8 h
+            ok[u][h] = true;
+            sld_slice<NWK>(sb + SL.kcodes + tk * KW * 4, KW, t * TDK * KB, true, ks[u][h]);
+            kn[u][h] = sldf(sb + SL.knorm + 4 * (noff + tk));
+            vn[u][h] = sldf(sb + SL.vnorm + 4 * (noff + tk));
+            gm[u][h] = 0.f;
+            sw[u][h] = 0u;
+            if constexpr (KF == KFMT_PROD) {
+              gm[u][h] = sldf(sb + SL.krn + 4 * (noff + tk));
+              sw[u][h] = sld32(sb + SL.ksign + (tk * KSW + t) * 4);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            sld_slice<NWV>(sb + SL.vcodes + (w0 + 16 * u + kv[i]) * VW * 4, VW, g * TDV * VB, true, vs[u][i]);
+        }
       } else {
-        oka = ka < cnt;
-        okb = kb2 < cnt;
-        sld_slice<NWK>(sb + SL.kcodes + ka * KW * 4, KW, t * TDK * KB, oka, ks0);
-        sld_slice<NWK>(sb + SL.kcodes + kb2 * KW * 4, KW, t * TDK * KB, okb, ks1);
-        auto norm_of = [&](uint32_t staged, const float* global, int lk, bool ok) {
-          return ok ? (lk < nn ? sldf(staged + 4 * (noff + lk)) : __ldg(global + rec0 + t0 + lk)) : 0.f;
+        auto norm_of = [&](uint32_t staged, const float* global, int lk, bool okk) {
+          return okk ? (lk < nn ? sldf(staged + 4 * (noff + lk)) : __ldg(global + rec0 + t0 + lk)) : 0.f;
         };
-        kn0 = norm_of(sb + SL.knorm, p.knorms, ka, oka); kn1 = norm_of(sb + SL.knorm, p.knorms, kb2, okb);
-        vn0 = norm_of(sb + SL.vnorm, p.vnorms, ka, oka); vn1 = norm_of(sb + SL.vnorm, p.vnorms, kb2, okb);
-        if constexpr (KF == KFMT_PROD) {
-          gm0 = norm_of(sb + SL.krn, p.krnorms, ka, oka);
-          gm1 = norm_of(sb + SL.krn, p.krnorms, kb2, okb);
-          sw0 = oka ? sld32(sb + SL.ksign + (ka * KSW + t) * 4) : 0u;
-          sw1 = okb ? sld32(sb + SL.ksign + (kb2 * KSW + t) * 4) : 0u;
-        }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int lk = u0 + kv[i];
-          sld_slice<NWV>(sb + SL.vcodes + lk * VW * 4, VW, g * TDV * VB, lk < cnt, vs[i]);
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int tk = w0 + 16 * u + 8 * h + pg;
+            const bool okk = tk < cnt;
+            ok[u][h] = okk;
+            sld_slice<NWK>(sb + SL.kcodes + tk * KW * 4, KW, t * TDK * KB, okk, ks[u][h]);
+            kn[u][h] = norm_of(sb + SL.knorm, p.knorms, tk, okk);
+            vn[u][h] = norm_of(sb + SL.vnorm, p.vnorms, tk, okk);
+            gm[u][h] = 0.f;
+            sw[u][h] = 0u;
+            if constexpr (KF == KFMT_PROD) {
+              gm[u][h] = norm_of(sb + SL.krn, p.krnorms, tk, okk);
+              sw[u][h] = okk ? sld32(sb + SL.ksign + (tk * KSW + t) * 4) : 0u;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int lk = w0 + 16 * u + kv[i];
+            sld_slice<NWV>(sb + SL.vcodes + lk * VW * 4, VW, g * TDV * VB, lk < cnt, vs[u][i]);
+          }
         }
       }
       __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(s)) : "memory");
-      if (u0 >= cnt) continue;
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
+      if (w0 >= cnt) continue;
 
-      // ---- scores: S[16 tokens x 8 columns], two accumulator chains (even / odd k-steps) ----
-      float acc[4] = {0.f, 0.f, 0.f, 0.f}, accb[4] = {0.f, 0.f, 0.f, 0.f};
-      float accl[4] = {0.f, 0.f, 0.f, 0.f}, acclb[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- scores: per unit S[16 tokens x 8 columns], two accumulator chains ----
+      float sc[U][4];
 #pragma unroll
-      for (int s2 = 0; s2 < KST; ++s2) {
-        uint32_t a0, a1, a2, a3;
-        if constexpr (KB == 4) {
-          // dims (4 s2, 4 s2 + 1) are byte 2 (s2 % 2) of word s2 / 2; (+2, +3) the next byte
-          const uint32_t w0 = ks0[s2 >> 1], w1 = ks1[s2 >> 1];
-          const int k = 2 * (s2 & 1);
-          a0 = tab_ld(tab_off(w0, klo, k));
-          a1 = tab_ld(tab_off(w1, klo, k));
-          a2 = tab_ld(tab_off(w0, klo, k + 1));
-          a3 = tab_ld(tab_off(w1, klo, k + 1));
-        } else {
-          a0 = tab_ld((pair_at<KB, NWK>(ks0, 4 * s2 * KB) << 8) | klo);
-          a1 = tab_ld((pair_at<KB, NWK>(ks1, 4 * s2 * KB) << 8) | klo);
-          a2 = tab_ld((pair_at<KB, NWK>(ks0, (4 * s2 + 2) * KB) << 8) | klo);
-          a3 = tab_ld((pair_at<KB, NWK>(ks1, (4 * s2 + 2) * KB) << 8) | klo);
-        }
-        if (s2 & 1) {
-          mma16816(accb, a0, a1, a2, a3, qh[s2][0], qh[s2][1]);
-          if constexpr (!PK) mma16816(acclb, a0, a1, a2, a3, ql[s2][0], ql[s2][1]);
-        } else {
-          mma16816(acc, a0, a1, a2, a3, qh[s2][0], qh[s2][1]);
-          if constexpr (!PK) mma16816(accl, a0, a1, a2, a3, ql[s2][0], ql[s2][1]);
-        }
-      }
+      for (int u = 0; u < U; ++u) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, accb[4] = {0.f, 0.f, 0.f, 0.f};
+        float accl[4] = {0.f, 0.f, 0.f, 0.f}, acclb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] += accb[i] + (accl[i] + acclb[i]);
-      float acc2[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (KF == KFMT_PROD) {
-#pragma unroll
-        for (int s2 = 0; s2 < KST; ++s2) {
-          const uint32_t a0 = tab_ld(luts_a + ((((sw0 >> (4 * s2)) & 3u) << 5) + lane) * 4);
-          const uint32_t a1 = tab_ld(luts_a + ((((sw1 >> (4 * s2)) & 3u) << 5) + lane) * 4);
-          const uint32_t a2 = tab_ld(luts_a + ((((sw0 >> (4 * s2 + 2)) & 3u) << 5) + lane) * 4);
-          const uint32_t a3 = tab_ld(luts_a + ((((sw1 >> (4 * s2 + 2)) & 3u) << 5) + lane) * 4);
-          mma16816(acc2, a0, a1, a2, a3, qb[s2][0], qb[s2][1]);
+        for (int k = 0; k < KST; ++k) {
+          uint32_t a0, a1, a2, a3;
+          if constexpr (KB == 4) {
+            // dims (4 k, 4 k + 1) are byte 2 (k % 2) of word k / 2; (+2, +3) the next byte
+            const uint32_t w0c = ks[u][0][k >> 1], w1c = ks[u][1][k >> 1];
+            const int bsel = 2 * (k & 1);
+            a0 = tab_ld(tab_off(w0c, klo, bsel));
+            a1 = tab_ld(tab_off(w1c, klo, bsel));
+            a2 = tab_ld(tab_off(w0c, klo, bsel + 1));
+            a3 = tab_ld(tab_off(w1c, klo, bsel + 1));
+          } else {
+            a0 = tab_ld((pair_at<KB, NWK>(ks[u][0], 4 * k * KB) << 8) | klo);
+            a1 = tab_ld((pair_at<KB, NWK>(ks[u][1], 4 * k * KB) << 8) | klo);
+            a2 = tab_ld((pair_at<KB, NWK>(ks[u][0], (4 * k + 2) * KB) << 8) | klo);
+            a3 = tab_ld((pair_at<KB, NWK>(ks[u][1], (4 * k + 2) * KB) << 8) | klo);
+          }
+          if (k & 1) {
+            mma16816(accb, a0, a1, a2, a3, qh[k][0], qh[k][1]);
+            if constexpr (!PK) mma16816(acclb, a0, a1, a2, a3, ql[k][0], ql[k][1]);
+          } else {
+            mma16816(acc, a0, a1, a2, a3, qh[k][0], qh[k][1]);
+            if constexpr (!PK) mma16816(accl, a0, a1, a2, a3, ql[k][0], ql[k][1]);
+          }
         }
-      }
-      value_half();                                  // unit i - 1 (independent of the scores)
-      if constexpr (PK) {
-        // columns c and c + 4 hold the hi and lo products of one head: lanes t and t ^ 2
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
-          if constexpr (KF == KFMT_PROD) acc2[i] += __shfl_xor_sync(0xffffffffu, acc2[i], 2);
+        for (int i = 0; i < 4; ++i) acc[i] += accb[i] + (accl[i] + acclb[i]);
+        float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (KF == KFMT_PROD) {
+#pragma unroll
+          for (int k = 0; k < KST; ++k) {
+            const uint32_t a0 = tab_ld(luts_a + ((((sw[u][0] >> (4 * k)) & 3u) << 5) + lane) * 4);
+            const uint32_t a1 = tab_ld(luts_a + ((((sw[u][1] >> (4 * k)) & 3u) << 5) + lane) * 4);
+            const uint32_t a2 = tab_ld(luts_a + ((((sw[u][0] >> (4 * k + 2)) & 3u) << 5) + lane) * 4);
+            const uint32_t a3 = tab_ld(luts_a + ((((sw[u][1] >> (4 * k + 2)) & 3u) << 5) + lane) * 4);
+            mma16816(acc2, a0, a1, a2, a3, qb[k][0], qb[k][1]);
+          }
         }
-      }
-      // acc[0], acc[1]: token row g, heads h0, h0 + 1; acc[2], acc[3]: token row g + 8
-      float sc[4];
-      {
-        const float kr[4] = {kn0, kn0, kn1, kn1};
-        const float gr[4] = {gm0, gm0, gm1, gm1};
+        if constexpr (PK) {
+          // columns c and c + 4 hold the hi and lo products of one head: lanes t and t ^ 2
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
+            if constexpr (KF == KFMT_PROD) acc2[i] += __shfl_xor_sync(0xffffffffu, acc2[i], 2);
+          }
+        }
+        // acc[0], acc[1]: token row g, heads h0, h0 + 1; acc[2], acc[3]: token row g + 8
         const float sa[4] = {sa0, sa1, sa0, sa1}, sbq[4] = {sb0, sb1, sb0, sb1};
-        const bool ok[4] = {oka, oka, okb, okb};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float v = sa[i] * acc[i];
-          if constexpr (KF == KFMT_PROD) v += gr[i] * sbq[i] * acc2[i];
-          sc[i] = ok[i] ? kr[i] * v : -INFINITY;
+          if constexpr (KF == KFMT_PROD) v += gm[u][i >> 1] * sbq[i] * acc2[i];
+          sc[u][i] = ok[u][i >> 1] ? kn[u][i >> 1] * v : -INFINITY;
         }
       }
-      // ---- online softmax per head (log2 domain), reduced over the 8 token rows; the
+      // ---- online softmax per head (log2 domain) over the warp's tokens; the row
       // reduction runs only when some score of the warp exceeds its running maximum ----
-      if (__any_sync(0xffffffffu, sc[0] > m0 || sc[2] > m0 || sc[1] > m1 || sc[3] > m1)) {
-        float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+      bool up = false;
+#pragma unroll
+      for (int u = 0; u < U; ++u) up = up || sc[u][0] > m0 || sc[u][2] > m0 || sc[u][1] > m1 || sc[u][3] > m1;
+      if (__any_sync(0xffffffffu, up)) {
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          mx0 = fmaxf(mx0, fmaxf(sc[u][0], sc[u][2]));
+          mx1 = fmaxf(mx1, fmaxf(sc[u][1], sc[u][3]));
+        }
 #pragma unroll
         for (int o2 = 4; o2 < 32; o2 <<= 1) {
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
@@ -597,28 +588,63 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           m1 = mn1;
         }
       }
-      const float p00 = c0ok ? ex2(sc[0] - m0) : 0.f, p01 = c1ok ? ex2(sc[1] - m1) : 0.f;
-      const float p10 = c0ok ? ex2(sc[2] - m0) : 0.f, p11 = c1ok ? ex2(sc[3] - m1) : 0.f;
-      l0 += p00 + p10;
-      l1 += p01 + p11;
-      // P^T (16 tokens x 8 columns) as the B operand of the next value half: transpose the
-      // two 8x8 halves
-      uint32_t pth, ptl, pbh, pbl;
-      split_pair(p00 * vn0, p01 * vn0, pth, ptl);
-      split_pair(p10 * vn1, p11 * vn1, pbh, pbl);
-      if constexpr (PK) {
-        pb0h = movmatrix_t(plo ? ptl : pth);
-        pb1h = movmatrix_t(plo ? pbl : pbh);
-      } else {
-        pb0h = movmatrix_t(pth); pb1h = movmatrix_t(pbh);
-        pb0l = movmatrix_t(ptl); pb1l = movmatrix_t(pbl);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float p00 = c0ok ? ex2(sc[u][0] - m0) : 0.f, p01 = c1ok ? ex2(sc[u][1] - m1) : 0.f;
+        const float p10 = c0ok ? ex2(sc[u][2] - m0) : 0.f, p11 = c1ok ? ex2(sc[u][3] - m1) : 0.f;
+        l0 += p00 + p10;
+        l1 += p01 + p11;
+        // P^T (16 tokens x 8 columns) as the B operand: transpose the two 8x8 halves
+        uint32_t pth, ptl, pbh, pbl;
+        split_pair(p00 * vn[u][0], p01 * vn[u][0], pth, ptl);
+        split_pair(p10 * vn[u][1], p11 * vn[u][1], pbh, pbl);
+        uint32_t b0h, b1h, b0l = 0u, b1l = 0u;
+        if constexpr (PK) {
+          b0h = movmatrix_t(plo ? ptl : pth);
+          b1h = movmatrix_t(plo ? pbl : pbh);
+        } else {
+          b0h = movmatrix_t(pth); b1h = movmatrix_t(pbh);
+          b0l = movmatrix_t(ptl); b1l = movmatrix_t(pbl);
+        }
+        // ---- O'^T[128 dims x 8 columns] += V_hat^T . P^T ----
+        // M-tile i: row g = dim TDV g + i (first word of the slice), row g + 8 = dim TDV g + 8 + i
+        if constexpr (VB == 4) {
+          // byte j of lo (hi) holds the codes of one token pair for dim 2j (2j + 1) of a word
+          uint32_t lo[2][2], hi[2][2];   // [token pair][word]
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+              const uint32_t x = vs[u][2 * kp][w], y = vs[u][2 * kp + 1][w];
+              lo[kp][w] = (x & 0x0F0F0F0Fu) | ((y << 4) & 0xF0F0F0F0u);
+              hi[kp][w] = ((x >> 4) & 0x0F0F0F0Fu) | (y & 0xF0F0F0F0u);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const int k = i >> 1;
+            const uint32_t a0 = tab_ld(tab_off((i & 1) ? hi[0][0] : lo[0][0], vlo, k));
+            const uint32_t a1 = tab_ld(tab_off((i & 1) ? hi[0][1] : lo[0][1], vlo, k));
+            const uint32_t a2 = tab_ld(tab_off((i & 1) ? hi[1][0] : lo[1][0], vlo, k));
+            const uint32_t a3 = tab_ld(tab_off((i & 1) ? hi[1][1] : lo[1][1], vlo, k));
+            mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
+            if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const uint32_t e00 = field_at<VB, NWV>(vs[u][0], i * VB) | (field_at<VB, NWV>(vs[u][1], i * VB) << VB);
+            const uint32_t e01 = field_at<VB, NWV>(vs[u][0], (8 + i) * VB) | (field_at<VB, NWV>(vs[u][1], (8 + i) * VB) << VB);
+            const uint32_t e10 = field_at<VB, NWV>(vs[u][2], i * VB) | (field_at<VB, NWV>(vs[u][3], i * VB) << VB);
+            const uint32_t e11 = field_at<VB, NWV>(vs[u][2], (8 + i) * VB) | (field_at<VB, NWV>(vs[u][3], (8 + i) * VB) << VB);
+            const uint32_t a0 = tab_ld((e00 << 8) | vlo), a1 = tab_ld((e01 << 8) | vlo);
+            const uint32_t a2 = tab_ld((e10 << 8) | vlo), a3 = tab_ld((e11 << 8) | vlo);
+            mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
+            if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
+          }
+        }
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int w = 0; w < NWV; ++w) pvs[i][w] = vs[i][w];
     }
-    value_half();                                    // the last unit of the item
 
     // ---- merge this item across the consumer warps (named barrier 1) ----
 #pragma unroll
@@ -626,33 +652,40 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
     }
-    float* wm = mrg + warp * 8 * (D + 2);           // [column][m, l, o'[D]]
-    if (g == 0) {
-      wm[(2 * t) * (D + 2)] = m0; wm[(2 * t) * (D + 2) + 1] = l0;
-      wm[(2 * t + 1) * (D + 2)] = m1; wm[(2 * t + 1) * (D + 2) + 1] = l1;
-    }
+    if constexpr (PK) {
+      // fold the lo columns (lanes t ^ 2) into the hi columns: lanes t < 2 keep heads 2t, 2t+1
 #pragma unroll
-    for (int i = 0; i < MT; ++i) {
-      wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = o[i][0];
-      wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = o[i][1];
-      wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][2];
-      wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][3];
+      for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[i][j] += __shfl_xor_sync(0xffffffffu, o[i][j], 2);
+    }
+    float* wm = mrg + warp * RW * (D + 2);           // [row][m, l, o'[D]]
+    if (!PK || t < 2) {
+      if (g == 0) {
+        wm[(2 * t) * (D + 2)] = m0; wm[(2 * t) * (D + 2) + 1] = l0;
+        wm[(2 * t + 1) * (D + 2)] = m1; wm[(2 * t + 1) * (D + 2) + 1] = l1;
+      }
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = o[i][0];
+        wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = o[i][1];
+        wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][2];
+        wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][3];
+      }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
     for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
       const int r = idx / D, j = idx - r * D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kTmaConsumerWarps; ++w) M = fmaxf(M, mrg[(w * 8 + r) * (D + 2)]);
+      for (int w = 0; w < NC; ++w) M = fmaxf(M, mrg[(w * RW + r) * (D + 2)]);
       float a = 0.f, L = 0.f;
 #pragma unroll
-      for (int w = 0; w < kTmaConsumerWarps; ++w) {
-        const float* row = mrg + (w * 8 + r) * (D + 2);
+      for (int w = 0; w < NC; ++w) {
+        const float* row = mrg + (w * RW + r) * (D + 2);
         const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
         L += f * row[1];
-        float ov = row[2 + j];
-        if constexpr (PK) ov += row[4 * (D + 2) + 2 + j];      // the lo column of head r
-        a += f * ov;
+        a += f * row[2 + j];
       }
       const int64_t qi = qbase + r;
       const int64_t pi = qi * p.n_chunks + chunk;

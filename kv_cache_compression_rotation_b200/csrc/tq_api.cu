@@ -278,7 +278,7 @@ DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t N
     // persistent bulk-copy kernel: about 16 work items per SM, chunks of whole 112-token
     // stages, and (when the shape allows) an item count that is a multiple of the SMs;
     // a work item covers one block of up to 8 query heads of a GQA group
-    const int64_t stage = tma_stage_tokens(kq->kind == TQ_KIND_PROD ? KFMT_PROD : KFMT_MSE);
+    const int64_t stage = tma_stage_tokens(kq->kind == TQ_KIND_PROD ? KFMT_PROD : KFMT_MSE, Hq / Hkv <= 4);
     const int64_t wu = units * tma_head_blocks(Hq / Hkv);
     int64_t n0 = std::max<int64_t>(1, (16 * sms + wu - 1) / wu);
     for (int64_t cand = n0; cand < n0 + 8 && cand <= Nmax; ++cand)
