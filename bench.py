@@ -393,6 +393,128 @@ def run_reference(args, rank, world):
             "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def _flush_l2(buf):
+    buf.zero_()
+
+
+def _timed(fn, stream, flush=None, reps=10, warm=3):
+    """Median device time (ms) of fn() over reps launches, L2 flushed before each."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(np.median(ts))
+
+
+def run_other(args):
+    """Secondary workloads of the scope table (one GPU, parts timed separately, L2 flushed
+    before every timed launch).  The headline line is the default 128k decode workload."""
+    import torch
+    import tq_inputs as ti
+    import kv_cache_compression_rotation_b200 as K
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = measured_peaks()
+    l2buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = lambda: _flush_l2(l2buf)
+    wl = args.workload
+    parts = {}
+    Dm = 128
+    if wl in ("c2", "c4"):
+        cfg = {"c2": (1, 8, 32, 32768, 2), "c4": (32, 8, 32, 8192, 4)}[wl]
+        Bw, Hkv, Hq, Nw, cfgno = cfg
+        n = Bw * Hkv * Nw
+        U = ti.haar_rotation(Dm, ti.SEEDS["basis"] + cfgno)
+        kx = ti.anisotropic_torch(n, Dm, U, ti.SEEDS["keys"] + cfgno, dev)
+        vx = ti.anisotropic_torch(n, Dm, U, ti.SEEDS["values"] + cfgno, dev)
+        q = ti.normal_torch((Bw, Hq, Dm), ti.SEEDS["queries"] + cfgno, dev, dtype=torch.bfloat16)
+        if wl == "c2":
+            rot = ti.haar_rotation(Dm, ti.SEEDS["rotation"] + cfgno)
+            S = ti.gaussian_matrix(Dm, Dm, ti.SEEDS["qjl"] + cfgno)
+            kq, vq = K.Quantizer.prod(rot, S, 3, device=dev), K.Quantizer.mse(rot, 3, device=dev)
+            desc = "decode-32k: B=1, Hkv=8, Hq=32, d=128, context 32768, TurboQuant-prod b=3 keys (m=128), mse b=3 values"
+        else:
+            ck = ti.anisotropic(4096, Dm, U.astype(np.float64), ti.SEEDS["calib_keys"] + cfgno).astype(np.float32)
+            cv = ti.anisotropic(4096, Dm, U.astype(np.float64), ti.SEEDS["calib_values"] + cfgno).astype(np.float32)
+            S4 = ti.gaussian_matrix(4, 4, ti.SEEDS["qjl"] + cfgno)
+            kvec, kval = K.spectral_calibrate(ck)
+            vvec, vval = K.spectral_calibrate(cv)
+            kq = K.Quantizer.spectral(kvec, kval, 4, list(K.waterfill(kval[:4], 12)), 1, True, S4, device=dev)
+            vq = K.Quantizer.spectral(vvec, vval, 4, list(K.waterfill(vval[:4], 12)), 1, False, None, device=dev)
+            desc = ("decode-8k spectral: B=32, Hkv=8, Hq=32, d=128, context 8192, eigenvector rotation from 4096 "
+                    "calibration vectors, water-filled top-4 bits + 1-bit tail, QJL on the top 4 (keys)")
+        Lk, Lv = kq.layout(), vq.layout()
+        kb = 4 * (Lk.code_words + Lk.sign_words + Lk.has_norms + Lk.has_rnorms)
+        vb = 4 * (Lv.code_words + Lv.sign_words + Lv.has_norms + Lv.has_rnorms)
+        kc, vc = kq.alloc(n, dev), vq.alloc(n, dev)
+        seq = torch.full((Bw,), Nw, dtype=torch.int32, device=dev)
+        ws = torch.empty(K.decode_workspace_bytes(kq, Bw, Hq, Hkv, Nw), dtype=torch.uint8, device=dev)
+        out = torch.empty((Bw, Hq, Dm), dtype=torch.float32, device=dev)
+        tk = _timed(lambda: K.quantize(kq, kx, kc), stream, flush)
+        tv = _timed(lambda: K.quantize(vq, vx, vc), stream, flush)
+        td = _timed(lambda: K.decode_attn(kq, vq, q, seq, kc, vc, Nw, Hkv, out=out, workspace=ws), stream, flush)
+        assert K.get_status() == 0
+        qk_b, qv_b, d_b = n * (Dm * 2 + kb), n * (Dm * 2 + vb), n * (kb + vb)
+        parts = {"quantize_k": {"ms": tk, "gbs": qk_b / tk / 1e6, "vectors_per_s": n / tk * 1e3},
+                 "quantize_v": {"ms": tv, "gbs": qv_b / tv / 1e6, "vectors_per_s": n / tv * 1e3},
+                 "decode_attn": {"ms": td, "gbs": d_b / td / 1e6, "frac": d_b / td / 1e6 / peak,
+                                 "bytes_per_token": kb + vb}}
+        value, unit, step_ms = (qk_b + qv_b + d_b) / (tk + tv + td) / 1e6, "GB/s", tk + tv + td
+    elif wl == "c1":
+        rot = ti.haar_rotation(Dm, ti.SEEDS["rotation"] + 1)
+        x = torch.from_numpy(ti.iid_normal((4096, Dm), ti.SEEDS["keys"] + 1) / math.sqrt(Dm)).float().to(dev)
+        qq = torch.from_numpy(ti.iid_normal((64, Dm), ti.SEEDS["queries"] + 1) / math.sqrt(Dm)).float().to(dev)
+        kq = K.Quantizer.mse(rot, 3, device=dev)
+        kc = kq.alloc(4096, dev)
+        tq = _timed(lambda: K.quantize(kq, x, kc), stream, None)
+        ts = _timed(lambda: K.score(kq, qq, kc, 4096), stream, None)
+        parts = {"quantize": {"ms": tq, "vectors_per_s": 4096 / tq * 1e3},
+                 "score": {"ms": ts, "estimates_per_s": 64 * 4096 / ts * 1e3}}
+        desc = "scores-4k: d=128, 4096 keys fp32 N(0,1/d), 64 queries, mse b=3 (launch-bound; parity config)"
+        value, unit, step_ms = 4096 / (tq + ts) * 1e3, "vectors/s", tq + ts
+    elif wl == "c5":
+        d5, nq5 = 1536, args.c5_queries
+        ndb = args.c5_db
+        rot = ti.haar_rotation(d5, ti.SEEDS["rotation"] + 5)
+        S = ti.gaussian_matrix(d5, d5, ti.SEEDS["qjl"] + 5)
+        g = torch.Generator(device=dev)
+        g.manual_seed(ti.SEEDS["db"] + 5)
+        db = torch.randn((ndb, d5), generator=g, device=dev)
+        db /= db.norm(dim=1, keepdim=True)
+        g.manual_seed(ti.SEEDS["db_queries"] + 5)
+        qs = torch.randn((nq5, d5), generator=g, device=dev)
+        qs /= qs.norm(dim=1, keepdim=True)
+        kq = K.Quantizer.prod(rot, S, args.c5_bits, device=dev)
+        kc = kq.alloc(ndb, dev)
+        tq = _timed(lambda: K.quantize(kq, db, kc), stream, flush, reps=3, warm=1)
+        ts = _timed(lambda: K.score(kq, qs, kc, ndb, topk=10), stream, None, reps=3, warm=1)
+        L = kq.layout()
+        rec = 4 * (L.code_words + L.sign_words + L.has_norms + L.has_rnorms)
+        parts = {"quantize": {"ms": tq, "vectors_per_s": ndb / tq * 1e3, "gbs": ndb * (d5 * 4 + rec) / tq / 1e6},
+                 "search_top10": {"ms": ts, "queries_per_s": nq5 / ts * 1e3,
+                                  "note": f"{nq5} queries x {ndb} records, CUDA-core estimator"}}
+        desc = (f"search: {ndb} x 1536 fp32 unit vectors, prod b={args.c5_bits} (m=1536), "
+                f"top-10 of {nq5} queries")
+        value, unit, step_ms = ndb / tq * 1e3, "vectors/s", tq
+    else:
+        raise SystemExit(f"unknown workload {wl}")
+    return {"metric": f"{wl} secondary workload", "value": value, "unit": unit, "n_gpus": 1, "steps": 10,
+            "warmup": 3, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": {"workload": desc, "l2": "flushed before each timed launch"},
+            "parts": parts, "peak_hbm_gbs": peak, "peak_source": peak_kind}
+
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -408,7 +530,19 @@ def main():
                     help="profiling aid: context length (the headline workload uses 131072)")
     ap.add_argument("--batch", type=int, default=B,
                     help="profiling aid: batch size (the headline workload uses 8)")
+    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5"],
+                    help="c3 (default): the 128k decode step of the headline; the others are the scope "
+                         "table's secondary workloads, timed per kernel")
+    ap.add_argument("--c5-queries", type=int, default=100)
+    ap.add_argument("--c5-db", type=int, default=1000000)
+    ap.add_argument("--c5-bits", type=int, default=2)
     args = ap.parse_args()
+    if args.workload != "c3":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the headline workload only"}))
+            return
+        print(json.dumps(run_other(args)))
+        return
     globals()["N"] = args.context
     globals()["B"] = args.batch
     world = int(os.environ.get("WORLD_SIZE", "1"))

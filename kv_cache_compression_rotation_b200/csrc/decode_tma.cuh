@@ -531,7 +531,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           }
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += accb[i] + (accl[i] + acclb[i]);
+        for (int i = 0; i < 4; ++i) acc[i] += PK ? accb[i] : accb[i] + (accl[i] + acclb[i]);
         float acc2[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (KF == KFMT_PROD) {
 #pragma unroll

@@ -52,14 +52,74 @@ __device__ __forceinline__ void spectral_dim_book(const SimtQuantParams& p, int 
   *sig = p.dim_sigma[j];
 }
 
-// Shared memory: xs[tv][d] f32 | ys[tv][d] f32 | code8[tv][d] u8 | nu[tv] | inv[tv] | gam[tv]
+// Tiled product on CUDA cores: out[v][j] = scale_v * sum_k A[v][k] M[j][k] for v < 8 * VPT
+// rows of A (shared memory, row stride lda, zero-padded to a multiple of 32 columns) and
+// j < mrows rows of M (global, row-major [mrows][d]).  M is staged through shared memory
+// in 32-column chunks of 128 rows (Ms, [32][kMsStride], transposed); thread (ty, tx) owns
+// rows ty * VPT .. + VPT - 1 and outputs tx + 32 q of each 128-row block.
+constexpr int kMsStride = 132;
+
+template <int VPT>
+__device__ __forceinline__ void tile_gemm(const float* A, int lda, const float* __restrict__ M, int mrows, int d,
+                                          float* out, int ldo, const float* rowscale, float* Ms) {
+  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
+  const int dp = (d + 31) & ~31;
+  for (int jb = 0; jb < mrows; jb += 128) {
+    float acc[VPT][4];
+#pragma unroll
+    for (int v = 0; v < VPT; ++v)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[v][q] = 0.f;
+    for (int k0 = 0; k0 < dp; k0 += 32) {
+      __syncthreads();                              // Ms is free
+      for (int i = tid; i < 32 * 128; i += kSimtThreads) {
+        const int jj = i >> 5, kk = i & 31, row = jb + jj, col = k0 + kk;
+        Ms[kk * kMsStride + jj] = (row < mrows && col < d) ? __ldg(M + static_cast<int64_t>(row) * d + col) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 2
+      for (int kk = 0; kk < 32; kk += 4) {
+        float4 a[VPT];
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) a[v] = *reinterpret_cast<const float4*>(A + (ty * VPT + v) * lda + k0 + kk);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          float b[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) b[q] = Ms[(kk + k4) * kMsStride + tx + 32 * q];
+#pragma unroll
+          for (int v = 0; v < VPT; ++v) {
+            const float av = k4 == 0 ? a[v].x : (k4 == 1 ? a[v].y : (k4 == 2 ? a[v].z : a[v].w));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[v][q] = fmaf(av, b[q], acc[v][q]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+      const float sc = rowscale ? rowscale[ty * VPT + v] : 1.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = jb + tx + 32 * q;
+        if (j < mrows) out[(ty * VPT + v) * ldo + j] = acc[v][q] * sc;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Shared memory: xs[tv][dp] f32 | ys[tv][yp] f32 | Ms[32][kMsStride] f32 | nu[tv] | inv[tv] |
+// gam[tv] | code8[tv][d] u8, with dp = d and yp = max(d, m) rounded up to 32 (zero padding).
 __global__ void __launch_bounds__(kSimtThreads)
 simt_quantize_kernel(SimtQuantParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int d = p.d, tv = p.tv;
+  const int dp = (d + 31) & ~31, yp = (max(d, p.m) + 31) & ~31;
   float* xs = reinterpret_cast<float*>(smem);
-  float* ys = xs + tv * d;
-  float* nu = ys + tv * d;
+  float* ys = xs + tv * dp;
+  float* Ms = ys + tv * yp;
+  float* nu = Ms + 32 * kMsStride;
   float* inv = nu + tv;
   float* gam = inv + tv;
   uint8_t* code8 = reinterpret_cast<uint8_t*>(gam + tv);
@@ -67,14 +127,14 @@ simt_quantize_kernel(SimtQuantParams p) {
   const int nv = static_cast<int>(min(static_cast<int64_t>(tv), p.n - v0));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  for (int i = tid; i < tv * d; i += kSimtThreads) {
-    const int v = i / d;
-    xs[i] = v < nv ? load_elem(p.x, p.dtype, (v0 + v) * d + (i - v * d)) : 0.f;
+  for (int i = tid; i < tv * dp; i += kSimtThreads) {
+    const int v = i / dp, k = i - v * dp;
+    xs[i] = (v < nv && k < d) ? load_elem(p.x, p.dtype, (v0 + v) * d + k) : 0.f;
   }
   __syncthreads();
   for (int v = warp; v < tv; v += kSimtThreads / 32) {
     float s = 0.f;
-    for (int k = lane; k < d; k += 32) s += xs[v * d + k] * xs[v * d + k];
+    for (int k = lane; k < d; k += 32) s += xs[v * dp + k] * xs[v * dp + k];
     s = warp_sum(s);
     if (lane == 0) {
       const float r = sqrtf(s);
@@ -84,28 +144,16 @@ simt_quantize_kernel(SimtQuantParams p) {
   }
   __syncthreads();
   // y = rot @ x (per vector), scaled to the unit sphere for mse / prod
-  for (int j = tid; j < d; j += kSimtThreads) {
-    const float* rrow = p.rot + static_cast<int64_t>(j) * d;
-    for (int vb = 0; vb < tv; vb += 8) {
-      float acc[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-      for (int k = 0; k < d; ++k) {
-        const float r = __ldg(rrow + k);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (vb + u < tv) acc[u] = fmaf(r, xs[(vb + u) * d + k], acc[u]);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (vb + u < tv) ys[(vb + u) * d + j] = acc[u] * inv[vb + u];
-    }
+  switch (tv / 8) {
+    case 1: tile_gemm<1>(xs, dp, p.rot, d, d, ys, yp, inv, Ms); break;
+    case 2: tile_gemm<2>(xs, dp, p.rot, d, d, ys, yp, inv, Ms); break;
+    case 3: tile_gemm<3>(xs, dp, p.rot, d, d, ys, yp, inv, Ms); break;
+    default: tile_gemm<4>(xs, dp, p.rot, d, d, ys, yp, inv, Ms); break;
   }
-  __syncthreads();
   // scalar codes (and residual for prod / spectral-qjl, kept in xs)
   for (int i = tid; i < tv * d; i += kSimtThreads) {
-    const int j = i % d;
-    const float y = ys[i];
+    const int v = i / d, j = i - v * d;
+    const float y = ys[v * yp + j];
     int c = 0;
     float chat = 0.f;
     if (p.kind == TQ_KIND_SPECTRAL) {
@@ -127,7 +175,7 @@ simt_quantize_kernel(SimtQuantParams p) {
       chat = __ldg(p.centroids + c);
     }
     code8[i] = static_cast<uint8_t>(c);
-    xs[i] = y - chat;   // residual (x no longer needed)
+    xs[v * dp + j] = y - chat;   // residual (x no longer needed; padding stays 0)
   }
   __syncthreads();
   // pack code words
@@ -155,10 +203,10 @@ simt_quantize_kernel(SimtQuantParams p) {
       float proj[TQ_MAX_TOP];
       float g2 = 0.f;
       if (p.qjl) {
-        for (int i = 0; i < k; ++i) g2 += xs[v * d + i] * xs[v * d + i];
+        for (int i = 0; i < k; ++i) g2 += xs[v * dp + i] * xs[v * dp + i];
         for (int i = 0; i < k; ++i) {
           float a = 0.f;
-          for (int kk = 0; kk < k; ++kk) a = fmaf(__ldg(p.S + i * k + kk), xs[v * d + kk], a);
+          for (int kk = 0; kk < k; ++kk) a = fmaf(__ldg(p.S + i * k + kk), xs[v * dp + kk], a);
           proj[i] = a;
         }
       }
@@ -205,22 +253,25 @@ simt_quantize_kernel(SimtQuantParams p) {
   }
   if (tid < nv && p.norms) p.norms[v0 + tid] = nu[tid];
   if (p.kind != TQ_KIND_PROD) return;
-  // prod: gamma = ||r||, signs of S r by warp ballot (32 rows of S per warp step)
+  // prod: gamma = ||r||, then S r for the tile (tiled product) and its signs by warp ballot
   for (int v = warp; v < tv; v += kSimtThreads / 32) {
     float s = 0.f;
-    for (int k = lane; k < d; k += 32) s += xs[v * d + k] * xs[v * d + k];
+    for (int k = lane; k < d; k += 32) s += xs[v * dp + k] * xs[v * dp + k];
     s = warp_sum(s);
     if (lane == 0) gam[v] = sqrtf(s);
   }
   __syncthreads();
   if (tid < nv && p.rnorms) p.rnorms[v0 + tid] = gam[tid];
-  for (int ib = warp * 32; ib < p.m; ib += kSimtThreads) {
-    const int i = ib + lane;
-    const float* srow = p.S + static_cast<int64_t>(min(i, p.m - 1)) * d;
-    for (int v = 0; v < nv; ++v) {
-      float a = 0.f;
-      for (int k = 0; k < d; ++k) a = fmaf(__ldg(srow + k), xs[v * d + k], a);
-      const unsigned bits = __ballot_sync(0xffffffffu, i < p.m && a >= 0.f);
+  switch (tv / 8) {
+    case 1: tile_gemm<1>(xs, dp, p.S, p.m, d, ys, yp, nullptr, Ms); break;
+    case 2: tile_gemm<2>(xs, dp, p.S, p.m, d, ys, yp, nullptr, Ms); break;
+    case 3: tile_gemm<3>(xs, dp, p.S, p.m, d, ys, yp, nullptr, Ms); break;
+    default: tile_gemm<4>(xs, dp, p.S, p.m, d, ys, yp, nullptr, Ms); break;
+  }
+  for (int v = warp; v < nv; v += kSimtThreads / 32) {
+    for (int ib = 0; ib < p.m; ib += 32) {
+      const int i = ib + lane;
+      const unsigned bits = __ballot_sync(0xffffffffu, i < p.m && ys[v * yp + min(i, p.m - 1)] >= 0.f);
       if (lane == 0) p.signs[(v0 + v) * p.sign_words + (ib >> 5)] = bits;
     }
   }

@@ -249,9 +249,18 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   p.norms = L.has_norms ? out.norms : nullptr;
   p.rnorms = L.has_rnorms ? out.rnorms : nullptr;
   const int d = q->d;
-  int tv = static_cast<int>(std::min<int64_t>(16, std::max<int64_t>(1, 180000 / (9 * d + 12))));
+  // vectors per CTA: a multiple of 8 (the tiled product's row groups), at most 32, within
+  // 200 KB of shared memory
+  const int dp = (d + 31) & ~31, yp = (std::max(d, p.m) + 31) & ~31;
+  auto smem_for = [&](int tvv) {
+    return static_cast<size_t>(tvv) * (dp + yp) * 4 + 32 * 132 * 4 + static_cast<size_t>(tvv) * 12 +
+           static_cast<size_t>(tvv) * d + 16;
+  };
+  int tv = 32;
+  while (tv > 8 && smem_for(tv) > 200 * 1024) tv -= 8;
+  if (smem_for(tv) > 220 * 1024) return fail(TQ_ERR_UNSUPPORTED, "d = %d too large for the general quantize kernel", d);
   p.tv = tv;
-  const size_t smem = static_cast<size_t>(tv) * d * 9 + static_cast<size_t>(tv) * 12 + 16;
+  const size_t smem = smem_for(tv);
   cudaError_t e = cudaFuncSetAttribute(simt_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "simt quantize attribute");
