@@ -5,9 +5,9 @@
 namespace tq {
 namespace {
 
-template <int B>
+template <int B, bool SPEC = false>
 cudaError_t go(const CUtensorMap& map, const UmmaQuantParams& p, int grid, cudaStream_t s) {
-  auto k = umma_quantize_kernel<B>;
+  auto k = umma_quantize_kernel<B, SPEC>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kUmmaSmemBytes));
   if (e != cudaSuccess) return e;
   k<<<grid, kUmmaThreads, kUmmaSmemBytes, s>>>(map, p);
@@ -18,6 +18,7 @@ cudaError_t go(const CUtensorMap& map, const UmmaQuantParams& p, int grid, cudaS
 
 cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& p, int bits, int grid,
                                  cudaStream_t s) {
+  if (bits == 0) return go<1, true>(map, p, grid, s);       // spectral records
   switch (bits) {
     case 1: return go<1>(map, p, grid, s);
     case 2: return go<2>(map, p, grid, s);

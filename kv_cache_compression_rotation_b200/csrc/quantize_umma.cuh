@@ -44,7 +44,10 @@ constexpr uint32_t kPiBytes = kUmmaD * kUmmaD * 2;                 // 32 KB per 
 constexpr long long kDrainLimit = 1ll << 28;
 // 32 cells over [-R, R): f in [0, 1] maps to floor(f * kCellSpan) in 0..31
 constexpr float kCellSpan = 31.9999f;
-constexpr uint32_t kUmmaSmemBytes = 1024 /*align slack*/ + 2 * kPiBytes + kUmmaStages * kXStageBytes + 256;
+// spectral tables: per top dim up to 63 thresholds and 64 centroids (top bits <= 6), S (<= 8 x 8)
+constexpr int kSpecMaxTopBits = 6;
+constexpr uint32_t kSpecTabBytes = (TQ_MAX_TOP * 64 * 2 + 64) * 4;
+constexpr uint32_t kUmmaSmemBytes = 1024 /*align slack*/ + 2 * kPiBytes + kUmmaStages * kXStageBytes + 256 + kSpecTabBytes;
 
 struct UmmaQuantParams {
   const float* rot;        // [128*128] fp32
@@ -55,6 +58,14 @@ struct UmmaQuantParams {
   float* norms;            // [n]
   int* status;
   long long wait_limit;
+  // spectral records (1-bit tail): top dims 0..k_top-1 with their own bits, QJL on them
+  int k_top, qjl;
+  int top_bits[TQ_MAX_TOP];
+  const float* dim_sigma;  // [128]
+  const float* unit_c;     // standard-normal codebooks (concatenated by bits)
+  const float* unit_t;
+  const float* S;          // [k_top*k_top] (qjl)
+  float* rnorms;           // [n] (qjl)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -164,27 +175,41 @@ __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B
   }
 }
 
-template <int B>
+// SPEC: spectral records instead of MSE codes (B unused): z = rot x without normalization;
+// tail dims take 1 bit, code (z_j > 0) (the 1-bit standard-normal boundary is 0); the top
+// dims are coded against sigma_j times their unit codebooks and get the QJL signs of
+// S (z_top - c_top); record = head word + 4 tail words (+ ||z_top - c_top||).
+template <int B, bool SPEC>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
 umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantParams p) {
   constexpr int K = 1 << B;
   constexpr int NB = K - 1;
   constexpr int W = kUmmaD * B / 32;             // code words per vector
+  // spectral codes compare raw (unnormalized) coordinates with boundaries at 0, where the
+  // data is densest: Pi takes three 16-bit terms (hi + lo + lo2, ~2^-26 relative) instead of
+  // two, and the ring one stage less so the shared memory stays the same
+  constexpr int NT = SPEC ? 3 : 2;
+  constexpr int NS = SPEC ? 3 : kUmmaStages;
+  static_assert(NT * kPiBytes + NS * kXStageBytes == 2 * kPiBytes + kUmmaStages * kXStageBytes, "smem");
   extern __shared__ unsigned char usm_raw[];
   const uint32_t raw = smem_u32(usm_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = usm_raw + (base - raw);
-  const uint32_t pi_hi = base, pi_lo = base + kPiBytes;
-  const uint32_t xs0 = base + 2 * kPiBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * kPiBytes + kUmmaStages * kXStageBytes);
+  const uint32_t pi_hi = base, pi_lo = base + kPiBytes, pi_lo2 = base + 2 * kPiBytes;
+  const uint32_t xs0 = base + NT * kPiBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + NT * kPiBytes + NS * kXStageBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kUmmaStages + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kUmmaStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kUmmaStages + 2 + b); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kUmmaStages + 4);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * NS + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tsm = reinterpret_cast<float*>(tmem_slot + 2);   // boundaries [NB]
+  // spectral: thresholds [top dim][64], centroids [top dim][64], S [64]
+  float* sthr = reinterpret_cast<float*>(sm + NT * kPiBytes + NS * kXStageBytes + 256);
+  float* scen = sthr + TQ_MAX_TOP * 64;
+  float* sS = scen + TQ_MAX_TOP * 64;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (p.n + kUmmaTileRows - 1) / kUmmaTileRows;
@@ -193,24 +218,37 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   for (int i = tid; i < kUmmaD * kUmmaD; i += kUmmaThreads) {
     const int nrow = i >> 7, k = i & 127;
     const float v = __ldg(p.rot + i);
-    uint16_t hi, lo;
+    uint16_t hi, lo, lo2;
     if (p.is_f16) {
       const __half h = __float2half_rn(v);
       const __half l = __float2half_rn(v - __half2float(h));
-      hi = __half_as_ushort(h); lo = __half_as_ushort(l);
+      const __half l2 = __float2half_rn(v - __half2float(h) - __half2float(l));
+      hi = __half_as_ushort(h); lo = __half_as_ushort(l); lo2 = __half_as_ushort(l2);
     } else {
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
       const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-      hi = __bfloat16_as_ushort(h); lo = __bfloat16_as_ushort(l);
+      const __nv_bfloat16 l2 = __float2bfloat16_rn(v - __bfloat162float(h) - __bfloat162float(l));
+      hi = __bfloat16_as_ushort(h); lo = __bfloat16_as_ushort(l); lo2 = __bfloat16_as_ushort(l2);
     }
     const int kb = k >> 6, kk = k & 63;
     const uint32_t off = kb * (kUmmaD * 128) + nrow * 128 + ((((kk >> 3) ^ (nrow & 7))) << 4) + (kk & 7) * 2;
     *reinterpret_cast<uint16_t*>(sm + off) = hi;
     *reinterpret_cast<uint16_t*>(sm + kPiBytes + off) = lo;
+    if (NT == 3) *reinterpret_cast<uint16_t*>(sm + 2 * kPiBytes + off) = lo2;
   }
-  if (tid < NB) tsm[tid] = __ldg(p.boundaries + tid);
+  if constexpr (SPEC) {
+    for (int i = tid; i < p.k_top * 64; i += kUmmaThreads) {
+      const int j = i >> 6, k = i & 63, b = p.top_bits[j];
+      const float sg = __ldg(p.dim_sigma + j);
+      sthr[i] = k < (1 << b) - 1 ? sg * __ldg(p.unit_t + unit_t_off(b) + k) : 3.0e38f;
+      scen[i] = k < (1 << b) ? sg * __ldg(p.unit_c + unit_c_off(b) + k) : 0.f;
+    }
+    if (p.qjl && tid < p.k_top * p.k_top) sS[tid] = __ldg(p.S + tid);
+  } else {
+    if (tid < NB) tsm[tid] = __ldg(p.boundaries + tid);
+  }
   if (tid == 0) {
-    for (int s = 0; s < kUmmaStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int s = 0; s < NS; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), 128); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -233,7 +271,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       int it = 0;
       int issued = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-        const int s = it % kUmmaStages, use = it / kUmmaStages;
+        const int s = it % NS, use = it / NS;
         if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, lim, p.status, abort_flag)) break;
         mbar_expect_tx(full_bar(s), kXStageBytes);
         const uint32_t dst = xs0 + s * kXStageBytes;
@@ -243,8 +281,8 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         ++issued;
       }
       // drain: every issued stage must land before the CTA can exit
-      for (int j = max(0, issued - kUmmaStages); j < issued; ++j) {
-        const int s = j % kUmmaStages, use = j / kUmmaStages;
+      for (int j = max(0, issued - NS); j < issued; ++j) {
+        const int s = j % NS, use = j / NS;
         for (long long i = 0; !mbar_try(full_bar(s), use & 1) && i < kDrainLimit; ++i) {}
       }
     }
@@ -253,9 +291,9 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       const uint32_t idesc = idesc_m128n128(p.is_f16);
       int it = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-        const int s = it % kUmmaStages, buf = it & 1, j = it >> 1;
+        const int s = it % NS, buf = it & 1, j = it >> 1;
         if (j > 0 && !mbar_wait(tempty_bar(buf), (j - 1) & 1, lim, p.status, abort_flag)) break;
-        if (!mbar_wait(full_bar(s), (it / kUmmaStages) & 1, lim, p.status, abort_flag)) break;
+        if (!mbar_wait(full_bar(s), (it / NS) & 1, lim, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t xa = xs0 + s * kXStageBytes;
         const uint32_t td = tmem_base + buf * 128;
@@ -265,6 +303,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           const uint32_t poff = (kk >> 2) * (kPiBytes / 2) + (kk & 3) * 32;
           umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_hi + poff), idesc, kk > 0 ? 1u : 0u);
           umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo + poff), idesc, 1u);
+          if (NT == 3) umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo2 + poff), idesc, 1u);
         }
         umma_commit(empty_bar(s));
         umma_commit(tfull_bar(buf));
@@ -313,6 +352,64 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 128;
       const int64_t v = tile * kUmmaTileRows + r;
+      if constexpr (SPEC) {
+        const int kt = p.k_top;
+        uint32_t tail[4];
+        float ztop[TQ_MAX_TOP];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float z[32];
+          tmem_ld32(taddr + 32 * c, z);
+          tmem_wait_ld();
+          uint32_t wbits = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) wbits |= (z[i] > 0.f ? 1u : 0u) << i;
+          if (c == 0) {
+#pragma unroll
+            for (int j = 0; j < TQ_MAX_TOP; ++j) ztop[j] = z[j];
+            wbits &= ~((1u << kt) - 1u);                // top dims carry no tail code
+          }
+          tail[c] = wbits;
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(buf));
+        uint32_t head = 0u;
+        int pos = 0;
+        float rr[TQ_MAX_TOP];
+        float g2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < TQ_MAX_TOP; ++j) {
+          rr[j] = 0.f;
+          if (j < kt) {
+            const int b = p.top_bits[j];
+            uint32_t cnt = 0u;
+            for (int k = 0; k < (1 << b) - 1; ++k) cnt += ztop[j] > sthr[j * 64 + k] ? 1u : 0u;
+            head |= cnt << pos;
+            pos += b;
+            rr[j] = ztop[j] - scen[j * 64 + cnt];
+            g2 = fmaf(rr[j], rr[j], g2);
+          }
+        }
+        if (p.qjl) {
+#pragma unroll
+          for (int i = 0; i < TQ_MAX_TOP; ++i) {
+            if (i < kt) {
+              float a = 0.f;
+#pragma unroll
+              for (int k = 0; k < TQ_MAX_TOP; ++k)
+                if (k < kt) a = fmaf(sS[i * kt + k], rr[k], a);
+              head |= (a >= 0.f ? 1u : 0u) << (pos + i);
+            }
+          }
+        }
+        if (v < p.n) {
+          uint32_t* dst = p.codes + v * 5;
+          dst[0] = head;
+          dst[1] = tail[0]; dst[2] = tail[1]; dst[3] = tail[2]; dst[4] = tail[3];
+          if (p.qjl) p.rnorms[v] = sqrtf(g2);
+        }
+        continue;
+      }
       // pass 1: ||y|| over the whole row (independent partial sums keep the FMA pipe busy)
       float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -178,8 +178,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+// spectral records the tensor-core kernel writes: 1-bit tail, top dims of <= 6 bits in one
+// head word, 4 tail words
+bool umma_spectral(const tq_quantizer* q) {
+  if (q->kind != TQ_KIND_SPECTRAL || q->tail_bits != 1 || q->k_top < 1 || q->k_top > TQ_MAX_TOP) return false;
+  int hb = q->qjl ? q->k_top : 0;
+  for (int j = 0; j < q->k_top; ++j) {
+    if (q->top_bits[j] < 1 || q->top_bits[j] > kSpecMaxTopBits) return false;
+    hb += q->top_bits[j];
+  }
+  return hb <= 32 && (!q->qjl || q->S);
+}
+
 bool umma_supported(const tq_quantizer* q, int dtype, int64_t n) {
-  if (q->kind != TQ_KIND_MSE || q->d != 128 || q->bits > 4) return false;
+  if (q->d != 128) return false;
+  if (q->kind == TQ_KIND_MSE ? q->bits > 4 : !umma_spectral(q)) return false;
   if (dtype != TQ_BF16 && dtype != TQ_F16) return false;
   if (n < 1 || n >= (1ll << 31) - 256) return false;
   if (std::getenv("TQ_FORCE_SIMT")) return false;
@@ -229,9 +242,15 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
     p.norms = out.norms;
     p.status = status;
     p.wait_limit = wait_limit();
+    if (q->kind == TQ_KIND_SPECTRAL) {
+      p.k_top = q->k_top; p.qjl = q->qjl;
+      for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];
+      p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids; p.unit_t = q->unit_boundaries;
+      p.S = q->S; p.rnorms = q->qjl ? out.rnorms : nullptr;
+    }
     const int64_t tiles = (n + 127) / 128;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
-    const cudaError_t e = launch_umma_quantize(map, p, q->bits, grid, stream);
+    const cudaError_t e = launch_umma_quantize(map, p, q->kind == TQ_KIND_SPECTRAL ? 0 : q->bits, grid, stream);
     return e == cudaSuccess ? TQ_OK : cuda_fail(e, "umma quantize launch");
   }
 
