@@ -1,5 +1,7 @@
-// Instantiations of decode_attn_kernel with keys in the spec format (D = 128).
+// Instantiations of the decode kernels for spectral keys and values (D = 128): the
+// bulk-copy staged kernel for 1-bit tails with one head word, the 4-warp kernel otherwise.
 #include "decode.cuh"
+#include "decode_tma.cuh"
 #include "launchers.h"
 
 namespace tq {
@@ -14,7 +16,21 @@ cudaError_t go(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <bool PK>
+cudaError_t go_tma(const DecodeParams& p, dim3 grid, cudaStream_t s, int* status, long long lim) {
+  auto k = decode_tma_kernel<KFMT_SPEC, 1, 1, PK>;
+  const size_t smem = decode_tma_smem_bytes(1, 1, KFMT_SPEC, PK);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k<<<grid, (tma_consumers(KFMT_SPEC, PK) + 1) * 32, smem, s>>>(p, status, lim);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_decode_spec_tma(const DecodeParams& p, dim3 grid, cudaStream_t s, int* status, long long lim) {
+  return p.G <= 4 ? go_tma<true>(p, grid, s, status, lim) : go_tma<false>(p, grid, s, status, lim);
+}
 
 cudaError_t launch_decode_spec(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s) {
   switch (kb * 10 + vb) {

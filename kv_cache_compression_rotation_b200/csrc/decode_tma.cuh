@@ -94,12 +94,15 @@ __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int k
   const int st = tma_stage_tokens(kf, pk);
   TmaStageLayout L{};
   uint32_t o = 0;
-  L.kcodes = o; o += st * kw * 4;
-  L.vcodes = o; o += st * vw * 4;
-  L.knorm = o; o += (st + 4) * 4;
-  L.vnorm = o; o += (st + 4) * 4;
+  // spectral records (20 bytes) are staged from the 16-byte boundary below the stage's first
+  // record: slack for the partial 16-byte blocks at both ends
+  const int slack = (kf == KFMT_SPEC) ? 32 : 0;
+  L.kcodes = o; o += st * kw * 4 + slack;
+  L.vcodes = o; o += st * vw * 4 + slack;
+  L.knorm = o; o += (kf == KFMT_SPEC) ? 0 : (st + 4) * 4;
+  L.vnorm = o; o += (kf == KFMT_SPEC) ? 0 : (st + 4) * 4;
   L.ksign = o; o += (kf == KFMT_PROD) ? st * ksw * 4 : 0;
-  L.krn = o; o += (kf == KFMT_PROD) ? (st + 4) * 4 : 0;
+  L.krn = o; o += (kf == KFMT_PROD || kf == KFMT_SPEC) ? (st + 4) * 4 : 0;
   L.bytes = o;
   return L;
 }
@@ -114,11 +117,13 @@ __host__ __device__ inline uint32_t tma_table_bytes(int kb, int vb) {
 __host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u : 8u; }
 __host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk) {
   const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf, pk)) * tma_merge_rows(pk) * (128u + 2u) * 4u;
-  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u;
+  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u + 510u * 4u + 8u;
   return (v + 127u) & ~127u;
 }
+// words of one record: the code stream, plus the head word of a spectral record
+__host__ __device__ constexpr int tma_record_words(int bits, int kf) { return 128 * bits / 32 + (kf == KFMT_SPEC ? 1 : 0); }
 inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, bool pk) {
-  const TmaStageLayout L = tma_stage_layout(128 * kb / 32, 128 * vb / 32, kf, 4, pk);
+  const TmaStageLayout L = tma_stage_layout(tma_record_words(kb, kf), tma_record_words(vb, kf), kf, 4, pk);
   const size_t want = 65536 + tma_table_bytes(kb, vb) + static_cast<size_t>(tma_stages(pk)) * L.bytes +
                       tma_misc_bytes(kf, pk);
   return want < 232448 ? want : 232448;
@@ -208,7 +213,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int NWV = (TDV * VB + 31) / 32;
   constexpr int MT = D / 16;                  // P.V M-tiles (16 dims each)
   constexpr int KLUT = 1 << (2 * KB), VLUT = 1 << (2 * VB);
-  constexpr int KW = D * KB / 32, VW = D * VB / 32;     // record words
+  constexpr bool SP = KF == KFMT_SPEC;                 // spectral keys and values (1-bit tails)
+  constexpr int KW = tma_record_words(KB, KF), VW = tma_record_words(VB, KF);   // record words
+  constexpr int TOFF = SP ? 32 : 0;                    // bit offset of the code stream in a record
   constexpr int KSW = 4;                                // prod sign words (m = 128)
   constexpr int HB = PK ? 4 : kTmaHeadBlock;            // query heads per work item
   constexpr int RW = static_cast<int>(tma_merge_rows(PK));   // merge rows per warp
@@ -258,6 +265,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   int* nb_off = nb_count + NS;                              // [NS] their offset in the stage
   volatile int* abort_flag = nb_off + NS;
   volatile int* consumers_stop = abort_flag + 1;   // uniform exit decision of the consumer warps
+  float* utab = reinterpret_cast<float*>(const_cast<int*>(consumers_stop) + 2);   // spectral unit codebooks [510]
   const uint32_t bar0 = tma_smem_u32(bars);
   const uint32_t nb_a = tma_smem_u32(nb_count);
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
@@ -304,11 +312,17 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     const int e = tid >> 5;
     luts[tid] = pack_half2((e & 1) ? 1.f : -1.f, (e & 2) ? 1.f : -1.f);
   }
+  if constexpr (SP)
+    for (int i = tid; i < 510; i += kTmaThreads) utab[i] = __ldg(p.unit_c + i);
   __syncthreads();
 
   if (warp == NC) {
     // ---------------- producer ----------------
-    if (lane == 0) {
+    // Bulk copies need 16-byte aligned sources, destinations and sizes.  MSE and PROD records
+    // are multiples of 16 bytes; spectral records (20 bytes) are copied word by word by the
+    // whole producer warp instead, and only their gamma array goes by bulk copy.
+    static_assert(SP || ((KW * 4) % 16 == 0 && (VW * 4) % 16 == 0), "record size");
+    if (SP || lane == 0) {
       int gs = 0;                                   // global stage counter of this CTA
       bool stop = false;
       for (int item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
@@ -317,7 +331,10 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         const int64_t rec0 = static_cast<int64_t>(bh) * p.Nmax;
         for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
           const int st = gs % NS, use = gs / NS;
-          if (use > 0 && !tma_mbar_wait(empty_bar(st), (use - 1) & 1, wait_lim, status, abort_flag)) {
+          bool free_ok = true;
+          if (use > 0 && lane == 0) free_ok = tma_mbar_wait(empty_bar(st), (use - 1) & 1, wait_lim, status, abort_flag);
+          if constexpr (SP) free_ok = __shfl_sync(0xffffffffu, free_ok, 0);
+          if (!free_ok) {
             stop = true;
             break;
           }
@@ -329,28 +346,67 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           const int off = static_cast<int>(r & 3);
           int nn = (off + cnt + 3) & ~3;
           if (r - off + nn > total_recs) nn = (off + cnt) & ~3;
-          nb_count[st] = max(0, nn - off);
-          nb_off[st] = off;
-          uint32_t bytes = cnt * (KW + VW) * 4 + 2 * nn * 4;
-          if (KF == KFMT_PROD) bytes += cnt * KSW * 4 + nn * 4;
           const uint32_t fb = full_bar(st);
-          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
           const uint32_t sb = stage_addr(st);
-          bulk_g2s(sb + SL.kcodes, p.kcodes + r * KW, cnt * KW * 4, fb);
-          bulk_g2s(sb + SL.vcodes, p.vcodes + r * VW, cnt * VW * 4, fb);
-          if (nn > 0) {
-            bulk_g2s(sb + SL.knorm, p.knorms + (r - off), nn * 4, fb);
-            bulk_g2s(sb + SL.vnorm, p.vnorms + (r - off), nn * 4, fb);
+          // spectral: the records' bytes [b0, b1) go from the 16-byte boundary below b0 by bulk
+          // copy up to the last 16-byte boundary inside the array; the few words past it
+          // (the array's last records) are copied by the warp's lanes
+          uint32_t sp_bytes = 0u;
+          int64_t ka0 = 0, kbe = 0, va0 = 0, vbe = 0;
+          if constexpr (SP) {
+            const int64_t kb0 = r * KW * 4, kb1 = (r + cnt) * KW * 4, kend = total_recs * KW * 4;
+            const int64_t vb0 = r * VW * 4, vb1 = (r + cnt) * VW * 4, vend = total_recs * VW * 4;
+            ka0 = kb0 & ~15ll;
+            kbe = min((kb1 + 15) & ~15ll, kend & ~15ll);
+            va0 = vb0 & ~15ll;
+            vbe = min((vb1 + 15) & ~15ll, vend & ~15ll);
+            sp_bytes = static_cast<uint32_t>((kbe - ka0) + (vbe - va0));
+            const unsigned char* kg = reinterpret_cast<const unsigned char*>(p.kcodes);
+            const unsigned char* vg = reinterpret_cast<const unsigned char*>(p.vcodes);
+            for (int64_t b = kbe + 4 * lane; b < kb1; b += 128)
+              *reinterpret_cast<uint32_t*>(gen(sb + SL.kcodes + static_cast<uint32_t>(b - ka0))) =
+                  __ldg(reinterpret_cast<const uint32_t*>(kg + b));
+            for (int64_t b = vbe + 4 * lane; b < vb1; b += 128)
+              *reinterpret_cast<uint32_t*>(gen(sb + SL.vcodes + static_cast<uint32_t>(b - va0))) =
+                  __ldg(reinterpret_cast<const uint32_t*>(vg + b));
+            __syncwarp();
           }
-          if (KF == KFMT_PROD) {
-            bulk_g2s(sb + SL.ksign, p.ksigns + r * KSW, cnt * KSW * 4, fb);
-            if (nn > 0) bulk_g2s(sb + SL.krn, p.krnorms + (r - off), nn * 4, fb);
+          if (lane == 0) {
+            nb_count[st] = max(0, nn - off);
+            nb_off[st] = off;
+            uint32_t bytes = SP ? sp_bytes : cnt * (KW + VW) * 4 + 2 * nn * 4;
+            if (KF == KFMT_PROD) bytes += cnt * KSW * 4 + nn * 4;
+            if (SP && p.krnorms) bytes += nn * 4;
+            // the arrival releases the word copies above (spectral) and expects the bulk bytes
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
+            if (!SP) {
+              bulk_g2s(sb + SL.kcodes, p.kcodes + r * KW, cnt * KW * 4, fb);
+              bulk_g2s(sb + SL.vcodes, p.vcodes + r * VW, cnt * VW * 4, fb);
+              if (nn > 0) {
+                bulk_g2s(sb + SL.knorm, p.knorms + (r - off), nn * 4, fb);
+                bulk_g2s(sb + SL.vnorm, p.vnorms + (r - off), nn * 4, fb);
+              }
+            }
+            if (SP) {
+              if (kbe > ka0)
+                bulk_g2s(sb + SL.kcodes, reinterpret_cast<const unsigned char*>(p.kcodes) + ka0,
+                         static_cast<uint32_t>(kbe - ka0), fb);
+              if (vbe > va0)
+                bulk_g2s(sb + SL.vcodes, reinterpret_cast<const unsigned char*>(p.vcodes) + va0,
+                         static_cast<uint32_t>(vbe - va0), fb);
+            }
+            if (SP && p.krnorms && nn > 0) bulk_g2s(sb + SL.krn, p.krnorms + (r - off), nn * 4, fb);
+            if (KF == KFMT_PROD) {
+              bulk_g2s(sb + SL.ksign, p.ksigns + r * KSW, cnt * KSW * 4, fb);
+              if (nn > 0) bulk_g2s(sb + SL.krn, p.krnorms + (r - off), nn * 4, fb);
+            }
           }
         }
       }
       // drain: the copies this CTA issued land before it may exit
-      for (int j = max(0, gs - NS); j < gs; ++j)
-        for (long long i = 0; !tma_mbar_try(full_bar(j % NS), (j / NS) & 1) && i < (1ll << 28); ++i) {}
+      if (lane == 0)
+        for (int j = max(0, gs - NS); j < gs; ++j)
+          for (long long i = 0; !tma_mbar_try(full_bar(j % NS), (j / NS) & 1) && i < (1ll << 28); ++i) {}
     }
     return;
   }
@@ -366,6 +422,36 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   const bool qlo = PK && g >= 4;                  // B column g carries a lo part
   const int h0 = PK ? 2 * (t & 1) : 2 * t;         // heads of accumulator columns 2t, 2t + 1
   const bool plo = PK && t >= 2;                  // accumulator columns 2t, 2t + 1 are lo parts
+  // spectral head words: this lane scores top dims 2t, 2t + 1 and QJL signs 2t, 2t + 1 of its
+  // key rows, and carries top value dim g (bit position, width, codebook offset; 0 = none)
+  int kh_pos[2] = {0, 0}, kh_nb[2] = {0, 0}, kh_off[2] = {0, 0}, ks_pos[2] = {0, 0};
+  bool ks_ok[2] = {false, false};
+  int vh_pos = 0, vh_nb = 0, vh_off = 0;
+  if constexpr (SP) {
+    // static indices only (a dynamically indexed array would live in local memory)
+    int acc = 0;
+#pragma unroll
+    for (int j = 0; j < TQ_MAX_TOP; ++j) {
+      const int b = j < p.k_top_k ? p.k_top_bits[j] : 0;
+      if (j == 2 * t) { kh_pos[0] = acc; kh_nb[0] = b; }
+      if (j == 2 * t + 1) { kh_pos[1] = acc; kh_nb[1] = b; }
+      acc += b;
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      kh_off[i] = kh_nb[i] ? unit_c_off(kh_nb[i]) : 0;
+      ks_pos[i] = acc + 2 * t + i;
+      ks_ok[i] = p.k_qjl && 2 * t + i < p.k_top_k;
+    }
+    acc = 0;
+#pragma unroll
+    for (int j = 0; j < TQ_MAX_TOP; ++j) {
+      const int b = j < p.v_top ? p.v_top_bits[j] : 0;
+      if (j == g) { vh_pos = acc; vh_nb = b; }
+      acc += b;
+    }
+    vh_off = vh_nb ? unit_c_off(vh_nb) : 0;
+  }
   int gs = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     int bh, hblk, chunk, k0, k1;
@@ -419,17 +505,33 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         }
       }
     }
+    // spectral head slots (B of the head MMA): slots 2t, 2t + 1 (top dims) and 2t + 8, 2t + 9
+    // (QJL) of column g
+    uint32_t qhb[2] = {0u, 0u};
+    if constexpr (SP) {
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+      if (hok) {
+        const float* qr = p.qb + (qbase + qcol) * p.qb_stride;
+        a[0] = qr[2 * t]; a[1] = qr[2 * t + 1]; a[2] = qr[2 * t + 8]; a[3] = qr[2 * t + 9];
+      }
+      uint32_t h01, l01, h23, l23;
+      split_pair(a[0], a[1], h01, l01);
+      split_pair(a[2], a[3], h23, l23);
+      qhb[0] = (PK && qlo) ? l01 : h01;
+      qhb[1] = (PK && qlo) ? l23 : h23;
+    }
     // this thread's score columns are heads h0, h0 + 1 of the block
     const bool c0ok = h0 < nh, c1ok = h0 + 1 < nh;
     const float sa0 = c0ok ? p.qs[(qbase + h0) * 2] * p.k_scale : 0.f;
     const float sa1 = c1ok ? p.qs[(qbase + h0 + 1) * 2] * p.k_scale : 0.f;
-    const float sb0 = c0ok ? p.qs[(qbase + h0) * 2 + 1] * p.qjl_coef : 0.f;
-    const float sb1 = c1ok ? p.qs[(qbase + h0 + 1) * 2 + 1] * p.qjl_coef : 0.f;
+    const float sb0 = c0ok ? p.qs[(qbase + h0) * 2 + 1] * (SP ? 1.f : p.qjl_coef) : 0.f;
+    const float sb1 = c1ok ? p.qs[(qbase + h0 + 1) * 2 + 1] * (SP ? 1.f : p.qjl_coef) : 0.f;
 
     float o[MT][4];
 #pragma unroll
     for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads h0, h0 + 1
+    float oh[4] = {0.f, 0.f, 0.f, 0.f};   // spectral: top value dim g (columns 2t, 2t + 1)
 
     for (int t0 = k0; t0 < k1; t0 += kTmaStageTokens, ++gs) {
       const int st = gs % NS;
@@ -438,12 +540,16 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       const int cnt = min(kTmaStageTokens, k1 - t0);
       const int nn = static_cast<int>(sld32(nb_a + 4u * st)), noff = static_cast<int>(sld32(nb_a + 4u * (NS + st)));
       const int w0 = warp * 16 * U;                  // first token of this warp (stage-local)
+      // spectral code arrays start at the 16-byte boundary below the stage's first record
+      const uint32_t kcb = sb + SL.kcodes + (SP ? static_cast<uint32_t>(((rec0 + t0) * KW * 4) & 15) : 0u);
+      const uint32_t vcb = sb + SL.vcodes + (SP ? static_cast<uint32_t>(((rec0 + t0) * VW * 4) & 15) : 0u);
       // ---- pull this warp's slices out of the stage ----
       bool ok[U][2];
       uint32_t ks[U][2][NWK];
       float kn[U][2], vn[U][2], gm[U][2];
       uint32_t sw[U][2];
       uint32_t vs[U][4][NWV];
+      uint32_t hk[U][2], hv[U][4];                   // spectral head words (keys by row, values by k-index)
       if (cnt == kTmaStageTokens && nn >= cnt) {
         // a whole stage with every norm staged (all but the last stage of a chunk): no
         // per-token checks
@@ -453,19 +559,25 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           for (int h = 0; h < 2; ++h) {
             const int tk = w0 + 16 * u + 8 * h + pg;     // token of score row g + 8 h
             ok[u][h] = true;
-            sld_slice<NWK>(sb + SL.kcodes + tk * KW * 4, KW, t * TDK * KB, true, ks[u][h]);
-            kn[u][h] = sldf(sb + SL.knorm + 4 * (noff + tk));
-            vn[u][h] = sldf(sb + SL.vnorm + 4 * (noff + tk));
+            sld_slice<NWK>(kcb + tk * KW * 4, KW, TOFF + t * TDK * KB, true, ks[u][h]);
+            kn[u][h] = SP ? 1.f : sldf(sb + SL.knorm + 4 * (noff + tk));
+            vn[u][h] = SP ? 1.f : sldf(sb + SL.vnorm + 4 * (noff + tk));
             gm[u][h] = 0.f;
             sw[u][h] = 0u;
+            if constexpr (SP) {
+              hk[u][h] = sld32(kcb + tk * KW * 4);
+              if (p.k_qjl) gm[u][h] = sldf(sb + SL.krn + 4 * (noff + tk));
+            }
             if constexpr (KF == KFMT_PROD) {
               gm[u][h] = sldf(sb + SL.krn + 4 * (noff + tk));
               sw[u][h] = sld32(sb + SL.ksign + (tk * KSW + t) * 4);
             }
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            sld_slice<NWV>(sb + SL.vcodes + (w0 + 16 * u + kv[i]) * VW * 4, VW, g * TDV * VB, true, vs[u][i]);
+          for (int i = 0; i < 4; ++i) {
+            sld_slice<NWV>(vcb + (w0 + 16 * u + kv[i]) * VW * 4, VW, TOFF + g * TDV * VB, true, vs[u][i]);
+            if constexpr (SP) hv[u][i] = sld32(vcb + (w0 + 16 * u + kv[i]) * VW * 4);
+          }
         }
       } else {
         auto norm_of = [&](uint32_t staged, const float* global, int lk, bool okk) {
@@ -478,11 +590,15 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             const int tk = w0 + 16 * u + 8 * h + pg;
             const bool okk = tk < cnt;
             ok[u][h] = okk;
-            sld_slice<NWK>(sb + SL.kcodes + tk * KW * 4, KW, t * TDK * KB, okk, ks[u][h]);
-            kn[u][h] = norm_of(sb + SL.knorm, p.knorms, tk, okk);
-            vn[u][h] = norm_of(sb + SL.vnorm, p.vnorms, tk, okk);
+            sld_slice<NWK>(kcb + tk * KW * 4, KW, TOFF + t * TDK * KB, okk, ks[u][h]);
+            kn[u][h] = SP ? 1.f : norm_of(sb + SL.knorm, p.knorms, tk, okk);
+            vn[u][h] = SP ? 1.f : norm_of(sb + SL.vnorm, p.vnorms, tk, okk);
             gm[u][h] = 0.f;
             sw[u][h] = 0u;
+            if constexpr (SP) {
+              hk[u][h] = okk ? sld32(kcb + tk * KW * 4) : 0u;
+              if (p.k_qjl) gm[u][h] = norm_of(sb + SL.krn, p.krnorms, tk, okk);
+            }
             if constexpr (KF == KFMT_PROD) {
               gm[u][h] = norm_of(sb + SL.krn, p.krnorms, tk, okk);
               sw[u][h] = okk ? sld32(sb + SL.ksign + (tk * KSW + t) * 4) : 0u;
@@ -491,7 +607,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int lk = w0 + 16 * u + kv[i];
-            sld_slice<NWV>(sb + SL.vcodes + lk * VW * 4, VW, g * TDV * VB, lk < cnt, vs[u][i]);
+            sld_slice<NWV>(vcb + lk * VW * 4, VW, TOFF + g * TDV * VB, lk < cnt, vs[u][i]);
+            if constexpr (SP) hv[u][i] = lk < cnt ? sld32(vcb + lk * VW * 4) : 0u;
           }
         }
       }
@@ -543,12 +660,33 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             mma16816(acc2, a0, a1, a2, a3, qb[k][0], qb[k][1]);
           }
         }
+        if constexpr (SP) {
+          // head slots of the spectral keys, one extra k-step: slots 2t, 2t+1 hold the top-dim
+          // codebook values, slots 2t+8, 2t+9 the QJL signs times gamma (split hi + lo)
+          float hvv[2][4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t w = hk[u][h];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              hvv[h][i] = kh_nb[i] ? utab[kh_off[i] + ((w >> kh_pos[i]) & ((1u << kh_nb[i]) - 1u))] : 0.f;
+              hvv[h][2 + i] = ks_ok[i] ? (((w >> ks_pos[i]) & 1u) ? gm[u][h] : -gm[u][h]) : 0.f;
+            }
+          }
+          uint32_t ah[4], al[4];
+          split_pair(hvv[0][0], hvv[0][1], ah[0], al[0]);
+          split_pair(hvv[1][0], hvv[1][1], ah[1], al[1]);
+          split_pair(hvv[0][2], hvv[0][3], ah[2], al[2]);
+          split_pair(hvv[1][2], hvv[1][3], ah[3], al[3]);
+          mma16816(acc2, ah[0], ah[1], ah[2], ah[3], qhb[0], qhb[1]);
+          mma16816(acc2, al[0], al[1], al[2], al[3], qhb[0], qhb[1]);
+        }
         if constexpr (PK) {
           // columns c and c + 4 hold the hi and lo products of one head: lanes t and t ^ 2
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
-            if constexpr (KF == KFMT_PROD) acc2[i] += __shfl_xor_sync(0xffffffffu, acc2[i], 2);
+            if constexpr (KF == KFMT_PROD || SP) acc2[i] += __shfl_xor_sync(0xffffffffu, acc2[i], 2);
           }
         }
         // acc[0], acc[1]: token row g, heads h0, h0 + 1; acc[2], acc[3]: token row g + 8
@@ -557,6 +695,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         for (int i = 0; i < 4; ++i) {
           float v = sa[i] * acc[i];
           if constexpr (KF == KFMT_PROD) v += gm[u][i >> 1] * sbq[i] * acc2[i];
+          if constexpr (SP) v += sbq[i] * acc2[i];
           sc[u][i] = ok[u][i >> 1] ? kn[u][i >> 1] * v : -INFINITY;
         }
       }
@@ -584,6 +723,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           l1 *= f1;
 #pragma unroll
           for (int i = 0; i < MT; ++i) { o[i][0] *= f0; o[i][2] *= f0; o[i][1] *= f1; o[i][3] *= f1; }
+          if constexpr (SP) { oh[0] *= f0; oh[1] *= f1; }
           m0 = mn0;
           m1 = mn1;
         }
@@ -605,6 +745,26 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         } else {
           b0h = movmatrix_t(pth); b1h = movmatrix_t(pbh);
           b0l = movmatrix_t(ptl); b1l = movmatrix_t(pbl);
+        }
+        if constexpr (SP) {
+          // top value dims: an extra M-tile whose row g is top dim g (rows g + 8 unused), k =
+          // the unit's tokens; values in the units of the table entries (c / v_scale)
+          float tv4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            tv4[i] = vh_nb ? utab[vh_off + ((hv[u][i] >> vh_pos) & ((1u << vh_nb) - 1u))] / p.v_scale : 0.f;
+          uint32_t vh0, vl0, vh2, vl2;
+          split_pair(tv4[0], tv4[1], vh0, vl0);
+          split_pair(tv4[2], tv4[3], vh2, vl2);
+          float ohx[4] = {oh[0], oh[1], 0.f, 0.f};
+          mma16816(ohx, vh0, 0u, vh2, 0u, b0h, b1h);
+          mma16816(ohx, vl0, 0u, vl2, 0u, b0h, b1h);
+          if constexpr (!PK) {
+            mma16816(ohx, vh0, 0u, vh2, 0u, b0l, b1l);
+            mma16816(ohx, vl0, 0u, vl2, 0u, b0l, b1l);
+          }
+          oh[0] = ohx[0];
+          oh[1] = ohx[1];
         }
         // ---- O'^T[128 dims x 8 columns] += V_hat^T . P^T ----
         // M-tile i: row g = dim TDV g + i (first word of the slice), row g + 8 = dim TDV g + 8 + i
@@ -671,6 +831,18 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = o[i][1];
         wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][2];
         wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][3];
+      }
+    }
+    if constexpr (SP) {
+      // the top value dims come from the head M-tile, not from the (zero) tail codes
+      if constexpr (PK) {
+        oh[0] += __shfl_xor_sync(0xffffffffu, oh[0], 2);
+        oh[1] += __shfl_xor_sync(0xffffffffu, oh[1], 2);
+      }
+      __syncwarp();
+      if ((!PK || t < 2) && vh_nb) {
+        wm[(2 * t) * (D + 2) + 2 + g] = oh[0];
+        wm[(2 * t + 1) * (D + 2) + 2 + g] = oh[1];
       }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");

@@ -20,6 +20,7 @@ cudaError_t launch_decode_mse(const DecodeParams& p, int kb, int vb, dim3 grid, 
 cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s,
                                int* status, long long lim);
 cudaError_t launch_decode_spec(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
+cudaError_t launch_decode_spec_tma(const DecodeParams& p, dim3 grid, cudaStream_t s, int* status, long long lim);
 
 // Tensor-core quantize (d = 128, 16-bit input, MSE bits 1..4).
 cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& p, int bits, int grid,

@@ -296,17 +296,24 @@ struct DecodePlan {
   size_t off_qa, off_qb, off_qs, off_ml, off_o, bytes;
 };
 
+// Spectral records the bulk-copy staged decode kernel reads: 1-bit tails and one head word.
+bool spectral_tma(const tq_quantizer* q) {
+  return q->kind == TQ_KIND_SPECTRAL && q->tail_bits == 1 && q->k_top <= TQ_MAX_TOP &&
+         spectral_head_bits(q) <= 32;
+}
+
 DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t Nmax) {
   DecodePlan P{};
   const int D = kq->d;
   const int64_t units = static_cast<int64_t>(B) * Hkv;
   const int64_t sms = sm_count();
   int64_t nch, cl;
-  if (kq->kind != TQ_KIND_SPECTRAL) {
+  if (kq->kind != TQ_KIND_SPECTRAL || spectral_tma(kq)) {
     // persistent bulk-copy kernel: about 16 work items per SM, chunks of whole 112-token
     // stages, and (when the shape allows) an item count that is a multiple of the SMs;
     // a work item covers one block of up to 8 query heads of a GQA group
-    const int64_t stage = tma_stage_tokens(kq->kind == TQ_KIND_PROD ? KFMT_PROD : KFMT_MSE, Hq / Hkv <= 4);
+    const int kf = kq->kind == TQ_KIND_PROD ? KFMT_PROD : (kq->kind == TQ_KIND_SPECTRAL ? KFMT_SPEC : KFMT_MSE);
+    const int64_t stage = tma_stage_tokens(kf, Hq / Hkv <= 4);
     const int64_t wu = units * tma_head_blocks(Hq / Hkv);
     int64_t n0 = std::max<int64_t>(1, (16 * sms + wu - 1) / wu);
     for (int64_t cand = n0; cand < n0 + 8 && cand <= Nmax; ++cand)
@@ -650,10 +657,17 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   dp.v_scale = vq->lut_scale > 0.f ? vq->lut_scale : 1.f;
   dp.part_ml = pml; dp.part_o = po;
   const int64_t items = static_cast<int64_t>(B) * Hkv * tma_head_blocks(G) * P.n_chunks;
-  const dim3 grid = kfmt == KFMT_SPEC ? dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv))
-                                      : dim3(static_cast<unsigned>(std::min<int64_t>(items, sm_count())));
+  const bool spec_tma = kfmt == KFMT_SPEC && spectral_tma(kq);   // the plan follows the keys
+  if (spec_tma && !spectral_tma(vq))
+    return fail(TQ_ERR_UNSUPPORTED, "spectral values need a head of at most 32 bits with 1-bit-tail keys");
+  const dim3 grid = (kfmt == KFMT_SPEC && !spec_tma)
+                        ? dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv))
+                        : dim3(static_cast<unsigned>(std::min<int64_t>(items, sm_count())));
   const size_t smem = decode_smem_bytes(D, kb, vb);
-  e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream, device_status_ptr(), wait_limit());
+  if (spec_tma)
+    e = launch_decode_spec_tma(dp, grid, stream, device_status_ptr(), wait_limit());
+  else
+    e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream, device_status_ptr(), wait_limit());
   if (e == cudaErrorNotSupported) return fail(TQ_ERR_UNSUPPORTED, "decode variant not built (kbits %d, vbits %d)", kb, vb);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
 
