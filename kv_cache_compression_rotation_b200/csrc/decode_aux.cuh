@@ -130,7 +130,7 @@ __device__ __forceinline__ void matvec8x128(const float* __restrict__ M, const f
   }
 }
 
-// qprep_kernel for MSE and PROD keys with d = 128 (same outputs).
+// qprep_kernel with d = 128 (same outputs, every key kind).
 __global__ void __launch_bounds__(256) qprep128_kernel(QPrepParams p) {
   __shared__ __align__(16) float xs[8 * 128], ys[8 * 128], us[8 * 128];
   const int r0 = blockIdx.x * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,6 +148,35 @@ __global__ void __launch_bounds__(256) qprep128_kernel(QPrepParams p) {
   }
   const int r = r0 + warp;                         // warp w normalizes row w
   if (r >= p.rows) return;
+  if (p.kind == TQ_KIND_SPECTRAL) {
+    // qa: sigma_j q'_j on the tail dims (0 on the top dims); qb slots 0..7: sigma_j q'_j of
+    // the top dims, slots 8..15: coef * (S q'_top)_i (QJL)
+    const float* y = ys + warp * 128;
+    float a4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = 4 * lane + i;
+      a4[i] = j < p.k_top ? 0.f : y[j] * __ldg(p.dim_sigma + j);
+    }
+    float ma = fmaxf(fmaxf(fabsf(a4[0]), fabsf(a4[1])), fmaxf(fabsf(a4[2]), fabsf(a4[3])));
+    ma = warp_max(ma);
+    const float sa = ma > 0.f ? ma : 1.f;
+    reinterpret_cast<float4*>(p.qa + static_cast<int64_t>(r) * 128)[lane] =
+        make_float4(a4[0] / sa, a4[1] / sa, a4[2] / sa, a4[3] / sa);
+    float bv = 0.f;                                 // lane i < 16: slot i
+    if (lane < p.k_top) bv = y[lane] * __ldg(p.dim_sigma + lane);
+    else if (lane >= 8 && lane < 8 + p.k_top && p.qjl) {
+      const int ii = lane - 8;
+      for (int k = 0; k < p.k_top; ++k) bv = fmaf(__ldg(p.S + ii * p.k_top + k), y[k], bv);
+      bv *= p.spec_coef;
+    }
+    if (lane >= 16) bv = 0.f;
+    float mb = warp_max(fabsf(bv));
+    const float sb = mb > 0.f ? mb : 1.f;
+    if (lane < p.qb_stride) p.qb[static_cast<int64_t>(r) * p.qb_stride + lane] = bv / sb;
+    if (lane == 0) { p.qs[r * 2] = sa; p.qs[r * 2 + 1] = sb; }
+    return;
+  }
   const float4 a = *reinterpret_cast<const float4*>(ys + warp * 128 + 4 * lane);
   float ma = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
   ma = warp_max(ma);

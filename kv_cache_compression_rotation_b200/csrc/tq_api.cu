@@ -612,7 +612,7 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   qp.spec_coef = static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, kq->k_top));
   qp.qa = qa; qp.qb = qb; qp.qs = qs; qp.qb_stride = P.qb_stride;
   const size_t qsm = static_cast<size_t>(2 * D + std::max(D, P.qb_stride)) * 4;
-  if (kq->kind != TQ_KIND_SPECTRAL && D == 128)
+  if (D == 128 && (kq->kind != TQ_KIND_SPECTRAL || kq->k_top <= 8))
     qprep128_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(qp);
   else
     qprep_kernel<<<rows, 128, qsm, stream>>>(qp);
