@@ -309,13 +309,17 @@ DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t N
   const int64_t sms = sm_count();
   int64_t nch, cl;
   if (kq->kind != TQ_KIND_SPECTRAL || spectral_tma(kq)) {
-    // persistent bulk-copy kernel: about 16 work items per SM, chunks of whole 112-token
-    // stages, and (when the shape allows) an item count that is a multiple of the SMs;
-    // a work item covers one block of up to 8 query heads of a GQA group
+    // persistent bulk-copy kernel: chunks of whole stages and (when the shape allows) an
+    // item count that is a multiple of the SMs; a work item covers one GQA group of up to
+    // 4 heads (packed columns) or one block of up to 8 heads
     const int kf = kq->kind == TQ_KIND_PROD ? KFMT_PROD : (kq->kind == TQ_KIND_SPECTRAL ? KFMT_SPEC : KFMT_MSE);
     const int64_t stage = tma_stage_tokens(kf, Hq / Hkv <= 4);
     const int64_t wu = units * tma_head_blocks(Hq / Hkv);
-    int64_t n0 = std::max<int64_t>(1, (16 * sms + wu - 1) / wu);
+    // at most ~16 items per SM, and items of at least ~4 stages when the context is short
+    // (each item ends in a cross-warp merge and writes one partial per head)
+    const int64_t stages_total = wu * ((Nmax + stage - 1) / stage);
+    const int64_t want = std::max<int64_t>(sms, std::min<int64_t>(16 * sms, stages_total / 4));
+    int64_t n0 = std::max<int64_t>(1, (want + wu - 1) / wu);
     for (int64_t cand = n0; cand < n0 + 8 && cand <= Nmax; ++cand)
       if ((wu * cand) % sms == 0) { n0 = cand; break; }
     cl = (Nmax + n0 - 1) / n0;
