@@ -198,14 +198,16 @@ __global__ void __launch_bounds__(256) qprep128_kernel(QPrepParams p) {
   if (lane == 0) { p.qs[r * 2] = sa; p.qs[r * 2 + 1] = sb; }
 }
 
-// combine_kernel with d = 128: 8 rows per CTA; dynamic shared memory holds the chunk
-// weights 2^(m_c - M) / L of the 8 rows ([8][n_chunks] floats).
+// combine_kernel with d = 128: 2 rows per CTA of 256 threads (many CTAs: the step is a
+// few microseconds of dependent loads); dynamic shared memory holds the chunk weights
+// 2^(m_c - M) / L of the 2 rows ([2][n_chunks] floats).
 __global__ void __launch_bounds__(256) combine128_kernel(CombineParams p) {
+  constexpr int R = 2;
   extern __shared__ __align__(16) float cw[];
-  __shared__ __align__(16) float ov[128 * 8];     // o' transposed: [j][row]
-  const int r0 = blockIdx.x * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ __align__(16) float ov[R * 128];      // o' per row
+  const int r0 = blockIdx.x * R, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nch = p.n_chunks;
-  {
+  if (warp < R) {
     float* w = cw + warp * nch;
     const int r = r0 + warp;
     if (r < p.rows) {
@@ -228,39 +230,24 @@ __global__ void __launch_bounds__(256) combine128_kernel(CombineParams p) {
     }
   }
   __syncthreads();
+  const int rr = tid >> 7, k = tid & 127;           // thread: row rr, dim k
+  const int r = r0 + rr;
   {
-    const int r = r0 + warp;                       // thread: row warp, dims 4 lane .. 4 lane + 3
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    float a = 0.f;
     if (r < p.rows) {
-      const float* w = cw + warp * nch;
-      const float4* po = reinterpret_cast<const float4*>(p.part_o + static_cast<int64_t>(r) * nch * 128) + lane;
-      for (int c = 0; c < nch; ++c) {
-        const float wc = w[c];
-        const float4 x = __ldg(po + c * 32);
-        a.x = fmaf(wc, x.x, a.x); a.y = fmaf(wc, x.y, a.y); a.z = fmaf(wc, x.z, a.z); a.w = fmaf(wc, x.w, a.w);
-      }
-      if (p.v_sigma) {
-        a.x *= p.v_sigma[4 * lane]; a.y *= p.v_sigma[4 * lane + 1];
-        a.z *= p.v_sigma[4 * lane + 2]; a.w *= p.v_sigma[4 * lane + 3];
-      }
+      const float* w = cw + rr * nch;
+      const float* po = p.part_o + static_cast<int64_t>(r) * nch * 128 + k;
+#pragma unroll 4
+      for (int c = 0; c < nch; ++c) a = fmaf(w[c], __ldg(po + c * 128), a);
+      if (p.v_sigma) a *= p.v_sigma[k];
     }
-    ov[(4 * lane) * 8 + warp] = a.x;
-    ov[(4 * lane + 1) * 8 + warp] = a.y;
-    ov[(4 * lane + 2) * 8 + warp] = a.z;
-    ov[(4 * lane + 3) * 8 + warp] = a.w;
+    ov[rr * 128 + k] = a;
   }
   __syncthreads();
-  const int k = tid & 127, rb = (tid >> 7) * 4;    // thread: output dim k of rows rb .. rb + 3
-  float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-  for (int j = 0; j < 128; ++j) {
-    const float m = __ldg(p.rot_v + j * 128 + k);
-    const float4 o = *reinterpret_cast<const float4*>(ov + j * 8 + rb);
-    o0 = fmaf(o.x, m, o0); o1 = fmaf(o.y, m, o1); o2 = fmaf(o.z, m, o2); o3 = fmaf(o.w, m, o3);
-  }
-  const float res[4] = {o0, o1, o2, o3};
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (r0 + rb + i < p.rows) p.out[static_cast<int64_t>(r0 + rb + i) * 128 + k] = res[i];
+  float o = 0.f;
+#pragma unroll 8
+  for (int j = 0; j < 128; ++j) o = fmaf(ov[rr * 128 + j], __ldg(p.rot_v + j * 128 + k), o);
+  if (r < p.rows) p.out[static_cast<int64_t>(r) * 128 + k] = o;
 }
 
 }  // namespace tq
