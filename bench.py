@@ -195,7 +195,8 @@ def run_tq(args, rank, world, local_rank):
     torch.backends.cuda.matmul.allow_tf32 = False
     seed_off = rank_seed_offset(rank)
     nvec, q_bytes, dec_bytes = algorithmic_bytes()
-    rot = ti.haar_rotation(D, ti.SEEDS["rotation"] + 3)
+    rot = (ti.hadamard_rotation(D, ti.SEEDS["rotation"] + 3) if args.rotation == "hadamard"
+           else ti.haar_rotation(D, ti.SEEDS["rotation"] + 3))
     U = ti.haar_rotation(D, ti.SEEDS["basis"] + 3)
     kq = K.Quantizer.mse(rot, BITS, device=dev)
     vq = K.Quantizer.mse(rot, BITS, device=dev)
@@ -309,7 +310,8 @@ def run_tq(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "decode-128k: B=8, Hkv=8, Hq=32 (GQA 4), d=128, context 131072, "
-                               "TurboQuant-mse b=4 keys+values, bf16 K/V anisotropic (80% variance in 4 dims)",
+                               "TurboQuant-mse b=4 keys+values, bf16 K/V anisotropic (80% variance in 4 dims)"
+                               + (", randomized Hadamard rotation" if args.rotation == "hadamard" else ""),
                    "global_batch": B * world, "seq_len": N, "parallelism": f"dp{world}",
                    "l2": "inputs (4.3 GB/step) larger than L2; no flush"},
         "parts": {
@@ -533,6 +535,8 @@ def main():
     ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5"],
                     help="c3 (default): the 128k decode step of the headline; the others are the scope "
                          "table's secondary workloads, timed per kernel")
+    ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
+                    help="rotation of the c3 workload: dense Haar (the headline) or randomized Hadamard")
     ap.add_argument("--c5-queries", type=int, default=100)
     ap.add_argument("--c5-db", type=int, default=1000000)
     ap.add_argument("--c5-bits", type=int, default=2)

@@ -99,6 +99,12 @@ typedef struct {
   float lut_scale;              /* decode/score: shared scale s of the half-precision codebook
                                    table (entries c_k / s); 0 means 1.  tq_lut_scale picks one
                                    that keeps every entry within ~1e-4 of c_k. */
+  int32_t rot_pm1;              /* non-zero: every entry of rot is +1/sqrt(d) or -1/sqrt(d) in
+                                   fp32 (a randomized Hadamard rotation H diag(s) / sqrt(d), the
+                                   launch kit's O(d log d) rotation mode).  The tensor-core
+                                   quantize then multiplies by the exact +-1 matrix in one pass and
+                                   rescales; an entry of another magnitude makes it report
+                                   TQ_ERR_INVALID_ARG through tq_get_status. */
 } tq_quantizer;
 
 /*

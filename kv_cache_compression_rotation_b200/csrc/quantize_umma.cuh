@@ -66,6 +66,9 @@ struct UmmaQuantParams {
   const float* unit_t;
   const float* S;          // [k_top*k_top] (qjl)
   float* rnorms;           // [n] (qjl)
+  // rotations with entries +-pm1_scale: one exact +-1 MMA operand, no low-order term
+  int pm1;
+  float pm1_scale;         // 1/sqrt(d) as fp32
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -217,7 +220,12 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   // Pi_hi / Pi_lo in the swizzled K-major layout: row = output dim n, k = input dim.
   for (int i = tid; i < kUmmaD * kUmmaD; i += kUmmaThreads) {
     const int nrow = i >> 7, k = i & 127;
-    const float v = __ldg(p.rot + i);
+    float v = __ldg(p.rot + i);
+    if (p.pm1) {
+      // the +-1 pattern is exact in both 16-bit types; the scale is applied to the norm
+      if (fabsf(v) != p.pm1_scale) report_status(p.status, TQ_ERR_INVALID_ARG);
+      v = v < 0.f ? -1.f : 1.f;
+    }
     uint16_t hi, lo, lo2;
     if (p.is_f16) {
       const __half h = __float2half_rn(v);
@@ -302,7 +310,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           const uint32_t koff = (kk >> 2) * (kXStageBytes / 2) + (kk & 3) * 32;
           const uint32_t poff = (kk >> 2) * (kPiBytes / 2) + (kk & 3) * 32;
           umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_hi + poff), idesc, kk > 0 ? 1u : 0u);
-          umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo + poff), idesc, 1u);
+          if (!p.pm1) umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo + poff), idesc, 1u);
           if (NT == 3) umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo2 + poff), idesc, 1u);
         }
         umma_commit(empty_bar(s));
@@ -424,8 +432,9 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           ss[(i + 2) & 3] = fmaf(vb[i], vb[i], ss[(i + 2) & 3]);
         }
       }
-      const float nu = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
-      const float inv = nu > 0.f ? 1.f / nu : 1.f;     // a zero row keeps u = 0
+      const float ny = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
+      const float nu = p.pm1 ? ny * p.pm1_scale : ny;  // ||x|| (the +-1 product is sqrt(d) Pi x)
+      const float inv = ny > 0.f ? 1.f / ny : 1.f;     // a zero row keeps u = 0
       uint32_t* dst = p.codes + v * W;
       // pass 2: codes of 32 coordinates at a time, B packed words per chunk
       if (use_cells) {
@@ -452,7 +461,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           if (v < p.n) store_words<B>(dst + c * B, wc);
         }
       } else {
-        const float nthr = nu > 0.f ? nu : 1.f;
+        const float nthr = ny > 0.f ? ny : 1.f;
 #pragma unroll
         for (int k = 0; k < NB; ++k) thr[k] = nthr * tsm[k];
 #pragma unroll 1

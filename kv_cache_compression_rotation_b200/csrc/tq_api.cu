@@ -242,6 +242,8 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
     p.norms = out.norms;
     p.status = status;
     p.wait_limit = wait_limit();
+    p.pm1 = q->kind == TQ_KIND_MSE && q->rot_pm1 != 0;
+    p.pm1_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(q->d)));
     if (q->kind == TQ_KIND_SPECTRAL) {
       p.k_top = q->k_top; p.qjl = q->qjl;
       for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];

@@ -48,7 +48,7 @@ class Quantizer_t(C.Structure):
         ("k_top", C.c_int32), ("tail_bits", C.c_int32), ("qjl", C.c_int32),
         ("top_bits", C.c_int32 * MAX_TOP),
         ("dim_sigma", C.c_void_p), ("unit_centroids", C.c_void_p), ("unit_boundaries", C.c_void_p),
-        ("lut_scale", C.c_float),
+        ("lut_scale", C.c_float), ("rot_pm1", C.c_int32),
     ]
 
 
@@ -195,7 +195,7 @@ class Quantizer:
 
     def __init__(self, kind: int, d: int, rot, *, bits=0, m=0, S=None, centroids=None, boundaries=None,
                  k_top=0, tail_bits=0, qjl=0, top_bits=(), dim_sigma=None, unit_c=None, unit_t=None,
-                 lut_scale=0.0):
+                 lut_scale=0.0, rot_pm1=None):
         self.kind, self.d, self.bits, self.m = kind, d, bits, m
         self._keep = [rot, S, centroids, boundaries, dim_sigma, unit_c, unit_t]
         self.rot, self.S, self.centroids, self.boundaries = rot, S, centroids, boundaries
@@ -204,7 +204,7 @@ class Quantizer:
         tb = (C.c_int32 * MAX_TOP)(*(list(top_bits) + [0] * (MAX_TOP - len(top_bits))))
         self.c = Quantizer_t(kind, d, bits, m, _dptr(rot), _dptr(S), _dptr(centroids), _dptr(boundaries),
                              k_top, tail_bits, qjl, tb, _dptr(dim_sigma), _dptr(unit_c), _dptr(unit_t),
-                             float(lut_scale))
+                             float(lut_scale), int(bool(rot_pm1)))
 
     @property
     def ref(self):
@@ -215,12 +215,19 @@ class Quantizer:
         import torch
         return torch.as_tensor(np.ascontiguousarray(a, dtype=np.float32), device=device).contiguous()
 
+    @staticmethod
+    def _is_pm1(rot) -> bool:
+        """True when every entry of rot is +-1/sqrt(d) in fp32 (Hadamard-type rotation)."""
+        r = np.asarray(rot, dtype=np.float32)
+        return bool(np.all(np.abs(r) == np.float32(1.0 / math.sqrt(r.shape[0]))))
+
     @classmethod
     def mse(cls, rot, bits: int, dist: str = "beta", sigma: float = 0.0, device="cuda"):
         d = rot.shape[0]
         c, t, _ = codebook_build(bits, dist, d=d, sigma=sigma)
         return cls(KIND_MSE, d, cls._dev(rot, device), bits=bits,
-                   centroids=cls._dev(c, device), boundaries=cls._dev(t, device), lut_scale=lut_scale(c))
+                   centroids=cls._dev(c, device), boundaries=cls._dev(t, device), lut_scale=lut_scale(c),
+                   rot_pm1=cls._is_pm1(rot))
 
     @classmethod
     def prod(cls, rot, S, bits: int, dist: str = "beta", sigma: float = 0.0, device="cuda"):

@@ -164,3 +164,30 @@ def test_decode_matches_score_logits():
     ref = (p @ vh).cpu().numpy()
     err = rel_rows(out.cpu().numpy().reshape(Hq, D), ref)
     assert np.all(err <= 1e-3)
+
+
+def test_decode_hadamard_rotation():
+    """Keys and values quantized with a randomized Hadamard rotation (tensor-core +-1 path);
+    decode reads them with the same dense rotation folded into the query and the output."""
+    B, Hq, Hkv, Nmax, seq_lens = 2, 8, 2, 2000, [2000, 1234]
+    rot = ti.hadamard_rotation(D, 1602)
+    kt, k64, vt, v64 = _cache_inputs(B, Hkv, Nmax, 31)
+    qt, q64 = _query(B, Hq, 31)
+    kq, vq = K.Quantizer.mse(rot, 4), K.Quantizer.mse(rot, 4)
+    sl = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
+    c, t, _ = lloyd_max(4, "beta", d=D)
+    okq = OQ.quantize_mse(k64, rot, c, t, 4)
+    ovq = OQ.quantize_mse(v64, rot, c, t, 4)
+    vh = OQ.dequantize_mse(ovq["idx"], ovq["norms"], rot, c)
+    ref = decode_attention(q64, seq_lens, Hkv,
+                           lambda b, h, qs: OQ.estimate_mse(qs, rot, okq["idx"][_rows(B, Hkv, Nmax, b, h, Nmax)],
+                                                            okq["norms"][_rows(B, Hkv, Nmax, b, h, Nmax)], c),
+                           lambda b, h, n: vh[_rows(B, Hkv, Nmax, b, h, n)], 1.0 / math.sqrt(D))
+    out = K.decode_attn(kq, vq, qt, sl, _dev_records(okq["codes"], okq["norms"]),
+                        _dev_records(ovq["codes"], ovq["norms"]), Nmax, Hkv).cpu().numpy()
+    assert K.get_status() == 0
+    err = rel_rows(out, ref)
+    assert np.all(err <= 1e-3), f"max row error {err.max():.3e}"
+    kc, vc = K.quantize(kq, kt), K.quantize(vq, vt)
+    err2 = rel_rows(K.decode_attn(kq, vq, qt, sl, kc, vc, Nmax, Hkv).cpu().numpy(), ref)
+    assert np.median(err2) <= 1e-3 and np.max(err2) <= 2e-2

@@ -79,6 +79,42 @@ def test_quantize_mse_parity(d, bits, dtype, n):
     assert np.all(err < 1e-5)
 
 
+@pytest.mark.parametrize("bits,dtype,n", [(4, "bf16", 128 * 148 + 77), (3, "bf16", 3000), (2, "f16", 2000),
+                                           (1, "bf16", 1000), (4, "f32", 700)])
+def test_quantize_mse_hadamard_parity(bits, dtype, n):
+    """Randomized Hadamard rotation (entries +-1/sqrt(d)): the tensor-core kernel multiplies by
+    the exact +-1 matrix; the oracle uses the dense rotation as given."""
+    d = 128
+    rot = ti.hadamard_rotation(d, 1500 + bits)
+    x, x64 = _inputs(n, d, dtype, 4500 + bits, zero_rows=[0])
+    q = K.Quantizer.mse(rot, bits)
+    assert q.c.rot_pm1 == 1
+    out = K.quantize(q, x)
+    torch.cuda.synchronize()
+    assert K.get_status() == 0
+    c, t, _ = lloyd_max(bits, "beta", d=d)
+    ref = OQ.quantize_mse(x64, rot, c, t, bits)
+    bad, exempt, _ = code_mismatches(as_u32(out.codes), ref["codes"], d, bits, ref["y"], t, skip_rows=[0])
+    assert bad == 0, f"{bad} code mismatches outside the band ({exempt} exempt)"
+    from oracle.quantizer import unpack_codes
+    assert np.all(unpack_codes(as_u32(out.codes)[0:1], d, bits) == (1 << (bits - 1)) - 1)
+    nrm = out.norms.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(nrm - ref["norms"]) <= 1e-5 * np.maximum(ref["norms"], 1e-30))
+
+
+def test_quantize_pm1_flag_rejects_other_rotations():
+    """rot_pm1 with a rotation whose entries are not +-1/sqrt(d) is reported, not trusted."""
+    d = 128
+    rot = ti.haar_rotation(d, 1502)
+    x, _ = _inputs(256, d, "bf16", 4600)
+    q = K.Quantizer.mse(rot, 4)
+    q.c.rot_pm1 = 1
+    K.quantize(q, x)
+    torch.cuda.synchronize()
+    assert K.get_status() == 1          # TQ_ERR_INVALID_ARG
+    assert K.get_status() == 0          # reading the status clears it
+
+
 @pytest.mark.parametrize("d,bits,m,dtype,n", [(128, 3, 128, "bf16", 2000), (64, 2, 64, "f32", 500),
                                               (128, 1, 128, "f32", 300), (128, 5, 256, "bf16", 400)])
 def test_quantize_prod_parity(d, bits, m, dtype, n):

@@ -30,7 +30,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "SEEDS", "haar_rotation", "gaussian_matrix", "kv_spectrum", "anisotropic",
+    "SEEDS", "haar_rotation", "hadamard_rotation", "gaussian_matrix", "kv_spectrum", "anisotropic",
     "iid_normal", "unit_gaussian", "to_bf16_f64", "anisotropic_torch", "normal_torch",
 ]
 
@@ -52,6 +52,20 @@ def haar_rotation(d: int, seed: int, dtype=np.float32) -> np.ndarray:
     q, r = np.linalg.qr(g)
     q = q * np.sign(np.diag(r))[None, :]
     return q.astype(dtype)
+
+
+def hadamard_rotation(d: int, seed: int) -> np.ndarray:
+    """Randomized Hadamard rotation H diag(s) / sqrt(d), d a power of two: H the Sylvester
+    Hadamard matrix, s i.i.d. random signs (the launch kit's O(d log d) rotation mode).  Every
+    entry is exactly +-float32(1/sqrt(d))."""
+    if d < 1 or d & (d - 1):
+        raise ValueError("d must be a power of two")
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    s = np.where(_rng(seed).random(d) < 0.5, -1.0, 1.0)
+    c = np.float32(1.0 / np.sqrt(d))
+    return (h * s[None, :]).astype(np.float32) * c
 
 
 def gaussian_matrix(m: int, d: int, seed: int, dtype=np.float32) -> np.ndarray:
