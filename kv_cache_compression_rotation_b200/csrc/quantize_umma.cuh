@@ -418,49 +418,68 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         }
         continue;
       }
-      // pass 1: ||y|| over the whole row (independent partial sums keep the FMA pipe busy)
-      float ss[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 4; c += 2) {
-        float va[32], vb[32];
-        tmem_ld32(taddr + 32 * c, va);
-        tmem_ld32(taddr + 32 * (c + 1), vb);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          ss[i & 3] = fmaf(va[i], va[i], ss[i & 3]);
-          ss[(i + 2) & 3] = fmaf(vb[i], vb[i], ss[(i + 2) & 3]);
-        }
-      }
-      const float ny = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
-      const float nu = p.pm1 ? ny * p.pm1_scale : ny;  // ||x|| (the +-1 product is sqrt(d) Pi x)
-      const float inv = ny > 0.f ? 1.f / ny : 1.f;     // a zero row keeps u = 0
       uint32_t* dst = p.codes + v * W;
-      // pass 2: codes of 32 coordinates at a time, B packed words per chunk
       if (use_cells) {
+        // the whole row comes out of TMEM in one go (128 registers), so the accumulator
+        // buffer goes back to the MMA warp before any of the arithmetic below
+        float y[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, y[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(tempty_bar(buf));
+        // pass 1: ||y|| over the whole row (independent partial sums keep the FMA pipe busy)
+        float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; c += 2) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            ss[i & 3] = fmaf(y[c][i], y[c][i], ss[i & 3]);
+            ss[(i + 2) & 3] = fmaf(y[c + 1][i], y[c + 1][i], ss[(i + 2) & 3]);
+          }
+        }
+        const float ny = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
+        const float nu = p.pm1 ? ny * p.pm1_scale : ny;  // ||x|| (the +-1 product is sqrt(d) Pi x)
+        const float inv = ny > 0.f ? 1.f / ny : 1.f;     // a zero row keeps u = 0
+        // pass 2: codes of 32 coordinates at a time, B packed words per chunk (the code
+        // fields are disjoint, so they are added into the words)
         const float fs = inv * cell_scale;
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float y[32];
-          tmem_ld32(taddr + 32 * c, y);
-          tmem_wait_ld();
           uint32_t wc[B];
 #pragma unroll
           for (int w = 0; w < B; ++w) wc[w] = 0u;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float f = __saturatef(fmaf(y[i], fs, 0.5f));
+            const float f = __saturatef(fmaf(y[c][i], fs, 0.5f));
             const float gcell = __fmaf_rz(f, kCellSpan, 8388608.0f);
             const uint32_t e = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gcell));
             // + 1 when f lies above the cell's boundary: the sign bit of (boundary - f)
             const uint32_t code = (e & 15u) + (__float_as_uint(__uint_as_float(e) - f) >> 31);
             const int pos = i * B;
-            wc[pos >> 5] |= code << (pos & 31);
-            if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
+            wc[pos >> 5] += code << (pos & 31);
+            if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] += code >> (32 - (pos & 31));
           }
           if (v < p.n) store_words<B>(dst + c * B, wc);
         }
+        if (v < p.n) p.norms[v] = nu;
       } else {
+        // thresholds against the unnormalized row: TMEM is read twice, 32 columns at a time
+        float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; c += 2) {
+          float va[32], vb[32];
+          tmem_ld32(taddr + 32 * c, va);
+          tmem_ld32(taddr + 32 * (c + 1), vb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            ss[i & 3] = fmaf(va[i], va[i], ss[i & 3]);
+            ss[(i + 2) & 3] = fmaf(vb[i], vb[i], ss[(i + 2) & 3]);
+          }
+        }
+        const float ny = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
+        const float nu = p.pm1 ? ny * p.pm1_scale : ny;
         const float nthr = ny > 0.f ? ny : 1.f;
 #pragma unroll
         for (int k = 0; k < NB; ++k) thr[k] = nthr * tsm[k];
@@ -483,10 +502,10 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           }
           if (v < p.n) store_words<B>(dst + c * B, wc);
         }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(buf));
+        if (v < p.n) p.norms[v] = nu;
       }
-      if (v < p.n) p.norms[v] = nu;
-      tc_fence_before();
-      mbar_arrive(tempty_bar(buf));
     }
   }
   tc_fence_before();
