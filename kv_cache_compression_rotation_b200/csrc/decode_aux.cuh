@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(QPrepParams p) {
   float* q2 = qr + p.D;          // [max(D,16)]
   __shared__ float red[2][4];
   const int r = blockIdx.x, tid = threadIdx.x, D = p.D;
+  pdl_trigger();   // the decode kernel may launch; it waits for this grid before reading q'
   for (int j = tid; j < D; j += 128) qin[j] = load_elem(p.q, p.dtype, static_cast<int64_t>(r) * D + j);
   __syncthreads();
   for (int j = tid; j < D; j += 128) {
@@ -62,6 +63,7 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
   float* ov = csm;                  // [D]
   __shared__ float sM, sL;
   const int r = blockIdx.x, tid = threadIdx.x, D = p.D;
+  pdl_wait();      // the partials come from the decode kernel before this one
   const float* ml = p.part_ml + static_cast<int64_t>(r) * p.n_chunks * 2;
   if (tid < 32) {
     float M = -INFINITY;
@@ -134,6 +136,7 @@ __device__ __forceinline__ void matvec8x128(const float* __restrict__ M, const f
 __global__ void __launch_bounds__(256) qprep128_kernel(QPrepParams p) {
   __shared__ __align__(16) float xs[8 * 128], ys[8 * 128], us[8 * 128];
   const int r0 = blockIdx.x * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();   // the decode kernel may launch; it waits for this grid before reading q'
   for (int i = tid; i < 8 * 128; i += 256) {
     const int r = i >> 7, j = i & 127;
     xs[i] = (r0 + r < p.rows) ? load_elem(p.q, p.dtype, static_cast<int64_t>(r0 + r) * 128 + j) : 0.f;
@@ -203,10 +206,23 @@ __global__ void __launch_bounds__(256) qprep128_kernel(QPrepParams p) {
 // 2^(m_c - M) / L of the 2 rows ([2][n_chunks] floats).
 __global__ void __launch_bounds__(256) combine128_kernel(CombineParams p) {
   constexpr int R = 2;
-  extern __shared__ __align__(16) float cw[];
+  extern __shared__ __align__(16) float cw[];       // [R][n_chunks] weights, then rot_V [128][128]
   __shared__ __align__(16) float ov[R * 128];      // o' per row
   const int r0 = blockIdx.x * R, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nch = p.n_chunks;
+  // rot_V is an input, not a decode result: its copy into shared memory is issued before
+  // the wait for the decode kernel and lands while that kernel drains
+  float* rv = cw + ((R * nch + 3) & ~3);
+  const uint32_t rv_s = static_cast<uint32_t>(__cvta_generic_to_shared(rv));
+  if ((reinterpret_cast<uintptr_t>(p.rot_v) & 15u) == 0) {
+    for (int i = tid; i < 128 * 128 / 4; i += 256)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(rv_s + 16u * i), "l"(p.rot_v + 4 * i) : "memory");
+  } else {
+    for (int i = tid; i < 128 * 128; i += 256)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(rv_s + 4u * i), "l"(p.rot_v + i) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  pdl_wait();      // the partials come from the decode kernel before this one
   if (warp < R) {
     float* w = cw + warp * nch;
     const int r = r0 + warp;
@@ -237,16 +253,17 @@ __global__ void __launch_bounds__(256) combine128_kernel(CombineParams p) {
     if (r < p.rows) {
       const float* w = cw + rr * nch;
       const float* po = p.part_o + static_cast<int64_t>(r) * nch * 128 + k;
-#pragma unroll 4
+#pragma unroll 8
       for (int c = 0; c < nch; ++c) a = fmaf(w[c], __ldg(po + c * 128), a);
       if (p.v_sigma) a *= p.v_sigma[k];
     }
     ov[rr * 128 + k] = a;
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   float o = 0.f;
 #pragma unroll 8
-  for (int j = 0; j < 128; ++j) o = fmaf(ov[rr * 128 + j], __ldg(p.rot_v + j * 128 + k), o);
+  for (int j = 0; j < 128; ++j) o = fmaf(ov[rr * 128 + j], rv[j * 128 + k], o);
   if (r < p.rows) p.out[static_cast<int64_t>(r) * 128 + k] = o;
 }
 

@@ -11,8 +11,8 @@ cudaError_t go_pk(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t s,
   smem = decode_tma_smem_bytes(KB, VB, KFMT_MSE, PK);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k<<<grid, (tma_consumers(KFMT_MSE, PK) + 1) * 32, smem, s>>>(p, status, lim);
-  return cudaGetLastError();
+  // the query preparation kernel runs just before: the prologue and the first copies overlap it
+  return launch_pdl(k, grid, dim3((tma_consumers(KFMT_MSE, PK) + 1) * 32), smem, s, p, status, lim);
 }
 
 // GQA groups of at most 4 heads take the packed-column variant

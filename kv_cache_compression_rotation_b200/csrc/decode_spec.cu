@@ -22,8 +22,8 @@ cudaError_t go_tma(const DecodeParams& p, dim3 grid, cudaStream_t s, int* status
   const size_t smem = decode_tma_smem_bytes(1, 1, KFMT_SPEC, PK);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k<<<grid, (tma_consumers(KFMT_SPEC, PK) + 1) * 32, smem, s>>>(p, status, lim);
-  return cudaGetLastError();
+  // the query preparation kernel runs just before: the prologue and the first copies overlap it
+  return launch_pdl(k, grid, dim3((tma_consumers(KFMT_SPEC, PK) + 1) * 32), smem, s, p, status, lim);
 }
 
 }  // namespace

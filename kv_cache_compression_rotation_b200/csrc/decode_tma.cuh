@@ -315,6 +315,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   if constexpr (SP)
     for (int i = tid; i < 510; i += kTmaThreads) utab[i] = __ldg(p.unit_c + i);
   __syncthreads();
+  pdl_trigger();   // the chunk combine may launch; it waits for this grid to complete
 
   if (warp == NC) {
     // ---------------- producer ----------------
@@ -452,6 +453,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     }
     vh_off = vh_nb ? unit_c_off(vh_nb) : 0;
   }
+  // the prepared queries come from the kernel before this one (the producer's copies of the
+  // cache do not depend on it and are already under way)
+  pdl_wait();
   int gs = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     int bh, hblk, chunk, k0, k1;

@@ -17,6 +17,14 @@ __device__ __forceinline__ void report_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic-serialization
+// attribute may begin while the kernel before it in the stream is still running:
+// pdl_wait() returns once that kernel has completed and its writes are visible, and
+// pdl_trigger() lets the kernel after this one begin launching.  Both are no-ops for a
+// kernel launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float load_elem(const void* base, int dtype, int64_t i) {
   if (dtype == TQ_F32) return __ldg(reinterpret_cast<const float*>(base) + i);
   if (dtype == TQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);

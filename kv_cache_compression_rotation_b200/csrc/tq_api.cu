@@ -682,17 +682,17 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
   cp.part_ml = pml; cp.part_o = po; cp.rot_v = vq->rot;
   cp.v_sigma = vq->kind == TQ_KIND_SPECTRAL ? vq->dim_sigma : nullptr;
   cp.out = out;
-  const size_t csm = static_cast<size_t>(2) * P.n_chunks * 4;
-  if (D == 128 && csm <= 160 * 1024) {
-    if (csm > 48 * 1024) {
-      e = cudaFuncSetAttribute(combine128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(csm));
-      if (e != cudaSuccess) return cuda_fail(e, "combine attribute");
-    }
-    combine128_kernel<<<(rows + 1) / 2, 256, csm, stream>>>(cp);
+  // combine128: weights of 2 rows, then rot_V (64 KB); both combines wait on the decode
+  // kernel inside (programmatic launch: their launch overlaps its tail)
+  const size_t csm = static_cast<size_t>((2 * P.n_chunks + 3) & ~3) * 4 + 128 * 128 * 4;
+  if (D == 128 && csm <= 200 * 1024) {
+    e = cudaFuncSetAttribute(combine128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(csm));
+    if (e != cudaSuccess) return cuda_fail(e, "combine attribute");
+    e = launch_pdl(combine128_kernel, dim3(static_cast<unsigned>((rows + 1) / 2)), dim3(256), csm, stream, cp);
   } else {
-    combine_kernel<<<rows, 128, static_cast<size_t>(D) * 4, stream>>>(cp);
+    e = launch_pdl(combine_kernel, dim3(static_cast<unsigned>(rows)), dim3(128), static_cast<size_t>(D) * 4, stream, cp);
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "combine launch");
 }
 
