@@ -247,9 +247,12 @@ tq_status tq_decode_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq
  *   first seq_lens[b] records, p = softmax(logit), out = sum_i p_i v_hat_i.
  * q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), caches laid out
  * [B][Hkv][Nmax] records, out [B*Hq*d] fp32.  Keys: MSE, PROD or SPECTRAL; values: MSE or
- * SPECTRAL (without qjl).  This build runs d in {64, 128}, code bits <= 4, PROD m = d,
+ * SPECTRAL (without qjl).  This build runs d = 128, code bits <= 4, PROD m = d,
  * Hq/Hkv in 1..16; other shapes give TQ_ERR_UNSUPPORTED.  Value norms must stay below
- * 6.0e4 (the probability-weighted norm is a half-precision MMA operand).
+ * 6.0e4 (the probability-weighted norm is a half-precision MMA operand).  The call
+ * enqueues three kernels (query preparation, decode, chunk combine); the last two use
+ * programmatic dependent launch, so each may start while the one before it drains, and
+ * every read of a predecessor's output waits for that kernel to complete.
  */
 tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const void* q,
                          int32_t dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,

@@ -428,17 +428,18 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(tempty_bar(buf));
-        // pass 1: ||y|| over the whole row (independent partial sums keep the FMA pipe busy)
-        float ss[4] = {0.f, 0.f, 0.f, 0.f};
+        // pass 1: ||y|| over the whole row, two coordinates per packed FMA (four independent
+        // pairs of partial sums keep the FMA pipe busy)
+        float2 s2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int c = 0; c < 4; c += 2) {
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            ss[i & 3] = fmaf(y[c][i], y[c][i], ss[i & 3]);
-            ss[(i + 2) & 3] = fmaf(y[c + 1][i], y[c + 1][i], ss[(i + 2) & 3]);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 v2 = make_float2(y[c][i], y[c][i + 1]);
+            s2[(i >> 1) & 3] = __ffma2_rn(v2, v2, s2[(i >> 1) & 3]);
           }
         }
-        const float ny = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
+        const float ny = sqrtf(((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) + ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y)));
         const float nu = p.pm1 ? ny * p.pm1_scale : ny;  // ||x|| (the +-1 product is sqrt(d) Pi x)
         const float inv = ny > 0.f ? 1.f / ny : 1.f;     // a zero row keeps u = 0
         // pass 2: codes of 32 coordinates at a time, B packed words per chunk (the code
@@ -450,15 +451,22 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
 #pragma unroll
           for (int w = 0; w < B; ++w) wc[w] = 0u;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float f = __saturatef(fmaf(y[c][i], fs, 0.5f));
-            const float gcell = __fmaf_rz(f, kCellSpan, 8388608.0f);
-            const uint32_t e = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gcell));
+          for (int i = 0; i < 32; i += 2) {
+            // two coordinates at a time: the cell index and the boundary difference go through
+            // packed FMAs (the same roundings as the scalar forms)
+            const float2 f2 = make_float2(__saturatef(fmaf(y[c][i], fs, 0.5f)), __saturatef(fmaf(y[c][i + 1], fs, 0.5f)));
+            const float2 g2 = __ffma2_rz(f2, make_float2(kCellSpan, kCellSpan), make_float2(8388608.0f, 8388608.0f));
+            const uint32_t e0 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(g2.x));
+            const uint32_t e1 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(g2.y));
             // + 1 when f lies above the cell's boundary: the sign bit of (boundary - f)
-            const uint32_t code = (e & 15u) + (__float_as_uint(__uint_as_float(e) - f) >> 31);
-            const int pos = i * B;
-            wc[pos >> 5] += code << (pos & 31);
-            if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] += code >> (32 - (pos & 31));
+            const float2 d2 = __ffma2_rn(f2, make_float2(-1.f, -1.f), make_float2(__uint_as_float(e0), __uint_as_float(e1)));
+            const uint32_t code[2] = {(e0 & 15u) + (__float_as_uint(d2.x) >> 31), (e1 & 15u) + (__float_as_uint(d2.y) >> 31)};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int pos = (i + h) * B;
+              wc[pos >> 5] += code[h] << (pos & 31);
+              if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] += code[h] >> (32 - (pos & 31));
+            }
           }
           if (v < p.n) store_words<B>(dst + c * B, wc);
         }
