@@ -87,7 +87,9 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(x0, x1);
   const float2 back = __half22float2(h);
-  const __half2 l = __floats2half2_rn(x0 - back.x, x1 - back.y);
+  // x - back in one packed FMA (the product by -1 is exact, so the rounding is the add's)
+  const float2 r = __ffma2_rn(back, make_float2(-1.f, -1.f), make_float2(x0, x1));
+  const __half2 l = __floats2half2_rn(r.x, r.y);
   hi = *reinterpret_cast<const uint32_t*>(&h);
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }

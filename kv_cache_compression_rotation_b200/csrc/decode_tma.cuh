@@ -694,13 +694,17 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           }
         }
         // acc[0], acc[1]: token row g, heads h0, h0 + 1; acc[2], acc[3]: token row g + 8
-        const float sa[4] = {sa0, sa1, sa0, sa1}, sbq[4] = {sb0, sb1, sb0, sb1};
+        // (one packed two-lane FMA per row and step)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float v = sa[i] * acc[i];
-          if constexpr (KF == KFMT_PROD) v += gm[u][i >> 1] * sbq[i] * acc2[i];
-          if constexpr (SP) v += sbq[i] * acc2[i];
-          sc[u][i] = ok[u][i >> 1] ? kn[u][i >> 1] * v : -INFINITY;
+        for (int h = 0; h < 2; ++h) {
+          float2 v = __fmul2_rn(make_float2(sa0, sa1), make_float2(acc[2 * h], acc[2 * h + 1]));
+          if constexpr (KF == KFMT_PROD)
+            v = __ffma2_rn(__fmul2_rn(make_float2(gm[u][h], gm[u][h]), make_float2(sb0, sb1)),
+                           make_float2(acc2[2 * h], acc2[2 * h + 1]), v);
+          if constexpr (SP) v = __ffma2_rn(make_float2(sb0, sb1), make_float2(acc2[2 * h], acc2[2 * h + 1]), v);
+          v = __fmul2_rn(make_float2(kn[u][h], kn[u][h]), v);
+          sc[u][2 * h] = ok[u][h] ? v.x : -INFINITY;
+          sc[u][2 * h + 1] = ok[u][h] ? v.y : -INFINITY;
         }
       }
       // ---- online softmax per head (log2 domain) over the warp's tokens; the row
@@ -725,8 +729,13 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           const float f0 = ex2(m0 - mn0), f1 = ex2(m1 - mn1);
           l0 *= f0;
           l1 *= f1;
+          const float2 f01 = make_float2(f0, f1);
 #pragma unroll
-          for (int i = 0; i < MT; ++i) { o[i][0] *= f0; o[i][2] *= f0; o[i][1] *= f1; o[i][3] *= f1; }
+          for (int i = 0; i < MT; ++i) {
+            const float2 a = __fmul2_rn(make_float2(o[i][0], o[i][1]), f01);
+            const float2 b = __fmul2_rn(make_float2(o[i][2], o[i][3]), f01);
+            o[i][0] = a.x; o[i][1] = a.y; o[i][2] = b.x; o[i][3] = b.y;
+          }
           if constexpr (SP) { oh[0] *= f0; oh[1] *= f1; }
           m0 = mn0;
           m1 = mn1;
@@ -734,14 +743,20 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const float p00 = c0ok ? ex2(sc[u][0] - m0) : 0.f, p01 = c1ok ? ex2(sc[u][1] - m1) : 0.f;
-        const float p10 = c0ok ? ex2(sc[u][2] - m0) : 0.f, p11 = c1ok ? ex2(sc[u][3] - m1) : 0.f;
-        l0 += p00 + p10;
-        l1 += p01 + p11;
+        const float2 nm = make_float2(-m0, -m1);
+        const float2 d0 = __fadd2_rn(make_float2(sc[u][0], sc[u][1]), nm);
+        const float2 d1 = __fadd2_rn(make_float2(sc[u][2], sc[u][3]), nm);
+        const float p00 = c0ok ? ex2(d0.x) : 0.f, p01 = c1ok ? ex2(d0.y) : 0.f;
+        const float p10 = c0ok ? ex2(d1.x) : 0.f, p11 = c1ok ? ex2(d1.y) : 0.f;
+        const float2 l01 = __fadd2_rn(make_float2(l0, l1), __fadd2_rn(make_float2(p00, p01), make_float2(p10, p11)));
+        l0 = l01.x;
+        l1 = l01.y;
         // P^T (16 tokens x 8 columns) as the B operand: transpose the two 8x8 halves
         uint32_t pth, ptl, pbh, pbl;
-        split_pair(p00 * vn[u][0], p01 * vn[u][0], pth, ptl);
-        split_pair(p10 * vn[u][1], p11 * vn[u][1], pbh, pbl);
+        const float2 pv0 = __fmul2_rn(make_float2(p00, p01), make_float2(vn[u][0], vn[u][0]));
+        const float2 pv1 = __fmul2_rn(make_float2(p10, p11), make_float2(vn[u][1], vn[u][1]));
+        split_pair(pv0.x, pv0.y, pth, ptl);
+        split_pair(pv1.x, pv1.y, pbh, pbl);
         uint32_t b0h, b1h, b0l = 0u, b1l = 0u;
         if constexpr (PK) {
           b0h = movmatrix_t(plo ? ptl : pth);
