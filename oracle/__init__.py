@@ -28,6 +28,8 @@ Modules:
 * :mod:`oracle.attention` -- decode attention (softmax(q.k_hat / sqrt(d)) v_hat)
   straight from the quantized records, and dense scores.
 * :mod:`oracle.search`    -- exhaustive top-k by estimated inner product.
+* :mod:`oracle.split`     -- outlier-channel split: independent TurboQuant instances
+  on channel groups (online outlier detection, per-group quantize, summed estimates).
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against closed forms,
 printed values, brute force or library routines, except where its docstring says

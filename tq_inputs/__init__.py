@@ -32,6 +32,7 @@ import numpy as np
 __all__ = [
     "SEEDS", "haar_rotation", "hadamard_rotation", "gaussian_matrix", "kv_spectrum", "anisotropic",
     "iid_normal", "unit_gaussian", "to_bf16_f64", "anisotropic_torch", "normal_torch",
+    "planted_outliers",
 ]
 
 # Seed plan: role base + workload number (1..5).
@@ -97,6 +98,14 @@ def anisotropic(n: int, d: int, basis: np.ndarray, seed: int, lam=None) -> np.nd
     lam = kv_spectrum(d) if lam is None else np.asarray(lam, dtype=np.float64)
     z = _rng(seed).standard_normal((n, d))
     return (z * np.sqrt(d * lam)[None, :]) @ basis.astype(np.float64).T
+
+
+def planted_outliers(n: int, d: int, channels, scale: float, seed: int) -> np.ndarray:
+    """float64 rows N(0, I) whose listed channels are multiplied by ``scale``: keys with a
+    few high-magnitude channels, the structure the outlier-channel split targets."""
+    x = _rng(seed).standard_normal((n, d))
+    x[:, np.asarray(channels, dtype=np.int64)] *= scale
+    return x
 
 
 def unit_gaussian(n: int, d: int, seed: int) -> np.ndarray:
