@@ -211,6 +211,54 @@ tq_status tq_quantize_spectral(const tq_quantizer* q, const void* x, int32_t dty
                                tq_packed out, tq_stream stream);
 
 /*
+ * Outlier-channel split (TurboQuant review, Method: for the KV-cache experiments the
+ * channels are split into an outlier group and the rest, each quantized by its own
+ * TurboQuant instance; the setting it calls 2.5-bit is 32 outlier channels at 3 bits plus
+ * 96 channels at 2 bits).  Group g reads channels cols[g][0 .. groups[g]->d) of every
+ * d-wide vector and is an independent MSE or PROD instance of dimension groups[g]->d,
+ * with its own rotation, codebook, norm and packed records.  The descriptor and the
+ * quantizers are host memory; cols[g] are DEVICE int32 arrays owned by the caller.
+ * Channel indices must lie in 0..d-1; an index outside that range is read as channel 0
+ * and sets the device status to TQ_ERR_INVALID_ARG (see tq_get_status).  For the
+ * estimates below to be those of the split, the groups must be disjoint and cover every
+ * channel; the library does not check this on the host (it would need a device read).
+ */
+#define TQ_MAX_GROUPS 4
+
+typedef struct {
+  int32_t n_groups;                           /* 1..TQ_MAX_GROUPS */
+  int32_t d;                                  /* width of the full vectors */
+  const tq_quantizer* groups[TQ_MAX_GROUPS];  /* kind TQ_KIND_MSE or TQ_KIND_PROD */
+  const int32_t* cols[TQ_MAX_GROUPS];         /* DEVICE, groups[g]->d channel indices */
+} tq_split;
+
+/*
+ * DEVICE.  Quantize n rows x [n*d] (dtype, row-major) group by group: out[g] receives
+ * the records of group g (layout from tq_record_layout(groups[g])), exactly what
+ * tq_quantize_mse / tq_quantize_prod would write for the gathered rows
+ * (x_v[cols[g][0]], ..., x_v[cols[g][d_g - 1]]).  out is a host array of n_groups
+ * packed descriptors.  Validation as for tq_quantize_mse, per group.
+ */
+tq_status tq_quantize_split(const tq_split* sp, const void* x, int32_t dtype, int64_t n,
+                            const tq_packed* out, tq_stream stream);
+
+/* Workspace bytes needed by tq_score_split. */
+tq_status tq_score_split_workspace(const tq_split* sp, int64_t nq, int64_t n, int32_t topk,
+                                   size_t* bytes);
+
+/*
+ * DEVICE.  Split inner-product estimates: est(q, x_i) = sum over the groups of the
+ * group's tq_score estimate for the gathered query q[cols[g]] against keys[g] (record i
+ * of every group belongs to vector i).  Output as tq_score: topk == 0 gives scores
+ * [nq*n] dense; topk in 1..32 gives the topk records of the summed estimate per query
+ * (descending, ties to the lower id).  keys is a host array of n_groups packed
+ * descriptors; workspace: device, >= tq_score_split_workspace bytes.
+ */
+tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int64_t nq,
+                         const tq_packed* keys, int64_t n, int32_t topk, float* scores,
+                         int32_t* ids, void* workspace, size_t ws_bytes, tq_stream stream);
+
+/*
  * DEVICE.  Reconstruction out [n*d] fp32: MSE x_hat = ||x|| rot^T c[code];
  * PROD adds ||x|| rot^T (sqrt(pi/2)/m ||r|| S^T (2s-1)) (unbiased);
  * SPECTRAL x_hat = rot^T c_hat (the QJL bits are not used).
@@ -229,7 +277,7 @@ tq_status tq_score_workspace(const tq_quantizer* q, int64_t nq, int64_t n, int32
  *   MSE       ||x|| <rot q, c[code]>
  *   PROD      ||x|| (<rot q, c_hat> + sqrt(pi/2)/m ||r|| <S rot q, 2s-1>)   (unbiased)
  *   SPECTRAL  sum_j (rot q)_j c_hat_j + sqrt(pi/2)/k ||r|| <S (rot q)_top, 2s-1>
- * topk == 0: scores [nq*n] fp32 dense, ids unused.  topk in 1..64: for each query the
+ * topk == 0: scores [nq*n] fp32 dense, ids unused.  topk in 1..32: for each query the
  * topk records by descending estimate, ties to the lower id: ids [nq*topk] int32,
  * scores [nq*topk].  workspace: device, >= tq_score_workspace bytes.
  */

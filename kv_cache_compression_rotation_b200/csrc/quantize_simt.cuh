@@ -44,6 +44,11 @@ struct SimtQuantParams {
   float* norms;
   float* rnorms;
   int tv;             // vectors per CTA
+  // input gather: element j of vector v is x[v * ld + (cols ? cols[j] : j)]; a column
+  // outside 0..ld-1 reads column 0 and reports TQ_ERR_INVALID_ARG to *status
+  int64_t ld;
+  const int32_t* cols;
+  int* status;
 };
 
 __device__ __forceinline__ void spectral_dim_book(const SimtQuantParams& p, int j, int* bits,
@@ -129,7 +134,19 @@ simt_quantize_kernel(SimtQuantParams p) {
 
   for (int i = tid; i < tv * dp; i += kSimtThreads) {
     const int v = i / dp, k = i - v * dp;
-    xs[i] = (v < nv && k < d) ? load_elem(p.x, p.dtype, (v0 + v) * d + k) : 0.f;
+    float xv = 0.f;
+    if (v < nv && k < d) {
+      int64_t col = k;
+      if (p.cols) {
+        col = __ldg(p.cols + k);
+        if (col < 0 || col >= p.ld) {
+          report_status(p.status, TQ_ERR_INVALID_ARG);
+          col = 0;
+        }
+      }
+      xv = load_elem(p.x, p.dtype, (v0 + v) * p.ld + col);
+    }
+    xs[i] = xv;
   }
   __syncthreads();
   for (int v = warp; v < tv; v += kSimtThreads / 32) {

@@ -35,6 +35,7 @@ struct ScoreParams {
   int qu_stride;
   int64_t nq, n;
   float* out;                 // [nq][n]
+  int accumulate;             // 1: add the estimates to out (split groups after the first)
 };
 
 __global__ void __launch_bounds__(kScoreThreads) score_dense_kernel(ScoreParams p) {
@@ -108,18 +109,34 @@ __global__ void __launch_bounds__(kScoreThreads) score_dense_kernel(ScoreParams 
 #pragma unroll
     for (int i = 0; i < kScoreQT; ++i) acc[i] *= nu;
   }
-  for (int i = 0; i < nqb; ++i) p.out[(q0 + i) * p.n + v] = acc[i];
+  for (int i = 0; i < nqb; ++i) {
+    float* o = p.out + (q0 + i) * p.n + v;
+    *o = p.accumulate ? *o + acc[i] : acc[i];
+  }
 }
 
 // Rotated queries for scoring: qr = rot @ q, qu = S @ qr (prod) or S_top @ qr_top.
+// Query element j of row r is q[r * ldq + (cols ? cols[j] : j)] (the split's gather; a
+// column outside 0..ldq-1 reads column 0 and reports TQ_ERR_INVALID_ARG to *status).
 __global__ void __launch_bounds__(128) score_qprep_kernel(const void* q, int dtype, int d, int kind,
                                                           const float* rot, const float* S, int m,
-                                                          int k_top, float* qr, float* qu, int qu_stride) {
+                                                          int k_top, float* qr, float* qu, int qu_stride,
+                                                          int64_t ldq, const int32_t* cols, int* status) {
   extern __shared__ __align__(16) float qsm2[];
   float* qin = qsm2;
   float* qo = qin + d;
   const int64_t r = blockIdx.x;
-  for (int j = threadIdx.x; j < d; j += 128) qin[j] = load_elem(q, dtype, r * d + j);
+  for (int j = threadIdx.x; j < d; j += 128) {
+    int64_t col = j;
+    if (cols) {
+      col = __ldg(cols + j);
+      if (col < 0 || col >= ldq) {
+        report_status(status, TQ_ERR_INVALID_ARG);
+        col = 0;
+      }
+    }
+    qin[j] = load_elem(q, dtype, r * ldq + col);
+  }
   __syncthreads();
   for (int j = threadIdx.x; j < d; j += 128) {
     float a = 0.f;

@@ -202,8 +202,11 @@ bool umma_supported(const tq_quantizer* q, int dtype, int64_t n) {
   return major == 10 && get_encode() != nullptr;
 }
 
+// ld / cols: element j of row v is x[v * ld + (cols ? cols[j] : j)] (cols: device; the
+// split's channel gather); a gather always takes the CUDA-core kernel.
 tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64_t n, tq_packed out,
-                          cudaStream_t stream, int want_kind) {
+                          cudaStream_t stream, int want_kind, int64_t ld, const int32_t* cols,
+                          const Range* extra_outs = nullptr, int n_extra = 0) {
   tq_status s = check_quantizer(q);
   if (s != TQ_OK) return s;
   if (q->kind != want_kind) return fail(TQ_ERR_INVALID_ARG, "quantizer kind does not match this entry point");
@@ -217,11 +220,14 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   if ((s = check_packed(out, L)) != TQ_OK) return s;
   Range outs[4];
   packed_ranges(out, L, n, outs);
-  const Range ins[1] = {{x, static_cast<size_t>(n) * q->d * dtype_size(dtype)}};
-  if ((s = check_no_alias(outs, 4, ins, 1)) != TQ_OK) return s;
+  // inputs: x, and the other groups' outputs of a split call (disjoint from this group's)
+  Range ins[1 + 4 * TQ_MAX_GROUPS];
+  ins[0] = {x, static_cast<size_t>(n) * static_cast<size_t>(ld) * dtype_size(dtype)};
+  for (int i = 0; i < n_extra; ++i) ins[1 + i] = extra_outs[i];
+  if ((s = check_no_alias(outs, 4, ins, 1 + n_extra)) != TQ_OK) return s;
   int* status = device_status_ptr();
 
-  if (umma_supported(q, dtype, n)) {
+  if (!cols && umma_supported(q, dtype, n)) {
     auto encode = get_encode();
     CUtensorMap map;
     const cuuint64_t gdim[2] = {128, static_cast<cuuint64_t>(n)};
@@ -269,6 +275,9 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   p.signs = out.signs; p.sign_words = L.sign_words;
   p.norms = L.has_norms ? out.norms : nullptr;
   p.rnorms = L.has_rnorms ? out.rnorms : nullptr;
+  p.ld = ld;
+  p.cols = cols;
+  p.status = status;
   const int d = q->d;
   // vectors per CTA: a multiple of 8 (the tiled product's row groups), at most 32, within
   // 200 KB of shared memory
@@ -418,17 +427,20 @@ tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out) {
 
 tq_status tq_quantize_mse(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
                           tq_stream stream) {
-  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_MSE);
+  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_MSE,
+                         q ? q->d : 0, nullptr);
 }
 
 tq_status tq_quantize_prod(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
                            tq_stream stream) {
-  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_PROD);
+  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_PROD,
+                         q ? q->d : 0, nullptr);
 }
 
 tq_status tq_quantize_spectral(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
                                tq_stream stream) {
-  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_SPECTRAL);
+  return quantize_common(q, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream), TQ_KIND_SPECTRAL,
+                         q ? q->d : 0, nullptr);
 }
 
 tq_status tq_dequantize(const tq_quantizer* q, tq_packed in, int64_t n, float* out, tq_stream stream) {
@@ -472,6 +484,33 @@ static int score_qu_stride(const tq_quantizer* q) {
   if (q->kind == TQ_KIND_PROD) return q->m;
   if (q->kind == TQ_KIND_SPECTRAL && q->qjl) return q->k_top;
   return 0;
+}
+
+// Estimator parameters of one quantizer's records (the rotated queries and the output are
+// filled in per launch).
+static ScoreParams score_params(const tq_quantizer* q, const tq_layout& L, const tq_packed& keys, int64_t n) {
+  const int qus = score_qu_stride(q);
+  ScoreParams p{};
+  p.kind = q->kind; p.d = q->d; p.m = qus;
+  p.bmse = q->kind == TQ_KIND_MSE ? q->bits : (q->kind == TQ_KIND_PROD ? q->bits - 1 : 0);
+  p.codes = keys.codes; p.code_words = L.code_words;
+  p.signs = keys.signs; p.sign_words = L.sign_words;
+  p.norms = keys.norms; p.rnorms = keys.rnorms;
+  p.centroids = q->centroids;
+  p.k_top = q->k_top; p.tail_bits = q->tail_bits; p.qjl = q->qjl;
+  for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];
+  p.head_words = q->kind == TQ_KIND_SPECTRAL ? (spectral_head_bits(q) + 31) / 32 : 0;
+  p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids;
+  p.coef = q->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / q->m)
+                                   : static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, q->k_top));
+  p.qu_stride = std::max(qus, 1);
+  p.n = n;
+  p.accumulate = 0;
+  return p;
+}
+
+static size_t score_smem(const ScoreParams& p) {
+  return static_cast<size_t>(kScoreQT) * (p.d + p.qu_stride) * 4 + 256 * 4;
 }
 
 tq_status tq_score_workspace(const tq_quantizer* q, int64_t nq, int64_t n, int32_t topk, size_t* bytes) {
@@ -522,25 +561,11 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
   float* dense = reinterpret_cast<float*>(
       ws + (static_cast<size_t>(nq) * d * 4 + 255) / 256 * 256 + (static_cast<size_t>(nq) * qus * 4 + 255) / 256 * 256);
   score_qprep_kernel<<<static_cast<unsigned>(nq), 128, 2 * d * 4, stream>>>(
-      qv, dtype, d, q->kind, q->rot, q->S, q->m, q->k_top, qr, qu, qus);
+      qv, dtype, d, q->kind, q->rot, q->S, q->m, q->k_top, qr, qu, qus, d, nullptr, device_status_ptr());
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "score qprep launch");
-  ScoreParams p{};
-  p.kind = q->kind; p.d = d; p.m = qus;
-  p.bmse = q->kind == TQ_KIND_MSE ? q->bits : (q->kind == TQ_KIND_PROD ? q->bits - 1 : 0);
-  p.codes = keys.codes; p.code_words = L.code_words;
-  p.signs = keys.signs; p.sign_words = L.sign_words;
-  p.norms = keys.norms; p.rnorms = keys.rnorms;
-  p.centroids = q->centroids;
-  p.k_top = q->k_top; p.tail_bits = q->tail_bits; p.qjl = q->qjl;
-  for (int j = 0; j < TQ_MAX_TOP; ++j) p.top_bits[j] = q->top_bits[j];
-  p.head_words = q->kind == TQ_KIND_SPECTRAL ? (spectral_head_bits(q) + 31) / 32 : 0;
-  p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids;
-  p.coef = q->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / q->m)
-                                   : static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, q->k_top));
-  p.qu_stride = std::max(qus, 1);
-  p.n = n;
-  const size_t smem = static_cast<size_t>(kScoreQT) * (d + p.qu_stride) * 4 + 256 * 4;
+  ScoreParams p = score_params(q, L, keys, n);
+  const size_t smem = score_smem(p);
   e = cudaFuncSetAttribute(score_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "score attribute");
   const int64_t qb = topk > 0 ? score_block(nq, n) : nq;
@@ -555,6 +580,157 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
     if (grid.y > 65535) return fail(TQ_ERR_UNSUPPORTED, "too many queries per block");
     score_dense_kernel<<<grid, kScoreThreads, smem, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+    if (topk > 0) {
+      if (topk <= 16) topk_kernel<16><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+      else topk_kernel<32><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+    }
+  }
+  return TQ_OK;
+}
+
+// ---- outlier-channel split ----
+static tq_status check_split(const tq_split* sp) {
+  if (!sp) return fail(TQ_ERR_INVALID_ARG, "split descriptor is NULL");
+  if (sp->n_groups < 1 || sp->n_groups > TQ_MAX_GROUPS)
+    return fail(TQ_ERR_INVALID_ARG, "n_groups must be 1..%d", TQ_MAX_GROUPS);
+  int64_t total = 0;
+  for (int g = 0; g < sp->n_groups; ++g) {
+    const tq_quantizer* q = sp->groups[g];
+    const tq_status s = check_quantizer(q);
+    if (s != TQ_OK) return s;
+    if (q->kind != TQ_KIND_MSE && q->kind != TQ_KIND_PROD)
+      return fail(TQ_ERR_UNSUPPORTED, "split groups are MSE or PROD instances");
+    if (!sp->cols[g]) return fail(TQ_ERR_INVALID_ARG, "cols[%d] is NULL", g);
+    if (reinterpret_cast<uintptr_t>(sp->cols[g]) & 3u) return fail(TQ_ERR_ALIGNMENT, "cols[%d] not 4-byte aligned", g);
+    total += q->d;
+  }
+  if (total != sp->d) return fail(TQ_ERR_INVALID_ARG, "the groups' widths add up to %lld, not d = %d",
+                                  static_cast<long long>(total), sp->d);
+  return TQ_OK;
+}
+
+tq_status tq_quantize_split(const tq_split* sp, const void* x, int32_t dtype, int64_t n, const tq_packed* out,
+                            tq_stream stream) {
+  tq_status s = check_split(sp);
+  if (s != TQ_OK) return s;
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return TQ_OK;
+  // every group's outputs must be disjoint from the other groups' (checked as inputs)
+  Range others[4 * TQ_MAX_GROUPS];
+  for (int g = 0; g < sp->n_groups; ++g) {
+    int k = 0;
+    for (int h = 0; h < sp->n_groups; ++h) {
+      if (h == g) continue;
+      if ((s = check_packed(out[h], layout_of(sp->groups[h]))) != TQ_OK) return s;
+      packed_ranges(out[h], layout_of(sp->groups[h]), n, others + k);
+      k += 4;
+    }
+    s = quantize_common(sp->groups[g], x, dtype, n, out[g], reinterpret_cast<cudaStream_t>(stream),
+                        sp->groups[g]->kind, sp->d, sp->cols[g], others, k);
+    if (s != TQ_OK) return s;
+  }
+  return TQ_OK;
+}
+
+// Workspace of tq_score_split: per group the gathered rotated queries (and S q' for PROD),
+// then, for top-k, one block of summed dense scores.
+static size_t split_ws_bytes(const tq_split* sp, int64_t nq, int64_t n, int32_t topk, size_t* off_qr, size_t* off_qu,
+                             size_t* off_dense) {
+  size_t b = 0;
+  for (int g = 0; g < sp->n_groups; ++g) {
+    off_qr[g] = b;
+    b += (static_cast<size_t>(nq) * sp->groups[g]->d * 4 + 255) / 256 * 256;
+    off_qu[g] = b;
+    b += (static_cast<size_t>(nq) * score_qu_stride(sp->groups[g]) * 4 + 255) / 256 * 256;
+  }
+  *off_dense = b;
+  if (topk > 0) b += static_cast<size_t>(score_block(nq, n)) * static_cast<size_t>(n) * 4 + 256;
+  return b + 256;
+}
+
+tq_status tq_score_split_workspace(const tq_split* sp, int64_t nq, int64_t n, int32_t topk, size_t* bytes) {
+  tq_status s = check_split(sp);
+  if (s != TQ_OK) return s;
+  if (!bytes || nq < 0 || n < 0 || topk < 0) return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
+  size_t a[TQ_MAX_GROUPS], b[TQ_MAX_GROUPS], c;
+  *bytes = split_ws_bytes(sp, nq, n, topk, a, b, &c);
+  return TQ_OK;
+}
+
+tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int64_t nq, const tq_packed* keys,
+                         int64_t n, int32_t topk, float* scores, int32_t* ids, void* workspace, size_t ws_bytes,
+                         tq_stream stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  tq_status s = check_split(sp);
+  if (s != TQ_OK) return s;
+  if (!keys) return fail(TQ_ERR_INVALID_ARG, "keys is NULL");
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (nq < 0 || n < 0) return fail(TQ_ERR_INVALID_ARG, "nq, n must be >= 0");
+  if (topk < 0 || topk > 32) return fail(TQ_ERR_UNSUPPORTED, "topk must be 0..32");
+  if (topk > 0 && topk > n) return fail(TQ_ERR_INVALID_ARG, "topk > n");
+  if (n > 0x7fffffff || nq > 0x7fffffff) return fail(TQ_ERR_INVALID_ARG, "sizes too large");
+  if (nq == 0 || n == 0) return TQ_OK;
+  if (!qv || !scores || (topk > 0 && !ids)) return fail(TQ_ERR_INVALID_ARG, "NULL query or output");
+  if (!aligned16(qv) || !aligned16(scores) || (ids && !aligned16(ids)))
+    return fail(TQ_ERR_ALIGNMENT, "query/output not 16-byte aligned");
+  size_t off_qr[TQ_MAX_GROUPS], off_qu[TQ_MAX_GROUPS], off_dense;
+  const size_t need = split_ws_bytes(sp, nq, n, topk, off_qr, off_qu, &off_dense);
+  if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  Range ins[4 * TQ_MAX_GROUPS + 2];
+  int nin = 0;
+  for (int g = 0; g < sp->n_groups; ++g) {
+    const tq_layout L = layout_of(sp->groups[g]);
+    if ((s = check_packed(keys[g], L)) != TQ_OK) return s;
+    packed_ranges(keys[g], L, n, ins + nin);
+    nin += 4;
+  }
+  ins[nin++] = {qv, static_cast<size_t>(nq) * sp->d * dtype_size(dtype)};
+  ins[nin++] = {workspace, ws_bytes};
+  const Range outs[2] = {{scores, topk > 0 ? static_cast<size_t>(nq) * topk * 4 : static_cast<size_t>(nq) * n * 4},
+                         {topk > 0 ? ids : nullptr, static_cast<size_t>(nq) * topk * 4}};
+  if ((s = check_no_alias(outs, 2, ins, nin)) != TQ_OK) return s;
+
+  char* ws = static_cast<char*>(workspace);
+  int* status = device_status_ptr();
+  ScoreParams P[TQ_MAX_GROUPS];
+  size_t smem = 0;
+  cudaError_t e;
+  for (int g = 0; g < sp->n_groups; ++g) {
+    const tq_quantizer* q = sp->groups[g];
+    const int qus = score_qu_stride(q);
+    float* qr = reinterpret_cast<float*>(ws + off_qr[g]);
+    float* qu = qus ? reinterpret_cast<float*>(ws + off_qu[g]) : nullptr;
+    score_qprep_kernel<<<static_cast<unsigned>(nq), 128, 2 * q->d * 4, stream>>>(
+        qv, dtype, q->d, q->kind, q->rot, q->S, q->m, q->k_top, qr, qu, qus, sp->d, sp->cols[g], status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score qprep launch");
+    P[g] = score_params(q, layout_of(q), keys[g], n);
+    P[g].qr = qr;
+    P[g].qu = qu;
+    P[g].accumulate = g > 0;
+    smem = std::max(smem, score_smem(P[g]));
+  }
+  e = cudaFuncSetAttribute(score_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "score attribute");
+  float* dense = reinterpret_cast<float*>(ws + off_dense);
+  const int64_t qb = topk > 0 ? score_block(nq, n) : nq;
+  for (int64_t q0 = 0; q0 < nq; q0 += qb) {
+    const int64_t nb = std::min(qb, nq - q0);
+    const dim3 grid(static_cast<unsigned>((n + kScoreThreads - 1) / kScoreThreads),
+                    static_cast<unsigned>((nb + kScoreQT - 1) / kScoreQT));
+    if (grid.y > 65535) return fail(TQ_ERR_UNSUPPORTED, "too many queries per block");
+    for (int g = 0; g < sp->n_groups; ++g) {
+      ScoreParams p = P[g];
+      const int d = sp->groups[g]->d;
+      p.qr = P[g].qr + q0 * d;
+      p.qu = P[g].qu ? P[g].qu + q0 * score_qu_stride(sp->groups[g]) : nullptr;
+      p.nq = nb;
+      p.out = topk > 0 ? dense : scores + q0 * n;
+      score_dense_kernel<<<grid, kScoreThreads, score_smem(p), stream>>>(p);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+    }
     if (topk > 0) {
       if (topk <= 16) topk_kernel<16><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
       else topk_kernel<32><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);

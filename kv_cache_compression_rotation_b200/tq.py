@@ -31,7 +31,7 @@ EXPORTS = [
     "tq_spectral_unit_codebooks", "tq_record_layout", "tq_quantize_mse", "tq_quantize_prod",
     "tq_quantize_spectral", "tq_dequantize", "tq_score_workspace", "tq_score",
     "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
-    "tq_decode_attn_fixed_ws",
+    "tq_decode_attn_fixed_ws", "tq_quantize_split", "tq_score_split_workspace", "tq_score_split",
 ]
 
 
@@ -54,6 +54,14 @@ class Quantizer_t(C.Structure):
 
 class Packed_t(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("signs", C.c_void_p), ("norms", C.c_void_p), ("rnorms", C.c_void_p)]
+
+
+MAX_GROUPS = 4
+
+
+class Split_t(C.Structure):
+    _fields_ = [("n_groups", C.c_int32), ("d", C.c_int32),
+                ("groups", C.POINTER(Quantizer_t) * MAX_GROUPS), ("cols", C.c_void_p * MAX_GROUPS)]
 
 
 class Layout_t(C.Structure):
@@ -96,6 +104,10 @@ def lib():
             "tq_get_status": ([vp], C.c_int),
             "tq_set_wait_limit": ([i64], C.c_int),
             "tq_lut_scale": ([f64p, i32, C.POINTER(C.c_float)], C.c_int),
+            "tq_quantize_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), vp], C.c_int),
+            "tq_score_split_workspace": ([C.POINTER(Split_t), i64, i64, i32, C.POINTER(C.c_size_t)], C.c_int),
+            "tq_score_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), i64, i32, vp, vp, vp,
+                                C.c_size_t, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -303,6 +315,56 @@ def score(q: Quantizer, qv, packed: Packed, n: int, topk: int = 0, stream=None):
         ids = torch.empty((nq, topk), dtype=torch.int32, device=qv.device)
     _check(lib().tq_score(q.ref, qv.data_ptr(), _dtype_code(qv), nq, packed.as_c(), n, topk, scores.data_ptr(),
                           _dptr(ids), work.data_ptr(), ws.value, _stream(stream)))
+    return scores if topk == 0 else (scores, ids)
+
+
+class Split:
+    """Outlier-channel split: group g is the quantizer ``groups[g]`` over the channels
+    ``cols[g]`` (int32 CUDA tensor) of d-wide vectors."""
+
+    def __init__(self, d: int, groups, cols):
+        assert 1 <= len(groups) == len(cols) <= MAX_GROUPS
+        self.d, self.groups, self.cols = d, list(groups), list(cols)
+        gp = (C.POINTER(Quantizer_t) * MAX_GROUPS)(*[C.pointer(q.c) for q in self.groups])
+        cp = (C.c_void_p * MAX_GROUPS)(*[_dptr(c) for c in self.cols])
+        self.c = Split_t(len(self.groups), d, gp, cp)
+
+    @property
+    def ref(self):
+        return C.byref(self.c)
+
+    def alloc(self, n: int, device="cuda"):
+        return [q.alloc(n, device) for q in self.groups]
+
+
+def _packed_array(packs):
+    return (Packed_t * len(packs))(*[p.as_c() for p in packs])
+
+
+def quantize_split(sp: Split, x, out=None, stream=None):
+    """tq_quantize_split of x [n, d]: one list entry of packed records per group."""
+    assert x.is_cuda and x.is_contiguous() and x.shape[-1] == sp.d
+    n = x.numel() // sp.d
+    out = sp.alloc(n, x.device) if out is None else out
+    _check(lib().tq_quantize_split(sp.ref, x.data_ptr(), _dtype_code(x), n, _packed_array(out), _stream(stream)))
+    return out
+
+
+def score_split(sp: Split, qv, packs, n: int, topk: int = 0, stream=None):
+    """Summed split estimates [nq, n], or (scores, ids) of the top-k when topk > 0."""
+    import torch
+    nq = qv.numel() // sp.d
+    ws = C.c_size_t(0)
+    _check(lib().tq_score_split_workspace(sp.ref, nq, n, topk, C.byref(ws)))
+    work = torch.empty(max(ws.value, 16), dtype=torch.uint8, device=qv.device)
+    if topk == 0:
+        scores = torch.empty((nq, n), dtype=torch.float32, device=qv.device)
+        ids = None
+    else:
+        scores = torch.empty((nq, topk), dtype=torch.float32, device=qv.device)
+        ids = torch.empty((nq, topk), dtype=torch.int32, device=qv.device)
+    _check(lib().tq_score_split(sp.ref, qv.data_ptr(), _dtype_code(qv), nq, _packed_array(packs), n, topk,
+                                scores.data_ptr(), _dptr(ids), work.data_ptr(), ws.value, _stream(stream)))
     return scores if topk == 0 else (scores, ids)
 
 

@@ -225,3 +225,42 @@ def test_lut_scale_tightens_half_precision_codebook(lib, bits):
     plain = np.max(np.abs(c.astype(np.float16).astype(np.float64) - c) / np.abs(c))
     scaled = np.max(np.abs((c / s).astype(np.float16).astype(np.float64) * s - c) / np.abs(c))
     assert scaled <= min(plain, 1.5e-4)
+
+
+def _split(groups, cols, d):
+    sp = T.Split_t()
+    sp.n_groups, sp.d = len(groups), d
+    for i, (q, c) in enumerate(zip(groups, cols)):
+        sp.groups[i] = C.pointer(q)
+        sp.cols[i] = c
+    return sp
+
+
+def test_split_validation_before_launch(lib):
+    qa, qb = _q(T.KIND_MSE, d=32, bits=3), _q(T.KIND_MSE, d=96, bits=2)
+    pks = (T.Packed_t * 2)(T.Packed_t(FAKE + 0x100000, None, FAKE + 0x200000, None),
+                           T.Packed_t(FAKE + 0x400000, None, FAKE + 0x500000, None))
+    x = FAKE + 0x700000
+    ok = _split([qa, qb], [FAKE + 0x800000, FAKE + 0x810000], 128)
+    assert lib.tq_quantize_split(C.byref(ok), x, 1, 0, pks, None) == 0            # n == 0: no launch
+    # widths that do not add up to d
+    assert lib.tq_quantize_split(C.byref(_split([qa, qb], [FAKE, FAKE], 127)), x, 1, 10, pks, None) == 1
+    # a NULL or misaligned channel list
+    assert lib.tq_quantize_split(C.byref(_split([qa, qb], [FAKE, None], 128)), x, 1, 10, pks, None) == 1
+    assert lib.tq_quantize_split(C.byref(_split([qa, qb], [FAKE, FAKE + 2], 128)), x, 1, 10, pks, None) == 3
+    # no groups, too many groups, a spectral group
+    assert lib.tq_quantize_split(C.byref(_split([], [], 128)), x, 1, 10, pks, None) == 1
+    sp = _split([qa, qb], [FAKE, FAKE], 128)
+    sp.n_groups = T.MAX_GROUPS + 1
+    assert lib.tq_quantize_split(C.byref(sp), x, 1, 10, pks, None) == 1
+    qs = _q(T.KIND_SPECTRAL, d=96, k_top=4, top_bits=[5, 3, 2, 2], tail_bits=1, dim_sigma=FAKE, unit_c=FAKE,
+            unit_t=FAKE)
+    assert lib.tq_quantize_split(C.byref(_split([qa, qs], [FAKE, FAKE], 128)), x, 1, 10, pks, None) == 2
+    # two groups writing into overlapping records
+    same = (T.Packed_t * 2)(pks[0], pks[0])
+    assert lib.tq_quantize_split(C.byref(ok), x, 1, 10, same, None) == 4
+    # score: workspace query, then a too-small workspace
+    ws = C.c_size_t(0)
+    assert lib.tq_score_split_workspace(C.byref(ok), 4, 1000, 10, C.byref(ws)) == 0 and ws.value > 4 * 128 * 4
+    assert lib.tq_score_split(C.byref(ok), FAKE + 0x900000, 0, 4, pks, 1000, 10, FAKE + 0xA00000,
+                              FAKE + 0xB00000, FAKE + 0xC00000, 16, None) == 8
