@@ -508,6 +508,33 @@ def run_other(args):
         desc = (f"search: {ndb} x 1536 fp32 unit vectors, prod b={args.c5_bits} (m=1536), "
                 f"top-10 of {nq5} queries")
         value, unit, step_ms = ndb / tq * 1e3, "vectors/s", tq
+    elif wl == "split":
+        # outlier-channel split of the KV setting: 32 channels at 3 bits + 96 at 2 bits
+        # (mse instances), keys with 32 planted high-magnitude channels whose list is given
+        # (a precomputed per-model list); quantize and dense estimates for 32 queries
+        n, nq = 8 * 32768, 32
+        planted = np.sort(np.random.Generator(np.random.PCG64(ti.SEEDS["basis"] + 6)).choice(Dm, 32, replace=False))
+        rest = np.setdiff1d(np.arange(Dm), planted)
+        x = ti.normal_torch((n, Dm), ti.SEEDS["keys"] + 6, dev)
+        x[:, torch.from_numpy(planted).to(dev)] *= 6.0
+        x = x.to(torch.bfloat16).contiguous()
+        qq = ti.normal_torch((nq, Dm), ti.SEEDS["queries"] + 6, dev)
+        groups = [K.Quantizer.mse(ti.haar_rotation(32, ti.SEEDS["rotation"] + 32), 3, device=dev),
+                  K.Quantizer.mse(ti.haar_rotation(96, ti.SEEDS["rotation"] + 96), 2, device=dev)]
+        cols = [torch.from_numpy(c.astype(np.int32)).to(dev) for c in (planted, rest)]
+        sp = K.Split(Dm, groups, cols)
+        out = sp.alloc(n, dev)
+        tq = _timed(lambda: K.quantize_split(sp, x, out), stream, flush)
+        ts = _timed(lambda: K.score_split(sp, qq, out, n), stream, flush)
+        assert K.get_status() == 0
+        rec = sum(4 * (L.code_words + L.has_norms) for L in (g.layout() for g in groups))
+        parts = {"quantize_split": {"ms": tq, "vectors_per_s": n / tq * 1e3, "gbs": n * (Dm * 2 + rec) / tq / 1e6,
+                                    "record_bytes": rec},
+                 "score_split": {"ms": ts, "estimates_per_s": nq * n / ts * 1e3,
+                                 "gbs": n * rec / ts / 1e6}}
+        desc = (f"outlier split: {n} bf16 keys d=128 with 32 planted channels (x6), groups 32 @ 3 bits + "
+                f"96 @ 2 bits (mse), dense estimates for {nq} queries (CUDA-core kernels)")
+        value, unit, step_ms = n / tq * 1e3, "vectors/s", tq
     else:
         raise SystemExit(f"unknown workload {wl}")
     return {"metric": f"{wl} secondary workload", "value": value, "unit": unit, "n_gpus": 1, "steps": 10,
@@ -532,7 +559,7 @@ def main():
                     help="profiling aid: context length (the headline workload uses 131072)")
     ap.add_argument("--batch", type=int, default=B,
                     help="profiling aid: batch size (the headline workload uses 8)")
-    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5"],
+    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5", "split"],
                     help="c3 (default): the 128k decode step of the headline; the others are the scope "
                          "table's secondary workloads, timed per kernel")
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
