@@ -258,6 +258,28 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
                          const tq_packed* keys, int64_t n, int32_t topk, float* scores,
                          int32_t* ids, void* workspace, size_t ws_bytes, tq_stream stream);
 
+/* Workspace bytes needed by tq_decode_attn_split for this shape. */
+tq_status tq_decode_attn_split_workspace(const tq_split* ks, const tq_split* vs, int32_t B,
+                                         int32_t Hq, int32_t Hkv, int64_t Nmax, size_t* bytes);
+
+/*
+ * DEVICE.  One decode-attention step over split caches (keys split by ks, values by vs;
+ * the splits may differ but have the same width d):
+ *   logit_i = scale * sum_g ||k_i,g|| <rot_g q[cols_g], c_g[code_i,g]>,  p = softmax(logit),
+ *   out[cols_g] = rot_g^T sum_i p_i ||v_i,g|| c_g[code_i,g]   for every value group g,
+ * over the first seq_lens[b] records of each (b, kv-head) row; query head h reads KV head
+ * h / (Hq/Hkv).  q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), kcache/vcache
+ * host arrays of one packed descriptor per group, each group's records laid out
+ * [B][Hkv][Nmax]; out [B*Hq*d] fp32.  This build runs MSE groups, d <= 256 and
+ * Hq/Hkv <= 8 on CUDA cores (TQ_ERR_UNSUPPORTED otherwise).  A value channel index out of
+ * range sets TQ_ERR_INVALID_ARG on the device and its output is not written.
+ */
+tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const void* q,
+                               int32_t dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,
+                               const int32_t* seq_lens, const tq_packed* kcache,
+                               const tq_packed* vcache, float scale, float* out, void* workspace,
+                               size_t ws_bytes, tq_stream stream);
+
 /*
  * DEVICE.  Reconstruction out [n*d] fp32: MSE x_hat = ||x|| rot^T c[code];
  * PROD adds ||x|| rot^T (sqrt(pi/2)/m ||r|| S^T (2s-1)) (unbiased);

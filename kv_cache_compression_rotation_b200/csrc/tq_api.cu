@@ -14,6 +14,7 @@
 
 #include "decode.cuh"
 #include "decode_aux.cuh"
+#include "decode_split.cuh"
 #include "decode_tma.cuh"
 #include "device_common.cuh"
 #include "launchers.h"
@@ -738,6 +739,149 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
     }
   }
   return TQ_OK;
+}
+
+// ---- decode attention over a split cache ----
+struct SplitDecodePlan {
+  int chunk_len, n_chunks;
+  size_t off_qr[TQ_MAX_GROUPS], off_ml, off_o, bytes;
+};
+
+static SplitDecodePlan plan_split_decode(const tq_split* ks, int B, int Hq, int64_t Nmax) {
+  SplitDecodePlan P{};
+  // at most 64 chunks per row: the partials stay small and the combine's weights fit in
+  // shared memory; chunks of at least 256 tokens
+  int64_t cl = (Nmax + 63) / 64;
+  cl = std::max<int64_t>(256, (cl + 31) / 32 * 32);
+  P.chunk_len = static_cast<int>(std::min<int64_t>(cl, 1 << 30));
+  P.n_chunks = static_cast<int>((Nmax + P.chunk_len - 1) / P.chunk_len);
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  size_t b = 0;
+  for (int g = 0; g < ks->n_groups; ++g) {
+    P.off_qr[g] = b;
+    b += (rows * ks->groups[g]->d * 4 + 255) / 256 * 256;
+  }
+  P.off_ml = b;
+  b += (rows * P.n_chunks * 2 * 4 + 255) / 256 * 256;
+  P.off_o = b;
+  b += (rows * P.n_chunks * static_cast<size_t>(ks->d) * 4 + 255) / 256 * 256;
+  P.bytes = b + 256;
+  return P;
+}
+
+static tq_status check_split_decode(const tq_split* ks, const tq_split* vs, int B, int Hq, int Hkv, int64_t Nmax) {
+  tq_status s = check_split(ks);
+  if (s != TQ_OK) return s;
+  if ((s = check_split(vs)) != TQ_OK) return s;
+  if (ks->d != vs->d) return fail(TQ_ERR_INVALID_ARG, "key and value splits have different widths");
+  if (ks->d > kSplitMaxD) return fail(TQ_ERR_UNSUPPORTED, "split decode runs d <= %d", kSplitMaxD);
+  for (int g = 0; g < ks->n_groups; ++g)
+    if (ks->groups[g]->kind != TQ_KIND_MSE) return fail(TQ_ERR_UNSUPPORTED, "split decode runs MSE key groups");
+  for (int g = 0; g < vs->n_groups; ++g)
+    if (vs->groups[g]->kind != TQ_KIND_MSE) return fail(TQ_ERR_UNSUPPORTED, "split decode runs MSE value groups");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nmax < 1) return fail(TQ_ERR_INVALID_ARG, "B, Hq, Hkv, Nmax must be >= 1");
+  if (Hq % Hkv) return fail(TQ_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (Hq / Hkv > kSplitMaxG) return fail(TQ_ERR_UNSUPPORTED, "Hq/Hkv > %d", kSplitMaxG);
+  if (static_cast<int64_t>(B) * Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "B*Hkv > 65535");
+  if (Nmax > (1ll << 30)) return fail(TQ_ERR_INVALID_ARG, "Nmax too large");
+  return TQ_OK;
+}
+
+tq_status tq_decode_attn_split_workspace(const tq_split* ks, const tq_split* vs, int32_t B, int32_t Hq, int32_t Hkv,
+                                         int64_t Nmax, size_t* bytes) {
+  tq_status s = check_split_decode(ks, vs, B, Hq, Hkv, Nmax);
+  if (s != TQ_OK) return s;
+  if (!bytes) return fail(TQ_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = plan_split_decode(ks, B, Hq, Nmax).bytes;
+  return TQ_OK;
+}
+
+tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const void* q, int32_t dtype, int32_t B,
+                               int32_t Hq, int32_t Hkv, int64_t Nmax, const int32_t* seq_lens,
+                               const tq_packed* kcache, const tq_packed* vcache, float scale, float* out,
+                               void* workspace, size_t ws_bytes, tq_stream stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  tq_status s = check_split_decode(ks, vs, B, Hq, Hkv, Nmax);
+  if (s != TQ_OK) return s;
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (!q || !seq_lens || !out || !kcache || !vcache) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(q) || !aligned16(seq_lens) || !aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "q/seq_lens/out alignment");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
+  const SplitDecodePlan P = plan_split_decode(ks, B, Hq, Nmax);
+  if (!workspace || ws_bytes < P.bytes) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", P.bytes);
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  const int64_t recs = static_cast<int64_t>(B) * Hkv * Nmax;
+  const int d = ks->d, G = Hq / Hkv, rows = B * Hq;
+  Range ins[8 * TQ_MAX_GROUPS + 3];
+  int nin = 0;
+  for (int g = 0; g < ks->n_groups; ++g) {
+    const tq_layout L = layout_of(ks->groups[g]);
+    if ((s = check_packed(kcache[g], L)) != TQ_OK) return s;
+    packed_ranges(kcache[g], L, recs, ins + nin);
+    nin += 4;
+  }
+  for (int g = 0; g < vs->n_groups; ++g) {
+    const tq_layout L = layout_of(vs->groups[g]);
+    if ((s = check_packed(vcache[g], L)) != TQ_OK) return s;
+    packed_ranges(vcache[g], L, recs, ins + nin);
+    nin += 4;
+  }
+  ins[nin++] = {q, static_cast<size_t>(rows) * d * dtype_size(dtype)};
+  ins[nin++] = {seq_lens, static_cast<size_t>(B) * 4};
+  ins[nin++] = {workspace, ws_bytes};
+  const Range outs[1] = {{out, static_cast<size_t>(rows) * d * 4}};
+  if ((s = check_no_alias(outs, 1, ins, nin)) != TQ_OK) return s;
+
+  char* ws = static_cast<char*>(workspace);
+  int* status = device_status_ptr();
+  SplitDecodeParams dp{};
+  dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.G = G; dp.d = d; dp.Nmax = Nmax;
+  dp.chunk_len = P.chunk_len; dp.n_chunks = P.n_chunks; dp.seq_lens = seq_lens;
+  dp.nkg = ks->n_groups; dp.nvg = vs->n_groups;
+  cudaError_t e;
+  int off = 0;
+  for (int g = 0; g < ks->n_groups; ++g) {
+    const tq_quantizer* kq = ks->groups[g];
+    float* qr = reinterpret_cast<float*>(ws + P.off_qr[g]);
+    score_qprep_kernel<<<static_cast<unsigned>(rows), 128, 2 * kq->d * 4, stream>>>(
+        q, dtype, kq->d, TQ_KIND_MSE, kq->rot, nullptr, 0, 0, qr, nullptr, 0, d, ks->cols[g], status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split qprep launch");
+    const tq_layout L = layout_of(kq);
+    dp.kd[g] = kq->d; dp.kbits[g] = kq->bits; dp.kwords[g] = L.code_words; dp.koff[g] = off;
+    dp.kcodes[g] = kcache[g].codes; dp.knorms[g] = kcache[g].norms; dp.kcent[g] = kq->centroids;
+    dp.qr[g] = qr;
+    off += kq->d;
+  }
+  off = 0;
+  for (int g = 0; g < vs->n_groups; ++g) {
+    const tq_quantizer* vq = vs->groups[g];
+    const tq_layout L = layout_of(vq);
+    dp.vd[g] = vq->d; dp.vbits[g] = vq->bits; dp.vwords[g] = L.code_words; dp.voff[g] = off;
+    dp.vcodes[g] = vcache[g].codes; dp.vnorms[g] = vcache[g].norms; dp.vcent[g] = vq->centroids;
+    off += vq->d;
+  }
+  dp.logit_scale = static_cast<float>(scale * kLog2e);
+  dp.part_ml = reinterpret_cast<float*>(ws + P.off_ml);
+  dp.part_o = reinterpret_cast<float*>(ws + P.off_o);
+  const size_t smem = split_decode_smem(G, d);
+  e = cudaFuncSetAttribute(split_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "split decode attribute");
+  split_decode_kernel<<<dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv)), kSplitDecThreads,
+                        smem, stream>>>(dp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split decode launch");
+
+  SplitCombineParams cp{};
+  cp.rows = rows; cp.d = d; cp.n_chunks = P.n_chunks; cp.nvg = vs->n_groups;
+  off = 0;
+  for (int g = 0; g < vs->n_groups; ++g) {
+    cp.vd[g] = vs->groups[g]->d; cp.voff[g] = off; cp.vrot[g] = vs->groups[g]->rot; cp.vcols[g] = vs->cols[g];
+    off += vs->groups[g]->d;
+  }
+  cp.status = status;
+  cp.part_ml = dp.part_ml; cp.part_o = dp.part_o; cp.out = out;
+  split_combine_kernel<<<static_cast<unsigned>(rows), 128, static_cast<size_t>(P.n_chunks + d) * 4, stream>>>(cp);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "split combine launch");
 }
 
 tq_status tq_decode_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,

@@ -32,6 +32,7 @@ EXPORTS = [
     "tq_quantize_spectral", "tq_dequantize", "tq_score_workspace", "tq_score",
     "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
     "tq_decode_attn_fixed_ws", "tq_quantize_split", "tq_score_split_workspace", "tq_score_split",
+    "tq_decode_attn_split_workspace", "tq_decode_attn_split",
 ]
 
 
@@ -108,6 +109,11 @@ def lib():
             "tq_score_split_workspace": ([C.POINTER(Split_t), i64, i64, i32, C.POINTER(C.c_size_t)], C.c_int),
             "tq_score_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), i64, i32, vp, vp, vp,
                                 C.c_size_t, vp], C.c_int),
+            "tq_decode_attn_split_workspace": ([C.POINTER(Split_t), C.POINTER(Split_t), i32, i32, i32, i64,
+                                                C.POINTER(C.c_size_t)], C.c_int),
+            "tq_decode_attn_split": ([C.POINTER(Split_t), C.POINTER(Split_t), vp, i32, i32, i32, i32, i64, vp,
+                                      C.POINTER(Packed_t), C.POINTER(Packed_t), C.c_float, vp, vp, C.c_size_t,
+                                      vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -366,6 +372,23 @@ def score_split(sp: Split, qv, packs, n: int, topk: int = 0, stream=None):
     _check(lib().tq_score_split(sp.ref, qv.data_ptr(), _dtype_code(qv), nq, _packed_array(packs), n, topk,
                                 scores.data_ptr(), _dptr(ids), work.data_ptr(), ws.value, _stream(stream)))
     return scores if topk == 0 else (scores, ids)
+
+
+def decode_attn_split(ks: Split, vs: Split, q, seq_lens, kpacks, vpacks, Nmax: int, Hkv: int, scale=None,
+                      out=None, stream=None):
+    """tq_decode_attn_split for q [B, Hq, d] over split caches (one packed list per split)."""
+    import torch
+    B, Hq, d = q.shape
+    assert d == ks.d == vs.d and q.is_contiguous()
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    ws = C.c_size_t(0)
+    _check(lib().tq_decode_attn_split_workspace(ks.ref, vs.ref, B, Hq, Hkv, Nmax, C.byref(ws)))
+    work = torch.empty(max(ws.value, 16), dtype=torch.uint8, device=q.device)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device) if out is None else out
+    _check(lib().tq_decode_attn_split(ks.ref, vs.ref, q.data_ptr(), _dtype_code(q), B, Hq, Hkv, Nmax,
+                                      seq_lens.data_ptr(), _packed_array(kpacks), _packed_array(vpacks),
+                                      float(scale), out.data_ptr(), work.data_ptr(), ws.value, _stream(stream)))
+    return out
 
 
 def decode_workspace_bytes(kq: Quantizer, B: int, Hq: int, Hkv: int, Nmax: int) -> int:

@@ -8,12 +8,13 @@ import numpy as np
 import pytest
 
 import tq_inputs as ti
+from oracle import attention as OA
 from oracle import quantizer as OQ
 from oracle import split as OS
 from oracle.codebook import lloyd_max
 from oracle.search import topk as otopk
 
-from _parity import as_u32, code_mismatches, sign_mismatches
+from _parity import as_u32, code_mismatches, rel_rows, sign_mismatches
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -131,3 +132,46 @@ def test_bad_channel_index_reports_status():
     torch.cuda.synchronize()
     assert K.get_status() == 1                            # TQ_ERR_INVALID_ARG
     assert K.get_status() == 0
+
+
+def _records_from_gpu(packs, groups, ins):
+    """The GPU's own records as oracle record dicts (codes unpacked, fp32 norms)."""
+    recs = []
+    for pk, ch, g in zip(packs, groups, ins):
+        idx = OQ.unpack_codes(as_u32(pk.codes), len(ch), g["bits"])
+        recs.append({"idx": idx, "norms": pk.norms.cpu().numpy().astype(np.float64)})
+    return recs
+
+
+@pytest.mark.parametrize("B,Hkv,Hq,Nmax,lens", [(2, 2, 8, 700, [700, 333]), (1, 4, 8, 3000, [2999]),
+                                                 (3, 1, 1, 300, [1, 300, 17])])
+def test_decode_attn_split_parity(B, Hkv, Hq, Nmax, lens):
+    # the attention step read straight from split caches against the oracle's split
+    # attention on the same records (keys with planted outlier channels, 32 @ 3 b + 96 @ 2 b
+    # for keys and values)
+    n = B * Hkv * Nmax
+    kx, k64, groups, ins, ks = _setup("mse", n, 4700 + Nmax)
+    vx64 = ti.iid_normal((n, D), 4800 + Nmax)
+    vxt, vx64 = ti.to_bf16_f64(vx64)
+    vx = vxt.cuda().contiguous()
+    vs = ks                                                # the same split for the values
+    kp = K.quantize_split(ks, kx)
+    vp = K.quantize_split(vs, vx)
+    q64 = ti.iid_normal((B, Hq, D), 4900 + Nmax)
+    q = torch.from_numpy(q64.astype(np.float32)).cuda()
+    seq = torch.tensor(lens, dtype=torch.int32).cuda()
+    o = K.decode_attn_split(ks, vs, q, seq, kp, vp, Nmax, Hkv).cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    assert K.get_status() == 0
+    kr, vr = _records_from_gpu(kp, groups, ins), _records_from_gpu(vp, groups, ins)
+
+    def rows(recs, b, h, n_):
+        base = (b * Hkv + h) * Nmax
+        return [{"idx": r["idx"][base:base + n_], "norms": r["norms"][base:base + n_]} for r in recs]
+
+    scale = 1.0 / np.sqrt(D)
+    ref = OA.decode_attention(q.cpu().numpy().astype(np.float64), lens, Hkv,
+                              lambda b, h, qs: OS.estimate_split(qs, rows(kr, b, h, lens[b]), groups, ins),
+                              lambda b, h, n_: OS.dequantize_split(rows(vr, b, h, n_), groups, ins, D), scale)
+    err = rel_rows(o, ref)
+    assert np.all(err <= 1e-3), f"max row error {err.max():.2e}"
