@@ -526,14 +526,23 @@ def run_other(args):
         out = sp.alloc(n, dev)
         tq = _timed(lambda: K.quantize_split(sp, x, out), stream, flush)
         ts = _timed(lambda: K.score_split(sp, qq, out, n), stream, flush)
+        # decode step over split K and V caches: B=1, Hkv=8, Hq=32, context 32768 (the same
+        # records serve as keys and values)
+        Bd, Hkvd, Hqd, Nd = 1, 8, 32, 32768
+        qd = ti.normal_torch((Bd, Hqd, Dm), ti.SEEDS["queries"] + 7, dev)
+        seqd = torch.full((Bd,), Nd, dtype=torch.int32, device=dev)
+        td = _timed(lambda: K.decode_attn_split(sp, sp, qd, seqd, out, out, Nd, Hkvd), stream, flush)
         assert K.get_status() == 0
         rec = sum(4 * (L.code_words + L.has_norms) for L in (g.layout() for g in groups))
         parts = {"quantize_split": {"ms": tq, "vectors_per_s": n / tq * 1e3, "gbs": n * (Dm * 2 + rec) / tq / 1e6,
                                     "record_bytes": rec},
                  "score_split": {"ms": ts, "estimates_per_s": nq * n / ts * 1e3,
-                                 "gbs": n * rec / ts / 1e6}}
+                                 "gbs": n * rec / ts / 1e6},
+                 "decode_attn_split": {"ms": td, "gbs": n * 2 * rec / td / 1e6,
+                                       "frac": n * 2 * rec / td / 1e6 / peak, "bytes_per_token": 2 * rec}}
         desc = (f"outlier split: {n} bf16 keys d=128 with 32 planted channels (x6), groups 32 @ 3 bits + "
-                f"96 @ 2 bits (mse), dense estimates for {nq} queries (CUDA-core kernels)")
+                f"96 @ 2 bits (mse), dense estimates for {nq} queries, decode B=1 Hkv=8 Hq=32 over 32768 "
+                f"tokens (CUDA-core kernels)")
         value, unit, step_ms = n / tq * 1e3, "vectors/s", tq
     else:
         raise SystemExit(f"unknown workload {wl}")
