@@ -264,3 +264,30 @@ def test_split_validation_before_launch(lib):
     assert lib.tq_score_split_workspace(C.byref(ok), 4, 1000, 10, C.byref(ws)) == 0 and ws.value > 4 * 128 * 4
     assert lib.tq_score_split(C.byref(ok), FAKE + 0x900000, 0, 4, pks, 1000, 10, FAKE + 0xA00000,
                               FAKE + 0xB00000, FAKE + 0xC00000, 16, None) == 8
+
+
+def test_split_decode_validation_before_launch(lib):
+    qa, qb = _q(T.KIND_MSE, d=32, bits=3), _q(T.KIND_MSE, d=96, bits=2)
+    sp = _split([qa, qb], [FAKE + 0x800000, FAKE + 0x810000], 128)
+    ws = C.c_size_t(0)
+    assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp), 2, 8, 2, 1000, C.byref(ws)) == 0
+    assert ws.value >= 2 * 8 * 128 * 4                               # at least the rotated queries
+    # GQA group too large, Hq not a multiple of Hkv, a prod group, mismatched widths
+    assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp), 1, 16, 1, 1000, C.byref(ws)) == 2
+    assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp), 1, 6, 4, 1000, C.byref(ws)) == 1
+    qp = _q(T.KIND_PROD, d=96, bits=3, m=96, S=FAKE)
+    spp = _split([qa, qp], [FAKE, FAKE], 128)
+    assert lib.tq_decode_attn_split_workspace(C.byref(spp), C.byref(sp), 1, 8, 1, 1000, C.byref(ws)) == 2
+    q64 = _q(T.KIND_MSE, d=64, bits=2)
+    sp96 = _split([qa, q64], [FAKE, FAKE], 96)
+    assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp96), 1, 8, 1, 1000, C.byref(ws)) == 1
+    # wider than this build
+    big = _split([_q(T.KIND_MSE, d=200, bits=2), _q(T.KIND_MSE, d=100, bits=2)], [FAKE, FAKE], 300)
+    assert lib.tq_decode_attn_split_workspace(C.byref(big), C.byref(big), 1, 8, 1, 1000, C.byref(ws)) == 2
+    # a workspace that is too small fails before any launch
+    pk = (T.Packed_t * 2)(T.Packed_t(FAKE + 0x100000, None, FAKE + 0x200000, None),
+                          T.Packed_t(FAKE + 0x300000, None, FAKE + 0x400000, None))
+    pv = (T.Packed_t * 2)(T.Packed_t(FAKE + 0x500000, None, FAKE + 0x600000, None),
+                          T.Packed_t(FAKE + 0x700000, None, FAKE + 0x780000, None))
+    assert lib.tq_decode_attn_split(C.byref(sp), C.byref(sp), FAKE + 0x900000, 1, 2, 8, 2, 1000, FAKE + 0xA00000,
+                                    pk, pv, C.c_float(0.1), FAKE + 0xB00000, FAKE + 0xC00000, 16, None) == 8
