@@ -30,6 +30,8 @@ Modules:
 * :mod:`oracle.search`    -- exhaustive top-k by estimated inner product.
 * :mod:`oracle.split`     -- outlier-channel split: independent TurboQuant instances
   on channel groups (online outlier detection, per-group quantize, summed estimates).
+* :mod:`oracle.sweep`     -- inner-product distortion of the mse and prod variants by
+  bit width (bias and total), on correlated query/key pairs.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against closed forms,
 printed values, brute force or library routines, except where its docstring says
