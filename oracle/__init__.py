@@ -32,6 +32,8 @@ Modules:
   on channel groups (online outlier detection, per-group quantize, summed estimates).
 * :mod:`oracle.sweep`     -- inner-product distortion of the mse and prod variants by
   bit width (bias and total), on correlated query/key pairs.
+* :mod:`oracle.serving`   -- paged-cache slots, and causal prefill attention over the
+  quantized cache (append-then-attend is the quantize and decode steps in sequence).
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against closed forms,
 printed values, brute force or library routines, except where its docstring says
