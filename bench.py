@@ -386,8 +386,12 @@ def run_reference(args, rank, world):
     val = float(np.mean([s["value"] for s in steps]))
     cb = dict(steps[-1])
     cb["value"] = val
+    # one full step of the workload (two quantize launches and the decode) at that rate
+    _, q_bytes, dec_bytes = algorithmic_bytes()
+    ms_step = (2 * q_bytes + dec_bytes) / (val * 1e9) * 1e3
     return {"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "decode-128k (bounded sample on host cores; see cpu_baseline.sample)",
                        "global_batch": B, "seq_len": N, "parallelism": "none"},
