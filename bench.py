@@ -421,6 +421,33 @@ def _timed(fn, stream, flush=None, reps=10, warm=3):
     return float(np.median(ts))
 
 
+def ip_sweep(K, dev, n: int = 4096, rho: float = 0.9, bits=range(1, 6), d: int = 128):
+    """Inner-product distortion by bit width through the library's quantize and estimator
+    (tq_score, the diagonal of the pair matrix): unit keys x and queries
+    y = rho x + sqrt(1 - rho^2) z with z a unit vector orthogonal to x.  Returns
+    {bits: {kind: {mean_sq, bias_sq}}} of the errors est(y_i, x_i) - <y_i, x_i>."""
+    import torch
+    import tq_inputs as ti
+    x = ti.normal_torch((n, d), ti.SEEDS["keys"] + 9, dev, dtype=torch.float64)
+    x /= x.norm(dim=1, keepdim=True)
+    z = ti.normal_torch((n, d), ti.SEEDS["queries"] + 9, dev, dtype=torch.float64)
+    z -= (z * x).sum(1, keepdim=True) * x
+    z /= z.norm(dim=1, keepdim=True)
+    y = rho * x + math.sqrt(1.0 - rho * rho) * z
+    exact = (x * y).sum(1)
+    rot = ti.haar_rotation(d, ti.SEEDS["rotation"] + 9)
+    S = ti.gaussian_matrix(d, d, ti.SEEDS["qjl"] + 9)
+    xf, yf = x.float().contiguous(), y.float().contiguous()
+    rows = {}
+    for b in bits:
+        for kind in ("mse", "prod"):
+            qz = K.Quantizer.mse(rot, b, device=dev) if kind == "mse" else K.Quantizer.prod(rot, S, b, device=dev)
+            est = K.score(qz, yf, K.quantize(qz, xf), n).diagonal().double()
+            err = est - exact
+            rows.setdefault(b, {})[kind] = {"mean_sq": float((err * err).mean()), "bias_sq": float(err.mean() ** 2)}
+    return rows
+
+
 def run_other(args):
     """Secondary workloads of the scope table (one GPU, parts timed separately, L2 flushed
     before every timed launch).  The headline line is the default 128k decode workload."""
@@ -548,6 +575,15 @@ def run_other(args):
                 f"96 @ 2 bits (mse), dense estimates for {nq} queries, decode B=1 Hkv=8 Hq=32 over 32768 "
                 f"tokens (CUDA-core kernels)")
         value, unit, step_ms = n / tq * 1e3, "vectors/s", tq
+    elif wl == "sweep":
+        n, rho = 4096, 0.9
+        rows = ip_sweep(K, dev, n, rho)
+        assert K.get_status() == 0
+        parts = {"ip_distortion": rows, "pairs": n, "rho": rho}
+        cross = [b for b in rows if rows[b]["prod"]["mean_sq"] < rows[b]["mse"]["mean_sq"]]
+        desc = (f"inner-product distortion sweep: {n} unit keys d=128, queries correlated with rho={rho}, "
+                f"mse and prod at 1..5 bits (quantize and tq_score estimates on the GPU)")
+        value, unit, step_ms = float(max(cross) if cross else 0), "bits where prod still wins (max)", 0.0
     else:
         raise SystemExit(f"unknown workload {wl}")
     return {"metric": f"{wl} secondary workload", "value": value, "unit": unit, "n_gpus": 1, "steps": 10,
@@ -572,7 +608,7 @@ def main():
                     help="profiling aid: context length (the headline workload uses 131072)")
     ap.add_argument("--batch", type=int, default=B,
                     help="profiling aid: batch size (the headline workload uses 8)")
-    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5", "split"],
+    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5", "split", "sweep"],
                     help="c3 (default): the 128k decode step of the headline; the others are the scope "
                          "table's secondary workloads, timed per kernel")
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
