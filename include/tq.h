@@ -44,7 +44,7 @@ typedef struct CUstream_st* tq_stream;
 typedef enum {
   TQ_OK = 0,
   TQ_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, inconsistent descriptor */
-  TQ_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+  TQ_ERR_UNSUPPORTED = 2,   /* valid request outside what libtq implements */
   TQ_ERR_ALIGNMENT = 3,     /* device pointer not 16-byte aligned */
   TQ_ERR_ALIAS = 4,         /* an output overlaps an input */
   TQ_ERR_CUDA = 5,          /* CUDA runtime error (message has the CUDA error string) */
@@ -270,7 +270,7 @@ tq_status tq_decode_attn_split_workspace(const tq_split* ks, const tq_split* vs,
  * over the first seq_lens[b] records of each (b, kv-head) row; query head h reads KV head
  * h / (Hq/Hkv).  q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), kcache/vcache
  * host arrays of one packed descriptor per group, each group's records laid out
- * [B][Hkv][Nmax]; out [B*Hq*d] fp32.  This build runs MSE groups, d <= 256 and
+ * [B][Hkv][Nmax]; out [B*Hq*d] fp32.  libtq runs MSE groups, d <= 256 and
  * Hq/Hkv <= 8 on CUDA cores (TQ_ERR_UNSUPPORTED otherwise).  A value channel index out of
  * range sets TQ_ERR_INVALID_ARG on the device and its output is not written.
  */
@@ -317,7 +317,7 @@ tq_status tq_decode_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq
  *   first seq_lens[b] records, p = softmax(logit), out = sum_i p_i v_hat_i.
  * q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), caches laid out
  * [B][Hkv][Nmax] records, out [B*Hq*d] fp32.  Keys: MSE, PROD or SPECTRAL; values: MSE or
- * SPECTRAL (without qjl).  This build runs d = 128, code bits <= 4, PROD m = d,
+ * SPECTRAL (without qjl).  libtq runs d = 128, code bits <= 4, PROD m = d,
  * Hq/Hkv in 1..16; other shapes give TQ_ERR_UNSUPPORTED.  Value norms must stay below
  * 6.0e4 (the probability-weighted norm is a half-precision MMA operand).  The call
  * enqueues three kernels (query preparation, decode, chunk combine); the last two use

@@ -216,7 +216,7 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   if (n == 0) return TQ_OK;
   if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
   if (!aligned16(x)) return fail(TQ_ERR_ALIGNMENT, "x is not 16-byte aligned");
-  if (q->d > 2048) return fail(TQ_ERR_UNSUPPORTED, "quantize supports d <= 2048 in this build");
+  if (q->d > 2048) return fail(TQ_ERR_UNSUPPORTED, "quantize supports d <= 2048");
   const tq_layout L = layout_of(q);
   if ((s = check_packed(out, L)) != TQ_OK) return s;
   Range outs[4];
@@ -368,7 +368,7 @@ tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int
   if (kq->d != vq->d) return fail(TQ_ERR_INVALID_ARG, "key and value d differ");
   if (Nmax > (1ll << 30)) return fail(TQ_ERR_INVALID_ARG, "Nmax too large");
   if (static_cast<int64_t>(B) * Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "B*Hkv > 65535");
-  if (kq->d != 128) return fail(TQ_ERR_UNSUPPORTED, "decode attention runs d = 128 in this build");
+  if (kq->d != 128) return fail(TQ_ERR_UNSUPPORTED, "decode attention runs d = 128 only");
   if (Hq / Hkv > 16) return fail(TQ_ERR_UNSUPPORTED, "Hq/Hkv > 16");
   if (vq->kind == TQ_KIND_PROD) return fail(TQ_ERR_UNSUPPORTED, "values as PROD are not built");
   if (vq->kind == TQ_KIND_SPECTRAL && vq->qjl) return fail(TQ_ERR_UNSUPPORTED, "spectral values with qjl");

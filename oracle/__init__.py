@@ -1,7 +1,7 @@
 """CPU oracle for the TurboQuant hot path -- TEST INFRASTRUCTURE ONLY.
 
 Plain, slow, float64 NumPy/SciPy restatement of what the method computes, used to
-judge the CUDA library.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+check the CUDA library.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it; the
 product path never does, and this package never imports the product.
 

@@ -196,7 +196,7 @@ def test_decode_validation_before_launch(lib):
     # Hq not a multiple of Hkv
     a2 = list(args); a2[3] = 3
     assert lib.tq_decode_attn(C.byref(kq), C.byref(vq), *a2, FAKE + 0x900000, ws.value, None) == 1
-    # head dim outside this build
+    # head dim outside what the decode supports
     k64 = _q(T.KIND_MSE, d=64, bits=4); v64 = _q(T.KIND_MSE, d=64, bits=4)
     assert lib.tq_decode_attn(C.byref(k64), C.byref(v64), *args, FAKE + 0x900000, 1 << 30, None) == 2
     # output aliasing the query
@@ -281,7 +281,7 @@ def test_split_decode_validation_before_launch(lib):
     q64 = _q(T.KIND_MSE, d=64, bits=2)
     sp96 = _split([qa, q64], [FAKE, FAKE], 96)
     assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp96), 1, 8, 1, 1000, C.byref(ws)) == 1
-    # wider than this build
+    # wider than the split decode supports
     big = _split([_q(T.KIND_MSE, d=200, bits=2), _q(T.KIND_MSE, d=100, bits=2)], [FAKE, FAKE], 300)
     assert lib.tq_decode_attn_split_workspace(C.byref(big), C.byref(big), 1, 8, 1, 1000, C.byref(ws)) == 2
     # a workspace that is too small fails before any launch
