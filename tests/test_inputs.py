@@ -1,4 +1,4 @@
-"""Pins of the seeded input generators that build rotations (no GPU)."""
+"""Pins of the seeded input generators (rotations, planted outlier channels; no GPU)."""
 import numpy as np
 import pytest
 
@@ -34,3 +34,10 @@ def test_hadamard_rotation_structure():
 def test_hadamard_rotation_rejects_non_power_of_two():
     with pytest.raises(ValueError):
         ti.hadamard_rotation(96, 1)
+
+
+def test_planted_outliers_scales_exactly_the_listed_channels():
+    base = ti.iid_normal((50, 16), 5)
+    x = ti.planted_outliers(50, 16, [2, 9], 6.0, 5)
+    for j in range(16):
+        np.testing.assert_array_equal(x[:, j], base[:, j] * (6.0 if j in (2, 9) else 1.0))
