@@ -343,7 +343,11 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
  *     needs about 4.9 MB).
  *   - The first call on a device, with that device current, looks up the array address
  *     (cudaGetSymbolAddress); make it before any latency-critical loop.  A failed lookup
- *     returns TQ_ERR_CUDA.
+ *     returns TQ_ERR_CUDA.  The address is kept per device and belongs to the device's
+ *     primary context: calls under another driver context, or after cudaDeviceReset,
+ *     are not supported.
+ *   - Shape and descriptor errors are those of tq_decode_attn and are checked first;
+ *     TQ_ERR_WORKSPACE means a valid shape whose scratch exceeds the array.
  *   - All calls on one device share the array: calls that can overlap in time (other
  *     streams, unordered host threads) race on it; calls in order on one stream do not.
  *     Nothing in it has to start at zero.
@@ -361,9 +365,13 @@ tq_status tq_get_status(tq_stream stream);
 
 /*
  * Test hook: iteration limit of every device-side bounded wait launched after this call
- * (0 = default, about 2^26 polls).  Lowering it makes waits that are not immediately
- * satisfied time out, which exercises the error path without hanging a GPU.
+ * (0 = default, about 2^24 polls).  Lowering it makes waits that are not immediately
+ * satisfied time out; TQ_WAIT_EXPIRE_AT_ONCE (-1) makes every bounded wait give up before
+ * its first poll, so a kernel with such a wait reports TQ_ERR_TIMEOUT on every launch.
+ * Either way the kernel drains the copies it issued, frees its tensor memory and exits;
+ * nothing hangs and the context stays usable.  Other negative values: TQ_ERR_INVALID_ARG.
  */
+#define TQ_WAIT_EXPIRE_AT_ONCE (-1)
 tq_status tq_set_wait_limit(int64_t polls);
 
 #ifdef __cplusplus

@@ -10,7 +10,9 @@
 //
 // The first call on a device (with that device current) looks up the array's address
 // with cudaGetSymbolAddress; that call should come before any latency-critical loop.
-// Every later call on the device reuses the address.  All calls on one device share the
+// Every later call on the device reuses the address, which belongs to the device's
+// primary context (the one the CUDA runtime uses): calls made under another driver
+// context, or after cudaDeviceReset of the device, are not supported.  All calls on one device share the
 // array, so two calls that can overlap in time (different streams, or different host
 // threads without ordering between them) race on it; calls issued in order on one
 // stream do not.  Nothing in the array needs to start at zero: each call writes every
@@ -37,8 +39,12 @@ extern "C" tq_status tq_decode_attn_fixed_ws(const tq_quantizer* kq, const tq_qu
                                              int32_t dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t Nmax,
                                              const int32_t* seq_lens, tq_packed kcache, tq_packed vcache,
                                              float scale, float* out, tq_stream stream) {
+  // the shape checks of tq_decode_attn come first, so a bad shape gets the same status
+  // from both entry points whatever its scratch size
+  tq_status s = tq::decode_shape_ok(kq, vq, B, Hq, Hkv, Nmax);
+  if (s != TQ_OK) return s;
   size_t need = 0;
-  tq_status s = tq_decode_attn_workspace(kq, B, Hq, Hkv, Nmax, &need);
+  s = tq_decode_attn_workspace(kq, B, Hq, Hkv, Nmax, &need);
   if (s != TQ_OK) return s;
   if (need > static_cast<size_t>(TQ_DECODE_FIXED_WS_BYTES))
     return tq::fail(TQ_ERR_WORKSPACE, "shape needs %zu scratch bytes; the fixed array holds %zu", need,

@@ -91,6 +91,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // Bounded wait; returns false (and records a timeout) if the limit ran out.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit, int* status,
                                           volatile int* abort_flag) {
+  if (limit < 0) {                 // test hook: every bounded wait expires at once
+    report_status(status, kDevTimeout);
+    *abort_flag = 1;
+    return false;
+  }
   for (long long i = 0;; ++i) {
     if (mbar_try(bar, parity)) return true;
     if (i >= limit || *abort_flag) {

@@ -49,7 +49,7 @@ int* device_status_ptr() {
 
 long long wait_limit() {
   const long long v = g_wait_limit.load();
-  return v > 0 ? v : kDefaultWaitLimit;
+  return v != 0 ? v : kDefaultWaitLimit;
 }
 
 namespace {
@@ -1030,7 +1030,7 @@ tq_status tq_get_status(tq_stream stream) {
 }
 
 tq_status tq_set_wait_limit(int64_t polls) {
-  if (polls < 0) return fail(TQ_ERR_INVALID_ARG, "polls < 0");
+  if (polls < -1) return fail(TQ_ERR_INVALID_ARG, "polls < -1");
   g_wait_limit.store(polls);
   return TQ_OK;
 }
@@ -1038,6 +1038,10 @@ tq_status tq_set_wait_limit(int64_t polls) {
 }  // extern "C"
 
 namespace tq {
+tq_status decode_shape_ok(const tq_quantizer* kq, const tq_quantizer* vq, int B, int Hq, int Hkv, int64_t Nmax) {
+  return check_decode_shape(kq, vq, B, Hq, Hkv, Nmax);
+}
+
 cudaError_t launch_decode(const DecodeParams& p, int kfmt, int kb, int vfmt, int vb, dim3 grid, size_t smem,
                           cudaStream_t stream, int* status, long long lim) {
   if (kfmt == KFMT_MSE && vfmt == VFMT_MSE) return launch_decode_mse(p, kb, vb, grid, smem, stream, status, lim);

@@ -19,6 +19,9 @@ tq_status spectral_calibrate(const float* X, int64_t n, int d, double* vecs, dou
 tq_status spectral_unit_codebooks(double* c_out, double* t_out);
 tq_status lut_scale(const double* values, int count, float* scale_out);
 
+// The shape and descriptor checks tq_decode_attn runs before anything else (tq_api.cu).
+tq_status decode_shape_ok(const tq_quantizer* kq, const tq_quantizer* vq, int B, int Hq, int Hkv, int64_t Nmax);
+
 // Device-side status word and wait limit (tq_api.cu).
 int* device_status_ptr();      // address of the current device's status word
 long long wait_limit();        // polls per bounded wait

@@ -33,9 +33,11 @@ import math
 import numpy as np
 
 from .codebook import lloyd_max
+from .quantizer import unpack_codes
 
 __all__ = ["calibrate", "waterfill", "build_descriptor", "quantize_spectral",
-           "dequantize_spectral", "estimate_spectral", "head_words", "record_words"]
+           "dequantize_spectral", "estimate_spectral", "head_words", "record_words",
+           "unpack_spectral"]
 
 
 def calibrate(X: np.ndarray):
@@ -122,6 +124,31 @@ def _pack_record(idx_row, s_row, desc) -> np.ndarray:
     for w in range(tw):
         out[hw + w] = (tail >> (32 * w)) & 0xFFFFFFFF
     return out
+
+
+def unpack_spectral(codes, desc):
+    """Inverse of the record layout: (idx [n, d], s [n, k_top]) from packed records."""
+    codes = np.asarray(codes, dtype=np.uint32)
+    n = codes.shape[0]
+    d = desc["bits"].shape[0]
+    k = desc["k_top"]
+    hw = head_words(desc)
+    tb = desc["tail_bits"]
+    # the tail is the plain LSB-first code stream of d fields (fields of dims < k are 0)
+    idx = unpack_codes(codes[:, hw:], d, tb)
+    idx[:, :k] = 0
+    s = np.zeros((n, k), dtype=np.int64)
+    for i in range(n):
+        head = sum(int(codes[i, w]) << (32 * w) for w in range(hw))
+        pos = 0
+        for j in range(k):
+            b = int(desc["bits"][j])
+            idx[i, j] = (head >> pos) & ((1 << b) - 1)
+            pos += b
+        if desc["qjl"]:
+            for j in range(k):
+                s[i, j] = (head >> (pos + j)) & 1
+    return idx, s
 
 
 def quantize_spectral(x, desc):

@@ -7,7 +7,7 @@ from oracle import quantizer as OQ
 from oracle.codebook import lloyd_max
 from oracle.search import topk as otopk
 
-from _parity import as_u32
+from _parity import adopt_mse, adopt_prod, as_u32
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -26,11 +26,12 @@ def test_scores_c1_mse_fp32():
     s = K.score(q, torch.from_numpy(qv).cuda(), pk, n).cpu().numpy().astype(np.float64)
     c, t, _ = lloyd_max(b, "beta", d=d)
     ref = OQ.quantize_mse(x.astype(np.float64), rot, c, t, b)
-    same = np.all(as_u32(pk.codes) == ref["codes"], axis=1)
-    est = OQ.estimate_mse(qv.astype(np.float64), rot, ref["idx"], ref["norms"], c)
+    # band-check the GPU's codes, then rescore every record with them
+    idx, exempt = adopt_mse(as_u32(pk.codes), ref, b, t)
+    assert exempt <= max(2, 1e-4 * n * d)
+    est = OQ.estimate_mse(qv.astype(np.float64), rot, idx, ref["norms"], c)
     scale = np.linalg.norm(qv, axis=1)[:, None] * np.linalg.norm(x, axis=1)[None, :]
-    assert np.all(np.abs(s - est)[:, same] <= 1e-3 * scale[:, same])
-    assert same.mean() > 0.99
+    assert np.all(np.abs(s - est) <= 1e-3 * scale)
     # quality context: estimates vs exact inner products (MSE stage is biased by 1 - D_3)
     exact = qv.astype(np.float64) @ x.astype(np.float64).T
     slope = np.sum(est * exact) / np.sum(exact * exact)
@@ -48,10 +49,9 @@ def test_scores_prod(d, bits, n, nq):
     s = K.score(q, torch.from_numpy(qv).cuda(), pk, n).cpu().numpy().astype(np.float64)
     c, t, _ = lloyd_max(bits - 1, "beta", d=d)
     ref = OQ.quantize_prod(x.astype(np.float64), rot, S, c, t, bits)
-    same = np.all(as_u32(pk.codes) == ref["codes"], axis=1) & np.all(as_u32(pk.signs) == ref["signs"], axis=1)
-    est = OQ.estimate_prod(qv.astype(np.float64), rot, S, ref["chat"], ref["s"], ref["norms"], ref["rnorms"])
-    assert np.all(np.abs(s - est)[:, same] <= 1e-3)       # unit-norm q and x
-    assert same.mean() > 0.99
+    a = adopt_prod(as_u32(pk.codes), as_u32(pk.signs), pk.rnorms.cpu().numpy(), ref, bits, c, t, S)
+    est = OQ.estimate_prod(qv.astype(np.float64), rot, S, a["chat"], a["s"], ref["norms"], a["rnorms"])
+    assert np.all(np.abs(s - est) <= 1e-3)       # unit-norm q and x: 1e-3 ||q|| ||x||
 
 
 @pytest.mark.parametrize("bits", [2, 4])
@@ -68,7 +68,8 @@ def test_topk_search(bits):
     vals, ids = vals.cpu().numpy().astype(np.float64), ids.cpu().numpy()
     c, t, _ = lloyd_max(bits - 1, "beta", d=d)
     ref = OQ.quantize_prod(x.astype(np.float64), rot, S, c, t, bits)
-    est = OQ.estimate_prod(qv.astype(np.float64), rot, S, ref["chat"], ref["s"], ref["norms"], ref["rnorms"])
+    a = adopt_prod(as_u32(pk.codes), as_u32(pk.signs), pk.rnorms.cpu().numpy(), ref, bits, c, t, S)
+    est = OQ.estimate_prod(qv.astype(np.float64), rot, S, a["chat"], a["s"], ref["norms"], a["rnorms"])
     rid, rval = otopk(est, k)
     tol = 1e-3
     for i in range(nq):

@@ -213,8 +213,6 @@ def test_score_validation(lib):
                         FAKE + 0x600000, ws.value, None) == 2   # topk > 32
     assert lib.tq_score(C.byref(q), FAKE + 0x300000, 0, 4, pk, 100, 10, FAKE + 0x400000, FAKE + 0x500000,
                         FAKE + 0x600000, 8, None) == 8          # workspace
-    assert lib.tq_set_wait_limit(-1) == 1
-    assert lib.tq_set_wait_limit(0) == 0
 
 
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
@@ -291,3 +289,10 @@ def test_split_decode_validation_before_launch(lib):
                           T.Packed_t(FAKE + 0x700000, None, FAKE + 0x780000, None))
     assert lib.tq_decode_attn_split(C.byref(sp), C.byref(sp), FAKE + 0x900000, 1, 2, 8, 2, 1000, FAKE + 0xA00000,
                                     pk, pv, C.c_float(0.1), FAKE + 0xB00000, FAKE + 0xC00000, 16, None) == 8
+
+
+def test_wait_limit_values(lib):
+    """0 restores the default, -1 is the expire-at-once test hook, below -1 is refused."""
+    assert lib.tq_set_wait_limit(-1) == 0
+    assert lib.tq_set_wait_limit(-2) == 1            # TQ_ERR_INVALID_ARG
+    assert lib.tq_set_wait_limit(0) == 0

@@ -131,3 +131,75 @@ def test_spectral_qjl_unbiased_over_S():
         out = SP.quantize_spectral(x, desc)
         est[i] = SP.estimate_spectral(q, desc, out["chat"], out["s"], out["rnorms"])[0, 0]
     assert abs(est.mean() - truth) <= 4 * est.std(ddof=1) / math.sqrt(trials)
+
+
+def _max_distortion(golden_dir, b):
+    """Unit-normal Lloyd-Max distortion of b bits, from the printed Max (1960) table."""
+    g = json.load(open(os.path.join(golden_dir, "lloyd_max_gaussian.json")))
+    return float(g["levels"][str(2 ** b)]["distortion"])
+
+
+def _recon_gap(dequant, golden_dir, n=20000):
+    """(mean squared reconstruction error - its expectation) / standard error.
+
+    The data are drawn from the generator's own eigenbasis, so rot = U^T holds the true
+    eigenvectors and z_j = (rot x)_j ~ N(0, lambda_j) independently.  With rot orthogonal,
+    ||x - rot^T c_hat||^2 = sum_j (z_j - c_hat_j)^2, whose expectation is
+    sum_j lambda_j D_{b_j} with D_b the textbook unit-normal distortion.
+    """
+    d = 128
+    U = ti.haar_rotation(d, 3004).astype(np.float64)
+    lam = d * ti.kv_spectrum(d)
+    desc = SP.build_descriptor(U.T, lam, 4, 8, 1, False)
+    bits = desc["bits"]
+    assert bits.max() <= 4, "the pin needs bit widths the printed table covers"
+    x = ti.anisotropic(n, d, U, 4104)
+    out = SP.quantize_spectral(x, desc)
+    err = np.sum((x - dequant(out["chat"], desc)) ** 2, axis=1)
+    expect = sum(lam[j] * _max_distortion(golden_dir, int(bits[j])) for j in range(d))
+    return (err.mean() - expect) / (err.std(ddof=1) / math.sqrt(n)), err.mean() / expect
+
+
+def test_dequantize_spectral_reconstruction_error(golden_dir):
+    """x_hat = rot^T c_hat: the squared error equals sum_j lambda_j D_{b_j} (printed D_b)."""
+    z, ratio = _recon_gap(SP.dequantize_spectral, golden_dir)
+    # the Monte-Carlo standard error (~0.25 % of the mean) dwarfs the table's rounding
+    assert abs(z) < 4.0, (z, ratio)
+
+
+def test_dequantize_spectral_pin_rejects_transposed_rotation(golden_dir):
+    """A planted mistake (x_hat = rot c_hat) must fail the reconstruction pin."""
+    z, ratio = _recon_gap(lambda chat, desc: np.asarray(chat) @ desc["rot"].T, golden_dir, n=4000)
+    assert ratio > 1.5 and z > 50.0
+
+
+def test_dequantize_spectral_permutation_by_hand():
+    """rot a permutation: dim j reads x[perm[j]] and its reconstruction returns there."""
+    d = 4
+    perm = [2, 0, 3, 1]                       # z_j = x[perm[j]]
+    rot = np.zeros((d, d))
+    for j, i in enumerate(perm):
+        rot[j, i] = 1.0
+    lam = np.array([4.0, 1.0, 0.25, 0.0625])  # sigma_j = 2, 1, 0.5, 0.25
+    desc = SP.build_descriptor(rot, lam, 0, 0, 1, False)
+    x = np.array([[0.3, -1.0, 2.0, -0.01]])
+    out = SP.quantize_spectral(x, desc)
+    a = math.sqrt(2.0 / math.pi)              # 1-bit unit-normal centroid magnitude
+    # dim 0 <- x[2] = 2.0 (sigma 2), dim 1 <- x[0] = 0.3 (sigma 1),
+    # dim 2 <- x[3] = -0.01 (sigma 0.5), dim 3 <- x[1] = -1.0 (sigma 0.25)
+    want = np.array([[1.0 * a, -0.25 * a, 2.0 * a, -0.5 * a]])
+    assert np.allclose(SP.dequantize_spectral(out["chat"], desc), want, rtol=1e-12, atol=0)
+
+
+def test_unpack_spectral_inverts_record_layout():
+    """Random codes and signs survive pack -> unpack (the record layout is a bijection)."""
+    d, U, desc = _spectral_setup()
+    rng = np.random.Generator(np.random.PCG64(12))
+    n = 40
+    idx = np.zeros((n, d), dtype=np.int64)
+    for j in range(d):
+        idx[:, j] = rng.integers(0, 1 << int(desc["bits"][j]), size=n)
+    s = rng.integers(0, 2, size=(n, 4))
+    words = np.stack([SP._pack_record(idx[i], s[i], desc) for i in range(n)])
+    gi, gs = SP.unpack_spectral(words, desc)
+    assert np.array_equal(gi, idx) and np.array_equal(gs, s)

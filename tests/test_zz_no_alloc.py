@@ -25,9 +25,8 @@ D = 128
 FIXED_BYTES = 8 << 20
 
 
-def _fixed(kq, vq, q, sl, kc, vc, Nmax, Hkv):
+def _fixed(kq, vq, q, sl, kc, vc, Nmax, Hkv, out):
     B, Hq, _ = q.shape
-    out = torch.full((B, Hq, D), float("nan"), dtype=torch.float32, device=q.device)
     st = T.lib().tq_decode_attn_fixed_ws(kq.ref, vq.ref, q.data_ptr(), T._dtype_code(q), B, Hq, Hkv, Nmax,
                                          sl.data_ptr(), kc.as_c(), vc.as_c(), C.c_float(1.0 / math.sqrt(D)),
                                          out.data_ptr(), None)
@@ -60,11 +59,22 @@ def test_fixed_scratch_matches_workspace_call(name, B, Hq, Hkv, Nmax, seq_lens, 
     del kx, vx
     sl = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
     ref = K.decode_attn(kq, vq, q, sl, kc, vc, Nmax, Hkv).cpu().numpy()
-    for _ in range(2):
-        out = _fixed(kq, vq, q, sl, kc, vc, Nmax, Hkv)
+    B_, Hq_, _ = q.shape
+    outs = [torch.full((B_, Hq_, D), float("nan"), dtype=torch.float32, device=q.device) for _ in range(2)]
+    torch.cuda.synchronize()
+    for i in range(2):
+        if i == 1:
+            # the first call did the address lookup; from here on neither the driver's view
+            # of free device memory nor torch's allocator may move
+            free0, _ = torch.cuda.mem_get_info()
+            torch0 = torch.cuda.memory_allocated()
+        _fixed(kq, vq, q, sl, kc, vc, Nmax, Hkv, outs[i])
         torch.cuda.synchronize()
+        if i == 1:
+            assert torch.cuda.mem_get_info()[0] == free0
+            assert torch.cuda.memory_allocated() == torch0
         assert K.get_status() == 0
-        o = out.cpu().numpy()
+        o = outs[i].cpu().numpy()
         assert np.all(np.isfinite(o))
         err = rel_rows(o, ref)
         assert np.all(err <= 1e-3), f"max row error {err.max():.3e}"
@@ -82,3 +92,15 @@ def test_fixed_scratch_rejects_oversize_shape():
                                          C.c_float(0.1), FAKE, None)
     assert st == 8
     assert b"fixed array" in T.lib().tq_last_error()
+
+
+def test_fixed_scratch_checks_shape_before_size():
+    """A bad shape gets tq_decode_attn's status even when its scratch would not fit."""
+    rot = ti.haar_rotation(D, 1002)
+    kq = K.Quantizer.mse(rot, 4)
+    vq = K.Quantizer.mse(rot, 4)
+    FAKE = 0x10000   # refused before any pointer is touched
+    pk = T.Packed_t(FAKE, None, FAKE, None)
+    st = T.lib().tq_decode_attn_fixed_ws(kq.ref, vq.ref, FAKE, T.BF16, 64, 60, 8, 1 << 20, FAKE, pk, pk,
+                                         C.c_float(0.1), FAKE, None)
+    assert st == 1                       # Hq not a multiple of Hkv: TQ_ERR_INVALID_ARG
