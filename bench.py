@@ -486,10 +486,8 @@ def run_other(args):
             ck = ti.anisotropic(4096, Dm, U.astype(np.float64), ti.SEEDS["calib_keys"] + cfgno).astype(np.float32)
             cv = ti.anisotropic(4096, Dm, U.astype(np.float64), ti.SEEDS["calib_values"] + cfgno).astype(np.float32)
             S4 = ti.gaussian_matrix(4, 4, ti.SEEDS["qjl"] + cfgno)
-            kvec, kval = K.spectral_calibrate(ck)
-            vvec, vval = K.spectral_calibrate(cv)
-            kq = K.Quantizer.spectral(kvec, kval, 4, list(K.waterfill(kval[:4], 12)), 1, True, S4, device=dev)
-            vq = K.Quantizer.spectral(vvec, vval, 4, list(K.waterfill(vval[:4], 12)), 1, False, None, device=dev)
+            kq, _ = K.Quantizer.spectral_calibrated(ck, 4, 12, 1, True, S4, device=dev)
+            vq, _ = K.Quantizer.spectral_calibrated(cv, 4, 12, 1, False, None, device=dev)
             desc = ("decode-8k spectral: B=32, Hkv=8, Hq=32, d=128, context 8192, eigenvector rotation from 4096 "
                     "calibration vectors, water-filled top-4 bits + 1-bit tail, QJL on the top 4 (keys)")
         Lk, Lv = kq.layout(), vq.layout()

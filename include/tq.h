@@ -182,6 +182,38 @@ tq_status tq_spectral_unit_codebooks(double* centroids_out, double* boundaries_o
  */
 tq_status tq_lut_scale(const double* values, int32_t count, float* scale_out);
 
+/*
+ * HOST.  Everything a SPECTRAL descriptor points at, from an eigen-decomposition
+ * (SpectralQuant thread, posts 4-6): eigvecs [d*d] (row j = eigenvector j, descending
+ * eigenvalue, as tq_spectral_calibrate writes them) and eigvals [d], host float64.
+ *   top_bits_out [k_top]       reverse water-filling of budget_bits over eigvals[0..k_top)
+ *                              (as tq_waterfill, negative eigenvalues taken as 0,
+ *                              dims capped at max_bits);
+ *   dim_sigma_out [d]          sqrt(max(eigvals_j, 0)), the scale of dim j's codebook;
+ *   rot_out [d*d]              the eigenvectors in fp32;
+ *   unit_centroids_out [510],
+ *   unit_boundaries_out [502]  the unit-normal codebooks of tq_spectral_unit_codebooks in fp32;
+ *   *lut_scale_out             tq_lut_scale of the tail_bits unit codebook.
+ * All outputs are host memory the caller allocated; copied to the device they are the
+ * descriptor's rot, dim_sigma, unit_centroids, unit_boundaries, top_bits and lut_scale.
+ * d 2..1024, k_top 1..TQ_MAX_TOP, tail_bits 1..4, max_bits 1..8; TQ_ERR_UNSUPPORTED when
+ * the top bits plus k_top sign bits exceed 32.
+ */
+tq_status tq_spectral_descriptor(const double* eigvecs, const double* eigvals, int32_t d, int32_t k_top,
+                                 int32_t budget_bits, int32_t tail_bits, int32_t max_bits, float* rot_out,
+                                 float* dim_sigma_out, float* unit_centroids_out, float* unit_boundaries_out,
+                                 int32_t* top_bits_out, float* lut_scale_out);
+
+/*
+ * HOST.  Calibration and descriptor in one call: tq_spectral_calibrate of the n host rows
+ * X [n*d] (fp32), then tq_spectral_descriptor of the result.  eigvals_out [d] (host,
+ * may be NULL) receives the eigenvalues.
+ */
+tq_status tq_spectral_prepare(const float* X, int64_t n, int32_t d, int32_t k_top, int32_t budget_bits,
+                              int32_t tail_bits, int32_t max_bits, float* rot_out, float* dim_sigma_out,
+                              float* unit_centroids_out, float* unit_boundaries_out, int32_t* top_bits_out,
+                              float* lut_scale_out, double* eigvals_out);
+
 /* HOST.  Words per record and which norm arrays a quantizer writes. */
 tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out);
 

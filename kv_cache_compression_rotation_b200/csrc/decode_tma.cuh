@@ -41,10 +41,19 @@ namespace tq {
 // two 16-token units of a stage (8 consumer warps, 3 stages of 256 tokens); otherwise one
 // unit (11 consumer warps for MSE keys, 4 stages).  PROD keys need more registers and run
 // 7 consumer warps.  Plus one producer warp.
-__host__ __device__ constexpr int tma_units(bool pk) { return pk ? 2 : 1; }
-__host__ __device__ constexpr int tma_consumers(int kf, bool pk) { return kf == KFMT_PROD ? 7 : (pk ? 8 : 11); }
+#ifndef TQ_DEC_PK_NC
+#define TQ_DEC_PK_NC 8
+#endif
+#ifndef TQ_DEC_PK_U
+#define TQ_DEC_PK_U 2
+#endif
+#ifndef TQ_DEC_PK_NS
+#define TQ_DEC_PK_NS 3
+#endif
+__host__ __device__ constexpr int tma_units(bool pk) { return pk ? TQ_DEC_PK_U : 1; }
+__host__ __device__ constexpr int tma_consumers(int kf, bool pk) { return kf == KFMT_PROD ? 7 : (pk ? TQ_DEC_PK_NC : 11); }
 __host__ __device__ constexpr int tma_stage_tokens(int kf, bool pk) { return tma_consumers(kf, pk) * 16 * tma_units(pk); }
-__host__ __device__ constexpr int tma_stages(bool pk) { return pk ? 3 : 4; }
+__host__ __device__ constexpr int tma_stages(bool pk) { return pk ? TQ_DEC_PK_NS : 4; }
 constexpr int kTmaHeadBlock = 8;     // query heads per work item (MMA N)
 
 __device__ __forceinline__ uint32_t tma_smem_u32(const void* p) {

@@ -366,4 +366,32 @@ tq_status spectral_unit_codebooks(double* c_out, double* t_out) {
   return TQ_OK;
 }
 
+tq_status spectral_descriptor(const double* vecs, const double* vals, int d, int k_top, int budget, int tail_bits,
+                              int max_bits, float* rot_out, float* sigma_out, float* unit_c_out, float* unit_t_out,
+                              int32_t* top_bits_out, float* lut_scale_out) {
+  if (!vecs || !vals || !rot_out || !sigma_out || !unit_c_out || !unit_t_out || !top_bits_out || !lut_scale_out)
+    return fail(TQ_ERR_INVALID_ARG, "spectral descriptor: null argument");
+  if (d < 2 || d > 1024 || k_top < 1 || k_top > TQ_MAX_TOP || k_top > d || budget < 0 || tail_bits < 1 ||
+      tail_bits > 4 || max_bits < 1 || max_bits > 8)
+    return fail(TQ_ERR_INVALID_ARG, "spectral descriptor: size out of range");
+  // bits of the signal dims: reverse water-filling over their eigenvalues (negative sample
+  // eigenvalues of a rank-deficient calibration count as zero variance)
+  std::vector<double> lam(d);
+  for (int j = 0; j < d; ++j) lam[j] = std::isfinite(vals[j]) ? std::max(vals[j], 0.0) : 0.0;
+  tq_status s = waterfill(lam.data(), k_top, budget, max_bits, top_bits_out);
+  if (s != TQ_OK) return s;
+  int top_sum = 0;
+  for (int j = 0; j < k_top; ++j) top_sum += top_bits_out[j];
+  if (top_sum + k_top > 32) return fail(TQ_ERR_UNSUPPORTED, "spectral descriptor: top bits + signs exceed one word");
+  // dim j's codebook is sqrt(lambda_j) times the unit-normal Lloyd-Max codebook
+  for (int j = 0; j < d; ++j) sigma_out[j] = static_cast<float>(std::sqrt(lam[j]));
+  for (size_t i = 0; i < static_cast<size_t>(d) * d; ++i) rot_out[i] = static_cast<float>(vecs[i]);
+  std::vector<double> uc(510), ut(502);
+  if ((s = spectral_unit_codebooks(uc.data(), ut.data())) != TQ_OK) return s;
+  for (int i = 0; i < 510; ++i) unit_c_out[i] = static_cast<float>(uc[i]);
+  for (int i = 0; i < 502; ++i) unit_t_out[i] = static_cast<float>(ut[i]);
+  // half-precision table of the tail codebook (the top dims are decoded in fp32)
+  return lut_scale(uc.data() + ((1 << tail_bits) - 2), 1 << tail_bits, lut_scale_out);
+}
+
 }  // namespace tq

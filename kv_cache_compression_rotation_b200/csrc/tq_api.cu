@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "decode.cuh"
 #include "decode_aux.cuh"
@@ -416,6 +417,28 @@ tq_status tq_spectral_unit_codebooks(double* centroids_out, double* boundaries_o
 
 tq_status tq_lut_scale(const double* values, int32_t count, float* scale_out) {
   return lut_scale(values, count, scale_out);
+}
+
+tq_status tq_spectral_descriptor(const double* eigvecs, const double* eigvals, int32_t d, int32_t k_top,
+                                 int32_t budget_bits, int32_t tail_bits, int32_t max_bits, float* rot_out,
+                                 float* dim_sigma_out, float* unit_centroids_out, float* unit_boundaries_out,
+                                 int32_t* top_bits_out, float* lut_scale_out) {
+  return spectral_descriptor(eigvecs, eigvals, d, k_top, budget_bits, tail_bits, max_bits, rot_out, dim_sigma_out,
+                             unit_centroids_out, unit_boundaries_out, top_bits_out, lut_scale_out);
+}
+
+tq_status tq_spectral_prepare(const float* X, int64_t n, int32_t d, int32_t k_top, int32_t budget_bits,
+                              int32_t tail_bits, int32_t max_bits, float* rot_out, float* dim_sigma_out,
+                              float* unit_centroids_out, float* unit_boundaries_out, int32_t* top_bits_out,
+                              float* lut_scale_out, double* eigvals_out) {
+  if (d < 2 || d > 1024) return fail(TQ_ERR_INVALID_ARG, "spectral prepare: d out of range");
+  std::vector<double> vecs(static_cast<size_t>(d) * d), vals(d);
+  tq_status s = spectral_calibrate(X, n, d, vecs.data(), vals.data());
+  if (s != TQ_OK) return s;
+  if (eigvals_out)
+    for (int j = 0; j < d; ++j) eigvals_out[j] = vals[j];
+  return spectral_descriptor(vecs.data(), vals.data(), d, k_top, budget_bits, tail_bits, max_bits, rot_out,
+                             dim_sigma_out, unit_centroids_out, unit_boundaries_out, top_bits_out, lut_scale_out);
 }
 
 tq_status tq_record_layout(const tq_quantizer* q, tq_layout* out) {

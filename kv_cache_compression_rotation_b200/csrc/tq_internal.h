@@ -18,6 +18,9 @@ tq_status waterfill(const double* lambda, int k, int budget, int max_bits, int32
 tq_status spectral_calibrate(const float* X, int64_t n, int d, double* vecs, double* vals);
 tq_status spectral_unit_codebooks(double* c_out, double* t_out);
 tq_status lut_scale(const double* values, int count, float* scale_out);
+tq_status spectral_descriptor(const double* vecs, const double* vals, int d, int k_top, int budget, int tail_bits,
+                              int max_bits, float* rot_out, float* sigma_out, float* unit_c_out, float* unit_t_out,
+                              int32_t* top_bits_out, float* lut_scale_out);
 
 // The shape and descriptor checks tq_decode_attn runs before anything else (tq_api.cu).
 tq_status decode_shape_ok(const tq_quantizer* kq, const tq_quantizer* vq, int B, int Hq, int Hkv, int64_t Nmax);

@@ -32,7 +32,7 @@ EXPORTS = [
     "tq_quantize_spectral", "tq_dequantize", "tq_score_workspace", "tq_score",
     "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
     "tq_decode_attn_fixed_ws", "tq_quantize_split", "tq_score_split_workspace", "tq_score_split",
-    "tq_decode_attn_split_workspace", "tq_decode_attn_split",
+    "tq_decode_attn_split_workspace", "tq_decode_attn_split", "tq_spectral_descriptor", "tq_spectral_prepare",
 ]
 
 
@@ -105,6 +105,10 @@ def lib():
             "tq_get_status": ([vp], C.c_int),
             "tq_set_wait_limit": ([i64], C.c_int),
             "tq_lut_scale": ([f64p, i32, C.POINTER(C.c_float)], C.c_int),
+            "tq_spectral_descriptor": ([f64p, f64p, i32, i32, i32, i32, i32, vp, vp, vp, vp, C.POINTER(i32),
+                                        C.POINTER(C.c_float)], C.c_int),
+            "tq_spectral_prepare": ([vp, i64, i32, i32, i32, i32, i32, vp, vp, vp, vp, C.POINTER(i32),
+                                     C.POINTER(C.c_float), f64p], C.c_int),
             "tq_quantize_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), vp], C.c_int),
             "tq_score_split_workspace": ([C.POINTER(Split_t), i64, i64, i32, C.POINTER(C.c_size_t)], C.c_int),
             "tq_score_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), i64, i32, vp, vp, vp,
@@ -261,15 +265,53 @@ class Quantizer:
                    centroids=cen, boundaries=bnd, lut_scale=sc)
 
     @classmethod
-    def spectral(cls, eigvecs, eigvals, k_top: int, top_bits, tail_bits: int, qjl: bool, S_top=None,
-                 device="cuda"):
-        d = eigvecs.shape[0]
-        uc, ut = spectral_unit_codebooks()
-        sig = np.sqrt(np.maximum(np.asarray(eigvals, dtype=np.float64), 0.0))
-        return cls(KIND_SPECTRAL, d, cls._dev(eigvecs, device), S=None if S_top is None else cls._dev(S_top, device),
-                   k_top=k_top, tail_bits=tail_bits, qjl=1 if qjl else 0, top_bits=list(top_bits),
+    def _spectral_from_host(cls, d, k_top, tail_bits, qjl, S_top, device, host):
+        rot, sig, uc, ut, top, lut = host
+        return cls(KIND_SPECTRAL, d, cls._dev(rot, device), S=None if S_top is None else cls._dev(S_top, device),
+                   k_top=k_top, tail_bits=tail_bits, qjl=1 if qjl else 0, top_bits=list(top[:k_top]),
                    dim_sigma=cls._dev(sig, device), unit_c=cls._dev(uc, device), unit_t=cls._dev(ut, device),
-                   lut_scale=lut_scale(uc[(1 << tail_bits) - 2:(1 << (tail_bits + 1)) - 2]))
+                   lut_scale=lut)
+
+    @staticmethod
+    def _spectral_outputs(d):
+        return (np.zeros((d, d), dtype=np.float32), np.zeros(d, dtype=np.float32), np.zeros(510, dtype=np.float32),
+                np.zeros(502, dtype=np.float32), np.zeros(MAX_TOP, dtype=np.int32))
+
+    @classmethod
+    def spectral(cls, eigvecs, eigvals, k_top: int, budget_bits: int, tail_bits: int, qjl: bool, S_top=None,
+                 max_bits: int = 8, device="cuda"):
+        """SPECTRAL descriptor from a given eigen-decomposition (rows of eigvecs, descending
+        eigvals): tq_spectral_descriptor water-fills the top bits and builds the scales and
+        codebooks; this wrapper only copies its outputs to the device."""
+        d = eigvecs.shape[0]
+        vecs = np.ascontiguousarray(eigvecs, dtype=np.float64)
+        vals = np.ascontiguousarray(eigvals, dtype=np.float64)
+        rot, sig, uc, ut, top = cls._spectral_outputs(d)
+        lut = C.c_float(0.0)
+        _check(lib().tq_spectral_descriptor(vecs.ctypes.data_as(C.POINTER(C.c_double)),
+                                            vals.ctypes.data_as(C.POINTER(C.c_double)), d, k_top, budget_bits,
+                                            tail_bits, max_bits, rot.ctypes.data, sig.ctypes.data, uc.ctypes.data,
+                                            ut.ctypes.data, top.ctypes.data_as(C.POINTER(C.c_int32)), C.byref(lut)))
+        return cls._spectral_from_host(d, k_top, tail_bits, qjl, S_top, device,
+                                       (rot, sig, uc, ut, top, float(lut.value)))
+
+    @classmethod
+    def spectral_calibrated(cls, X, k_top: int, budget_bits: int, tail_bits: int, qjl: bool, S_top=None,
+                            max_bits: int = 8, device="cuda"):
+        """SPECTRAL descriptor straight from calibration rows X [n, d] (tq_spectral_prepare:
+        calibration, water-filling, scales and codebooks in the library).  Returns
+        (quantizer, eigenvalues)."""
+        X = np.ascontiguousarray(X, dtype=np.float32)
+        n, d = X.shape
+        rot, sig, uc, ut, top = cls._spectral_outputs(d)
+        vals = np.zeros(d, dtype=np.float64)
+        lut = C.c_float(0.0)
+        _check(lib().tq_spectral_prepare(X.ctypes.data, n, d, k_top, budget_bits, tail_bits, max_bits,
+                                         rot.ctypes.data, sig.ctypes.data, uc.ctypes.data, ut.ctypes.data,
+                                         top.ctypes.data_as(C.POINTER(C.c_int32)), C.byref(lut),
+                                         vals.ctypes.data_as(C.POINTER(C.c_double))))
+        q = cls._spectral_from_host(d, k_top, tail_bits, qjl, S_top, device, (rot, sig, uc, ut, top, float(lut.value)))
+        return q, vals
 
     def layout(self) -> Layout_t:
         L = Layout_t()

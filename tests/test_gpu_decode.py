@@ -155,9 +155,9 @@ def test_decode_spectral_parity():
     kt, k64 = ti.to_bf16_f64(kx)
     vt, v64 = ti.to_bf16_f64(vx)
     qt, q64 = _query(B, Hq, 4)
-    top = list(dk["bits"][:4])
-    kq = K.Quantizer.spectral(rot, lam, 4, top, 1, True, S4)
-    vq = K.Quantizer.spectral(rot, lam, 4, top, 1, False, None)
+    kq = K.Quantizer.spectral(rot, lam, 4, 12, 1, True, S4)
+    vq = K.Quantizer.spectral(rot, lam, 4, 12, 1, False, None)
+    assert list(kq.top_bits) == list(dk["bits"][:4]) == list(vq.top_bits)
     sl = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
     ok = OSP.quantize_spectral(k64, dk)
     ov = OSP.quantize_spectral(v64, dv)

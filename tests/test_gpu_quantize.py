@@ -1,4 +1,5 @@
 """GPU parity: quantize / dequantize through the C ABI against the oracle."""
+import functools
 import math
 
 import numpy as np
@@ -7,7 +8,7 @@ import pytest
 import tq_inputs as ti
 from oracle import quantizer as OQ
 from oracle import spectral as OSP
-from oracle.codebook import lloyd_max
+from oracle.codebook import lloyd_max as _lloyd_max
 
 from _parity import adopt_spectral, as_u32, code_mismatches, sign_mismatches
 
@@ -15,6 +16,11 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 K = pytest.importorskip("kv_cache_compression_rotation_b200")
+
+
+@functools.lru_cache(maxsize=None)
+def lloyd_max(bits, dist, d=None):
+    return _lloyd_max(bits, dist, d=d)
 
 
 def _inputs(n, d, dtype, seed, zero_rows=()):
@@ -47,6 +53,8 @@ MSE_CASES = [
     (32, 5, "f32", 300),
     (96, 6, "bf16", 100),
     (1536, 4, "bf16", 64),
+    (64, 7, "f32", 200),          # the top of the ABI's MSE range (CUDA-core kernel)
+    (64, 8, "bf16", 150),
 ]
 
 
@@ -116,7 +124,9 @@ def test_quantize_pm1_flag_rejects_other_rotations():
 
 
 @pytest.mark.parametrize("d,bits,m,dtype,n", [(128, 3, 128, "bf16", 2000), (64, 2, 64, "f32", 500),
-                                              (128, 1, 128, "f32", 300), (128, 5, 256, "bf16", 400)])
+                                              (128, 1, 128, "f32", 300), (128, 5, 256, "bf16", 400),
+                                              (64, 6, 64, "f32", 200), (64, 7, 64, "bf16", 200),
+                                              (64, 8, 96, "f32", 150), (64, 9, 64, "bf16", 150)])
 def test_quantize_prod_parity(d, bits, m, dtype, n):
     rot = ti.haar_rotation(d, 1100 + d)
     S = ti.gaussian_matrix(m, d, 2000 + d)
@@ -162,7 +172,8 @@ def test_quantize_spectral_parity(qjl):
     d, n = 128, 3000
     U, rot, lam, S4, desc = _spectral_desc(qjl)
     xt, x64 = ti.to_bf16_f64(ti.anisotropic(n, d, U, 4004))
-    q = K.Quantizer.spectral(rot, lam, 4, list(desc["bits"][:4]), 1, qjl, S4 if qjl else None)
+    q = K.Quantizer.spectral(rot, lam, 4, 12, 1, qjl, S4 if qjl else None)
+    assert list(q.top_bits) == list(desc["bits"][:4])      # the library's water-filling
     out = K.quantize(q, xt.cuda())
     ref = OSP.quantize_spectral(x64, desc)
     # coordinate by coordinate: a differing code must be a neighbour with the oracle's z_j

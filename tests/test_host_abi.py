@@ -296,3 +296,66 @@ def test_wait_limit_values(lib):
     assert lib.tq_set_wait_limit(-1) == 0
     assert lib.tq_set_wait_limit(-2) == 1            # TQ_ERR_INVALID_ARG
     assert lib.tq_set_wait_limit(0) == 0
+
+
+def test_spectral_descriptor_matches_oracle(lib):
+    """tq_spectral_descriptor: water-filled bits, per-dim scales and codebooks as the oracle's
+    build_descriptor computes them from the same eigen-decomposition."""
+    d, n = 128, 4096
+    U = ti.haar_rotation(d, 3004).astype(np.float64)
+    X = ti.anisotropic(n, d, U, 7000).astype(np.float32)
+    vo, wo = OSP.calibrate(X.astype(np.float64))
+    desc = OSP.build_descriptor(vo, wo, 4, 12, 1, True)
+    rot = np.zeros((d, d), np.float32)
+    sig = np.zeros(d, np.float32)
+    uc = np.zeros(510, np.float32)
+    ut = np.zeros(502, np.float32)
+    top = np.zeros(8, np.int32)
+    lut = C.c_float(0)
+    dp = C.POINTER(C.c_double)
+    st = lib.tq_spectral_descriptor(vo.ctypes.data_as(dp), wo.ctypes.data_as(dp), d, 4, 12, 1, 8, rot.ctypes.data,
+                                    sig.ctypes.data, uc.ctypes.data, ut.ctypes.data,
+                                    top.ctypes.data_as(C.POINTER(C.c_int32)), C.byref(lut))
+    assert st == 0
+    assert list(top[:4]) == list(desc["bits"][:4]) == [5, 3, 2, 2]
+    assert np.allclose(sig, desc["sigma"], rtol=1e-7, atol=0)
+    assert np.array_equal(rot, vo.astype(np.float32))
+    for b in range(1, 7):
+        co, to, _ = lloyd_max(b, "gaussian", sigma=1.0)
+        off_c, off_t = (1 << b) - 2, (1 << b) - b - 1
+        assert np.allclose(uc[off_c:off_c + (1 << b)], co, rtol=1e-6, atol=1e-7)
+        assert np.allclose(ut[off_t:off_t + (1 << b) - 1], to, rtol=1e-6, atol=1e-7)
+    assert 1.0 <= lut.value < 2.0
+    # a negative sample eigenvalue is a zero variance: scale 0, no bits from water-filling
+    w2 = wo.copy()
+    w2[2] = -1e-3
+    st = lib.tq_spectral_descriptor(vo.ctypes.data_as(dp), w2.ctypes.data_as(dp), d, 4, 12, 1, 8, rot.ctypes.data,
+                                    sig.ctypes.data, uc.ctypes.data, ut.ctypes.data,
+                                    top.ctypes.data_as(C.POINTER(C.c_int32)), C.byref(lut))
+    assert st == 0 and sig[2] == 0.0 and top[2] == 0
+    # top bits plus sign bits must fit one head word
+    st = lib.tq_spectral_descriptor(vo.ctypes.data_as(dp), wo.ctypes.data_as(dp), d, 8, 40, 1, 8, rot.ctypes.data,
+                                    sig.ctypes.data, uc.ctypes.data, ut.ctypes.data,
+                                    top.ctypes.data_as(C.POINTER(C.c_int32)), C.byref(lut))
+    assert st == 2
+
+
+def test_spectral_prepare_is_calibrate_then_descriptor(lib):
+    d, n = 128, 4096
+    U = ti.haar_rotation(d, 3004).astype(np.float64)
+    X = ti.anisotropic(n, d, U, 7000).astype(np.float32)
+    vecs, vals = K.spectral_calibrate(X)
+    rot = np.zeros((d, d), np.float32)
+    sig = np.zeros(d, np.float32)
+    uc = np.zeros(510, np.float32)
+    ut = np.zeros(502, np.float32)
+    top = np.zeros(8, np.int32)
+    lut = C.c_float(0)
+    ev = np.zeros(d)
+    st = lib.tq_spectral_prepare(X.ctypes.data, n, d, 4, 12, 1, 8, rot.ctypes.data, sig.ctypes.data, uc.ctypes.data,
+                                 ut.ctypes.data, top.ctypes.data_as(C.POINTER(C.c_int32)), C.byref(lut),
+                                 ev.ctypes.data_as(C.POINTER(C.c_double)))
+    assert st == 0
+    assert np.array_equal(ev, vals) and np.array_equal(rot, vecs.astype(np.float32))
+    assert np.array_equal(sig, np.sqrt(np.maximum(vals, 0)).astype(np.float32))
+    assert list(top[:4]) == list(K.waterfill(vals[:4], 12))
