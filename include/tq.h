@@ -348,9 +348,11 @@ tq_status tq_decode_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq
  *   for query head h (KV head h / (Hq/Hkv)), logit_i = scale * est(q_h, k_i) over the
  *   first seq_lens[b] records, p = softmax(logit), out = sum_i p_i v_hat_i.
  * q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), caches laid out
- * [B][Hkv][Nmax] records, out [B*Hq*d] fp32.  Keys: MSE, PROD or SPECTRAL; values: MSE or
- * SPECTRAL (without qjl).  libtq runs d = 128, code bits <= 4, PROD m = d,
- * Hq/Hkv in 1..16; other shapes give TQ_ERR_UNSUPPORTED.  Value norms must stay below
+ * [B][Hkv][Nmax] records, out [B*Hq*d] fp32.  Keys: MSE, PROD or SPECTRAL; values: MSE,
+ * PROD or SPECTRAL (without qjl).  Values as PROD use their unbiased reconstruction
+ * ||v|| rot^T (c[code] + sqrt(pi/2)/m ||r|| S^T (2s-1)) (review, Method; the sign part is
+ * accumulated in the sketch domain and mapped back once per row).  libtq runs d = 128,
+ * code bits <= 4, PROD m = d, Hq/Hkv in 1..16; other shapes give TQ_ERR_UNSUPPORTED.  Value norms must stay below
  * 6.0e4 (the probability-weighted norm is a half-precision MMA operand).  The call
  * enqueues three kernels (query preparation, decode, chunk combine); the last two use
  * programmatic dependent launch, so each may start while the one before it drains, and
@@ -361,6 +363,64 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
                          const int32_t* seq_lens, tq_packed kcache, tq_packed vcache,
                          float scale, float* out, void* workspace, size_t ws_bytes,
                          tq_stream stream);
+
+/*
+ * Paged record pool (TurboQuant review, "Comparison": serving engines keep the cache in
+ * pages and quantize the tokens generated during decoding into it).  Every record array of
+ * a pool (codes, signs, norms, rnorms) holds num_pages pages; page p holds page_size
+ * consecutive records for each KV head, so token t of sequence b and KV head h is record
+ *     (block_table[b * max_pages + t / page_size] * Hkv + h) * page_size + t % page_size.
+ * block_table is a DEVICE int32 array [B][max_pages] owned by the caller; page ids must
+ * lie in 0..num_pages-1 (a page id out of range is read as page 0 and sets the device
+ * status to TQ_ERR_INVALID_ARG).  page_size is a multiple of 16.
+ */
+typedef struct {
+  const int32_t* block_table;
+  int32_t page_size;
+  int32_t max_pages;
+  int64_t num_pages;
+} tq_pages;
+
+/*
+ * DEVICE.  One decode step over a paged cache, appending the step's token first (review,
+ * "Comparison": decode-time tokens are quantized too).  For every (b, kv-head h):
+ *   1. k_new / v_new row b * Hkv + h ([B*Hkv*d], dtype) is quantized with kq / vq into
+ *      the record of token seq_lens[b] - 1 (its slot from the block table);
+ *   2. attention as tq_decode_attn over tokens 0..seq_lens[b]-1 of the pool.
+ * k_new and v_new may both be NULL (no append).  seq_lens [B] device int32 counts the
+ * tokens including the appended one (1..max_pages*page_size).  Workspace: the bytes
+ * tq_decode_attn_workspace gives for Nmax = max_pages * page_size.  Keys MSE or PROD,
+ * values MSE (spectral records are not paged: TQ_ERR_UNSUPPORTED).  The append runs as
+ * one extra kernel per array before the attention kernels, in stream order.
+ */
+tq_status tq_decode_attn_paged(const tq_quantizer* kq, const tq_quantizer* vq, const void* q,
+                               const void* k_new, const void* v_new, int32_t dtype, int32_t B, int32_t Hq,
+                               int32_t Hkv, const int32_t* seq_lens, const tq_pages* pages,
+                               tq_packed kpool, tq_packed vpool, float scale, float* out, void* workspace,
+                               size_t ws_bytes, tq_stream stream);
+
+/* Workspace bytes needed by tq_prefill_attn for this shape. */
+tq_status tq_prefill_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq, int32_t Hkv, int32_t T,
+                                    int64_t Nmax, size_t* bytes);
+
+/*
+ * DEVICE.  Causal prefill attention over the packed cache (TurboQuant launch kit, X thread
+ * and Show HN post: prefill at long context runs over the compressed cache).  For a block
+ * of T queries per sequence, q [B][Hq][T][d] (dtype), query (b, h, i) sits at absolute
+ * position q_pos[b * T + i] (DEVICE int32 [B][T], 0-based) and attends, with the decode
+ * step's scale and GQA map, to the cached tokens 0..q_pos[b*T+i] of its KV head:
+ *   out[b][h][i] = sum_{t <= pos} softmax_t(scale * est(q, k_t)) v_hat_t.
+ * kv_lens [B] (device int32) is the number of cached tokens of each sequence; every
+ * position must be below it.  The cache is the packed [B][Hkv][Nmax] layout (pages NULL)
+ * or a paged pool (pages non-NULL, Nmax ignored and taken as max_pages * page_size).
+ * out [B][Hq][T][d] fp32.  Keys MSE or PROD, values MSE, d = 128.  The cache must already
+ * hold the block's own tokens (quantize them first, as for decode).
+ */
+tq_status tq_prefill_attn(const tq_quantizer* kq, const tq_quantizer* vq, const void* q, int32_t dtype,
+                          int32_t B, int32_t Hq, int32_t Hkv, int32_t T, const int32_t* q_pos,
+                          const int32_t* kv_lens, const tq_pages* pages, int64_t Nmax, tq_packed kcache,
+                          tq_packed vcache, float scale, float* out, void* workspace, size_t ws_bytes,
+                          tq_stream stream);
 
 /* Size of the fixed device scratch array behind tq_decode_attn_fixed_ws (8 MiB per device). */
 #define TQ_DECODE_FIXED_WS_BYTES (8u << 20)

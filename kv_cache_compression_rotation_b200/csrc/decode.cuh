@@ -38,7 +38,7 @@ constexpr int kDecWarps = kDecThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int { KFMT_MSE = 0, KFMT_PROD = 1, KFMT_SPEC = 2 };
-enum : int { VFMT_MSE = 0, VFMT_SPEC = 2 };
+enum : int { VFMT_MSE = 0, VFMT_PROD = 1, VFMT_SPEC = 2 };
 
 struct DecodeParams {
   int B, Hq, Hkv, G;
@@ -76,6 +76,19 @@ struct DecodeParams {
   // partial results
   float* part_ml;       // [B*Hq][n_chunks][2]
   float* part_o;        // [B*Hq][n_chunks][D]
+  // paged pool (block_table != nullptr): token t of (b, kv-head h) is record
+  // (block_table[b * max_pages + t / page] * Hkv + h) * page + t % page of every array
+  const int32_t* block_table;
+  int page, max_pages;
+  int64_t num_pages;
+  // causal query rows (prefill): row r = (b * Hq_rows + ...) sees tokens t < q_pos[b * T + r % T] + 1
+  const int32_t* q_pos;
+  int T;
+  // values quantized as prod: sign words [recs][4], gamma [recs], S [128*128], sqrt(pi/2)/m
+  const uint32_t* vsigns;
+  const float* vrnorms;
+  const float* vS;
+  float v_coef;
 };
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {

@@ -100,11 +100,11 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
 }
 
 struct TmaStageLayout {
-  uint32_t kcodes, vcodes, knorm, vnorm, ksign, krn, bytes;
+  uint32_t kcodes, vcodes, knorm, vnorm, ksign, krn, vsign, vrn, bytes;
 };
 
 // Byte offsets of the arrays of one stage (all 16-byte aligned).
-__host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int kf, int ksw, bool pk) {
+__host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int kf, int ksw, bool pk, bool vpr = false) {
   const int st = tma_stage_tokens(kf, pk);
   TmaStageLayout L{};
   uint32_t o = 0;
@@ -117,6 +117,8 @@ __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int k
   L.vnorm = o; o += (kf == KFMT_SPEC) ? 0 : (st + 4) * 4;
   L.ksign = o; o += (kf == KFMT_PROD) ? st * ksw * 4 : 0;
   L.krn = o; o += (kf == KFMT_PROD || kf == KFMT_SPEC) ? (st + 4) * 4 : 0;
+  L.vsign = o; o += vpr ? st * 4 * 4 : 0;          // values as prod: 4 sign words and gamma
+  L.vrn = o; o += vpr ? (st + 4) * 4 : 0;
   L.bytes = o;
   return L;
 }
@@ -129,17 +131,18 @@ __host__ __device__ inline uint32_t tma_table_bytes(int kb, int vb) {
   return (1u << (2 * (kb > vb ? kb : vb))) * 256u;
 }
 __host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u : 8u; }
-__host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk) {
+__host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk, bool vpr = false) {
   const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf, pk)) * tma_merge_rows(pk) * (128u + 2u) * 4u;
-  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u + 510u * 4u + 8u;
+  // values as prod: the merged sign-domain sums of up to 8 rows
+  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u + 510u * 4u + 8u + (vpr ? 8u * 128u * 4u : 0u);
   return (v + 127u) & ~127u;
 }
 // words of one record: the code stream, plus the head word of a spectral record
 __host__ __device__ constexpr int tma_record_words(int bits, int kf) { return 128 * bits / 32 + (kf == KFMT_SPEC ? 1 : 0); }
-inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, bool pk) {
-  const TmaStageLayout L = tma_stage_layout(tma_record_words(kb, kf), tma_record_words(vb, kf), kf, 4, pk);
+inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, bool pk, bool vpr = false) {
+  const TmaStageLayout L = tma_stage_layout(tma_record_words(kb, kf), tma_record_words(vb, kf), kf, 4, pk, vpr);
   const size_t want = 65536 + tma_table_bytes(kb, vb) + static_cast<size_t>(tma_stages(pk)) * L.bytes +
-                      tma_misc_bytes(kf, pk);
+                      tma_misc_bytes(kf, pk, vpr);
   return want < 232448 ? want : 232448;
 }
 
@@ -211,7 +214,14 @@ __device__ __forceinline__ float ex2(float x) {
 // instruction (summed across lanes t and t ^ 2), and P's hi / lo split rides in the same
 // columns of the value MMA (summed in the merge).  Without PK the 8 columns are 8 heads and
 // the hi / lo parts take separate MMAs.
-template <int KF, int KB, int VB, bool PK>
+// CZ (prefill): query row r only sees tokens below its causal limit q_pos[b * T + r % T] + 1;
+// a work item stops at the largest limit of its rows.
+// VPR: values quantized as TurboQuant-prod (VB = bits of their MSE stage, m = d = 128 sign
+// bits and gamma per value).  The unbiased reconstruction adds sqrt(pi/2)/m gamma S^T (2s-1)
+// to c[code] (rotated domain), so the step also accumulates the sign-domain sum
+// a = sum_i p_i ||v_i|| gamma_i (2 s_i - 1) with a third MMA per unit (A = the +-1 signs), and
+// the merge of an item folds sqrt(pi/2)/m S^T a into its partial o'.
+template <int KF, int KB, int VB, bool PK, bool CZ = false, bool VPR = false>
 __global__ void __launch_bounds__((tma_consumers(KF, PK) + 1) * 32, 1)
 decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int NC = tma_consumers(KF, PK);   // consumer warps
@@ -242,7 +252,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   // Table entry e is 256 B: the key value pair for lanes 0..31, then the value pair.  With the
   // table base B (a multiple of 64 KB), the lookup address of a code pair byte x for this lane
   // is B | x << 8 | lane * 4 [+ 128]: one byte permute, no add.
-  const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW, PK);
+  const TmaStageLayout SL = tma_stage_layout(KW, VW, KF, KSW, PK, VPR);
   const uint32_t base = tma_smem_u32(tsm_);
   uint32_t dyn;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
@@ -256,7 +266,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     after += bytes;
     return a0;
   };
-  const uint32_t miscA = place(tma_misc_bytes(KF, PK));
+  const uint32_t miscA = place(tma_misc_bytes(KF, PK, VPR));
   uint32_t stA[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
   for (int i = 0; i < NS; ++i) stA[i] = place(SL.bytes);
@@ -280,6 +290,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   volatile int* abort_flag = nb_off + NS;
   volatile int* consumers_stop = abort_flag + 1;   // uniform exit decision of the consumer warps
   float* utab = reinterpret_cast<float*>(const_cast<int*>(consumers_stop) + 2);   // spectral unit codebooks [510]
+  float* asum = utab + 510;                        // values as prod: merged sign-domain sums [8][128]
   const uint32_t bar0 = tma_smem_u32(bars);
   const uint32_t nb_a = tma_smem_u32(nb_count);
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
@@ -291,6 +302,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   const int nhb = PK ? 1 : tma_head_blocks(G);
   const int n_items = p.B * p.Hkv * nhb * p.n_chunks;
   const int64_t total_recs = static_cast<int64_t>(p.B) * p.Hkv * p.Nmax;
+  // causal limit of query row r (prefill)
+  auto row_limit = [&](int bb, int64_t r) { return p.q_pos[bb * p.T + static_cast<int>(r % p.T)] + 1; };
   // item -> (bh, head block, chunk, token range)
   auto item_range = [&](int item, int& bh, int& hblk, int& chunk, int& k0, int& k1) {
     chunk = item % p.n_chunks;
@@ -298,7 +311,15 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     hblk = rest % nhb;
     bh = rest / nhb;
     const int bb = bh / p.Hkv;
-    const int len = static_cast<int>(min(static_cast<int64_t>(p.seq_lens[bb]), p.Nmax));
+    int len = static_cast<int>(min(static_cast<int64_t>(p.seq_lens[bb]), p.Nmax));
+    if constexpr (CZ) {
+      // no token past the block's largest causal limit is visible to any of its rows
+      const int hb = PK ? 4 : kTmaHeadBlock;
+      const int64_t r0 = static_cast<int64_t>(bb) * p.Hq + (bh - bb * p.Hkv) * G + hblk * hb;
+      int mx = 0;
+      for (int c = 0; c < min(hb, G - hblk * hb); ++c) mx = max(mx, row_limit(bb, r0 + c));
+      len = min(len, mx);
+    }
     k0 = chunk * p.chunk_len;
     k1 = min(len, k0 + p.chunk_len);
   };
@@ -386,11 +407,56 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
                   __ldg(reinterpret_cast<const uint32_t*>(vg + b));
             __syncwarp();
           }
+          if (!SP && p.block_table) {
+            // paged pool: the stage is cut at page boundaries and each piece copied from its
+            // page (pages hold a multiple of 16 tokens and stages start on multiples of 16, so
+            // every piece is 16-byte aligned; norms are copied in whole groups of 4, which the
+            // page holds)
+            if (lane == 0) {
+              const int bb = bh / p.Hkv, hk = bh - bb * p.Hkv;
+              nb_count[st] = cnt;
+              nb_off[st] = 0;
+              uint32_t bytes = 0u;
+              for (int tt = t0; tt < t0 + cnt;) {
+                const int seg = min(t0 + cnt, (tt / p.page + 1) * p.page) - tt, nseg = (seg + 3) & ~3;
+                bytes += seg * (KW + VW) * 4 + 2 * nseg * 4;
+                if (KF == KFMT_PROD) bytes += seg * KSW * 4 + nseg * 4;
+                if (VPR) bytes += seg * 16 + nseg * 4;
+                tt += seg;
+              }
+              asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
+              for (int tt = t0; tt < t0 + cnt;) {
+                const int pi = tt / p.page, seg = min(t0 + cnt, (pi + 1) * p.page) - tt, nseg = (seg + 3) & ~3;
+                int pg = p.block_table[static_cast<int64_t>(bb) * p.max_pages + pi];
+                if (pg < 0 || pg >= p.num_pages) {            // a bad page id reads page 0
+                  report_status(status, TQ_ERR_INVALID_ARG);
+                  pg = 0;
+                }
+                const int64_t rr = (static_cast<int64_t>(pg) * p.Hkv + hk) * p.page + (tt - pi * p.page);
+                const uint32_t so = static_cast<uint32_t>(tt - t0);
+                bulk_g2s(sb + SL.kcodes + so * KW * 4, p.kcodes + rr * KW, seg * KW * 4, fb);
+                bulk_g2s(sb + SL.vcodes + so * VW * 4, p.vcodes + rr * VW, seg * VW * 4, fb);
+                bulk_g2s(sb + SL.knorm + so * 4, p.knorms + rr, nseg * 4, fb);
+                bulk_g2s(sb + SL.vnorm + so * 4, p.vnorms + rr, nseg * 4, fb);
+                if (KF == KFMT_PROD) {
+                  bulk_g2s(sb + SL.ksign + so * KSW * 4, p.ksigns + rr * KSW, seg * KSW * 4, fb);
+                  bulk_g2s(sb + SL.krn + so * 4, p.krnorms + rr, nseg * 4, fb);
+                }
+                if (VPR) {
+                  bulk_g2s(sb + SL.vsign + so * 16, p.vsigns + rr * 4, seg * 16, fb);
+                  bulk_g2s(sb + SL.vrn + so * 4, p.vrnorms + rr, nseg * 4, fb);
+                }
+                tt += seg;
+              }
+            }
+            continue;
+          }
           if (lane == 0) {
             nb_count[st] = max(0, nn - off);
             nb_off[st] = off;
             uint32_t bytes = SP ? sp_bytes : cnt * (KW + VW) * 4 + 2 * nn * 4;
             if (KF == KFMT_PROD) bytes += cnt * KSW * 4 + nn * 4;
+            if (VPR) bytes += cnt * 16 + nn * 4;
             if (SP && p.krnorms) bytes += nn * 4;
             // the arrival releases the word copies above (spectral) and expects the bulk bytes
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
@@ -414,6 +480,10 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             if (KF == KFMT_PROD) {
               bulk_g2s(sb + SL.ksign, p.ksigns + r * KSW, cnt * KSW * 4, fb);
               if (nn > 0) bulk_g2s(sb + SL.krn, p.krnorms + (r - off), nn * 4, fb);
+            }
+            if (VPR) {
+              bulk_g2s(sb + SL.vsign, p.vsigns + r * 4, cnt * 16, fb);
+              if (nn > 0) bulk_g2s(sb + SL.vrn, p.vrnorms + (r - off), nn * 4, fb);
             }
           }
         }
@@ -501,7 +571,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         ql[k][0] = l01; ql[k][1] = l23;
       }
     }
-    uint32_t qb[KST][2];
+    uint32_t qb[KST][2], qbl[PK ? 1 : KST][2];     // QJL operand (hi; lo without packed columns)
     if constexpr (KF == KFMT_PROD) {
 #pragma unroll
       for (int k = 0; k < KST; ++k) {
@@ -518,8 +588,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           qb[k][0] = qlo ? l01 : h01;
           qb[k][1] = qlo ? l23 : h23;
         } else {
-          qb[k][0] = pack_half2(a[0], a[1]);
-          qb[k][1] = pack_half2(a[2], a[3]);
+          split_pair(a[0], a[1], qb[k][0], qbl[k][0]);
+          split_pair(a[2], a[3], qb[k][1], qbl[k][1]);
         }
       }
     }
@@ -540,6 +610,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     }
     // this thread's score columns are heads h0, h0 + 1 of the block
     const bool c0ok = h0 < nh, c1ok = h0 + 1 < nh;
+    int lim0 = 0x7fffffff, lim1 = 0x7fffffff;      // causal limits of those rows (prefill)
+    if constexpr (CZ) {
+      if (c0ok) lim0 = row_limit(bb, qbase + h0);
+      if (c1ok) lim1 = row_limit(bb, qbase + h0 + 1);
+    }
     const float sa0 = c0ok ? p.qs[(qbase + h0) * 2] * p.k_scale : 0.f;
     const float sa1 = c1ok ? p.qs[(qbase + h0 + 1) * 2] * p.k_scale : 0.f;
     const float sb0 = c0ok ? p.qs[(qbase + h0) * 2 + 1] * (SP ? 1.f : p.qjl_coef) : 0.f;
@@ -548,6 +623,10 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     float o[MT][4];
 #pragma unroll
     for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    // values as prod: sign-domain sums, row g = sign index TDV g + i, row g + 8 = TDV g + 8 + i
+    float os[VPR ? MT : 1][4];
+#pragma unroll
+    for (int i = 0; i < (VPR ? MT : 1); ++i) os[i][0] = os[i][1] = os[i][2] = os[i][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads h0, h0 + 1
     float oh[4] = {0.f, 0.f, 0.f, 0.f};   // spectral: top value dim g (columns 2t, 2t + 1)
 
@@ -568,6 +647,10 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       uint32_t sw[U][2];
       uint32_t vs[U][4][NWV];
       uint32_t hk[U][2], hv[U][4];                   // spectral head words (keys by row, values by k-index)
+      // values as prod: this thread's 16 sign bits (signs TDV g ..) of the value-operand tokens,
+      // and gamma of the score-row tokens
+      uint32_t vsw[VPR ? U : 1][4];
+      float vgm[VPR ? U : 1][2];
       if (cnt == kTmaStageTokens && nn >= cnt) {
         // a whole stage with every norm staged (all but the last stage of a chunk): no
         // per-token checks
@@ -590,11 +673,14 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
               gm[u][h] = sldf(sb + SL.krn + 4 * (noff + tk));
               sw[u][h] = sld32(sb + SL.ksign + (tk * KSW + t) * 4);
             }
+            if constexpr (VPR) vgm[u][h] = sldf(sb + SL.vrn + 4 * (noff + tk));
           }
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             sld_slice<NWV>(vcb + (w0 + 16 * u + kv[i]) * VW * 4, VW, TOFF + g * TDV * VB, true, vs[u][i]);
             if constexpr (SP) hv[u][i] = sld32(vcb + (w0 + 16 * u + kv[i]) * VW * 4);
+            if constexpr (VPR)
+              vsw[u][i] = (sld32(sb + SL.vsign + ((w0 + 16 * u + kv[i]) * 4 + (g >> 1)) * 4) >> (16 * (g & 1))) & 0xFFFFu;
           }
         }
       } else {
@@ -621,12 +707,15 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
               gm[u][h] = norm_of(sb + SL.krn, p.krnorms, tk, okk);
               sw[u][h] = okk ? sld32(sb + SL.ksign + (tk * KSW + t) * 4) : 0u;
             }
+            if constexpr (VPR) vgm[u][h] = norm_of(sb + SL.vrn, p.vrnorms, tk, okk);
           }
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int lk = w0 + 16 * u + kv[i];
             sld_slice<NWV>(vcb + lk * VW * 4, VW, TOFF + g * TDV * VB, lk < cnt, vs[u][i]);
             if constexpr (SP) hv[u][i] = lk < cnt ? sld32(vcb + lk * VW * 4) : 0u;
+            if constexpr (VPR)
+              vsw[u][i] = lk < cnt ? (sld32(sb + SL.vsign + (lk * 4 + (g >> 1)) * 4) >> (16 * (g & 1))) & 0xFFFFu : 0u;
           }
         }
       }
@@ -676,6 +765,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             const uint32_t a2 = tab_ld(luts_a + ((((sw[u][0] >> (4 * k + 2)) & 3u) << 5) + lane) * 4);
             const uint32_t a3 = tab_ld(luts_a + ((((sw[u][1] >> (4 * k + 2)) & 3u) << 5) + lane) * 4);
             mma16816(acc2, a0, a1, a2, a3, qb[k][0], qb[k][1]);
+            if constexpr (!PK) mma16816(acc2, a0, a1, a2, a3, qbl[k][0], qbl[k][1]);
           }
         }
         if constexpr (SP) {
@@ -717,8 +807,14 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
                            make_float2(acc2[2 * h], acc2[2 * h + 1]), v);
           if constexpr (SP) v = __ffma2_rn(make_float2(sb0, sb1), make_float2(acc2[2 * h], acc2[2 * h + 1]), v);
           v = __fmul2_rn(make_float2(kn[u][h], kn[u][h]), v);
-          sc[u][2 * h] = ok[u][h] ? v.x : -INFINITY;
-          sc[u][2 * h + 1] = ok[u][h] ? v.y : -INFINITY;
+          if constexpr (CZ) {
+            const int tok = t0 + w0 + 16 * u + 8 * h + pg;     // absolute token of score row g + 8 h
+            sc[u][2 * h] = (ok[u][h] && tok < lim0) ? v.x : -INFINITY;
+            sc[u][2 * h + 1] = (ok[u][h] && tok < lim1) ? v.y : -INFINITY;
+          } else {
+            sc[u][2 * h] = ok[u][h] ? v.x : -INFINITY;
+            sc[u][2 * h + 1] = ok[u][h] ? v.y : -INFINITY;
+          }
         }
       }
       // ---- online softmax per head (log2 domain) over the warp's tokens; the row
@@ -740,7 +836,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         }
         const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
         if (mn0 > m0 || mn1 > m1) {
-          const float f0 = ex2(m0 - mn0), f1 = ex2(m1 - mn1);
+          // (causal rows: a row still fully masked keeps max -inf and nothing to rescale)
+          const float f0 = (CZ && m0 == -INFINITY) ? 0.f : ex2(m0 - mn0);
+          const float f1 = (CZ && m1 == -INFINITY) ? 0.f : ex2(m1 - mn1);
           l0 *= f0;
           l1 *= f1;
           const float2 f01 = make_float2(f0, f1);
@@ -751,13 +849,24 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             o[i][0] = a.x; o[i][1] = a.y; o[i][2] = b.x; o[i][3] = b.y;
           }
           if constexpr (SP) { oh[0] *= f0; oh[1] *= f1; }
+          if constexpr (VPR) {
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+              const float2 a = __fmul2_rn(make_float2(os[i][0], os[i][1]), f01);
+              const float2 b = __fmul2_rn(make_float2(os[i][2], os[i][3]), f01);
+              os[i][0] = a.x; os[i][1] = a.y; os[i][2] = b.x; os[i][3] = b.y;
+            }
+          }
           m0 = mn0;
           m1 = mn1;
         }
       }
+      // a causal row whose tokens of this warp are all masked keeps max -inf: its
+      // probabilities are exp2(-inf - 0) = 0, not exp2(-inf + inf)
+      const float ms0 = (CZ && m0 == -INFINITY) ? 0.f : m0, ms1 = (CZ && m1 == -INFINITY) ? 0.f : m1;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const float2 nm = make_float2(-m0, -m1);
+        const float2 nm = make_float2(-ms0, -ms1);
         const float2 d0 = __fadd2_rn(make_float2(sc[u][0], sc[u][1]), nm);
         const float2 d1 = __fadd2_rn(make_float2(sc[u][2], sc[u][3]), nm);
         const float p00 = c0ok ? ex2(d0.x) : 0.f, p01 = c1ok ? ex2(d0.y) : 0.f;
@@ -798,6 +907,43 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           }
           oh[0] = ohx[0];
           oh[1] = ohx[1];
+        }
+        if constexpr (VPR) {
+          // ---- A^T[128 signs x 8 columns] += (2 s - 1)^T . (P gamma)^T ----
+          // weights p ||v|| gamma of the score rows, split and transposed like P
+          const float2 pw0 = __fmul2_rn(pv0, make_float2(vgm[u][0], vgm[u][0]));
+          const float2 pw1 = __fmul2_rn(pv1, make_float2(vgm[u][1], vgm[u][1]));
+          uint32_t wth, wtl, wbh, wbl;
+          split_pair(pw0.x, pw0.y, wth, wtl);
+          split_pair(pw1.x, pw1.y, wbh, wbl);
+          uint32_t c0h, c1h, c0l = 0u, c1l = 0u;
+          if constexpr (PK) {
+            c0h = movmatrix_t(plo ? wtl : wth);
+            c1h = movmatrix_t(plo ? wbl : wbh);
+          } else {
+            c0h = movmatrix_t(wth); c1h = movmatrix_t(wbh);
+            c0l = movmatrix_t(wtl); c1l = movmatrix_t(wbl);
+          }
+          // bit j of token kv[0] (kv[2]) at bit 2 j, of kv[1] (kv[3]) at bit 2 j + 1: the A entry
+          // pair of rows (sign i, tokens k, k + 1) is a 2-bit index into the +-1 pair table
+          auto spread = [](uint32_t v) {
+            v = (v | (v << 8)) & 0x00FF00FFu;
+            v = (v | (v << 4)) & 0x0F0F0F0Fu;
+            v = (v | (v << 2)) & 0x33333333u;
+            return (v | (v << 1)) & 0x55555555u;
+          };
+          const uint32_t z01 = spread(vsw[u][0]) | (spread(vsw[u][1]) << 1);
+          const uint32_t z23 = spread(vsw[u][2]) | (spread(vsw[u][3]) << 1);
+          const uint32_t lane4 = luts_a + static_cast<uint32_t>(lane) * 4u;
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const uint32_t a0 = tab_ld(lane4 + ((z01 >> (2 * i)) & 3u) * 128u);
+            const uint32_t a1 = tab_ld(lane4 + ((z01 >> (16 + 2 * i)) & 3u) * 128u);
+            const uint32_t a2 = tab_ld(lane4 + ((z23 >> (2 * i)) & 3u) * 128u);
+            const uint32_t a3 = tab_ld(lane4 + ((z23 >> (16 + 2 * i)) & 3u) * 128u);
+            mma16816(os[i], a0, a1, a2, a3, c0h, c1h);
+            if constexpr (!PK) mma16816(os[i], a0, a1, a2, a3, c0l, c1l);
+          }
         }
         // ---- O'^T[128 dims x 8 columns] += V_hat^T . P^T ----
         // M-tile i: row g = dim TDV g + i (first word of the slice), row g + 8 = dim TDV g + 8 + i
@@ -896,6 +1042,50 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       const int64_t pi = qi * p.n_chunks + chunk;
       if (j == 0) { p.part_ml[pi * 2] = M; p.part_ml[pi * 2 + 1] = L; }
       p.part_o[pi * D + j] = a * p.v_scale;
+    }
+    if constexpr (VPR) {
+      // fold sqrt(pi/2)/m S^T a into the partial: merge the warps' sign-domain sums with the
+      // same chunk weights, then one matrix-vector product per row with S from global memory
+      if constexpr (PK) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) os[i][j] += __shfl_xor_sync(0xffffffffu, os[i][j], 2);
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");   // every warp has read mrg
+      if (!PK || t < 2) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = os[i][0];
+          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = os[i][1];
+          wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = os[i][2];
+          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = os[i][3];
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+      for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
+        const int r = idx / D, j = idx - r * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NC; ++w) M = fmaxf(M, mrg[(w * RW + r) * (D + 2)]);
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < NC; ++w) {
+          const float* row = mrg + (w * RW + r) * (D + 2);
+          const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
+          a += f * row[2 + j];
+        }
+        asum[r * D + j] = a;
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+      for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
+        const int r = idx / D, j = idx - r * D;
+        float c = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) c = fmaf(__ldg(p.vS + i * D + j), asum[r * D + i], c);
+        const int64_t pi = (qbase + r) * p.n_chunks + chunk;
+        p.part_o[pi * D + j] += p.v_coef * c;
+      }
     }
     // every consumer warp takes the same exit decision: one thread samples the abort
     // flag between the two barriers (a warp that timed out still reaches both)

@@ -39,9 +39,18 @@ cudaError_t launch_decode_prod(const DecodeParams& p, int kb, int vb, dim3 grid,
                                int* status, long long lim);
 cudaError_t launch_decode_spec(const DecodeParams& p, int kb, int vb, dim3 grid, size_t smem, cudaStream_t s);
 cudaError_t launch_decode_spec_tma(const DecodeParams& p, dim3 grid, cudaStream_t s, int* status, long long lim);
+// Values quantized as prod (MSE-stage bits 1..4, m = 128): MSE / PROD keys.
+cudaError_t launch_decode_vprod(const DecodeParams& p, int kfmt, int kb, int vb, dim3 grid, cudaStream_t s,
+                                int* status, long long lim);
+// Causal query blocks (prefill): MSE / PROD keys (bits of the MSE stage 1..4), MSE values.
+cudaError_t launch_decode_causal(const DecodeParams& p, int kfmt, int kb, int vb, dim3 grid, cudaStream_t s,
+                                 int* status, long long lim);
 
 // Tensor-core quantize (d = 128, 16-bit input, MSE bits 1..4).
 cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& p, int bits, int grid,
                                  cudaStream_t stream);
+// TurboQuant-prod with m = d = 128: the rotation and the QJL projection on the tensor cores
+cudaError_t launch_umma_quantize_prod(const CUtensorMap& map, const UmmaQuantParams& p, int mse_bits, int grid,
+                                      cudaStream_t s);
 
 }  // namespace tq

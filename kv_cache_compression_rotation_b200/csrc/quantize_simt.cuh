@@ -49,7 +49,25 @@ struct SimtQuantParams {
   int64_t ld;
   const int32_t* cols;
   int* status;
+  // output rows: record v goes to slot orow(v) (paged append: vector v = b * Hkv + h is the
+  // newest token seq_lens[b] - 1 of (b, h), placed through the block table)
+  const int32_t* pg_table;    // [B][pg_max] page ids, or nullptr (record v at slot v)
+  const int32_t* pg_seq;      // [B] token counts including the appended one
+  int pg_size, pg_max, pg_hkv;
+  int64_t pg_num;
 };
+
+// Record slot of output vector v; -1 when the block table or the length is out of range
+// (reported as TQ_ERR_INVALID_ARG by the caller of this function, and nothing is written).
+__device__ __forceinline__ int64_t simt_out_row(const SimtQuantParams& p, int64_t v) {
+  if (!p.pg_table) return v;
+  const int b = static_cast<int>(v / p.pg_hkv), h = static_cast<int>(v - static_cast<int64_t>(b) * p.pg_hkv);
+  const int t = p.pg_seq[b] - 1;
+  if (t < 0 || t >= p.pg_size * p.pg_max) return -1;
+  const int pg = p.pg_table[static_cast<int64_t>(b) * p.pg_max + t / p.pg_size];
+  if (pg < 0 || pg >= p.pg_num) return -1;
+  return (static_cast<int64_t>(pg) * p.pg_hkv + h) * p.pg_size + t % p.pg_size;
+}
 
 __device__ __forceinline__ void spectral_dim_book(const SimtQuantParams& p, int j, int* bits,
                                                   float* sig) {
@@ -213,7 +231,8 @@ simt_quantize_kernel(SimtQuantParams p) {
         if (pos >= 0) word |= static_cast<uint32_t>(c << pos);
         else word |= static_cast<uint32_t>(c >> (-pos));
       }
-      p.codes[(v0 + v) * p.code_words + hw + w] = word;
+      const int64_t o = simt_out_row(p, v0 + v);
+      if (o >= 0) p.codes[o * p.code_words + hw + w] = word;
     }
     if (tid < tv && tid < nv) {
       const int v = tid;
@@ -241,12 +260,15 @@ simt_quantize_kernel(SimtQuantParams p) {
       for (int j = 0; j < k; ++j) put(code8[v * d + j], p.top_bits[j]);
       if (p.qjl)
         for (int i = 0; i < k; ++i) put(proj[i] >= 0.f ? 1u : 0u, 1);
-      uint32_t* dst = p.codes + (v0 + v) * p.code_words;
-      for (int w = 0; w < hw; ++w) {
-        const uint64_t src = head[w >> 1];
-        dst[w] = static_cast<uint32_t>((w & 1) ? (src >> 32) : src);
+      const int64_t orow = simt_out_row(p, v0 + v);
+      if (orow >= 0) {
+        uint32_t* dst = p.codes + orow * p.code_words;
+        for (int w = 0; w < hw; ++w) {
+          const uint64_t src = head[w >> 1];
+          dst[w] = static_cast<uint32_t>((w & 1) ? (src >> 32) : src);
+        }
+        if (p.qjl && p.rnorms) p.rnorms[orow] = sqrtf(g2);
       }
-      if (p.qjl && p.rnorms) p.rnorms[v0 + v] = sqrtf(g2);
       (void)extra;
     }
     return;
@@ -265,10 +287,15 @@ simt_quantize_kernel(SimtQuantParams p) {
         if (pos >= 0) word |= static_cast<uint32_t>(c << pos);
         else word |= static_cast<uint32_t>(c >> (-pos));
       }
-      p.codes[(v0 + v) * W + w] = word;
+      const int64_t o = simt_out_row(p, v0 + v);
+      if (o >= 0) p.codes[o * W + w] = word;
     }
   }
-  if (tid < nv && p.norms) p.norms[v0 + tid] = nu[tid];
+  if (tid < nv) {
+    const int64_t o = simt_out_row(p, v0 + tid);
+    if (o < 0) report_status(p.status, TQ_ERR_INVALID_ARG);
+    else if (p.norms) p.norms[o] = nu[tid];
+  }
   if (p.kind != TQ_KIND_PROD) return;
   // prod: gamma = ||r||, then S r for the tile (tiled product) and its signs by warp ballot
   for (int v = warp; v < tv; v += kSimtThreads / 32) {
@@ -278,7 +305,10 @@ simt_quantize_kernel(SimtQuantParams p) {
     if (lane == 0) gam[v] = sqrtf(s);
   }
   __syncthreads();
-  if (tid < nv && p.rnorms) p.rnorms[v0 + tid] = gam[tid];
+  if (tid < nv && p.rnorms) {
+    const int64_t o = simt_out_row(p, v0 + tid);
+    if (o >= 0) p.rnorms[o] = gam[tid];
+  }
   switch (tv / 8) {
     case 1: tile_gemm<1>(xs, dp, p.S, p.m, d, ys, yp, nullptr, Ms); break;
     case 2: tile_gemm<2>(xs, dp, p.S, p.m, d, ys, yp, nullptr, Ms); break;
@@ -289,7 +319,8 @@ simt_quantize_kernel(SimtQuantParams p) {
     for (int ib = 0; ib < p.m; ib += 32) {
       const int i = ib + lane;
       const unsigned bits = __ballot_sync(0xffffffffu, i < p.m && ys[v * yp + min(i, p.m - 1)] >= 0.f);
-      if (lane == 0) p.signs[(v0 + v) * p.sign_words + (ib >> 5)] = bits;
+      const int64_t o = simt_out_row(p, v0 + v);
+      if (lane == 0 && o >= 0) p.signs[o * p.sign_words + (ib >> 5)] = bits;
     }
   }
 }

@@ -5,12 +5,13 @@
 namespace tq {
 namespace {
 
-template <int B, bool SPEC = false>
+template <int B, bool SPEC = false, bool PRODK = false>
 cudaError_t go(const CUtensorMap& map, const UmmaQuantParams& p, int grid, cudaStream_t s) {
-  auto k = umma_quantize_kernel<B, SPEC>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kUmmaSmemBytes));
+  auto k = umma_quantize_kernel<B, SPEC, PRODK>;
+  const uint32_t smem = PRODK ? kUmmaProdSmemBytes : kUmmaSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k<<<grid, kUmmaThreads, kUmmaSmemBytes, s>>>(map, p);
+  k<<<grid, kUmmaThreads, smem, s>>>(map, p);
   return cudaGetLastError();
 }
 
@@ -24,6 +25,17 @@ cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& 
     case 2: return go<2>(map, p, grid, s);
     case 3: return go<3>(map, p, grid, s);
     case 4: return go<4>(map, p, grid, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+cudaError_t launch_umma_quantize_prod(const CUtensorMap& map, const UmmaQuantParams& p, int mse_bits, int grid,
+                                      cudaStream_t s) {
+  switch (mse_bits) {
+    case 1: return go<1, false, true>(map, p, grid, s);
+    case 2: return go<2, false, true>(map, p, grid, s);
+    case 3: return go<3, false, true>(map, p, grid, s);
+    case 4: return go<4, false, true>(map, p, grid, s);
     default: return cudaErrorNotSupported;
   }
 }

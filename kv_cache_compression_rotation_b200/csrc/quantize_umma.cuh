@@ -23,6 +23,15 @@
 // code = (#boundaries below the cell) + (u > boundary in the cell).  A codebook whose
 // gaps are narrower than the cells falls back to counting all boundaries.
 // ||y|| equals ||x|| up to the orthogonality of the fp32 Pi (~1e-7 relative).
+// TurboQuant-prod (PRODK instantiation, m = d = 128): the (b-1)-bit MSE stage as above,
+// then the QJL projection of the unit-scale residual r = u - c[code] is a second tensor-
+// core product Z[128 x 128] = R . S^T.  The epilogue writes r as fp16 hi + lo parts into
+// tensor memory, where it is the A operand (S hi + lo in shared memory is B); the three
+// products R_hi S_hi + R_hi S_lo + R_lo S_hi keep every projection within ~1e-6 ||S_i|| ||r||
+// of the fp32 value, far inside the 1e-5 ||S_i|| sign band.  Tensor memory, per epilogue
+// group (tile parity): a 128-column accumulator that holds Y and then Z (the projection
+// overwrites Y once the group has read it) and 128 columns of R_hi | R_lo, 512 in all; the
+// accumulator goes back to the MMA warp after the group has read Z.
 // Every mbarrier wait is bounded; on timeout the CTA records TQ_ERR_TIMEOUT, drains
 // what it issued, frees TMEM and exits.
 #pragma once
@@ -48,6 +57,9 @@ constexpr float kCellSpan = 31.9999f;
 constexpr int kSpecMaxTopBits = 6;
 constexpr uint32_t kSpecTabBytes = (TQ_MAX_TOP * 64 * 2 + 64) * 4;
 constexpr uint32_t kUmmaSmemBytes = 1024 /*align slack*/ + 2 * kPiBytes + kUmmaStages * kXStageBytes + 256 + kSpecTabBytes;
+// prod: Pi hi + lo and S hi + lo (fp16), a 3-stage ring, barriers and the centroid table
+constexpr int kProdStages = 3;
+constexpr uint32_t kUmmaProdSmemBytes = 1024 + 4 * kPiBytes + kProdStages * kXStageBytes + 256 + 64 * 4;
 
 struct UmmaQuantParams {
   const float* rot;        // [128*128] fp32
@@ -69,6 +81,9 @@ struct UmmaQuantParams {
   // rotations with entries +-pm1_scale: one exact +-1 MMA operand, no low-order term
   int pm1;
   float pm1_scale;         // 1/sqrt(d) as fp32
+  // prod (m = 128): S [128*128] fp32 is the field S above; MSE-stage centroids, sign words
+  const float* centroids;  // [2^B]
+  uint32_t* signs;         // [n][4]
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -146,6 +161,27 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64
       ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// Same, with the A operand read from tensor memory (M rows = lanes, K 16-bit elements
+// packed two per 32-bit column).
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+      ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                ::"r"(bar) : "memory");
@@ -187,7 +223,7 @@ __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B
 // tail dims take 1 bit, code (z_j > 0) (the 1-bit standard-normal boundary is 0); the top
 // dims are coded against sigma_j times their unit codebooks and get the QJL signs of
 // S (z_top - c_top); record = head word + 4 tail words (+ ||z_top - c_top||).
-template <int B, bool SPEC>
+template <int B, bool SPEC, bool PRODK = false>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
 umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantParams p) {
   constexpr int K = 1 << B;
@@ -197,25 +233,36 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   // data is densest: Pi takes three 16-bit terms (hi + lo + lo2, ~2^-26 relative) instead of
   // two, and the ring one stage less so the shared memory stays the same
   constexpr int NT = SPEC ? 3 : 2;
-  constexpr int NS = SPEC ? 3 : kUmmaStages;
-  static_assert(NT * kPiBytes + NS * kXStageBytes == 2 * kPiBytes + kUmmaStages * kXStageBytes, "smem");
+  constexpr int NS = SPEC ? 3 : (PRODK ? kProdStages : kUmmaStages);
+  // 32 KB operand blocks before the ring: Pi terms, and for prod S hi + lo
+  constexpr int NPI = PRODK ? 4 : NT;
+  static_assert(PRODK || NT * kPiBytes + NS * kXStageBytes == 2 * kPiBytes + kUmmaStages * kXStageBytes, "smem");
+  static_assert(!PRODK || 1024 + NPI * kPiBytes + NS * kXStageBytes + 256 + 64 * 4 <= kUmmaProdSmemBytes, "smem");
+  constexpr uint32_t kTmemCols = PRODK ? 512u : 256u;
+  // prod tensor-memory columns of buffer b: Y then Z at 128 b, R_hi at 256 + 128 b, R_lo 64 after
+  constexpr uint32_t kR = 256u;
   extern __shared__ unsigned char usm_raw[];
   const uint32_t raw = smem_u32(usm_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = usm_raw + (base - raw);
   const uint32_t pi_hi = base, pi_lo = base + kPiBytes, pi_lo2 = base + 2 * kPiBytes;
-  const uint32_t xs0 = base + NT * kPiBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + NT * kPiBytes + NS * kXStageBytes);
+  const uint32_t s_hi = base + 2 * kPiBytes, s_lo = base + 3 * kPiBytes;   // prod only
+  const uint32_t xs0 = base + NPI * kPiBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + NPI * kPiBytes + NS * kXStageBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * NS + 2 + b); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 4);
+  // prod, per buffer: R written (count 128), Z committed (1)
+  auto rfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 4 + b); };
+  auto zfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 6 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + (PRODK ? 8 : 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tsm = reinterpret_cast<float*>(tmem_slot + 2);   // boundaries [NB]
   // spectral: thresholds [top dim][64], centroids [top dim][64], S [64]
-  float* sthr = reinterpret_cast<float*>(sm + NT * kPiBytes + NS * kXStageBytes + 256);
+  float* sthr = reinterpret_cast<float*>(sm + NPI * kPiBytes + NS * kXStageBytes + 256);
+  float* pcen = sthr;                                     // prod: MSE-stage centroids [2^B]
   float* scen = sthr + TQ_MAX_TOP * 64;
   float* sS = scen + TQ_MAX_TOP * 64;
 
@@ -260,9 +307,25 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   } else {
     if (tid < NB) tsm[tid] = __ldg(p.boundaries + tid);
   }
+  if constexpr (PRODK) {
+    // S_hi / S_lo (fp16) in the same swizzled K-major layout: row = projection i, k = dim
+    for (int i = tid; i < kUmmaD * kUmmaD; i += kUmmaThreads) {
+      const int nrow = i >> 7, k = i & 127;
+      const float v = __ldg(p.S + i);
+      const __half h = __float2half_rn(v);
+      const __half l = __float2half_rn(v - __half2float(h));
+      const int kb = k >> 6, kk = k & 63;
+      const uint32_t off = kb * (kUmmaD * 128) + nrow * 128 + ((((kk >> 3) ^ (nrow & 7))) << 4) + (kk & 7) * 2;
+      *reinterpret_cast<uint16_t*>(sm + 2 * kPiBytes + off) = __half_as_ushort(h);
+      *reinterpret_cast<uint16_t*>(sm + 3 * kPiBytes + off) = __half_as_ushort(l);
+    }
+    if (tid < K) pcen[tid] = __ldg(p.centroids + tid);
+  }
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), 128); }
+    if (PRODK)
+      for (int b = 0; b < 2; ++b) { mbar_init(rfull_bar(b), 128); mbar_init(zfull_bar(b), 1); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -270,7 +333,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(tmem_slot)), "r"(256) : "memory");
+                 ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
@@ -302,8 +365,29 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_m128n128(p.is_f16);
-      int it = 0;
-      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      // prod: Z(t) = R(t) . S^T once the epilogue of tile t has written R(t) (three fp16
+      // products: R_hi S_hi + R_hi S_lo + R_lo S_hi), into tile t's accumulator
+      int zt = 0;                                   // next tile whose Z is issued
+      auto issue_z = [&]() {
+        const int zb = zt & 1;
+        if (!mbar_wait(rfull_bar(zb), (zt >> 1) & 1, lim, p.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t zidesc = idesc_m128n128(1);
+        const uint32_t zd = tmem_base + zb * 128, ra = tmem_base + kR + zb * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t boff = (kk >> 2) * (kPiBytes / 2) + (kk & 3) * 32;
+          umma_f16_ts(zd, ra + kk * 8, sw128_desc(s_hi + boff), zidesc, kk > 0 ? 1u : 0u);
+          umma_f16_ts(zd, ra + kk * 8, sw128_desc(s_lo + boff), zidesc, 1u);
+          umma_f16_ts(zd, ra + 64 + kk * 8, sw128_desc(s_hi + boff), zidesc, 1u);
+        }
+        umma_commit(zfull_bar(zb));
+        ++zt;
+        return true;
+      };
+      int it = 0;                                   // rotations issued
+      bool zok = true;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         const int s = it % NS, buf = it & 1, j = it >> 1;
         if (j > 0 && !mbar_wait(tempty_bar(buf), (j - 1) & 1, lim, p.status, abort_flag)) break;
         if (!mbar_wait(full_bar(s), (it / NS) & 1, lim, p.status, abort_flag)) break;
@@ -320,12 +404,18 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         }
         umma_commit(empty_bar(s));
         umma_commit(tfull_bar(buf));
+        ++it;
+        // the previous tile's projection, issued behind this tile's rotation
+        if (PRODK && it > 1 && !(zok = issue_z())) break;
       }
+      if (PRODK && zok && zt < it) zok = issue_z();      // the last tile
       // wait for the tensor core to finish everything issued before TMEM is freed
       if (it > 0) {
         const int last = it - 1;
         for (long long i = 0; !mbar_try(tfull_bar(last & 1), (last >> 1) & 1) && i < kDrainLimit; ++i) {}
       }
+      if (PRODK && zt > 0)
+        for (long long i = 0; !mbar_try(zfull_bar((zt - 1) & 1), ((zt - 1) >> 1) & 1) && i < kDrainLimit; ++i) {}
     }
   } else {
     const int grp = (warp - 2) >> 2;                   // 0: warps 2-5, 1: warps 6-9
@@ -365,6 +455,104 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 128;
       const int64_t v = tile * kUmmaTileRows + r;
+      if constexpr (PRODK) {
+        float y[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, y[c]);
+        tmem_wait_ld();
+        // (the accumulator stays with this group: Z lands in it next)
+        float2 s2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 v2 = make_float2(y[c][i], y[c][i + 1]);
+            s2[(i >> 1) & 3] = __ffma2_rn(v2, v2, s2[(i >> 1) & 3]);
+          }
+        }
+        const float ny = sqrtf(((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) + ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y)));
+        const float inv = ny > 0.f ? 1.f / ny : 1.f;
+        const float fs = inv * cell_scale;
+        const float ccen = lane < K ? pcen[lane] : 0.f;   // centroid of code `lane`
+        // this group's R columns were last read by its previous tile's projection, which
+        // completed before that tile's Z was read
+        const uint32_t rowaddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16);
+        const uint32_t rcol = rowaddr + kR + buf * 128;
+        float2 g2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t wc[B], hw[16], lw[16];
+#pragma unroll
+          for (int w = 0; w < B; ++w) wc[w] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            uint32_t code[2];
+            if (use_cells) {
+              const float2 f2 = make_float2(__saturatef(fmaf(y[c][i], fs, 0.5f)), __saturatef(fmaf(y[c][i + 1], fs, 0.5f)));
+              const float2 gg = __ffma2_rz(f2, make_float2(kCellSpan, kCellSpan), make_float2(8388608.0f, 8388608.0f));
+              const uint32_t e0 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gg.x));
+              const uint32_t e1 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gg.y));
+              const float2 d2 = __ffma2_rn(f2, make_float2(-1.f, -1.f), make_float2(__uint_as_float(e0), __uint_as_float(e1)));
+              code[0] = (e0 & 15u) + (__float_as_uint(d2.x) >> 31);
+              code[1] = (e1 & 15u) + (__float_as_uint(d2.y) >> 31);
+            } else {
+              uint32_t c0 = 0u, c1 = 0u;
+#pragma unroll
+              for (int k = 0; k < NB; ++k) {
+                c0 += y[c][i] * inv > tsm[k] ? 1u : 0u;
+                c1 += y[c][i + 1] * inv > tsm[k] ? 1u : 0u;
+              }
+              code[0] = c0; code[1] = c1;
+            }
+            // unit-scale residual r = u - c[code] and its fp16 hi + lo parts (the A operand)
+            const float ch0 = __shfl_sync(0xffffffffu, ccen, static_cast<int>(code[0]));
+            const float ch1 = __shfl_sync(0xffffffffu, ccen, static_cast<int>(code[1]));
+            const float2 rr = __ffma2_rn(make_float2(y[c][i], y[c][i + 1]), make_float2(inv, inv), make_float2(-ch0, -ch1));
+            g2 = __ffma2_rn(rr, rr, g2);
+            // hi = half2(r), lo = half2(r - hi): one paired conversion each, one packed FMA
+            const __half2 h2 = __floats2half2_rn(rr.x, rr.y);
+            const float2 back = __half22float2(h2);
+            const float2 res = __ffma2_rn(back, make_float2(-1.f, -1.f), rr);
+            const __half2 l2 = __floats2half2_rn(res.x, res.y);
+            hw[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+            lw[i >> 1] = *reinterpret_cast<const uint32_t*>(&l2);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int pos = (i + h) * B;
+              wc[pos >> 5] += code[h] << (pos & 31);
+              if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] += code[h] >> (32 - (pos & 31));
+            }
+          }
+          tmem_st16(rcol + 16 * c, hw);
+          tmem_st16(rcol + 64 + 16 * c, lw);
+          if (v < p.n) store_words<B>(p.codes + v * W + c * B, wc);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(rfull_bar(buf));
+        if (v < p.n) {
+          p.norms[v] = ny;
+          p.rnorms[v] = sqrtf(g2.x + g2.y);
+        }
+        // sign bits of the projection, (S r)_i >= 0
+        if (!mbar_wait(zfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
+        tc_fence_after();
+        uint32_t sw[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float z[32];
+          tmem_ld32(taddr + 32 * c, z);
+          tmem_wait_ld();
+          uint32_t wbits = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) wbits |= (z[i] >= 0.f ? 1u : 0u) << i;
+          sw[c] = wbits;
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(buf));                   // the accumulator is free again
+        if (v < p.n) *reinterpret_cast<uint4*>(p.signs + v * 4) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+        continue;
+      }
       if constexpr (SPEC) {
         const int kt = p.k_top;
         uint32_t tail[4];
@@ -525,7 +713,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(256) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
   }
 }
 

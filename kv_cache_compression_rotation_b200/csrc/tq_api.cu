@@ -192,9 +192,16 @@ bool umma_spectral(const tq_quantizer* q) {
   return hb <= 32 && (!q->qjl || q->S);
 }
 
+// prod records the tensor-core kernel writes: m = d = 128, 1..4 MSE bits plus the QJL signs
+bool umma_prod(const tq_quantizer* q) {
+  return q->kind == TQ_KIND_PROD && q->m == 128 && q->bits >= 2 && q->bits <= 5 && q->S && q->centroids &&
+         q->boundaries;
+}
+
 bool umma_supported(const tq_quantizer* q, int dtype, int64_t n) {
   if (q->d != 128) return false;
-  if (q->kind == TQ_KIND_MSE ? q->bits > 4 : !umma_spectral(q)) return false;
+  if (q->kind == TQ_KIND_MSE ? q->bits > 4 : (q->kind == TQ_KIND_PROD ? !umma_prod(q) : !umma_spectral(q)))
+    return false;
   if (dtype != TQ_BF16 && dtype != TQ_F16) return false;
   if (n < 1 || n >= (1ll << 31) - 256) return false;
   if (std::getenv("TQ_FORCE_SIMT")) return false;
@@ -206,9 +213,17 @@ bool umma_supported(const tq_quantizer* q, int dtype, int64_t n) {
 
 // ld / cols: element j of row v is x[v * ld + (cols ? cols[j] : j)] (cols: device; the
 // split's channel gather); a gather always takes the CUDA-core kernel.
+// Paged output of an append: vector v = b * Hkv + h goes to the record of token
+// seq[b] - 1 of (b, h) in the pool (see tq_pages).
+struct PagedOut {
+  const tq_pages* pages;
+  const int32_t* seq;
+  int Hkv;
+};
+
 tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64_t n, tq_packed out,
                           cudaStream_t stream, int want_kind, int64_t ld, const int32_t* cols,
-                          const Range* extra_outs = nullptr, int n_extra = 0) {
+                          const Range* extra_outs = nullptr, int n_extra = 0, const PagedOut* pgo = nullptr) {
   tq_status s = check_quantizer(q);
   if (s != TQ_OK) return s;
   if (q->kind != want_kind) return fail(TQ_ERR_INVALID_ARG, "quantizer kind does not match this entry point");
@@ -221,7 +236,7 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   const tq_layout L = layout_of(q);
   if ((s = check_packed(out, L)) != TQ_OK) return s;
   Range outs[4];
-  packed_ranges(out, L, n, outs);
+  packed_ranges(out, L, pgo ? pgo->pages->num_pages * pgo->Hkv * pgo->pages->page_size : n, outs);
   // inputs: x, and the other groups' outputs of a split call (disjoint from this group's)
   Range ins[1 + 4 * TQ_MAX_GROUPS];
   ins[0] = {x, static_cast<size_t>(n) * static_cast<size_t>(ld) * dtype_size(dtype)};
@@ -229,7 +244,7 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   if ((s = check_no_alias(outs, 4, ins, 1 + n_extra)) != TQ_OK) return s;
   int* status = device_status_ptr();
 
-  if (!cols && umma_supported(q, dtype, n)) {
+  if (!cols && !pgo && umma_supported(q, dtype, n)) {
     auto encode = get_encode();
     CUtensorMap map;
     const cuuint64_t gdim[2] = {128, static_cast<cuuint64_t>(n)};
@@ -258,9 +273,14 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
       p.dim_sigma = q->dim_sigma; p.unit_c = q->unit_centroids; p.unit_t = q->unit_boundaries;
       p.S = q->S; p.rnorms = q->qjl ? out.rnorms : nullptr;
     }
+    if (q->kind == TQ_KIND_PROD) {
+      p.S = q->S; p.centroids = q->centroids; p.signs = out.signs; p.rnorms = out.rnorms;
+    }
     const int64_t tiles = (n + 127) / 128;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
-    const cudaError_t e = launch_umma_quantize(map, p, q->kind == TQ_KIND_SPECTRAL ? 0 : q->bits, grid, stream);
+    const cudaError_t e = q->kind == TQ_KIND_PROD
+                              ? launch_umma_quantize_prod(map, p, q->bits - 1, grid, stream)
+                              : launch_umma_quantize(map, p, q->kind == TQ_KIND_SPECTRAL ? 0 : q->bits, grid, stream);
     return e == cudaSuccess ? TQ_OK : cuda_fail(e, "umma quantize launch");
   }
 
@@ -280,6 +300,10 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
   p.ld = ld;
   p.cols = cols;
   p.status = status;
+  if (pgo) {
+    p.pg_table = pgo->pages->block_table; p.pg_seq = pgo->seq; p.pg_size = pgo->pages->page_size;
+    p.pg_max = pgo->pages->max_pages; p.pg_hkv = pgo->Hkv; p.pg_num = pgo->pages->num_pages;
+  }
   const int d = q->d;
   // vectors per CTA: a multiple of 8 (the tiled product's row groups), at most 32, within
   // 200 KB of shared memory
@@ -315,7 +339,7 @@ bool spectral_tma(const tq_quantizer* q) {
          spectral_head_bits(q) <= 32;
 }
 
-DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t Nmax) {
+DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t Nmax, bool causal = false) {
   DecodePlan P{};
   const int D = kq->d;
   const int64_t units = static_cast<int64_t>(B) * Hkv;
@@ -326,7 +350,7 @@ DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t N
     // item count that is a multiple of the SMs; a work item covers one GQA group of up to
     // 4 heads (packed columns) or one block of up to 8 heads
     const int kf = kq->kind == TQ_KIND_PROD ? KFMT_PROD : (kq->kind == TQ_KIND_SPECTRAL ? KFMT_SPEC : KFMT_MSE);
-    const int64_t stage = tma_stage_tokens(kf, Hq / Hkv <= 4);
+    const int64_t stage = tma_stage_tokens(kf, Hq / Hkv <= 4 && !causal);
     const int64_t wu = units * tma_head_blocks(Hq / Hkv);
     // at most ~16 items per SM, and items of at least ~4 stages when the context is short
     // (each item ends in a cross-warp merge and writes one partial per head)
@@ -360,7 +384,8 @@ DecodePlan plan_decode(const tq_quantizer* kq, int B, int Hq, int Hkv, int64_t N
   return P;
 }
 
-tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int B, int Hq, int Hkv, int64_t Nmax) {
+tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int B, int Hq, int Hkv, int64_t Nmax,
+                             int max_group = 16) {
   tq_status s = check_quantizer(kq);
   if (s != TQ_OK) return s;
   if ((s = check_quantizer(vq)) != TQ_OK) return s;
@@ -370,8 +395,9 @@ tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int
   if (Nmax > (1ll << 30)) return fail(TQ_ERR_INVALID_ARG, "Nmax too large");
   if (static_cast<int64_t>(B) * Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "B*Hkv > 65535");
   if (kq->d != 128) return fail(TQ_ERR_UNSUPPORTED, "decode attention runs d = 128 only");
-  if (Hq / Hkv > 16) return fail(TQ_ERR_UNSUPPORTED, "Hq/Hkv > 16");
-  if (vq->kind == TQ_KIND_PROD) return fail(TQ_ERR_UNSUPPORTED, "values as PROD are not built");
+  if (Hq / Hkv > max_group) return fail(TQ_ERR_UNSUPPORTED, "Hq/Hkv > %d", max_group);
+  if (vq->kind == TQ_KIND_PROD && (vq->m != 128 || vq->bits < 2 || vq->bits > 5 || !vq->S))
+    return fail(TQ_ERR_UNSUPPORTED, "PROD values need m = d and 2..5 bits");
   if (vq->kind == TQ_KIND_SPECTRAL && vq->qjl) return fail(TQ_ERR_UNSUPPORTED, "spectral values with qjl");
   if ((kq->kind == TQ_KIND_SPECTRAL) != (vq->kind == TQ_KIND_SPECTRAL))
     return fail(TQ_ERR_UNSUPPORTED, "spectral keys need spectral values (and the reverse)");
@@ -382,6 +408,210 @@ tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int
   if (kq->kind == TQ_KIND_SPECTRAL && (kq->tail_bits > 2 || kq->tail_bits != vq->tail_bits))
     return fail(TQ_ERR_UNSUPPORTED, "spectral tail bits must be equal and <= 2");
   return TQ_OK;
+}
+
+// One attention step over the packed cache, shared by the decode entry points and the
+// causal prefill (whose query rows are the (head, position) pairs of a block: Hq counts
+// rows per sequence, T the positions per head).
+struct DecodeCall {
+  const tq_quantizer* kq;
+  const tq_quantizer* vq;
+  const void* q;
+  int dtype, B, Hq, Hkv;
+  int64_t Nmax;
+  const int32_t* seq_lens;
+  tq_packed kc, vc;
+  float scale;
+  float* out;
+  void* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+  const tq_pages* pages;     // paged pool, or nullptr
+  const void* k_new;         // paged append (decode), or nullptr
+  const void* v_new;
+  const int32_t* q_pos;      // causal rows (prefill), or nullptr
+  int T;
+};
+
+tq_status check_pages(const tq_pages* pg) {
+  if (!pg || !pg->block_table) return fail(TQ_ERR_INVALID_ARG, "pages or block_table is NULL");
+  if (!aligned16(pg->block_table)) return fail(TQ_ERR_ALIGNMENT, "block_table not 16-byte aligned");
+  if (pg->page_size < 16 || pg->page_size % 16) return fail(TQ_ERR_INVALID_ARG, "page_size must be a multiple of 16");
+  if (pg->max_pages < 1 || pg->num_pages < 1) return fail(TQ_ERR_INVALID_ARG, "max_pages and num_pages must be >= 1");
+  if (static_cast<int64_t>(pg->max_pages) * pg->page_size > (1ll << 30))
+    return fail(TQ_ERR_INVALID_ARG, "max_pages * page_size too large");
+  if (pg->num_pages > (1ll << 31) - 1) return fail(TQ_ERR_INVALID_ARG, "num_pages too large");
+  return TQ_OK;
+}
+
+tq_status decode_run(const DecodeCall& c) {
+  const tq_quantizer* kq = c.kq;
+  const tq_quantizer* vq = c.vq;
+  const void* q = c.q;
+  const int dtype = c.dtype, B = c.B, Hq = c.Hq, Hkv = c.Hkv;
+  const int64_t Nmax = c.Nmax;
+  const int32_t* seq_lens = c.seq_lens;
+  const tq_packed kc = c.kc, vc = c.vc;
+  const float scale = c.scale;
+  float* out = c.out;
+  void* workspace = c.ws;
+  const size_t ws_bytes = c.ws_bytes;
+  cudaStream_t stream = c.stream;
+  const bool causal = c.q_pos != nullptr;
+  tq_status s = check_decode_shape(kq, vq, B, Hq, Hkv, Nmax, causal ? (1 << 30) : 16);
+  if (s != TQ_OK) return s;
+  if ((c.pages || causal) && (kq->kind == TQ_KIND_SPECTRAL || vq->kind == TQ_KIND_SPECTRAL))
+    return fail(TQ_ERR_UNSUPPORTED, "paged and causal attention take MSE or PROD keys and MSE or PROD values");
+  if (causal && vq->kind == TQ_KIND_PROD) return fail(TQ_ERR_UNSUPPORTED, "causal attention takes MSE values");
+  if (causal && c.q_pos && !aligned16(c.q_pos)) return fail(TQ_ERR_ALIGNMENT, "q_pos alignment");
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
+  if (!aligned16(q) || !aligned16(seq_lens) || !aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "q/seq_lens/out alignment");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
+  if (!(kq->lut_scale >= 0.f) || !(vq->lut_scale >= 0.f) || !std::isfinite(kq->lut_scale) || !std::isfinite(vq->lut_scale))
+    return fail(TQ_ERR_INVALID_ARG, "lut_scale must be finite and >= 0");
+  const tq_layout LK = layout_of(kq), LV = layout_of(vq);
+  if ((s = check_packed(kc, LK)) != TQ_OK) return s;
+  if ((s = check_packed(vc, LV)) != TQ_OK) return s;
+  const DecodePlan P = plan_decode(kq, B, Hq, Hkv, Nmax, causal);
+  if (!workspace || ws_bytes < P.bytes) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", P.bytes);
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  const int64_t recs = c.pages ? c.pages->num_pages * Hkv * c.pages->page_size : static_cast<int64_t>(B) * Hkv * Nmax;
+  Range ins[14];
+  packed_ranges(kc, LK, recs, ins);
+  packed_ranges(vc, LV, recs, ins + 4);
+  ins[8] = {q, static_cast<size_t>(B) * Hq * kq->d * dtype_size(dtype)};
+  ins[9] = {seq_lens, static_cast<size_t>(B) * 4};
+  ins[10] = {workspace, ws_bytes};
+  int n_ins = 11;
+  if (c.pages) ins[n_ins++] = {c.pages->block_table, static_cast<size_t>(B) * c.pages->max_pages * 4};
+  if (causal) ins[n_ins++] = {c.q_pos, static_cast<size_t>(B) * c.T * 4};
+  const Range outs[1] = {{out, static_cast<size_t>(B) * Hq * kq->d * 4}};
+  if ((s = check_no_alias(outs, 1, ins, n_ins)) != TQ_OK) return s;
+
+  if (c.k_new) {
+    // the step's own token: quantized into its slot of the pool before the attention reads it
+    const PagedOut po{c.pages, seq_lens, Hkv};
+    const Range news[2] = {{c.k_new, static_cast<size_t>(B) * Hkv * kq->d * dtype_size(dtype)},
+                           {c.v_new, static_cast<size_t>(B) * Hkv * kq->d * dtype_size(dtype)}};
+    if ((s = check_no_alias(outs, 1, news, 2)) != TQ_OK) return s;
+    Range vouts[4];
+    packed_ranges(vc, LV, recs, vouts);
+    s = quantize_common(kq, c.k_new, dtype, static_cast<int64_t>(B) * Hkv, kc, stream, kq->kind, kq->d, nullptr,
+                        vouts, 4, &po);
+    if (s != TQ_OK) return s;
+    Range kouts[4];
+    packed_ranges(kc, LK, recs, kouts);
+    s = quantize_common(vq, c.v_new, dtype, static_cast<int64_t>(B) * Hkv, vc, stream, vq->kind, vq->d, nullptr,
+                        kouts, 4, &po);
+    if (s != TQ_OK) return s;
+  }
+
+  const int D = kq->d, G = Hq / Hkv, rows = B * Hq;
+  char* ws = static_cast<char*>(workspace);
+  float* qa = reinterpret_cast<float*>(ws + P.off_qa);
+  float* qb = reinterpret_cast<float*>(ws + P.off_qb);
+  float* qs = reinterpret_cast<float*>(ws + P.off_qs);
+  float* pml = reinterpret_cast<float*>(ws + P.off_ml);
+  float* po = reinterpret_cast<float*>(ws + P.off_o);
+
+  QPrepParams qp{};
+  qp.q = q; qp.dtype = dtype; qp.rows = rows; qp.D = D; qp.kind = kq->kind;
+  qp.scale = scale * kLog2e;
+  qp.rot = kq->rot; qp.S = kq->S; qp.m = kq->m;
+  qp.dim_sigma = kq->dim_sigma; qp.k_top = kq->k_top; qp.qjl = kq->qjl;
+  qp.spec_coef = static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, kq->k_top));
+  qp.qa = qa; qp.qb = qb; qp.qs = qs; qp.qb_stride = P.qb_stride;
+  const size_t qsm = static_cast<size_t>(2 * D + std::max(D, P.qb_stride)) * 4;
+  if (D == 128 && (kq->kind != TQ_KIND_SPECTRAL || kq->k_top <= 8))
+    qprep128_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(qp);
+  else
+    qprep_kernel<<<rows, 128, qsm, stream>>>(qp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "qprep launch");
+
+  DecodeParams dp{};
+  dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.G = G; dp.Nmax = Nmax;
+  dp.chunk_len = P.chunk_len; dp.n_chunks = P.n_chunks; dp.seq_lens = seq_lens;
+  dp.kcodes = kc.codes; dp.k_words = LK.code_words; dp.ksigns = kc.signs; dp.k_sign_words = LK.sign_words;
+  dp.knorms = kc.norms; dp.krnorms = kc.rnorms;
+  dp.vcodes = vc.codes; dp.v_words = LV.code_words; dp.vnorms = vc.norms;
+  dp.unit_c = kq->kind == TQ_KIND_SPECTRAL ? kq->unit_centroids : nullptr;
+  int kfmt, kb, vfmt, vb;
+  if (kq->kind == TQ_KIND_SPECTRAL) {
+    kfmt = KFMT_SPEC; kb = kq->tail_bits;
+    dp.k_code_off = (spectral_head_bits(kq) + 31) / 32;
+    dp.kc = kq->unit_centroids + unit_c_off(kb);
+    dp.k_top_k = kq->k_top; dp.k_qjl = kq->qjl;
+    for (int j = 0; j < TQ_MAX_TOP; ++j) dp.k_top_bits[j] = kq->top_bits[j];
+  } else {
+    kfmt = kq->kind == TQ_KIND_PROD ? KFMT_PROD : KFMT_MSE;
+    kb = kq->kind == TQ_KIND_PROD ? kq->bits - 1 : kq->bits;
+    dp.k_code_off = 0;
+    dp.kc = kq->centroids;
+  }
+  if (vq->kind == TQ_KIND_SPECTRAL) {
+    vfmt = VFMT_SPEC; vb = vq->tail_bits;
+    dp.v_code_off = (spectral_head_bits(vq) + 31) / 32;
+    dp.vc = vq->unit_centroids + unit_c_off(vb);
+    dp.v_top = vq->k_top;
+    for (int j = 0; j < TQ_MAX_TOP; ++j) dp.v_top_bits[j] = vq->top_bits[j];
+    if (!dp.unit_c) dp.unit_c = vq->unit_centroids;
+  } else if (vq->kind == TQ_KIND_PROD) {
+    vfmt = VFMT_PROD; vb = vq->bits - 1;
+    dp.v_code_off = 0;
+    dp.vc = vq->centroids;
+    dp.vsigns = vc.signs; dp.vrnorms = vc.rnorms; dp.vS = vq->S;
+    dp.v_coef = static_cast<float>(std::sqrt(M_PI / 2.0) / vq->m);
+  } else {
+    vfmt = VFMT_MSE; vb = vq->bits;
+    dp.v_code_off = 0;
+    dp.vc = vq->centroids;
+  }
+  dp.qa = qa; dp.qb = qb; dp.qs = qs; dp.qb_stride = P.qb_stride;
+  dp.qjl_coef = kq->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / kq->m) : 0.f;
+  dp.k_scale = kq->lut_scale > 0.f ? kq->lut_scale : 1.f;
+  dp.v_scale = vq->lut_scale > 0.f ? vq->lut_scale : 1.f;
+  dp.part_ml = pml; dp.part_o = po;
+  const int64_t items = static_cast<int64_t>(B) * Hkv * tma_head_blocks(G) * P.n_chunks;
+  const bool spec_tma = kfmt == KFMT_SPEC && spectral_tma(kq);   // the plan follows the keys
+  if (spec_tma && !spectral_tma(vq))
+    return fail(TQ_ERR_UNSUPPORTED, "spectral values need a head of at most 32 bits with 1-bit-tail keys");
+  const dim3 grid = (kfmt == KFMT_SPEC && !spec_tma)
+                        ? dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv))
+                        : dim3(static_cast<unsigned>(std::min<int64_t>(items, sm_count())));
+  const size_t smem = decode_smem_bytes(D, kb, vb);
+  if (c.pages) {
+    dp.block_table = c.pages->block_table; dp.page = c.pages->page_size; dp.max_pages = c.pages->max_pages;
+    dp.num_pages = c.pages->num_pages;
+  }
+  if (causal) { dp.q_pos = c.q_pos; dp.T = c.T; }
+  if (spec_tma)
+    e = launch_decode_spec_tma(dp, grid, stream, device_status_ptr(), wait_limit());
+  else if (causal)
+    e = launch_decode_causal(dp, kfmt, kb, vb, grid, stream, device_status_ptr(), wait_limit());
+  else
+    e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream, device_status_ptr(), wait_limit());
+  if (e == cudaErrorNotSupported) return fail(TQ_ERR_UNSUPPORTED, "decode variant not built (kbits %d, vbits %d)", kb, vb);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+
+  CombineParams cp{};
+  cp.rows = rows; cp.D = D; cp.n_chunks = P.n_chunks;
+  cp.part_ml = pml; cp.part_o = po; cp.rot_v = vq->rot;
+  cp.v_sigma = vq->kind == TQ_KIND_SPECTRAL ? vq->dim_sigma : nullptr;
+  cp.out = out;
+  // combine128: weights of 2 rows, then rot_V (64 KB); both combines wait on the decode
+  // kernel inside (programmatic launch: their launch overlaps its tail)
+  const size_t csm = static_cast<size_t>((2 * P.n_chunks + 3) & ~3) * 4 + 128 * 128 * 4;
+  if (D == 128 && csm <= 200 * 1024) {
+    e = cudaFuncSetAttribute(combine128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(csm));
+    if (e != cudaSuccess) return cuda_fail(e, "combine attribute");
+    e = launch_pdl(combine128_kernel, dim3(static_cast<unsigned>((rows + 1) / 2)), dim3(256), csm, stream, cp);
+  } else {
+    e = launch_pdl(combine_kernel, dim3(static_cast<unsigned>(rows)), dim3(128), static_cast<size_t>(D) * 4, stream, cp);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "combine launch");
 }
 
 }  // namespace
@@ -920,123 +1150,57 @@ tq_status tq_decode_attn(const tq_quantizer* kq, const tq_quantizer* vq, const v
                          int32_t Hq, int32_t Hkv, int64_t Nmax, const int32_t* seq_lens, tq_packed kc,
                          tq_packed vc, float scale, float* out, void* workspace, size_t ws_bytes,
                          tq_stream stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  tq_status s = check_decode_shape(kq, vq, B, Hq, Hkv, Nmax);
+  DecodeCall c{};
+  c.kq = kq; c.vq = vq; c.q = q; c.dtype = dtype; c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.Nmax = Nmax;
+  c.seq_lens = seq_lens; c.kc = kc; c.vc = vc; c.scale = scale; c.out = out; c.ws = workspace;
+  c.ws_bytes = ws_bytes; c.stream = reinterpret_cast<cudaStream_t>(stream_);
+  return decode_run(c);
+}
+
+tq_status tq_decode_attn_paged(const tq_quantizer* kq, const tq_quantizer* vq, const void* q, const void* k_new,
+                               const void* v_new, int32_t dtype, int32_t B, int32_t Hq, int32_t Hkv,
+                               const int32_t* seq_lens, const tq_pages* pages, tq_packed kpool, tq_packed vpool,
+                               float scale, float* out, void* workspace, size_t ws_bytes, tq_stream stream_) {
+  tq_status s = check_pages(pages);
   if (s != TQ_OK) return s;
-  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
-  if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
-  if (!aligned16(q) || !aligned16(seq_lens) || !aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "q/seq_lens/out alignment");
-  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
-  if (!(kq->lut_scale >= 0.f) || !(vq->lut_scale >= 0.f) || !std::isfinite(kq->lut_scale) || !std::isfinite(vq->lut_scale))
-    return fail(TQ_ERR_INVALID_ARG, "lut_scale must be finite and >= 0");
-  const tq_layout LK = layout_of(kq), LV = layout_of(vq);
-  if ((s = check_packed(kc, LK)) != TQ_OK) return s;
-  if ((s = check_packed(vc, LV)) != TQ_OK) return s;
-  const DecodePlan P = plan_decode(kq, B, Hq, Hkv, Nmax);
-  if (!workspace || ws_bytes < P.bytes) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", P.bytes);
-  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
-  const int64_t recs = static_cast<int64_t>(B) * Hkv * Nmax;
-  Range ins[11];
-  packed_ranges(kc, LK, recs, ins);
-  packed_ranges(vc, LV, recs, ins + 4);
-  ins[8] = {q, static_cast<size_t>(B) * Hq * kq->d * dtype_size(dtype)};
-  ins[9] = {seq_lens, static_cast<size_t>(B) * 4};
-  ins[10] = {workspace, ws_bytes};
-  const Range outs[1] = {{out, static_cast<size_t>(B) * Hq * kq->d * 4}};
-  if ((s = check_no_alias(outs, 1, ins, 11)) != TQ_OK) return s;
+  if ((k_new == nullptr) != (v_new == nullptr)) return fail(TQ_ERR_INVALID_ARG, "k_new and v_new go together");
+  if (!seq_lens || !aligned16(seq_lens)) return fail(TQ_ERR_ALIGNMENT, "seq_lens NULL or not 16-byte aligned");
+  DecodeCall c{};
+  c.kq = kq; c.vq = vq; c.q = q; c.dtype = dtype; c.B = B; c.Hq = Hq; c.Hkv = Hkv;
+  c.Nmax = static_cast<int64_t>(pages->max_pages) * pages->page_size;
+  c.seq_lens = seq_lens; c.kc = kpool; c.vc = vpool; c.scale = scale; c.out = out; c.ws = workspace;
+  c.ws_bytes = ws_bytes; c.stream = reinterpret_cast<cudaStream_t>(stream_); c.pages = pages;
+  c.k_new = k_new; c.v_new = v_new;
+  return decode_run(c);
+}
 
-  const int D = kq->d, G = Hq / Hkv, rows = B * Hq;
-  char* ws = static_cast<char*>(workspace);
-  float* qa = reinterpret_cast<float*>(ws + P.off_qa);
-  float* qb = reinterpret_cast<float*>(ws + P.off_qb);
-  float* qs = reinterpret_cast<float*>(ws + P.off_qs);
-  float* pml = reinterpret_cast<float*>(ws + P.off_ml);
-  float* po = reinterpret_cast<float*>(ws + P.off_o);
+tq_status tq_prefill_attn_workspace(const tq_quantizer* kq, int32_t B, int32_t Hq, int32_t Hkv, int32_t T,
+                                    int64_t Nmax, size_t* bytes) {
+  tq_status s = check_quantizer(kq);
+  if (s != TQ_OK) return s;
+  if (!bytes || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Nmax < 1 || static_cast<int64_t>(Hq) * T > (1 << 24))
+    return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
+  *bytes = plan_decode(kq, B, Hq * T, Hkv, Nmax, true).bytes;
+  return TQ_OK;
+}
 
-  QPrepParams qp{};
-  qp.q = q; qp.dtype = dtype; qp.rows = rows; qp.D = D; qp.kind = kq->kind;
-  qp.scale = scale * kLog2e;
-  qp.rot = kq->rot; qp.S = kq->S; qp.m = kq->m;
-  qp.dim_sigma = kq->dim_sigma; qp.k_top = kq->k_top; qp.qjl = kq->qjl;
-  qp.spec_coef = static_cast<float>(std::sqrt(M_PI / 2.0) / std::max(1, kq->k_top));
-  qp.qa = qa; qp.qb = qb; qp.qs = qs; qp.qb_stride = P.qb_stride;
-  const size_t qsm = static_cast<size_t>(2 * D + std::max(D, P.qb_stride)) * 4;
-  if (D == 128 && (kq->kind != TQ_KIND_SPECTRAL || kq->k_top <= 8))
-    qprep128_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(qp);
-  else
-    qprep_kernel<<<rows, 128, qsm, stream>>>(qp);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "qprep launch");
-
-  DecodeParams dp{};
-  dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.G = G; dp.Nmax = Nmax;
-  dp.chunk_len = P.chunk_len; dp.n_chunks = P.n_chunks; dp.seq_lens = seq_lens;
-  dp.kcodes = kc.codes; dp.k_words = LK.code_words; dp.ksigns = kc.signs; dp.k_sign_words = LK.sign_words;
-  dp.knorms = kc.norms; dp.krnorms = kc.rnorms;
-  dp.vcodes = vc.codes; dp.v_words = LV.code_words; dp.vnorms = vc.norms;
-  dp.unit_c = kq->kind == TQ_KIND_SPECTRAL ? kq->unit_centroids : nullptr;
-  int kfmt, kb, vfmt, vb;
-  if (kq->kind == TQ_KIND_SPECTRAL) {
-    kfmt = KFMT_SPEC; kb = kq->tail_bits;
-    dp.k_code_off = (spectral_head_bits(kq) + 31) / 32;
-    dp.kc = kq->unit_centroids + unit_c_off(kb);
-    dp.k_top_k = kq->k_top; dp.k_qjl = kq->qjl;
-    for (int j = 0; j < TQ_MAX_TOP; ++j) dp.k_top_bits[j] = kq->top_bits[j];
-  } else {
-    kfmt = kq->kind == TQ_KIND_PROD ? KFMT_PROD : KFMT_MSE;
-    kb = kq->kind == TQ_KIND_PROD ? kq->bits - 1 : kq->bits;
-    dp.k_code_off = 0;
-    dp.kc = kq->centroids;
+tq_status tq_prefill_attn(const tq_quantizer* kq, const tq_quantizer* vq, const void* q, int32_t dtype, int32_t B,
+                          int32_t Hq, int32_t Hkv, int32_t T, const int32_t* q_pos, const int32_t* kv_lens,
+                          const tq_pages* pages, int64_t Nmax, tq_packed kcache, tq_packed vcache, float scale,
+                          float* out, void* workspace, size_t ws_bytes, tq_stream stream_) {
+  if (T < 1 || Hq < 1 || static_cast<int64_t>(Hq) * T > (1 << 24)) return fail(TQ_ERR_INVALID_ARG, "T out of range");
+  if (!q_pos || !aligned16(q_pos)) return fail(TQ_ERR_ALIGNMENT, "q_pos NULL or not 16-byte aligned");
+  if (pages) {
+    tq_status s = check_pages(pages);
+    if (s != TQ_OK) return s;
+    Nmax = static_cast<int64_t>(pages->max_pages) * pages->page_size;
   }
-  if (vq->kind == TQ_KIND_SPECTRAL) {
-    vfmt = VFMT_SPEC; vb = vq->tail_bits;
-    dp.v_code_off = (spectral_head_bits(vq) + 31) / 32;
-    dp.vc = vq->unit_centroids + unit_c_off(vb);
-    dp.v_top = vq->k_top;
-    for (int j = 0; j < TQ_MAX_TOP; ++j) dp.v_top_bits[j] = vq->top_bits[j];
-    if (!dp.unit_c) dp.unit_c = vq->unit_centroids;
-  } else {
-    vfmt = VFMT_MSE; vb = vq->bits;
-    dp.v_code_off = 0;
-    dp.vc = vq->centroids;
-  }
-  dp.qa = qa; dp.qb = qb; dp.qs = qs; dp.qb_stride = P.qb_stride;
-  dp.qjl_coef = kq->kind == TQ_KIND_PROD ? static_cast<float>(std::sqrt(M_PI / 2.0) / kq->m) : 0.f;
-  dp.k_scale = kq->lut_scale > 0.f ? kq->lut_scale : 1.f;
-  dp.v_scale = vq->lut_scale > 0.f ? vq->lut_scale : 1.f;
-  dp.part_ml = pml; dp.part_o = po;
-  const int64_t items = static_cast<int64_t>(B) * Hkv * tma_head_blocks(G) * P.n_chunks;
-  const bool spec_tma = kfmt == KFMT_SPEC && spectral_tma(kq);   // the plan follows the keys
-  if (spec_tma && !spectral_tma(vq))
-    return fail(TQ_ERR_UNSUPPORTED, "spectral values need a head of at most 32 bits with 1-bit-tail keys");
-  const dim3 grid = (kfmt == KFMT_SPEC && !spec_tma)
-                        ? dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv))
-                        : dim3(static_cast<unsigned>(std::min<int64_t>(items, sm_count())));
-  const size_t smem = decode_smem_bytes(D, kb, vb);
-  if (spec_tma)
-    e = launch_decode_spec_tma(dp, grid, stream, device_status_ptr(), wait_limit());
-  else
-    e = launch_decode(dp, kfmt, kb, vfmt, vb, grid, smem, stream, device_status_ptr(), wait_limit());
-  if (e == cudaErrorNotSupported) return fail(TQ_ERR_UNSUPPORTED, "decode variant not built (kbits %d, vbits %d)", kb, vb);
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-
-  CombineParams cp{};
-  cp.rows = rows; cp.D = D; cp.n_chunks = P.n_chunks;
-  cp.part_ml = pml; cp.part_o = po; cp.rot_v = vq->rot;
-  cp.v_sigma = vq->kind == TQ_KIND_SPECTRAL ? vq->dim_sigma : nullptr;
-  cp.out = out;
-  // combine128: weights of 2 rows, then rot_V (64 KB); both combines wait on the decode
-  // kernel inside (programmatic launch: their launch overlaps its tail)
-  const size_t csm = static_cast<size_t>((2 * P.n_chunks + 3) & ~3) * 4 + 128 * 128 * 4;
-  if (D == 128 && csm <= 200 * 1024) {
-    e = cudaFuncSetAttribute(combine128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(csm));
-    if (e != cudaSuccess) return cuda_fail(e, "combine attribute");
-    e = launch_pdl(combine128_kernel, dim3(static_cast<unsigned>((rows + 1) / 2)), dim3(256), csm, stream, cp);
-  } else {
-    e = launch_pdl(combine_kernel, dim3(static_cast<unsigned>(rows)), dim3(128), static_cast<size_t>(D) * 4, stream, cp);
-  }
-  if (e == cudaSuccess) e = cudaGetLastError();
-  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "combine launch");
+  DecodeCall c{};
+  c.kq = kq; c.vq = vq; c.q = q; c.dtype = dtype; c.B = B; c.Hq = Hq * T; c.Hkv = Hkv; c.Nmax = Nmax;
+  c.seq_lens = kv_lens; c.kc = kcache; c.vc = vcache; c.scale = scale; c.out = out; c.ws = workspace;
+  c.ws_bytes = ws_bytes; c.stream = reinterpret_cast<cudaStream_t>(stream_); c.pages = pages;
+  c.q_pos = q_pos; c.T = T;
+  return decode_run(c);
 }
 
 tq_status tq_get_status(tq_stream stream) {
@@ -1067,6 +1231,7 @@ tq_status decode_shape_ok(const tq_quantizer* kq, const tq_quantizer* vq, int B,
 
 cudaError_t launch_decode(const DecodeParams& p, int kfmt, int kb, int vfmt, int vb, dim3 grid, size_t smem,
                           cudaStream_t stream, int* status, long long lim) {
+  if (vfmt == VFMT_PROD) return launch_decode_vprod(p, kfmt, kb, vb, grid, stream, status, lim);
   if (kfmt == KFMT_MSE && vfmt == VFMT_MSE) return launch_decode_mse(p, kb, vb, grid, smem, stream, status, lim);
   if (kfmt == KFMT_PROD && vfmt == VFMT_MSE) return launch_decode_prod(p, kb, vb, grid, smem, stream, status, lim);
   if (kfmt == KFMT_SPEC && vfmt == VFMT_SPEC) return launch_decode_spec(p, kb, vb, grid, smem, stream);

@@ -33,6 +33,7 @@ EXPORTS = [
     "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
     "tq_decode_attn_fixed_ws", "tq_quantize_split", "tq_score_split_workspace", "tq_score_split",
     "tq_decode_attn_split_workspace", "tq_decode_attn_split", "tq_spectral_descriptor", "tq_spectral_prepare",
+    "tq_decode_attn_paged", "tq_prefill_attn_workspace", "tq_prefill_attn",
 ]
 
 
@@ -63,6 +64,11 @@ MAX_GROUPS = 4
 class Split_t(C.Structure):
     _fields_ = [("n_groups", C.c_int32), ("d", C.c_int32),
                 ("groups", C.POINTER(Quantizer_t) * MAX_GROUPS), ("cols", C.c_void_p * MAX_GROUPS)]
+
+
+class Pages_t(C.Structure):
+    _fields_ = [("block_table", C.c_void_p), ("page_size", C.c_int32), ("max_pages", C.c_int32),
+                ("num_pages", C.c_int64)]
 
 
 class Layout_t(C.Structure):
@@ -109,6 +115,11 @@ def lib():
                                         C.POINTER(C.c_float)], C.c_int),
             "tq_spectral_prepare": ([vp, i64, i32, i32, i32, i32, i32, vp, vp, vp, vp, C.POINTER(i32),
                                      C.POINTER(C.c_float), f64p], C.c_int),
+            "tq_decode_attn_paged": ([qp, qp, vp, vp, vp, i32, i32, i32, i32, vp, C.POINTER(Pages_t), Packed_t,
+                                      Packed_t, C.c_float, vp, vp, C.c_size_t, vp], C.c_int),
+            "tq_prefill_attn_workspace": ([qp, i32, i32, i32, i32, i64, C.POINTER(C.c_size_t)], C.c_int),
+            "tq_prefill_attn": ([qp, qp, vp, i32, i32, i32, i32, i32, vp, vp, C.POINTER(Pages_t), i64, Packed_t,
+                                 Packed_t, C.c_float, vp, vp, C.c_size_t, vp], C.c_int),
             "tq_quantize_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), vp], C.c_int),
             "tq_score_split_workspace": ([C.POINTER(Split_t), i64, i64, i32, C.POINTER(C.c_size_t)], C.c_int),
             "tq_score_split": ([C.POINTER(Split_t), vp, i32, i64, C.POINTER(Packed_t), i64, i32, vp, vp, vp,
@@ -452,6 +463,64 @@ def decode_attn(kq: Quantizer, vq: Quantizer, q, seq_lens, kcache: Packed, vcach
     _check(lib().tq_decode_attn(kq.ref, vq.ref, q.data_ptr(), _dtype_code(q), B, Hq, Hkv, Nmax,
                                 seq_lens.data_ptr(), kcache.as_c(), vcache.as_c(), float(scale), out.data_ptr(),
                                 workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out
+
+
+class Pages:
+    """Paged record pool: block_table int32 [B, max_pages] CUDA tensor of page ids, page_size
+    tokens per page (a multiple of 16), num_pages pages; token t of (b, kv-head h) is record
+    (block_table[b, t // page_size] * Hkv + h) * page_size + t % page_size of every array."""
+
+    def __init__(self, block_table, page_size: int, num_pages: int):
+        assert block_table.dtype.is_floating_point is False and block_table.is_contiguous()
+        self.block_table, self.page_size, self.num_pages = block_table, page_size, num_pages
+        self.max_pages = block_table.shape[1]
+        self.c = Pages_t(block_table.data_ptr(), page_size, self.max_pages, num_pages)
+
+    @property
+    def ref(self):
+        return C.byref(self.c)
+
+    def records(self, Hkv: int) -> int:
+        return self.num_pages * Hkv * self.page_size
+
+
+def decode_attn_paged(kq: Quantizer, vq: Quantizer, q, seq_lens, pages: Pages, kpool: Packed, vpool: Packed,
+                      Hkv: int, k_new=None, v_new=None, scale: Optional[float] = None, out=None, workspace=None,
+                      stream=None):
+    """tq_decode_attn_paged: append k_new / v_new [B*Hkv, d] (optional) as token seq_lens[b]-1,
+    then one decode step over the pool; q [B, Hq, d]."""
+    import torch
+    B, Hq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = decode_workspace_bytes(kq, B, Hq, Hkv, pages.max_pages * pages.page_size)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device) if out is None else out
+    _check(lib().tq_decode_attn_paged(kq.ref, vq.ref, q.data_ptr(), _dptr(k_new), _dptr(v_new), _dtype_code(q), B, Hq,
+                                      Hkv, seq_lens.data_ptr(), pages.ref, kpool.as_c(), vpool.as_c(), float(scale),
+                                      out.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out
+
+
+def prefill_attn(kq: Quantizer, vq: Quantizer, q, q_pos, kv_lens, kcache: Packed, vcache: Packed, Hkv: int,
+                 Nmax: int = 0, pages: Optional[Pages] = None, scale: Optional[float] = None, out=None,
+                 workspace=None, stream=None):
+    """tq_prefill_attn: causal attention of q [B, Hq, T, d] at positions q_pos [B, T] over the
+    packed cache ([B, Hkv, Nmax] records, or a paged pool)."""
+    import torch
+    B, Hq, T, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    n = pages.max_pages * pages.page_size if pages is not None else Nmax
+    ws = C.c_size_t(0)
+    _check(lib().tq_prefill_attn_workspace(kq.ref, B, Hq, Hkv, T, n, C.byref(ws)))
+    if workspace is None or workspace.numel() < ws.value:
+        workspace = torch.empty(max(ws.value, 16), dtype=torch.uint8, device=q.device)
+    out = torch.empty((B, Hq, T, d), dtype=torch.float32, device=q.device) if out is None else out
+    _check(lib().tq_prefill_attn(kq.ref, vq.ref, q.data_ptr(), _dtype_code(q), B, Hq, Hkv, T, q_pos.data_ptr(),
+                                 kv_lens.data_ptr(), pages.ref if pages is not None else None, Nmax, kcache.as_c(),
+                                 vcache.as_c(), float(scale), out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)))
     return out
 
 

@@ -237,3 +237,50 @@ def test_decode_hadamard_rotation():
     ref2 = _rescored_reference(q64, seq_lens, B, Hkv, Nmax, rot, None, "mse", 4, 4, kc, vc, okq, ovq, c, t, c, t)
     err2 = rel_rows(out2, ref2)
     assert np.all(err2 <= 1e-3), f"max row error {err2.max():.3e}"
+
+
+PROD_VALUE_CASES = [
+    # name, B, Hq, Hkv, Nmax, seq_lens, key kind, key bits, value bits (values as prod)
+    ("pv-mse4-prod3", 2, 8, 2, 1500, [1500, 733], "mse", 4, 3),
+    ("pv-prod3-prod3", 1, 32, 8, 1100, [1100], "prod", 3, 3),
+    ("pv-g8", 1, 8, 1, 900, [900], "mse", 3, 4),
+    ("pv-g1-bits2", 2, 4, 4, 700, [1, 699], "mse", 2, 2),
+    ("pv-prod5", 1, 8, 2, 600, [600], "prod", 4, 5),
+]
+
+
+@pytest.mark.parametrize("name,B,Hq,Hkv,Nmax,seq_lens,kk,bk,bv", PROD_VALUE_CASES, ids=[c[0] for c in PROD_VALUE_CASES])
+def test_decode_prod_values(name, B, Hq, Hkv, Nmax, seq_lens, kk, bk, bv):
+    """Values quantized as TurboQuant-prod: the step uses their unbiased reconstruction
+    ||v|| Pi^T (c[code] + sqrt(pi/2)/m ||r|| S^T (2s - 1)).  GPU quantize -> GPU decode, the
+    oracle rescoring with the GPU's band-checked key and value records, 1e-3 per row."""
+    seed = sum(ord(ch) for ch in name) % 89
+    rot = ti.haar_rotation(D, 1003)
+    S = ti.gaussian_matrix(D, D, 2003)
+    Sv = ti.gaussian_matrix(D, D, 2103)
+    kt, k64, vt, v64 = _cache_inputs(B, Hkv, Nmax, seed)
+    qt, q64 = _query(B, Hq, seed)
+    kq = K.Quantizer.prod(rot, S, bk) if kk == "prod" else K.Quantizer.mse(rot, bk)
+    vq = K.Quantizer.prod(rot, Sv, bv)
+    sl = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
+    kc, vc = K.quantize(kq, kt), K.quantize(vq, vt)
+    out = K.decode_attn(kq, vq, qt, sl, kc, vc, Nmax, Hkv).cpu().numpy()
+    assert K.get_status() == 0
+    ck, tk, _ = lloyd_max(bk - 1 if kk == "prod" else bk, "beta", d=D)
+    cv, tv, _ = lloyd_max(bv - 1, "beta", d=D)
+    okq = OQ.quantize_prod(k64, rot, S, ck, tk, bk) if kk == "prod" else OQ.quantize_mse(k64, rot, ck, tk, bk)
+    ovq = OQ.quantize_prod(v64, rot, Sv, cv, tv, bv)
+    _check_norms(kc, okq)
+    _check_norms(vc, ovq)
+    if kk == "prod":
+        a = adopt_prod(as_u32(kc.codes), as_u32(kc.signs), kc.rnorms.cpu().numpy(), okq, bk, ck, tk, S)
+        ks = lambda r, qs: OQ.estimate_prod(qs, rot, S, a["chat"][r], a["s"][r], okq["norms"][r], a["rnorms"][r])
+    else:
+        kidx, _ = adopt_mse(as_u32(kc.codes), okq, bk, tk)
+        ks = lambda r, qs: OQ.estimate_mse(qs, rot, kidx[r], okq["norms"][r], ck)
+    av = adopt_prod(as_u32(vc.codes), as_u32(vc.signs), vc.rnorms.cpu().numpy(), ovq, bv, cv, tv, Sv)
+    vh = OQ.dequantize_prod(av["chat"], av["s"], ovq["norms"], av["rnorms"], rot, Sv)
+    ref = decode_attention(q64, seq_lens, Hkv, lambda b, h, qs: ks(_rows(B, Hkv, Nmax, b, h, Nmax), qs),
+                           lambda b, h, n: vh[_rows(B, Hkv, Nmax, b, h, n)], 1.0 / math.sqrt(D))
+    err = rel_rows(out, ref)
+    assert np.all(err <= 1e-3), f"max row error {err.max():.3e}"

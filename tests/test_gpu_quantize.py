@@ -126,7 +126,11 @@ def test_quantize_pm1_flag_rejects_other_rotations():
 @pytest.mark.parametrize("d,bits,m,dtype,n", [(128, 3, 128, "bf16", 2000), (64, 2, 64, "f32", 500),
                                               (128, 1, 128, "f32", 300), (128, 5, 256, "bf16", 400),
                                               (64, 6, 64, "f32", 200), (64, 7, 64, "bf16", 200),
-                                              (64, 8, 96, "f32", 150), (64, 9, 64, "bf16", 150)])
+                                              (64, 8, 96, "f32", 150), (64, 9, 64, "bf16", 150),
+                                              # d = m = 128 with 16-bit input: the tensor-core kernel
+                                              # (rotation and QJL projection on tcgen05), ragged tiles
+                                              (128, 2, 128, "bf16", 128 * 148 + 5), (128, 4, 128, "f16", 3001),
+                                              (128, 5, 128, "bf16", 1000), (128, 3, 128, "f16", 1)])
 def test_quantize_prod_parity(d, bits, m, dtype, n):
     rot = ti.haar_rotation(d, 1100 + d)
     S = ti.gaussian_matrix(m, d, 2000 + d)
