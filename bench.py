@@ -533,13 +533,15 @@ def run_other(args):
         qs /= qs.norm(dim=1, keepdim=True)
         kq = K.Quantizer.prod(rot, S, args.c5_bits, device=dev)
         kc = kq.alloc(ndb, dev)
-        tq = _timed(lambda: K.quantize(kq, db, kc), stream, flush, reps=3, warm=1)
+        wsq = torch.empty(max(16, K.tq_quantize_workspace_bytes(kq, db)), dtype=torch.uint8, device=dev)
+        tq = _timed(lambda: K.quantize_ws(kq, db, kc, workspace=wsq), stream, flush, reps=3, warm=1)
         ts = _timed(lambda: K.score(kq, qs, kc, ndb, topk=10), stream, None, reps=3, warm=1)
         L = kq.layout()
         rec = 4 * (L.code_words + L.sign_words + L.has_norms + L.has_rnorms)
         parts = {"quantize": {"ms": tq, "vectors_per_s": ndb / tq * 1e3, "gbs": ndb * (d5 * 4 + rec) / tq / 1e6},
                  "search_top10": {"ms": ts, "queries_per_s": nq5 / ts * 1e3,
                                   "note": f"{nq5} queries x {ndb} records, CUDA-core estimator"}}
+        parts["quantize"]["note"] = "tq_quantize_ws: rotation and QJL projection as split-precision tcgen05 products"
         desc = (f"search: {ndb} x 1536 fp32 unit vectors, prod b={args.c5_bits} (m=1536), "
                 f"top-10 of {nq5} queries")
         value, unit, step_ms = ndb / tq * 1e3, "vectors/s", tq
@@ -579,6 +581,53 @@ def run_other(args):
                 f"96 @ 2 bits (mse), dense estimates for {nq} queries, decode B=1 Hkv=8 Hq=32 over 32768 "
                 f"tokens (CUDA-core kernels)")
         value, unit, step_ms = n / tq * 1e3, "vectors/s", tq
+    elif wl == "serving":
+        # serving forms at the 128k decode shapes: one decode step over a paged pool with the
+        # step's token appended in the same call (pages of 256 tokens, shuffled block table),
+        # and causal prefill of a 1024-token block at the end of a 32k context
+        Bw, Hkv, Hq, Nw, P = 8, 8, 32, 131072, 256
+        rot = ti.haar_rotation(Dm, ti.SEEDS["rotation"] + 3)
+        U = ti.haar_rotation(Dm, ti.SEEDS["basis"] + 3)
+        kq, vq = K.Quantizer.mse(rot, 4, device=dev), K.Quantizer.mse(rot, 4, device=dev)
+        max_pages = Nw // P
+        num_pages = Bw * max_pages
+        table = np.random.Generator(np.random.PCG64(ti.SEEDS["basis"] + 9)).permutation(num_pages)
+        pages = K.Pages(torch.from_numpy(table.reshape(Bw, max_pages).astype(np.int32)).to(dev), P, num_pages)
+        n = pages.records(Hkv)
+        kx = ti.anisotropic_torch(n, Dm, U, ti.SEEDS["keys"] + 3, dev)
+        vx = ti.anisotropic_torch(n, Dm, U, ti.SEEDS["values"] + 3, dev)
+        kpool, vpool = K.quantize(kq, kx), K.quantize(vq, vx)       # every slot holds a record
+        del kx, vx
+        knew = ti.normal_torch((Bw * Hkv, Dm), ti.SEEDS["keys"] + 13, dev, dtype=torch.bfloat16)
+        vnew = ti.normal_torch((Bw * Hkv, Dm), ti.SEEDS["values"] + 13, dev, dtype=torch.bfloat16)
+        q = ti.normal_torch((Bw, Hq, Dm), ti.SEEDS["queries"] + 3, dev, dtype=torch.bfloat16)
+        seq = torch.full((Bw,), Nw, dtype=torch.int32, device=dev)
+        ws = torch.empty(K.decode_workspace_bytes(kq, Bw, Hq, Hkv, Nw), dtype=torch.uint8, device=dev)
+        out = torch.empty((Bw, Hq, Dm), dtype=torch.float32, device=dev)
+        td = _timed(lambda: K.decode_attn_paged(kq, vq, q, seq, pages, kpool, vpool, Hkv, k_new=knew, v_new=vnew,
+                                                out=out, workspace=ws), stream, flush)
+        # prefill: B=1, 32k cached tokens, the last T=1024 positions
+        Np, T = 32768, 1024
+        kc1 = K.Packed(kpool.codes[:Hkv * Np], None, kpool.norms[:Hkv * Np], None)
+        vc1 = K.Packed(vpool.codes[:Hkv * Np], None, vpool.norms[:Hkv * Np], None)
+        qp = ti.normal_torch((1, Hq, T, Dm), ti.SEEDS["queries"] + 14, dev, dtype=torch.bfloat16)
+        pos = torch.arange(Np - T, Np, dtype=torch.int32, device=dev).reshape(1, T)
+        kvl = torch.tensor([Np], dtype=torch.int32, device=dev)
+        outp = torch.empty((1, Hq, T, Dm), dtype=torch.float32, device=dev)
+        tp = _timed(lambda: K.prefill_attn(kq, vq, qp, pos, kvl, kc1, vc1, Hkv, Nmax=Np, out=outp), stream, flush,
+                    reps=5, warm=2)
+        assert K.get_status() == 0
+        dec_b = Bw * Hkv * Nw * 136
+        # causal work: query i sees (Np - T + i + 1) tokens, for every head
+        visible = sum(Np - T + i + 1 for i in range(T)) * Hq
+        parts = {"decode_attn_paged": {"ms": td, "gbs": dec_b / td / 1e6, "frac": dec_b / td / 1e6 / peak,
+                                       "note": "includes the append of 64 new key and value vectors"},
+                 "prefill_attn": {"ms": tp, "queries_per_s": Hq * T / tp * 1e3,
+                                  "score_pairs_per_s": visible / tp * 1e3,
+                                  "note": f"B=1, Hq=32, Hkv=8, {T} queries at positions {Np - T}..{Np - 1}"}}
+        desc = (f"serving: paged decode B=8, Hkv=8, Hq=32, context 131072, pages of {P} tokens, append in the "
+                f"call; causal prefill of {T} queries over a 32768-token packed cache")
+        value, unit, step_ms = dec_b / td / 1e6, "GB/s", td
     elif wl == "sweep":
         n, rho = 4096, 0.9
         rows = ip_sweep(K, dev, n, rho)
@@ -613,7 +662,7 @@ def main():
                     help="profiling aid: context length (the headline workload uses 131072)")
     ap.add_argument("--batch", type=int, default=B,
                     help="profiling aid: batch size (the headline workload uses 8)")
-    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5", "split", "sweep"],
+    ap.add_argument("--workload", default="c3", choices=["c3", "c1", "c2", "c4", "c5", "split", "sweep", "serving"],
                     help="c3 (default): the 128k decode step of the headline; the others are the scope "
                          "table's secondary workloads, timed per kernel")
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],

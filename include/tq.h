@@ -243,6 +243,25 @@ tq_status tq_quantize_spectral(const tq_quantizer* q, const void* x, int32_t dty
                                tq_packed out, tq_stream stream);
 
 /*
+ * Workspace bytes that tq_quantize_ws needs for n vectors of this quantizer and dtype; 0
+ * when the call takes the same kernels as tq_quantize_mse / _prod / _spectral.
+ */
+tq_status tq_quantize_workspace(const tq_quantizer* q, int32_t dtype, int64_t n, size_t* bytes);
+
+/*
+ * DEVICE.  Quantize with caller-provided device scratch: the records are exactly those of
+ * tq_quantize_mse / tq_quantize_prod / tq_quantize_spectral (by q->kind).  For fp32 input
+ * with d a multiple of 256 (up to 4096; the review's d = 1536 vector-search embeddings),
+ * MSE with 1..4 bits or PROD with 2..5 bits and m = d, the rotation and the QJL projection
+ * run on the tensor cores as split-precision products (x, Pi, S and the residual split
+ * into bf16 hi + lo parts in the workspace, three products per pair, fp32 accumulation),
+ * in passes of up to 32768 vectors; the workspace holds the split operands of one pass.
+ * Other shapes ignore the workspace.  workspace: device, >= tq_quantize_workspace bytes.
+ */
+tq_status tq_quantize_ws(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
+                         void* workspace, size_t ws_bytes, tq_stream stream);
+
+/*
  * Outlier-channel split (TurboQuant review, Method: for the KV-cache experiments the
  * channels are split into an outlier group and the rest, each quantized by its own
  * TurboQuant instance; the setting it calls 2.5-bit is 32 outlier channels at 3 bits plus

@@ -26,6 +26,7 @@ inline cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t
 
 struct DecodeParams;
 struct UmmaQuantParams;
+struct SplitGemmParams;
 
 // Launch decode_attn_kernel for (key format, key bits, value format, value bits) at D = 128.
 // Returns cudaErrorNotSupported (without launching) for a combination that is not built.
@@ -49,6 +50,20 @@ cudaError_t launch_decode_causal(const DecodeParams& p, int kfmt, int kb, int vb
 // Tensor-core quantize (d = 128, 16-bit input, MSE bits 1..4).
 cudaError_t launch_umma_quantize(const CUtensorMap& map, const UmmaQuantParams& p, int bits, int grid,
                                  cudaStream_t stream);
+// Split-precision product for wide vectors: maps = {A_hi, A_lo, B_hi, B_lo}; epi 0 writes
+// codes (bits 1..4) and the QJL residual, epi 1 the sign words.
+cudaError_t launch_split_gemm(const CUtensorMap* maps, const SplitGemmParams& p, int epi, int bits, int grid,
+                              cudaStream_t s);
+// Tensor-core estimator operands: [a | b] rows as bf16 hi + lo; records decoded to
+// [c[code] | coef * gamma * (2s - 1)] rows as bf16 hi + lo.
+cudaError_t launch_split_cat(const float* a, int da, const float* b, int db, int64_t rows, uint16_t* hi,
+                             uint16_t* lo, cudaStream_t s);
+cudaError_t launch_expand_records(const uint32_t* codes, int code_words, const uint32_t* signs, int sign_words,
+                                  const float* rnorms, const float* centroids, float coef, int64_t n, int d, int m,
+                                  int bits, uint16_t* hi, uint16_t* lo, cudaStream_t s);
+// fp32 rows -> bf16 hi + lo parts (and row norms when norms != nullptr).
+cudaError_t launch_split_rows(const float* x, int64_t rows, int d, uint16_t* hi, uint16_t* lo, float* norms,
+                              cudaStream_t s);
 // TurboQuant-prod with m = d = 128: the rotation and the QJL projection on the tensor cores
 cudaError_t launch_umma_quantize_prod(const CUtensorMap& map, const UmmaQuantParams& p, int mse_bits, int grid,
                                       cudaStream_t s);

@@ -17,6 +17,7 @@
 #include "decode_aux.cuh"
 #include "decode_split.cuh"
 #include "decode_tma.cuh"
+#include "gemm_umma.cuh"
 #include "device_common.cuh"
 #include "launchers.h"
 #include "quantize_simt.cuh"
@@ -312,7 +313,8 @@ tq_status quantize_common(const tq_quantizer* q, const void* x, int dtype, int64
     return static_cast<size_t>(tvv) * (dp + yp) * 4 + 32 * 132 * 4 + static_cast<size_t>(tvv) * 12 +
            static_cast<size_t>(tvv) * d + 16;
   };
-  int tv = 32;
+  // a few vectors (a decode step's append) spread over more CTAs
+  int tv = n <= 16 * 148 ? 8 : 32;
   while (tv > 8 && smem_for(tv) > 200 * 1024) tv -= 8;
   if (smem_for(tv) > 220 * 1024) return fail(TQ_ERR_UNSUPPORTED, "d = %d too large for the general quantize kernel", d);
   p.tv = tv;
@@ -407,6 +409,114 @@ tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int
   if (vq->kind == TQ_KIND_MSE && vq->bits > 4) return fail(TQ_ERR_UNSUPPORTED, "value bits > 4");
   if (kq->kind == TQ_KIND_SPECTRAL && (kq->tail_bits > 2 || kq->tail_bits != vq->tail_bits))
     return fail(TQ_ERR_UNSUPPORTED, "spectral tail bits must be equal and <= 2");
+  return TQ_OK;
+}
+
+// ---- wide vectors on the tensor cores (split-precision products, workspace) ----
+
+// fp32 input, d a multiple of 256 (<= 4096): MSE with 1..4 bits, or PROD with 2..5 bits and m = d.
+bool wide_supported(const tq_quantizer* q, int dtype) {
+  if (dtype != TQ_F32 || q->d < 256 || q->d % 256 || q->d > 4096) return false;
+  if (q->kind == TQ_KIND_MSE) return q->bits >= 1 && q->bits <= 4;
+  if (q->kind == TQ_KIND_PROD) return q->bits >= 2 && q->bits <= 5 && q->m == q->d && q->S;
+  return false;
+}
+
+constexpr int64_t kWideBatch = 32768;     // vectors per pass of the workspace
+
+struct WidePlan {
+  size_t pi, s, xh, xl, rh, rl, nx, r2, bytes;
+  int64_t nb;
+};
+
+WidePlan plan_wide(const tq_quantizer* q, int64_t n) {
+  WidePlan P{};
+  const int64_t d = q->d, m = q->kind == TQ_KIND_PROD ? q->m : 0;
+  P.nb = std::max<int64_t>(1, std::min<int64_t>(n, kWideBatch));
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t off = 0;
+  P.pi = off; off = al(off + 2 * d * d * 2);
+  P.s = off; off = al(off + 2 * m * d * 2);
+  P.xh = off; off = al(off + P.nb * d * 2);
+  P.xl = off; off = al(off + P.nb * d * 2);
+  P.rh = off; off = al(off + (m ? P.nb * d * 2 : 0));
+  P.rl = off; off = al(off + (m ? P.nb * d * 2 : 0));
+  P.nx = off; off = al(off + P.nb * 4);
+  P.r2 = off; off = al(off + P.nb * (d / 256) * 4);
+  P.bytes = off;
+  return P;
+}
+
+// 2D bf16 tensor map of a row-major [rows][cols] array with a 64-column x box_rows box.
+tq_status bf16_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+  auto encode = get_encode();
+  if (!encode) return fail(TQ_ERR_UNSUPPORTED, "tensor maps unavailable");
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols * 2)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TQ_OK : fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+}
+
+tq_status quantize_wide(const tq_quantizer* q, const float* x, int64_t n, tq_packed out, char* ws,
+                        cudaStream_t stream) {
+  const WidePlan P = plan_wide(q, n);
+  const int d = q->d;
+  const bool prod = q->kind == TQ_KIND_PROD;
+  const int m = prod ? q->m : 0;
+  const int bmse = prod ? q->bits - 1 : q->bits;
+  const tq_layout L = layout_of(q);
+  auto u16 = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  // rotation (and S) split once per call
+  cudaError_t e = launch_split_rows(q->rot, d, d, u16(P.pi), u16(P.pi) + static_cast<size_t>(d) * d, nullptr, stream);
+  if (e == cudaSuccess && prod)
+    e = launch_split_rows(q->S, m, d, u16(P.s), u16(P.s) + static_cast<size_t>(m) * d, nullptr, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "split launch");
+  CUtensorMap pimaps[2], smaps[2];
+  tq_status s;
+  if ((s = bf16_map(&pimaps[0], u16(P.pi), d, d, 256)) != TQ_OK) return s;
+  if ((s = bf16_map(&pimaps[1], u16(P.pi) + static_cast<size_t>(d) * d, d, d, 256)) != TQ_OK) return s;
+  if (prod) {
+    if ((s = bf16_map(&smaps[0], u16(P.s), m, d, 256)) != TQ_OK) return s;
+    if ((s = bf16_map(&smaps[1], u16(P.s) + static_cast<size_t>(m) * d, m, d, 256)) != TQ_OK) return s;
+  }
+  int* status = device_status_ptr();
+  for (int64_t v0 = 0; v0 < n; v0 += P.nb) {
+    const int64_t nb = std::min<int64_t>(P.nb, n - v0);
+    e = launch_split_rows(x + v0 * d, nb, d, u16(P.xh), u16(P.xl), f32(P.nx), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "split launch");
+    CUtensorMap maps[4];
+    if ((s = bf16_map(&maps[0], u16(P.xh), nb, d, 128)) != TQ_OK) return s;
+    if ((s = bf16_map(&maps[1], u16(P.xl), nb, d, 128)) != TQ_OK) return s;
+    maps[2] = pimaps[0];
+    maps[3] = pimaps[1];
+    SplitGemmParams g{};
+    g.M = nb; g.N = d; g.K = d; g.status = status; g.wait_limit = wait_limit();
+    g.rnorm_x = f32(P.nx); g.boundaries = q->boundaries; g.centroids = q->centroids;
+    g.codes = out.codes + v0 * L.code_words; g.code_words = L.code_words;
+    g.norms = out.norms + v0;
+    if (prod) { g.r_hi = u16(P.rh); g.r_lo = u16(P.rl); g.r2_part = f32(P.r2); }
+    const int64_t work = (nb + 127) / 128 * (d / 256);
+    const int grid = static_cast<int>(std::min<int64_t>(work, sm_count()));
+    e = launch_split_gemm(maps, g, GEMM_EPI_QUANT, bmse, grid, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wide rotation launch");
+    if (!prod) continue;
+    if ((s = bf16_map(&maps[0], u16(P.rh), nb, d, 128)) != TQ_OK) return s;
+    if ((s = bf16_map(&maps[1], u16(P.rl), nb, d, 128)) != TQ_OK) return s;
+    maps[2] = smaps[0];
+    maps[3] = smaps[1];
+    SplitGemmParams z{};
+    z.M = nb; z.N = m; z.K = d; z.status = status; z.wait_limit = wait_limit();
+    z.signs = out.signs + v0 * L.sign_words; z.rnorms = out.rnorms + v0;
+    z.r2_in = f32(P.r2); z.r2_chunks = d / 256;
+    const int64_t zwork = (nb + 127) / 128 * (m / 256);
+    e = launch_split_gemm(maps, z, GEMM_EPI_SIGNS, 1, static_cast<int>(std::min<int64_t>(zwork, sm_count())), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wide projection launch");
+  }
   return TQ_OK;
 }
 
@@ -697,6 +807,37 @@ tq_status tq_quantize_spectral(const tq_quantizer* q, const void* x, int32_t dty
                          q ? q->d : 0, nullptr);
 }
 
+tq_status tq_quantize_workspace(const tq_quantizer* q, int32_t dtype, int64_t n, size_t* bytes) {
+  tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (!bytes || n < 0) return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
+  *bytes = wide_supported(q, dtype) && n > 0 ? plan_wide(q, n).bytes : 0;
+  return TQ_OK;
+}
+
+tq_status tq_quantize_ws(const tq_quantizer* q, const void* x, int32_t dtype, int64_t n, tq_packed out,
+                         void* workspace, size_t ws_bytes, tq_stream stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  tq_status s = check_quantizer(q);
+  if (s != TQ_OK) return s;
+  if (q->kind == TQ_KIND_SPECTRAL || n <= 0 || !wide_supported(q, dtype))
+    return quantize_common(q, x, dtype, n, out, stream, q->kind, q->d, nullptr);
+  if (q->kind == TQ_KIND_PROD && q->bits > 1 && (!q->centroids || !q->boundaries))
+    return fail(TQ_ERR_INVALID_ARG, "codebook is NULL");
+  if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
+  if (!aligned16(x)) return fail(TQ_ERR_ALIGNMENT, "x is not 16-byte aligned");
+  const tq_layout L = layout_of(q);
+  if ((s = check_packed(out, L)) != TQ_OK) return s;
+  const WidePlan P = plan_wide(q, n);
+  if (!workspace || ws_bytes < P.bytes) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", P.bytes);
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  Range outs[4];
+  packed_ranges(out, L, n, outs);
+  const Range ins[2] = {{x, static_cast<size_t>(n) * q->d * 4}, {workspace, ws_bytes}};
+  if ((s = check_no_alias(outs, 4, ins, 2)) != TQ_OK) return s;
+  return quantize_wide(q, static_cast<const float*>(x), n, out, static_cast<char*>(workspace), stream);
+}
+
 tq_status tq_dequantize(const tq_quantizer* q, tq_packed in, int64_t n, float* out, tq_stream stream) {
   tq_status s = check_quantizer(q);
   if (s != TQ_OK) return s;
@@ -740,6 +881,43 @@ static int score_qu_stride(const tq_quantizer* q) {
   return 0;
 }
 
+// Estimates on the tensor cores: MSE (1..4 bits) or PROD (2..5 bits, m = d) records with d a
+// multiple of 256, against at least 4096 records.  Queries [q' | S q'] and decoded records
+// [c[code] | sqrt(pi/2)/m gamma (2s - 1)] become split-precision operands of one product;
+// the column scale is the record norm.
+static bool score_wide(const tq_quantizer* q, int64_t n) {
+  if (q->d < 256 || q->d % 256 || q->d > 4096 || n < 4096 || std::getenv("TQ_FORCE_SIMT")) return false;
+  if (q->kind == TQ_KIND_MSE) return q->bits >= 1 && q->bits <= 4;
+  if (q->kind == TQ_KIND_PROD) return q->bits >= 2 && q->bits <= 5 && q->m == q->d;
+  return false;
+}
+
+struct ScoreWidePlan {
+  size_t qr, qu, ah, al, bh, bl, dense, bytes;
+  int64_t qb;
+  int K;
+};
+
+static ScoreWidePlan plan_score_wide(const tq_quantizer* q, int64_t nq, int64_t n, int topk) {
+  ScoreWidePlan P{};
+  const int64_t d = q->d, m = q->kind == TQ_KIND_PROD ? q->m : 0;
+  P.K = static_cast<int>(d + m);
+  int64_t qb = (1ll << 28) / std::max<int64_t>(n, 1) / 128 * 128;
+  qb = std::max<int64_t>(128, std::min<int64_t>(1024, qb));
+  P.qb = std::min<int64_t>(qb, (nq + 127) / 128 * 128);
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t off = 0;
+  P.qr = off; off = al(off + nq * d * 4);
+  P.qu = off; off = al(off + nq * std::max<int64_t>(m, 1) * 4);
+  P.ah = off; off = al(off + P.qb * P.K * 2);
+  P.al = off; off = al(off + P.qb * P.K * 2);
+  P.bh = off; off = al(off + n * P.K * 2);
+  P.bl = off; off = al(off + n * P.K * 2);
+  P.dense = off; off = al(off + (topk > 0 ? P.qb * n * 4 : 0));
+  P.bytes = off;
+  return P;
+}
+
 // Estimator parameters of one quantizer's records (the rotated queries and the output are
 // filled in per launch).
 static ScoreParams score_params(const tq_quantizer* q, const tq_layout& L, const tq_packed& keys, int64_t n) {
@@ -771,6 +949,10 @@ tq_status tq_score_workspace(const tq_quantizer* q, int64_t nq, int64_t n, int32
   tq_status s = check_quantizer(q);
   if (s != TQ_OK) return s;
   if (!bytes || nq < 0 || n < 0) return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
+  if (score_wide(q, n) && nq > 0) {
+    *bytes = plan_score_wide(q, nq, n, topk).bytes;
+    return TQ_OK;
+  }
   size_t b = static_cast<size_t>(nq) * q->d * 4 + 256;
   b += static_cast<size_t>(nq) * score_qu_stride(q) * 4 + 256;
   if (topk > 0) b += static_cast<size_t>(score_block(nq, n)) * static_cast<size_t>(n) * 4 + 256;
@@ -810,6 +992,45 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
   const int d = q->d;
   const int qus = score_qu_stride(q);
   char* ws = static_cast<char*>(workspace);
+  if (score_wide(q, n)) {
+    const ScoreWidePlan P = plan_score_wide(q, nq, n, topk);
+    float* qr = reinterpret_cast<float*>(ws + P.qr);
+    float* qu = reinterpret_cast<float*>(ws + P.qu);
+    const int m = q->kind == TQ_KIND_PROD ? q->m : 0;
+    auto u16 = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+    score_qprep_kernel<<<static_cast<unsigned>(nq), 128, 2 * d * 4, stream>>>(
+        qv, dtype, d, q->kind, q->rot, q->S, q->m, q->k_top, qr, m ? qu : nullptr, qus, d, nullptr, device_status_ptr());
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "score qprep launch");
+    const int bm = q->kind == TQ_KIND_PROD ? q->bits - 1 : q->bits;
+    const float coef = m ? static_cast<float>(std::sqrt(M_PI / 2.0) / m) : 0.f;
+    e = launch_expand_records(keys.codes, L.code_words, keys.signs, L.sign_words, keys.rnorms, q->centroids, coef, n,
+                              d, m, bm, u16(P.bh), u16(P.bl), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "record expansion launch");
+    CUtensorMap maps[4];
+    if ((s = bf16_map(&maps[2], u16(P.bh), n, P.K, 256)) != TQ_OK) return s;
+    if ((s = bf16_map(&maps[3], u16(P.bl), n, P.K, 256)) != TQ_OK) return s;
+    float* dense = reinterpret_cast<float*>(ws + P.dense);
+    for (int64_t q0 = 0; q0 < nq; q0 += P.qb) {
+      const int64_t nb = std::min(P.qb, nq - q0);
+      e = launch_split_cat(qr + q0 * d, d, qu + q0 * m, m, nb, u16(P.ah), u16(P.al), stream);
+      if (e != cudaSuccess) return cuda_fail(e, "query split launch");
+      if ((s = bf16_map(&maps[0], u16(P.ah), nb, P.K, 128)) != TQ_OK) return s;
+      if ((s = bf16_map(&maps[1], u16(P.al), nb, P.K, 128)) != TQ_OK) return s;
+      SplitGemmParams g{};
+      g.M = nb; g.N = static_cast<int>(n); g.K = P.K; g.status = device_status_ptr(); g.wait_limit = wait_limit();
+      g.out = topk > 0 ? dense : scores + q0 * n; g.ldo = n; g.col_scale = keys.norms;
+      const int64_t work = (nb + 127) / 128 * ((n + 255) / 256);
+      e = launch_split_gemm(maps, g, GEMM_EPI_SCORE, 1, static_cast<int>(std::min<int64_t>(work, sm_count())), stream);
+      if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
+      if (topk > 0) {
+        if (topk <= 16) topk_kernel<16><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+        else topk_kernel<32><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+      }
+    }
+    return TQ_OK;
+  }
   float* qr = reinterpret_cast<float*>(ws);
   float* qu = qus ? reinterpret_cast<float*>(ws + (static_cast<size_t>(nq) * d * 4 + 255) / 256 * 256) : nullptr;
   float* dense = reinterpret_cast<float*>(

@@ -33,7 +33,8 @@ EXPORTS = [
     "tq_decode_attn_workspace", "tq_decode_attn", "tq_get_status", "tq_set_wait_limit", "tq_lut_scale",
     "tq_decode_attn_fixed_ws", "tq_quantize_split", "tq_score_split_workspace", "tq_score_split",
     "tq_decode_attn_split_workspace", "tq_decode_attn_split", "tq_spectral_descriptor", "tq_spectral_prepare",
-    "tq_decode_attn_paged", "tq_prefill_attn_workspace", "tq_prefill_attn",
+    "tq_decode_attn_paged", "tq_prefill_attn_workspace", "tq_prefill_attn", "tq_quantize_workspace",
+    "tq_quantize_ws",
 ]
 
 
@@ -100,6 +101,8 @@ def lib():
             "tq_quantize_mse": ([qp, vp, i32, i64, Packed_t, vp], C.c_int),
             "tq_quantize_prod": ([qp, vp, i32, i64, Packed_t, vp], C.c_int),
             "tq_quantize_spectral": ([qp, vp, i32, i64, Packed_t, vp], C.c_int),
+            "tq_quantize_workspace": ([qp, i32, i64, C.POINTER(C.c_size_t)], C.c_int),
+            "tq_quantize_ws": ([qp, vp, i32, i64, Packed_t, vp, C.c_size_t, vp], C.c_int),
             "tq_dequantize": ([qp, Packed_t, i64, vp, vp], C.c_int),
             "tq_score_workspace": ([qp, i64, i64, i32, C.POINTER(C.c_size_t)], C.c_int),
             "tq_score": ([qp, vp, i32, i64, Packed_t, i64, i32, vp, vp, vp, C.c_size_t, vp], C.c_int),
@@ -349,6 +352,28 @@ def quantize(q: Quantizer, x, out: Optional[Packed] = None, stream=None) -> Pack
     fn = {KIND_MSE: lib().tq_quantize_mse, KIND_PROD: lib().tq_quantize_prod,
           KIND_SPECTRAL: lib().tq_quantize_spectral}[q.kind]
     _check(fn(q.ref, x.data_ptr(), _dtype_code(x), n, out.as_c(), _stream(stream)))
+    return out
+
+
+def tq_quantize_workspace_bytes(q: Quantizer, x) -> int:
+    ws = C.c_size_t(0)
+    _check(lib().tq_quantize_workspace(q.ref, _dtype_code(x), x.numel() // q.d, C.byref(ws)))
+    return ws.value
+
+
+def quantize_ws(q: Quantizer, x, out: Optional[Packed] = None, workspace=None, stream=None) -> Packed:
+    """tq_quantize_ws: the same records as quantize(), with device scratch (wide fp32 vectors
+    take the tensor-core split-precision path)."""
+    import torch
+    assert x.is_cuda and x.is_contiguous() and x.shape[-1] == q.d
+    n = x.numel() // q.d
+    out = q.alloc(n, x.device) if out is None else out
+    ws = C.c_size_t(0)
+    _check(lib().tq_quantize_workspace(q.ref, _dtype_code(x), n, C.byref(ws)))
+    if workspace is None or workspace.numel() < ws.value:
+        workspace = torch.empty(max(ws.value, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().tq_quantize_ws(q.ref, x.data_ptr(), _dtype_code(x), n, out.as_c(), workspace.data_ptr(),
+                                workspace.numel(), _stream(stream)))
     return out
 
 

@@ -3,7 +3,8 @@ of d = 1536 (the stand-in for the review's OpenAI3 d=1536 embeddings), TurboQuan
 b = 2 and b = 4 with m = 1536 QJL rows, exhaustive top-10 of the first 100 queries, in the
 launch configuration bench.py times (``--workload c5``).
 
-The oracle cannot quantize the whole database in a test, so the check is on samples and
+The database is quantized with tq_quantize_ws (rotation and QJL projection on the tensor
+cores).  The oracle cannot quantize the whole database in a test, so the check is on samples and
 on properties that hold at any size:
   * sampled records (3000 random ids plus every id the GPU returns) are band-checked
     against the oracle's quantization of the same rows, and the oracle's estimates with
@@ -51,7 +52,7 @@ def database():
 def test_search1m_top10(database, bits):
     w = database
     kq = K.Quantizer.prod(w["rot"], w["S"], bits)
-    kc = K.quantize(kq, w["db"])
+    kc = K.quantize_ws(kq, w["db"])         # tensor-core rotation and projection (split precision)
     vals, ids = K.score(kq, w["qs"], kc, NDB, topk=TOP)
     dense = K.score(kq, w["qs"], kc, NDB)
     torch.cuda.synchronize()

@@ -189,3 +189,57 @@ def test_quantize_spectral_parity(qjl):
     xh = K.dequantize(q, out, n).cpu().numpy()
     xr = OSP.dequantize_spectral(a["chat"], desc)
     assert np.max(np.abs(xh - xr)) < 1e-4 * np.max(np.abs(xr))
+
+
+@pytest.mark.parametrize("d,kind,bits,n", [(1536, "prod", 2, 3000), (1536, "prod", 4, 1000), (256, "prod", 3, 777),
+                                           (1536, "mse", 3, 500), (512, "mse", 1, 129), (256, "prod", 5, 1)])
+def test_quantize_wide_tensor_core_parity(d, kind, bits, n):
+    """tq_quantize_ws on fp32 vectors with d a multiple of 256: the rotation and the QJL
+    projection as split-precision tensor-core products; records band-checked against the
+    oracle (codes and signs), norms and residual norms to 1e-5."""
+    from _parity import adopt_mse, adopt_prod
+    rot = ti.haar_rotation(d, 1200 + d)
+    S = ti.gaussian_matrix(d, d, 2200 + d)
+    x = ti.unit_gaussian(n, d, 4200 + d + bits) * 3.0
+    if n > 5:
+        x[3] = 0.0                                  # a zero vector
+    xt = torch.from_numpy(x.astype(np.float32)).cuda()
+    x64 = xt.double().cpu().numpy()
+    q = K.Quantizer.prod(rot, S, bits) if kind == "prod" else K.Quantizer.mse(rot, bits)
+    out = K.quantize_ws(q, xt)
+    torch.cuda.synchronize()
+    assert K.get_status() == 0
+    nrm = out.norms.cpu().numpy().astype(np.float64)
+    ref_n = np.linalg.norm(x64, axis=1)
+    assert np.all(np.abs(nrm - ref_n) <= 1e-5 * np.maximum(ref_n, 1e-30))
+    skip = [3] if n > 5 else []
+    if kind == "mse":
+        c, t, _ = lloyd_max(bits, "beta", d=d)
+        ref = OQ.quantize_mse(x64, rot, c, t, bits)
+        if skip:
+            ref["codes"][3] = as_u32(out.codes)[3]   # the zero row: checked below
+        adopt_mse(as_u32(out.codes), ref, bits, t)
+    else:
+        c, t, _ = lloyd_max(bits - 1, "beta", d=d)
+        ref = OQ.quantize_prod(x64, rot, S, c, t, bits)
+        keep = np.ones(n, dtype=bool)
+        keep[skip] = False
+        sub = {k: (v[keep] if isinstance(v, np.ndarray) and v.shape[:1] == (n,) else v) for k, v in ref.items()}
+        a = adopt_prod(as_u32(out.codes)[keep], as_u32(out.signs)[keep], out.rnorms.cpu().numpy()[keep], sub, bits,
+                       c, t, S)
+        assert a["idx"].shape == (keep.sum(), d)
+    from oracle.quantizer import unpack_codes
+    bm = bits - 1 if kind == "prod" else bits
+    for r in skip:                                   # u = 0: every code is the middle one
+        assert np.all(unpack_codes(as_u32(out.codes)[r:r + 1], d, bm) == (1 << (bm - 1)) - 1)
+
+
+def test_quantize_ws_matches_plain_call_elsewhere():
+    """Shapes outside the wide path: tq_quantize_ws writes the records tq_quantize_* writes."""
+    d, n = 128, 1000
+    rot = ti.haar_rotation(d, 1301)
+    xt = torch.from_numpy(ti.iid_normal((n, d), 4301).astype(np.float32)).to(torch.bfloat16).cuda()
+    q = K.Quantizer.mse(rot, 4)
+    a, b = K.quantize(q, xt), K.quantize_ws(q, xt)
+    torch.cuda.synchronize()
+    assert torch.equal(a.codes, b.codes) and torch.equal(a.norms, b.norms)

@@ -81,3 +81,30 @@ def test_topk_search(bits):
         must = rid[i][rval[i] > kth + 2 * tol]
         assert set(must.tolist()) <= set(ids[i].tolist())
         assert np.all(est[i, ids[i]] >= kth - 2 * tol)
+
+
+@pytest.mark.parametrize("d,kind,bits,n,nq", [(1536, "prod", 2, 5000, 7), (256, "mse", 3, 4500, 130),
+                                              (512, "prod", 5, 4099, 3)])
+def test_scores_wide_tensor_core(d, kind, bits, n, nq):
+    """Dense estimates on the tensor cores (d a multiple of 256, at least 4096 records): every
+    (query, record) estimate equals the oracle's on the GPU's band-checked records to 1e-3
+    (unit-norm queries and records); the ragged last column tile and query tile included."""
+    rot = ti.haar_rotation(d, 1405 + d)
+    S = ti.gaussian_matrix(d, d, 2405 + d)
+    x = ti.unit_gaussian(n, d, 8100 + d).astype(np.float32)
+    qv = ti.unit_gaussian(nq, d, 8101 + d).astype(np.float32)
+    q = K.Quantizer.prod(rot, S, bits) if kind == "prod" else K.Quantizer.mse(rot, bits)
+    pk = K.quantize(q, torch.from_numpy(x).cuda())
+    s = K.score(q, torch.from_numpy(qv).cuda(), pk, n).cpu().numpy().astype(np.float64)
+    assert K.get_status() == 0
+    if kind == "prod":
+        c, t, _ = lloyd_max(bits - 1, "beta", d=d)
+        ref = OQ.quantize_prod(x.astype(np.float64), rot, S, c, t, bits)
+        a = adopt_prod(as_u32(pk.codes), as_u32(pk.signs), pk.rnorms.cpu().numpy(), ref, bits, c, t, S)
+        est = OQ.estimate_prod(qv.astype(np.float64), rot, S, a["chat"], a["s"], ref["norms"], a["rnorms"])
+    else:
+        c, t, _ = lloyd_max(bits, "beta", d=d)
+        ref = OQ.quantize_mse(x.astype(np.float64), rot, c, t, bits)
+        idx, _ = adopt_mse(as_u32(pk.codes), ref, bits, t)
+        est = OQ.estimate_mse(qv.astype(np.float64), rot, idx, ref["norms"], c)
+    assert np.max(np.abs(s - est)) <= 1e-3
