@@ -540,7 +540,8 @@ def run_other(args):
         rec = 4 * (L.code_words + L.sign_words + L.has_norms + L.has_rnorms)
         parts = {"quantize": {"ms": tq, "vectors_per_s": ndb / tq * 1e3, "gbs": ndb * (d5 * 4 + rec) / tq / 1e6},
                  "search_top10": {"ms": ts, "queries_per_s": nq5 / ts * 1e3,
-                                  "note": f"{nq5} queries x {ndb} records, CUDA-core estimator"}}
+                                  "note": f"{nq5} queries x {ndb} records: records decoded once per call, "
+                                          "estimates as one split-precision tcgen05 product, top-10 per query"}}
         parts["quantize"]["note"] = "tq_quantize_ws: rotation and QJL projection as split-precision tcgen05 products"
         desc = (f"search: {ndb} x 1536 fp32 unit vectors, prod b={args.c5_bits} (m=1536), "
                 f"top-10 of {nq5} queries")

@@ -456,17 +456,18 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 128;
       const int64_t v = tile * kUmmaTileRows + r;
       if constexpr (PRODK) {
-        float y[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, y[c]);
-        tmem_wait_ld();
-        // (the accumulator stays with this group: Z lands in it next)
+        // tensor memory is read twice (||y||, then the codes 32 columns at a time), so one
+        // 32-coordinate body serves all four chunks (a small loop body keeps the
+        // instruction stream in cache; the accumulator stays with this group: Z lands in it)
         float2 s2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
+          float yv[32];
+          tmem_ld32(taddr + 32 * c, yv);
+          tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float2 v2 = make_float2(y[c][i], y[c][i + 1]);
+            const float2 v2 = make_float2(yv[i], yv[i + 1]);
             s2[(i >> 1) & 3] = __ffma2_rn(v2, v2, s2[(i >> 1) & 3]);
           }
         }
@@ -479,8 +480,11 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         const uint32_t rowaddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16);
         const uint32_t rcol = rowaddr + kR + buf * 128;
         float2 g2 = make_float2(0.f, 0.f);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
+          float y[1][32];
+          tmem_ld32(taddr + 32 * c, y[0]);
+          tmem_wait_ld();
           uint32_t wc[B], hw[16], lw[16];
 #pragma unroll
           for (int w = 0; w < B; ++w) wc[w] = 0u;
@@ -488,7 +492,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           for (int i = 0; i < 32; i += 2) {
             uint32_t code[2];
             if (use_cells) {
-              const float2 f2 = make_float2(__saturatef(fmaf(y[c][i], fs, 0.5f)), __saturatef(fmaf(y[c][i + 1], fs, 0.5f)));
+              const float2 f2 = make_float2(__saturatef(fmaf(y[0][i], fs, 0.5f)), __saturatef(fmaf(y[0][i + 1], fs, 0.5f)));
               const float2 gg = __ffma2_rz(f2, make_float2(kCellSpan, kCellSpan), make_float2(8388608.0f, 8388608.0f));
               const uint32_t e0 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gg.x));
               const uint32_t e1 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gg.y));
@@ -499,15 +503,15 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
               uint32_t c0 = 0u, c1 = 0u;
 #pragma unroll
               for (int k = 0; k < NB; ++k) {
-                c0 += y[c][i] * inv > tsm[k] ? 1u : 0u;
-                c1 += y[c][i + 1] * inv > tsm[k] ? 1u : 0u;
+                c0 += y[0][i] * inv > tsm[k] ? 1u : 0u;
+                c1 += y[0][i + 1] * inv > tsm[k] ? 1u : 0u;
               }
               code[0] = c0; code[1] = c1;
             }
             // unit-scale residual r = u - c[code] and its fp16 hi + lo parts (the A operand)
             const float ch0 = __shfl_sync(0xffffffffu, ccen, static_cast<int>(code[0]));
             const float ch1 = __shfl_sync(0xffffffffu, ccen, static_cast<int>(code[1]));
-            const float2 rr = __ffma2_rn(make_float2(y[c][i], y[c][i + 1]), make_float2(inv, inv), make_float2(-ch0, -ch1));
+            const float2 rr = __ffma2_rn(make_float2(y[0][i], y[0][i + 1]), make_float2(inv, inv), make_float2(-ch0, -ch1));
             g2 = __ffma2_rn(rr, rr, g2);
             // hi = half2(r), lo = half2(r - hi): one paired conversion each, one packed FMA
             const __half2 h2 = __floats2half2_rn(rr.x, rr.y);
