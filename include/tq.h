@@ -251,7 +251,7 @@ tq_status tq_quantize_workspace(const tq_quantizer* q, int32_t dtype, int64_t n,
 /*
  * DEVICE.  Quantize with caller-provided device scratch: the records are exactly those of
  * tq_quantize_mse / tq_quantize_prod / tq_quantize_spectral (by q->kind).  For fp32 input
- * with d a multiple of 256 (up to 4096; the review's d = 1536 vector-search embeddings),
+ * with d a multiple of 128 (up to 4096; the review's d = 1536 vector-search embeddings),
  * MSE with 1..4 bits or PROD with 2..5 bits and m = d, the rotation and the QJL projection
  * run on the tensor cores as split-precision products (x, Pi, S and the residual split
  * into bf16 hi + lo parts in the workspace, three products per pair, fp32 accumulation),

@@ -41,13 +41,20 @@ __global__ void __launch_bounds__(256) split_rows_kernel(const float* __restrict
 }
 
 
+template <int EPI, int B, int TN>
+cudaError_t go_tn(const CUtensorMap* maps, const SplitGemmParams& p, int grid, cudaStream_t s) {
+  auto k = split_gemm_kernel<EPI, B, TN>;
+  const uint32_t smem = gemm_smem_bytes(TN);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k<<<grid, kGemmThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+  return cudaGetLastError();
+}
+
+// N tiles of 256 columns, or of 128 when N is not a multiple of 256
 template <int EPI, int B>
 cudaError_t go(const CUtensorMap* maps, const SplitGemmParams& p, int grid, cudaStream_t s) {
-  auto k = split_gemm_kernel<EPI, B>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGemmSmemBytes));
-  if (e != cudaSuccess) return e;
-  k<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(maps[0], maps[1], maps[2], maps[3], p);
-  return cudaGetLastError();
+  return gemm_tile_n(p.N) == 256 ? go_tn<EPI, B, 256>(maps, p, grid, s) : go_tn<EPI, B, 128>(maps, p, grid, s);
 }
 
 // Queries for the tensor-core estimator: row r of [qr | qu] (fp32, d + m columns) as bf16

@@ -1,4 +1,4 @@
-// Split-precision tensor-core product for wide vectors (d a multiple of 256, e.g. 1536):
+// Split-precision tensor-core product for fp32 vectors (d a multiple of 128, e.g. 128 or 1536):
 //
 //   C[M x N] = A[M x K] . B[N x K]^T   with A = A_hi + A_lo and B = B_hi + B_lo in bf16,
 //   accumulated as A_hi B_hi + A_hi B_lo + A_lo B_hi in fp32 (tensor memory).
@@ -7,12 +7,13 @@
 // fp32 product's scale, so a rotated coordinate of a unit vector is exact far inside the
 // 1e-5 decision band (TurboQuant review, "Method": y = Pi x / ||x||, then per-coordinate
 // Lloyd-Max codes; the QJL variant projects the residual with S).  Rows of A are vectors
-// (128 per tile), N is cut into 256-wide chunks, K runs in 64-wide stages.
+// (128 per tile), N is cut into TN-wide chunks (256, or 128 when N is not a multiple of
+// 256), K runs in 64-wide stages.
 //
 // Roles in a persistent CTA (one per SM), 192 threads:
-//   warp 0      TMA producer: A_hi, A_lo (128 x 64) and B_hi, B_lo (256 x 64) per stage
-//   warp 1      TMEM allocator (512 columns: two 256-column accumulators) and MMA issuer
-//   warps 2-5   epilogue: one row per thread, the 256 accumulator columns of a tile
+//   warp 0      TMA producer: A_hi, A_lo (128 x 64) and B_hi, B_lo (TN x 64) per stage
+//   warp 1      TMEM allocator (512 columns: two TN-column accumulators) and MMA issuer
+//   warps 2-5   epilogue: one row per thread, the TN accumulator columns of a tile
 // Epilogues:
 //   QUANT  y = acc / ||x||: codes against the Lloyd-Max boundaries, packed LSB-first into
 //          the record's stream; with a QJL stage, the residual r = y - c[code] as bf16
@@ -34,18 +35,22 @@ namespace tq {
 constexpr int kGemmThreads = 192;
 constexpr int kGemmStages = 2;
 constexpr int kGemmTileM = 128;
-constexpr int kGemmTileN = 256;
 constexpr int kGemmTileK = 64;
 constexpr uint32_t kGemmAStage = kGemmTileM * kGemmTileK * 2;     // 16 KB per part
-constexpr uint32_t kGemmBStage = kGemmTileN * kGemmTileK * 2;     // 32 KB per part
-constexpr uint32_t kGemmStageBytes = 2 * kGemmAStage + 2 * kGemmBStage;
-constexpr uint32_t kGemmSmemBytes = 1024 + kGemmStages * kGemmStageBytes + 256 + 512 * 4;
+__host__ __device__ constexpr uint32_t gemm_b_stage(int tn) { return static_cast<uint32_t>(tn) * kGemmTileK * 2; }
+__host__ __device__ constexpr uint32_t gemm_stage_bytes(int tn) { return 2 * kGemmAStage + 2 * gemm_b_stage(tn); }
+__host__ __device__ constexpr uint32_t gemm_smem_bytes(int tn) {
+  return 1024 + kGemmStages * gemm_stage_bytes(tn) + 256 + 512 * 4;
+}
 
 enum : int { GEMM_EPI_QUANT = 0, GEMM_EPI_SIGNS = 1, GEMM_EPI_SCORE = 2 };
 
+// Column tile of a product with N output columns (the SCORE epilogue takes any N).
+__host__ __device__ constexpr int gemm_tile_n(int n) { return n % 256 == 0 || n > 4096 ? 256 : 128; }
+
 struct SplitGemmParams {
   int64_t M;               // rows (vectors)
-  int N, K;                // output columns and contraction length (multiples of 256 and 64)
+  int N, K;                // output columns and contraction length (multiples of TN and 64)
   int* status;
   long long wait_limit;
   // QUANT
@@ -56,7 +61,7 @@ struct SplitGemmParams {
   int code_words;
   uint16_t* r_hi;          // [M][K] bf16 residual parts (QJL stage), or nullptr
   uint16_t* r_lo;
-  float* r2_part;          // [M][N / 256] parts of ||r||^2
+  float* r2_part;          // [M][N / TN] parts of ||r||^2
   float* norms;            // [M] record norms (written once, by column chunk 0)
   // SIGNS
   uint32_t* signs;         // [M][N / 32]
@@ -69,9 +74,9 @@ struct SplitGemmParams {
   const float* col_scale;  // [N]
 };
 
-// Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = 256.
-__device__ __forceinline__ uint32_t idesc_m128n256_bf16() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+// Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = tn.
+__device__ __forceinline__ uint32_t idesc_m128_bf16(uint32_t tn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((tn >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 __device__ __forceinline__ void tma_load_2d_g(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -80,12 +85,15 @@ __device__ __forceinline__ void tma_load_2d_g(uint32_t dst, const CUtensorMap* m
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
 
-template <int EPI, int B>
+template <int EPI, int B, int TN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                   const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
                   const SplitGemmParams p) {
   constexpr int NS = kGemmStages;
+  constexpr uint32_t kGemmBStage = gemm_b_stage(TN), kGemmStageBytes = gemm_stage_bytes(TN);
+  constexpr int kGemmTileN = TN;
+  constexpr int NCH = TN / 32;                   // 32-column chunks of a tile
   constexpr int NB = (1 << B) - 1;
   extern __shared__ unsigned char gsm_raw[];
   const uint32_t raw = smem_u32(gsm_raw);
@@ -155,14 +163,14 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_m128n256_bf16();
+      const uint32_t idesc = idesc_m128_bf16(TN);
       int it = 0, t = 0;                           // stage uses, tiles
       bool stop = false;
       for (int64_t w = blockIdx.x; w < n_work && !stop; w += gridDim.x, ++t) {
         const int buf = t & 1, j = t >> 1;
         if (j > 0 && !mbar_wait(tempty_bar(buf), (j - 1) & 1, lim, p.status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t td = tmem_base + buf * 256;
+        const uint32_t td = tmem_base + buf * TN;
         for (int ks = 0; ks < k_steps; ++ks, ++it) {
           const int s = it % NS;
           if (!mbar_wait(full_bar(s), (it / NS) & 1, lim, p.status, abort_flag)) { stop = true; break; }
@@ -198,13 +206,13 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
       tc_fence_after();
       const int64_t v = (w / n_tiles) * kGemmTileM + r;
       const int nt = static_cast<int>(w % n_tiles);
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 256;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * TN;
       if constexpr (EPI == GEMM_EPI_QUANT) {
         const float nx = v < p.M ? __ldg(p.rnorm_x + v) : 0.f;
         const float inv = nx > 0.f ? 1.f / nx : 0.f;   // a zero row keeps y = 0
         float g2 = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {                  // 32 columns at a time
+        for (int c = 0; c < NCH; ++c) {                  // 32 columns at a time
           float y[32];
           tmem_ld32(taddr + 32 * c, y);
           tmem_wait_ld();
@@ -255,7 +263,7 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
         }
       } else if constexpr (EPI == GEMM_EPI_SCORE) {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < NCH; ++c) {
           float z[32];
           tmem_ld32(taddr + 32 * c, z);
           tmem_wait_ld();
@@ -276,9 +284,9 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
         tc_fence_before();
         mbar_arrive(tempty_bar(buf));
       } else {
-        uint32_t sw[8];
+        uint32_t sw[NCH];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < NCH; ++c) {
           float z[32];
           tmem_ld32(taddr + 32 * c, z);
           tmem_wait_ld();
@@ -290,9 +298,9 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
         tc_fence_before();
         mbar_arrive(tempty_bar(buf));
         if (v < p.M) {
-          uint4* dst = reinterpret_cast<uint4*>(p.signs + v * (p.N / 32) + nt * 8);
-          dst[0] = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-          dst[1] = make_uint4(sw[4], sw[5], sw[6], sw[7]);
+          uint4* dst = reinterpret_cast<uint4*>(p.signs + v * (p.N / 32) + nt * NCH);
+#pragma unroll
+          for (int q = 0; q < NCH / 4; ++q) dst[q] = make_uint4(sw[4 * q], sw[4 * q + 1], sw[4 * q + 2], sw[4 * q + 3]);
           if (nt == 0) {
             float g2 = 0.f;
             for (int q = 0; q < p.r2_chunks; ++q) g2 += p.r2_in[v * p.r2_chunks + q];

@@ -28,10 +28,10 @@
 // core product Z[128 x 128] = R . S^T.  The epilogue writes r as fp16 hi + lo parts into
 // tensor memory, where it is the A operand (S hi + lo in shared memory is B); the three
 // products R_hi S_hi + R_hi S_lo + R_lo S_hi keep every projection within ~1e-6 ||S_i|| ||r||
-// of the fp32 value, far inside the 1e-5 ||S_i|| sign band.  Tensor memory, per epilogue
-// group (tile parity): a 128-column accumulator that holds Y and then Z (the projection
-// overwrites Y once the group has read it) and 128 columns of R_hi | R_lo, 512 in all; the
-// accumulator goes back to the MMA warp after the group has read Z.
+// of the fp32 value, far inside the 1e-5 ||S_i|| sign band.  Tensor memory: one Y
+// accumulator (128 columns, handed back as soon as an epilogue group has read its row),
+// one Z accumulator (128) and one R_hi | R_lo block per epilogue group (2 x 128), 512 in
+// all; the groups overlap their code and residual arithmetic and meet only on Y and Z.
 // Every mbarrier wait is bounded; on timeout the CTA records TQ_ERR_TIMEOUT, drains
 // what it issued, frees TMEM and exits.
 #pragma once
@@ -239,8 +239,8 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   static_assert(PRODK || NT * kPiBytes + NS * kXStageBytes == 2 * kPiBytes + kUmmaStages * kXStageBytes, "smem");
   static_assert(!PRODK || 1024 + NPI * kPiBytes + NS * kXStageBytes + 256 + 64 * 4 <= kUmmaProdSmemBytes, "smem");
   constexpr uint32_t kTmemCols = PRODK ? 512u : 256u;
-  // prod tensor-memory columns of buffer b: Y then Z at 128 b, R_hi at 256 + 128 b, R_lo 64 after
-  constexpr uint32_t kR = 256u;
+  // prod tensor-memory columns: Y 0..127, Z 128..255, R_hi of group b at 256 + 128 b, R_lo 64 after
+  constexpr uint32_t kZcol = 128u, kR = 256u;
   extern __shared__ unsigned char usm_raw[];
   const uint32_t raw = smem_u32(usm_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -254,9 +254,11 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * NS + 2 + b); };
-  // prod, per buffer: R written (count 128), Z committed (1)
+  // prod: R of group b written (count 128), Z committed (1), Z read (count 128); Y uses the
+  // tfull / tempty pair of buffer 0 as its single full / empty barrier
   auto rfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 4 + b); };
-  auto zfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 6 + b); };
+  auto zfull_bar = [&]() { return bar0 + 8u * (2 * NS + 6); };
+  auto zempty_bar = [&]() { return bar0 + 8u * (2 * NS + 7); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + (PRODK ? 8 : 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tsm = reinterpret_cast<float*>(tmem_slot + 2);   // boundaries [NB]
@@ -324,8 +326,11 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), 128); }
-    if (PRODK)
-      for (int b = 0; b < 2; ++b) { mbar_init(rfull_bar(b), 128); mbar_init(zfull_bar(b), 1); }
+    if (PRODK) {
+      for (int b = 0; b < 2; ++b) mbar_init(rfull_bar(b), 128);
+      mbar_init(zfull_bar(), 1);
+      mbar_init(zempty_bar(), 128);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -365,15 +370,16 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_m128n128(p.is_f16);
-      // prod: Z(t) = R(t) . S^T once the epilogue of tile t has written R(t) (three fp16
-      // products: R_hi S_hi + R_hi S_lo + R_lo S_hi), into tile t's accumulator
+      // prod: Z(t) = R(t) . S^T once the epilogue of tile t has written R(t) and tile t - 1's
+      // Z has been read (three fp16 products: R_hi S_hi + R_hi S_lo + R_lo S_hi)
       int zt = 0;                                   // next tile whose Z is issued
       auto issue_z = [&]() {
         const int zb = zt & 1;
         if (!mbar_wait(rfull_bar(zb), (zt >> 1) & 1, lim, p.status, abort_flag)) return false;
+        if (zt > 0 && !mbar_wait(zempty_bar(), (zt - 1) & 1, lim, p.status, abort_flag)) return false;
         tc_fence_after();
         const uint32_t zidesc = idesc_m128n128(1);
-        const uint32_t zd = tmem_base + zb * 128, ra = tmem_base + kR + zb * 128;
+        const uint32_t zd = tmem_base + kZcol, ra = tmem_base + kR + zb * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t boff = (kk >> 2) * (kPiBytes / 2) + (kk & 3) * 32;
@@ -381,14 +387,15 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           umma_f16_ts(zd, ra + kk * 8, sw128_desc(s_lo + boff), zidesc, 1u);
           umma_f16_ts(zd, ra + 64 + kk * 8, sw128_desc(s_hi + boff), zidesc, 1u);
         }
-        umma_commit(zfull_bar(zb));
+        umma_commit(zfull_bar());
         ++zt;
         return true;
       };
       int it = 0;                                   // rotations issued
       bool zok = true;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int s = it % NS, buf = it & 1, j = it >> 1;
+        // prod: one Y accumulator (buffer 0, a phase per tile); otherwise two, by tile parity
+        const int s = it % NS, buf = PRODK ? 0 : (it & 1), j = PRODK ? it : (it >> 1);
         if (j > 0 && !mbar_wait(tempty_bar(buf), (j - 1) & 1, lim, p.status, abort_flag)) break;
         if (!mbar_wait(full_bar(s), (it / NS) & 1, lim, p.status, abort_flag)) break;
         tc_fence_after();
@@ -412,10 +419,11 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       // wait for the tensor core to finish everything issued before TMEM is freed
       if (it > 0) {
         const int last = it - 1;
-        for (long long i = 0; !mbar_try(tfull_bar(last & 1), (last >> 1) & 1) && i < kDrainLimit; ++i) {}
+        const int lb = PRODK ? 0 : (last & 1), lp = PRODK ? (last & 1) : ((last >> 1) & 1);
+        for (long long i = 0; !mbar_try(tfull_bar(lb), lp) && i < kDrainLimit; ++i) {}
       }
       if (PRODK && zt > 0)
-        for (long long i = 0; !mbar_try(zfull_bar((zt - 1) & 1), ((zt - 1) >> 1) & 1) && i < kDrainLimit; ++i) {}
+        for (long long i = 0; !mbar_try(zfull_bar(), (zt - 1) & 1) && i < kDrainLimit; ++i) {}
     }
   } else {
     const int grp = (warp - 2) >> 2;                   // 0: warps 2-5, 1: warps 6-9
@@ -451,23 +459,26 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       const int buf = it & 1;
       if (buf != grp) continue;
       const int j = it >> 1;
-      if (!mbar_wait(tfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
+      // prod: the single Y accumulator completes once per tile
+      if (!mbar_wait(tfull_bar(PRODK ? 0 : buf), PRODK ? (it & 1) : (j & 1), lim, p.status, abort_flag)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + buf * 128;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + (PRODK ? 0u : buf * 128u);
       const int64_t v = tile * kUmmaTileRows + r;
       if constexpr (PRODK) {
-        // tensor memory is read twice (||y||, then the codes 32 columns at a time), so one
-        // 32-coordinate body serves all four chunks (a small loop body keeps the
-        // instruction stream in cache; the accumulator stays with this group: Z lands in it)
+        // the whole row comes out of tensor memory at once and Y goes straight back to the
+        // MMA warp (the next tile's rotation runs while this group computes)
+        float y[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, y[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(tempty_bar(0));
         float2 s2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float yv[32];
-          tmem_ld32(taddr + 32 * c, yv);
-          tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float2 v2 = make_float2(yv[i], yv[i + 1]);
+            const float2 v2 = make_float2(y[c][i], y[c][i + 1]);
             s2[(i >> 1) & 3] = __ffma2_rn(v2, v2, s2[(i >> 1) & 3]);
           }
         }
@@ -480,11 +491,8 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
         const uint32_t rowaddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16);
         const uint32_t rcol = rowaddr + kR + buf * 128;
         float2 g2 = make_float2(0.f, 0.f);
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float y[1][32];
-          tmem_ld32(taddr + 32 * c, y[0]);
-          tmem_wait_ld();
           uint32_t wc[B], hw[16], lw[16];
 #pragma unroll
           for (int w = 0; w < B; ++w) wc[w] = 0u;
@@ -492,7 +500,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           for (int i = 0; i < 32; i += 2) {
             uint32_t code[2];
             if (use_cells) {
-              const float2 f2 = make_float2(__saturatef(fmaf(y[0][i], fs, 0.5f)), __saturatef(fmaf(y[0][i + 1], fs, 0.5f)));
+              const float2 f2 = make_float2(__saturatef(fmaf(y[c][i], fs, 0.5f)), __saturatef(fmaf(y[c][i + 1], fs, 0.5f)));
               const float2 gg = __ffma2_rz(f2, make_float2(kCellSpan, kCellSpan), make_float2(8388608.0f, 8388608.0f));
               const uint32_t e0 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gg.x));
               const uint32_t e1 = __shfl_sync(0xffffffffu, cell_entry, __float_as_int(gg.y));
@@ -503,15 +511,15 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
               uint32_t c0 = 0u, c1 = 0u;
 #pragma unroll
               for (int k = 0; k < NB; ++k) {
-                c0 += y[0][i] * inv > tsm[k] ? 1u : 0u;
-                c1 += y[0][i + 1] * inv > tsm[k] ? 1u : 0u;
+                c0 += y[c][i] * inv > tsm[k] ? 1u : 0u;
+                c1 += y[c][i + 1] * inv > tsm[k] ? 1u : 0u;
               }
               code[0] = c0; code[1] = c1;
             }
             // unit-scale residual r = u - c[code] and its fp16 hi + lo parts (the A operand)
             const float ch0 = __shfl_sync(0xffffffffu, ccen, static_cast<int>(code[0]));
             const float ch1 = __shfl_sync(0xffffffffu, ccen, static_cast<int>(code[1]));
-            const float2 rr = __ffma2_rn(make_float2(y[0][i], y[0][i + 1]), make_float2(inv, inv), make_float2(-ch0, -ch1));
+            const float2 rr = __ffma2_rn(make_float2(y[c][i], y[c][i + 1]), make_float2(inv, inv), make_float2(-ch0, -ch1));
             g2 = __ffma2_rn(rr, rr, g2);
             // hi = half2(r), lo = half2(r - hi): one paired conversion each, one packed FMA
             const __half2 h2 = __floats2half2_rn(rr.x, rr.y);
@@ -539,13 +547,13 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           p.rnorms[v] = sqrtf(g2.x + g2.y);
         }
         // sign bits of the projection, (S r)_i >= 0
-        if (!mbar_wait(zfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
+        if (!mbar_wait(zfull_bar(), it & 1, lim, p.status, abort_flag)) break;
         tc_fence_after();
         uint32_t sw[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float z[32];
-          tmem_ld32(taddr + 32 * c, z);
+          tmem_ld32(rowaddr + kZcol + 32 * c, z);
           tmem_wait_ld();
           uint32_t wbits = 0u;
 #pragma unroll
@@ -553,7 +561,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           sw[c] = wbits;
         }
         tc_fence_before();
-        mbar_arrive(tempty_bar(buf));                   // the accumulator is free again
+        mbar_arrive(zempty_bar());                      // Z is free for the next tile
         if (v < p.n) *reinterpret_cast<uint4*>(p.signs + v * 4) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
         continue;
       }

@@ -414,9 +414,9 @@ tq_status check_decode_shape(const tq_quantizer* kq, const tq_quantizer* vq, int
 
 // ---- wide vectors on the tensor cores (split-precision products, workspace) ----
 
-// fp32 input, d a multiple of 256 (<= 4096): MSE with 1..4 bits, or PROD with 2..5 bits and m = d.
+// fp32 input, d a multiple of 128 (<= 4096): MSE with 1..4 bits, or PROD with 2..5 bits and m = d.
 bool wide_supported(const tq_quantizer* q, int dtype) {
-  if (dtype != TQ_F32 || q->d < 256 || q->d % 256 || q->d > 4096) return false;
+  if (dtype != TQ_F32 || q->d < 128 || q->d % 128 || q->d > 4096) return false;
   if (q->kind == TQ_KIND_MSE) return q->bits >= 1 && q->bits <= 4;
   if (q->kind == TQ_KIND_PROD) return q->bits >= 2 && q->bits <= 5 && q->m == q->d && q->S;
   return false;
@@ -442,7 +442,7 @@ WidePlan plan_wide(const tq_quantizer* q, int64_t n) {
   P.rh = off; off = al(off + (m ? P.nb * d * 2 : 0));
   P.rl = off; off = al(off + (m ? P.nb * d * 2 : 0));
   P.nx = off; off = al(off + P.nb * 4);
-  P.r2 = off; off = al(off + P.nb * (d / 256) * 4);
+  P.r2 = off; off = al(off + P.nb * (d / gemm_tile_n(static_cast<int>(d))) * 4);
   P.bytes = off;
   return P;
 }
@@ -500,7 +500,7 @@ tq_status quantize_wide(const tq_quantizer* q, const float* x, int64_t n, tq_pac
     g.codes = out.codes + v0 * L.code_words; g.code_words = L.code_words;
     g.norms = out.norms + v0;
     if (prod) { g.r_hi = u16(P.rh); g.r_lo = u16(P.rl); g.r2_part = f32(P.r2); }
-    const int64_t work = (nb + 127) / 128 * (d / 256);
+    const int64_t work = (nb + 127) / 128 * (d / gemm_tile_n(d));
     const int grid = static_cast<int>(std::min<int64_t>(work, sm_count()));
     e = launch_split_gemm(maps, g, GEMM_EPI_QUANT, bmse, grid, stream);
     if (e != cudaSuccess) return cuda_fail(e, "wide rotation launch");
@@ -512,8 +512,8 @@ tq_status quantize_wide(const tq_quantizer* q, const float* x, int64_t n, tq_pac
     SplitGemmParams z{};
     z.M = nb; z.N = m; z.K = d; z.status = status; z.wait_limit = wait_limit();
     z.signs = out.signs + v0 * L.sign_words; z.rnorms = out.rnorms + v0;
-    z.r2_in = f32(P.r2); z.r2_chunks = d / 256;
-    const int64_t zwork = (nb + 127) / 128 * (m / 256);
+    z.r2_in = f32(P.r2); z.r2_chunks = d / gemm_tile_n(d);
+    const int64_t zwork = (nb + 127) / 128 * (m / gemm_tile_n(m));
     e = launch_split_gemm(maps, z, GEMM_EPI_SIGNS, 1, static_cast<int>(std::min<int64_t>(zwork, sm_count())), stream);
     if (e != cudaSuccess) return cuda_fail(e, "wide projection launch");
   }
@@ -882,11 +882,11 @@ static int score_qu_stride(const tq_quantizer* q) {
 }
 
 // Estimates on the tensor cores: MSE (1..4 bits) or PROD (2..5 bits, m = d) records with d a
-// multiple of 256, against at least 4096 records.  Queries [q' | S q'] and decoded records
+// multiple of 128, against at least 4096 records.  Queries [q' | S q'] and decoded records
 // [c[code] | sqrt(pi/2)/m gamma (2s - 1)] become split-precision operands of one product;
 // the column scale is the record norm.
 static bool score_wide(const tq_quantizer* q, int64_t n) {
-  if (q->d < 256 || q->d % 256 || q->d > 4096 || n < 4096 || std::getenv("TQ_FORCE_SIMT")) return false;
+  if (q->d < 128 || q->d % 128 || q->d > 4096 || n < 4096 || std::getenv("TQ_FORCE_SIMT")) return false;
   if (q->kind == TQ_KIND_MSE) return q->bits >= 1 && q->bits <= 4;
   if (q->kind == TQ_KIND_PROD) return q->bits >= 2 && q->bits <= 5 && q->m == q->d;
   return false;
@@ -1020,7 +1020,8 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
       SplitGemmParams g{};
       g.M = nb; g.N = static_cast<int>(n); g.K = P.K; g.status = device_status_ptr(); g.wait_limit = wait_limit();
       g.out = topk > 0 ? dense : scores + q0 * n; g.ldo = n; g.col_scale = keys.norms;
-      const int64_t work = (nb + 127) / 128 * ((n + 255) / 256);
+      const int64_t tn = gemm_tile_n(static_cast<int>(n));
+      const int64_t work = (nb + 127) / 128 * ((n + tn - 1) / tn);
       e = launch_split_gemm(maps, g, GEMM_EPI_SCORE, 1, static_cast<int>(std::min<int64_t>(work, sm_count())), stream);
       if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
       if (topk > 0) {

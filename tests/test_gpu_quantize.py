@@ -192,9 +192,10 @@ def test_quantize_spectral_parity(qjl):
 
 
 @pytest.mark.parametrize("d,kind,bits,n", [(1536, "prod", 2, 3000), (1536, "prod", 4, 1000), (256, "prod", 3, 777),
-                                           (1536, "mse", 3, 500), (512, "mse", 1, 129), (256, "prod", 5, 1)])
+                                           (1536, "mse", 3, 500), (512, "mse", 1, 129), (256, "prod", 5, 1),
+                                           (128, "mse", 3, 4096), (384, "prod", 3, 300), (128, "prod", 2, 257)])
 def test_quantize_wide_tensor_core_parity(d, kind, bits, n):
-    """tq_quantize_ws on fp32 vectors with d a multiple of 256: the rotation and the QJL
+    """tq_quantize_ws on fp32 vectors with d a multiple of 128: the rotation and the QJL
     projection as split-precision tensor-core products; records band-checked against the
     oracle (codes and signs), norms and residual norms to 1e-5."""
     from _parity import adopt_mse, adopt_prod
