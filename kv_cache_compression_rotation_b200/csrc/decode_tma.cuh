@@ -54,6 +54,7 @@ __host__ __device__ constexpr int tma_units(bool pk) { return pk ? TQ_DEC_PK_U :
 __host__ __device__ constexpr int tma_consumers(int kf, bool pk) { return kf == KFMT_PROD ? 7 : (pk ? TQ_DEC_PK_NC : 11); }
 __host__ __device__ constexpr int tma_stage_tokens(int kf, bool pk) { return tma_consumers(kf, pk) * 16 * tma_units(pk); }
 __host__ __device__ constexpr int tma_stages(bool pk) { return pk ? TQ_DEC_PK_NS : 4; }
+static_assert(TQ_DEC_PK_NS >= 2 && TQ_DEC_PK_NS <= 8, "decode ring depth");
 constexpr int kTmaHeadBlock = 8;     // query heads per work item (MMA N)
 
 __device__ __forceinline__ uint32_t tma_smem_u32(const void* p) {
@@ -267,16 +268,24 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     return a0;
   };
   const uint32_t miscA = place(tma_misc_bytes(KF, PK, VPR));
-  uint32_t stA[4] = {0u, 0u, 0u, 0u};
+  // equal-size stages: the first st_gap of them sit back to back in the gap, the rest back
+  // to back after the table
+  uint32_t st_first = 0u, st_after = 0u;
+  int st_gap = 0;
 #pragma unroll
-  for (int i = 0; i < NS; ++i) stA[i] = place(SL.bytes);
+  for (int i = 0; i < NS; ++i) {
+    const uint32_t a = place(SL.bytes);
+    if (i == 0) st_first = a;
+    if (a < tabA) ++st_gap;
+    else if (i == st_gap) st_after = a;
+  }
   if (after > base + dyn) {                       // the request did not cover this layout
     if (threadIdx.x == 0) report_status(status, TQ_ERR_UNSUPPORTED);
     return;
   }
   auto stage_addr = [&](int st) {
-    return NS == 3 ? (st == 0 ? stA[0] : (st == 1 ? stA[1] : stA[2]))
-                   : (st < 2 ? (st == 0 ? stA[0] : stA[1]) : (st == 2 ? stA[2] : stA[3]));
+    return st < st_gap ? st_first + static_cast<uint32_t>(st) * SL.bytes
+                       : st_after + static_cast<uint32_t>(st - st_gap) * SL.bytes;
   };
   auto gen = [&](uint32_t a) { return tsm_ + (a - base); };   // generic pointer of a shared address
   uint32_t* tab_g = reinterpret_cast<uint32_t*>(gen(tabA));

@@ -254,12 +254,14 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * NS + 2 + b); };
-  // prod: R of group b written (count 128), Z committed (1), Z read (count 128); Y uses the
-  // tfull / tempty pair of buffer 0 as its single full / empty barrier
+  // prod: R of group b written (count 128), Z of group b's tile committed (1), Z read
+  // (count 128).  Y is one buffer: its full barrier is the group's tfull (each group waits
+  // only for its own tiles, so a parity wait never passes on a phase of the other group),
+  // its empty barrier tempty(0), waited in tile order by the MMA warp alone.
   auto rfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 4 + b); };
-  auto zfull_bar = [&]() { return bar0 + 8u * (2 * NS + 6); };
-  auto zempty_bar = [&]() { return bar0 + 8u * (2 * NS + 7); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + (PRODK ? 8 : 4));
+  auto zfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 6 + b); };
+  auto zempty_bar = [&]() { return bar0 + 8u * (2 * NS + 8); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + (PRODK ? 10 : 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tsm = reinterpret_cast<float*>(tmem_slot + 2);   // boundaries [NB]
   // spectral: thresholds [top dim][64], centroids [top dim][64], S [64]
@@ -327,8 +329,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
     for (int s = 0; s < NS; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), 128); }
     if (PRODK) {
-      for (int b = 0; b < 2; ++b) mbar_init(rfull_bar(b), 128);
-      mbar_init(zfull_bar(), 1);
+      for (int b = 0; b < 2; ++b) { mbar_init(rfull_bar(b), 128); mbar_init(zfull_bar(b), 1); }
       mbar_init(zempty_bar(), 128);
     }
     *abort_flag = 0;
@@ -387,7 +388,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           umma_f16_ts(zd, ra + kk * 8, sw128_desc(s_lo + boff), zidesc, 1u);
           umma_f16_ts(zd, ra + 64 + kk * 8, sw128_desc(s_hi + boff), zidesc, 1u);
         }
-        umma_commit(zfull_bar());
+        umma_commit(zfull_bar(zb));
         ++zt;
         return true;
       };
@@ -410,7 +411,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           if (NT == 3) umma_f16(td, sw128_desc(xa + koff), sw128_desc(pi_lo2 + poff), idesc, 1u);
         }
         umma_commit(empty_bar(s));
-        umma_commit(tfull_bar(buf));
+        umma_commit(tfull_bar(PRODK ? (it & 1) : buf));
         ++it;
         // the previous tile's projection, issued behind this tile's rotation
         if (PRODK && it > 1 && !(zok = issue_z())) break;
@@ -419,11 +420,10 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       // wait for the tensor core to finish everything issued before TMEM is freed
       if (it > 0) {
         const int last = it - 1;
-        const int lb = PRODK ? 0 : (last & 1), lp = PRODK ? (last & 1) : ((last >> 1) & 1);
-        for (long long i = 0; !mbar_try(tfull_bar(lb), lp) && i < kDrainLimit; ++i) {}
+        for (long long i = 0; !mbar_try(tfull_bar(last & 1), (last >> 1) & 1) && i < kDrainLimit; ++i) {}
       }
       if (PRODK && zt > 0)
-        for (long long i = 0; !mbar_try(zfull_bar(), (zt - 1) & 1) && i < kDrainLimit; ++i) {}
+        for (long long i = 0; !mbar_try(zfull_bar((zt - 1) & 1), ((zt - 1) >> 1) & 1) && i < kDrainLimit; ++i) {}
     }
   } else {
     const int grp = (warp - 2) >> 2;                   // 0: warps 2-5, 1: warps 6-9
@@ -459,8 +459,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
       const int buf = it & 1;
       if (buf != grp) continue;
       const int j = it >> 1;
-      // prod: the single Y accumulator completes once per tile
-      if (!mbar_wait(tfull_bar(PRODK ? 0 : buf), PRODK ? (it & 1) : (j & 1), lim, p.status, abort_flag)) break;
+      if (!mbar_wait(tfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lanebase) << 16) + (PRODK ? 0u : buf * 128u);
       const int64_t v = tile * kUmmaTileRows + r;
@@ -547,7 +546,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           p.rnorms[v] = sqrtf(g2.x + g2.y);
         }
         // sign bits of the projection, (S r)_i >= 0
-        if (!mbar_wait(zfull_bar(), it & 1, lim, p.status, abort_flag)) break;
+        if (!mbar_wait(zfull_bar(buf), j & 1, lim, p.status, abort_flag)) break;
         tc_fence_after();
         uint32_t sw[4];
 #pragma unroll

@@ -478,11 +478,12 @@ tq_status quantize_wide(const tq_quantizer* q, const float* x, int64_t n, tq_pac
   if (e != cudaSuccess) return cuda_fail(e, "split launch");
   CUtensorMap pimaps[2], smaps[2];
   tq_status s;
-  if ((s = bf16_map(&pimaps[0], u16(P.pi), d, d, 256)) != TQ_OK) return s;
-  if ((s = bf16_map(&pimaps[1], u16(P.pi) + static_cast<size_t>(d) * d, d, d, 256)) != TQ_OK) return s;
+  // B operands: one box is one column tile of the product (the kernel's B stage)
+  if ((s = bf16_map(&pimaps[0], u16(P.pi), d, d, gemm_tile_n(d))) != TQ_OK) return s;
+  if ((s = bf16_map(&pimaps[1], u16(P.pi) + static_cast<size_t>(d) * d, d, d, gemm_tile_n(d))) != TQ_OK) return s;
   if (prod) {
-    if ((s = bf16_map(&smaps[0], u16(P.s), m, d, 256)) != TQ_OK) return s;
-    if ((s = bf16_map(&smaps[1], u16(P.s) + static_cast<size_t>(m) * d, m, d, 256)) != TQ_OK) return s;
+    if ((s = bf16_map(&smaps[0], u16(P.s), m, d, gemm_tile_n(m))) != TQ_OK) return s;
+    if ((s = bf16_map(&smaps[1], u16(P.s) + static_cast<size_t>(m) * d, m, d, gemm_tile_n(m))) != TQ_OK) return s;
   }
   int* status = device_status_ptr();
   for (int64_t v0 = 0; v0 < n; v0 += P.nb) {
@@ -1008,8 +1009,9 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
                               d, m, bm, u16(P.bh), u16(P.bl), stream);
     if (e != cudaSuccess) return cuda_fail(e, "record expansion launch");
     CUtensorMap maps[4];
-    if ((s = bf16_map(&maps[2], u16(P.bh), n, P.K, 256)) != TQ_OK) return s;
-    if ((s = bf16_map(&maps[3], u16(P.bl), n, P.K, 256)) != TQ_OK) return s;
+    const int tn = gemm_tile_n(static_cast<int>(n));      // B box = one column tile
+    if ((s = bf16_map(&maps[2], u16(P.bh), n, P.K, tn)) != TQ_OK) return s;
+    if ((s = bf16_map(&maps[3], u16(P.bl), n, P.K, tn)) != TQ_OK) return s;
     float* dense = reinterpret_cast<float*>(ws + P.dense);
     for (int64_t q0 = 0; q0 < nq; q0 += P.qb) {
       const int64_t nb = std::min(P.qb, nq - q0);
@@ -1020,7 +1022,6 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
       SplitGemmParams g{};
       g.M = nb; g.N = static_cast<int>(n); g.K = P.K; g.status = device_status_ptr(); g.wait_limit = wait_limit();
       g.out = topk > 0 ? dense : scores + q0 * n; g.ldo = n; g.col_scale = keys.norms;
-      const int64_t tn = gemm_tile_n(static_cast<int>(n));
       const int64_t work = (nb + 127) / 128 * ((n + tn - 1) / tn);
       e = launch_split_gemm(maps, g, GEMM_EPI_SCORE, 1, static_cast<int>(std::min<int64_t>(work, sm_count())), stream);
       if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
