@@ -316,13 +316,16 @@ tq_status tq_decode_attn_split_workspace(const tq_split* ks, const tq_split* vs,
 /*
  * DEVICE.  One decode-attention step over split caches (keys split by ks, values by vs;
  * the splits may differ but have the same width d):
- *   logit_i = scale * sum_g ||k_i,g|| <rot_g q[cols_g], c_g[code_i,g]>,  p = softmax(logit),
+ *   logit_i = scale * sum_g est_g(q[cols_g], k_i,g),  p = softmax(logit),
  *   out[cols_g] = rot_g^T sum_i p_i ||v_i,g|| c_g[code_i,g]   for every value group g,
+ * where est_g is the group's estimate: ||k|| <rot_g q', c_g[code]> for an MSE group, plus
+ * ||k|| sqrt(pi/2)/m ||r|| <S_g rot_g q', 2s - 1> for a PROD group (TurboQuant review,
+ * Method: the outlier and non-outlier channels are independent instances),
  * over the first seq_lens[b] records of each (b, kv-head) row; query head h reads KV head
  * h / (Hq/Hkv).  q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), kcache/vcache
  * host arrays of one packed descriptor per group, each group's records laid out
- * [B][Hkv][Nmax]; out [B*Hq*d] fp32.  libtq runs MSE groups, d <= 256 and
- * Hq/Hkv <= 8 on CUDA cores (TQ_ERR_UNSUPPORTED otherwise).  A value channel index out of
+ * [B][Hkv][Nmax]; out [B*Hq*d] fp32.  libtq runs MSE or PROD key groups, MSE value
+ * groups, d <= 256 and Hq/Hkv <= 8 (TQ_ERR_UNSUPPORTED otherwise).  A value channel index out of
  * range sets TQ_ERR_INVALID_ARG on the device and its output is not written.
  */
 tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const void* q,

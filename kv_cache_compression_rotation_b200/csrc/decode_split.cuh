@@ -13,7 +13,9 @@
 // warp per token at a time, lanes over the concatenated rotated coordinates, online
 // softmax in the log2 domain, and the per-warp P.V accumulators in shared memory;
 // split_combine_kernel merges the chunks and applies each value group's Pi_g^T,
-// scattering to the group's channels.  MSE groups only.
+// scattering to the group's channels.  Key groups are MSE or PROD instances: a PROD group
+// adds its QJL term sqrt(pi/2)/m_g ||r|| <S_g Pi_g q[cols_g], 2s - 1> to the group's
+// estimate (times ||k_g||); value groups are MSE.
 #pragma once
 
 #include "device_common.cuh"
@@ -35,6 +37,12 @@ struct SplitDecodeParams {
   const float* knorms[TQ_MAX_GROUPS];
   const float* kcent[TQ_MAX_GROUPS];
   const float* qr[TQ_MAX_GROUPS];      // [B*Hq][kd[g]]: Pi_g q[cols_g]
+  // PROD key groups (km = 0 for MSE): kbits is the MSE stage's width (0: no codes)
+  int km[TQ_MAX_GROUPS], ksw[TQ_MAX_GROUPS], kuoff[TQ_MAX_GROUPS], mu;   // mu = sum of km
+  const uint32_t* ksigns[TQ_MAX_GROUPS];
+  const float* krnorms[TQ_MAX_GROUPS];
+  const float* qu[TQ_MAX_GROUPS];      // [B*Hq][km[g]]: S_g Pi_g q[cols_g]
+  float kcoef[TQ_MAX_GROUPS];          // sqrt(pi/2) / m_g
   int vd[TQ_MAX_GROUPS], vbits[TQ_MAX_GROUPS], vwords[TQ_MAX_GROUPS], voff[TQ_MAX_GROUPS];
   const uint32_t* vcodes[TQ_MAX_GROUPS];
   const float* vnorms[TQ_MAX_GROUPS];
@@ -45,9 +53,10 @@ struct SplitDecodeParams {
 };
 
 // Shared memory (floats): q'[G][d] | key codebooks [4][256] | value codebooks [4][256] |
-// per-warp max [4][G], sum [4][G] | per-warp P.V [4][G][d]
-__host__ __device__ inline size_t split_decode_smem(int G, int d) {
-  return (static_cast<size_t>(G) * d + 2 * TQ_MAX_GROUPS * 256 + 2 * 4 * G + 4 * static_cast<size_t>(G) * d) * 4;
+// per-warp max [4][G], sum [4][G] | per-warp P.V [4][G][d] | S q'[G][mu] (PROD key groups)
+__host__ __device__ inline size_t split_decode_smem(int G, int d, int mu = 0) {
+  return (static_cast<size_t>(G) * d + 2 * TQ_MAX_GROUPS * 256 + 2 * 4 * G + 4 * static_cast<size_t>(G) * d +
+          static_cast<size_t>(G) * mu) * 4;
 }
 
 __global__ void __launch_bounds__(kSplitDecThreads) split_decode_kernel(const SplitDecodeParams p) {
@@ -59,6 +68,7 @@ __global__ void __launch_bounds__(kSplitDecThreads) split_decode_kernel(const Sp
   float* wm = cbv + TQ_MAX_GROUPS * 256;
   float* wl = wm + 4 * G;
   float* wo = wl + 4 * G;
+  float* su = wo + 4 * G * d;
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.Hkv, hk = bh - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -71,9 +81,16 @@ __global__ void __launch_bounds__(kSplitDecThreads) split_decode_kernel(const Sp
       if (j >= p.koff[g] && j < p.koff[g] + p.kd[g]) v = p.qr[g][(row0 + h) * p.kd[g] + (j - p.koff[g])];
     sq[i] = v;
   }
+  for (int i = tid; i < G * p.mu; i += kSplitDecThreads) {
+    const int h = i / p.mu, j = i - h * p.mu;
+    float v = 0.f;
+    for (int g = 0; g < p.nkg; ++g)
+      if (p.km[g] && j >= p.kuoff[g] && j < p.kuoff[g] + p.km[g]) v = p.qu[g][(row0 + h) * p.km[g] + (j - p.kuoff[g])];
+    su[i] = v;
+  }
   for (int i = tid; i < TQ_MAX_GROUPS * 256; i += kSplitDecThreads) {
     const int g = i >> 8, e = i & 255;
-    cbk[i] = (g < p.nkg && e < (1 << p.kbits[g])) ? p.kcent[g][e] : 0.f;
+    cbk[i] = (g < p.nkg && p.kbits[g] > 0 && e < (1 << p.kbits[g])) ? p.kcent[g][e] : 0.f;
     cbv[i] = (g < p.nvg && e < (1 << p.vbits[g])) ? p.vcent[g][e] : 0.f;
   }
   for (int i = tid; i < 4 * G * d; i += kSplitDecThreads) wo[i] = 0.f;
@@ -91,14 +108,28 @@ __global__ void __launch_bounds__(kSplitDecThreads) split_decode_kernel(const Sp
 #pragma unroll
     for (int h = 0; h < kSplitMaxG; ++h) s[h] = 0.f;
     for (int g = 0; g < p.nkg; ++g) {
-      const uint32_t* w = p.kcodes[g] + rec * p.kwords[g];
       const float nk = p.knorms[g][rec];
-      for (int jj = lane; jj < p.kd[g]; jj += 32) {
-        const float c = nk * cbk[g * 256 + stream_bits(w, jj * p.kbits[g], p.kbits[g])];
-        const int j = p.koff[g] + jj;
+      if (p.kbits[g] > 0) {
+        const uint32_t* w = p.kcodes[g] + rec * p.kwords[g];
+        for (int jj = lane; jj < p.kd[g]; jj += 32) {
+          const float c = nk * cbk[g * 256 + stream_bits(w, jj * p.kbits[g], p.kbits[g])];
+          const int j = p.koff[g] + jj;
 #pragma unroll
-        for (int h = 0; h < kSplitMaxG; ++h)
-          if (h < G) s[h] = fmaf(sq[h * d + j], c, s[h]);
+          for (int h = 0; h < kSplitMaxG; ++h)
+            if (h < G) s[h] = fmaf(sq[h * d + j], c, s[h]);
+        }
+      }
+      if (p.km[g]) {
+        // QJL term: ||k_g|| sqrt(pi/2)/m ||r|| sum_i (S q')_i (2 s_i - 1)
+        const uint32_t* sw = p.ksigns[g] + rec * p.ksw[g];
+        const float f = nk * p.kcoef[g] * p.krnorms[g][rec];
+        for (int i = lane; i < p.km[g]; i += 32) {
+          const float c = ((sw[i >> 5] >> (i & 31)) & 1u) ? f : -f;
+          const int j = p.kuoff[g] + i;
+#pragma unroll
+          for (int h = 0; h < kSplitMaxG; ++h)
+            if (h < G) s[h] = fmaf(su[h * p.mu + j], c, s[h]);
+        }
       }
     }
     float f[kSplitMaxG], pr[kSplitMaxG];

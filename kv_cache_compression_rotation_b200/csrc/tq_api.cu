@@ -1220,7 +1220,8 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
 // ---- decode attention over a split cache ----
 struct SplitDecodePlan {
   int chunk_len, n_chunks;
-  size_t off_qr[TQ_MAX_GROUPS], off_ml, off_o, bytes;
+  size_t off_qr[TQ_MAX_GROUPS], off_qu[TQ_MAX_GROUPS], off_ml, off_o, bytes;
+  int mu;                    // sum of the PROD key groups' m
 };
 
 static SplitDecodePlan plan_split_decode(const tq_split* ks, int B, int Hq, int64_t Nmax) {
@@ -1236,6 +1237,10 @@ static SplitDecodePlan plan_split_decode(const tq_split* ks, int B, int Hq, int6
   for (int g = 0; g < ks->n_groups; ++g) {
     P.off_qr[g] = b;
     b += (rows * ks->groups[g]->d * 4 + 255) / 256 * 256;
+    const int m = ks->groups[g]->kind == TQ_KIND_PROD ? ks->groups[g]->m : 0;
+    P.off_qu[g] = b;
+    b += (rows * m * 4 + 255) / 256 * 256;
+    P.mu += m;
   }
   P.off_ml = b;
   b += (rows * P.n_chunks * 2 * 4 + 255) / 256 * 256;
@@ -1252,7 +1257,8 @@ static tq_status check_split_decode(const tq_split* ks, const tq_split* vs, int 
   if (ks->d != vs->d) return fail(TQ_ERR_INVALID_ARG, "key and value splits have different widths");
   if (ks->d > kSplitMaxD) return fail(TQ_ERR_UNSUPPORTED, "split decode runs d <= %d", kSplitMaxD);
   for (int g = 0; g < ks->n_groups; ++g)
-    if (ks->groups[g]->kind != TQ_KIND_MSE) return fail(TQ_ERR_UNSUPPORTED, "split decode runs MSE key groups");
+    if (ks->groups[g]->kind != TQ_KIND_MSE && ks->groups[g]->kind != TQ_KIND_PROD)
+      return fail(TQ_ERR_UNSUPPORTED, "split decode runs MSE or PROD key groups");
   for (int g = 0; g < vs->n_groups; ++g)
     if (vs->groups[g]->kind != TQ_KIND_MSE) return fail(TQ_ERR_UNSUPPORTED, "split decode runs MSE value groups");
   if (B < 1 || Hq < 1 || Hkv < 1 || Nmax < 1) return fail(TQ_ERR_INVALID_ARG, "B, Hq, Hkv, Nmax must be >= 1");
@@ -1315,19 +1321,29 @@ tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const voi
   dp.chunk_len = P.chunk_len; dp.n_chunks = P.n_chunks; dp.seq_lens = seq_lens;
   dp.nkg = ks->n_groups; dp.nvg = vs->n_groups;
   cudaError_t e;
-  int off = 0;
+  int off = 0, uoff = 0;
   for (int g = 0; g < ks->n_groups; ++g) {
     const tq_quantizer* kq = ks->groups[g];
+    const bool prod = kq->kind == TQ_KIND_PROD;
     float* qr = reinterpret_cast<float*>(ws + P.off_qr[g]);
+    float* qu = prod ? reinterpret_cast<float*>(ws + P.off_qu[g]) : nullptr;
     score_qprep_kernel<<<static_cast<unsigned>(rows), 128, 2 * kq->d * 4, stream>>>(
-        q, dtype, kq->d, TQ_KIND_MSE, kq->rot, nullptr, 0, 0, qr, nullptr, 0, d, ks->cols[g], status);
+        q, dtype, kq->d, kq->kind, kq->rot, prod ? kq->S : nullptr, prod ? kq->m : 0, 0, qr, qu, prod ? kq->m : 0, d,
+        ks->cols[g], status);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split qprep launch");
     const tq_layout L = layout_of(kq);
-    dp.kd[g] = kq->d; dp.kbits[g] = kq->bits; dp.kwords[g] = L.code_words; dp.koff[g] = off;
+    dp.kd[g] = kq->d; dp.kbits[g] = prod ? kq->bits - 1 : kq->bits; dp.kwords[g] = L.code_words; dp.koff[g] = off;
     dp.kcodes[g] = kcache[g].codes; dp.knorms[g] = kcache[g].norms; dp.kcent[g] = kq->centroids;
     dp.qr[g] = qr;
+    if (prod) {
+      dp.km[g] = kq->m; dp.ksw[g] = L.sign_words; dp.kuoff[g] = uoff;
+      dp.ksigns[g] = kcache[g].signs; dp.krnorms[g] = kcache[g].rnorms; dp.qu[g] = qu;
+      dp.kcoef[g] = static_cast<float>(std::sqrt(M_PI / 2.0) / kq->m);
+      uoff += kq->m;
+    }
     off += kq->d;
   }
+  dp.mu = P.mu;
   off = 0;
   for (int g = 0; g < vs->n_groups; ++g) {
     const tq_quantizer* vq = vs->groups[g];
@@ -1339,7 +1355,8 @@ tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const voi
   dp.logit_scale = static_cast<float>(scale * kLog2e);
   dp.part_ml = reinterpret_cast<float*>(ws + P.off_ml);
   dp.part_o = reinterpret_cast<float*>(ws + P.off_o);
-  const size_t smem = split_decode_smem(G, d);
+  const size_t smem = split_decode_smem(G, d, P.mu);
+  if (smem > 227 * 1024) return fail(TQ_ERR_UNSUPPORTED, "split decode: shared memory for Hq/Hkv and widths too large");
   e = cudaFuncSetAttribute(split_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "split decode attribute");
   split_decode_kernel<<<dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv)), kSplitDecThreads,

@@ -135,26 +135,43 @@ def test_bad_channel_index_reports_status():
 
 
 def _records_from_gpu(packs, groups, ins):
-    """The GPU's own records as oracle record dicts (codes unpacked, fp32 norms)."""
+    """The GPU's own records as oracle record dicts (codes unpacked, fp32 norms; a PROD
+    group adds c[idx], its sign bits and its residual norms)."""
     recs = []
     for pk, ch, g in zip(packs, groups, ins):
-        idx = OQ.unpack_codes(as_u32(pk.codes), len(ch), g["bits"])
-        recs.append({"idx": idx, "norms": pk.norms.cpu().numpy().astype(np.float64)})
+        nrm = pk.norms.cpu().numpy().astype(np.float64)
+        if g["kind"] == "mse":
+            idx = OQ.unpack_codes(as_u32(pk.codes), len(ch), g["bits"])
+            recs.append({"idx": idx, "norms": nrm})
+        else:
+            idx = OQ.unpack_codes(as_u32(pk.codes), len(ch), g["bits"] - 1)
+            m = g["S"].shape[0]
+            recs.append({"idx": idx, "norms": nrm, "chat": np.asarray(g["centroids"], dtype=np.float64)[idx],
+                         "s": OQ.unpack_signs(as_u32(pk.signs), m),
+                         "rnorms": pk.rnorms.cpu().numpy().astype(np.float64)})
     return recs
 
 
-@pytest.mark.parametrize("B,Hkv,Hq,Nmax,lens", [(2, 2, 8, 700, [700, 333]), (1, 4, 8, 3000, [2999]),
-                                                 (3, 1, 1, 300, [1, 300, 17])])
-def test_decode_attn_split_parity(B, Hkv, Hq, Nmax, lens):
+@pytest.mark.parametrize("kkind,B,Hkv,Hq,Nmax,lens", [("mse", 2, 2, 8, 700, [700, 333]),
+                                                       ("mse", 1, 4, 8, 3000, [2999]),
+                                                       ("mse", 3, 1, 1, 300, [1, 300, 17]),
+                                                       ("prod", 2, 2, 8, 700, [700, 333]),
+                                                       ("prod", 1, 2, 4, 2100, [2100]),
+                                                       ("prod", 3, 1, 1, 300, [1, 300, 17])])
+def test_decode_attn_split_parity(kkind, B, Hkv, Hq, Nmax, lens):
     # the attention step read straight from split caches against the oracle's split
     # attention on the same records (keys with planted outlier channels, 32 @ 3 b + 96 @ 2 b
-    # for keys and values)
+    # MSE or TurboQuant-prod instances; values split the same way, MSE)
     n = B * Hkv * Nmax
-    kx, k64, groups, ins, ks = _setup("mse", n, 4700 + Nmax)
+    kx, k64, groups, kins, ks = _setup(kkind, n, 4700 + Nmax)
     vx64 = ti.iid_normal((n, D), 4800 + Nmax)
     vxt, vx64 = ti.to_bf16_f64(vx64)
     vx = vxt.cuda().contiguous()
-    vs = ks                                                # the same split for the values
+    if kkind == "mse":
+        vins, vs = kins, ks                                # the same split for the values
+    else:
+        _, _, vgroups, vins, vs = _setup("mse", 2000, 4750)
+        assert all(np.array_equal(a, b) for a, b in zip(groups, vgroups))
     kp = K.quantize_split(ks, kx)
     vp = K.quantize_split(vs, vx)
     q64 = ti.iid_normal((B, Hq, D), 4900 + Nmax)
@@ -163,15 +180,15 @@ def test_decode_attn_split_parity(B, Hkv, Hq, Nmax, lens):
     o = K.decode_attn_split(ks, vs, q, seq, kp, vp, Nmax, Hkv).cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
     assert K.get_status() == 0
-    kr, vr = _records_from_gpu(kp, groups, ins), _records_from_gpu(vp, groups, ins)
+    kr, vr = _records_from_gpu(kp, groups, kins), _records_from_gpu(vp, groups, vins)
 
     def rows(recs, b, h, n_):
         base = (b * Hkv + h) * Nmax
-        return [{"idx": r["idx"][base:base + n_], "norms": r["norms"][base:base + n_]} for r in recs]
+        return [{k: v[base:base + n_] for k, v in r.items()} for r in recs]
 
     scale = 1.0 / np.sqrt(D)
     ref = OA.decode_attention(q.cpu().numpy().astype(np.float64), lens, Hkv,
-                              lambda b, h, qs: OS.estimate_split(qs, rows(kr, b, h, lens[b]), groups, ins),
-                              lambda b, h, n_: OS.dequantize_split(rows(vr, b, h, n_), groups, ins, D), scale)
+                              lambda b, h, qs: OS.estimate_split(qs, rows(kr, b, h, lens[b]), groups, kins),
+                              lambda b, h, n_: OS.dequantize_split(rows(vr, b, h, n_), groups, vins, D), scale)
     err = rel_rows(o, ref)
     assert np.all(err <= 1e-3), f"max row error {err.max():.2e}"
