@@ -64,6 +64,10 @@ cudaError_t launch_expand_records(const uint32_t* codes, int code_words, const u
 // fp32 rows -> bf16 hi + lo parts (and row norms when norms != nullptr).
 cudaError_t launch_split_rows(const float* x, int64_t rows, int d, uint16_t* hi, uint16_t* lo, float* norms,
                               cudaStream_t s);
+// Split-cache decode on the tensor cores: two MSE groups per record, 32 rotated dims at 3
+// bits then 96 at 2 bits (keys and values), GQA groups of at most 4 heads.
+struct SplitMmaParams;
+cudaError_t launch_decode_split_mma(const SplitMmaParams& p, int grid, cudaStream_t s, int* status, long long lim);
 // TurboQuant-prod with m = d = 128: the rotation and the QJL projection on the tensor cores
 cudaError_t launch_umma_quantize_prod(const CUtensorMap& map, const UmmaQuantParams& p, int mse_bits, int grid,
                                       cudaStream_t s);

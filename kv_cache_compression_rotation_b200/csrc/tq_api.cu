@@ -16,6 +16,7 @@
 #include "decode.cuh"
 #include "decode_aux.cuh"
 #include "decode_split.cuh"
+#include "decode_split_mma.cuh"
 #include "decode_tma.cuh"
 #include "gemm_umma.cuh"
 #include "device_common.cuh"
@@ -1219,17 +1220,47 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
 
 // ---- decode attention over a split cache ----
 struct SplitDecodePlan {
+  bool fast;                 // the tensor-core kernel (decode_split_mma.cuh)
   int chunk_len, n_chunks;
   size_t off_qr[TQ_MAX_GROUPS], off_qu[TQ_MAX_GROUPS], off_ml, off_o, bytes;
   int mu;                    // sum of the PROD key groups' m
 };
 
-static SplitDecodePlan plan_split_decode(const tq_split* ks, int B, int Hq, int64_t Nmax) {
+// The tensor-core split decode takes the 2.5-bit outlier split of the KV experiments: two
+// MSE groups, 32 rotated dims at 3 bits then 96 at 2 bits, for keys and values alike;
+// GQA groups of at most 4 heads; rows of a multiple of 4 records (16-byte aligned copies).
+static bool split_mma_ok(const tq_split* ks, const tq_split* vs, int G, int64_t Nmax) {
+  auto shape = [](const tq_split* s) {
+    return s->d == 128 && s->n_groups == 2 && s->groups[0]->kind == TQ_KIND_MSE &&
+           s->groups[1]->kind == TQ_KIND_MSE && s->groups[0]->d == 32 && s->groups[0]->bits == 3 &&
+           s->groups[1]->d == 96 && s->groups[1]->bits == 2;
+  };
+  return shape(ks) && shape(vs) && G <= 4 && Nmax % 4 == 0;
+}
+
+static SplitDecodePlan plan_split_decode(const tq_split* ks, const tq_split* vs, int B, int Hq, int Hkv,
+                                         int64_t Nmax) {
   SplitDecodePlan P{};
-  // at most 64 chunks per row: the partials stay small and the combine's weights fit in
-  // shared memory; chunks of at least 256 tokens
-  int64_t cl = (Nmax + 63) / 64;
-  cl = std::max<int64_t>(256, (cl + 31) / 32 * 32);
+  P.fast = split_mma_ok(ks, vs, Hq / Hkv, Nmax);
+  int64_t cl;
+  if (P.fast) {
+    // persistent kernel: chunks of whole 256-token stages, ~16 items per SM at most and
+    // items of at least ~4 stages, an item count that is a multiple of the SMs when the
+    // shape allows (as the packed-cache decode plans its work)
+    const int64_t stage = kSmStage, sms = sm_count(), wu = static_cast<int64_t>(B) * Hkv;
+    const int64_t stages_total = wu * ((Nmax + stage - 1) / stage);
+    const int64_t want = std::max<int64_t>(sms, std::min<int64_t>(16 * sms, stages_total / 4));
+    int64_t n0 = std::max<int64_t>(1, (want + wu - 1) / wu);
+    for (int64_t cand = n0; cand < n0 + 8 && cand <= Nmax; ++cand)
+      if ((wu * cand) % sms == 0) { n0 = cand; break; }
+    cl = (Nmax + n0 - 1) / n0;
+    cl = std::max<int64_t>(stage, (cl + stage - 1) / stage * stage);
+  } else {
+    // at most 64 chunks per row: the partials stay small and the combine's weights fit in
+    // shared memory; chunks of at least 256 tokens
+    cl = (Nmax + 63) / 64;
+    cl = std::max<int64_t>(256, (cl + 31) / 32 * 32);
+  }
   P.chunk_len = static_cast<int>(std::min<int64_t>(cl, 1 << 30));
   P.n_chunks = static_cast<int>((Nmax + P.chunk_len - 1) / P.chunk_len);
   const size_t rows = static_cast<size_t>(B) * Hq;
@@ -1274,7 +1305,7 @@ tq_status tq_decode_attn_split_workspace(const tq_split* ks, const tq_split* vs,
   tq_status s = check_split_decode(ks, vs, B, Hq, Hkv, Nmax);
   if (s != TQ_OK) return s;
   if (!bytes) return fail(TQ_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = plan_split_decode(ks, B, Hq, Nmax).bytes;
+  *bytes = plan_split_decode(ks, vs, B, Hq, Hkv, Nmax).bytes;
   return TQ_OK;
 }
 
@@ -1289,7 +1320,7 @@ tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const voi
   if (!q || !seq_lens || !out || !kcache || !vcache) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
   if (!aligned16(q) || !aligned16(seq_lens) || !aligned16(out)) return fail(TQ_ERR_ALIGNMENT, "q/seq_lens/out alignment");
   if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
-  const SplitDecodePlan P = plan_split_decode(ks, B, Hq, Nmax);
+  const SplitDecodePlan P = plan_split_decode(ks, vs, B, Hq, Hkv, Nmax);
   if (!workspace || ws_bytes < P.bytes) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", P.bytes);
   if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
   const int64_t recs = static_cast<int64_t>(B) * Hkv * Nmax;
@@ -1355,13 +1386,34 @@ tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const voi
   dp.logit_scale = static_cast<float>(scale * kLog2e);
   dp.part_ml = reinterpret_cast<float*>(ws + P.off_ml);
   dp.part_o = reinterpret_cast<float*>(ws + P.off_o);
-  const size_t smem = split_decode_smem(G, d, P.mu);
-  if (smem > 227 * 1024) return fail(TQ_ERR_UNSUPPORTED, "split decode: shared memory for Hq/Hkv and widths too large");
-  e = cudaFuncSetAttribute(split_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return cuda_fail(e, "split decode attribute");
-  split_decode_kernel<<<dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv)), kSplitDecThreads,
-                        smem, stream>>>(dp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split decode launch");
+  if (P.fast) {
+    SplitMmaParams mp{};
+    mp.B = B; mp.Hq = Hq; mp.Hkv = Hkv; mp.G = G; mp.Nmax = Nmax;
+    mp.chunk_len = P.chunk_len; mp.n_chunks = P.n_chunks; mp.seq_lens = seq_lens;
+    for (int g = 0; g < 2; ++g) {
+      mp.kc[g] = kcache[g].codes; mp.kn[g] = kcache[g].norms;
+      mp.vc[g] = vcache[g].codes; mp.vn[g] = vcache[g].norms;
+      mp.kcent[g] = ks->groups[g]->centroids; mp.vcent[g] = vs->groups[g]->centroids;
+      mp.kscale[g] = ks->groups[g]->lut_scale > 0.f ? ks->groups[g]->lut_scale : 1.f;
+      mp.vscale[g] = vs->groups[g]->lut_scale > 0.f ? vs->groups[g]->lut_scale : 1.f;
+      mp.qr[g] = dp.qr[g];
+    }
+    mp.logit_scale = dp.logit_scale;
+    mp.part_ml = dp.part_ml;
+    mp.part_o = dp.part_o;
+    const int64_t items = static_cast<int64_t>(B) * Hkv * P.n_chunks;
+    const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
+    e = launch_decode_split_mma(mp, grid, stream, status, wait_limit());
+    if (e != cudaSuccess) return cuda_fail(e, "split decode launch");
+  } else {
+    const size_t smem = split_decode_smem(G, d, P.mu);
+    if (smem > 227 * 1024) return fail(TQ_ERR_UNSUPPORTED, "split decode: shared memory for Hq/Hkv and widths too large");
+    e = cudaFuncSetAttribute(split_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "split decode attribute");
+    split_decode_kernel<<<dim3(static_cast<unsigned>(P.n_chunks), static_cast<unsigned>(B * Hkv)), kSplitDecThreads,
+                          smem, stream>>>(dp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split decode launch");
+  }
 
   SplitCombineParams cp{};
   cp.rows = rows; cp.d = d; cp.n_chunks = P.n_chunks; cp.nvg = vs->n_groups;

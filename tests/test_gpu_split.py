@@ -152,9 +152,14 @@ def _records_from_gpu(packs, groups, ins):
     return recs
 
 
+# MSE splits with GQA groups of at most 4 heads and rows of a multiple of 4 records take the
+# tensor-core kernel; 8 heads per group or an odd row length the CUDA-core one
 @pytest.mark.parametrize("kkind,B,Hkv,Hq,Nmax,lens", [("mse", 2, 2, 8, 700, [700, 333]),
                                                        ("mse", 1, 4, 8, 3000, [2999]),
                                                        ("mse", 3, 1, 1, 300, [1, 300, 17]),
+                                                       ("mse", 2, 4, 16, 4100, [4100, 2055]),
+                                                       ("mse", 1, 2, 6, 1028, [1027]),
+                                                       ("mse", 1, 1, 8, 501, [501]),
                                                        ("prod", 2, 2, 8, 700, [700, 333]),
                                                        ("prod", 1, 2, 4, 2100, [2100]),
                                                        ("prod", 3, 1, 1, 300, [1, 300, 17])])

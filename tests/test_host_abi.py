@@ -270,12 +270,14 @@ def test_split_decode_validation_before_launch(lib):
     ws = C.c_size_t(0)
     assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp), 2, 8, 2, 1000, C.byref(ws)) == 0
     assert ws.value >= 2 * 8 * 128 * 4                               # at least the rotated queries
-    # GQA group too large, Hq not a multiple of Hkv, a prod group, mismatched widths
+    # GQA group too large, Hq not a multiple of Hkv, a prod value group (prod key groups
+    # are taken), mismatched widths
     assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp), 1, 16, 1, 1000, C.byref(ws)) == 2
     assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp), 1, 6, 4, 1000, C.byref(ws)) == 1
     qp = _q(T.KIND_PROD, d=96, bits=3, m=96, S=FAKE)
     spp = _split([qa, qp], [FAKE, FAKE], 128)
-    assert lib.tq_decode_attn_split_workspace(C.byref(spp), C.byref(sp), 1, 8, 1, 1000, C.byref(ws)) == 2
+    assert lib.tq_decode_attn_split_workspace(C.byref(spp), C.byref(sp), 1, 8, 1, 1000, C.byref(ws)) == 0
+    assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(spp), 1, 8, 1, 1000, C.byref(ws)) == 2
     q64 = _q(T.KIND_MSE, d=64, bits=2)
     sp96 = _split([qa, q64], [FAKE, FAKE], 96)
     assert lib.tq_decode_attn_split_workspace(C.byref(sp), C.byref(sp96), 1, 8, 1, 1000, C.byref(ws)) == 1
