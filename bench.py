@@ -573,16 +573,36 @@ def run_other(args):
         seqd = torch.full((Bd,), Nd, dtype=torch.int32, device=dev)
         td = _timed(lambda: K.decode_attn_split(sp, sp, qd, seqd, out, out, Nd, Hkvd), stream, flush)
         assert K.get_status() == 0
+        # and at the 128k decode shapes: B=8, Hkv=8, Hq=32, context 131072 (738 MB of split
+        # K and V records)
+        Bb, Nb = 8, 131072
+        nb = Bb * Hkvd * Nb
+        xb = ti.normal_torch((nb, Dm), ti.SEEDS["keys"] + 8, dev)
+        xb[:, torch.from_numpy(planted).to(dev)] *= 6.0
+        xb = xb.to(torch.bfloat16).contiguous()
+        outb = sp.alloc(nb, dev)
+        K.quantize_split(sp, xb, outb)
+        del xb
+        qb = ti.normal_torch((Bb, Hqd, Dm), ti.SEEDS["queries"] + 8, dev)
+        seqb = torch.full((Bb,), Nb, dtype=torch.int32, device=dev)
+        tb = _timed(lambda: K.decode_attn_split(sp, sp, qb, seqb, outb, outb, Nb, Hkvd), stream, flush)
+        assert K.get_status() == 0
         rec = sum(4 * (L.code_words + L.has_norms) for L in (g.layout() for g in groups))
         parts = {"quantize_split": {"ms": tq, "vectors_per_s": n / tq * 1e3, "gbs": n * (Dm * 2 + rec) / tq / 1e6,
                                     "record_bytes": rec},
                  "score_split": {"ms": ts, "estimates_per_s": nq * n / ts * 1e3,
                                  "gbs": n * rec / ts / 1e6},
                  "decode_attn_split": {"ms": td, "gbs": n * 2 * rec / td / 1e6,
-                                       "frac": n * 2 * rec / td / 1e6 / peak, "bytes_per_token": 2 * rec}}
+                                       "frac": n * 2 * rec / td / 1e6 / peak, "bytes_per_token": 2 * rec,
+                                       "shape": "B=1 Hkv=8 Hq=32, 32768 tokens"},
+                 "decode_attn_split_128k": {"ms": tb, "gbs": nb * 2 * rec / tb / 1e6,
+                                            "frac": nb * 2 * rec / tb / 1e6 / peak, "bytes_per_token": 2 * rec,
+                                            "shape": "B=8 Hkv=8 Hq=32, 131072 tokens",
+                                            "note": "tq_decode_attn_split = 2 query preps + tensor-core decode + "
+                                                    "combine with the per-group inverse rotations"}}
         desc = (f"outlier split: {n} bf16 keys d=128 with 32 planted channels (x6), groups 32 @ 3 bits + "
-                f"96 @ 2 bits (mse), dense estimates for {nq} queries, decode B=1 Hkv=8 Hq=32 over 32768 "
-                f"tokens (CUDA-core kernels)")
+                f"96 @ 2 bits (mse), dense estimates for {nq} queries (CUDA cores), decode over split K and V "
+                f"caches (tensor cores) at B=1 x 32768 and B=8 x 131072 tokens, Hkv=8, Hq=32")
         value, unit, step_ms = n / tq * 1e3, "vectors/s", tq
     elif wl == "serving":
         # serving forms at the 128k decode shapes: one decode step over a paged pool with the

@@ -64,6 +64,10 @@ cudaError_t launch_expand_records(const uint32_t* codes, int code_words, const u
 // fp32 rows -> bf16 hi + lo parts (and row norms when norms != nullptr).
 cudaError_t launch_split_rows(const float* x, int64_t rows, int d, uint16_t* hi, uint16_t* lo, float* norms,
                               cudaStream_t s);
+// Outlier split (32 channels at b0 bits + 96 at b1 bits, (3, 2) or (4, 3)) as one
+// tensor-core pass over 16-bit rows of 128 channels.
+cudaError_t launch_umma_quantize_split(const CUtensorMap& map, const UmmaQuantParams& p, int b0, int b1, int grid,
+                                       cudaStream_t s);
 // Split-cache decode on the tensor cores: two MSE groups per record, 32 rotated dims at 3
 // bits then 96 at 2 bits (keys and values), GQA groups of at most 4 heads.
 struct SplitMmaParams;

@@ -5,9 +5,9 @@
 namespace tq {
 namespace {
 
-template <int B, bool SPEC = false, bool PRODK = false>
+template <int B, bool SPEC = false, bool PRODK = false, int B1 = 0>
 cudaError_t go(const CUtensorMap& map, const UmmaQuantParams& p, int grid, cudaStream_t s) {
-  auto k = umma_quantize_kernel<B, SPEC, PRODK>;
+  auto k = umma_quantize_kernel<B, SPEC, PRODK, B1>;
   const uint32_t smem = PRODK ? kUmmaProdSmemBytes : kUmmaSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -38,6 +38,13 @@ cudaError_t launch_umma_quantize_prod(const CUtensorMap& map, const UmmaQuantPar
     case 4: return go<4, false, true>(map, p, grid, s);
     default: return cudaErrorNotSupported;
   }
+}
+
+cudaError_t launch_umma_quantize_split(const CUtensorMap& map, const UmmaQuantParams& p, int b0, int b1, int grid,
+                                       cudaStream_t s) {
+  if (b0 == 3 && b1 == 2) return go<3, false, false, 2>(map, p, grid, s);
+  if (b0 == 4 && b1 == 3) return go<4, false, false, 3>(map, p, grid, s);
+  return cudaErrorNotSupported;
 }
 
 }  // namespace tq

@@ -84,6 +84,15 @@ struct UmmaQuantParams {
   // prod (m = 128): S [128*128] fp32 is the field S above; MSE-stage centroids, sign words
   const float* centroids;  // [2^B]
   uint32_t* signs;         // [n][4]
+  // outlier split (B1 instantiation): rot is Pi_0 [32*32] of the channels cols0, rot1 Pi_1
+  // [96*96] of cols1; group 0 records (B bits) go to codes / norms, group 1 (B1 bits) to
+  // codes1 / norms1
+  const float* rot1;
+  const int32_t* cols0;
+  const int32_t* cols1;
+  const float* boundaries1;
+  uint32_t* codes1;        // [n][3 * B1]
+  float* norms1;           // [n]
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -223,7 +232,12 @@ __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B
 // tail dims take 1 bit, code (z_j > 0) (the 1-bit standard-normal boundary is 0); the top
 // dims are coded against sigma_j times their unit codebooks and get the QJL signs of
 // S (z_top - c_top); record = head word + 4 tail words (+ ||z_top - c_top||).
-template <int B, bool SPEC, bool PRODK = false>
+// B1 > 0: the outlier-channel split of the KV experiments (TurboQuant review, Method) as
+// one pass over the full 128-channel rows: the operand is the block rotation whose rows
+// 0..31 are Pi_0 scattered over the channels cols0 and rows 32..127 Pi_1 over cols1, so
+// Y = [Pi_0 x[cols0] | Pi_1 x[cols1]] (the zero entries add nothing); each group is then
+// coded with its own norm ||y_g|| = ||x[cols_g]||, boundaries and width (B, then B1 bits).
+template <int B, bool SPEC, bool PRODK = false, int B1 = 0>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
 umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantParams p) {
   constexpr int K = 1 << B;
@@ -273,10 +287,36 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (p.n + kUmmaTileRows - 1) / kUmmaTileRows;
 
+  // split: the block rotation is zero outside the scattered group rows
+  if constexpr (B1 > 0) {
+    for (int i = tid; i < static_cast<int>(2 * kPiBytes / 4); i += kUmmaThreads) reinterpret_cast<uint32_t*>(sm)[i] = 0u;
+    __syncthreads();
+  }
   // Pi_hi / Pi_lo in the swizzled K-major layout: row = output dim n, k = input dim.
-  for (int i = tid; i < kUmmaD * kUmmaD; i += kUmmaThreads) {
-    const int nrow = i >> 7, k = i & 127;
-    float v = __ldg(p.rot + i);
+  for (int i = tid; i < (B1 > 0 ? 32 * 32 + 96 * 96 : kUmmaD * kUmmaD); i += kUmmaThreads) {
+    int nrow = i >> 7, k = i & 127;
+    float v;
+    if constexpr (B1 > 0) {
+      // row r of Pi_0 (first 1024 entries) or of Pi_1, entry j -> channel cols_g[j]
+      int j, col;
+      if (i < 32 * 32) {
+        nrow = i >> 5; j = i & 31;
+        col = __ldg(p.cols0 + j);
+        v = __ldg(p.rot + i);
+      } else {
+        const int i2 = i - 32 * 32, r = i2 / 96;
+        nrow = 32 + r; j = i2 - r * 96;
+        col = __ldg(p.cols1 + j);
+        v = __ldg(p.rot1 + i2);
+      }
+      if (col < 0 || col >= kUmmaD) {           // a channel out of range contributes nothing
+        report_status(p.status, TQ_ERR_INVALID_ARG);
+        continue;
+      }
+      k = col;
+    } else {
+      v = __ldg(p.rot + i);
+    }
     if (p.pm1) {
       // the +-1 pattern is exact in both 16-bit types; the scale is applied to the norm
       if (fabsf(v) != p.pm1_scale) report_status(p.status, TQ_ERR_INVALID_ARG);
@@ -310,6 +350,7 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
     if (p.qjl && tid < p.k_top * p.k_top) sS[tid] = __ldg(p.S + tid);
   } else {
     if (tid < NB) tsm[tid] = __ldg(p.boundaries + tid);
+    if (B1 > 0 && tid < (1 << B1) - 1) sthr[tid] = __ldg(p.boundaries1 + tid);
   }
   if constexpr (PRODK) {
     // S_hi / S_lo (fp16) in the same swizzled K-major layout: row = projection i, k = dim
@@ -620,6 +661,63 @@ umma_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const UmmaQuantPa
           dst[1] = tail[0]; dst[2] = tail[1]; dst[3] = tail[2]; dst[4] = tail[3];
           if (p.qjl) p.rnorms[v] = sqrtf(g2);
         }
+        continue;
+      }
+      if constexpr (B1 > 0) {
+        // split: group 0 = chunk 0 (B bits), group 1 = chunks 1..3 (B1 bits), each coded
+        // against its own norm times its boundaries (unnormalized coordinates)
+        constexpr int NB1 = (1 << B1) - 1;
+        float y[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, y[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(tempty_bar(buf));
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s0[i & 3] = fmaf(y[0][i], y[0][i], s0[i & 3]);
+#pragma unroll
+        for (int c = 1; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s1[i & 3] = fmaf(y[c][i], y[c][i], s1[i & 3]);
+        const float n0 = sqrtf((s0[0] + s0[1]) + (s0[2] + s0[3])), n1 = sqrtf((s1[0] + s1[1]) + (s1[2] + s1[3]));
+        float th0[NB], th1[NB1];
+#pragma unroll
+        for (int k = 0; k < NB; ++k) th0[k] = (n0 > 0.f ? n0 : 1.f) * tsm[k];   // a zero group codes u = 0
+#pragma unroll
+        for (int k = 0; k < NB1; ++k) th1[k] = (n1 > 0.f ? n1 : 1.f) * sthr[k];
+        {
+          uint32_t wc[B];
+#pragma unroll
+          for (int w = 0; w < B; ++w) wc[w] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            uint32_t cnt = 0u;
+#pragma unroll
+            for (int k = 0; k < NB; ++k) cnt += y[0][i] > th0[k] ? 1u : 0u;
+            const int pos = i * B;
+            wc[pos >> 5] |= cnt << (pos & 31);
+            if ((pos & 31) + B > 32) wc[(pos >> 5) + 1] |= cnt >> (32 - (pos & 31));
+          }
+          if (v < p.n) store_words<B>(p.codes + v * B, wc);
+        }
+#pragma unroll
+        for (int c = 1; c < 4; ++c) {
+          uint32_t wc[B1];
+#pragma unroll
+          for (int w = 0; w < B1; ++w) wc[w] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            uint32_t cnt = 0u;
+#pragma unroll
+            for (int k = 0; k < NB1; ++k) cnt += y[c][i] > th1[k] ? 1u : 0u;
+            const int pos = i * B1;
+            wc[pos >> 5] |= cnt << (pos & 31);
+            if ((pos & 31) + B1 > 32) wc[(pos >> 5) + 1] |= cnt >> (32 - (pos & 31));
+          }
+          if (v < p.n) store_words<B1>(p.codes1 + v * (3 * B1) + (c - 1) * B1, wc);
+        }
+        if (v < p.n) { p.norms[v] = n0; p.norms1[v] = n1; }
         continue;
       }
       uint32_t* dst = p.codes + v * W;

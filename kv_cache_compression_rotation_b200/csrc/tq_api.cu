@@ -1088,6 +1088,60 @@ static tq_status check_split(const tq_split* sp) {
   return TQ_OK;
 }
 
+// The outlier split of the KV experiments on the tensor cores: two MSE groups, 32 channels
+// at 3 bits + 96 at 2 (or 4 + 3), 16-bit rows of 128 channels.
+static bool umma_split(const tq_split* sp, int dtype, int64_t n) {
+  if (sp->d != 128 || sp->n_groups != 2) return false;
+  const tq_quantizer* a = sp->groups[0];
+  const tq_quantizer* b = sp->groups[1];
+  if (a->kind != TQ_KIND_MSE || b->kind != TQ_KIND_MSE || a->d != 32 || b->d != 96) return false;
+  if (!((a->bits == 3 && b->bits == 2) || (a->bits == 4 && b->bits == 3))) return false;
+  tq_quantizer probe = *a;                        // the hardware and size checks of the d = 128 path
+  probe.d = 128;
+  probe.bits = 2;
+  return umma_supported(&probe, dtype, n);
+}
+
+static tq_status quantize_split_umma(const tq_split* sp, const void* x, int dtype, int64_t n, const tq_packed* out,
+                                     cudaStream_t stream) {
+  tq_status s;
+  const tq_layout L0 = layout_of(sp->groups[0]), L1 = layout_of(sp->groups[1]);
+  if ((s = check_packed(out[0], L0)) != TQ_OK) return s;
+  if ((s = check_packed(out[1], L1)) != TQ_OK) return s;
+  if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
+  if (!aligned16(x)) return fail(TQ_ERR_ALIGNMENT, "x is not 16-byte aligned");
+  Range outs[8];
+  packed_ranges(out[0], L0, n, outs);
+  packed_ranges(out[1], L1, n, outs + 4);
+  const Range ins[1] = {{x, static_cast<size_t>(n) * 128 * dtype_size(dtype)}};
+  if ((s = check_no_alias(outs, 8, ins, 1)) != TQ_OK) return s;     // and the groups' outputs pairwise
+  auto encode = get_encode();
+  CUtensorMap map;
+  const cuuint64_t gdim[2] = {128, static_cast<cuuint64_t>(n)};
+  const cuuint64_t gstride[1] = {256};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(&map, dtype == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                            2, const_cast<void*>(x), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  UmmaQuantParams p{};
+  p.rot = sp->groups[0]->rot; p.rot1 = sp->groups[1]->rot;
+  p.cols0 = sp->cols[0]; p.cols1 = sp->cols[1];
+  p.boundaries = sp->groups[0]->boundaries; p.boundaries1 = sp->groups[1]->boundaries;
+  p.n = n;
+  p.is_f16 = dtype == TQ_F16;
+  p.codes = out[0].codes; p.norms = out[0].norms;
+  p.codes1 = out[1].codes; p.norms1 = out[1].norms;
+  p.status = device_status_ptr();
+  p.wait_limit = wait_limit();
+  const int64_t tiles = (n + 127) / 128;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
+  const cudaError_t e = launch_umma_quantize_split(map, p, sp->groups[0]->bits, sp->groups[1]->bits, grid, stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "split quantize launch");
+}
+
 tq_status tq_quantize_split(const tq_split* sp, const void* x, int32_t dtype, int64_t n, const tq_packed* out,
                             tq_stream stream) {
   tq_status s = check_split(sp);
@@ -1095,6 +1149,8 @@ tq_status tq_quantize_split(const tq_split* sp, const void* x, int32_t dtype, in
   if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
   if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
   if (n == 0) return TQ_OK;
+  if (dtype < TQ_F32 || dtype > TQ_F16) return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+  if (umma_split(sp, dtype, n)) return quantize_split_umma(sp, x, dtype, n, out, reinterpret_cast<cudaStream_t>(stream));
   // every group's outputs must be disjoint from the other groups' (checked as inputs)
   Range others[4 * TQ_MAX_GROUPS];
   for (int g = 0; g < sp->n_groups; ++g) {

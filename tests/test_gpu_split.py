@@ -25,8 +25,11 @@ D = 128
 PLANTED = np.sort(np.random.Generator(np.random.PCG64(77)).choice(D, 32, replace=False))
 
 
-def _setup(kind, n, seed, dtype="bf16"):
+def _setup(kind, n, seed, dtype="bf16", bits=(3, 2), zero_rows=False):
     x = ti.planted_outliers(n, D, PLANTED, 6.0, seed)
+    if zero_rows:
+        x[3] = 0.0                                      # a zero row
+        x[5, PLANTED] = 0.0                             # a row whose outlier group is zero
     if dtype == "bf16":
         xt, x64 = ti.to_bf16_f64(x)
     else:
@@ -34,7 +37,6 @@ def _setup(kind, n, seed, dtype="bf16"):
         xt, x64 = torch.from_numpy(x32), x32.astype(np.float64)
     groups = OS.split_groups(D, OS.outlier_channels(x64, 32))
     assert np.array_equal(groups[0], PLANTED)
-    bits = [3, 2]
     ins, qs = [], []
     for g, (ch, b) in enumerate(zip(groups, bits)):
         dg = len(ch)
@@ -54,9 +56,13 @@ def _setup(kind, n, seed, dtype="bf16"):
     return xt.cuda().contiguous(), x64, groups, ins, sp
 
 
-@pytest.mark.parametrize("kind,n,dtype", [("mse", 3000, "bf16"), ("mse", 777, "f32"), ("prod", 1500, "bf16")])
-def test_quantize_split_parity(kind, n, dtype):
-    x, x64, groups, ins, sp = _setup(kind, n, 4300 + n, dtype)
+# 16-bit MSE splits of 32 @ 3 + 96 @ 2 or 32 @ 4 + 96 @ 3 bits take the tensor-core pass over
+# whole rows; fp32 rows and prod groups the CUDA-core kernel with the gather on the load
+@pytest.mark.parametrize("kind,n,dtype,bits", [("mse", 3000, "bf16", (3, 2)), ("mse", 777, "f32", (3, 2)),
+                                               ("prod", 1500, "bf16", (3, 2)), ("mse", 1500, "bf16", (4, 3)),
+                                               ("mse", 129, "bf16", (3, 2))])
+def test_quantize_split_parity(kind, n, dtype, bits):
+    x, x64, groups, ins, sp = _setup(kind, n, 4300 + n, dtype, bits, zero_rows=True)
     out = K.quantize_split(sp, x)
     torch.cuda.synchronize()
     assert K.get_status() == 0
@@ -78,10 +84,10 @@ def test_quantize_split_parity(kind, n, dtype):
 
 
 def test_quantize_split_equals_gathered_single_instances():
-    # the split call writes exactly what the single-instance call writes for the gathered
-    # rows (same kernel, gather on the load)
+    # on the CUDA-core path (fp32 rows) the split call writes exactly what the single-instance
+    # call writes for the gathered rows (same kernel, gather on the load)
     n = 1000
-    x, x64, groups, ins, sp = _setup("mse", n, 4400)
+    x, x64, groups, ins, sp = _setup("mse", n, 4400, "f32")
     out = K.quantize_split(sp, x)
     for g, ch in enumerate(groups):
         xg = x[:, torch.from_numpy(np.asarray(ch)).cuda()].contiguous().float()
