@@ -4,10 +4,11 @@
 // (decode.cuh): logit = scale * est(q, k_i), online softmax, o' = sum p ||v|| c[code_v].
 //
 // Streaming.  Persistent CTAs (one per SM) walk work items (batch * kv-head, head block,
-// context chunk).  One producer warp copies each item in stages of 16 tokens per consumer warp with
-// cp.async.bulk (key codes, value codes, norms; prod adds sign words and residual norms)
-// into a 4-deep shared-memory ring; 11 (prod: 7) consumer warps each take 16 tokens of a stage,
-// pull their record slices into registers, release the stage and compute.
+// context chunk).  One producer warp copies each item in stages of 16 tokens per consumer
+// warp and unit with cp.async.bulk (key codes, value codes, norms; prod adds sign words and
+// residual norms) into a shared-memory ring (2 or 4 deep, see the work split below); 11
+// (prod: 7) consumer warps each take one or two 16-token units of a stage, pull their record
+// slices into registers, release the stage and compute.
 //
 // Math per 16-token unit, all on mma.sync m16n8k16 (fp16 in, fp32 accumulate):
 //   scores  S[16 tokens x 8 columns] = K_hat[16 x 128] . Q'^T     (A = table-decoded keys)
@@ -38,17 +39,18 @@
 namespace tq {
 
 // Work split.  With packed columns (GQA groups of at most 4 heads) every consumer warp takes
-// two 16-token units of a stage (8 consumer warps, 3 stages of 256 tokens); otherwise one
-// unit (11 consumer warps for MSE keys, 4 stages).  PROD keys need more registers and run
+// two 16-token units of a stage (11 consumer warps, 2 stages of 352 tokens: more warps to
+// interleave measured faster than a deeper ring, 8 warps x 3 stages of 256 tokens); otherwise
+// one unit (11 consumer warps for MSE keys, 4 stages).  PROD keys need more registers and run
 // 7 consumer warps.  Plus one producer warp.
 #ifndef TQ_DEC_PK_NC
-#define TQ_DEC_PK_NC 8
+#define TQ_DEC_PK_NC 11
 #endif
 #ifndef TQ_DEC_PK_U
 #define TQ_DEC_PK_U 2
 #endif
 #ifndef TQ_DEC_PK_NS
-#define TQ_DEC_PK_NS 3
+#define TQ_DEC_PK_NS 2
 #endif
 __host__ __device__ constexpr int tma_units(bool pk) { return pk ? TQ_DEC_PK_U : 1; }
 __host__ __device__ constexpr int tma_consumers(int kf, bool pk) { return kf == KFMT_PROD ? 7 : (pk ? TQ_DEC_PK_NC : 11); }
