@@ -20,6 +20,12 @@
 // Table decoding: one 32-bit shared load turns a pair of codes into half2 codebook values
 // (table replicated per lane, so a warp's 32 loads hit 32 banks; the table sits at a
 // 64 KB-aligned shared address, so one byte permute of the code word is the address).
+// 1-bit codes (TurboQuant-mse b=1, the MSE stage of b=2 prod, spectral 1-bit tails) take
+// a whole byte per lookup instead: one 128-bit load returns 8 decoded values, the A
+// registers of two key k-steps (the byte holds 8 consecutive dims of one token), or all
+// four A registers of a value M-tile (the byte holds one dim of the 4 tokens of the lane's
+// two rows, bit-transposed per unit); those entries keep 8 lane slots of 16 bytes, which a
+// 128-bit load of 32 lanes reads in four conflict-free passes.
 // Precision: the query operand and P are split hi + lo (one accumulator), table entries
 // are c / s with a searched shared scale s (see tq_lut_scale).
 // Token order inside a unit: score rows r and r + 8 hold tokens tau(r) and 8 + tau(r), with
@@ -131,7 +137,8 @@ __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int k
 // (merge buffer, sign table, barriers) and as many stages as fit go into the gap below
 // the table, the rest after it; the kernel checks the layout against the allocation.
 __host__ __device__ inline uint32_t tma_table_bytes(int kb, int vb) {
-  return (1u << (2 * (kb > vb ? kb : vb))) * 256u;
+  // 1-bit codes index the table by whole bytes
+  return (kb == 1 || vb == 1) ? 65536u : (1u << (2 * (kb > vb ? kb : vb))) * 256u;
 }
 __host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u : 8u; }
 __host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk, bool vpr = false) {
@@ -165,6 +172,12 @@ __device__ __forceinline__ uint32_t sld32(uint32_t a) {
   return v;
 }
 __device__ __forceinline__ float sldf(uint32_t a) { return __uint_as_float(sld32(a)); }
+// 128-bit table load (1-bit entries).
+__device__ __forceinline__ uint4 tab_ld128(uint32_t addr) {
+  uint4 v;
+  asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
 
 // Slice of NW words of a record in shared memory starting at word w0 (aligned slices).
 template <int NW>
@@ -247,7 +260,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int HB = PK ? 4 : kTmaHeadBlock;            // query heads per work item
   constexpr int RW = static_cast<int>(tma_merge_rows(PK));   // merge rows per warp
   constexpr int CONSUMERS = NC * 32;
-  constexpr int NE = KLUT > VLUT ? KLUT : VLUT;        // table entries
+  constexpr int NE = (KB == 1 || VB == 1) ? 256 : (KLUT > VLUT ? KLUT : VLUT);   // table entries
   constexpr uint32_t TAB = static_cast<uint32_t>(NE) * 256u;
   extern __shared__ __align__(128) unsigned char tsm_[];
 
@@ -344,13 +357,25 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int i = tid; i < NE * 64; i += kTmaThreads) {
-    const int e = i >> 6;
+    const int e = i >> 6, j = i & 3;               // j: word of a 16-byte slot (1-bit entries)
     uint32_t val = 0u;
     if ((i & 32) == 0) {
-      if (e < KLUT)
+      if constexpr (KB == 1) {
+        // byte e = codes of 8 consecutive dims: word j holds dims 2j, 2j + 1
+        val = pack_half2(__ldg(p.kc + ((e >> (2 * j)) & 1)) / p.k_scale,
+                         __ldg(p.kc + ((e >> (2 * j + 1)) & 1)) / p.k_scale);
+      } else if (e < KLUT) {
         val = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) / p.k_scale, __ldg(p.kc + (e >> KB)) / p.k_scale);
-    } else if (e < VLUT) {
-      val = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
+      }
+    } else {
+      if constexpr (VB == 1) {
+        // byte e: bits 0-3 = one dim of the lane's 4 tokens (row g), bits 4-7 = row g + 8;
+        // words = A registers a0 (row g, tokens 0, 1), a1 (row g + 8), a2 (row g, tokens 2, 3), a3
+        const int b = (j == 0) ? 0 : (j == 1) ? 4 : (j == 2) ? 2 : 6;
+        val = pack_half2(__ldg(p.vc + ((e >> b) & 1)) / p.v_scale, __ldg(p.vc + ((e >> (b + 1)) & 1)) / p.v_scale);
+      } else if (e < VLUT) {
+        val = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
+      }
     }
     tab_g[i] = val;
   }
@@ -513,6 +538,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   // value-operand k-indices 2t, 2t+1, 2t+8, 2t+9 are the tokens of score rows 2t, 2t+1, ...
   const int kv[4] = {t, t ^ 5, 8 + t, 8 + (t ^ 5)};
   const uint32_t klo = tabA | static_cast<uint32_t>(lane) * 4u, vlo = klo + 128u;
+  // 16-byte slots of the 1-bit entries: 8 per half row
+  const uint32_t k1lo = tabA | (static_cast<uint32_t>(lane & 7) << 4), v1lo = k1lo + 128u;
   // MMA column of this lane's B operand (g) and of its accumulators (2t, 2t + 1)
   const int qcol = PK ? (g & 3) : g;               // head (in the block) of B column g
   const bool qlo = PK && g >= 4;                  // B column g carries a lo part
@@ -740,10 +767,24 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       for (int u = 0; u < U; ++u) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, accb[4] = {0.f, 0.f, 0.f, 0.f};
         float accl[4] = {0.f, 0.f, 0.f, 0.f}, acclb[4] = {0.f, 0.f, 0.f, 0.f};
+        // 1-bit keys: byte j of a row's 32-dim slice decodes k-steps 2j and 2j + 1 at once
+        uint32_t kq[KB == 1 ? 2 : 1][KB == 1 ? KST : 1][2];
+        if constexpr (KB == 1) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < KST / 2; ++j) {
+              const uint4 r = tab_ld128(__byte_perm(ks[u][h][0], k1lo, 0x7604u | (static_cast<uint32_t>(j) << 4)));
+              kq[h][2 * j][0] = r.x; kq[h][2 * j][1] = r.y;
+              kq[h][2 * j + 1][0] = r.z; kq[h][2 * j + 1][1] = r.w;
+            }
+        }
 #pragma unroll
         for (int k = 0; k < KST; ++k) {
           uint32_t a0, a1, a2, a3;
-          if constexpr (KB == 4) {
+          if constexpr (KB == 1) {
+            a0 = kq[0][k][0]; a1 = kq[1][k][0]; a2 = kq[0][k][1]; a3 = kq[1][k][1];
+          } else if constexpr (KB == 4) {
             // dims (4 k, 4 k + 1) are byte 2 (k % 2) of word k / 2; (+2, +3) the next byte
             const uint32_t w0c = ks[u][0][k >> 1], w1c = ks[u][1][k >> 1];
             const int bsel = 2 * (k & 1);
@@ -979,6 +1020,23 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             const uint32_t a3 = tab_ld(tab_off((i & 1) ? hi[1][1] : lo[1][1], vlo, k));
             mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
             if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
+          }
+        } else if constexpr (VB == 1) {
+          // bit-transpose the 4 tokens' 16-dim slices: byte i of zl (i < 4) / zh holds dim i
+          // (bits 0-3, one per token) and dim 8 + i (bits 4-7) of the M-tile's two rows
+          auto spread4 = [](uint32_t x) { return (x * 0x00204081u) & 0x01010101u; };   // bit k -> 8k
+          uint32_t zl = 0u, zh = 0u;
+#pragma unroll
+          for (int tau = 0; tau < 4; ++tau) {
+            const uint32_t sv = vs[u][tau][0];
+            zl |= (spread4(sv & 15u) << tau) | (spread4((sv >> 8) & 15u) << (4 + tau));
+            zh |= (spread4((sv >> 4) & 15u) << tau) | (spread4((sv >> 12) & 15u) << (4 + tau));
+          }
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const uint4 r = tab_ld128(__byte_perm(i < 4 ? zl : zh, v1lo, 0x7604u | (static_cast<uint32_t>(i & 3) << 4)));
+            mma16816(o[i], r.x, r.y, r.z, r.w, b0h, b1h);
+            if constexpr (!PK) mma16816(o[i], r.x, r.y, r.z, r.w, b0l, b1l);
           }
         } else {
 #pragma unroll

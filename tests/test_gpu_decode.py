@@ -91,6 +91,9 @@ DECODE_CASES = [
     ("g16", 1, 32, 2, 900, [900], "mse", 3, 2),
     ("one-token", 3, 8, 2, 64, [1, 2, 64], "mse", 4, 4),
     ("bits1", 1, 8, 2, 1000, [999], "mse", 1, 1),
+    ("bits1-g8", 1, 16, 2, 700, [700], "mse", 1, 1),
+    ("bits4-1", 2, 8, 2, 900, [900, 451], "mse", 4, 1),
+    ("bits1-3", 1, 8, 2, 800, [800], "mse", 1, 3),
     ("bits2-4", 2, 8, 2, 800, [800, 17], "mse", 2, 4),
     ("prod2", 1, 8, 2, 1500, [1500], "prod", 2, 4),
     ("prod5", 1, 8, 2, 600, [600], "prod", 5, 3),
