@@ -28,9 +28,9 @@
 //   3 bits  one 6-bit pair -> half2: 64 entries of 256 bytes (32 lane slots each side)
 //
 // Streaming is that of decode_tma_kernel: persistent CTAs over (batch * kv-head, context
-// chunk) items, a producer warp copying 256-token stages (the four record arrays and four
-// norm arrays) into a 3-deep ring with bulk copies, 8 consumer warps of two 16-token units
-// each, mma.sync m16n8k16 with packed hi / lo query columns (GQA groups of at most 4 heads),
+// chunk) items, a producer warp copying stages of 32 tokens per consumer warp (the four
+// record arrays and four norm arrays) into a ring with bulk copies, consumer warps of two
+// 16-token units each, mma.sync m16n8k16 with packed hi / lo query columns (GQA groups of at most 4 heads),
 // an online softmax in the log2 domain, and a cross-warp merge per item into chunk partials
 // that split_combine_kernel merges (with each value group's Pi_g^T and channel scatter).
 // Every wait is bounded (TQ_ERR_TIMEOUT); a CTA that times out drains its copies.
@@ -40,9 +40,18 @@
 
 namespace tq {
 
-constexpr int kSmNC = 8;                          // consumer warps
+// 11 consumer warps and the producer: 3 warps per scheduler (measured faster than 8 or 10
+// consumer warps with a 3-deep ring)
+#ifndef TQ_SPLIT_NC
+#define TQ_SPLIT_NC 11
+#endif
+#ifndef TQ_SPLIT_NS
+#define TQ_SPLIT_NS 2
+#endif
+constexpr int kSmNC = TQ_SPLIT_NC;                // consumer warps
 constexpr int kSmU = 2;                           // 16-token units per consumer warp and stage
-constexpr int kSmNS = 3;                          // ring stages
+constexpr int kSmNS = TQ_SPLIT_NS;                // ring stages
+static_assert(kSmNS >= 2 && kSmNS <= 4, "split decode ring depth");
 constexpr int kSmStage = kSmNC * 16 * kSmU;       // tokens per stage
 constexpr int kSmThreads = (kSmNC + 1) * 32;
 constexpr int kSmRows = 4;                        // query heads per item (packed columns)
