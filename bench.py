@@ -583,6 +583,7 @@ def run_other(args):
         outb = sp.alloc(nb, dev)
         K.quantize_split(sp, xb, outb)
         del xb
+        torch.cuda.empty_cache()
         qb = ti.normal_torch((Bb, Hqd, Dm), ti.SEEDS["queries"] + 8, dev)
         seqb = torch.full((Bb,), Nb, dtype=torch.int32, device=dev)
         tb = _timed(lambda: K.decode_attn_split(sp, sp, qb, seqb, outb, outb, Nb, Hkvd), stream, flush)

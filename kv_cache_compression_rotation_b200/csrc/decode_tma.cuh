@@ -144,7 +144,7 @@ __host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u 
 __host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk, bool vpr = false) {
   const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf, pk)) * tma_merge_rows(pk) * (128u + 2u) * 4u;
   // values as prod: the merged sign-domain sums of up to 8 rows
-  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u + 510u * 4u + 8u + (vpr ? 8u * 128u * 4u : 0u);
+  const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u + 1024u * 4u + 8u + (vpr ? 8u * 128u * 4u : 0u);
   return (v + 127u) & ~127u;
 }
 // words of one record: the code stream, plus the head word of a spectral record
@@ -313,8 +313,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   int* nb_off = nb_count + NS;                              // [NS] their offset in the stage
   volatile int* abort_flag = nb_off + NS;
   volatile int* consumers_stop = abort_flag + 1;   // uniform exit decision of the consumer warps
-  float* utab = reinterpret_cast<float*>(const_cast<int*>(consumers_stop) + 2);   // spectral unit codebooks [510]
-  float* asum = utab + 510;                        // values as prod: merged sign-domain sums [8][128]
+  // spectral unit codebooks [512]: the 510 entries, then zeros (the entry of a dim with no
+  // top code); for values the same divided by the value table scale
+  float* utab = reinterpret_cast<float*>(const_cast<int*>(consumers_stop) + 2);
+  float* utabv = utab + 512;
+  float* asum = utabv + 512;                       // values as prod: merged sign-domain sums [8][128]
   const uint32_t bar0 = tma_smem_u32(bars);
   const uint32_t nb_a = tma_smem_u32(nb_count);
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
@@ -384,7 +387,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     luts[tid] = pack_half2((e & 1) ? 1.f : -1.f, (e & 2) ? 1.f : -1.f);
   }
   if constexpr (SP)
-    for (int i = tid; i < 510; i += kTmaThreads) utab[i] = __ldg(p.unit_c + i);
+    for (int i = tid; i < 512; i += kTmaThreads) {
+      const float c = i < 510 ? __ldg(p.unit_c + i) : 0.f;
+      utab[i] = c;
+      utabv[i] = c / p.v_scale;
+    }
   __syncthreads();
   pdl_trigger();   // the chunk combine may launch; it waits for this grid to complete
 
@@ -547,9 +554,13 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   const bool plo = PK && t >= 2;                  // accumulator columns 2t, 2t + 1 are lo parts
   // spectral head words: this lane scores top dims 2t, 2t + 1 and QJL signs 2t, 2t + 1 of its
   // key rows, and carries top value dim g (bit position, width, codebook offset; 0 = none)
-  int kh_pos[2] = {0, 0}, kh_nb[2] = {0, 0}, kh_off[2] = {0, 0}, ks_pos[2] = {0, 0};
-  bool ks_ok[2] = {false, false};
-  int vh_pos = 0, vh_nb = 0, vh_off = 0;
+  // (branch-free: a dim without a top code reads the zero entry with an empty mask, a sign
+  // outside the QJL dims is scaled by 0)
+  int kh_pos[2] = {0, 0}, kh_nb[2] = {0, 0}, kh_off[2] = {510, 510}, ks_pos[2] = {0, 0};
+  uint32_t kh_mask[2] = {0u, 0u};
+  float ks_f[2] = {0.f, 0.f};
+  int vh_pos = 0, vh_nb = 0, vh_off = 510;
+  uint32_t vh_mask = 0u;
   if constexpr (SP) {
     // static indices only (a dynamically indexed array would live in local memory)
     int acc = 0;
@@ -562,9 +573,10 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      kh_off[i] = kh_nb[i] ? unit_c_off(kh_nb[i]) : 0;
+      kh_off[i] = kh_nb[i] ? unit_c_off(kh_nb[i]) : 510;
+      kh_mask[i] = kh_nb[i] ? (1u << kh_nb[i]) - 1u : 0u;
       ks_pos[i] = acc + 2 * t + i;
-      ks_ok[i] = p.k_qjl && 2 * t + i < p.k_top_k;
+      ks_f[i] = (p.k_qjl && 2 * t + i < p.k_top_k) ? 1.f : 0.f;
     }
     acc = 0;
 #pragma unroll
@@ -573,7 +585,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       if (j == g) { vh_pos = acc; vh_nb = b; }
       acc += b;
     }
-    vh_off = vh_nb ? unit_c_off(vh_nb) : 0;
+    vh_off = vh_nb ? unit_c_off(vh_nb) : 510;
+    vh_mask = vh_nb ? (1u << vh_nb) - 1u : 0u;
   }
   // the prepared queries come from the kernel before this one (the producer's copies of the
   // cache do not depend on it and are already under way)
@@ -829,8 +842,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             const uint32_t w = hk[u][h];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-              hvv[h][i] = kh_nb[i] ? utab[kh_off[i] + ((w >> kh_pos[i]) & ((1u << kh_nb[i]) - 1u))] : 0.f;
-              hvv[h][2 + i] = ks_ok[i] ? (((w >> ks_pos[i]) & 1u) ? gm[u][h] : -gm[u][h]) : 0.f;
+              hvv[h][i] = utab[kh_off[i] + ((w >> kh_pos[i]) & kh_mask[i])];
+              hvv[h][2 + i] = (((w >> ks_pos[i]) & 1u) ? gm[u][h] : -gm[u][h]) * ks_f[i];
             }
           }
           uint32_t ah[4], al[4];
@@ -946,7 +959,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           float tv4[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            tv4[i] = vh_nb ? utab[vh_off + ((hv[u][i] >> vh_pos) & ((1u << vh_nb) - 1u))] / p.v_scale : 0.f;
+            tv4[i] = utabv[vh_off + ((hv[u][i] >> vh_pos) & vh_mask)];
           uint32_t vh0, vl0, vh2, vl2;
           split_pair(tv4[0], tv4[1], vh0, vl0);
           split_pair(tv4[2], tv4[3], vh2, vl2);
