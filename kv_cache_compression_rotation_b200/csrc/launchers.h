@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "tq.h"
+
 namespace tq {
 
 // Launch `k` with programmatic stream serialization: it may start (and run what precedes
@@ -68,6 +70,26 @@ cudaError_t launch_split_rows(const float* x, int64_t rows, int d, uint16_t* hi,
 // tensor-core pass over 16-bit rows of 128 channels.
 cudaError_t launch_umma_quantize_split(const CUtensorMap& map, const UmmaQuantParams& p, int b0, int b1, int grid,
                                        cudaStream_t s);
+// Operands of the tensor-core estimator over outlier-split records: per group the rotated
+// (and S-projected, PROD) queries and the records, concatenated along K (see score_split_tc.cu).
+struct SplitScoreGroups {
+  int n;                                   // groups
+  int d[TQ_MAX_GROUPS], m[TQ_MAX_GROUPS];  // MSE-part and QJL-part widths (m = 0 for MSE)
+  int bits[TQ_MAX_GROUPS];                 // MSE-stage bits (0: no codes)
+  int code_words[TQ_MAX_GROUPS], sign_words[TQ_MAX_GROUPS];
+  const float* qr[TQ_MAX_GROUPS];          // [nq][d_g] (the block of queries of this pass)
+  const float* qu[TQ_MAX_GROUPS];          // [nq][m_g]
+  const uint32_t* codes[TQ_MAX_GROUPS];
+  const uint32_t* signs[TQ_MAX_GROUPS];
+  const float* norms[TQ_MAX_GROUPS];
+  const float* rnorms[TQ_MAX_GROUPS];
+  const float* centroids[TQ_MAX_GROUPS];
+  float coef[TQ_MAX_GROUPS];               // sqrt(pi/2) / m_g
+};
+cudaError_t launch_split_score_queries(const SplitScoreGroups& G, int64_t nq, int K, uint16_t* qh, uint16_t* ql,
+                                       cudaStream_t s);
+cudaError_t launch_split_score_records(const SplitScoreGroups& G, int64_t n, int K, uint16_t* rh, uint16_t* rl,
+                                       float* ones, cudaStream_t s);
 // Split-cache decode on the tensor cores: two MSE groups per record, 32 rotated dims at 3
 // bits then 96 at 2 bits (keys and values), GQA groups of at most 4 heads.
 struct SplitMmaParams;

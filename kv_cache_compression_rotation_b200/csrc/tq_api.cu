@@ -1170,26 +1170,76 @@ tq_status tq_quantize_split(const tq_split* sp, const void* x, int32_t dtype, in
 
 // Workspace of tq_score_split: per group the gathered rotated queries (and S q' for PROD),
 // then, for top-k, one block of summed dense scores.
-static size_t split_ws_bytes(const tq_split* sp, int64_t nq, int64_t n, int32_t topk, size_t* off_qr, size_t* off_qu,
-                             size_t* off_dense) {
+// The summed estimates on the tensor cores (score_split_tc.cu): MSE (1..4 bits) or PROD
+// (2..5 bits, m = d) groups whose widths d_g + m_g add up to a multiple of 64 (at most 4096),
+// against at least 4096 records.
+static bool split_score_tc(const tq_split* sp, int64_t n, int* K) {
+  if (n < 4096 || std::getenv("TQ_FORCE_SIMT")) return false;
+  int k = 0;
+  for (int g = 0; g < sp->n_groups; ++g) {
+    const tq_quantizer* q = sp->groups[g];
+    if (q->kind == TQ_KIND_MSE) {
+      if (q->bits < 1 || q->bits > 4) return false;
+      k += q->d;
+    } else if (q->kind == TQ_KIND_PROD) {
+      if (q->bits < 2 || q->bits > 5 || q->m != q->d) return false;
+      k += 2 * q->d;
+    } else {
+      return false;
+    }
+  }
+  if (k % 64 || k > 4096) return false;
+  if (K) *K = k;
+  return true;
+}
+
+// Workspace of tq_score_split: per group the gathered, rotated queries (and S q' for PROD);
+// then either the tensor-core operands (query block and records as bf16 hi + lo, a column
+// of ones) or the CUDA-core estimator's block of dense scores; top-k keeps one block of
+// summed dense scores.
+struct SplitScorePlan {
+  size_t qr[TQ_MAX_GROUPS], qu[TQ_MAX_GROUPS], ah, al, bh, bl, ones, dense, bytes;
+  bool tc;
+  int K;
+  int64_t qb;                // queries per pass
+};
+
+static SplitScorePlan plan_split_score(const tq_split* sp, int64_t nq, int64_t n, int32_t topk) {
+  SplitScorePlan P{};
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
   size_t b = 0;
   for (int g = 0; g < sp->n_groups; ++g) {
-    off_qr[g] = b;
-    b += (static_cast<size_t>(nq) * sp->groups[g]->d * 4 + 255) / 256 * 256;
-    off_qu[g] = b;
-    b += (static_cast<size_t>(nq) * score_qu_stride(sp->groups[g]) * 4 + 255) / 256 * 256;
+    P.qr[g] = b;
+    b = al(b + static_cast<size_t>(nq) * sp->groups[g]->d * 4);
+    P.qu[g] = b;
+    b = al(b + static_cast<size_t>(nq) * score_qu_stride(sp->groups[g]) * 4);
   }
-  *off_dense = b;
-  if (topk > 0) b += static_cast<size_t>(score_block(nq, n)) * static_cast<size_t>(n) * 4 + 256;
-  return b + 256;
+  P.tc = split_score_tc(sp, n, &P.K);
+  if (P.tc) {
+    int64_t qb = (1ll << 28) / std::max<int64_t>(n, 1) / 128 * 128;
+    qb = std::max<int64_t>(128, std::min<int64_t>(1024, qb));
+    P.qb = std::min<int64_t>(qb, (nq + 127) / 128 * 128);
+    P.ah = b; b = al(b + P.qb * P.K * 2);
+    P.al = b; b = al(b + P.qb * P.K * 2);
+    P.bh = b; b = al(b + static_cast<size_t>(n) * P.K * 2);
+    P.bl = b; b = al(b + static_cast<size_t>(n) * P.K * 2);
+    P.ones = b; b = al(b + static_cast<size_t>(n) * 4);
+    P.dense = b;
+    if (topk > 0) b = al(b + static_cast<size_t>(P.qb) * n * 4);
+  } else {
+    P.qb = topk > 0 ? score_block(nq, n) : nq;
+    P.dense = b;
+    if (topk > 0) b += static_cast<size_t>(P.qb) * static_cast<size_t>(n) * 4 + 256;
+  }
+  P.bytes = b + 256;
+  return P;
 }
 
 tq_status tq_score_split_workspace(const tq_split* sp, int64_t nq, int64_t n, int32_t topk, size_t* bytes) {
   tq_status s = check_split(sp);
   if (s != TQ_OK) return s;
   if (!bytes || nq < 0 || n < 0 || topk < 0) return fail(TQ_ERR_INVALID_ARG, "bad workspace query");
-  size_t a[TQ_MAX_GROUPS], b[TQ_MAX_GROUPS], c;
-  *bytes = split_ws_bytes(sp, nq, n, topk, a, b, &c);
+  *bytes = plan_split_score(sp, nq, n, topk).bytes;
   return TQ_OK;
 }
 
@@ -1209,8 +1259,8 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
   if (!qv || !scores || (topk > 0 && !ids)) return fail(TQ_ERR_INVALID_ARG, "NULL query or output");
   if (!aligned16(qv) || !aligned16(scores) || (ids && !aligned16(ids)))
     return fail(TQ_ERR_ALIGNMENT, "query/output not 16-byte aligned");
-  size_t off_qr[TQ_MAX_GROUPS], off_qu[TQ_MAX_GROUPS], off_dense;
-  const size_t need = split_ws_bytes(sp, nq, n, topk, off_qr, off_qu, &off_dense);
+  const SplitScorePlan PL = plan_split_score(sp, nq, n, topk);
+  const size_t need = PL.bytes;
   if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
   if (!aligned16(workspace)) return fail(TQ_ERR_ALIGNMENT, "workspace not 16-byte aligned");
   Range ins[4 * TQ_MAX_GROUPS + 2];
@@ -1235,8 +1285,8 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
   for (int g = 0; g < sp->n_groups; ++g) {
     const tq_quantizer* q = sp->groups[g];
     const int qus = score_qu_stride(q);
-    float* qr = reinterpret_cast<float*>(ws + off_qr[g]);
-    float* qu = qus ? reinterpret_cast<float*>(ws + off_qu[g]) : nullptr;
+    float* qr = reinterpret_cast<float*>(ws + PL.qr[g]);
+    float* qu = qus ? reinterpret_cast<float*>(ws + PL.qu[g]) : nullptr;
     score_qprep_kernel<<<static_cast<unsigned>(nq), 128, 2 * q->d * 4, stream>>>(
         qv, dtype, q->d, q->kind, q->rot, q->S, q->m, q->k_top, qr, qu, qus, sp->d, sp->cols[g], status);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score qprep launch");
@@ -1246,10 +1296,58 @@ tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int6
     P[g].accumulate = g > 0;
     smem = std::max(smem, score_smem(P[g]));
   }
+  float* dense = reinterpret_cast<float*>(ws + PL.dense);
+  if (PL.tc) {
+    // one split-precision product of [queries of every group] x [decoded records of every group]
+    auto u16 = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+    float* ones = reinterpret_cast<float*>(ws + PL.ones);
+    SplitScoreGroups G{};
+    G.n = sp->n_groups;
+    for (int g = 0; g < sp->n_groups; ++g) {
+      const tq_quantizer* q = sp->groups[g];
+      const tq_layout L = layout_of(q);
+      const bool prod = q->kind == TQ_KIND_PROD;
+      G.d[g] = q->d; G.m[g] = prod ? q->m : 0;
+      G.bits[g] = prod ? q->bits - 1 : q->bits;
+      G.code_words[g] = L.code_words; G.sign_words[g] = L.sign_words;
+      G.codes[g] = keys[g].codes; G.signs[g] = keys[g].signs;
+      G.norms[g] = keys[g].norms; G.rnorms[g] = keys[g].rnorms;
+      G.centroids[g] = q->centroids;
+      G.coef[g] = prod ? static_cast<float>(std::sqrt(M_PI / 2.0) / q->m) : 0.f;
+    }
+    e = launch_split_score_records(G, n, PL.K, u16(PL.bh), u16(PL.bl), ones, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "split record expansion launch");
+    CUtensorMap maps[4];
+    const int tn = gemm_tile_n(static_cast<int>(n));       // B box = one column tile
+    if ((s = bf16_map(&maps[2], u16(PL.bh), n, PL.K, tn)) != TQ_OK) return s;
+    if ((s = bf16_map(&maps[3], u16(PL.bl), n, PL.K, tn)) != TQ_OK) return s;
+    for (int64_t q0 = 0; q0 < nq; q0 += PL.qb) {
+      const int64_t nb = std::min(PL.qb, nq - q0);
+      for (int g = 0; g < sp->n_groups; ++g) {
+        G.qr[g] = P[g].qr + q0 * G.d[g];
+        G.qu[g] = P[g].qu ? P[g].qu + q0 * G.m[g] : nullptr;
+      }
+      e = launch_split_score_queries(G, nb, PL.K, u16(PL.ah), u16(PL.al), stream);
+      if (e != cudaSuccess) return cuda_fail(e, "split query operand launch");
+      if ((s = bf16_map(&maps[0], u16(PL.ah), nb, PL.K, 128)) != TQ_OK) return s;
+      if ((s = bf16_map(&maps[1], u16(PL.al), nb, PL.K, 128)) != TQ_OK) return s;
+      SplitGemmParams gp{};
+      gp.M = nb; gp.N = static_cast<int>(n); gp.K = PL.K; gp.status = status; gp.wait_limit = wait_limit();
+      gp.out = topk > 0 ? dense : scores + q0 * n; gp.ldo = n; gp.col_scale = ones;
+      const int64_t work = (nb + 127) / 128 * ((n + tn - 1) / tn);
+      e = launch_split_gemm(maps, gp, GEMM_EPI_SCORE, 1, static_cast<int>(std::min<int64_t>(work, sm_count())), stream);
+      if (e != cudaSuccess) return cuda_fail(e, "split estimate launch");
+      if (topk > 0) {
+        if (topk <= 16) topk_kernel<16><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+        else topk_kernel<32><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+      }
+    }
+    return TQ_OK;
+  }
   e = cudaFuncSetAttribute(score_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "score attribute");
-  float* dense = reinterpret_cast<float*>(ws + off_dense);
-  const int64_t qb = topk > 0 ? score_block(nq, n) : nq;
+  const int64_t qb = PL.qb;
   for (int64_t q0 = 0; q0 < nq; q0 += qb) {
     const int64_t nb = std::min(qb, nq - q0);
     const dim3 grid(static_cast<unsigned>((n + kScoreThreads - 1) / kScoreThreads),
