@@ -574,19 +574,22 @@ def run_other(args):
         td = _timed(lambda: K.decode_attn_split(sp, sp, qd, seqd, out, out, Nd, Hkvd), stream, flush)
         assert K.get_status() == 0
         # and at the 128k decode shapes: B=8, Hkv=8, Hq=32, context 131072 (738 MB of split
-        # K and V records)
+        # K and V records, separate caches)
         Bb, Nb = 8, 131072
         nb = Bb * Hkvd * Nb
-        xb = ti.normal_torch((nb, Dm), ti.SEEDS["keys"] + 8, dev)
-        xb[:, torch.from_numpy(planted).to(dev)] *= 6.0
-        xb = xb.to(torch.bfloat16).contiguous()
-        outb = sp.alloc(nb, dev)
-        K.quantize_split(sp, xb, outb)
-        del xb
-        torch.cuda.empty_cache()
+        caches = []
+        for j in range(2):
+            xb = ti.normal_torch((nb, Dm), ti.SEEDS["keys" if j == 0 else "values"] + 8, dev)
+            xb[:, torch.from_numpy(planted).to(dev)] *= 6.0
+            xb = xb.to(torch.bfloat16).contiguous()
+            caches.append(sp.alloc(nb, dev))
+            K.quantize_split(sp, xb, caches[-1])
+            del xb
+            torch.cuda.empty_cache()
+        kb_c, vb_c = caches
         qb = ti.normal_torch((Bb, Hqd, Dm), ti.SEEDS["queries"] + 8, dev)
         seqb = torch.full((Bb,), Nb, dtype=torch.int32, device=dev)
-        tb = _timed(lambda: K.decode_attn_split(sp, sp, qb, seqb, outb, outb, Nb, Hkvd), stream, flush)
+        tb = _timed(lambda: K.decode_attn_split(sp, sp, qb, seqb, kb_c, vb_c, Nb, Hkvd), stream, flush)
         assert K.get_status() == 0
         rec = sum(4 * (L.code_words + L.has_norms) for L in (g.layout() for g in groups))
         parts = {"quantize_split": {"ms": tq, "vectors_per_s": n / tq * 1e3, "gbs": n * (Dm * 2 + rec) / tq / 1e6,
