@@ -138,7 +138,7 @@ __host__ __device__ inline TmaStageLayout tma_stage_layout(int kw, int vw, int k
 // the table, the rest after it; the kernel checks the layout against the allocation.
 __host__ __device__ inline uint32_t tma_table_bytes(int kb, int vb) {
   // 1-bit codes index the table by whole bytes
-  return (kb == 1 || vb == 1) ? 65536u : (1u << (2 * (kb > vb ? kb : vb))) * 256u;
+  return (kb <= 2 || vb <= 2) ? 65536u : (1u << (2 * (kb > vb ? kb : vb))) * 256u;
 }
 __host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u : 8u; }
 __host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk, bool vpr = false) {
@@ -172,6 +172,12 @@ __device__ __forceinline__ uint32_t sld32(uint32_t a) {
   return v;
 }
 __device__ __forceinline__ float sldf(uint32_t a) { return __uint_as_float(sld32(a)); }
+// 64-bit table load (2-bit entries).
+__device__ __forceinline__ uint2 tab_ld64(uint32_t addr) {
+  uint2 v;
+  asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
 // 128-bit table load (1-bit entries).
 __device__ __forceinline__ uint4 tab_ld128(uint32_t addr) {
   uint4 v;
@@ -260,7 +266,7 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int HB = PK ? 4 : kTmaHeadBlock;            // query heads per work item
   constexpr int RW = static_cast<int>(tma_merge_rows(PK));   // merge rows per warp
   constexpr int CONSUMERS = NC * 32;
-  constexpr int NE = (KB == 1 || VB == 1) ? 256 : (KLUT > VLUT ? KLUT : VLUT);   // table entries
+  constexpr int NE = (KB <= 2 || VB <= 2) ? 256 : (KLUT > VLUT ? KLUT : VLUT);   // table entries
   constexpr uint32_t TAB = static_cast<uint32_t>(NE) * 256u;
   extern __shared__ __align__(128) unsigned char tsm_[];
 
@@ -367,6 +373,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         // byte e = codes of 8 consecutive dims: word j holds dims 2j, 2j + 1
         val = pack_half2(__ldg(p.kc + ((e >> (2 * j)) & 1)) / p.k_scale,
                          __ldg(p.kc + ((e >> (2 * j + 1)) & 1)) / p.k_scale);
+      } else if constexpr (KB == 2) {
+        // byte e = codes of 4 consecutive dims: word i & 1 holds dims (0, 1) or (2, 3)
+        const int w = i & 1;
+        val = pack_half2(__ldg(p.kc + ((e >> (4 * w)) & 3)) / p.k_scale,
+                         __ldg(p.kc + ((e >> (4 * w + 2)) & 3)) / p.k_scale);
       } else if (e < KLUT) {
         val = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) / p.k_scale, __ldg(p.kc + (e >> KB)) / p.k_scale);
       }
@@ -376,6 +387,12 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         // words = A registers a0 (row g, tokens 0, 1), a1 (row g + 8), a2 (row g, tokens 2, 3), a3
         const int b = (j == 0) ? 0 : (j == 1) ? 4 : (j == 2) ? 2 : 6;
         val = pack_half2(__ldg(p.vc + ((e >> b) & 1)) / p.v_scale, __ldg(p.vc + ((e >> (b + 1)) & 1)) / p.v_scale);
+      } else if constexpr (VB == 2) {
+        // byte e: bits 0-3 = one dim of a token pair (row g), bits 4-7 = row g + 8: words =
+        // A registers of the pair in rows g and g + 8
+        const int w = i & 1;
+        val = pack_half2(__ldg(p.vc + ((e >> (4 * w)) & 3)) / p.v_scale,
+                         __ldg(p.vc + ((e >> (4 * w + 2)) & 3)) / p.v_scale);
       } else if (e < VLUT) {
         val = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
       }
@@ -547,6 +564,9 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   const uint32_t klo = tabA | static_cast<uint32_t>(lane) * 4u, vlo = klo + 128u;
   // 16-byte slots of the 1-bit entries: 8 per half row
   const uint32_t k1lo = tabA | (static_cast<uint32_t>(lane & 7) << 4), v1lo = k1lo + 128u;
+  // 8-byte slots of the 2-bit entries: 16 per half row (a 64-bit load of 32 lanes takes two
+  // passes, so 16 slots keep it conflict-free)
+  const uint32_t k2lo = tabA | (static_cast<uint32_t>(lane & 15) << 3), v2lo = k2lo + 128u;
   // MMA column of this lane's B operand (g) and of its accumulators (2t, 2t + 1)
   const int qcol = PK ? (g & 3) : g;               // head (in the block) of B column g
   const bool qlo = PK && g >= 4;                  // B column g carries a lo part
@@ -797,6 +817,12 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           uint32_t a0, a1, a2, a3;
           if constexpr (KB == 1) {
             a0 = kq[0][k][0]; a1 = kq[1][k][0]; a2 = kq[0][k][1]; a3 = kq[1][k][1];
+          } else if constexpr (KB == 2) {
+            // dims 4k .. 4k + 3 of a row are byte k % 4 of word k / 4: one 64-bit lookup per row
+            const uint32_t sel = 0x7604u | (static_cast<uint32_t>(k & 3) << 4);
+            const uint2 r0 = tab_ld64(__byte_perm(ks[u][0][k >> 2], k2lo, sel));
+            const uint2 r1 = tab_ld64(__byte_perm(ks[u][1][k >> 2], k2lo, sel));
+            a0 = r0.x; a2 = r0.y; a1 = r1.x; a3 = r1.y;
           } else if constexpr (KB == 4) {
             // dims (4 k, 4 k + 1) are byte 2 (k % 2) of word k / 2; (+2, +3) the next byte
             const uint32_t w0c = ks[u][0][k >> 1], w1c = ks[u][1][k >> 1];
@@ -1033,6 +1059,31 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             const uint32_t a3 = tab_ld(tab_off((i & 1) ? hi[1][1] : lo[1][1], vlo, k));
             mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
             if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
+          }
+        } else if constexpr (VB == 2) {
+          // interleave the 2-bit codes of a token pair: byte i of z (zl: i < 4, zh: i >= 4)
+          // holds dim i of both tokens (bits 0-3) and dim 8 + i (bits 4-7), one 64-bit
+          // lookup per pair and M-tile
+          auto spread = [](uint32_t x) {           // 2-bit fields j = 0..3 of a byte -> bits 8j
+            x = (x | (x << 12)) & 0x000F000Fu;
+            return (x | (x << 6)) & 0x03030303u;
+          };
+          uint32_t zl[2], zh[2];
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+            const uint32_t a = vs[u][2 * pr][0], b = vs[u][2 * pr + 1][0];
+            zl[pr] = spread(a & 0xFFu) | (spread(b & 0xFFu) << 2) | (spread((a >> 16) & 0xFFu) << 4) |
+                     (spread((b >> 16) & 0xFFu) << 6);
+            zh[pr] = spread((a >> 8) & 0xFFu) | (spread((b >> 8) & 0xFFu) << 2) | (spread(a >> 24) << 4) |
+                     (spread(b >> 24) << 6);
+          }
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const uint32_t sel = 0x7604u | (static_cast<uint32_t>(i & 3) << 4);
+            const uint2 r0 = tab_ld64(__byte_perm(i < 4 ? zl[0] : zh[0], v2lo, sel));
+            const uint2 r1 = tab_ld64(__byte_perm(i < 4 ? zl[1] : zh[1], v2lo, sel));
+            mma16816(o[i], r0.x, r0.y, r1.x, r1.y, b0h, b1h);
+            if constexpr (!PK) mma16816(o[i], r0.x, r0.y, r1.x, r1.y, b0l, b1l);
           }
         } else if constexpr (VB == 1) {
           // bit-transpose the 4 tokens' 16-dim slices: byte i of zl (i < 4) / zh holds dim i
