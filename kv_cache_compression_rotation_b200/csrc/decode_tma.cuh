@@ -172,6 +172,18 @@ __device__ __forceinline__ uint32_t sld32(uint32_t a) {
   return v;
 }
 __device__ __forceinline__ float sldf(uint32_t a) { return __uint_as_float(sld32(a)); }
+// Bits [pos, pos + W) of a word slice moved to bit `to`, the rest cleared.  pos and to are
+// compile-time after unrolling, so this is one shift (a funnel shift across two words) and
+// a mask that folds into the OR forming the table address.
+template <int W, int NW>
+__device__ __forceinline__ uint32_t field_to(const uint32_t (&seg)[NW], int pos, int to) {
+  const int wi = pos >> 5, sh = pos & 31;
+  constexpr uint32_t m = (1u << W) - 1u;
+  if (sh + W > 32 && wi + 1 < NW) return (__funnelshift_r(seg[wi], seg[wi + 1], sh) << to) & (m << to);
+  const uint32_t x = seg[wi];
+  return (sh >= to ? (x >> (sh - to)) : (x << (to - sh))) & (m << to);
+}
+
 // 64-bit table load (2-bit entries).
 __device__ __forceinline__ uint2 tab_ld64(uint32_t addr) {
   uint2 v;
@@ -832,10 +844,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
             a2 = tab_ld(tab_off(w0c, klo, bsel + 1));
             a3 = tab_ld(tab_off(w1c, klo, bsel + 1));
           } else {
-            a0 = tab_ld((pair_at<KB, NWK>(ks[u][0], 4 * k * KB) << 8) | klo);
-            a1 = tab_ld((pair_at<KB, NWK>(ks[u][1], 4 * k * KB) << 8) | klo);
-            a2 = tab_ld((pair_at<KB, NWK>(ks[u][0], (4 * k + 2) * KB) << 8) | klo);
-            a3 = tab_ld((pair_at<KB, NWK>(ks[u][1], (4 * k + 2) * KB) << 8) | klo);
+            // the code pair's 2 KB bits placed straight at the entry index bits 8..
+            a0 = tab_ld(field_to<2 * KB, NWK>(ks[u][0], 4 * k * KB, 8) | klo);
+            a1 = tab_ld(field_to<2 * KB, NWK>(ks[u][1], 4 * k * KB, 8) | klo);
+            a2 = tab_ld(field_to<2 * KB, NWK>(ks[u][0], (4 * k + 2) * KB, 8) | klo);
+            a3 = tab_ld(field_to<2 * KB, NWK>(ks[u][1], (4 * k + 2) * KB, 8) | klo);
           }
           if (k & 1) {
             mma16816(accb, a0, a1, a2, a3, qh[k][0], qh[k][1]);
@@ -1105,12 +1118,14 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         } else {
 #pragma unroll
           for (int i = 0; i < MT; ++i) {
-            const uint32_t e00 = field_at<VB, NWV>(vs[u][0], i * VB) | (field_at<VB, NWV>(vs[u][1], i * VB) << VB);
-            const uint32_t e01 = field_at<VB, NWV>(vs[u][0], (8 + i) * VB) | (field_at<VB, NWV>(vs[u][1], (8 + i) * VB) << VB);
-            const uint32_t e10 = field_at<VB, NWV>(vs[u][2], i * VB) | (field_at<VB, NWV>(vs[u][3], i * VB) << VB);
-            const uint32_t e11 = field_at<VB, NWV>(vs[u][2], (8 + i) * VB) | (field_at<VB, NWV>(vs[u][3], (8 + i) * VB) << VB);
-            const uint32_t a0 = tab_ld((e00 << 8) | vlo), a1 = tab_ld((e01 << 8) | vlo);
-            const uint32_t a2 = tab_ld((e10 << 8) | vlo), a3 = tab_ld((e11 << 8) | vlo);
+            // entry index (code of the first token | code of the second << VB) at bits 8..
+            auto vaddr = [&](const uint32_t (&x)[NWV], const uint32_t (&y)[NWV], int pos) {
+              return field_to<VB, NWV>(x, pos, 8) | field_to<VB, NWV>(y, pos, 8 + VB) | vlo;
+            };
+            const uint32_t a0 = tab_ld(vaddr(vs[u][0], vs[u][1], i * VB));
+            const uint32_t a1 = tab_ld(vaddr(vs[u][0], vs[u][1], (8 + i) * VB));
+            const uint32_t a2 = tab_ld(vaddr(vs[u][2], vs[u][3], i * VB));
+            const uint32_t a3 = tab_ld(vaddr(vs[u][2], vs[u][3], (8 + i) * VB));
             mma16816(o[i], a0, a1, a2, a3, b0h, b1h);
             if constexpr (!PK) mma16816(o[i], a0, a1, a2, a3, b0l, b1l);
           }
