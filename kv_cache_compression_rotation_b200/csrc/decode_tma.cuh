@@ -377,36 +377,40 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // entries c / s: one reciprocal per thread, a product per value (the table is up to 64 KB,
+  // refilled by every CTA; the product is within an fp32 ulp of the quotient, far below
+  // the entries' fp16 rounding)
+  const float kinv = 1.f / p.k_scale, vinv = 1.f / p.v_scale;
   for (int i = tid; i < NE * 64; i += kTmaThreads) {
     const int e = i >> 6, j = i & 3;               // j: word of a 16-byte slot (1-bit entries)
     uint32_t val = 0u;
     if ((i & 32) == 0) {
       if constexpr (KB == 1) {
         // byte e = codes of 8 consecutive dims: word j holds dims 2j, 2j + 1
-        val = pack_half2(__ldg(p.kc + ((e >> (2 * j)) & 1)) / p.k_scale,
-                         __ldg(p.kc + ((e >> (2 * j + 1)) & 1)) / p.k_scale);
+        val = pack_half2(__ldg(p.kc + ((e >> (2 * j)) & 1)) * kinv,
+                         __ldg(p.kc + ((e >> (2 * j + 1)) & 1)) * kinv);
       } else if constexpr (KB == 2) {
         // byte e = codes of 4 consecutive dims: word i & 1 holds dims (0, 1) or (2, 3)
         const int w = i & 1;
-        val = pack_half2(__ldg(p.kc + ((e >> (4 * w)) & 3)) / p.k_scale,
-                         __ldg(p.kc + ((e >> (4 * w + 2)) & 3)) / p.k_scale);
+        val = pack_half2(__ldg(p.kc + ((e >> (4 * w)) & 3)) * kinv,
+                         __ldg(p.kc + ((e >> (4 * w + 2)) & 3)) * kinv);
       } else if (e < KLUT) {
-        val = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) / p.k_scale, __ldg(p.kc + (e >> KB)) / p.k_scale);
+        val = pack_half2(__ldg(p.kc + (e & ((1 << KB) - 1))) * kinv, __ldg(p.kc + (e >> KB)) * kinv);
       }
     } else {
       if constexpr (VB == 1) {
         // byte e: bits 0-3 = one dim of the lane's 4 tokens (row g), bits 4-7 = row g + 8;
         // words = A registers a0 (row g, tokens 0, 1), a1 (row g + 8), a2 (row g, tokens 2, 3), a3
         const int b = (j == 0) ? 0 : (j == 1) ? 4 : (j == 2) ? 2 : 6;
-        val = pack_half2(__ldg(p.vc + ((e >> b) & 1)) / p.v_scale, __ldg(p.vc + ((e >> (b + 1)) & 1)) / p.v_scale);
+        val = pack_half2(__ldg(p.vc + ((e >> b) & 1)) * vinv, __ldg(p.vc + ((e >> (b + 1)) & 1)) * vinv);
       } else if constexpr (VB == 2) {
         // byte e: bits 0-3 = one dim of a token pair (row g), bits 4-7 = row g + 8: words =
         // A registers of the pair in rows g and g + 8
         const int w = i & 1;
-        val = pack_half2(__ldg(p.vc + ((e >> (4 * w)) & 3)) / p.v_scale,
-                         __ldg(p.vc + ((e >> (4 * w + 2)) & 3)) / p.v_scale);
+        val = pack_half2(__ldg(p.vc + ((e >> (4 * w)) & 3)) * vinv,
+                         __ldg(p.vc + ((e >> (4 * w + 2)) & 3)) * vinv);
       } else if (e < VLUT) {
-        val = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) / p.v_scale, __ldg(p.vc + (e >> VB)) / p.v_scale);
+        val = pack_half2(__ldg(p.vc + (e & ((1 << VB) - 1))) * vinv, __ldg(p.vc + (e >> VB)) * vinv);
       }
     }
     tab_g[i] = val;
