@@ -285,10 +285,14 @@ typedef struct {
 
 /*
  * DEVICE.  Quantize n rows x [n*d] (dtype, row-major) group by group: out[g] receives
- * the records of group g (layout from tq_record_layout(groups[g])), exactly what
- * tq_quantize_mse / tq_quantize_prod would write for the gathered rows
- * (x_v[cols[g][0]], ..., x_v[cols[g][d_g - 1]]).  out is a host array of n_groups
- * packed descriptors.  Validation as for tq_quantize_mse, per group.
+ * the records of group g (layout from tq_record_layout(groups[g])), the quantization by
+ * groups[g] of the gathered rows (x_v[cols[g][0]], ..., x_v[cols[g][d_g - 1]]): what
+ * tq_quantize_mse / tq_quantize_prod write for those rows, up to the code of a coordinate
+ * within rounding of a boundary when the two calls run different kernels.  16-bit rows
+ * of the outlier split of the KV experiments (d = 128, two MSE groups: 32 channels at 3
+ * bits then 96 at 2, or 4 then 3) take one tensor-core pass over whole rows; other splits
+ * gather their channels on the loads of the CUDA-core kernel.  out is a host array of
+ * n_groups packed descriptors.  Validation as for tq_quantize_mse, per group.
  */
 tq_status tq_quantize_split(const tq_split* sp, const void* x, int32_t dtype, int64_t n,
                             const tq_packed* out, tq_stream stream);
@@ -303,7 +307,10 @@ tq_status tq_score_split_workspace(const tq_split* sp, int64_t nq, int64_t n, in
  * of every group belongs to vector i).  Output as tq_score: topk == 0 gives scores
  * [nq*n] dense; topk in 1..32 gives the topk records of the summed estimate per query
  * (descending, ties to the lower id).  keys is a host array of n_groups packed
- * descriptors; workspace: device, >= tq_score_split_workspace bytes.
+ * descriptors; workspace: device, >= tq_score_split_workspace bytes.  From 4096 records
+ * (MSE groups of 1..4 bits or PROD groups of 2..5 bits with m = d, total width of the
+ * groups' parts a multiple of 64) the estimates are one split-precision tensor-core
+ * product; otherwise the CUDA-core estimator adds the groups.
  */
 tq_status tq_score_split(const tq_split* sp, const void* qv, int32_t dtype, int64_t nq,
                          const tq_packed* keys, int64_t n, int32_t topk, float* scores,
@@ -325,7 +332,10 @@ tq_status tq_decode_attn_split_workspace(const tq_split* ks, const tq_split* vs,
  * h / (Hq/Hkv).  q [B*Hq*d] (dtype), seq_lens [B] device int32 (1..Nmax), kcache/vcache
  * host arrays of one packed descriptor per group, each group's records laid out
  * [B][Hkv][Nmax]; out [B*Hq*d] fp32.  libtq runs MSE or PROD key groups, MSE value
- * groups, d <= 256 and Hq/Hkv <= 8 (TQ_ERR_UNSUPPORTED otherwise).  A value channel index out of
+ * groups, d <= 256 and Hq/Hkv <= 8 (TQ_ERR_UNSUPPORTED otherwise).  The outlier split
+ * of the KV experiments for keys and values (d = 128, two MSE groups: 32 rotated dims at
+ * 3 bits then 96 at 2) with Hq/Hkv <= 4 and Nmax a multiple of 4 runs on the tensor
+ * cores; other shapes on CUDA cores.  A value channel index out of
  * range sets TQ_ERR_INVALID_ARG on the device and its output is not written.
  */
 tq_status tq_decode_attn_split(const tq_split* ks, const tq_split* vs, const void* q,
