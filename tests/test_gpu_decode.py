@@ -96,6 +96,7 @@ DECODE_CASES = [
     ("bits1-3", 1, 8, 2, 800, [800], "mse", 1, 3),
     ("bits2-4", 2, 8, 2, 800, [800, 17], "mse", 2, 4),
     ("bits2", 1, 8, 2, 900, [900], "mse", 2, 2),
+    ("bits2-g8", 2, 16, 2, 500, [500, 263], "mse", 2, 2),
     ("bits3-2-g8", 1, 16, 2, 600, [600], "mse", 3, 2),
     ("prod2", 1, 8, 2, 1500, [1500], "prod", 2, 4),
     ("prod5", 1, 8, 2, 600, [600], "prod", 5, 3),
