@@ -93,22 +93,33 @@ __device__ __forceinline__ void lds64(uint32_t a, uint32_t& x, uint32_t& y) {
   asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x), "=r"(y) : "r"(a));
 }
 
+// Where the lane's 12-bit key field of 3-bit k-step kl starts (bit 48 kl + 12 t): word jb =
+// 48 kl / 32 or the one after it (up), at bit s of that word.  When it starts in word jb + 1
+// it ends there too (s + 12 <= 32), so the field is always the funnel of (jb or jb + 1, jb + 1).
+struct Field3 {
+  bool up;
+  uint32_t s;
+};
+__device__ __forceinline__ Field3 field3(int kl, int t) {
+  const int pos = 48 * kl + 12 * t, jb = (48 * kl) >> 5;
+  return Field3{(pos >> 5) > jb, static_cast<uint32_t>(pos & 31)};
+}
+
 // Key operand of one k-step for one token row: the lane's 4-code field of local k-step kl
 // (dims 16 kl + 4t .. + 3 of its group) -> (dims 0,1) and (dims 2,3) as half2.
 template <int B, int W>
-__device__ __forceinline__ void key_pairs(const uint32_t (&w)[W], int kl, uint32_t sel, uint32_t tlo, int t,
+__device__ __forceinline__ void key_pairs(const uint32_t (&w)[W], int kl, uint32_t sel, uint32_t tlo, Field3 f,
                                           uint32_t& lo, uint32_t& hi) {
   if constexpr (B == 2) {
     // byte t of word kl holds the 4 codes: one 64-bit lookup
     lds64(__byte_perm(w[kl], tlo, sel), lo, hi);
   } else {
     static_assert(B == 3, "key field width");
-    // 12 bits at bit 48 kl + 12 t: a 64-bit window of the two words from word jb
     const int jb = (48 * kl) >> 5;
-    const uint64_t win = (static_cast<uint64_t>(w[jb + 1]) << 32) | w[jb];
-    const uint32_t x = static_cast<uint32_t>(win >> (48 * kl - 32 * jb + 12 * t));
-    lo = tab_ld(tlo | ((x & 63u) << 8));
-    hi = tab_ld(tlo | (((x >> 6) & 63u) << 8));
+    const uint32_t x = __funnelshift_r(f.up ? w[jb + 1] : w[jb], w[jb + 1], f.s);
+    // the two 6-bit pair indices placed at the entry bits 8..13
+    lo = tab_ld(tlo | ((x << 8) & 0x3F00u));
+    hi = tab_ld(tlo | ((x << 2) & 0x3F00u));
   }
 }
 
@@ -124,7 +135,7 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
   static_assert(D0 % 16 == 0 && D0 > 0 && D0 < 128, "group widths");
   static_assert(B0 == 3 && B1 == 2, "instantiated for the 3-bit outlier / 2-bit rest split");
   static_assert(W0 * 32 == D0 * B0 && W1 * 32 == D1 * B1, "whole words per group record");
-  static_assert(L0 * B0 <= 32 && L1 * B1 <= 32, "value field fits a word");
+  static_assert(L0 * B0 + 11 <= 32 && L1 * B1 <= 32, "value fields fit a word (group 0 shifted by up to 11)");
   static_assert(L1 % 4 == 0, "2-bit value runs of whole bytes");
   extern __shared__ __align__(128) unsigned char ssm_[];
 
@@ -278,6 +289,9 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
   constexpr uint32_t M0 = (1u << (L0 * B0)) - 1u;
   constexpr uint32_t M1 = L1 * B1 == 32 ? 0xFFFFFFFFu : (1u << (L1 * B1)) - 1u;
   const float lk0 = p.logit_scale * p.kscale[0], lk1 = p.logit_scale * p.kscale[1];
+  Field3 f3[KS0];
+#pragma unroll
+  for (int k = 0; k < KS0; ++k) f3[k] = field3(k, t);
 
   pdl_wait();
   int gs = 0;
@@ -287,7 +301,9 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
     const int bb = bh / p.Hkv, hk = bh - bb * p.Hkv;
     const int nh = min(kSmRows, G);
     const int64_t qbase = static_cast<int64_t>(bb) * p.Hq + static_cast<int64_t>(hk) * G;
-    // query operand: k-step k covers dims 16k + 4t .. + 3 (group 0 for k < KS0)
+    // query operand: k-step k covers dims 16k + 4t .. + 3 (group 0 for k < KS0), times the
+    // group's logit factor (scale log2(e) and its table scale), so that a score row is the
+    // two groups' accumulators weighted by the token's norms alone
     const bool hok = qcol < nh;
     uint32_t qh[8][2];
 #pragma unroll
@@ -297,7 +313,8 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
         const float* src = k < KS0 ? p.qr[0] + (qbase + qcol) * D0 + 16 * k + 4 * t
                                    : p.qr[1] + (qbase + qcol) * D1 + 16 * (k - KS0) + 4 * t;
         const float4 v = __ldg(reinterpret_cast<const float4*>(src));
-        a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+        const float f = k < KS0 ? lk0 : lk1;
+        a[0] = v.x * f; a[1] = v.y * f; a[2] = v.z * f; a[3] = v.w * f;
       }
       uint32_t h01, l01, h23, l23;
       split_pair(a[0], a[1], h01, l01);
@@ -317,7 +334,8 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
       const uint32_t sb = stage_addr(st);
       const int cnt = static_cast<int>(sld32(tma_smem_u32(cnt_st + st)));
       const int w0 = warp * 16 * U;
-      // ---- this warp's slices ----
+      // ---- this warp's slices (no per-token checks when the warp's tokens are all in the stage) ----
+      const bool whole = w0 + 16 * U <= cnt;
       bool ok[U][2];
       uint32_t kw0[U][2][W0], kw1[U][2][W1];
       float kn0[U][2], kn1[U][2], vn0[U][2], vn1[U][2];
@@ -327,7 +345,7 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int tk = w0 + 16 * u + 8 * h + g;
-          ok[u][h] = tk < cnt;
+          ok[u][h] = whole || tk < cnt;
 #pragma unroll
           for (int j = 0; j < W0; ++j) kw0[u][h][j] = sld32(sb + oK0 + (tk * W0 + j) * 4);
           static_assert(W1 % 2 == 0, "8-byte aligned group-1 records");
@@ -338,16 +356,25 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
             kw1[u][h][j] = x;
             kw1[u][h][j + 1] = y;
           }
-          kn0[u][h] = ok[u][h] ? sldf(sb + oKN0 + 4 * tk) : 0.f;
-          kn1[u][h] = ok[u][h] ? sldf(sb + oKN1 + 4 * tk) : 0.f;
-          vn0[u][h] = ok[u][h] ? sldf(sb + oVN0 + 4 * tk) : 0.f;
-          vn1[u][h] = ok[u][h] ? sldf(sb + oVN1 + 4 * tk) : 0.f;
+          if (whole) {
+            kn0[u][h] = sldf(sb + oKN0 + 4 * tk);
+            kn1[u][h] = sldf(sb + oKN1 + 4 * tk);
+            vn0[u][h] = sldf(sb + oVN0 + 4 * tk);
+            vn1[u][h] = sldf(sb + oVN1 + 4 * tk);
+          } else {
+            kn0[u][h] = ok[u][h] ? sldf(sb + oKN0 + 4 * tk) : 0.f;
+            kn1[u][h] = ok[u][h] ? sldf(sb + oKN1 + 4 * tk) : 0.f;
+            vn0[u][h] = ok[u][h] ? sldf(sb + oVN0 + 4 * tk) : 0.f;
+            vn1[u][h] = ok[u][h] ? sldf(sb + oVN1 + 4 * tk) : 0.f;
+          }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int tk = w0 + 16 * u + kv[i];
           const uint32_t r0 = sb + oV0 + tk * W0 * 4, r1 = sb + oV1 + tk * W1 * 4;
-          f0[u][i] = __funnelshift_r(sld32(r0 + 4 * vw0), sld32(r0 + 4 * vw0n), vs0) & M0;
+          // codes of group 0 at bit 8 (tokens kv 0, 2) or 11 (kv 1, 3): the pair index of a dim
+          // is then two masked shifts of the pair's words
+          f0[u][i] = (__funnelshift_r(sld32(r0 + 4 * vw0), sld32(r0 + 4 * vw0n), vs0) & M0) << (i & 1 ? 11 : 8);
           f1[u][i] = __funnelshift_r(sld32(r1 + 4 * vw1), sld32(r1 + 4 * vw1n), vs1) & M1;
         }
       }
@@ -355,74 +382,90 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
       if (w0 >= cnt) continue;
 
+      // ---- scores of both units: group 0 k-steps into acc0, group 1 into acc1 / acc2 ----
+      float sc[U][4];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        // ---- scores: group 0 k-steps into acc0, group 1 into acc1 ----
         float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < KS0; ++k) {
           uint32_t a0, a1, a2, a3;
-          key_pairs<B0, W0>(kw0[u][0], k, sel_t, k3lo, t, a0, a2);
-          key_pairs<B0, W0>(kw0[u][1], k, sel_t, k3lo, t, a1, a3);
+          key_pairs<B0, W0>(kw0[u][0], k, sel_t, k3lo, f3[k], a0, a2);
+          key_pairs<B0, W0>(kw0[u][1], k, sel_t, k3lo, f3[k], a1, a3);
           mma16816(acc0, a0, a1, a2, a3, qh[k][0], qh[k][1]);
         }
 #pragma unroll
         for (int k = 0; k < KS1; ++k) {
           uint32_t a0, a1, a2, a3;
-          key_pairs<B1, W1>(kw1[u][0], k, sel_t, k2lo, t, a0, a2);
-          key_pairs<B1, W1>(kw1[u][1], k, sel_t, k2lo, t, a1, a3);
+          key_pairs<B1, W1>(kw1[u][0], k, sel_t, k2lo, Field3{}, a0, a2);
+          key_pairs<B1, W1>(kw1[u][1], k, sel_t, k2lo, Field3{}, a1, a3);
           if (k & 1) mma16816(acc2, a0, a1, a2, a3, qh[KS0 + k][0], qh[KS0 + k][1]);
           else mma16816(acc1, a0, a1, a2, a3, qh[KS0 + k][0], qh[KS0 + k][1]);
         }
-        float sc[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc1[i] += acc2[i];
-          acc0[i] += __shfl_xor_sync(0xffffffffu, acc0[i], 2);    // hi + lo columns
-          acc1[i] += __shfl_xor_sync(0xffffffffu, acc1[i], 2);
-        }
+        // row h: ||k_0|| acc0 + ||k_1|| acc1 on this lane's hi or lo columns, then the
+        // partner lane's half (lanes t and t ^ 2 hold the same token rows)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float a = kn0[u][h] * lk0, b = kn1[u][h] * lk1;
-          const float v0 = fmaf(a, acc0[2 * h], b * acc1[2 * h]);
-          const float v1 = fmaf(a, acc0[2 * h + 1], b * acc1[2 * h + 1]);
-          sc[2 * h] = ok[u][h] ? v0 : -INFINITY;
-          sc[2 * h + 1] = ok[u][h] ? v1 : -INFINITY;
+          const float2 s1 = __fadd2_rn(make_float2(acc1[2 * h], acc1[2 * h + 1]), make_float2(acc2[2 * h], acc2[2 * h + 1]));
+          float2 v = __ffma2_rn(make_float2(kn0[u][h], kn0[u][h]), make_float2(acc0[2 * h], acc0[2 * h + 1]),
+                                __fmul2_rn(make_float2(kn1[u][h], kn1[u][h]), s1));
+          v.x += __shfl_xor_sync(0xffffffffu, v.x, 2);
+          v.y += __shfl_xor_sync(0xffffffffu, v.y, 2);
+          sc[u][2 * h] = ok[u][h] ? v.x : -INFINITY;
+          sc[u][2 * h + 1] = ok[u][h] ? v.y : -INFINITY;
         }
-        // ---- online softmax (log2 domain) ----
-        const bool up = sc[0] > m0 || sc[2] > m0 || sc[1] > m1 || sc[3] > m1;
-        if (__any_sync(0xffffffffu, up)) {
-          float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+      }
+      // ---- online softmax (log2 domain), one maximum check per stage ----
+      bool up = false;
 #pragma unroll
-          for (int o2 = 4; o2 < 32; o2 <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
-          }
-          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-          if (mn0 > m0 || mn1 > m1) {
-            const float fa = ex2(m0 - mn0), fb = ex2(m1 - mn1);
-            l0 *= fa;
-            l1 *= fb;
+      for (int u = 0; u < U; ++u) up = up || sc[u][0] > m0 || sc[u][2] > m0 || sc[u][1] > m1 || sc[u][3] > m1;
+      if (__any_sync(0xffffffffu, up)) {
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              o[i][0] *= fa; o[i][1] *= fb; o[i][2] *= fa; o[i][3] *= fb;
-            }
-            m0 = mn0;
-            m1 = mn1;
-          }
+        for (int u = 0; u < U; ++u) {
+          mx0 = fmaxf(mx0, fmaxf(sc[u][0], sc[u][2]));
+          mx1 = fmaxf(mx1, fmaxf(sc[u][1], sc[u][3]));
         }
-        const float p00 = c0ok ? ex2(sc[0] - m0) : 0.f, p01 = c1ok ? ex2(sc[1] - m1) : 0.f;
-        const float p10 = c0ok ? ex2(sc[2] - m0) : 0.f, p11 = c1ok ? ex2(sc[3] - m1) : 0.f;
-        l0 += p00 + p10;
-        l1 += p01 + p11;
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        if (mn0 > m0 || mn1 > m1) {
+          const float2 f = make_float2(ex2(m0 - mn0), ex2(m1 - mn1));
+          l0 *= f.x;
+          l1 *= f.y;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 x = __fmul2_rn(make_float2(o[i][0], o[i][1]), f);
+            const float2 y = __fmul2_rn(make_float2(o[i][2], o[i][3]), f);
+            o[i][0] = x.x; o[i][1] = x.y; o[i][2] = y.x; o[i][3] = y.y;
+          }
+          m0 = mn0;
+          m1 = mn1;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float2 nm = make_float2(-m0, -m1);
+        const float2 d0 = __fadd2_rn(make_float2(sc[u][0], sc[u][1]), nm);
+        const float2 d1 = __fadd2_rn(make_float2(sc[u][2], sc[u][3]), nm);
+        const float p00 = c0ok ? ex2(d0.x) : 0.f, p01 = c1ok ? ex2(d0.y) : 0.f;
+        const float p10 = c0ok ? ex2(d1.x) : 0.f, p11 = c1ok ? ex2(d1.y) : 0.f;
+        const float2 ls = __fadd2_rn(make_float2(l0, l1), __fadd2_rn(make_float2(p00, p01), make_float2(p10, p11)));
+        l0 = ls.x;
+        l1 = ls.y;
         // P^T per value group (the group's norm rides in P): transpose the two 8x8 halves
         uint32_t bg[2][2];
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
           const float n0 = gg ? vn1[u][0] : vn0[u][0], n1 = gg ? vn1[u][1] : vn0[u][1];
+          const float2 pt = __fmul2_rn(make_float2(p00, p01), make_float2(n0, n0));
+          const float2 pb = __fmul2_rn(make_float2(p10, p11), make_float2(n1, n1));
           uint32_t th, tl, bh2, bl2;
-          split_pair(p00 * n0, p01 * n0, th, tl);
-          split_pair(p10 * n1, p11 * n1, bh2, bl2);
+          split_pair(pt.x, pt.y, th, tl);
+          split_pair(pb.x, pb.y, bh2, bl2);
           bg[gg][0] = movmatrix_t(plo ? tl : th);
           bg[gg][1] = movmatrix_t(plo ? bl2 : bh2);
         }
@@ -434,8 +477,7 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
           for (int r = 0; r < 4; ++r) {
             const int dl = 2 * i + (r & 1);                 // run dim of the row
             const int pr = r >> 1;                          // token pair (kv 0,1) or (kv 2,3)
-            const uint32_t idx = ((f0[u][2 * pr] >> (3 * dl)) & 7u) | (((f0[u][2 * pr + 1] >> (3 * dl)) & 7u) << 3);
-            a[r] = tab_ld(v3lo | (idx << 8));
+            a[r] = tab_ld((v3lo | ((f0[u][2 * pr] >> (3 * dl)) & 0x700u)) | ((f0[u][2 * pr + 1] >> (3 * dl)) & 0x3800u));
           }
           mma16816(o[i], a[0], a[1], a[2], a[3], bg[0][0], bg[0][1]);
         }
