@@ -80,7 +80,7 @@ __host__ __device__ constexpr uint32_t sm_stage_bytes(int d0, int b0, int b1) {
   return static_cast<uint32_t>(kSmStage) * (2u * 4u * (sm_words(d0, b0) + sm_words(128 - d0, b1)) + 16u);
 }
 __host__ __device__ constexpr uint32_t sm_misc_bytes() {
-  return (kSmNC * kSmRows * (128u + 2u) * 4u + 2u * kSmNS * 8u + 64u + 127u) & ~127u;
+  return (kSmNC * kSmRows * (128u + 2u) * 4u + 2u * kSmNS * 8u + 64u + 2u * kSmNC * kSmRows * 4u + 127u) & ~127u;
 }
 inline size_t decode_split_mma_smem(int d0, int b0, int b1) {
   const size_t want = 65536 + sm_table_bytes(b0) + sm_table_bytes(b1) + static_cast<size_t>(kSmNS) *
@@ -181,6 +181,7 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * NS);
   volatile int* consumers_stop = abort_flag + 1;
   int* cnt_st = const_cast<int*>(consumers_stop) + 1;             // [NS] tokens of each stage
+  float* mxb = reinterpret_cast<float*>(gen(miscA + NC * kSmRows * (D + 2) * 4 + 2 * NS * 8 + 64));   // [2][warp][4] maxima
   const uint32_t bar0 = tma_smem_u32(bars);
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
   auto empty_bar = [&](int st) { return bar0 + 8u * (NS + st); };
@@ -294,8 +295,8 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
   for (int k = 0; k < KS0; ++k) f3[k] = field3(k, t);
 
   pdl_wait();
-  int gs = 0;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  int gs = 0, ipar = 0;                          // ipar: parity of this CTA's item count
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ipar ^= 1) {
     int bh, chunk, k0, k1;
     item_range(item, bh, chunk, k0, k1);
     const int bb = bh / p.Hkv, hk = bh - bb * p.Hkv;
@@ -512,11 +513,30 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
     for (int i = 0; i < 8; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) o[i][j] += __shfl_xor_sync(0xffffffffu, o[i][j], 2);
-    float* wm = mrg + warp * kSmRows * (D + 2);
+    // each warp publishes its row maxima, scales its own partial by 2^(m_w - M) in registers
+    // and writes it; the item's partial is then a plain sum over the warps in a fixed order
+    // (maxima in a buffer per item parity: a warp may publish the next item's while a slower
+    // one still reads these)
+    float* mb = mxb + ipar * (NC * kSmRows);        // [warp][4 rows]
+    if (t < 2 && g == 0) {
+      mb[warp * kSmRows + 2 * t] = m0;
+      mb[warp * kSmRows + 2 * t + 1] = m1;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+    // one exit decision for every consumer warp, sampled between the two barriers
+    if (tid == 0) *consumers_stop = *abort_flag;
+    float* wm = mrg + warp * kSmRows * (D + 2);      // [row][-, l, o'[D]]
     if (t < 2) {
+      float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NC; ++w) {
+        M0 = fmaxf(M0, mb[w * kSmRows + 2 * t]);
+        M1 = fmaxf(M1, mb[w * kSmRows + 2 * t + 1]);
+      }
+      const float2 f = make_float2(m0 == -INFINITY ? 0.f : ex2(m0 - M0), m1 == -INFINITY ? 0.f : ex2(m1 - M1));
       if (g == 0) {
-        wm[(2 * t) * (D + 2)] = m0; wm[(2 * t) * (D + 2) + 1] = l0;
-        wm[(2 * t + 1) * (D + 2)] = m1; wm[(2 * t + 1) * (D + 2) + 1] = l1;
+        wm[(2 * t) * (D + 2) + 1] = l0 * f.x;
+        wm[(2 * t + 1) * (D + 2) + 1] = l1 * f.y;
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -529,32 +549,38 @@ decode_split_mma_kernel(const SplitMmaParams p, int* status, long long wait_lim)
           da = D0 + L1 * g + 4 * mm + par;
           db = da + 2;
         }
-        wm[(2 * t) * (D + 2) + 2 + da] = o[i][0];
-        wm[(2 * t + 1) * (D + 2) + 2 + da] = o[i][1];
-        wm[(2 * t) * (D + 2) + 2 + db] = o[i][2];
-        wm[(2 * t + 1) * (D + 2) + 2 + db] = o[i][3];
+        const float2 x = __fmul2_rn(make_float2(o[i][0], o[i][1]), f);
+        const float2 y = __fmul2_rn(make_float2(o[i][2], o[i][3]), f);
+        wm[(2 * t) * (D + 2) + 2 + da] = x.x;
+        wm[(2 * t + 1) * (D + 2) + 2 + da] = x.y;
+        wm[(2 * t) * (D + 2) + 2 + db] = y.x;
+        wm[(2 * t + 1) * (D + 2) + 2 + db] = y.y;
       }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
     for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
       const int r = idx / D, j = idx - r * D;
-      float M = -INFINITY;
+      float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int w = 0; w < NC; ++w) M = fmaxf(M, mrg[(w * kSmRows + r) * (D + 2)]);
-      float a = 0.f, L = 0.f;
-#pragma unroll
-      for (int w = 0; w < NC; ++w) {
-        const float* row = mrg + (w * kSmRows + r) * (D + 2);
-        const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
-        L += f * row[1];
-        a += f * row[2 + j];
+      for (int w = 0; w < NC; w += 2) {
+        s0 += mrg[(w * kSmRows + r) * (D + 2) + 2 + j];
+        if (w + 1 < NC) s1 += mrg[((w + 1) * kSmRows + r) * (D + 2) + 2 + j];
       }
       const int64_t pi = (qbase + r) * p.n_chunks + chunk;
-      if (j == 0) { p.part_ml[pi * 2] = M; p.part_ml[pi * 2 + 1] = L; }
-      p.part_o[pi * D + j] = a * (j < D0 ? p.vscale[0] : p.vscale[1]);
+      if (j == 0) {
+        float M = -INFINITY, L = 0.f;
+#pragma unroll
+        for (int w = 0; w < NC; ++w) {
+          M = fmaxf(M, mb[w * kSmRows + r]);
+          L += mrg[(w * kSmRows + r) * (D + 2) + 1];
+        }
+        p.part_ml[pi * 2] = M;
+        p.part_ml[pi * 2 + 1] = L;
+      }
+      p.part_o[pi * D + j] = (s0 + s1) * (j < D0 ? p.vscale[0] : p.vscale[1]);
     }
-    if (tid == 0) *consumers_stop = *abort_flag;
-    asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+    // the next writes of mrg come after the next item's first barrier, which every thread
+    // reaches only after this loop
     if (*consumers_stop) break;
   }
 }

@@ -628,7 +628,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   // cache do not depend on it and are already under way)
   pdl_wait();
   int gs = 0;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  int ipar = 0;                                   // parity of this CTA's item count (merge buffers)
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ipar ^= 1) {
     int bh, hblk, chunk, k0, k1;
     item_range(item, bh, hblk, chunk, k0, k1);
     const int bb = bh / p.Hkv, hk = bh - bb * p.Hkv;
@@ -1150,68 +1151,96 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[i][j] += __shfl_xor_sync(0xffffffffu, o[i][j], 2);
     }
-    float* wm = mrg + warp * RW * (D + 2);           // [row][m, l, o'[D]]
-    if (!PK || t < 2) {
-      if (g == 0) {
-        wm[(2 * t) * (D + 2)] = m0; wm[(2 * t) * (D + 2) + 1] = l0;
-        wm[(2 * t + 1) * (D + 2)] = m1; wm[(2 * t + 1) * (D + 2) + 1] = l1;
+    if constexpr (!SP && !VPR) {
+      // Each warp publishes its row maxima m_w, then scales its own partial (l, o') by
+      // 2^(m_w - M) in registers (M = the row maximum over the warps), so the item's partial
+      // is a plain sum over the warps in a fixed order.  The maxima go to a buffer per item
+      // parity: a warp may publish the next item's while a slower one still reads these.
+      static_assert(2 * NC * RW <= 1024, "merge maxima fit the spectral codebook area");
+      float* mb = utab + ipar * (NC * RW);          // [warp][RW rows]
+      const bool wr = !PK || t < 2;                 // lanes holding rows 2t, 2t + 1
+      if (wr && g == 0) {
+        mb[warp * RW + 2 * t] = m0;
+        mb[warp * RW + 2 * t + 1] = m1;
       }
+      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+      // one exit decision for every consumer warp, sampled between the two barriers (a warp
+      // that timed out still reaches both) and read after the second
+      if (tid == 0) *consumers_stop = *abort_flag;
+      float* wm = mrg + warp * RW * (D + 2);         // [row][-, l, o'[D]]
+      if (wr) {
+        float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < MT; ++i) {
-        wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = o[i][0];
-        wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = o[i][1];
-        wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][2];
-        wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][3];
-      }
-    }
-    if constexpr (SP) {
-      // the top value dims come from the head M-tile, not from the (zero) tail codes
-      if constexpr (PK) {
-        oh[0] += __shfl_xor_sync(0xffffffffu, oh[0], 2);
-        oh[1] += __shfl_xor_sync(0xffffffffu, oh[1], 2);
-      }
-      __syncwarp();
-      if ((!PK || t < 2) && vh_nb) {
-        wm[(2 * t) * (D + 2) + 2 + g] = oh[0];
-        wm[(2 * t + 1) * (D + 2) + 2 + g] = oh[1];
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
-    for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
-      const int r = idx / D, j = idx - r * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NC; ++w) M = fmaxf(M, mrg[(w * RW + r) * (D + 2)]);
-      float a = 0.f, L = 0.f;
-#pragma unroll
-      for (int w = 0; w < NC; ++w) {
-        const float* row = mrg + (w * RW + r) * (D + 2);
-        const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
-        L += f * row[1];
-        a += f * row[2 + j];
-      }
-      const int64_t qi = qbase + r;
-      const int64_t pi = qi * p.n_chunks + chunk;
-      if (j == 0) { p.part_ml[pi * 2] = M; p.part_ml[pi * 2 + 1] = L; }
-      p.part_o[pi * D + j] = a * p.v_scale;
-    }
-    if constexpr (VPR) {
-      // fold sqrt(pi/2)/m S^T a into the partial: merge the warps' sign-domain sums with the
-      // same chunk weights, then one matrix-vector product per row with S from global memory
-      if constexpr (PK) {
-#pragma unroll
-        for (int i = 0; i < MT; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) os[i][j] += __shfl_xor_sync(0xffffffffu, os[i][j], 2);
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");   // every warp has read mrg
-      if (!PK || t < 2) {
+        for (int w = 0; w < NC; ++w) {
+          M0 = fmaxf(M0, mb[w * RW + 2 * t]);
+          M1 = fmaxf(M1, mb[w * RW + 2 * t + 1]);
+        }
+        // a row this warp never saw (causal masking) keeps max -inf and weight 0
+        const float2 f = make_float2(m0 == -INFINITY ? 0.f : ex2(m0 - M0), m1 == -INFINITY ? 0.f : ex2(m1 - M1));
+        if (g == 0) {
+          wm[(2 * t) * (D + 2) + 1] = l0 * f.x;
+          wm[(2 * t + 1) * (D + 2) + 1] = l1 * f.y;
+        }
 #pragma unroll
         for (int i = 0; i < MT; ++i) {
-          wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = os[i][0];
-          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = os[i][1];
-          wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = os[i][2];
-          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = os[i][3];
+          const float2 x = __fmul2_rn(make_float2(o[i][0], o[i][1]), f);
+          const float2 y = __fmul2_rn(make_float2(o[i][2], o[i][3]), f);
+          wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = x.x;
+          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = x.y;
+          wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = y.x;
+          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = y.y;
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+      for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
+        const int r = idx / D, j = idx - r * D;
+        float s0 = 0.f, s1 = 0.f;                    // two chains over the warps
+#pragma unroll
+        for (int w = 0; w < NC; w += 2) {
+          s0 += mrg[(w * RW + r) * (D + 2) + 2 + j];
+          if (w + 1 < NC) s1 += mrg[((w + 1) * RW + r) * (D + 2) + 2 + j];
+        }
+        const int64_t pi = (qbase + r) * p.n_chunks + chunk;
+        if (j == 0) {
+          float M = -INFINITY, L = 0.f;
+#pragma unroll
+          for (int w = 0; w < NC; ++w) {
+            M = fmaxf(M, mb[w * RW + r]);
+            L += mrg[(w * RW + r) * (D + 2) + 1];
+          }
+          p.part_ml[pi * 2] = M;
+          p.part_ml[pi * 2 + 1] = L;
+        }
+        p.part_o[pi * D + j] = (s0 + s1) * p.v_scale;
+      }
+      // the next writes of mrg come after the next item's first barrier, which every thread
+      // reaches only after this loop
+      if (*consumers_stop) break;
+    } else {
+      float* wm = mrg + warp * RW * (D + 2);           // [row][m, l, o'[D]]
+      if (!PK || t < 2) {
+        if (g == 0) {
+          wm[(2 * t) * (D + 2)] = m0; wm[(2 * t) * (D + 2) + 1] = l0;
+          wm[(2 * t + 1) * (D + 2)] = m1; wm[(2 * t + 1) * (D + 2) + 1] = l1;
+        }
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = o[i][0];
+          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = o[i][1];
+          wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][2];
+          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = o[i][3];
+        }
+      }
+      if constexpr (SP) {
+        // the top value dims come from the head M-tile, not from the (zero) tail codes
+        if constexpr (PK) {
+          oh[0] += __shfl_xor_sync(0xffffffffu, oh[0], 2);
+          oh[1] += __shfl_xor_sync(0xffffffffu, oh[1], 2);
+        }
+        __syncwarp();
+        if ((!PK || t < 2) && vh_nb) {
+          wm[(2 * t) * (D + 2) + 2 + g] = oh[0];
+          wm[(2 * t + 1) * (D + 2) + 2 + g] = oh[1];
         }
       }
       asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
@@ -1220,30 +1249,69 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NC; ++w) M = fmaxf(M, mrg[(w * RW + r) * (D + 2)]);
-        float a = 0.f;
+        float a = 0.f, L = 0.f;
 #pragma unroll
         for (int w = 0; w < NC; ++w) {
           const float* row = mrg + (w * RW + r) * (D + 2);
           const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
+          L += f * row[1];
           a += f * row[2 + j];
         }
-        asum[r * D + j] = a;
+        const int64_t qi = qbase + r;
+        const int64_t pi = qi * p.n_chunks + chunk;
+        if (j == 0) { p.part_ml[pi * 2] = M; p.part_ml[pi * 2 + 1] = L; }
+        p.part_o[pi * D + j] = a * p.v_scale;
       }
-      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
-      for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
-        const int r = idx / D, j = idx - r * D;
-        float c = 0.f;
+      if constexpr (VPR) {
+        // fold sqrt(pi/2)/m S^T a into the partial: merge the warps' sign-domain sums with the
+        // same chunk weights, then one matrix-vector product per row with S from global memory
+        if constexpr (PK) {
+#pragma unroll
+          for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) os[i][j] += __shfl_xor_sync(0xffffffffu, os[i][j], 2);
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");   // every warp has read mrg
+        if (!PK || t < 2) {
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = os[i][0];
+            wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = os[i][1];
+            wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = os[i][2];
+            wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = os[i][3];
+          }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+        for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
+          const int r = idx / D, j = idx - r * D;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < NC; ++w) M = fmaxf(M, mrg[(w * RW + r) * (D + 2)]);
+          float a = 0.f;
+#pragma unroll
+          for (int w = 0; w < NC; ++w) {
+            const float* row = mrg + (w * RW + r) * (D + 2);
+            const float f = (row[0] == -INFINITY) ? 0.f : exp2f(row[0] - M);
+            a += f * row[2 + j];
+          }
+          asum[r * D + j] = a;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+        for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
+          const int r = idx / D, j = idx - r * D;
+          float c = 0.f;
 #pragma unroll 8
-        for (int i = 0; i < D; ++i) c = fmaf(__ldg(p.vS + i * D + j), asum[r * D + i], c);
-        const int64_t pi = (qbase + r) * p.n_chunks + chunk;
-        p.part_o[pi * D + j] += p.v_coef * c;
+          for (int i = 0; i < D; ++i) c = fmaf(__ldg(p.vS + i * D + j), asum[r * D + i], c);
+          const int64_t pi = (qbase + r) * p.n_chunks + chunk;
+          p.part_o[pi * D + j] += p.v_coef * c;
+        }
       }
+      // every consumer warp takes the same exit decision: one thread samples the abort
+      // flag between the two barriers (a warp that timed out still reaches both)
+      if (tid == 0) *consumers_stop = *abort_flag;
+      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+      if (*consumers_stop) break;
     }
-    // every consumer warp takes the same exit decision: one thread samples the abort
-    // flag between the two barriers (a warp that timed out still reaches both)
-    if (tid == 0) *consumers_stop = *abort_flag;
-    asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
-    if (*consumers_stop) break;
   }
 }
 
