@@ -58,11 +58,20 @@ namespace tq {
 #ifndef TQ_DEC_PK_NS
 #define TQ_DEC_PK_NS 2
 #endif
+// Ring depth for MSE keys and values with packed columns.  Three stages fit (the half-size
+// merge buffer and one stage below the 64 KB-aligned table, two after it) but measured no
+// faster than two at the 128k-token shapes: the consumers' instruction stream sets the time.
+#ifndef TQ_DEC_PK_NS_MSE
+#define TQ_DEC_PK_NS_MSE 2
+#endif
 __host__ __device__ constexpr int tma_units(bool pk) { return pk ? TQ_DEC_PK_U : 1; }
 __host__ __device__ constexpr int tma_consumers(int kf, bool pk) { return kf == KFMT_PROD ? 7 : (pk ? TQ_DEC_PK_NC : 11); }
 __host__ __device__ constexpr int tma_stage_tokens(int kf, bool pk) { return tma_consumers(kf, pk) * 16 * tma_units(pk); }
-__host__ __device__ constexpr int tma_stages(bool pk) { return pk ? TQ_DEC_PK_NS : 4; }
-static_assert(TQ_DEC_PK_NS >= 2 && TQ_DEC_PK_NS <= 8, "decode ring depth");
+__host__ __device__ constexpr int tma_stages(int kf, bool pk, bool vpr) {
+  return pk ? ((kf == KFMT_MSE && !vpr) ? TQ_DEC_PK_NS_MSE : TQ_DEC_PK_NS) : 4;
+}
+static_assert(TQ_DEC_PK_NS >= 2 && TQ_DEC_PK_NS <= 4 && TQ_DEC_PK_NS_MSE >= 2 && TQ_DEC_PK_NS_MSE <= 4,
+              "decode ring depth");
 constexpr int kTmaHeadBlock = 8;     // query heads per work item (MMA N)
 
 __device__ __forceinline__ uint32_t tma_smem_u32(const void* p) {
@@ -141,8 +150,13 @@ __host__ __device__ inline uint32_t tma_table_bytes(int kb, int vb) {
   return (kb <= 2 || vb <= 2) ? 65536u : (1u << (2 * (kb > vb ? kb : vb))) * 256u;
 }
 __host__ __device__ constexpr uint32_t tma_merge_rows(bool pk) { return pk ? 4u : 8u; }
+// Floats per merge row: m, l and o'[128] for the spectral and values-as-prod merge; l and
+// half of o' for the others, whose merge runs in two halves of the dims.
+__host__ __device__ constexpr uint32_t tma_merge_row_floats(int kf, bool vpr) {
+  return (kf == KFMT_SPEC || vpr) ? 128u + 2u : 64u + 1u;
+}
 __host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk, bool vpr = false) {
-  const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf, pk)) * tma_merge_rows(pk) * (128u + 2u) * 4u;
+  const uint32_t merge = static_cast<uint32_t>(tma_consumers(kf, pk)) * tma_merge_rows(pk) * tma_merge_row_floats(kf, vpr) * 4u;
   // values as prod: the merged sign-domain sums of up to 8 rows
   const uint32_t v = merge + 4u * 32u * 4u + 2u * 4u * 8u + 2u * 4u * 4u + 16u + 1024u * 4u + 8u + (vpr ? 8u * 128u * 4u : 0u);
   return (v + 127u) & ~127u;
@@ -151,7 +165,7 @@ __host__ __device__ inline uint32_t tma_misc_bytes(int kf, bool pk, bool vpr = f
 __host__ __device__ constexpr int tma_record_words(int bits, int kf) { return 128 * bits / 32 + (kf == KFMT_SPEC ? 1 : 0); }
 inline size_t decode_tma_smem_bytes(int kb, int vb, int kf, bool pk, bool vpr = false) {
   const TmaStageLayout L = tma_stage_layout(tma_record_words(kb, kf), tma_record_words(vb, kf), kf, 4, pk, vpr);
-  const size_t want = 65536 + tma_table_bytes(kb, vb) + static_cast<size_t>(tma_stages(pk)) * L.bytes +
+  const size_t want = 65536 + tma_table_bytes(kb, vb) + static_cast<size_t>(tma_stages(kf, pk, vpr)) * L.bytes +
                       tma_misc_bytes(kf, pk, vpr);
   return want < 232448 ? want : 232448;
 }
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__((tma_consumers(KF, PK) + 1) * 32, 1)
 decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   constexpr int NC = tma_consumers(KF, PK);   // consumer warps
   constexpr int U = tma_units(PK);            // 16-token units per consumer warp per stage
-  constexpr int NS = tma_stages(PK);          // ring stages
+  constexpr int NS = tma_stages(KF, PK, VPR);  // ring stages
   constexpr int kTmaThreads = (NC + 1) * 32;
   constexpr int kTmaStageTokens = tma_stage_tokens(KF, PK);
   constexpr int D = 128;
@@ -322,8 +336,8 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
   };
   auto gen = [&](uint32_t a) { return tsm_ + (a - base); };   // generic pointer of a shared address
   uint32_t* tab_g = reinterpret_cast<uint32_t*>(gen(tabA));
-  float* mrg = reinterpret_cast<float*>(gen(miscA));             // [warp][RW rows][m, l, o'[D]]
-  const uint32_t mrg_bytes = NC * RW * (D + 2) * 4;
+  float* mrg = reinterpret_cast<float*>(gen(miscA));             // [warp][RW rows][merge row]
+  const uint32_t mrg_bytes = NC * RW * tma_merge_row_floats(KF, VPR) * 4;
   uint32_t* luts = reinterpret_cast<uint32_t*>(gen(miscA + mrg_bytes));
   const uint32_t luts_a = miscA + mrg_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gen(miscA + mrg_bytes + 512));
@@ -1167,7 +1181,11 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
       // one exit decision for every consumer warp, sampled between the two barriers (a warp
       // that timed out still reaches both) and read after the second
       if (tid == 0) *consumers_stop = *abort_flag;
-      float* wm = mrg + warp * RW * (D + 2);         // [row][-, l, o'[D]]
+      // the partials go through the buffer in two halves of the dims: half hf holds dims
+      // TDV g + 8 hf + i (i < 8) of every lane group g at local index 8 g + i, after l
+      constexpr int HW = D / 2 + 1;
+      float* wm = mrg + warp * RW * HW;              // [row][l, o' half]
+      float2 f = make_float2(0.f, 0.f);
       if (wr) {
         float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
@@ -1176,42 +1194,46 @@ decode_tma_kernel(const DecodeParams p, int* status, long long wait_lim) {
           M1 = fmaxf(M1, mb[w * RW + 2 * t + 1]);
         }
         // a row this warp never saw (causal masking) keeps max -inf and weight 0
-        const float2 f = make_float2(m0 == -INFINITY ? 0.f : ex2(m0 - M0), m1 == -INFINITY ? 0.f : ex2(m1 - M1));
+        f = make_float2(m0 == -INFINITY ? 0.f : ex2(m0 - M0), m1 == -INFINITY ? 0.f : ex2(m1 - M1));
         if (g == 0) {
-          wm[(2 * t) * (D + 2) + 1] = l0 * f.x;
-          wm[(2 * t + 1) * (D + 2) + 1] = l1 * f.y;
-        }
-#pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          const float2 x = __fmul2_rn(make_float2(o[i][0], o[i][1]), f);
-          const float2 y = __fmul2_rn(make_float2(o[i][2], o[i][3]), f);
-          wm[(2 * t) * (D + 2) + 2 + TDV * g + i] = x.x;
-          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + i] = x.y;
-          wm[(2 * t) * (D + 2) + 2 + TDV * g + 8 + i] = y.x;
-          wm[(2 * t + 1) * (D + 2) + 2 + TDV * g + 8 + i] = y.y;
+          wm[(2 * t) * HW] = l0 * f.x;
+          wm[(2 * t + 1) * HW] = l1 * f.y;
         }
       }
-      asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
-      for (int idx = tid; idx < nh * D; idx += CONSUMERS) {
-        const int r = idx / D, j = idx - r * D;
-        float s0 = 0.f, s1 = 0.f;                    // two chains over the warps
 #pragma unroll
-        for (int w = 0; w < NC; w += 2) {
-          s0 += mrg[(w * RW + r) * (D + 2) + 2 + j];
-          if (w + 1 < NC) s1 += mrg[((w + 1) * RW + r) * (D + 2) + 2 + j];
-        }
-        const int64_t pi = (qbase + r) * p.n_chunks + chunk;
-        if (j == 0) {
-          float M = -INFINITY, L = 0.f;
+      for (int hf = 0; hf < 2; ++hf) {
+        if (hf) asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");   // first half read
+        if (wr) {
 #pragma unroll
-          for (int w = 0; w < NC; ++w) {
-            M = fmaxf(M, mb[w * RW + r]);
-            L += mrg[(w * RW + r) * (D + 2) + 1];
+          for (int i = 0; i < MT; ++i) {
+            const float2 x = __fmul2_rn(make_float2(o[i][2 * hf], o[i][2 * hf + 1]), f);
+            wm[(2 * t) * HW + 1 + 8 * g + i] = x.x;
+            wm[(2 * t + 1) * HW + 1 + 8 * g + i] = x.y;
           }
-          p.part_ml[pi * 2] = M;
-          p.part_ml[pi * 2 + 1] = L;
         }
-        p.part_o[pi * D + j] = (s0 + s1) * p.v_scale;
+        asm volatile("bar.sync 1, %0;" ::"r"(CONSUMERS) : "memory");
+        for (int idx = tid; idx < nh * (D / 2); idx += CONSUMERS) {
+          const int r = idx / (D / 2), jl = idx - r * (D / 2);
+          const int j = TDV * (jl >> 3) + 8 * hf + (jl & 7);
+          float s0 = 0.f, s1 = 0.f;                  // two chains over the warps
+#pragma unroll
+          for (int w = 0; w < NC; w += 2) {
+            s0 += mrg[(w * RW + r) * HW + 1 + jl];
+            if (w + 1 < NC) s1 += mrg[((w + 1) * RW + r) * HW + 1 + jl];
+          }
+          const int64_t pi = (qbase + r) * p.n_chunks + chunk;
+          if (hf == 0 && jl == 0) {
+            float M = -INFINITY, L = 0.f;
+#pragma unroll
+            for (int w = 0; w < NC; ++w) {
+              M = fmaxf(M, mb[w * RW + r]);
+              L += mrg[(w * RW + r) * HW];
+            }
+            p.part_ml[pi * 2] = M;
+            p.part_ml[pi * 2 + 1] = L;
+          }
+          p.part_o[pi * D + j] = (s0 + s1) * p.v_scale;
+        }
       }
       // the next writes of mrg come after the next item's first barrier, which every thread
       // reaches only after this loop
