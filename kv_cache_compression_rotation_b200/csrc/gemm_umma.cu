@@ -113,6 +113,72 @@ __global__ void __launch_bounds__(256) expand_records_kernel(const uint32_t* __r
   }
 }
 
+// The same records, 8 consecutive values per lane and step with one 16-byte store of each
+// part: d and m multiples of 8, hi and lo 16-byte aligned.  The hi / lo rounding is that of
+// expand_records_kernel value by value.
+template <int B>
+__global__ void __launch_bounds__(256) expand_records8_kernel(const uint32_t* __restrict__ codes, int code_words,
+                                                              const uint32_t* __restrict__ signs, int sign_words,
+                                                              const float* __restrict__ rnorms,
+                                                              const float* __restrict__ centroids, float coef,
+                                                              int64_t n, int d, int m, uint16_t* __restrict__ hi,
+                                                              uint16_t* __restrict__ lo) {
+  constexpr uint32_t kMask = (1u << B) - 1u;
+  __shared__ float cs[1 << B];
+  if (threadIdx.x < (1u << B)) cs[threadIdx.x] = __ldg(centroids + threadIdx.x);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t rec = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (rec >= n) return;
+  const int64_t k = d + m;
+  const uint32_t* cw = codes + rec * code_words;
+  uint4* h = reinterpret_cast<uint4*>(hi + rec * k);
+  uint4* l = reinterpret_cast<uint4*>(lo + rec * k);
+  for (int gi = lane; gi < d / 8; gi += 32) {
+    // codes of dims 8 gi .. 8 gi + 7: 8 B bits from bit 8 gi B of the stream
+    const int pos = gi * 8 * B, w = pos >> 5, sh = pos & 31;
+    uint32_t bits = cw[w] >> sh;
+    if (sh + 8 * B > 32) bits |= cw[w + 1] << (32 - sh);
+    uint32_t hv[4], lv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = cs[(bits >> (2 * j * B)) & kMask];
+      const float b = cs[(bits >> ((2 * j + 1) * B)) & kMask];
+      const __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+      const float2 back = __bfloat1622float2(hb);
+      const __nv_bfloat162 lb = __floats2bfloat162_rn(a - back.x, b - back.y);
+      hv[j] = *reinterpret_cast<const uint32_t*>(&hb);
+      lv[j] = *reinterpret_cast<const uint32_t*>(&lb);
+    }
+    h[gi] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    l[gi] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+  }
+  if (m > 0) {
+    const float g = coef * rnorms[rec];
+    const __nv_bfloat16 gh = __float2bfloat16_rn(g);
+    const __nv_bfloat16 gl = __float2bfloat16_rn(g - __bfloat162float(gh));
+    const uint32_t ph = __bfloat16_as_ushort(gh), pl = __bfloat16_as_ushort(gl);
+    const uint32_t ph2 = ph | (ph << 16), pl2 = pl | (pl << 16);
+    // byte gi of the sign words holds signs 8 gi .. 8 gi + 7 (LSB first)
+    const unsigned char* sb = reinterpret_cast<const unsigned char*>(signs + rec * sign_words);
+    uint4* h2 = reinterpret_cast<uint4*>(hi + rec * k + d);
+    uint4* l2 = reinterpret_cast<uint4*>(lo + rec * k + d);
+    for (int gi = lane; gi < m / 8; gi += 32) {
+      const uint32_t ns = ~static_cast<uint32_t>(sb[gi]);   // set bit: a negative sign
+      uint32_t hv[4], lv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // -x flips the sign bit of a bf16 (gamma >= 0): bit 15 of the low half, 31 of the high
+        const uint32_t flip = (((ns >> (2 * j)) & 1u) << 15) | (((ns >> (2 * j + 1)) & 1u) << 31);
+        hv[j] = ph2 ^ flip;
+        lv[j] = pl2 ^ flip;
+      }
+      h2[gi] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      l2[gi] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_split_cat(const float* a, int da, const float* b, int db, int64_t rows, uint16_t* hi,
@@ -126,6 +192,17 @@ cudaError_t launch_expand_records(const uint32_t* codes, int code_words, const u
                                   const float* rnorms, const float* centroids, float coef, int64_t n, int d, int m,
                                   int bits, uint16_t* hi, uint16_t* lo, cudaStream_t s) {
   const unsigned blocks = static_cast<unsigned>((n + 7) / 8);
+  const bool vec = d % 8 == 0 && m % 8 == 0 && ((reinterpret_cast<uintptr_t>(hi) | reinterpret_cast<uintptr_t>(lo)) & 15u) == 0;
+  if (vec) {
+    switch (bits) {
+      case 1: expand_records8_kernel<1><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
+      case 2: expand_records8_kernel<2><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
+      case 3: expand_records8_kernel<3><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
+      case 4: expand_records8_kernel<4><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
+      default: return cudaErrorNotSupported;
+    }
+    return cudaGetLastError();
+  }
   switch (bits) {
     case 1: expand_records_kernel<1><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
     case 2: expand_records_kernel<2><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;

@@ -213,4 +213,112 @@ __global__ void __launch_bounds__(128) topk_kernel(const float* scores, int64_t 
   }
 }
 
+// y[i][j] = sum_k A[j][k] x[i][k] for queries i < nx and rows j < rows (A fp32 [rows][d], x
+// [nx][ldx] in the given dtype, d a multiple of 128): the query rotation and projection of the
+// tensor-core estimator.  A block takes kMvQ queries (in shared memory) and kMvRows rows, one
+// warp per row at a time: the lanes read the row with coalesced 16-byte loads and reduce the
+// kMvQ dot products with shuffles.
+constexpr int kMvQ = 8, kMvRows = 32;
+__global__ void __launch_bounds__(128) rows_matvec_kernel(const float* __restrict__ A, int rows, int d,
+                                                          const void* x, int dtype, int64_t nx, int64_t ldx,
+                                                          float* __restrict__ y, int64_t ldy) {
+  extern __shared__ __align__(16) float xs[];      // [kMvQ][d]
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * kMvQ;
+  for (int e = threadIdx.x; e < kMvQ * d; e += 128) {
+    const int qi = e / d, k = e - qi * d;
+    xs[e] = (i0 + qi < nx) ? load_elem(x, dtype, (i0 + qi) * ldx + k) : 0.f;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float4* xs4 = reinterpret_cast<const float4*>(xs);
+#pragma unroll 1
+  for (int jj = 0; jj < kMvRows / 4; ++jj) {
+    const int j = blockIdx.x * kMvRows + warp * (kMvRows / 4) + jj;
+    if (j >= rows) break;
+    const float4* a4 = reinterpret_cast<const float4*>(A + static_cast<int64_t>(j) * d);
+    float acc[kMvQ];
+#pragma unroll
+    for (int qi = 0; qi < kMvQ; ++qi) acc[qi] = 0.f;
+    for (int k4 = lane; k4 < d / 4; k4 += 32) {
+      const float4 a = __ldg(a4 + k4);
+#pragma unroll
+      for (int qi = 0; qi < kMvQ; ++qi) {
+        const float4 v = xs4[qi * (d / 4) + k4];
+        acc[qi] = fmaf(a.x, v.x, fmaf(a.y, v.y, fmaf(a.z, v.z, fmaf(a.w, v.w, acc[qi]))));
+      }
+    }
+    float mine = 0.f;                               // lane qi keeps query qi's sum
+#pragma unroll
+    for (int qi = 0; qi < kMvQ; ++qi) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[qi] += __shfl_xor_sync(0xffffffffu, acc[qi], o);
+      if (lane == qi) mine = acc[qi];
+    }
+    if (lane < kMvQ && i0 + lane < nx) y[(i0 + lane) * ldy + j] = mine;
+  }
+}
+
+// Top-K of row segments: CTA (s, r) takes candidates [s L, min((s + 1) L, len)) of row r,
+// scores from `scores` and ids from `ids` (or the positions when ids is null), and writes its
+// best k_out in the order of the whole search (descending score, ascending id) to
+// out[((out_row0 + r) * gridDim.x + s) * k_out ..].  Run over the dense rows in segments and
+// then once over the segments' K candidates, it gives the same top-k as one pass over the row
+// (every member of the row's top-k is in its segment's top-K).
+template <int K>
+__global__ void __launch_bounds__(128) topk_seg_kernel(const float* scores, const int32_t* ids, int64_t len,
+                                                       int64_t seg, int k_out, float* out_s, int32_t* out_i,
+                                                       int64_t out_row0) {
+  __shared__ float ss[128][K];
+  __shared__ int32_t si[128][K];
+  const int64_t r = blockIdx.y, b = static_cast<int64_t>(blockIdx.x) * seg;
+  const int64_t e = min(len, b + seg);
+  const float* row = scores + r * len;
+  const int32_t* idr = ids ? ids + r * len : nullptr;
+  float bs[K];
+  int32_t bi[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) { bs[i] = -INFINITY; bi[i] = 0x7fffffff; }
+  for (int64_t j = b + threadIdx.x; j < e; j += 128) {
+    const float s = row[j];
+    const int32_t id = idr ? idr[j] : static_cast<int32_t>(j);
+    if (s > bs[K - 1] || (s == bs[K - 1] && id < bi[K - 1])) {
+      float cs = s;
+      int32_t ci = id;
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        const bool better = cs > bs[i] || (cs == bs[i] && ci < bi[i]);
+        if (better) {
+          const float ts = bs[i]; const int32_t ti = bi[i];
+          bs[i] = cs; bi[i] = ci; cs = ts; ci = ti;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < K; ++i) { ss[threadIdx.x][i] = bs[i]; si[threadIdx.x][i] = bi[i]; }
+  __syncthreads();
+  for (int stride = 64; stride > 0; stride >>= 1) {
+    if (threadIdx.x < stride) {
+      const int a = threadIdx.x, c = threadIdx.x + stride;
+      float ms[K];
+      int32_t mi[K];
+      int ia = 0, ic = 0;
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        const bool takeA = ss[a][ia] > ss[c][ic] || (ss[a][ia] == ss[c][ic] && si[a][ia] < si[c][ic]);
+        if (takeA) { ms[i] = ss[a][ia]; mi[i] = si[a][ia]; ++ia; }
+        else { ms[i] = ss[c][ic]; mi[i] = si[c][ic]; ++ic; }
+      }
+#pragma unroll
+      for (int i = 0; i < K; ++i) { ss[a][i] = ms[i]; si[a][i] = mi[i]; }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < k_out) {
+    const int64_t o = ((out_row0 + r) * gridDim.x + blockIdx.x) * k_out + threadIdx.x;
+    out_s[o] = ss[0][threadIdx.x];
+    out_i[o] = si[0][threadIdx.x];
+  }
+}
+
 }  // namespace tq

@@ -895,10 +895,17 @@ static bool score_wide(const tq_quantizer* q, int64_t n) {
 }
 
 struct ScoreWidePlan {
-  size_t qr, qu, ah, al, bh, bl, dense, bytes;
+  size_t qr, qu, ah, al, bh, bl, dense, cand, bytes;
   int64_t qb;
   int K;
+  int seg_n;                    // top-k segments per dense row
 };
+
+// Top-k over a dense row runs in segments of ~16k estimates (one CTA each), then over the
+// segments' candidates.
+static int topk_segments(int64_t n) {
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(64, (n + 16383) / 16384)));
+}
 
 static ScoreWidePlan plan_score_wide(const tq_quantizer* q, int64_t nq, int64_t n, int topk) {
   ScoreWidePlan P{};
@@ -916,6 +923,8 @@ static ScoreWidePlan plan_score_wide(const tq_quantizer* q, int64_t nq, int64_t 
   P.bh = off; off = al(off + n * P.K * 2);
   P.bl = off; off = al(off + n * P.K * 2);
   P.dense = off; off = al(off + (topk > 0 ? P.qb * n * 4 : 0));
+  P.seg_n = topk_segments(n);
+  P.cand = off; off = al(off + (topk > 0 ? P.qb * P.seg_n * 32 * 8 : 0));   // scores, then ids
   P.bytes = off;
   return P;
 }
@@ -1000,10 +1009,20 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
     float* qu = reinterpret_cast<float*>(ws + P.qu);
     const int m = q->kind == TQ_KIND_PROD ? q->m : 0;
     auto u16 = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
-    score_qprep_kernel<<<static_cast<unsigned>(nq), 128, 2 * d * 4, stream>>>(
-        qv, dtype, d, q->kind, q->rot, q->S, q->m, q->k_top, qr, m ? qu : nullptr, qus, d, nullptr, device_status_ptr());
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "score qprep launch");
+    // q' = Pi q and S q' (PROD), fp32
+    const size_t mv_smem = static_cast<size_t>(kMvQ) * d * 4;
+    cudaError_t e = cudaFuncSetAttribute(rows_matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(mv_smem));
+    if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
+    const dim3 mv_grid(static_cast<unsigned>((d + kMvRows - 1) / kMvRows), static_cast<unsigned>((nq + kMvQ - 1) / kMvQ));
+    if (mv_grid.y > 65535) return fail(TQ_ERR_UNSUPPORTED, "too many queries");
+    rows_matvec_kernel<<<mv_grid, 128, mv_smem, stream>>>(q->rot, d, d, qv, dtype, nq, d, qr, d);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "query rotation launch");
+    if (m) {
+      const dim3 sg(static_cast<unsigned>((m + kMvRows - 1) / kMvRows), mv_grid.y);
+      rows_matvec_kernel<<<sg, 128, mv_smem, stream>>>(q->S, m, d, qr, TQ_F32, nq, d, qu, qus);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "query projection launch");
+    }
     const int bm = q->kind == TQ_KIND_PROD ? q->bits - 1 : q->bits;
     const float coef = m ? static_cast<float>(std::sqrt(M_PI / 2.0) / m) : 0.f;
     e = launch_expand_records(keys.codes, L.code_words, keys.signs, L.sign_words, keys.rnorms, q->centroids, coef, n,
@@ -1027,8 +1046,21 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
       e = launch_split_gemm(maps, g, GEMM_EPI_SCORE, 1, static_cast<int>(std::min<int64_t>(work, sm_count())), stream);
       if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
       if (topk > 0) {
-        if (topk <= 16) topk_kernel<16><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
-        else topk_kernel<32><<<static_cast<unsigned>(nb), 128, 0, stream>>>(dense, n, topk, q0, scores, ids);
+        // the segments' best K (pass 1), then the top-k of those candidates (pass 2)
+        const int S = P.seg_n;
+        const int64_t seg = (n + S - 1) / S;
+        float* cs = reinterpret_cast<float*>(ws + P.cand);
+        int32_t* ci = reinterpret_cast<int32_t*>(ws + P.cand + static_cast<size_t>(P.qb) * S * 32 * 4);
+        const dim3 g1(static_cast<unsigned>(S), static_cast<unsigned>(nb)), g2(1, static_cast<unsigned>(nb));
+        if (topk <= 16) {
+          topk_seg_kernel<16><<<g1, 128, 0, stream>>>(dense, nullptr, n, seg, 16, cs, ci, 0);
+          topk_seg_kernel<16><<<g2, 128, 0, stream>>>(cs, ci, static_cast<int64_t>(S) * 16, static_cast<int64_t>(S) * 16,
+                                                      topk, scores, ids, q0);
+        } else {
+          topk_seg_kernel<32><<<g1, 128, 0, stream>>>(dense, nullptr, n, seg, 32, cs, ci, 0);
+          topk_seg_kernel<32><<<g2, 128, 0, stream>>>(cs, ci, static_cast<int64_t>(S) * 32, static_cast<int64_t>(S) * 32,
+                                                      topk, scores, ids, q0);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
       }
     }
