@@ -108,3 +108,31 @@ def test_scores_wide_tensor_core(d, kind, bits, n, nq):
         idx, _ = adopt_mse(as_u32(pk.codes), ref, bits, t)
         est = OQ.estimate_mse(qv.astype(np.float64), rot, idx, ref["norms"], c)
     assert np.max(np.abs(s - est)) <= 1e-3
+
+
+def test_topk_segments_ties():
+    """The tensor-core path takes the top-k over segments of ~16k estimates and then over their
+    candidates; the result must be that of one pass over the row: descending estimate, ties to
+    the lower id.  n = 40,000 makes three segments (boundaries at 13,334 and 26,668); one record
+    is copied to ids in all three and is query 0, so its copies tie at the top.  The reference is
+    a host top-k of the same call's dense estimates."""
+    d, n, nq, k = 256, 40000, 6, 12
+    rot = ti.haar_rotation(d, 1406)
+    x = ti.unit_gaussian(n, d, 8102).astype(np.float32)
+    dup = [5, 123, 13333, 13334, 20000, 26668, 39999]
+    x[dup] = x[123]
+    qv = ti.unit_gaussian(nq, d, 8103).astype(np.float32)
+    qv[0] = x[123]
+    q = K.Quantizer.mse(rot, 3)
+    pk = K.quantize(q, torch.from_numpy(x).cuda())
+    qt = torch.from_numpy(qv).cuda()
+    dense = K.score(q, qt, pk, n).cpu().numpy()
+    vals, ids = K.score(q, qt, pk, n, topk=k)
+    vals, ids = vals.cpu().numpy(), ids.cpu().numpy()
+    assert K.get_status() == 0
+    for i in range(nq):
+        order = np.lexsort((np.arange(n), -dense[i].astype(np.float64)))[:k]
+        assert ids[i].tolist() == order.tolist(), f"query {i}"
+        assert np.array_equal(vals[i], dense[i, order])
+    # the copies carry equal records, hence equal estimates, and lead query 0 in id order
+    assert ids[0][:len(dup)].tolist() == sorted(dup)
