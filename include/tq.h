@@ -366,6 +366,9 @@ tq_status tq_score_workspace(const tq_quantizer* q, int64_t nq, int64_t n, int32
  * topk == 0: scores [nq*n] fp32 dense, ids unused.  topk in 1..32: for each query the
  * topk records by descending estimate, ties to the lower id: ids [nq*topk] int32,
  * scores [nq*topk].  workspace: device, >= tq_score_workspace bytes.
+ * From 4096 records with d a multiple of 128 (MSE 1..4 bits, PROD 2..5 bits with m = d) the
+ * estimates are one split-precision tensor-core product; its top-k keeps the best of
+ * segments of ~16k estimates and then of their candidates (the one-pass result).
  */
 tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t nq,
                    tq_packed keys, int64_t n, int32_t topk, float* scores, int32_t* ids,
