@@ -58,16 +58,19 @@ cudaError_t go(const CUtensorMap* maps, const SplitGemmParams& p, int grid, cuda
 }
 
 // Queries for the tensor-core estimator: row r of [qr | qu] (fp32, d + m columns) as bf16
-// hi + lo parts.
+// hi + lo parts.  While *sym is nonzero (records expanded as +-1 in units of c[1]) the qr
+// columns carry that centroid.
 __global__ void __launch_bounds__(256) split_cat_kernel(const float* __restrict__ a, int da,
                                                         const float* __restrict__ b, int db, int64_t rows,
-                                                        uint16_t* __restrict__ hi, uint16_t* __restrict__ lo) {
+                                                        uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
+                                                        const int* sym, const float* centroids) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const int k = da + db;
   if (i >= rows * k) return;
   const int64_t r = i / k;
   const int c = static_cast<int>(i - r * k);
-  const float v = c < da ? a[r * da + c] : b[r * db + (c - da)];
+  const float sa = (sym && *sym) ? __ldg(centroids + 1) : 1.f;
+  const float v = c < da ? a[r * da + c] * sa : b[r * db + (c - da)];
   const __nv_bfloat16 h = __float2bfloat16_rn(v);
   hi[i] = __bfloat16_as_ushort(h);
   lo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
@@ -115,18 +118,22 @@ __global__ void __launch_bounds__(256) expand_records_kernel(const uint32_t* __r
 
 // The same records, 8 consecutive values per lane and step with one 16-byte store of each
 // part: d and m multiples of 8, hi and lo 16-byte aligned.  The hi / lo rounding is that of
-// expand_records_kernel value by value.
+// expand_records_kernel value by value.  1-bit codes with c[0] = -c[1] (sym_flag given):
+// the d code columns are written as exactly +-1 (units of c[1], which the queries then
+// carry) with no lo part, and *sym_flag = 1 tells the query split and the product so.
 template <int B>
 __global__ void __launch_bounds__(256) expand_records8_kernel(const uint32_t* __restrict__ codes, int code_words,
                                                               const uint32_t* __restrict__ signs, int sign_words,
                                                               const float* __restrict__ rnorms,
                                                               const float* __restrict__ centroids, float coef,
                                                               int64_t n, int d, int m, uint16_t* __restrict__ hi,
-                                                              uint16_t* __restrict__ lo) {
+                                                              uint16_t* __restrict__ lo, int* sym_flag) {
   constexpr uint32_t kMask = (1u << B) - 1u;
   __shared__ float cs[1 << B];
   if (threadIdx.x < (1u << B)) cs[threadIdx.x] = __ldg(centroids + threadIdx.x);
   __syncthreads();
+  const bool sym = B == 1 && sym_flag != nullptr && cs[0] == -cs[1];
+  if (sym_flag && blockIdx.x == 0 && threadIdx.x == 0) *sym_flag = sym ? 1 : 0;
   const int lane = threadIdx.x & 31;
   const int64_t rec = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (rec >= n) return;
@@ -139,6 +146,15 @@ __global__ void __launch_bounds__(256) expand_records8_kernel(const uint32_t* __
     const int pos = gi * 8 * B, w = pos >> 5, sh = pos & 31;
     uint32_t bits = cw[w] >> sh;
     if (sh + 8 * B > 32) bits |= cw[w + 1] << (32 - sh);
+    if (sym) {
+      // bf16 -1 is 0xBF80; code 1 (+1) clears the sign bit
+      uint32_t hv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        hv[j] = 0xBF80BF80u ^ (((bits >> (2 * j)) & 1u) << 15) ^ (((bits >> (2 * j + 1)) & 1u) << 31);
+      h[gi] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      continue;
+    }
     uint32_t hv[4], lv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -182,26 +198,32 @@ __global__ void __launch_bounds__(256) expand_records8_kernel(const uint32_t* __
 }  // namespace
 
 cudaError_t launch_split_cat(const float* a, int da, const float* b, int db, int64_t rows, uint16_t* hi,
-                             uint16_t* lo, cudaStream_t s) {
+                             uint16_t* lo, cudaStream_t s, const int* sym, const float* centroids) {
   const int64_t total = rows * (da + db);
-  split_cat_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(a, da, b, db, rows, hi, lo);
+  split_cat_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(a, da, b, db, rows, hi, lo, sym,
+                                                                                centroids);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expand_records(const uint32_t* codes, int code_words, const uint32_t* signs, int sign_words,
                                   const float* rnorms, const float* centroids, float coef, int64_t n, int d, int m,
-                                  int bits, uint16_t* hi, uint16_t* lo, cudaStream_t s) {
+                                  int bits, uint16_t* hi, uint16_t* lo, int* sym_flag, cudaStream_t s) {
   const unsigned blocks = static_cast<unsigned>((n + 7) / 8);
   const bool vec = d % 8 == 0 && m % 8 == 0 && ((reinterpret_cast<uintptr_t>(hi) | reinterpret_cast<uintptr_t>(lo)) & 15u) == 0;
   if (vec) {
     switch (bits) {
-      case 1: expand_records8_kernel<1><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
-      case 2: expand_records8_kernel<2><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
-      case 3: expand_records8_kernel<3><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
-      case 4: expand_records8_kernel<4><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;
+      case 1: expand_records8_kernel<1><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo, sym_flag); break;
+      case 2: expand_records8_kernel<2><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo, sym_flag); break;
+      case 3: expand_records8_kernel<3><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo, sym_flag); break;
+      case 4: expand_records8_kernel<4><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo, sym_flag); break;
       default: return cudaErrorNotSupported;
     }
     return cudaGetLastError();
+  }
+  // the value-by-value kernel always writes both parts
+  if (sym_flag) {
+    const cudaError_t e = cudaMemsetAsync(sym_flag, 0, sizeof(int), s);
+    if (e != cudaSuccess) return e;
   }
   switch (bits) {
     case 1: expand_records_kernel<1><<<blocks, 256, 0, s>>>(codes, code_words, signs, sign_words, rnorms, centroids, coef, n, d, m, hi, lo); break;

@@ -72,6 +72,10 @@ struct SplitGemmParams {
   float* out;              // [M][ldo]
   int64_t ldo;
   const float* col_scale;  // [N]
+  // SCORE: while *lo_skip_flag is nonzero the B lo part is zero in columns [0, lo_skip_k) of
+  // K (records exactly +-1 there), so those lo loads and their products are not issued
+  const int* lo_skip_flag;
+  int lo_skip_k;           // multiple of 64
 };
 
 // Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = tn.
@@ -114,6 +118,8 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
   const int n_tiles = (p.N + kGemmTileN - 1) / kGemmTileN;
   const int64_t n_work = m_tiles * n_tiles;
   const int k_steps = p.K / kGemmTileK;
+  // first K column whose B lo part is read (a flag written by the record expansion)
+  const int k_lo0 = (EPI == GEMM_EPI_SCORE && p.lo_skip_flag && *p.lo_skip_flag) ? p.lo_skip_k : 0;
 
   if constexpr (EPI == GEMM_EPI_QUANT) {
     if (tid < NB) tab[tid] = __ldg(p.boundaries + tid);
@@ -147,13 +153,14 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
         for (int ks = 0; ks < k_steps; ++ks, ++it) {
           const int s = it % NS, use = it / NS;
           if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, lim, p.status, abort_flag)) { stop = true; break; }
-          mbar_expect_tx(full_bar(s), kGemmStageBytes);
           const uint32_t st = base + s * kGemmStageBytes;
           const int k0 = ks * kGemmTileK;
+          const bool lo = k0 >= k_lo0;
+          mbar_expect_tx(full_bar(s), lo ? kGemmStageBytes : kGemmStageBytes - kGemmBStage);
           tma_load_2d_g(st, &a_hi, k0, row, full_bar(s));
           tma_load_2d_g(st + kGemmAStage, &a_lo, k0, row, full_bar(s));
           tma_load_2d_g(st + 2 * kGemmAStage, &b_hi, k0, col, full_bar(s));
-          tma_load_2d_g(st + 2 * kGemmAStage + kGemmBStage, &b_lo, k0, col, full_bar(s));
+          if (lo) tma_load_2d_g(st + 2 * kGemmAStage + kGemmBStage, &b_lo, k0, col, full_bar(s));
           ++issued;
         }
       }
@@ -177,12 +184,13 @@ split_gemm_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constan
           tc_fence_after();
           const uint32_t st = base + s * kGemmStageBytes;
           const uint32_t ah = st, al = st + kGemmAStage, bh = st + 2 * kGemmAStage, bl = bh + kGemmBStage;
+          const bool lo = ks * kGemmTileK >= k_lo0;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t ko = kk * 32;
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             umma_f16(td, sw128_desc(ah + ko), sw128_desc(bh + ko), idesc, acc);
-            umma_f16(td, sw128_desc(ah + ko), sw128_desc(bl + ko), idesc, 1u);
+            if (lo) umma_f16(td, sw128_desc(ah + ko), sw128_desc(bl + ko), idesc, 1u);
             umma_f16(td, sw128_desc(al + ko), sw128_desc(bh + ko), idesc, 1u);
           }
           umma_commit(empty_bar(s));

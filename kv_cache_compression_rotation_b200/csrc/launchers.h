@@ -59,10 +59,10 @@ cudaError_t launch_split_gemm(const CUtensorMap* maps, const SplitGemmParams& p,
 // Tensor-core estimator operands: [a | b] rows as bf16 hi + lo; records decoded to
 // [c[code] | coef * gamma * (2s - 1)] rows as bf16 hi + lo.
 cudaError_t launch_split_cat(const float* a, int da, const float* b, int db, int64_t rows, uint16_t* hi,
-                             uint16_t* lo, cudaStream_t s);
+                             uint16_t* lo, cudaStream_t s, const int* sym = nullptr, const float* centroids = nullptr);
 cudaError_t launch_expand_records(const uint32_t* codes, int code_words, const uint32_t* signs, int sign_words,
                                   const float* rnorms, const float* centroids, float coef, int64_t n, int d, int m,
-                                  int bits, uint16_t* hi, uint16_t* lo, cudaStream_t s);
+                                  int bits, uint16_t* hi, uint16_t* lo, int* sym_flag, cudaStream_t s);
 // fp32 rows -> bf16 hi + lo parts (and row norms when norms != nullptr).
 cudaError_t launch_split_rows(const float* x, int64_t rows, int d, uint16_t* hi, uint16_t* lo, float* norms,
                               cudaStream_t s);

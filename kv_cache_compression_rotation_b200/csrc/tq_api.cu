@@ -895,7 +895,7 @@ static bool score_wide(const tq_quantizer* q, int64_t n) {
 }
 
 struct ScoreWidePlan {
-  size_t qr, qu, ah, al, bh, bl, dense, cand, bytes;
+  size_t qr, qu, ah, al, bh, bl, dense, cand, sym, bytes;
   int64_t qb;
   int K;
   int seg_n;                    // top-k segments per dense row
@@ -925,6 +925,7 @@ static ScoreWidePlan plan_score_wide(const tq_quantizer* q, int64_t nq, int64_t 
   P.dense = off; off = al(off + (topk > 0 ? P.qb * n * 4 : 0));
   P.seg_n = topk_segments(n);
   P.cand = off; off = al(off + (topk > 0 ? P.qb * P.seg_n * 32 * 8 : 0));   // scores, then ids
+  P.sym = off; off = al(off + 4);                  // records expanded as +-1 (int flag)
   P.bytes = off;
   return P;
 }
@@ -1025,8 +1026,9 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
     }
     const int bm = q->kind == TQ_KIND_PROD ? q->bits - 1 : q->bits;
     const float coef = m ? static_cast<float>(std::sqrt(M_PI / 2.0) / m) : 0.f;
+    int* sym = reinterpret_cast<int*>(ws + P.sym);
     e = launch_expand_records(keys.codes, L.code_words, keys.signs, L.sign_words, keys.rnorms, q->centroids, coef, n,
-                              d, m, bm, u16(P.bh), u16(P.bl), stream);
+                              d, m, bm, u16(P.bh), u16(P.bl), sym, stream);
     if (e != cudaSuccess) return cuda_fail(e, "record expansion launch");
     CUtensorMap maps[4];
     const int tn = gemm_tile_n(static_cast<int>(n));      // B box = one column tile
@@ -1035,13 +1037,14 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
     float* dense = reinterpret_cast<float*>(ws + P.dense);
     for (int64_t q0 = 0; q0 < nq; q0 += P.qb) {
       const int64_t nb = std::min(P.qb, nq - q0);
-      e = launch_split_cat(qr + q0 * d, d, qu + q0 * m, m, nb, u16(P.ah), u16(P.al), stream);
+      e = launch_split_cat(qr + q0 * d, d, qu + q0 * m, m, nb, u16(P.ah), u16(P.al), stream, sym, q->centroids);
       if (e != cudaSuccess) return cuda_fail(e, "query split launch");
       if ((s = bf16_map(&maps[0], u16(P.ah), nb, P.K, 128)) != TQ_OK) return s;
       if ((s = bf16_map(&maps[1], u16(P.al), nb, P.K, 128)) != TQ_OK) return s;
       SplitGemmParams g{};
       g.M = nb; g.N = static_cast<int>(n); g.K = P.K; g.status = device_status_ptr(); g.wait_limit = wait_limit();
       g.out = topk > 0 ? dense : scores + q0 * n; g.ldo = n; g.col_scale = keys.norms;
+      g.lo_skip_flag = sym; g.lo_skip_k = d;
       const int64_t work = (nb + 127) / 128 * ((n + tn - 1) / tn);
       e = launch_split_gemm(maps, g, GEMM_EPI_SCORE, 1, static_cast<int>(std::min<int64_t>(work, sm_count())), stream);
       if (e != cudaSuccess) return cuda_fail(e, "estimate launch");

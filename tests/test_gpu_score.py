@@ -84,7 +84,8 @@ def test_topk_search(bits):
 
 
 @pytest.mark.parametrize("d,kind,bits,n,nq", [(1536, "prod", 2, 5000, 7), (256, "mse", 3, 4500, 130),
-                                              (512, "prod", 5, 4099, 3), (512, "mse", 2, 4100, 9)])
+                                              (512, "prod", 5, 4099, 3), (512, "mse", 2, 4100, 9),
+                                              (384, "mse", 1, 4500, 6)])
 def test_scores_wide_tensor_core(d, kind, bits, n, nq):
     """Dense estimates on the tensor cores (d a multiple of 128, at least 4096 records): every
     (query, record) estimate equals the oracle's on the GPU's band-checked records to 1e-3
