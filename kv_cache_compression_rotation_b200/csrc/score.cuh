@@ -215,15 +215,15 @@ __global__ void __launch_bounds__(128) topk_kernel(const float* scores, int64_t 
 
 // y[i][j] = sum_k A[j][k] x[i][k] for queries i < nx and rows j < rows (A fp32 [rows][d], x
 // [nx][ldx] in the given dtype, d a multiple of 128): the query rotation and projection of the
-// tensor-core estimator.  A block takes kMvQ queries (in shared memory) and kMvRows rows, one
-// warp per row at a time: the lanes read the row with coalesced 16-byte loads and reduce the
-// kMvQ dot products with shuffles.
+// tensor-core estimator.  Block (x, y) takes queries kMvQ x .. (in shared memory) and rows
+// kMvRows y .., one warp per row at a time: the lanes read the row with coalesced 16-byte
+// loads and reduce the kMvQ dot products with shuffles.
 constexpr int kMvQ = 8, kMvRows = 32;
 __global__ void __launch_bounds__(128) rows_matvec_kernel(const float* __restrict__ A, int rows, int d,
                                                           const void* x, int dtype, int64_t nx, int64_t ldx,
                                                           float* __restrict__ y, int64_t ldy) {
   extern __shared__ __align__(16) float xs[];      // [kMvQ][d]
-  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * kMvQ;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kMvQ;
   for (int e = threadIdx.x; e < kMvQ * d; e += 128) {
     const int qi = e / d, k = e - qi * d;
     xs[e] = (i0 + qi < nx) ? load_elem(x, dtype, (i0 + qi) * ldx + k) : 0.f;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(128) rows_matvec_kernel(const float* __restric
   const float4* xs4 = reinterpret_cast<const float4*>(xs);
 #pragma unroll 1
   for (int jj = 0; jj < kMvRows / 4; ++jj) {
-    const int j = blockIdx.x * kMvRows + warp * (kMvRows / 4) + jj;
+    const int j = blockIdx.y * kMvRows + warp * (kMvRows / 4) + jj;
     if (j >= rows) break;
     const float4* a4 = reinterpret_cast<const float4*>(A + static_cast<int64_t>(j) * d);
     float acc[kMvQ];

@@ -1015,12 +1015,12 @@ tq_status tq_score(const tq_quantizer* q, const void* qv, int32_t dtype, int64_t
     cudaError_t e = cudaFuncSetAttribute(rows_matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(mv_smem));
     if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
-    const dim3 mv_grid(static_cast<unsigned>((d + kMvRows - 1) / kMvRows), static_cast<unsigned>((nq + kMvQ - 1) / kMvQ));
-    if (mv_grid.y > 65535) return fail(TQ_ERR_UNSUPPORTED, "too many queries");
+    // queries along x (up to 2^31 - 1 blocks), row blocks along y (d <= 4096: at most 128)
+    const dim3 mv_grid(static_cast<unsigned>((nq + kMvQ - 1) / kMvQ), static_cast<unsigned>((d + kMvRows - 1) / kMvRows));
     rows_matvec_kernel<<<mv_grid, 128, mv_smem, stream>>>(q->rot, d, d, qv, dtype, nq, d, qr, d);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "query rotation launch");
     if (m) {
-      const dim3 sg(static_cast<unsigned>((m + kMvRows - 1) / kMvRows), mv_grid.y);
+      const dim3 sg(mv_grid.x, static_cast<unsigned>((m + kMvRows - 1) / kMvRows));
       rows_matvec_kernel<<<sg, 128, mv_smem, stream>>>(q->S, m, d, qr, TQ_F32, nq, d, qu, qus);
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "query projection launch");
     }
